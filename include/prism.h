@@ -1,0 +1,237 @@
+/*
+ * prism.h — C ABI of the Prism dynamic block-sparse attention hot path for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Prism ("Prism: Dynamic Sparse Attention for Native 2K Joint Video-Audio
+ * Generation Model Training"; README of Tencent-Hunyuan/Prism, section
+ * "Overview") organises the video token grid into spatiotemporal macro-zones,
+ * gives every zone one 64-token block shape chosen from the video features'
+ * channel variance and the norm of the audio-to-video (a2v) bridge residual,
+ * represents blocks by block-level (mean-pooled) features, selects key blocks
+ * per query block with a hybrid top-k + cumulative-mass rule, and runs exact
+ * attention over the selected blocks only, forward and backward.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Token order is raster over the latent grid (T, H, W):
+ *   token n = (t * H + h) * W + w.
+ * - Zones tile the grid in raster (zt, zh, zw) order; zone z covers
+ *   [zt*Zt, zt*Zt+Zt) x [zh*Zh, ...) x [zw*Zw, ...).
+ * - A block shape is (bt, bh, bw) with bt*bh*bw == 64 dividing the zone
+ *   extents. The blocks of zone z are numbered raster over the zone's
+ *   (Zt/bt, Zh/bh, Zw/bw) sub-grid; global block id = z * blocks_per_zone +
+ *   local id, blocks_per_zone = Zt*Zh*Zw/64. Tokens inside a block are raster
+ *   (t, h, w). Query and key blocks use the same partition.
+ * - Q, K, V, O, dO, dQ, dK, dV are token-major [N, heads, head_dim] with a
+ *   token stride of `tok_stride` elements (>= heads*head_dim, a multiple of 8)
+ *   and contiguous heads and channels.
+ * - Pointers marked "device" must be device memory of the current device;
+ *   "host" pointers are read (or written) before the call returns. The
+ *   library never allocates or frees device memory: scratch comes from the
+ *   caller's workspace `ws` of `ws_bytes` bytes (256-byte aligned), sized by
+ *   prism_workspace_size(). Work is enqueued on `stream` (a cudaStream_t; NULL
+ *   is the legacy default stream) and is asynchronous unless stated.
+ * - Every call validates its arguments on the host and returns a status; no
+ *   exception crosses the ABI. Device-side faults are avoided by design:
+ *   device waits are bounded and report PRISM_ERR_TIMEOUT, index checks
+ *   report PRISM_ERR_DEVICE, through prism_check_device_status().
+ * - Not re-entrant on one workspace: calls that share `ws` must be ordered on
+ *   one stream.
+ */
+#ifndef PRISM_H_
+#define PRISM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PRISM_OK = 0,
+  PRISM_ERR_ARG = 1,         /* NULL where a pointer is required, bad scalar */
+  PRISM_ERR_SHAPE = 2,       /* grid / zone / candidate geometry invalid */
+  PRISM_ERR_DTYPE = 3,       /* dtype not supported for this argument */
+  PRISM_ERR_WORKSPACE = 4,   /* ws NULL, misaligned or smaller than required */
+  PRISM_ERR_CAPACITY = 5,    /* col_cap smaller than the number of kept pairs */
+  PRISM_ERR_CUDA = 6,        /* a CUDA runtime / driver call failed */
+  PRISM_ERR_TIMEOUT = 7,     /* a bounded device wait gave up */
+  PRISM_ERR_DEVICE = 8,      /* a device-side index check failed */
+  PRISM_ERR_UNSUPPORTED = 9  /* size outside what the kernels implement */
+} prism_status;
+
+typedef enum { PRISM_BF16 = 0, PRISM_FP32 = 1 } prism_dtype;
+
+typedef struct {
+  int32_t t, h, w;
+} prism_dim3;
+
+/* Token-grid geometry shared by the block-level entry points.
+ * grid: latent token grid (T, H, W); zone: macro-zone extents (Zt, Zh, Zw),
+ * dividing the grid, with Zt*Zh*Zw a multiple of 64 and at most 512;
+ * cand: host array of n_cand (1..16) candidate block shapes. */
+typedef struct {
+  prism_dim3 grid;
+  prism_dim3 zone;
+  const prism_dim3* cand;
+  int32_t n_cand;
+} prism_geometry;
+
+/* Constants of the zone shape rule (see prism_zone_shapes). */
+typedef struct {
+  float w_audio;  /* weight of the audio term, default 1 */
+  float gamma;    /* isotropy penalty, default 0.25 */
+  float gate_max; /* cap G of the audio gate, default 4 */
+} prism_shape_params;
+
+/* Which call a workspace is sized for. */
+typedef enum {
+  PRISM_OP_ZONE_SHAPES = 0,
+  PRISM_OP_BLOCK_SELECT = 1,
+  PRISM_OP_BSA_FWD = 2,
+  PRISM_OP_BSA_BWD = 3
+} prism_op;
+
+/* Human-readable name of a status. Never NULL. */
+const char* prism_status_string(prism_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t prism_version(void);
+
+/* Number of zones and of blocks for a geometry (host only, no GPU work). */
+prism_status prism_geometry_counts(const prism_geometry* geo, int32_t* n_zones, int32_t* n_blocks);
+
+/* Workspace bytes needed by `op`. `nnz` is the number of selected
+ * (query block, key block) pairs summed over heads (row_ptr[heads*n_blocks]),
+ * used by PRISM_OP_BSA_BWD only. `in_dtype` is the dtype of Q/K/V (fp32
+ * inputs need bf16 staging copies). Host only. */
+prism_status prism_workspace_size(prism_op op, const prism_geometry* geo, int32_t heads, int32_t head_dim,
+                                  int32_t feat_c, int32_t res_c, prism_dtype in_dtype, int64_t nnz,
+                                  size_t* bytes);
+
+/* Reads and clears the device status word kept in `ws` (synchronises
+ * `stream`). Returns PRISM_ERR_TIMEOUT or PRISM_ERR_DEVICE if a kernel that
+ * used this workspace reported one, else PRISM_OK. */
+prism_status prism_check_device_status(void* ws, void* stream);
+
+/*
+ * a1 + a2 — macro-zone tiling and per-zone block shape.
+ * Cites: README "Overview" (zones; video feature variance along the channel
+ * and a2v feature norms; finer partitioning along axes of rapid visual change
+ * and strong audio-visual coupling); walkthrough (wmrh.cn/news/72296) section
+ * "桥接残差反哺稀疏注意力" (per-token L2 norm of the unscaled a2v residual as
+ * the audio-influence proxy; sounding regions get finer blocks) and section
+ * "三者如何协同" (candidate shapes, one per zone).
+ *
+ * The rule (no formula is printed; this is the library's documented
+ * reading): for zone z and axis a in (t, h, w), V_a = mean over channels and
+ * over lines parallel to a of the population variance of the feature along
+ * the line; r(n) = ||res[n, :]||_2, A_a = mean over lines parallel to a of
+ * the population variance of r; g = clamp(mean_z r / mean_grid r - 1, 0,
+ * gate_max); S_a = 3 V_a / (sum V + 1e-12) + w_audio * g * 3 A_a / (sum A +
+ * 1e-12), renormalised to sum 3 (all ones when zero); cost(c) = sum_a S_a *
+ * log2(ext_{c,a}) + gamma * sum_a (log2(ext_{c,a}) - 2)^2; the zone takes the
+ * argmin, ties to the lower candidate index.
+ *
+ * feat: device [N, feat_c] row stride feat_ld elements (bf16 or fp32), or
+ *       NULL; res: device [N, res_c] row stride res_ld, or NULL. Both NULL:
+ *       every zone takes candidate 0. Row strides are multiples of 8 elements
+ *       and feat_c / res_c multiples of 64.
+ * params: host, NULL for the defaults.
+ * zone_shape: device int32 [n_zones] out (candidate index per zone).
+ * zone_margin: device float [n_zones] out (second-best minus best cost), or
+ *       NULL.
+ */
+prism_status prism_zone_shapes(const prism_geometry* geo, const void* feat, int64_t feat_ld, int32_t feat_c,
+                               prism_dtype feat_dtype, const void* res, int64_t res_ld, int32_t res_c,
+                               prism_dtype res_dtype, const prism_shape_params* params, int32_t* zone_shape,
+                               float* zone_margin, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * a3 — block partition and mean pooling ("block-level features", README
+ * "Overview"): q_pool[h, b, :] = mean of the 64 rows Q[n, h, :] of block b,
+ * likewise k_pool.
+ * zone_shape: device int32 [n_zones] (from prism_zone_shapes).
+ * q, k: device [N, heads, head_dim], bf16 or fp32, token stride tok_stride.
+ * q_pool, k_pool: device float [heads, n_blocks, head_dim] out.
+ * head_dim is 64 or 128.
+ */
+prism_status prism_block_pool(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
+                              prism_dtype dtype, int32_t heads, int32_t head_dim, int64_t tok_stride, float* q_pool,
+                              float* k_pool, void* stream);
+
+/*
+ * a4 + a5 — block scoring and hybrid selection (walkthrough section
+ * "三者如何协同": the gating step takes the k highest-scoring blocks, then
+ * extends along the CDF until cdf_threshold, default 0.20; README "Overview":
+ * hybrid selection sets each query's sparsity; Sol-Attn abstract on the
+ * Prism paper page: blocks ranked by a block proxy score).
+ *
+ * For head h and query block I: s_J = scale * q_pool[h,I] . k_pool[h,J] over
+ * all key blocks J; p = softmax(s); blocks ranked by p descending, ties to the
+ * lower J; m = max(top_k, min{m : p_(1) + ... + p_(m) >= cdf_threshold});
+ * top_k >= n_blocks or cdf_threshold >= 1 keeps every block. Scores are never
+ * written to memory.
+ *
+ * q_pool, k_pool: device float [heads, n_blocks, head_dim].
+ * top_k >= 1; cdf_threshold >= 0.
+ * mask: device uint32 [heads, n_blocks, ceil(n_blocks/32)] out; bit (J % 32)
+ *       of word J / 32 of row (h, I) is set when J is kept.
+ * kept: device int32 [heads, n_blocks] out (m per row).
+ * row_ptr: device int32 [heads*n_blocks + 1] out, CSR offsets over the rows
+ *       taken in (h, I) order.
+ * col_idx: device int32 [col_cap] out, kept J of each row ascending; NULL to
+ *       skip (then col_cap is ignored).
+ * total_kept: host int64 out (synchronises `stream`), or NULL. When col_idx
+ *       is given and the total exceeds col_cap the call returns
+ *       PRISM_ERR_CAPACITY after the sync, with col_idx untouched (this check
+ *       needs total_kept != NULL; without it the fill clips at col_cap and
+ *       reports PRISM_ERR_DEVICE through prism_check_device_status).
+ */
+prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
+                                int32_t head_dim, float scale, int32_t top_k, float cdf_threshold, uint32_t* mask,
+                                int32_t* kept, int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
+                                int64_t* total_kept, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * a6 — block-sparse attention forward (Sol-Attn abstract: compute only the
+ * selected key/value blocks): for every query token i of block I,
+ * O_i = sum over key tokens j of the blocks in row (h, I) of the CSR of
+ * softmax_j(scale * q_i . k_j) v_j, and lse[h, i] = log sum_j exp(scale q_i.k_j)
+ * (natural log). Exact up to bf16 operand rounding; fp32 accumulation.
+ *
+ * zone_shape: device int32 [n_zones].
+ * q, k, v: device [N, heads, head_dim], bf16 (fp32 inputs are rounded to bf16
+ *       in the workspace), token stride tok_stride. head_dim 64 or 128.
+ * row_ptr, col_idx: device CSR from prism_block_select (rows with no block
+ *       give O = 0 and lse = -inf).
+ * o: device [N, heads, head_dim] out, same dtype as q, token stride tok_stride.
+ * lse: device float [heads, N] out.
+ */
+prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
+                           const void* v, prism_dtype dtype, int32_t heads, int32_t head_dim, int64_t tok_stride,
+                           float scale, const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * a7 — block-sparse attention backward (Prism trains natively with the
+ * sparse attention, README "Overview"), selection held fixed:
+ * D_i = sum_c dO_ic O_ic; P_ij = exp(scale q_i.k_j - lse_i) on the selected
+ * blocks; dV_j = sum_i P_ij dO_i; dS_ij = P_ij (dO_i . v_j - D_i);
+ * dQ_i = scale sum_j dS_ij k_j; dK_j = scale sum_i dS_ij q_i.
+ * Arguments as prism_bsa_fwd; o and lse are the forward's outputs; dout is
+ * device [N, heads, head_dim]; dq, dk, dv are device outs like q. nnz =
+ * row_ptr[heads*n_blocks] (for workspace sizing; checked against ws_bytes).
+ */
+prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
+                           const void* v, const void* o, const float* lse, const void* dout, prism_dtype dtype,
+                           int32_t heads, int32_t head_dim, int64_t tok_stride, float scale, const int32_t* row_ptr,
+                           const int32_t* col_idx, int64_t nnz, void* dq, void* dk, void* dv, void* ws,
+                           size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_H_ */

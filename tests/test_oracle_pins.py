@@ -1,0 +1,359 @@
+"""Pins for the CPU oracle, independent of the oracle's own code paths.
+
+Each test fixes a value from something other than the oracle itself: closed
+forms, library routines (torch SDPA in fp64, scipy logsumexp), brute force over
+subsets, finite differences, and invariants that follow from the Prism pages'
+statements (finer blocks along axes of rapid variation; (4,4,4) is the
+isotropic shape; (8,2,4) for vertical detail; (2,4,8) for fast motion; hybrid
+top-k then CDF selection with default threshold 0.20).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import logsumexp
+
+from oracle import prism_oracle as O
+from dynamic_block_sparse_shape_b200.synth import DEFAULT_CANDIDATES
+
+CAND = list(DEFAULT_CANDIDATES)
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = line.split("=", 1)
+                out[k.strip()] = v.strip()
+    return out
+
+
+# ----------------------------------------------------------------- tiling
+def test_zone_tokens_are_a_partition():
+    grid, zone = (8, 16, 24), (4, 8, 8)
+    nz = np.prod(O.zone_counts(grid, zone))
+    seen = np.concatenate([O.zone_token_ids(grid, zone, z).ravel() for z in range(nz)])
+    assert np.array_equal(np.sort(seen), np.arange(np.prod(grid)))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_blocks_are_64_token_boxes_partitioning_the_grid(seed):
+    grid, zone = (8, 16, 16), (8, 8, 8)
+    rng = np.random.default_rng(seed)
+    nz = np.prod(O.zone_counts(grid, zone))
+    shape_idx = rng.integers(0, len(CAND), nz)
+    blocks = O.block_tokens(grid, zone, CAND, shape_idx)
+    T, H, W = grid
+    assert np.array_equal(np.sort(blocks.ravel()), np.arange(T * H * W))
+    for b, toks in enumerate(blocks):
+        t, r = np.divmod(toks, H * W)
+        h, w = np.divmod(r, W)
+        ext = (t.max() - t.min() + 1, h.max() - h.min() + 1, w.max() - w.min() + 1)
+        assert ext == CAND[shape_idx[b // 8]]
+        # raster (t, h, w) order inside the block
+        assert np.all(np.diff(toks) > 0)
+
+
+def test_block_ids_explicit_444():
+    # zone 8x8x8 on an 8x8x8 grid with (4,4,4): block 1 is the box w in 4..7.
+    blocks = O.block_tokens((8, 8, 8), (8, 8, 8), [(4, 4, 4)], [0])
+    assert blocks[0][:5].tolist() == [0, 1, 2, 3, 8]
+    assert blocks[1][0] == 4 and blocks[2][0] == 32 and blocks[4][0] == 256
+    assert blocks[7][-1] == 511
+
+
+# ----------------------------------------------------------------- statistics
+def test_line_variance_closed_forms():
+    t = np.arange(8)[:, None, None, None] * np.ones((8, 8, 8, 1))
+    # alternating sign along t: population variance 1 along t, 0 elsewhere
+    V = O.line_variance((-1.0) ** t)
+    assert np.allclose(V, [1.0, 0.0, 0.0], atol=1e-15)
+    # linear ramp 0..7 along h: variance (8^2-1)/12
+    h = np.arange(8)[None, :, None, None] * np.ones((8, 8, 8, 2))
+    assert np.allclose(O.line_variance(h), [0.0, 63.0 / 12.0, 0.0], atol=1e-12)
+    # two full periods of a quarter-wave along w: variance 1/2 for any phase
+    w = np.arange(8)[None, None, :, None]
+    X = np.sin(np.pi / 2 * w + np.array([0.3, 1.1, 2.9])[None, None, None, :]) * np.ones((8, 8, 8, 3))
+    assert np.allclose(O.line_variance(X), [0.0, 0.0, 0.5], atol=1e-12)
+
+
+def test_token_norms_closed_form():
+    R = np.array([[3.0, 4.0, 0.0], [0.0, 0.0, 0.0], [1.0, 1.0, 1.0]])
+    assert np.allclose(O.token_norms(R), [5.0, 0.0, math.sqrt(3.0)])
+
+
+# ----------------------------------------------------------------- shape rule
+def _choice(V, A=(0, 0, 0), m=0.0, mbar=1.0, cand=CAND):
+    c = O.shape_cost(np.array(V, float), np.array(A, float), m, mbar, cand)
+    return cand[int(np.argmin(c))]
+
+
+def test_isotropic_zone_takes_444():
+    g = _golden("pages_constants.txt")
+    assert tuple(int(x) for x in g["isotropic_shape"].split(",")) == (4, 4, 4)
+    assert _choice([1.0, 1.0, 1.0]) == (4, 4, 4)
+    assert _choice([0.0, 0.0, 0.0]) == (4, 4, 4)
+
+
+def test_named_shapes_of_the_walkthrough():
+    g = _golden("pages_constants.txt")
+    vertical = tuple(int(x) for x in g["vertical_detail_shape"].split(","))
+    motion = tuple(int(x) for x in g["fast_motion_shape"].split(","))
+    # h varies most, then w, then t: the vertical-detail shape
+    assert _choice([0.5, 1.5, 1.0]) == vertical
+    # t varies most, then h, then w: the fast-motion shape
+    assert _choice([1.5, 1.0, 0.5]) == motion
+    assert vertical in CAND and motion in CAND
+
+
+def test_variation_along_one_axis_gives_finest_extent_there():
+    for a in range(3):
+        V = [0.0, 0.0, 0.0]
+        V[a] = 1.0
+        s = _choice(V)
+        assert s[a] == min(c[a] for c in CAND)
+
+
+def test_shape_rule_permutes_with_axes():
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        V = rng.random(3)
+        A = rng.random(3)
+        base = _choice(V, A, m=2.5, mbar=1.0)
+        for perm in itertools.permutations(range(3)):
+            got = _choice(V[list(perm)], A[list(perm)], m=2.5, mbar=1.0)
+            # candidate costs are distinct for random stats, so the argmin moves with the axes
+            assert got == tuple(base[p] for p in perm)
+
+
+def test_shape_rule_scale_invariant():
+    rng = np.random.default_rng(6)
+    for _ in range(100):
+        V, A = rng.random(3), rng.random(3)
+        m, mbar = 3.0 * rng.random(), 1.0
+        ref = _choice(V, A, m, mbar)
+        assert _choice(7.5 * V, A, m, mbar) == ref
+        assert _choice(V, 0.01 * A, m, mbar) == ref
+        assert _choice(V, 4.0 * A, 9.0 * m, 9.0 * mbar) == ref  # scaling R scales m and mbar alike
+
+
+def test_audio_gate_only_acts_above_the_mean_norm():
+    V = [1.0, 1.0, 1.0]
+    A = [0.0, 1.0, 0.0]
+    assert _choice(V, A, m=0.9, mbar=1.0) == (4, 4, 4)  # quieter than average: no audio term
+    s = _choice(V, A, m=3.0, mbar=1.0)  # sounding zone with norm varying along h
+    assert s[1] < 4  # finer along h
+
+
+def test_finer_with_more_variation_monotone():
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        V = rng.random(3)
+        a = rng.integers(3)
+        before = _choice(V)[a]
+        V2 = V.copy()
+        V2[a] *= 1.0 + 3.0 * rng.random()
+        assert _choice(V2)[a] <= before
+
+
+def test_zone_statistics_end_to_end_on_planted_zones():
+    # two zones on a 8x8x16 grid: zone 0 oscillates along t, zone 1 along w.
+    grid, zone = (8, 8, 16), (8, 8, 8)
+    T, H, W = grid
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    F = np.where(w < 8, (-1.0) ** t, (-1.0) ** w).reshape(-1, 1) * np.ones((1, 4))
+    idx, margin, st = O.zone_shapes(grid, zone, CAND, F=F)
+    assert CAND[idx[0]] == (1, 8, 8) and CAND[idx[1]] == (8, 8, 1)
+    assert np.allclose(st["V"][0], [1, 0, 0]) and np.allclose(st["V"][1], [0, 0, 1])
+    assert np.all(margin > 0.1)
+    # no signal at all: candidate 0 everywhere
+    idx0, _, _ = O.zone_shapes(grid, zone, CAND)
+    assert np.all(idx0 == 0)
+
+
+# ----------------------------------------------------------------- pooling
+def test_pooling_of_a_linear_field_is_its_value_at_the_block_centre():
+    grid, zone = (8, 8, 16), (8, 8, 8)
+    T, H, W = grid
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    coef = np.array([[0.5, -1.0, 2.0, 0.25], [1.5, 0.0, -0.5, 3.0]])  # (a_t, a_h, a_w, c) per channel
+    X = np.stack([coef[c, 0] * t + coef[c, 1] * h + coef[c, 2] * w + coef[c, 3] for c in range(2)], -1)
+    X = X.reshape(-1, 1, 2)
+    shape_idx = [1, 5]
+    blocks = O.block_tokens(grid, zone, CAND, shape_idx)
+    pooled = O.block_pool(X, blocks)  # [1, nb, 2]
+    for b, toks in enumerate(blocks):
+        tt, r = np.divmod(toks, H * W)
+        hh, ww = np.divmod(r, W)
+        centre = np.array([(tt.min() + tt.max()) / 2, (hh.min() + hh.max()) / 2, (ww.min() + ww.max()) / 2])
+        expect = coef[:, :3] @ centre + coef[:, 3]
+        assert np.allclose(pooled[0, b], expect, atol=1e-12)
+
+
+# ----------------------------------------------------------------- selection
+def _brute_force_selection(p, k, tau):
+    """Smallest m such that SOME subset of size m carries mass >= tau (the
+    top-m subset carries the most), floored at k; the kept set is the size-m
+    subset of largest mass. Enumerates all subsets."""
+    n = len(p)
+    if k >= n or tau >= 1.0:
+        return set(range(n))
+    best = {}
+    for m in range(1, n + 1):
+        best[m] = max(itertools.combinations(range(n), m), key=lambda S: sum(p[i] for i in S))
+    m_min = next((m for m in range(1, n + 1) if sum(p[i] for i in best[m]) >= tau), n)
+    return set(best[max(k, m_min)])
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_selection_matches_subset_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(3, 10))
+    s = rng.normal(0, 1.5, n)
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    for k in (1, 2, 3):
+        for tau in (0.05, 0.2, 0.5, 0.9, 1.0):
+            kept, m, m_star, gap, margin = O.select_row(s, k, tau)
+            assert set(kept.tolist()) == _brute_force_selection(p, k, tau)
+            assert m >= min(k, n)
+
+
+def test_selection_invariants_and_special_cases():
+    rng = np.random.default_rng(3)
+    H, nb, d = 2, 16, 8
+    qp, kp = rng.normal(size=(H, nb, d)), rng.normal(size=(H, nb, d))
+    sc = 1 / math.sqrt(d)
+    s = O.block_logits(qp, kp, sc)
+    # tau = 1 or k = nb: dense
+    assert O.block_select(qp, kp, sc, 1, 1.0)["mask"].all()
+    assert O.block_select(qp, kp, sc, nb, 0.2)["mask"].all()
+    # tau -> 0: exactly the k largest logits
+    r = O.block_select(qp, kp, sc, 3, 1e-12)
+    for h in range(H):
+        for i in range(nb):
+            top = set(np.argsort(-s[h, i], kind="stable")[:3].tolist())
+            assert set(np.nonzero(r["mask"][h, i])[0].tolist()) == top
+    # minimal prefix: C_{m*-1} < tau <= C_{m*}; kept >= k
+    r = O.block_select(qp, kp, sc, 2, 0.3)
+    for h in range(H):
+        for i in range(nb):
+            row = s[h, i]
+            p = np.exp(row - row.max())
+            p /= p.sum()
+            kept = np.nonzero(r["mask"][h, i])[0]
+            assert len(kept) >= 2
+            order = np.argsort(-row, kind="stable")
+            C = np.cumsum(p[order])
+            m_star = int(np.searchsorted(C, 0.3)) + 1
+            assert C[m_star - 1] >= 0.3 and (m_star == 1 or C[m_star - 2] < 0.3)
+            assert len(kept) == max(2, m_star)
+
+
+def test_default_cdf_threshold_from_the_pages():
+    g = _golden("pages_constants.txt")
+    assert float(g["cdf_threshold_default"]) == 0.20
+
+
+# ----------------------------------------------------------------- attention
+def _tiny_problem(seed=0, N=128, H=2, d=16, nblocks=None):
+    rng = np.random.default_rng(seed)
+    Q, K, V, dO = (rng.normal(size=(N, H, d)) for _ in range(4))
+    return Q, K, V, dO
+
+
+def _sdpa(Q, K, V, allowed, scale):
+    q = torch.tensor(Q).permute(1, 0, 2)
+    k = torch.tensor(K).permute(1, 0, 2)
+    v = torch.tensor(V).permute(1, 0, 2)
+    out = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.tensor(allowed), scale=scale)
+    return out.permute(1, 0, 2).numpy()
+
+
+def test_dense_selection_equals_full_attention():
+    Q, K, V, _ = _tiny_problem()
+    N, H, d = Q.shape
+    allowed = np.ones((H, N, N), bool)
+    Oo, lse = O.masked_attention_fwd(Q, K, V, allowed, 1 / math.sqrt(d))
+    assert np.allclose(Oo, _sdpa(Q, K, V, allowed, 1 / math.sqrt(d)), atol=1e-12)
+    S = np.einsum("ihd,jhd->hij", Q, K) / math.sqrt(d)
+    assert np.allclose(lse, logsumexp(S, axis=-1), atol=1e-12)
+
+
+def test_masked_attention_matches_library_with_block_mask():
+    grid, zone = (4, 8, 8), (4, 8, 8)
+    rng = np.random.default_rng(1)
+    N, H, d = 256, 2, 16
+    Q, K, V = (rng.normal(size=(N, H, d)) for _ in range(3))
+    blocks = O.block_tokens(grid, zone, [(4, 4, 4)], [0])
+    bm = rng.random((H, 4, 4)) < 0.5
+    bm[:, np.arange(4), rng.integers(0, 4, 4)] = True  # every row keeps a block
+    allowed = O.token_mask(bm, blocks, N)
+    sc = 1 / math.sqrt(d)
+    Oo, lse = O.masked_attention_fwd(Q, K, V, allowed, sc)
+    assert np.allclose(Oo, _sdpa(Q, K, V, allowed, sc), atol=1e-12)
+    S = np.where(allowed, np.einsum("ihd,jhd->hij", Q, K) * sc, -np.inf)
+    assert np.allclose(lse, logsumexp(S, axis=-1), atol=1e-12)
+
+
+def test_masked_attention_backward_matches_autograd_and_finite_differences():
+    rng = np.random.default_rng(2)
+    N, H, d = 64, 1, 8
+    Q, K, V, dO = (rng.normal(size=(N, H, d)) for _ in range(4))
+    allowed = rng.random((H, N, N)) < 0.4
+    allowed[:, np.arange(N), np.arange(N)] = True
+    sc = 1 / math.sqrt(d)
+    Oo, lse = O.masked_attention_fwd(Q, K, V, allowed, sc)
+    dQ, dK, dV = O.masked_attention_bwd(Q, K, V, Oo, lse, dO, allowed, sc)
+    # library autograd in fp64
+    q, k, v = (torch.tensor(x).permute(1, 0, 2).requires_grad_(True) for x in (Q, K, V))
+    out = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.tensor(allowed), scale=sc)
+    (out * torch.tensor(dO).permute(1, 0, 2)).sum().backward()
+    assert np.allclose(dQ, q.grad.permute(1, 0, 2).numpy(), atol=1e-10)
+    assert np.allclose(dK, k.grad.permute(1, 0, 2).numpy(), atol=1e-10)
+    assert np.allclose(dV, v.grad.permute(1, 0, 2).numpy(), atol=1e-10)
+    # central finite differences on a few coordinates
+    def loss(Qx, Kx, Vx):
+        return float((O.masked_attention_fwd(Qx, Kx, Vx, allowed, sc)[0] * dO).sum())
+    h = 1e-6
+    for (arr_i, grad) in ((0, dQ), (1, dK), (2, dV)):
+        for _ in range(5):
+            i, j = rng.integers(N), rng.integers(d)
+            args = [Q.copy(), K.copy(), V.copy()]
+            args[arr_i][i, 0, j] += h
+            lp = loss(*args)
+            args[arr_i][i, 0, j] -= 2 * h
+            lm = loss(*args)
+            assert abs((lp - lm) / (2 * h) - grad[i, 0, j]) < 1e-6
+
+
+def test_sampled_rows_equal_masked_dense_form():
+    grid, zone = (4, 8, 16), (4, 8, 8)
+    rng = np.random.default_rng(4)
+    N, H, d = 512, 2, 16
+    Q, K, V, dO = (rng.normal(size=(N, H, d)) for _ in range(4))
+    blocks = O.block_tokens(grid, zone, [(4, 4, 4)], [0, 0])
+    nb = blocks.shape[0]
+    bm = rng.random((H, nb, nb)) < 0.5
+    bm[:, np.arange(nb), np.arange(nb)] = True
+    sc = 1 / math.sqrt(d)
+    allowed = O.token_mask(bm, blocks, N)
+    Oo, lse = O.masked_attention_fwd(Q, K, V, allowed, sc)
+    dQ, dK, dV = O.masked_attention_bwd(Q, K, V, Oo, lse, dO, allowed, sc)
+    cache = {}
+    for h in range(H):
+        for I in range(nb):
+            rr = O.attention_block_rows(Q, K, V, blocks, np.nonzero(bm[h, I])[0], h, I, sc, dO=dO)
+            assert np.allclose(rr["O"], Oo[blocks[I], h], atol=1e-12)
+            assert np.allclose(rr["lse"], lse[h, blocks[I]], atol=1e-12)
+            assert np.allclose(rr["dQ"], dQ[blocks[I], h], atol=1e-12)
+        for J in range(nb):
+            gk, gv = O.attention_kv_block_grads(Q, K, V, dO, blocks, bm[h], h, J, sc, row_cache=cache)
+            assert np.allclose(gk, dK[blocks[J], h], atol=1e-12)
+            assert np.allclose(gv, dV[blocks[J], h], atol=1e-12)
