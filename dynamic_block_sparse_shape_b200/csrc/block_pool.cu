@@ -1,0 +1,110 @@
+// a3: block partition and mean pooling ("block-level features", Prism README
+// "Overview"; mean pooling as the block feature).
+//
+// One CTA per (block, tensor): each thread owns 8 consecutive channels of the
+// token row [heads * head_dim] and walks the block's 64 tokens (bt rows of bh
+// runs of bw contiguous tokens), accumulating in fp32 with 16-byte loads.
+// The output layout is [heads, n_blocks, head_dim] fp32.
+#include <cuda_bf16.h>
+
+#include "host.h"
+
+namespace prism {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float* x);
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float* x) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float* x) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(1024) pool_kernel(const Geo g, const int32_t* __restrict__ zone_shape,
+                                                    const T* __restrict__ q, const T* __restrict__ k,
+                                                    int64_t tok_stride, int head_dim, float* __restrict__ qp,
+                                                    float* __restrict__ kp, int* status) {
+  const int b = blockIdx.x;
+  const T* src = blockIdx.y ? k : q;
+  float* dst = blockIdx.y ? kp : qp;
+  const int c0 = threadIdx.x * 8;
+  const int head = c0 / head_dim, dd = c0 - head * head_dim;
+  float* out = dst + (size_t(head) * g.n_blocks + b) * head_dim + dd;
+  const int shape = zone_shape[zone_of_block(g, b)];
+  if (shape < 0 || shape >= g.n_cand) {
+    if (threadIdx.x == 0) atomicOr(status, kDevErrBounds);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = __int_as_float(0x7fc00000);
+    return;
+  }
+  const BlockBox bb = block_box(g, shape, b);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int rt = 0; rt < bb.bt; ++rt) {
+    for (int rh = 0; rh < bb.bh; ++rh) {
+      const int64_t n0 = (int64_t(bb.t0 + rt) * g.H + bb.h0 + rh) * g.W + bb.w0;
+      const T* row = src + n0 * tok_stride + c0;
+#pragma unroll 4
+      for (int rw = 0; rw < bb.bw; ++rw) {
+        float x[8];
+        load8<T>(row + int64_t(rw) * tok_stride, x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += x[i];
+      }
+    }
+  }
+  const float inv = 1.0f / 64.0f;
+  reinterpret_cast<float4*>(out)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  reinterpret_cast<float4*>(out)[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+}
+
+}  // namespace
+}  // namespace prism
+
+using namespace prism;
+
+extern "C" prism_status prism_block_pool(const prism_geometry* geo, const int32_t* zone_shape, const void* q,
+                                         const void* k, prism_dtype dtype, int32_t heads, int32_t head_dim,
+                                         int64_t tok_stride, float* q_pool, float* k_pool, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  Geo g;
+  prism_status st = make_geo(geo, &g);
+  if (st != PRISM_OK) return st;
+  if (!zone_shape || !q || !k || !q_pool || !k_pool) return PRISM_ERR_ARG;
+  if (dtype != PRISM_BF16 && dtype != PRISM_FP32) return PRISM_ERR_DTYPE;
+  if (head_dim != 64 && head_dim != 128) return PRISM_ERR_UNSUPPORTED;
+  if (heads < 1 || int64_t(heads) * head_dim > 8192) return PRISM_ERR_UNSUPPORTED;
+  if (tok_stride < int64_t(heads) * head_dim || tok_stride % 8) return PRISM_ERR_ARG;
+  const size_t es = dtype == PRISM_FP32 ? 4 : 2;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k) % 16) return PRISM_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(q_pool) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16) return PRISM_ERR_ARG;
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
+  (void)es;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(g.n_blocks, 2);
+  const int threads = heads * head_dim / 8;
+  if (dtype == PRISM_BF16)
+    pool_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(g, zone_shape, static_cast<const __nv_bfloat16*>(q),
+                                                         static_cast<const __nv_bfloat16*>(k), tok_stride, head_dim,
+                                                         q_pool, k_pool, ws_status(ws));
+  else
+    pool_kernel<float><<<grid, threads, 0, s>>>(g, zone_shape, static_cast<const float*>(q),
+                                                static_cast<const float*>(k), tok_stride, head_dim, q_pool, k_pool,
+                                                ws_status(ws));
+  return cuda_status(cudaGetLastError());
+}

@@ -1,0 +1,336 @@
+// a4 + a5: block scoring and hybrid top-k + cumulative-mass selection.
+//
+// Prism walkthrough (wmrh.cn/news/72296), section "三者如何协同": the gating
+// step keeps the k highest-scoring blocks, then extends along the CDF of the
+// block scores until cdf_threshold (default 0.20). Prism README "Overview":
+// the hybrid rule sets each query's sparsity. Sol-Attn abstract on the Prism
+// paper page: computing and materialising the proxy scores is the routing
+// overhead, so the scores here live only in shared memory.
+//
+// select_kernel: one CTA = 8 query blocks of one head (one warp each).
+//   1. logits s_J = scale * qbar_I . kbar_J for all J, fp32 FFMA, with the
+//      key features staged transposed in shared memory (2 keys x 4 rows per
+//      thread per channel);
+//   2. per row: max, p_J = exp(s_J - max) in place, Z = sum p (fp64);
+//   3. the mass threshold: bisection on the float bits of p for
+//      u* = max{u : sum_{key_J >= u} p_J >= tau * Z}; ties at u* are taken in
+//      ascending J until the mass is reached -> m*;
+//   4. m = max(k, m*); if m > m*, a bisection on counts finds the m-th key;
+//   5. the kept set (ranked by p descending, ties to the lower J) is written
+//      as a bitmask row with warp ballots, and kept[row] = m.
+// scan_kernel: exclusive scan of kept into the CSR row_ptr (one CTA).
+// fill_kernel: one warp per row expands the bitmask into ascending col_idx.
+#include <cfloat>
+#include <cmath>
+
+#include "host.h"
+
+namespace prism {
+namespace {
+
+constexpr int kSelRows = 8;
+constexpr int kSelThreads = 256;
+constexpr int kKeyTile = 256;
+constexpr int kDChunk = 32;
+constexpr int kKtPitch = kKeyTile + 2;
+constexpr int kSelMaxBlocks = 5120;
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Mass of the entries whose key is >= u (fp64, warp-reduced).
+__device__ __forceinline__ double mass_at_least(const float* p, int nb, uint32_t u, int lane) {
+  double acc = 0;
+  for (int j = lane; j < nb; j += 32) {
+    const float v = p[j];
+    if (__float_as_uint(v) >= u) acc += double(v);
+  }
+  return warp_sum_d(acc);
+}
+__device__ __forceinline__ int count_at_least(const float* p, int nb, uint32_t u, int lane) {
+  int c = 0;
+  for (int j = lane; j < nb; j += 32) c += __float_as_uint(p[j]) >= u;
+  return warp_sum_i(c);
+}
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+    select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int nb, int d, float scale, int top_k,
+                  float tau, uint32_t* __restrict__ mask, int32_t* __restrict__ kept) {
+  extern __shared__ __align__(16) float sm[];
+  float* srow = sm;                                  // [kSelRows][nb]
+  float* kT = srow + size_t(kSelRows) * nb;          // [kDChunk][kKtPitch]
+  float* qT = kT + kDChunk * kKtPitch;               // [d][kSelRows]
+  const int head = blockIdx.y;
+  const int I0 = blockIdx.x * kSelRows;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* qh = qp + size_t(head) * nb * d;
+  const float* kh = kp + size_t(head) * nb * d;
+  for (int i = tid; i < kSelRows * d; i += kSelThreads) {
+    const int r = i / d, c = i - r * d;
+    qT[c * kSelRows + r] = (I0 + r < nb) ? qh[size_t(I0 + r) * d + c] : 0.f;
+  }
+  // ---- 1. logits
+  const int kpair = tid & 127, rh = tid >> 7;
+  for (int key0 = 0; key0 < nb; key0 += kKeyTile) {
+    float acc[4][2] = {{0, 0}, {0, 0}, {0, 0}, {0, 0}};
+    for (int c0 = 0; c0 < d; c0 += kDChunk) {
+      __syncthreads();
+      // stage kT[c][j] = kbar[key0 + j][c0 + c], 256 keys x 32 channels
+      for (int i = tid; i < kKeyTile * (kDChunk / 4); i += kSelThreads) {
+        const int j = i >> 3, q4 = i & 7;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (key0 + j < nb) v = __ldg(reinterpret_cast<const float4*>(kh + size_t(key0 + j) * d + c0) + q4);
+        kT[(q4 * 4 + 0) * kKtPitch + j] = v.x;
+        kT[(q4 * 4 + 1) * kKtPitch + j] = v.y;
+        kT[(q4 * 4 + 2) * kKtPitch + j] = v.z;
+        kT[(q4 * 4 + 3) * kKtPitch + j] = v.w;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int c = 0; c < kDChunk; ++c) {
+        const float2 kv = *reinterpret_cast<const float2*>(kT + c * kKtPitch + 2 * kpair);
+        const float4 qv = *reinterpret_cast<const float4*>(qT + (c0 + c) * kSelRows + 4 * rh);
+        acc[0][0] = fmaf(qv.x, kv.x, acc[0][0]); acc[0][1] = fmaf(qv.x, kv.y, acc[0][1]);
+        acc[1][0] = fmaf(qv.y, kv.x, acc[1][0]); acc[1][1] = fmaf(qv.y, kv.y, acc[1][1]);
+        acc[2][0] = fmaf(qv.z, kv.x, acc[2][0]); acc[2][1] = fmaf(qv.z, kv.y, acc[2][1]);
+        acc[3][0] = fmaf(qv.w, kv.x, acc[3][0]); acc[3][1] = fmaf(qv.w, kv.y, acc[3][1]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int key = key0 + 2 * kpair + j;
+        if (key < nb) srow[size_t(4 * rh + i) * nb + key] = acc[i][j] * scale;
+      }
+  }
+  __syncthreads();
+  // ---- 2..5. one warp per query block
+  const int I = I0 + warp;
+  if (I >= nb) return;
+  float* p = srow + size_t(warp) * nb;
+  const int words = (nb + 31) >> 5;
+  uint32_t* mrow = mask + (size_t(head) * nb + I) * words;
+  float mx = -INFINITY;
+  for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, p[j]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  double zacc = 0;
+  for (int j = lane; j < nb; j += 32) {
+    float e = expf(p[j] - mx);
+    if (!(e >= 0.f)) e = 0.f;  // NaN logits carry no mass
+    p[j] = e;
+    zacc += double(e);
+  }
+  const double Z = warp_sum_d(zacc);
+  __syncwarp();
+  if (top_k >= nb || tau >= 1.0f) {
+    for (int w = lane; w < words; w += 32) {
+      const int rem = nb - 32 * w;
+      mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+    }
+    if (lane == 0) kept[size_t(head) * nb + I] = nb;
+    return;
+  }
+  const double target = double(tau) * Z;
+  // u*: largest key with mass(key >= u) >= target.
+  uint32_t u_star;
+  int m_star;
+  if (target <= 0.0) {
+    // C_1 >= tau already: the single largest entry (ties -> lowest J).
+    uint32_t best = 0;
+    for (int j = lane; j < nb; j += 32) best = max(best, __float_as_uint(p[j]));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+    u_star = best;
+    m_star = count_at_least(p, nb, u_star + 1, lane) + 1;
+  } else {
+    uint32_t lo = 0, hi = 0x3F800001u;  // mass(>= lo) >= target, mass(>= hi) < target
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      if (mass_at_least(p, nb, mid, lane) >= target) lo = mid; else hi = mid;
+    }
+    u_star = lo;
+    const double above = mass_at_least(p, nb, u_star + 1, lane);
+    const int above_cnt = count_at_least(p, nb, u_star + 1, lane);
+    // walk the entries tied at u_star in ascending J
+    double run = above;
+    int rank = 0;
+    bool found = false;
+    for (int base = 0; base < nb && !found; base += 32) {
+      const int j = base + lane;
+      const bool tie = j < nb && __float_as_uint(p[j]) == u_star;
+      uint32_t bal = __ballot_sync(0xffffffffu, tie);
+      while (bal) {
+        const int src = __ffs(bal) - 1;
+        bal &= bal - 1;
+        (void)src;
+        run += double(__uint_as_float(u_star));  // every tied entry has p = u_star
+        ++rank;
+        if (run >= target) { found = true; break; }
+      }
+    }
+    if (!found) rank = max(rank, 1);
+    m_star = above_cnt + rank;
+  }
+  const int m = max(min(top_k, nb), m_star);
+  uint32_t u_final;
+  int keep_ties;  // number of entries tied at u_final to keep, lowest J first
+  if (m == m_star) {
+    u_final = u_star;
+    keep_ties = m - count_at_least(p, nb, u_star + 1, lane);
+  } else {
+    uint32_t lo = 0, hi = 0x7F800001u;  // count(>= lo) >= m, count(>= hi) < m
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      if (count_at_least(p, nb, mid, lane) >= m) lo = mid; else hi = mid;
+    }
+    u_final = lo;
+    keep_ties = m - count_at_least(p, nb, u_final + 1, lane);
+  }
+  int tie_run = 0;
+  for (int w = 0; w < words; ++w) {
+    const int j = 32 * w + lane;
+    const uint32_t key = j < nb ? __float_as_uint(p[j]) : 0u;
+    const bool tie = j < nb && key == u_final;
+    const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+    const int my_rank = tie_run + __popc(tb & ((1u << lane) - 1u));
+    const bool keep = j < nb && (key > u_final || (tie && my_rank < keep_ties));
+    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+    tie_run += __popc(tb);
+    if (lane == 0) mrow[w] = kb;
+  }
+  if (lane == 0) kept[size_t(head) * nb + I] = m;
+}
+
+// Exclusive scan of n ints into out[0..n] (out[n] = total), one CTA.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ in, int n, int32_t* __restrict__ out) {
+  __shared__ int64_t part[1024];
+  const int tid = threadIdx.x;
+  const int per = (n + 1023) / 1024;
+  const int b = tid * per, e = min(n, b + per);
+  int64_t s = 0;
+  for (int i = b; i < e; ++i) s += in[i];
+  part[tid] = s;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const int64_t v = tid >= off ? part[tid - off] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  int64_t run = part[tid] - s;
+  for (int i = b; i < e; ++i) {
+    out[i] = int32_t(run);
+    run += in[i];
+  }
+  if (tid == 1023) out[n] = int32_t(part[1023]);
+}
+
+__global__ void __launch_bounds__(256) fill_kernel(const uint32_t* __restrict__ mask, const int32_t* __restrict__ row_ptr,
+                                                   int rows, int nb, int64_t cap, int32_t* __restrict__ col_idx,
+                                                   int* status) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int words = (nb + 31) >> 5;
+  const uint32_t* mrow = mask + size_t(row) * words;
+  int64_t pos = row_ptr[row];
+  const int64_t end = row_ptr[row + 1];
+  if (end > cap || end < pos) {
+    if (lane == 0) atomicOr(status, kDevErrCapacity);
+    return;
+  }
+  for (int w0 = 0; w0 < words; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t bits = w < words ? mrow[w] : 0u;
+    const int cnt = __popc(bits);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int64_t at = pos + incl - cnt;
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (at < end) col_idx[at] = 32 * w + bit;
+      ++at;
+    }
+    pos += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+}  // namespace
+
+size_t block_select_ws_bytes() { return kWsHeader; }
+
+cudaError_t launch_exclusive_scan(const int32_t* in, int n, int32_t* out, cudaStream_t s) {
+  scan_kernel<<<1, 1024, 0, s>>>(in, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mask_to_lists(const uint32_t* mask, const int32_t* row_ptr, int rows, int nb, int64_t cap,
+                                 int32_t* idx, int* status, cudaStream_t s) {
+  fill_kernel<<<unsigned((int64_t(rows) * 32 + 255) / 256), 256, 0, s>>>(mask, row_ptr, rows, nb, cap, idx, status);
+  return cudaGetLastError();
+}
+
+}  // namespace prism
+
+using namespace prism;
+
+extern "C" prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
+                                           int32_t head_dim, float scale, int32_t top_k, float cdf_threshold,
+                                           uint32_t* mask, int32_t* kept, int32_t* row_ptr, int32_t* col_idx,
+                                           int64_t col_cap, int64_t* total_kept, void* ws, size_t ws_bytes,
+                                           void* stream) {
+  if (!q_pool || !k_pool || !mask || !kept || !row_ptr) return PRISM_ERR_ARG;
+  if (heads < 1 || n_blocks < 1 || top_k < 1) return PRISM_ERR_ARG;
+  if (!(cdf_threshold >= 0.f) || !(scale > 0.f) || !std::isfinite(scale)) return PRISM_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return PRISM_ERR_UNSUPPORTED;
+  if (n_blocks > kSelMaxBlocks) return PRISM_ERR_UNSUPPORTED;
+  if (int64_t(heads) * n_blocks * n_blocks >= (int64_t(1) << 31)) return PRISM_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(q_pool) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16) return PRISM_ERR_ARG;
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
+  if (col_idx && col_cap < 0) return PRISM_ERR_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t smem = (size_t(kSelRows) * n_blocks + kDChunk * kKtPitch + size_t(head_dim) * kSelRows) * sizeof(float);
+  if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  const dim3 grid((n_blocks + kSelRows - 1) / kSelRows, heads);
+  select_kernel<<<grid, kSelThreads, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, top_k, cdf_threshold, mask,
+                                                kept);
+  const int rows = heads * n_blocks;
+  if (launch_exclusive_scan(kept, rows, row_ptr, s) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (total_kept) {
+    int32_t tot = 0;
+    if (cudaMemcpyAsync(&tot, row_ptr + rows, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PRISM_ERR_CUDA;
+    *total_kept = tot;
+    if (col_idx && tot > col_cap) return PRISM_ERR_CAPACITY;
+  }
+  if (col_idx) {
+    if (launch_mask_to_lists(mask, row_ptr, rows, n_blocks, col_cap, col_idx, ws_status(ws), s) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+extern "C" prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* row_ptr, int32_t rows,
+                                          int32_t n_blocks, int32_t* col_idx, int64_t col_cap, void* ws,
+                                          size_t ws_bytes, void* stream) {
+  if (!mask || !row_ptr || !col_idx || rows < 1 || n_blocks < 1 || col_cap < 0) return PRISM_ERR_ARG;
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
+  return cuda_status(launch_mask_to_lists(mask, row_ptr, rows, n_blocks, col_cap, col_idx, ws_status(ws),
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}

@@ -1,0 +1,751 @@
+// a7: block-sparse attention backward with the block selection held fixed.
+//
+// Prism is a training method (README "Overview": natively training joint
+// video-audio models with the sparse attention), so the attention over the
+// selected blocks needs dQ, dK and dV. With P_ij = exp(scale q_i.k_j - lse_i)
+// on the selected blocks and D_i = rowsum(dO_i * O_i):
+//   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i . v_j - D_i),
+//   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i.
+//
+// Kernels:
+//   prep        one CTA per (block, head): D in block order and the forward
+//               LSE converted to log2 units in block order;
+//   csc_scatter the CSR selection transposed into a bitmask [head, J, I];
+//               csc_count + scan + list fill give the CSC (ascending I);
+//   dq          one CTA per (query block, head), q-stationary: per step of two
+//               selected key blocks, S = Q K^T and dP = dO V^T (.ws M=64,
+//               N=128), then dS in the softmax warps, then dQ += dS K (.ws
+//               M=64, N=d); dQ lives in TMEM for the whole row;
+//   dkdv        one CTA per (key block, head), kv-stationary over the query
+//               blocks that selected it: S^T = K Q^T, dP^T = V dO^T, then
+//               P^T, dS^T in the softmax warps, then dV += P^T dO and
+//               dK += dS^T Q (.ws M=64, N=d); dK, dV live in TMEM.
+// Splitting dQ from dK/dV costs one recomputation of S and dP but needs no
+// atomics and is deterministic.
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "bsa_common.cuh"
+#include "host.h"
+
+namespace prism {
+namespace {
+
+constexpr int kKB = 2;
+constexpr int kSoftWarps = 8;
+constexpr int kBwdThreads = 64 + 32 * kSoftWarps;
+
+struct BwdParams {
+  CUtensorMap mq[kMaxCand];
+  CUtensorMap mk[kMaxCand];
+  CUtensorMap mv[kMaxCand];
+  CUtensorMap mdo[kMaxCand];
+  Geo g;
+  const int32_t* zone_shape;
+  const int32_t* ptr;  // CSR row_ptr (dq) or CSC col_ptr (dkdv), over (head, block)
+  const int32_t* idx;  // CSR col_idx (dq) or CSC row_idx (dkdv)
+  const float* lse2;   // [heads, n_blocks, 64] LSE * log2(e), block order
+  const float* dvec;   // [heads, n_blocks, 64] rowsum(dO * O), block order
+  void* out0;          // dq   | dk
+  void* out1;          //      | dv
+  int* status;
+  int64_t tok_stride;  // of the outputs, elements
+  float scale_log2;
+  float scale;
+  int out_fp32;
+};
+
+// ----------------------------------------------------------------------- dq
+template <int D>
+struct DqSmem {
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kDO = D * 128;
+  static constexpr uint32_t kHalf = kKB * D * 128;  // K (or V) of one stage
+  static constexpr uint32_t kStage0 = 2 * D * 128;
+  static constexpr uint32_t kStageBytes = 2 * kHalf;
+  static constexpr uint32_t kDS0 = kStage0 + 2 * kStageBytes;
+  static constexpr uint32_t kDSBytes = kKB * kBoxBytes;
+  static constexpr uint32_t kBar = kDS0 + 2 * kDSBytes;
+  static constexpr uint32_t kTotal = kBar + 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_constant__ BwdParams P) {
+  using L = DqSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  uint64_t* qd_full = bars + 0;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_free = bars + 7;
+  uint64_t* ds_full = bars + 9;
+  uint64_t* ds_free = bars + 11;
+  uint64_t* mma_done = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+
+  const Geo& g = P.g;
+  const int I = blockIdx.x, head = blockIdx.y;
+  const int row = head * g.n_blocks + I;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = P.status;
+  const int beg = P.ptr[row];
+  int cnt = P.ptr[row + 1] - beg;
+  if (cnt < 0 || cnt > g.n_blocks) {
+    if (threadIdx.x == 0) atomicOr(status, kDevErrBounds);
+    cnt = 0;
+  }
+  const int nsteps = (cnt + kKB - 1) / kKB;
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kSoftWarps);
+      mbar_init(&ds_full[i], kSoftWarps);
+      mbar_init(&ds_free[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tdQ = tbase + 256;
+
+  if (warp == 0) {
+    if (lane == 0 && nsteps > 0) {
+      const int sI = safe_shape(g, P.zone_shape, I, status);
+      const BlockBox qb = block_box(g, sI, I);
+      mbar_arrive_expect_tx(qd_full, 2 * D * 128);
+      for (int dh = 0; dh < D / 64; ++dh) {
+        tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+        tma_load_5d(sm + L::kDO + dh * kBoxBytes, &P.mdo[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+      }
+      int issued = 0;
+      for (int j = 0; j < nsteps; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait_abortable(&kv_empty[st], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
+        uint8_t* stage = sm + L::kStage0 + st * L::kStageBytes;
+        mbar_arrive_expect_tx(&kv_full[st], L::kStageBytes);
+        for (int slot = 0; slot < kKB; ++slot) {
+          int e = j * kKB + slot;
+          if (e >= cnt) e = j * kKB;
+          int J = P.idx[beg + e];
+          if (J < 0 || J >= g.n_blocks) {
+            atomicOr(status, kDevErrBounds);
+            J = 0;
+          }
+          const int sJ = safe_shape(g, P.zone_shape, J, status);
+          const BlockBox kb = block_box(g, sJ, J);
+          for (int dh = 0; dh < D / 64; ++dh) {
+            const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
+            tma_load_5d(stage + off, &P.mk[sJ], &kv_full[st], dh * 64, head, kb.w0, kb.h0, kb.t0);
+            tma_load_5d(stage + L::kHalf + off, &P.mv[sJ], &kv_full[st], dh * 64, head, kb.w0, kb.h0, kb.t0);
+          }
+        }
+        ++issued;
+      }
+      mbar_wait(qd_full, 0, status);
+      for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nsteps > 0) {
+      const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
+      const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
+      const uint32_t sQ = smem_u32(sm + L::kQ), sDO = smem_u32(sm + L::kDO);
+      bool ok = mbar_wait_abortable(qd_full, 0, status, abort_flag);
+      auto issue_dq = [&](int i) -> bool {
+        const int pb = i & 1;
+        if (!mbar_wait_abortable(&ds_full[pb], (i >> 1) & 1, status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t sDS = smem_u32(sm + L::kDS0 + pb * L::kDSBytes);
+        const uint32_t sK = smem_u32(sm + L::kStage0 + (i & 1) * L::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+          mma_ws(tdQ, kmajor_desc(sDS, kk, kBoxBytes), mnmajor_desc(sK, kk, kBoxBytes, kKB * kBoxBytes), idQ,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&kv_empty[i & 1]);
+        mma_commit(&ds_free[pb]);
+        return true;
+      };
+      for (int j = 0; j < nsteps && ok; ++j) {
+        const int st = j & 1, sb = j & 1;
+        if (!mbar_wait_abortable(&kv_full[st], (j >> 1) & 1, status, abort_flag)) break;
+        if (!mbar_wait_abortable(&s_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t sK = smem_u32(sm + L::kStage0 + st * L::kStageBytes);
+        const uint32_t sV = sK + L::kHalf;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws(tbase + sb * 64, kmajor_desc(sQ, kk, kBoxBytes), kmajor_desc(sK, kk, kKB * kBoxBytes), idS,
+                 kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws(tbase + 128 + sb * 64, kmajor_desc(sDO, kk, kBoxBytes), kmajor_desc(sV, kk, kKB * kBoxBytes), idS,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(&s_full[sb]);
+        if (j >= 1 && !issue_dq(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) issue_dq(nsteps - 1);
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, status);
+    }
+  } else {
+    const int sw = warp - 2, sp = warp & 3, ch = sw >> 2;
+    const int Ln = sp * 32 + lane;
+    const int m = Ln & 63, kh = Ln >> 6;
+    const uint32_t lane_off = uint32_t(sp * 32) << 16;
+    const float lse2 = P.lse2[size_t(row) * 64 + m];
+    const float dm = P.dvec[size_t(row) * 64 + m];
+    for (int j = 0; j < nsteps; ++j) {
+      const int sb = j & 1;
+      mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
+      tc_fence_after();
+      uint32_t rs[32], rp[32];
+      tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
+      tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
+      const bool valid = (j * kKB + kh) < cnt && lse2 > -INFINITY;
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float d0 = 0.f, d1 = 0.f;
+        if (valid) {
+          const float p0 = fast_exp2(__uint_as_float(rs[2 * i]) * P.scale_log2 - lse2);
+          const float p1 = fast_exp2(__uint_as_float(rs[2 * i + 1]) * P.scale_log2 - lse2);
+          d0 = p0 * (__uint_as_float(rp[2 * i]) - dm);
+          d1 = p1 * (__uint_as_float(rp[2 * i + 1]) - dm);
+        }
+        pk[i] = pack_bf16x2(d0, d1);
+      }
+      if (j >= 2) mbar_wait_abortable(&ds_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag);
+      uint8_t* pt = sm + L::kDS0 + sb * L::kDSBytes + kh * kBoxBytes;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_full[sb]);
+    }
+    if (nsteps > 0) mbar_wait_abortable(&ds_free[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, status, abort_flag);
+    tc_fence_after();
+    const bool ok = *abort_flag == 0;
+    constexpr int NC = D / 4;
+    float v[NC];
+    if (nsteps > 0) {
+      tmem_ld_f<NC>(tdQ + lane_off + ch * NC, v);
+#pragma unroll
+      for (int i = 0; i < NC; ++i) v[i] = ok ? v[i] * P.scale : 0.f;
+    } else {
+#pragma unroll
+      for (int i = 0; i < NC; ++i) v[i] = 0.f;
+    }
+    const int sI = safe_shape(g, P.zone_shape, I, status);
+    const int tok = block_token(g, block_box(g, sI, I), m);
+    store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * (D / 2) + ch * NC, v, P.out_fp32);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// --------------------------------------------------------------------- dkdv
+template <int D>
+struct DkvSmem {
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = D * 128;
+  static constexpr uint32_t kHalf = kKB * D * 128;  // Q (or dO) of one stage
+  static constexpr uint32_t kLD = 2 * kHalf;        // lse2 [slot][64], D [slot][64]
+  static constexpr uint32_t kStageBytes = 2 * kHalf + 1024;
+  static constexpr uint32_t kStage0 = 2 * D * 128;
+  static constexpr uint32_t kPT = kStage0 + 2 * kStageBytes;
+  static constexpr uint32_t kPBytes = kKB * kBoxBytes;
+  static constexpr uint32_t kDST = kPT + kPBytes;
+  static constexpr uint32_t kBar = kDST + kPBytes;
+  static constexpr uint32_t kTotal = kBar + 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_constant__ BwdParams P) {
+  using L = DkvSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* st_full = bars + 1;
+  uint64_t* st_empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_free = bars + 7;
+  uint64_t* ps_full = bars + 9;
+  uint64_t* ps_free = bars + 10;
+  uint64_t* mma_done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
+
+  const Geo& g = P.g;
+  const int J = blockIdx.x, head = blockIdx.y;
+  const int col = head * g.n_blocks + J;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = P.status;
+  const int beg = P.ptr[col];
+  int cnt = P.ptr[col + 1] - beg;
+  if (cnt < 0 || cnt > g.n_blocks) {
+    if (threadIdx.x == 0) atomicOr(status, kDevErrBounds);
+    cnt = 0;
+  }
+  const int nsteps = (cnt + kKB - 1) / kKB;
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&st_full[i], 1);
+      mbar_init(&st_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kSoftWarps);
+    }
+    mbar_init(ps_full, kSoftWarps);
+    mbar_init(ps_free, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tdV = tbase + 256, tdK = tbase + 384;
+
+  if (warp == 0) {
+    if (lane == 0 && nsteps > 0) {
+      const int sJ = safe_shape(g, P.zone_shape, J, status);
+      const BlockBox kb = block_box(g, sJ, J);
+      mbar_arrive_expect_tx(kv_full, 2 * D * 128);
+      for (int dh = 0; dh < D / 64; ++dh) {
+        tma_load_5d(sm + L::kK + dh * kBoxBytes, &P.mk[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
+        tma_load_5d(sm + L::kV + dh * kBoxBytes, &P.mv[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
+      }
+      int issued = 0;
+      for (int j = 0; j < nsteps; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait_abortable(&st_empty[st], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
+        uint8_t* stage = sm + L::kStage0 + st * L::kStageBytes;
+        mbar_arrive_expect_tx(&st_full[st], 2 * L::kHalf + kKB * 2 * 256);
+        for (int slot = 0; slot < kKB; ++slot) {
+          int e = j * kKB + slot;
+          if (e >= cnt) e = j * kKB;
+          int I = P.idx[beg + e];
+          if (I < 0 || I >= g.n_blocks) {
+            atomicOr(status, kDevErrBounds);
+            I = 0;
+          }
+          const int sI = safe_shape(g, P.zone_shape, I, status);
+          const BlockBox qb = block_box(g, sI, I);
+          for (int dh = 0; dh < D / 64; ++dh) {
+            const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
+            tma_load_5d(stage + off, &P.mq[sI], &st_full[st], dh * 64, head, qb.w0, qb.h0, qb.t0);
+            tma_load_5d(stage + L::kHalf + off, &P.mdo[sI], &st_full[st], dh * 64, head, qb.w0, qb.h0, qb.t0);
+          }
+          const size_t rowoff = (size_t(head) * g.n_blocks + I) * 64;
+          bulk_load(stage + L::kLD + slot * 256, P.lse2 + rowoff, 256, &st_full[st]);
+          bulk_load(stage + L::kLD + 512 + slot * 256, P.dvec + rowoff, 256, &st_full[st]);
+        }
+        ++issued;
+      }
+      mbar_wait(kv_full, 0, status);
+      for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i) mbar_wait(&st_full[i & 1], (i >> 1) & 1, status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nsteps > 0) {
+      const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
+      const uint32_t idO = idesc_bf16_f32(64, D, false, true);
+      const uint32_t sK = smem_u32(sm + L::kK), sV = smem_u32(sm + L::kV);
+      const uint32_t sPT = smem_u32(sm + L::kPT), sDST = smem_u32(sm + L::kDST);
+      bool ok = mbar_wait_abortable(kv_full, 0, status, abort_flag);
+      auto issue_kv = [&](int i) -> bool {
+        if (!mbar_wait_abortable(ps_full, i & 1, status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(sm + L::kStage0 + (i & 1) * L::kStageBytes);
+        const uint32_t sDO = sQ + L::kHalf;
+#pragma unroll
+        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+          mma_ws(tdV, kmajor_desc(sPT, kk, kBoxBytes), mnmajor_desc(sDO, kk, kBoxBytes, kKB * kBoxBytes), idO,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+          mma_ws(tdK, kmajor_desc(sDST, kk, kBoxBytes), mnmajor_desc(sQ, kk, kBoxBytes, kKB * kBoxBytes), idO,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&st_empty[i & 1]);
+        mma_commit(ps_free);
+        return true;
+      };
+      for (int j = 0; j < nsteps && ok; ++j) {
+        const int st = j & 1, sb = j & 1;
+        if (!mbar_wait_abortable(&st_full[st], (j >> 1) & 1, status, abort_flag)) break;
+        if (!mbar_wait_abortable(&s_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(sm + L::kStage0 + st * L::kStageBytes);
+        const uint32_t sDO = sQ + L::kHalf;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws(tbase + sb * 64, kmajor_desc(sK, kk, kBoxBytes), kmajor_desc(sQ, kk, kKB * kBoxBytes), idS,
+                 kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws(tbase + 128 + sb * 64, kmajor_desc(sV, kk, kBoxBytes), kmajor_desc(sDO, kk, kKB * kBoxBytes), idS,
+                 kk > 0 ? 1u : 0u);
+        mma_commit(&s_full[sb]);
+        if (j >= 1 && !issue_kv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) issue_kv(nsteps - 1);
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, status);
+    }
+  } else {
+    const int sw = warp - 2, sp = warp & 3, ch = sw >> 2;
+    const int Ln = sp * 32 + lane;
+    const int m = Ln & 63, kh = Ln >> 6;
+    const uint32_t lane_off = uint32_t(sp * 32) << 16;
+    for (int j = 0; j < nsteps; ++j) {
+      const int sb = j & 1;
+      mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
+      tc_fence_after();
+      uint32_t rs[32], rp[32];
+      tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
+      tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
+      const bool valid = (j * kKB + kh) < cnt;
+      // the per-query LSE / D rows arrived by bulk copy on st_full: observe it
+      mbar_wait_abortable(&st_full[sb], (j >> 1) & 1, status, abort_flag);
+      const float* ld = reinterpret_cast<const float*>(sm + L::kStage0 + (j & 1) * L::kStageBytes + L::kLD);
+      const float* l2 = ld + kh * 64 + ch * 32;
+      const float* dd = ld + 128 + kh * 64 + ch * 32;
+      uint32_t pp[16], pd[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+        if (valid) {
+          const float a0 = l2[2 * i], a1 = l2[2 * i + 1];
+          p0 = a0 > -INFINITY ? fast_exp2(__uint_as_float(rs[2 * i]) * P.scale_log2 - a0) : 0.f;
+          p1 = a1 > -INFINITY ? fast_exp2(__uint_as_float(rs[2 * i + 1]) * P.scale_log2 - a1) : 0.f;
+          d0 = p0 * (__uint_as_float(rp[2 * i]) - dd[2 * i]);
+          d1 = p1 * (__uint_as_float(rp[2 * i + 1]) - dd[2 * i + 1]);
+        }
+        pp[i] = pack_bf16x2(p0, p1);
+        pd[i] = pack_bf16x2(d0, d1);
+      }
+      if (j >= 1) mbar_wait_abortable(ps_free, (j - 1) & 1, status, abort_flag);
+      uint8_t* pt = sm + L::kPT + kh * kBoxBytes;
+      uint8_t* dt = sm + L::kDST + kh * kBoxBytes;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
+            make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
+        *reinterpret_cast<uint4*>(dt + sw128_offset(m, ch * 4 + q)) =
+            make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ps_full);
+    }
+    if (nsteps > 0) mbar_wait_abortable(ps_free, (nsteps - 1) & 1, status, abort_flag);
+    tc_fence_after();
+    const bool ok = *abort_flag == 0;
+    constexpr int NC = D / 4;
+    float vv[NC], vk[NC];
+    if (nsteps > 0) {
+      tmem_ld_f<NC>(tdV + lane_off + ch * NC, vv);
+      tmem_ld_f<NC>(tdK + lane_off + ch * NC, vk);
+#pragma unroll
+      for (int i = 0; i < NC; ++i) {
+        vv[i] = ok ? vv[i] : 0.f;
+        vk[i] = ok ? vk[i] * P.scale : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NC; ++i) vv[i] = vk[i] = 0.f;
+    }
+    const int sJ = safe_shape(g, P.zone_shape, J, status);
+    const int tok = block_token(g, block_box(g, sJ, J), m);
+    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * (D / 2) + ch * NC;
+    store_row<NC>(P.out0, off, vk, P.out_fp32);
+    store_row<NC>(P.out1, off, vv, P.out_fp32);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// --------------------------------------------------------------------- prep
+template <typename T>
+__device__ __forceinline__ float dot_chunk(const T* a, const T* b, int n);
+template <>
+__device__ __forceinline__ float dot_chunk<__nv_bfloat16>(const __nv_bfloat16* a, const __nv_bfloat16* b, int n) {
+  float s = 0.f;
+  for (int i = 0; i < n; i += 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(a + i);
+    const uint4 v = *reinterpret_cast<const uint4*>(b + i);
+    const uint32_t x[4] = {u.x, u.y, u.z, u.w}, y[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      s = fmaf(__uint_as_float(x[q] << 16), __uint_as_float(y[q] << 16), s);
+      s = fmaf(__uint_as_float(x[q] & 0xFFFF0000u), __uint_as_float(y[q] & 0xFFFF0000u), s);
+    }
+  }
+  return s;
+}
+template <>
+__device__ __forceinline__ float dot_chunk<float>(const float* a, const float* b, int n) {
+  float s = 0.f;
+  for (int i = 0; i < n; i += 4) {
+    const float4 u = *reinterpret_cast<const float4*>(a + i);
+    const float4 v = *reinterpret_cast<const float4*>(b + i);
+    s = fmaf(u.x, v.x, fmaf(u.y, v.y, fmaf(u.z, v.z, fmaf(u.w, v.w, s))));
+  }
+  return s;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const Geo g, const int32_t* __restrict__ zone_shape,
+                                                       const T* __restrict__ o, const T* __restrict__ dout,
+                                                       int64_t tok_stride, int head_dim, const float* __restrict__ lse,
+                                                       float* __restrict__ lse2_blk, float* __restrict__ d_blk,
+                                                       int* status) {
+  const int b = blockIdx.x, head = blockIdx.y;
+  const int r = threadIdx.x >> 2, part = threadIdx.x & 3;
+  const int s = safe_shape(g, zone_shape, b, status);
+  const int tok = block_token(g, block_box(g, s, b), r);
+  const int n = head_dim / 4;
+  const int64_t off = int64_t(tok) * tok_stride + int64_t(head) * head_dim + part * n;
+  float acc = dot_chunk<T>(o + off, dout + off, n);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  if (part == 0) {
+    const size_t at = (size_t(head) * g.n_blocks + b) * 64 + r;
+    d_blk[at] = acc;
+    const int N = g.T * g.H * g.W;
+    lse2_blk[at] = lse[int64_t(head) * N + tok] * 1.4426950408889634f;
+  }
+}
+
+// ---------------------------------------------------------------------- CSC
+__global__ void __launch_bounds__(256) csc_scatter_kernel(const int32_t* __restrict__ row_ptr,
+                                                          const int32_t* __restrict__ col_idx, int heads, int nb,
+                                                          uint32_t* __restrict__ tmask, int* status) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (row >= heads * nb) return;
+  const int head = row / nb, I = row - head * nb;
+  const int words = (nb + 31) >> 5;
+  const int b = row_ptr[row], e = row_ptr[row + 1];
+  for (int k = b + lane; k < e; k += 32) {
+    const int J = col_idx[k];
+    if (J < 0 || J >= nb) {
+      atomicOr(status, kDevErrBounds);
+      continue;
+    }
+    atomicOr(&tmask[(size_t(head) * nb + J) * words + (I >> 5)], 1u << (I & 31));
+  }
+}
+
+__global__ void __launch_bounds__(256) popc_rows_kernel(const uint32_t* __restrict__ mask, int rows, int words,
+                                                        int32_t* __restrict__ cnt) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  int c = 0;
+  for (int w = lane; w < words; w += 32) c += __popc(mask[size_t(row) * words + w]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) cnt[row] = c;
+}
+
+struct BwdWs {
+  size_t stage_q, stage_k, stage_v, stage_do, lse2, dvec, tmask, ccnt, cptr, ridx, total;
+};
+
+BwdWs bwd_ws_layout(const Geo& g, int heads, int head_dim, prism_dtype dtype, int64_t nnz) {
+  WsCarver c;
+  BwdWs w{};
+  if (dtype == PRISM_FP32) {
+    const size_t t = size_t(g.T) * g.H * g.W * heads * head_dim * 2;
+    w.stage_q = c.take(t);
+    w.stage_k = c.take(t);
+    w.stage_v = c.take(t);
+    w.stage_do = c.take(t);
+  }
+  const size_t rows = size_t(heads) * g.n_blocks;
+  w.lse2 = c.take(rows * 64 * 4);
+  w.dvec = c.take(rows * 64 * 4);
+  w.tmask = c.take(rows * ((g.n_blocks + 31) / 32) * 4);
+  w.ccnt = c.take(rows * 4);
+  w.cptr = c.take((rows + 1) * 4);
+  w.ridx = c.take(size_t(nnz > 0 ? nnz : 1) * 4);
+  w.total = c.off;
+  return w;
+}
+
+}  // namespace
+
+prism_status stage_bf16(const void* src, prism_dtype dtype, int64_t tok_stride, int C, int64_t n_tokens,
+                        __nv_bfloat16* dst, cudaStream_t s);
+
+size_t bsa_bwd_ws_bytes(const Geo& g, int heads, int head_dim, prism_dtype dtype, int64_t nnz) {
+  return bwd_ws_layout(g, heads, head_dim, dtype, nnz).total;
+}
+
+}  // namespace prism
+
+using namespace prism;
+
+extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q,
+                                      const void* k, const void* v, const void* o, const float* lse,
+                                      const void* dout, prism_dtype dtype, int32_t heads, int32_t head_dim,
+                                      int64_t tok_stride, float scale, const int32_t* row_ptr,
+                                      const int32_t* col_idx, int64_t nnz, void* dq, void* dk, void* dv, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  Geo g;
+  prism_status st = make_geo(geo, &g);
+  if (st != PRISM_OK) return st;
+  if (!zone_shape || !q || !k || !v || !o || !lse || !dout || !row_ptr || !col_idx || !dq || !dk || !dv)
+    return PRISM_ERR_ARG;
+  if (dtype != PRISM_BF16 && dtype != PRISM_FP32) return PRISM_ERR_DTYPE;
+  if (head_dim != 64 && head_dim != 128) return PRISM_ERR_UNSUPPORTED;
+  if (heads < 1 || heads > 65535) return PRISM_ERR_UNSUPPORTED;
+  if (tok_stride < int64_t(heads) * head_dim || tok_stride % 8) return PRISM_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return PRISM_ERR_ARG;
+  if (nnz < 0 || nnz > int64_t(heads) * g.n_blocks * g.n_blocks) return PRISM_ERR_ARG;
+  for (const void* p : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                        static_cast<const void*>(dv)})
+    if (reinterpret_cast<uintptr_t>(p) % 16) return PRISM_ERR_ARG;
+  const BwdWs W = bwd_ws_layout(g, heads, head_dim, dtype, nnz);
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < W.total) return PRISM_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  int* status = ws_status(ws);
+  const int64_t N = int64_t(g.T) * g.H * g.W;
+  const int C = heads * head_dim;
+  const void *qb = q, *kb = k, *vb = v, *dob = dout;
+  int64_t in_stride = tok_stride;
+  if (dtype == PRISM_FP32) {
+    auto* sq = reinterpret_cast<__nv_bfloat16*>(w8 + W.stage_q);
+    auto* sk = reinterpret_cast<__nv_bfloat16*>(w8 + W.stage_k);
+    auto* sv = reinterpret_cast<__nv_bfloat16*>(w8 + W.stage_v);
+    auto* sdo = reinterpret_cast<__nv_bfloat16*>(w8 + W.stage_do);
+    if ((st = stage_bf16(q, dtype, tok_stride, C, N, sq, s)) != PRISM_OK) return st;
+    if ((st = stage_bf16(k, dtype, tok_stride, C, N, sk, s)) != PRISM_OK) return st;
+    if ((st = stage_bf16(v, dtype, tok_stride, C, N, sv, s)) != PRISM_OK) return st;
+    if ((st = stage_bf16(dout, dtype, tok_stride, C, N, sdo, s)) != PRISM_OK) return st;
+    qb = sq; kb = sk; vb = sv; dob = sdo;
+    in_stride = C;
+  }
+  float* lse2 = reinterpret_cast<float*>(w8 + W.lse2);
+  float* dvec = reinterpret_cast<float*>(w8 + W.dvec);
+  uint32_t* tmask = reinterpret_cast<uint32_t*>(w8 + W.tmask);
+  int32_t* ccnt = reinterpret_cast<int32_t*>(w8 + W.ccnt);
+  int32_t* cptr = reinterpret_cast<int32_t*>(w8 + W.cptr);
+  int32_t* ridx = reinterpret_cast<int32_t*>(w8 + W.ridx);
+  const dim3 grid(g.n_blocks, heads);
+  if (dtype == PRISM_BF16)
+    bwd_prep_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g, zone_shape, static_cast<const __nv_bfloat16*>(o),
+                                                        static_cast<const __nv_bfloat16*>(dout), tok_stride, head_dim,
+                                                        lse, lse2, dvec, status);
+  else
+    bwd_prep_kernel<float><<<grid, 256, 0, s>>>(g, zone_shape, static_cast<const float*>(o),
+                                                static_cast<const float*>(dout), tok_stride, head_dim, lse, lse2,
+                                                dvec, status);
+  const int rows = heads * g.n_blocks;
+  const int words = (g.n_blocks + 31) / 32;
+  if (cudaMemsetAsync(tmask, 0, size_t(rows) * words * 4, s) != cudaSuccess) return PRISM_ERR_CUDA;
+  csc_scatter_kernel<<<unsigned((int64_t(rows) * 32 + 255) / 256), 256, 0, s>>>(row_ptr, col_idx, heads, g.n_blocks,
+                                                                                 tmask, status);
+  popc_rows_kernel<<<unsigned((int64_t(rows) * 32 + 255) / 256), 256, 0, s>>>(tmask, rows, words, ccnt);
+  if (launch_exclusive_scan(ccnt, rows, cptr, s) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (launch_mask_to_lists(tmask, cptr, rows, g.n_blocks, nnz, ridx, status, s) != cudaSuccess) return PRISM_ERR_CUDA;
+
+  BwdParams P;
+  std::memset(&P, 0, sizeof(P));
+  for (int c = 0; c < g.n_cand; ++c) {
+    const int bt = g.cand[c][0], bh = g.cand[c][1], bw = g.cand[c][2];
+    if ((st = encode_block_map(&P.mq[c], qb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+    if ((st = encode_block_map(&P.mk[c], kb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+    if ((st = encode_block_map(&P.mv[c], vb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+    if ((st = encode_block_map(&P.mdo[c], dob, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+  }
+  P.g = g;
+  P.zone_shape = zone_shape;
+  P.lse2 = lse2;
+  P.dvec = dvec;
+  P.status = status;
+  P.tok_stride = tok_stride;
+  P.scale_log2 = scale * 1.4426950408889634f;
+  P.scale = scale;
+  P.out_fp32 = dtype == PRISM_FP32;
+  // dQ: q-stationary over the CSR
+  P.ptr = row_ptr;
+  P.idx = col_idx;
+  P.out0 = dq;
+  P.out1 = nullptr;
+  if (head_dim == 128) {
+    const size_t smem = DqSmem<128>::kTotal + 1024;
+    if (cudaFuncSetAttribute(bsa_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+    bsa_dq_kernel<128><<<grid, kBwdThreads, smem, s>>>(P);
+  } else {
+    const size_t smem = DqSmem<64>::kTotal + 1024;
+    if (cudaFuncSetAttribute(bsa_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+    bsa_dq_kernel<64><<<grid, kBwdThreads, smem, s>>>(P);
+  }
+  if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
+  // dK, dV: kv-stationary over the CSC
+  P.ptr = cptr;
+  P.idx = ridx;
+  P.out0 = dk;
+  P.out1 = dv;
+  if (head_dim == 128) {
+    const size_t smem = DkvSmem<128>::kTotal + 1024;
+    if (cudaFuncSetAttribute(bsa_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return PRISM_ERR_CUDA;
+    bsa_dkdv_kernel<128><<<grid, kBwdThreads, smem, s>>>(P);
+  } else {
+    const size_t smem = DkvSmem<64>::kTotal + 1024;
+    if (cudaFuncSetAttribute(bsa_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return PRISM_ERR_CUDA;
+    bsa_dkdv_kernel<64><<<grid, kBwdThreads, smem, s>>>(P);
+  }
+  return cuda_status(cudaGetLastError());
+}

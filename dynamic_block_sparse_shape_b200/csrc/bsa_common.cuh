@@ -1,0 +1,87 @@
+// Pieces shared by the block-sparse attention kernels (forward and backward).
+//
+// Tiles. A 64-token block of one head is gathered by TMA as head_dim/64 boxes
+// of (64 channels, 1 head, bw, bh, bt) from the token-major tensor; each box
+// lands as 64 rows x 128 bytes with the 128-byte swizzle (8-row atoms of 1 KB),
+// rows in raster (t, h, w) order, i.e. the K-major operand layout of tcgen05.
+//
+// MMA shape. A query block has 64 rows. tcgen05.mma with M = 64 runs at half
+// rate, while the weight-stationary form (.ws) with M = 64 uses the full
+// 128-lane datapath by splitting N over the two lane halves: accumulator
+// element (m, n) of an M=64 x N tile sits at TMEM lane m + 64 * (n >= N/2),
+// column n mod N/2. Every product here is .ws M = 64 with fp32 accumulation.
+#pragma once
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace prism {
+
+constexpr int kBoxBytes = 64 * 128;  // one 64-row x 128-byte swizzled box
+
+__device__ __forceinline__ void mma_ws(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.ws.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// K-major descriptor for the k-th 16-element step of a [n_box][rows][128 B]
+// operand whose boxes sit box_stride bytes apart (64 channels per box).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kstep, uint32_t box_stride) {
+  return sdesc_sw128(base + uint32_t(kstep >> 2) * box_stride + uint32_t(kstep & 3) * 32u, 16, 1024);
+}
+
+// MN-major descriptor for the k-th 16-row step of an operand made of 64-row
+// x 128-byte boxes whose rows run along the contraction index: box
+// (slot, n_box) sits at base + slot * slot_stride + n_box * n_stride, where a
+// slot covers 64 contraction rows and n_box the 64-column slices along N.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kstep, uint32_t slot_stride, uint32_t n_stride) {
+  return sdesc_sw128(base + uint32_t(kstep >> 2) * slot_stride + uint32_t(kstep & 3) * 2048u, n_stride, 1024);
+}
+
+__device__ __forceinline__ int safe_shape(const Geo& g, const int32_t* zone_shape, int b, int* status) {
+  int s = zone_shape[b / g.bpz];
+  if (s < 0 || s >= g.n_cand) {
+    atomicOr(status, kDevErrBounds);
+    s = 0;
+  }
+  return s;
+}
+
+// Store 32 (or 16) fp32 values as bf16 or fp32 at dst (16-byte aligned).
+template <int NC>
+__device__ __forceinline__ void store_row(void* dst, int64_t off, const float* v, bool fp32) {
+  if (fp32) {
+    float4* d = reinterpret_cast<float4*>(static_cast<float*>(dst) + off);
+#pragma unroll
+    for (int i = 0; i < NC / 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + off);
+#pragma unroll
+    for (int i = 0; i < NC / 8; ++i)
+      d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                        pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  }
+}
+
+// TMEM load of NC (32 or 16) consecutive columns into floats.
+template <int NC>
+__device__ __forceinline__ void tmem_ld_f(uint32_t taddr, float* v) {
+  uint32_t r[NC];
+  if constexpr (NC == 32) tmem_ld32(taddr, r);
+  else tmem_ld16(taddr, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < NC; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace prism

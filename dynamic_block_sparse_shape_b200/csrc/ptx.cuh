@@ -8,14 +8,9 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-namespace prism {
+#include "common.cuh"
 
-// Error bits written into the device status word.
-enum : int {
-  kDevErrTimeout = 1,   // an mbarrier wait gave up
-  kDevErrBounds = 2,    // an index fell outside its buffer (skipped)
-  kDevErrCapacity = 4,  // a list outgrew its buffer (truncated)
-};
+namespace prism {
 
 // Wall-clock limit of one bounded wait, in nanoseconds (about 2 s).
 #ifndef PRISM_WAIT_LIMIT_NS
@@ -72,6 +67,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// Bounded wait that gives up at once when another warp of the CTA already
+// gave up (`abort` is a shared-memory flag), and raises the flag on its own
+// timeout. Keeps every warp's control flow (named barriers, step counts)
+// identical while bounding the total time spent after a failure.
+// A timeout anywhere on the device (the kDevErrTimeout bit of *status) also
+// makes every later wait give up at once, so a systematic failure costs one
+// wait limit, not one per CTA.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t parity, int* status,
+                                                    volatile int* abort) {
+  if (*abort) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  if (*reinterpret_cast<volatile int*>(status) & kDevErrTimeout) {
+    *abort = 1;
+    return false;
+  }
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (*reinterpret_cast<volatile int*>(status) & kDevErrTimeout) {
+      *abort = 1;
+      return false;
+    }
+    if (global_timer_ns() - t0 > PRISM_WAIT_LIMIT_NS) {
+      atomicOr(status, kDevErrTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -107,6 +134,16 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Untiled bulk copy global -> shared (16-byte aligned addresses, size a
+// multiple of 16), completion counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

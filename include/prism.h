@@ -44,6 +44,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define PRISM_API __attribute__((visibility("default")))
+#else
+#define PRISM_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -94,26 +100,26 @@ typedef enum {
 } prism_op;
 
 /* Human-readable name of a status. Never NULL. */
-const char* prism_status_string(prism_status s);
+PRISM_API const char* prism_status_string(prism_status s);
 
 /* Library version, major*10000 + minor*100 + patch. */
-int32_t prism_version(void);
+PRISM_API int32_t prism_version(void);
 
 /* Number of zones and of blocks for a geometry (host only, no GPU work). */
-prism_status prism_geometry_counts(const prism_geometry* geo, int32_t* n_zones, int32_t* n_blocks);
+PRISM_API prism_status prism_geometry_counts(const prism_geometry* geo, int32_t* n_zones, int32_t* n_blocks);
 
 /* Workspace bytes needed by `op`. `nnz` is the number of selected
  * (query block, key block) pairs summed over heads (row_ptr[heads*n_blocks]),
  * used by PRISM_OP_BSA_BWD only. `in_dtype` is the dtype of Q/K/V (fp32
  * inputs need bf16 staging copies). Host only. */
-prism_status prism_workspace_size(prism_op op, const prism_geometry* geo, int32_t heads, int32_t head_dim,
+PRISM_API prism_status prism_workspace_size(prism_op op, const prism_geometry* geo, int32_t heads, int32_t head_dim,
                                   int32_t feat_c, int32_t res_c, prism_dtype in_dtype, int64_t nnz,
                                   size_t* bytes);
 
 /* Reads and clears the device status word kept in `ws` (synchronises
  * `stream`). Returns PRISM_ERR_TIMEOUT or PRISM_ERR_DEVICE if a kernel that
  * used this workspace reported one, else PRISM_OK. */
-prism_status prism_check_device_status(void* ws, void* stream);
+PRISM_API prism_status prism_check_device_status(void* ws, void* stream);
 
 /*
  * a1 + a2 — macro-zone tiling and per-zone block shape.
@@ -143,7 +149,7 @@ prism_status prism_check_device_status(void* ws, void* stream);
  * zone_margin: device float [n_zones] out (second-best minus best cost), or
  *       NULL.
  */
-prism_status prism_zone_shapes(const prism_geometry* geo, const void* feat, int64_t feat_ld, int32_t feat_c,
+PRISM_API prism_status prism_zone_shapes(const prism_geometry* geo, const void* feat, int64_t feat_ld, int32_t feat_c,
                                prism_dtype feat_dtype, const void* res, int64_t res_ld, int32_t res_c,
                                prism_dtype res_dtype, const prism_shape_params* params, int32_t* zone_shape,
                                float* zone_margin, void* ws, size_t ws_bytes, void* stream);
@@ -155,11 +161,14 @@ prism_status prism_zone_shapes(const prism_geometry* geo, const void* feat, int6
  * zone_shape: device int32 [n_zones] (from prism_zone_shapes).
  * q, k: device [N, heads, head_dim], bf16 or fp32, token stride tok_stride.
  * q_pool, k_pool: device float [heads, n_blocks, head_dim] out.
- * head_dim is 64 or 128.
+ * head_dim is 64 or 128; heads * head_dim <= 8192.
+ * ws: workspace of at least prism_workspace_size(PRISM_OP_BLOCK_SELECT, ...)
+ *       bytes; only its status word is used (an out-of-range zone_shape entry
+ *       leaves that block's pooled rows as NaN and reports PRISM_ERR_DEVICE).
  */
-prism_status prism_block_pool(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
+PRISM_API prism_status prism_block_pool(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
                               prism_dtype dtype, int32_t heads, int32_t head_dim, int64_t tok_stride, float* q_pool,
-                              float* k_pool, void* stream);
+                              float* k_pool, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * a4 + a5 — block scoring and hybrid selection (walkthrough section
@@ -189,10 +198,22 @@ prism_status prism_block_pool(const prism_geometry* geo, const int32_t* zone_sha
  *       needs total_kept != NULL; without it the fill clips at col_cap and
  *       reports PRISM_ERR_DEVICE through prism_check_device_status).
  */
-prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
+PRISM_API prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
                                 int32_t head_dim, float scale, int32_t top_k, float cdf_threshold, uint32_t* mask,
                                 int32_t* kept, int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
                                 int64_t* total_kept, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Expands a selection bitmask (as written by prism_block_select) into the
+ * CSR column lists: col_idx[row_ptr[r] .. row_ptr[r+1]) = the set bits of row
+ * r, ascending. Use it after a prism_block_select call made with
+ * col_idx = NULL and total_kept to size col_idx. Rows past col_cap are left
+ * unwritten and reported through prism_check_device_status.
+ * mask: device uint32 [rows, ceil(n_blocks/32)]; row_ptr: device int32
+ * [rows+1]; col_idx: device int32 [col_cap] out.
+ */
+PRISM_API prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* row_ptr, int32_t rows, int32_t n_blocks,
+                                         int32_t* col_idx, int64_t col_cap, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * a6 — block-sparse attention forward (Sol-Attn abstract: compute only the
@@ -209,7 +230,7 @@ prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_
  * o: device [N, heads, head_dim] out, same dtype as q, token stride tok_stride.
  * lse: device float [heads, N] out.
  */
-prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
+PRISM_API prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
                            const void* v, prism_dtype dtype, int32_t heads, int32_t head_dim, int64_t tok_stride,
                            float scale, const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
                            void* ws, size_t ws_bytes, void* stream);
@@ -224,7 +245,7 @@ prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape,
  * device [N, heads, head_dim]; dq, dk, dv are device outs like q. nnz =
  * row_ptr[heads*n_blocks] (for workspace sizing; checked against ws_bytes).
  */
-prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
+PRISM_API prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
                            const void* v, const void* o, const float* lse, const void* dout, prism_dtype dtype,
                            int32_t heads, int32_t head_dim, int64_t tok_stride, float scale, const int32_t* row_ptr,
                            const int32_t* col_idx, int64_t nnz, void* dq, void* dk, void* dv, void* ws,

@@ -298,30 +298,35 @@ def token_mask(block_mask, blocks, n_tokens):
 
 def masked_attention_fwd(Q, K, V, allowed, scale):
     """O [N, heads, d] and LSE [heads, N] of softmax attention with logits
-    scale * q.k set to -inf where ``allowed`` is False."""
-    Q, K, V = (np.asarray(x, np.float64) for x in (Q, K, V))
-    S = scale * np.einsum("ihd,jhd->hij", Q, K)
+    scale * q.k set to -inf where ``allowed`` is False. A query with no allowed
+    key (an empty selection, which the hybrid rule never produces since
+    k >= 1) gets O = 0 and LSE = -inf, and contributes no gradient."""
+    Qh, Kh, Vh = (np.asarray(x, np.float64).transpose(1, 0, 2) for x in (Q, K, V))  # [heads, N, d]
+    S = scale * (Qh @ Kh.transpose(0, 2, 1))
     S = np.where(allowed, S, -np.inf)
-    mx = S.max(axis=-1, keepdims=True)
+    empty = ~np.asarray(allowed).any(axis=-1, keepdims=True)  # a query with no selected key
+    mx = np.where(empty, 0.0, S.max(axis=-1, keepdims=True))
     P = np.exp(S - mx)
     l = P.sum(axis=-1, keepdims=True)
-    O = np.einsum("hij,jhd->ihd", P / l, V)
-    lse = (mx + np.log(l))[..., 0]
+    O = (np.where(empty, 0.0, P / np.where(empty, 1.0, l)) @ Vh).transpose(1, 0, 2)
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, mx + np.log(l))[..., 0]
     return O, lse
 
 
 def masked_attention_bwd(Q, K, V, O, lse, dO, allowed, scale):
     """dQ, dK, dV of the masked attention with the mask held fixed."""
-    Q, K, V, O, dO = (np.asarray(x, np.float64) for x in (Q, K, V, O, dO))
-    S = scale * np.einsum("ihd,jhd->hij", Q, K)
-    P = np.where(allowed, np.exp(S - np.asarray(lse, np.float64)[..., None]), 0.0)
-    dV = np.einsum("hij,ihd->jhd", P, dO)
-    dP = np.einsum("ihd,jhd->hij", dO, V)
-    D = np.einsum("ihd,ihd->hi", dO, O)
+    Qh, Kh, Vh, Oh, dOh = (np.asarray(x, np.float64).transpose(1, 0, 2) for x in (Q, K, V, O, dO))
+    S = scale * (Qh @ Kh.transpose(0, 2, 1))
+    with np.errstate(over="ignore", invalid="ignore"):
+        P = np.where(allowed, np.exp(S - np.asarray(lse, np.float64)[..., None]), 0.0)
+    dV = P.transpose(0, 2, 1) @ dOh
+    dP = dOh @ Vh.transpose(0, 2, 1)
+    D = (dOh * Oh).sum(axis=-1)
     dS = P * (dP - D[..., None])
-    dQ = scale * np.einsum("hij,jhd->ihd", dS, K)
-    dK = scale * np.einsum("hij,ihd->jhd", dS, Q)
-    return dQ, dK, dV
+    dQ = scale * (dS @ Kh)
+    dK = scale * (dS.transpose(0, 2, 1) @ Qh)
+    return dQ.transpose(1, 0, 2), dK.transpose(1, 0, 2), dV.transpose(1, 0, 2)
 
 
 # --------------------------------------------------------------------------

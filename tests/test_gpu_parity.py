@@ -1,0 +1,244 @@
+"""GPU parity: every C-ABI entry point against the fp64 CPU oracle.
+
+Inputs come from the seeded generators in dynamic_block_sparse_shape_b200.synth
+(or plain seeded torch draws) and are shared by both sides; expected values are
+computed by ``oracle/`` only. Integer outputs (zone shapes, block masks, CSR)
+are compared bit-exactly where the oracle's margins say the answer is robust
+to rounding; floating outputs within max-abs 2e-2 / mean-abs 2e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dynamic_block_sparse_shape_b200 as P
+from dynamic_block_sparse_shape_b200 import synth
+from oracle import prism_oracle as O
+from tests.gpu_util import (CDF_MARGIN, LOGIT_GAP, assert_close, csr_from_mask, f64, mask_bits_to_bool,
+                            require_gpu, scale_for)
+
+pytestmark = pytest.mark.gpu
+
+CAND = tuple(synth.DEFAULT_CANDIDATES)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _oracle_attention(q, k, v, do, blocks, mask, scale):
+    N = q.shape[0]
+    allowed = O.token_mask(mask, blocks, N)
+    Oo, lse = O.masked_attention_fwd(q, k, v, allowed, scale)
+    dq, dk, dv = O.masked_attention_bwd(q, k, v, Oo, lse, do, allowed, scale)
+    return Oo, lse, dq, dk, dv
+
+
+def _check_attention(geo, zone_shape_np, q, k, v, do, mask, with_bwd=True):
+    """Run bsa_fwd / bsa_bwd on the CSR of `mask` and compare with the oracle."""
+    dev = q.device
+    H, d = q.shape[1], q.shape[2]
+    sc = scale_for(d)
+    blocks = O.block_tokens(geo.grid, geo.zone, geo.cand, zone_shape_np)
+    zs = torch.tensor(zone_shape_np, dtype=torch.int32, device=dev)
+    row_ptr, col_idx, nnz = csr_from_mask(mask, dev)
+    ws = P.Workspace(dev)
+    o, lse = P.bsa_fwd(geo, zs, q, k, v, sc, row_ptr, col_idx, ws=ws)
+    qd, kd, vd, dod = (f64(t) for t in (q, k, v, do))
+    Or, lser, dqr, dkr, dvr = _oracle_attention(qd, kd, vd, dod, blocks, mask, sc)
+    res = {"O": assert_close("O", f64(o), Or)}
+    lse_g = f64(lse)
+    fin = np.isfinite(lser)
+    assert np.array_equal(np.isfinite(lse_g), fin)
+    res["lse"] = assert_close("LSE", lse_g[fin], lser[fin])
+    if with_bwd:
+        dq, dk, dv = P.bsa_bwd(geo, zs, q, k, v, o, lse, do, sc, row_ptr, col_idx, nnz, ws=ws)
+        res["dQ"] = assert_close("dQ", f64(dq), dqr)
+        res["dK"] = assert_close("dK", f64(dk), dkr)
+        res["dV"] = assert_close("dV", f64(dv), dvr)
+    P.check_device_status(ws)
+    return res
+
+
+# --------------------------------------------------------------------------- tiny
+def test_tiny_end_to_end():
+    """The fixed-shape fp32 workload: grid 4x8x8, one zone, (4,4,4), k=1, tau=0.2."""
+    wl = synth.WORKLOADS["tiny"]
+    x = synth.qkv(wl)  # CPU generator, fp32
+    dev = torch.device("cuda")
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    geo = P.Geometry(wl.grid, wl.zone, tuple(synth.candidates_for(wl)))
+    ws = P.Workspace(dev)
+    zs, margin = P.zone_shapes(geo, ws=ws)
+    idx_r, _, _ = O.zone_shapes(wl.grid, wl.zone, geo.cand)
+    assert np.array_equal(zs.cpu().numpy(), idx_r)
+    qp, kp = P.block_pool(geo, zs, q, k, ws=ws)
+    blocks = O.block_tokens(wl.grid, wl.zone, geo.cand, idx_r)
+    qpr, kpr = O.block_pool(f64(q), blocks), O.block_pool(f64(k), blocks)
+    assert np.abs(f64(qp) - qpr).max() < 1e-5 and np.abs(f64(kp) - kpr).max() < 1e-5
+    sc = scale_for(wl.head_dim)
+    sel = P.block_select(qp, kp, sc, wl.top_k, wl.cdf_threshold, ws=ws)
+    ref = O.block_select(qpr, kpr, sc, wl.top_k, wl.cdf_threshold)
+    got = mask_bits_to_bool(sel["mask"], blocks.shape[0])
+    assert np.array_equal(got, ref["mask"])
+    assert np.array_equal(sel["kept"].cpu().numpy(), ref["kept"])
+    # the GPU CSR lists the oracle's kept blocks in ascending order
+    rp = sel["row_ptr"].cpu().numpy()
+    ci = sel["col_idx"].cpu().numpy()
+    H, nb = ref["kept"].shape
+    for r in range(H * nb):
+        assert ci[rp[r]:rp[r + 1]].tolist() == np.nonzero(ref["mask"].reshape(H * nb, nb)[r])[0].tolist()
+    _check_attention(geo, idx_r, q, k, v, do, ref["mask"])
+
+
+# --------------------------------------------------------------------------- attention
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("density", [0.12, 0.5, 1.0])
+def test_attention_random_masks_all_shapes(d, density):
+    """Every candidate shape in use, ragged rows (odd counts, one empty row)."""
+    grid, zone = (8, 16, 24), (8, 8, 8)
+    geo = P.Geometry(grid, zone, CAND)
+    nz, nb = geo.counts()
+    rng = np.random.default_rng(int(1000 * density) + d)
+    zone_shape = np.arange(nz) % len(CAND)
+    rng.shuffle(zone_shape)
+    H = 2
+    mask = rng.random((H, nb, nb)) < density
+    mask[:, np.arange(nb), rng.integers(0, nb, nb)] = True
+    mask[0, 3, :] = False  # an empty row
+    mask[1, 5, :] = False
+    mask[1, 5, 7] = True  # a single-block row
+    gen = torch.Generator().manual_seed(7 + d)
+    N = geo.n_tokens
+    dev = torch.device("cuda")
+    q, k, v, do = (torch.randn((N, H, d), generator=gen).to(torch.bfloat16).to(dev) for _ in range(4))
+    _check_attention(geo, zone_shape, q, k, v, do, mask)
+
+
+def test_attention_strided_tokens():
+    """Q/K/V/O as views with a token stride larger than heads*head_dim."""
+    grid, zone = (8, 8, 16), (8, 8, 8)
+    geo = P.Geometry(grid, zone, CAND)
+    nz, nb = geo.counts()
+    H, d = 2, 128
+    N = geo.n_tokens
+    rng = np.random.default_rng(3)
+    zone_shape = np.array([1, 5])
+    mask = rng.random((H, nb, nb)) < 0.4
+    mask[:, np.arange(nb), np.arange(nb)] = True
+    dev = torch.device("cuda")
+    gen = torch.Generator().manual_seed(11)
+    base = torch.randn((N, 4, H, d), generator=gen).to(torch.bfloat16).to(dev)  # packed q|k|v|do
+    q, k, v, do = base[:, 0], base[:, 1], base[:, 2], base[:, 3]
+    blocks = O.block_tokens(grid, zone, CAND, zone_shape)
+    zs = torch.tensor(zone_shape, dtype=torch.int32, device=dev)
+    row_ptr, col_idx, nnz = csr_from_mask(mask, dev)
+    sc = scale_for(d)
+    o = torch.empty((N, 4, H, d), dtype=torch.bfloat16, device=dev)[:, 1]
+    o, lse = P.bsa_fwd(geo, zs, q, k, v, sc, row_ptr, col_idx, out=o)
+    Or, lser, _, _, _ = _oracle_attention(f64(q), f64(k), f64(v), f64(do), blocks, mask, sc)
+    assert_close("O strided", f64(o), Or)
+
+
+# --------------------------------------------------------------------------- pooling
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_block_pool_all_shapes(dtype):
+    grid, zone = (16, 16, 24), (8, 8, 8)
+    geo = P.Geometry(grid, zone, CAND)
+    nz, nb = geo.counts()
+    zone_shape = np.arange(nz) % len(CAND)
+    H, d = 24, 128
+    gen = torch.Generator().manual_seed(5)
+    dev = torch.device("cuda")
+    q = torch.randn((geo.n_tokens, H, d), generator=gen).to(dtype).to(dev)
+    k = torch.randn((geo.n_tokens, H, d), generator=gen).to(dtype).to(dev)
+    zs = torch.tensor(zone_shape, dtype=torch.int32, device=dev)
+    qp, kp = P.block_pool(geo, zs, q, k)
+    blocks = O.block_tokens(grid, zone, CAND, zone_shape)
+    assert np.abs(f64(qp) - O.block_pool(f64(q), blocks)).max() < 2e-6
+    assert np.abs(f64(kp) - O.block_pool(f64(k), blocks)).max() < 2e-6
+
+
+# --------------------------------------------------------------------------- selection
+def _selection_parity(qp, kp, sc, top_k, tau):
+    sel = P.block_select(qp, kp, sc, top_k, tau)
+    H, nb, _ = qp.shape
+    ref = O.block_select(f64(qp), f64(kp), sc, top_k, tau)
+    got = mask_bits_to_bool(sel["mask"], nb)
+    kept = sel["kept"].cpu().numpy()
+    qual = (ref["gap"] > LOGIT_GAP) & (ref["margin"] > CDF_MARGIN)
+    assert np.array_equal(got[qual], ref["mask"][qual])
+    assert np.array_equal(kept[qual], ref["kept"][qual])
+    # every row: kept >= k, popcount == kept, and any difference from the
+    # oracle lies among blocks whose logits are within LOGIT_GAP of the boundary
+    assert np.all(kept >= min(top_k, nb))
+    assert np.array_equal(got.sum(axis=2), kept)
+    s = O.block_logits(f64(qp), f64(kp), sc)
+    for h, i in zip(*np.nonzero(~qual)):
+        diff = got[h, i] ^ ref["mask"][h, i]
+        if diff.any():
+            order = np.sort(s[h, i])[::-1]
+            bound = order[min(ref["kept"][h, i], nb) - 1]
+            assert np.all(np.abs(s[h, i][diff] - bound) < 5e-2)
+    # CSR matches the mask
+    rp = sel["row_ptr"].cpu().numpy()
+    assert rp[-1] == kept.sum() and sel["total"] == kept.sum()
+    return int(qual.sum()), qual.size
+
+
+@pytest.mark.parametrize("top_k,tau", [(1, 0.05), (4, 0.2), (16, 0.5), (4, 1.0), (4, 0.0), (2000, 0.2)])
+def test_block_select_synthetic_720p_heads(top_k, tau):
+    wl = synth.WORKLOADS["720p"]
+    import dataclasses
+    wl = dataclasses.replace(wl, heads=2)
+    x = synth.qkv(wl)
+    geo = P.Geometry(wl.grid, wl.zone, CAND)
+    dev = torch.device("cuda")
+    q, k = x["q"].to(dev), x["k"].to(dev)
+    N = wl.n_tokens
+    zs, _ = P.zone_shapes(geo, feat=q.view(N, -1))
+    qp, kp = P.block_pool(geo, zs, q, k)
+    n_q, n = _selection_parity(qp, kp, scale_for(wl.head_dim), top_k, tau)
+    assert n_q > 0.2 * n
+
+
+def test_block_select_ragged_block_count():
+    """n_blocks not a multiple of 8 or 32 (tail rows and words)."""
+    gen = torch.Generator().manual_seed(9)
+    dev = torch.device("cuda")
+    for nb in (37, 1, 65, 200):
+        qp = torch.randn((3, nb, 64), generator=gen).to(dev)
+        kp = torch.randn((3, nb, 64), generator=gen).to(dev)
+        _selection_parity(qp, kp, 0.125, 3, 0.3)
+
+
+# --------------------------------------------------------------------------- zone shapes
+def test_zone_shapes_features_and_residual():
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["1080p"], grid=(16, 32, 48))
+    dev = torch.device("cuda")
+    F = synth.video_features(wl, device=dev)
+    R, _ = synth.a2v_residual(wl, device=dev)
+    geo = P.Geometry(wl.grid, wl.zone, CAND)
+    for feat, res in ((F, R), (F, None), (None, R)):
+        zs, margin = P.zone_shapes(geo, feat=feat, res=res)
+        idx_r, margin_r, st = O.zone_shapes(wl.grid, wl.zone, CAND, F=None if feat is None else f64(feat),
+                                            R=None if res is None else f64(res))
+        got = zs.cpu().numpy()
+        qual = margin_r > 1e-3
+        assert qual.mean() > 0.5
+        assert np.array_equal(got[qual], idx_r[qual])
+        assert np.allclose(margin.cpu().numpy()[qual], margin_r[qual], rtol=1e-3, atol=1e-4)
+
+
+def test_zone_shapes_fp32_features_match_bf16():
+    dev = torch.device("cuda")
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["1080p"], grid=(8, 16, 32))
+    F = synth.video_features(wl, device=dev)
+    geo = P.Geometry(wl.grid, wl.zone, CAND)
+    a, ma = P.zone_shapes(geo, feat=F)
+    b, mb = P.zone_shapes(geo, feat=F.float())
+    assert torch.equal(a, b)

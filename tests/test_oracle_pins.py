@@ -357,3 +357,20 @@ def test_sampled_rows_equal_masked_dense_form():
             gk, gv = O.attention_kv_block_grads(Q, K, V, dO, blocks, bm[h], h, J, sc, row_cache=cache)
             assert np.allclose(gk, dK[blocks[J], h], atol=1e-12)
             assert np.allclose(gv, dV[blocks[J], h], atol=1e-12)
+
+
+def test_empty_selection_row_is_zero_with_no_gradient():
+    rng = np.random.default_rng(8)
+    N, H, d = 32, 1, 4
+    Q, K, V, dO = (rng.normal(size=(N, H, d)) for _ in range(4))
+    allowed = rng.random((H, N, N)) < 0.5
+    allowed[0, 5, :] = False
+    Oo, lse = O.masked_attention_fwd(Q, K, V, allowed, 0.5)
+    assert np.all(Oo[5] == 0.0) and lse[0, 5] == -np.inf
+    dQ, dK, dV = O.masked_attention_bwd(Q, K, V, Oo, lse, dO, allowed, 0.5)
+    assert np.all(np.isfinite(dK)) and np.all(np.isfinite(dV)) and np.all(dQ[5] == 0.0)
+    # removing the empty query changes no key gradient
+    keep = np.arange(N) != 5
+    O2, l2 = O.masked_attention_fwd(Q[keep], K, V, allowed[:, keep], 0.5)
+    _, dK2, dV2 = O.masked_attention_bwd(Q[keep], K, V, O2, l2, dO[keep], allowed[:, keep], 0.5)
+    assert np.allclose(dK, dK2) and np.allclose(dV, dV2)
