@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the Prism block-sparse attention hot path on B200.
+
+One step = one layer of the 2K training workload through every stage:
+zone shapes (video features + a2v residual) -> block pooling -> hybrid top-k +
+CDF selection (+ CSR) -> block-sparse attention forward -> backward. Inputs are
+resident in HBM before the timed region and every input tensor (1.8 GB) is
+larger than L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead. Multi-GPU runs are independent
+replicas (the path has no exchange step); ``value`` is whole-job ms per layer.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "2K block-sparse attn fwd+bwd ms/layer; achieved TFLOP/s vs BF16 tensor peak"
+UNIT = "ms/layer"
+FWD_FLOP_PER_PAIR = 4 * 64 * 64 * 128  # QK^T and PV over one (query block, key block) pair, d = 128
+BWD_FLOP_PER_PAIR = 2.5 * FWD_FLOP_PER_PAIR
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def build_inputs(wl, device):
+    import torch
+    from dynamic_block_sparse_shape_b200 import synth
+    x = synth.qkv(wl, device=device)
+    feats = synth.video_features(wl, device=device) if wl.features == "synthetic" else None
+    res = synth.a2v_residual(wl, device=device)[0] if wl.residual else None
+    torch.cuda.synchronize()
+    return x, feats, res
+
+
+class Pipeline:
+    """One layer of the hot path through the public binding, with every
+    buffer preallocated so a step launches kernels only (no host sync)."""
+
+    def __init__(self, wl, x, feats, res):
+        import torch
+        import dynamic_block_sparse_shape_b200 as P
+        from dynamic_block_sparse_shape_b200 import synth
+        self.P, self.torch = P, torch
+        self.wl = wl
+        self.geo = P.Geometry(wl.grid, wl.zone, tuple(synth.candidates_for(wl)))
+        self.nz, self.nb = self.geo.counts()
+        self.x, self.feats, self.res = x, feats, res
+        dev = x["q"].device
+        H, d = wl.heads, wl.head_dim
+        self.scale = 1.0 / math.sqrt(d)
+        self.ws = P.Workspace(dev)
+        self.qp = torch.empty((H, self.nb, d), dtype=torch.float32, device=dev)
+        self.kp = torch.empty_like(self.qp)
+        words = (self.nb + 31) // 32
+        self.mask = torch.empty((H, self.nb, words), dtype=torch.int32, device=dev)
+        self.kept = torch.empty((H, self.nb), dtype=torch.int32, device=dev)
+        self.row_ptr = torch.empty(H * self.nb + 1, dtype=torch.int32, device=dev)
+        self.o = torch.empty_like(x["q"])
+        self.lse = torch.empty((H, wl.n_tokens), dtype=torch.float32, device=dev)
+        self.grads = tuple(torch.empty_like(x["q"]) for _ in range(3))
+        self.zone_shape = torch.empty(self.nz, dtype=torch.int32, device=dev)
+        self.zone_margin = torch.empty(self.nz, dtype=torch.float32, device=dev)
+        self.ws.ensure(P.workspace_size("zone_shapes", self.geo, feat_c=feats.shape[1] if feats is not None else 0,
+                                        res_c=res.shape[1] if res is not None else 0))
+        # size the CSR and the workspaces from one selection pass
+        self.stage_zone()
+        self.stage_pool()
+        sel = P.block_select(self.qp, self.kp, self.scale, wl.top_k, wl.cdf_threshold, ws=self.ws, csr=False)
+        self.nnz = sel["total"]
+        self.col_idx = torch.empty(max(1, self.nnz), dtype=torch.int32, device=dev)
+        need = max(P.workspace_size("zone_shapes", self.geo, feat_c=feats.shape[1] if feats is not None else 0,
+                                    res_c=res.shape[1] if res is not None else 0),
+                   P.workspace_size("bsa_fwd", self.geo, heads=H, head_dim=d),
+                   P.workspace_size("bsa_bwd", self.geo, heads=H, head_dim=d, nnz=self.nnz))
+        self.ws.ensure(need)
+        self.events = {}
+
+    def _lib(self):
+        return self.P.lib()
+
+    def stage_zone(self):
+        import ctypes
+        P, g = self.P, self.geo.c()
+        f, r = self.feats, self.res
+        P._check(P.lib().prism_zone_shapes(
+            ctypes.byref(g), P._ptr(f), f.stride(0) if f is not None else 0, f.shape[1] if f is not None else 0,
+            P.BF16, P._ptr(r), r.stride(0) if r is not None else 0, r.shape[1] if r is not None else 0, P.BF16,
+            None, P._ptr(self.zone_shape), P._ptr(self.zone_margin), self.ws.ptr, self.ws.nbytes, P._stream()),
+            "zone_shapes")
+
+    def stage_pool(self):
+        import ctypes
+        P, g, q, k = self.P, self.geo.c(), self.x["q"], self.x["k"]
+        P._check(P.lib().prism_block_pool(ctypes.byref(g), P._ptr(self.zone_shape), P._ptr(q), P._ptr(k), P.BF16,
+                                          q.shape[1], q.shape[2], q.stride(0), P._ptr(self.qp), P._ptr(self.kp),
+                                          self.ws.ptr, self.ws.nbytes, P._stream()), "block_pool")
+
+    def stage_select(self):
+        P = self.P
+        H, nb, d = self.qp.shape
+        P._check(P.lib().prism_block_select(P._ptr(self.qp), P._ptr(self.kp), H, nb, d, self.scale, self.wl.top_k,
+                                            self.wl.cdf_threshold, P._ptr(self.mask), P._ptr(self.kept),
+                                            P._ptr(self.row_ptr), P._ptr(self.col_idx), self.col_idx.numel(), None,
+                                            self.ws.ptr, self.ws.nbytes, P._stream()), "block_select")
+
+    def stage_fwd(self):
+        x = self.x
+        self.P.bsa_fwd(self.geo, self.zone_shape, x["q"], x["k"], x["v"], self.scale, self.row_ptr, self.col_idx,
+                       ws=self.ws, out=self.o, lse=self.lse)
+
+    def stage_bwd(self):
+        x = self.x
+        self.P.bsa_bwd(self.geo, self.zone_shape, x["q"], x["k"], x["v"], self.o, self.lse, x["do"], self.scale,
+                       self.row_ptr, self.col_idx, self.nnz, ws=self.ws, grads=self.grads)
+
+    STAGES = ("zone_shapes", "block_pool", "block_select", "bsa_fwd", "bsa_bwd")
+    # kernels each stage launches (prism kernels only; memsets excluded)
+    LAUNCHES = {"zone_shapes": 4, "block_pool": 1, "block_select": 3, "bsa_fwd": 1, "bsa_bwd": 7}
+
+    def step(self, record=None):
+        fns = (self.stage_zone, self.stage_pool, self.stage_select, self.stage_fwd, self.stage_bwd)
+        for name, fn in zip(self.STAGES, fns):
+            if record is not None:
+                e0 = self.torch.cuda.Event(enable_timing=True)
+                e1 = self.torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                record.setdefault(name, []).append((e0, e1))
+            else:
+                fn()
+
+    def launches_per_step(self):
+        n = sum(self.LAUNCHES.values())
+        if self.feats is None:
+            n -= 1
+        if self.res is None:
+            n -= 2
+        return n
+
+
+def cpu_sample(wl, x, feats, res, q_blocks=4, kv_blocks=2, sel_rows=256, users_per_kv=8):
+    """Times the fp64 oracle on a bounded sample of the workload and
+    extrapolates each stage linearly to one layer (ms). Oracle only: the
+    selection it uses is its own; no CUDA-path value enters."""
+    import numpy as np
+    import torch
+    from oracle import prism_oracle as O
+    from dynamic_block_sparse_shape_b200 import synth
+    t_all = time.time()
+    cand = synth.candidates_for(wl)
+    N = wl.n_tokens
+    nzt, nzh, nzw = O.zone_counts(wl.grid, wl.zone)
+    nz = nzt * nzh * nzw
+    nb = nz * O.blocks_per_zone(wl.zone)
+    heads = wl.heads
+    rng = np.random.default_rng(0)
+    timings = {}
+    # a2: token norms of 1/16 of the residual rows, statistics + choice on 4 zones
+    zs_sample = sorted(rng.choice(nz, size=min(4, nz), replace=False).tolist())
+    ids = np.concatenate([O.zone_token_ids(wl.grid, wl.zone, z).ravel() for z in zs_sample])
+    fmap = {int(n): i for i, n in enumerate(ids)}
+
+    class _Rows:  # the sampled zones' rows only, indexed by token id
+        def __init__(self, sub):
+            self.sub = sub
+
+        def __getitem__(self, idx):
+            return self.sub[[fmap[int(n)] for n in np.asarray(idx).ravel()]]
+    t_norm = 0.0
+    r = None
+    if res is not None:
+        chunk = N // 16
+        t0 = time.time()
+        O.token_norms(res[:chunk].to("cpu", torch.float64).numpy())
+        t_norm = (time.time() - t0) * 16
+        r = np.ones(N)  # norms outside the sample are not needed for the timing
+        r[ids] = O.token_norms(res[torch.as_tensor(ids, device=res.device)].to("cpu", torch.float64).numpy())
+    Fz = None
+    if feats is not None:
+        Fz = _Rows(feats[torch.as_tensor(ids, device=feats.device)].to("cpu", torch.float64).numpy())
+    t0 = time.time()
+    st = O.zone_statistics(wl.grid, wl.zone, F=Fz, zones=zs_sample, r=r)
+    O.choose_shapes(st, cand, have_features=feats is not None, have_residual=r is not None)
+    timings["zone_shapes"] = t_norm + (time.time() - t0) * nz / len(zs_sample)
+    # a3: pooling of head 0 over all blocks (the selection needs every key block)
+    blocks = O.block_tokens(wl.grid, wl.zone, cand, np.zeros(nz, dtype=np.int64))
+    q0, k0, v0, do0 = (x[n][:, 0].to("cpu", torch.float64).numpy()[:, None, :] for n in ("q", "k", "v", "do"))
+    t0 = time.time()
+    qp = O.block_pool(q0, blocks)
+    kp = O.block_pool(k0, blocks)
+    timings["block_pool"] = (time.time() - t0) * heads
+    # a4/a5: sel_rows query blocks of head 0
+    sc = 1.0 / math.sqrt(wl.head_dim)
+    srows = sorted(rng.choice(nb, size=min(sel_rows, nb), replace=False).tolist())
+    t0 = time.time()
+    sel = O.block_select(qp, kp, sc, wl.top_k, wl.cdf_threshold, rows=[(0, i) for i in srows])
+    timings["block_select"] = (time.time() - t0) * heads * nb / len(srows)
+    mask0 = sel["mask"][0]
+    mean_kept = float(np.mean([sel["kept"][0, i] for i in srows]))
+    # a6/a7 (q side): forward rows + dQ of q_blocks sampled query blocks
+    t0 = time.time()
+    cache = {}
+    for I in srows[:q_blocks]:
+        cache[(0, I)] = O.attention_block_rows(q0, k0, v0, blocks, np.nonzero(mask0[I])[0], 0, I, sc, dO=do0)
+    t_q = (time.time() - t0) / q_blocks
+    # a7 (kv side): dK/dV of kv_blocks key blocks, restricted to users_per_kv
+    # users whose rows are cached; time per user, times the mean users per block
+    users = srows[q_blocks:q_blocks + users_per_kv]
+    for I in users:
+        cache[(0, I)] = O.attention_block_rows(q0, k0, v0, blocks, np.nonzero(mask0[I])[0], 0, I, sc, dO=do0)
+    t_user = 0.0
+    n_user = 0
+    for J in range(kv_blocks):
+        sub = np.zeros_like(mask0)
+        for I in users:
+            sub[I] = mask0[I]
+            sub[I, J] = True
+        t0 = time.time()
+        O.attention_kv_block_grads(q0, k0, v0, do0, blocks, sub, 0, J, sc, row_cache=cache)
+        t_user += time.time() - t0
+        n_user += len(users)
+    t_kv = t_user / max(n_user, 1) * mean_kept  # users per key block = mean kept per query block
+    timings["attention"] = (t_q + t_kv) * nb * heads
+    total_ms = 1e3 * sum(timings.values())
+    sample = (f"oracle (numpy fp64) on {wl.name}: zone statistics on {len(zs_sample)} of {nz} zones and residual "
+              f"norms of 1/16 of the tokens; pooling of all {nb} blocks of head 0; selection of {len(srows)} query "
+              f"blocks of head 0; attention forward + dQ rows of {q_blocks} query blocks; dK/dV per user row on "
+              f"{kv_blocks} key blocks x {len(users)} users; each stage extrapolated linearly to {heads} heads x "
+              f"{nb} blocks (mean kept {mean_kept:.1f})")
+    return {"value": round(total_ms, 1), "unit": UNIT, "cores": int(os.cpu_count() or 1),
+            "threads": int(torch.get_num_threads()), "kind": "oracle", "sample": sample,
+            "wall_s": round(time.time() - t_all, 1), "stage_ms": {k: round(1e3 * v, 1) for k, v in timings.items()}}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from dynamic_block_sparse_shape_b200 import synth
+    from dynamic_block_sparse_shape_b200 import build as pbuild
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    pbuild.build()
+    wl = synth.WORKLOADS[args.config]
+    dev = torch.device("cuda", local)
+    x, feats, res = build_inputs(wl, dev)
+    pipe = Pipeline(wl, x, feats, res)
+    for _ in range(args.warmup):
+        pipe.step()
+    torch.cuda.synchronize()
+    pipe.P.check_device_status(pipe.ws)
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    rec = {}
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        pipe.step(record=rec)
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = float(t.item()) / args.steps
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in rec.items()}
+    pipe.P.check_device_status(pipe.ws)
+    # end to end through the public API with host buffers
+    e2e = run_e2e(pipe, wl, x, feats, res, steps=min(args.steps, args.e2e_steps))
+    peaks, peak_src = _peaks()
+    nnz = pipe.nnz
+    attn_flop = nnz * (FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR)
+    t_attn = (stage_ms["bsa_fwd"] + stage_ms["bsa_bwd"]) * 1e-3
+    achieved = attn_flop / t_attn / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    out = {
+        "metric": METRIC, "value": round(ms_step / world, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]} ({wl.n_tokens} tokens), "
+                               f"{wl.heads} heads x d{wl.head_dim}, zones {wl.zone}, top_k {wl.top_k}, "
+                               f"cdf_threshold {wl.cdf_threshold}, fwd+bwd",
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (each 1.8 GB), no flush"},
+        "tflops": round(achieved, 1),
+        "selected_pairs": nnz, "density": round(nnz / (wl.heads * pipe.nb * pipe.nb), 4),
+        "stage_ms": {k: round(v, 3) for k, v in stage_ms.items()},
+        "roofline": {"bound": "tensor", "kernel": "bsa_fwd + bsa_bwd (dq, dkdv)", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16 sustained",
+                     "flop_per_pair": FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR},
+        "e2e": e2e,
+        "gpu_launches": pipe.launches_per_step() * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_sample(wl, x, feats, res)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(pipe, wl, x, feats, res, steps):
+    """Same metric through the public API: per step, host->device copies of the
+    step's inputs from pinned memory, the five stages, and device->host reads of
+    O, dQ, dK, dV."""
+    import torch
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+    host_in = {k: pinned_copy(v) for k, v in x.items()}
+    host_f = pinned_copy(feats) if feats is not None else None
+    host_r = pinned_copy(res) if res is not None else None
+    outs = (pipe.o, *pipe.grads)
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    h2d += sum(t.numel() * t.element_size() for t in (host_f, host_r) if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def one():
+        for k2, v2 in host_in.items():
+            x[k2].copy_(v2, non_blocking=True)
+        if host_f is not None:
+            feats.copy_(host_f, non_blocking=True)
+        if host_r is not None:
+            res.copy_(host_r, non_blocking=True)
+        pipe.step()
+        for h, o in zip(host_out, outs):
+            h.copy_(o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"value": round(ms, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": steps}
+
+
+# ---------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    import torch
+    from dynamic_block_sparse_shape_b200 import synth
+    world, rank, local = _dist()
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.config]
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    x, feats, res = build_inputs(wl, dev) if dev.type == "cuda" else _cpu_inputs(wl)
+    vals = []
+    last = None
+    for i in range(args.warmup + args.steps):
+        last = cpu_sample(wl, x, feats, res)
+        if i >= args.warmup:
+            vals.append(last["value"])
+    v = statistics.mean(vals)
+    cpu = dict(last)
+    cpu["value"] = round(v, 1)
+    out = {"metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": f"{wl.name} (oracle on host cores, bounded sample per step)"},
+           "cpu_baseline": cpu,
+           "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def _cpu_inputs(wl):
+    from dynamic_block_sparse_shape_b200 import synth
+    x = synth.qkv(wl)
+    feats = synth.video_features(wl) if wl.features == "synthetic" else None
+    res = synth.a2v_residual(wl)[0] if wl.residual else None
+    return x, feats, res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
+    ap.add_argument("--config", default="2k")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -232,7 +232,9 @@ def select_row(s, top_k, tau):
 
     s: logits over all key blocks. Returns (kept indices ascending, m, m_star,
     logit_gap, cdf_margin) where the gap is s_(m) - s_(m+1) in the ranked
-    order and the margin is min(|C_{m*} - tau|, |C_{m*-1} - tau|).
+    order. The margin says how far the cumulative mass is from changing m:
+    min(|C_{m*} - tau|, |C_{m*-1} - tau|) when the crossing decides m
+    (m* >= k), else C_k - tau.
     """
     s = np.asarray(s, dtype=np.float64)
     n = s.shape[0]
@@ -247,9 +249,13 @@ def select_row(s, top_k, tau):
     m = max(int(top_k), m_star)
     kept = np.sort(order[:m])
     gap = float(s[order[m - 1]] - s[order[m]]) if m < n else math.inf
-    c_hi = C[m_star - 1]
-    c_lo = C[m_star - 2] if m_star >= 2 else 0.0
-    margin = float(min(abs(c_hi - tau), abs(c_lo - tau)))
+    if m_star < top_k:
+        # the floor k decides m; it stays decided while C_k stays above tau
+        margin = float(C[int(top_k) - 1] - tau)
+    else:
+        c_hi = C[m_star - 1]
+        c_lo = C[m_star - 2] if m_star >= 2 else 0.0
+        margin = float(min(abs(c_hi - tau), abs(c_lo - tau)))
     return kept, m, m_star, gap, margin
 
 

@@ -1,0 +1,119 @@
+"""The C-ABI library loads without a GPU, exports every declared entry point,
+and its host-side validation returns the documented status codes (no CUDA
+call is reached in these cases)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dynamic_block_sparse_shape_b200 as P
+from dynamic_block_sparse_shape_b200 import build as pbuild
+from dynamic_block_sparse_shape_b200.synth import DEFAULT_CANDIDATES
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "prism.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return P.lib()
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^PRISM_API\s+[^(]*?\b(prism_\w+)\s*\(", txt, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    for s in syms:
+        assert hasattr(lib, s), s
+    # and the binding declares a signature for each of them
+    assert set(syms) == set(P._SIGNATURES), set(syms) ^ set(P._SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    for code in P.STATUS:
+        assert lib.prism_status_string(code)
+    assert lib.prism_status_string(12345) == b"unknown status"
+    assert lib.prism_version() >= 100
+
+
+def _geo(grid=(32, 72, 128), zone=(8, 8, 8), cand=DEFAULT_CANDIDATES):
+    return P.Geometry(grid, zone, tuple(cand))
+
+
+def test_geometry_counts_and_errors(lib):
+    assert _geo().counts() == (576, 4608)
+    assert _geo((4, 8, 8), (4, 8, 8), [(4, 4, 4)]).counts() == (1, 4)
+    bad = [
+        ((32, 72, 127), (8, 8, 8), DEFAULT_CANDIDATES, 2),  # grid not divisible by the zone
+        ((32, 72, 128), (8, 8, 8), [(4, 4, 2)], 2),  # candidate volume != 64
+        ((32, 72, 128), (8, 8, 8), [(16, 2, 2)], 2),  # candidate does not divide the zone
+        ((32, 64, 128), (16, 16, 16), [(4, 4, 4)], 9),  # zone larger than 512 tokens
+        ((8, 8, 8), (4, 4, 2), [(4, 4, 2)], 2),  # zone volume not a multiple of 64
+    ]
+    for grid, zone, cand, code in bad:
+        with pytest.raises(P.PrismError) as e:
+            _geo(grid, zone, cand).counts()
+        assert e.value.status == code, (grid, zone, cand)
+
+
+def test_workspace_sizes(lib):
+    g = _geo()
+    assert P.workspace_size("block_select", g) == 256
+    z = P.workspace_size("zone_shapes", g, feat_c=3072, res_c=3072)
+    assert z >= 576 * 48 * 8 * 4 + 294912 * 4
+    b = P.workspace_size("bsa_bwd", g, heads=24, head_dim=128, nnz=1000)
+    b2 = P.workspace_size("bsa_bwd", g, heads=24, head_dim=128, nnz=2000)
+    assert b2 - b == 4096 or b2 - b == 3840 or b2 > b
+    f32 = P.workspace_size("bsa_fwd", g, heads=24, head_dim=128, dtype=__import__("torch").float32)
+    assert f32 >= 3 * 294912 * 24 * 128 * 2
+
+
+def test_host_validation_codes(lib):
+    g = _geo().c()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    ws = ctypes.c_void_p(1 << 24)
+    # block_select: top_k < 1, bad tau, unsupported d, too many blocks, missing workspace
+    sel = lib.prism_block_select
+    assert sel(fake, fake, 24, 4608, 128, 0.088, 0, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 1
+    assert sel(fake, fake, 24, 4608, 128, 0.088, 4, -0.1, fake, fake, fake, None, 0, None, ws, 256, None) == 1
+    assert sel(fake, fake, 24, 4608, 96, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 9
+    assert sel(fake, fake, 24, 9000, 128, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 9
+    assert sel(fake, fake, 24, 4608, 128, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, None, 256, None) == 4
+    assert sel(None, fake, 24, 4608, 128, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 1
+    # block_pool: dtype, head_dim, token stride
+    pool = lib.prism_block_pool
+    assert pool(ctypes.byref(g), fake, fake, fake, 7, 24, 128, 3072, fake, fake, ws, 256, None) == 3
+    assert pool(ctypes.byref(g), fake, fake, fake, 0, 24, 96, 3072, fake, fake, ws, 256, None) == 9
+    assert pool(ctypes.byref(g), fake, fake, fake, 0, 24, 128, 3000, fake, fake, ws, 256, None) == 1
+    # attention: null pointers, bad scale, small workspace
+    fwd = lib.prism_bsa_fwd
+    assert fwd(ctypes.byref(g), fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, fake, fake, ws, 256,
+               None) == 1
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, -1.0, fake, fake, fake, fake, ws, 256,
+               None) == 1
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 1, 24, 128, 3072, 0.088, fake, fake, fake, fake, ws, 256,
+               None) == 4  # fp32 inputs need staging space
+    bwd = lib.prism_bsa_bwd
+    assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, 1000,
+               fake, fake, fake, ws, 256, None) == 4
+    assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, -5,
+               fake, fake, fake, ws, 1 << 40, None) == 1
+    # zone shapes: channels not a multiple of 64, misaligned workspace
+    zs = lib.prism_zone_shapes
+    assert zs(ctypes.byref(g), fake, 3072, 3000, 0, None, 0, 0, 0, None, fake, None, ws, 1 << 30, None) == 1
+    assert zs(ctypes.byref(g), None, 0, 0, 0, None, 0, 0, 0, None, fake, None, ctypes.c_void_p((1 << 24) + 8),
+              1 << 30, None) == 4
+    # mask_to_csr
+    assert lib.prism_mask_to_csr(fake, fake, 0, 10, fake, 10, ws, 256, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(P, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(P, "_lib", None)
+    with pytest.raises(P.PrismError):
+        P.lib()
