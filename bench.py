@@ -101,7 +101,11 @@ def build_inputs(wl, device):
     import torch
     from dynamic_block_sparse_shape_b200 import synth
     x = synth.qkv(wl, device=device)
-    feats = synth.video_features(wl, device=device) if wl.features == "synthetic" else None
+    feats = None
+    if wl.features == "synthetic":
+        feats = synth.video_features(wl, device=device)
+    elif wl.features == "q":
+        feats = x["q"].view(wl.n_tokens, -1)
     res = synth.a2v_residual(wl, device=device)[0] if wl.residual else None
     torch.cuda.synchronize()
     return x, feats, res
@@ -350,7 +354,7 @@ def run_gpu(args):
     stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in rec.items()}
     pipe.P.check_device_status(pipe.ws)
     # end to end through the public API with host buffers
-    e2e = run_e2e(pipe, wl, x, feats, res, steps=min(args.steps, args.e2e_steps))
+    e2e = None if args.no_e2e else run_e2e(pipe, wl, x, feats, res, steps=min(args.steps, args.e2e_steps))
     peaks, peak_src = _peaks()
     nnz = pipe.nnz
     attn_flop = nnz * (FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR)
@@ -378,7 +382,8 @@ def run_gpu(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_sample(wl, x, feats, res)
+        out["cpu_baseline"] = cpu_sample(wl, x, feats, res, q_blocks=24, kv_blocks=4, sel_rows=1024,
+                                         users_per_kv=16)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -460,7 +465,8 @@ def run_reference(args):
 def _cpu_inputs(wl):
     from dynamic_block_sparse_shape_b200 import synth
     x = synth.qkv(wl)
-    feats = synth.video_features(wl) if wl.features == "synthetic" else None
+    feats = synth.video_features(wl) if wl.features == "synthetic" else (
+        x["q"].view(wl.n_tokens, -1) if wl.features == "q" else None)
     res = synth.a2v_residual(wl)[0] if wl.residual else None
     return x, feats, res
 
@@ -474,6 +480,7 @@ def main():
     ap.add_argument("--config", default="2k")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -61,6 +61,9 @@ WORKLOADS = {
     "1080p": Workload("1080p", (16, 72, 128), 24, 128, "bf16", (8, 8, 8), 4, 0.20, False, "synthetic", True,
                       seed=2),
     "2k": Workload("2k", (32, 72, 128), 24, 128, "bf16", (8, 8, 8), 4, 0.20, True, "synthetic", True, seed=3),
+    # the 2K grid with 2 heads and Q as the feature input: every attention tensor (151 MB) is still
+    # larger than L2, and the whole working set (~1.3 GB) is small enough for profiler captures
+    "2k-2h": Workload("2k-2h", (32, 72, 128), 2, 128, "bf16", (8, 8, 8), 4, 0.20, True, "q", False, seed=3),
 }
 
 
