@@ -64,12 +64,16 @@ def test_static_scratch_matches_workspace_entry_point_twice():
 def test_static_scratch_rejects_grids_beyond_its_size():
     require_gpu()
     dev = torch.device("cuda")
-    # 64x128x128 tokens need about 7.4 MB of scratch with 3072 channels
+    # 64x128x128 tokens: the residual norms alone need 4 MiB, beyond the
+    # static scratch. The residual buffer has the full size the geometry
+    # declares (8 channels, 16 MB), so nothing could read out of bounds even
+    # if the size check were missing.
     geo = P.Geometry((64, 128, 128), (8, 8, 8), tuple(synth.DEFAULT_CANDIDATES))
     nz, _ = geo.counts()
-    feat = torch.empty((16, 3072), dtype=torch.bfloat16, device=dev)  # never read: the size check fails first
+    res = torch.zeros((geo.n_tokens, 8), dtype=torch.bfloat16, device=dev)
     shape = torch.empty(nz, dtype=torch.int32, device=dev)
     g = geo.c()
-    st = P.lib().prism_zone_shapes_static(ctypes.byref(g), P._ptr(feat), 3072, 3072, P.BF16, None, 0, 0, P.BF16, None,
+    st = P.lib().prism_zone_shapes_static(ctypes.byref(g), None, 0, 0, P.BF16, P._ptr(res), 8, 8, P.BF16, None,
                                           P._ptr(shape), None, P._stream())
     assert P.STATUS[st] == "PRISM_ERR_UNSUPPORTED"
+    torch.cuda.synchronize()
