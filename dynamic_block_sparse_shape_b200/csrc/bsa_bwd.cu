@@ -58,16 +58,24 @@ struct BwdParams {
 };
 
 // ----------------------------------------------------------------------- dq
+// Rings: K (3 slots, held until the dQ product of its step completes), V (2
+// slots, held until the dP product), score buffers S/dP (3 each, TMEM),
+// dS (one shared-memory buffer). The producer and the issuer poll every
+// barrier they could act on and start whichever operation is ready.
+constexpr int kDqKSlots = 3;
+constexpr int kDqVSlots = 2;
+constexpr int kDqSBufs = 3;
+
 template <int D>
 struct DqSmem {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kDO = D * 128;
-  static constexpr uint32_t kHalf = kKB * D * 128;  // K (or V) of one stage
-  static constexpr uint32_t kStage0 = 2 * D * 128;
-  static constexpr uint32_t kStageBytes = 2 * kHalf;
-  static constexpr uint32_t kDS0 = kStage0 + 2 * kStageBytes;
+  static constexpr uint32_t kSlotBytes = kKB * D * 128;  // K (or V) of one step, [dh][block][64][128 B]
+  static constexpr uint32_t kK0 = 2 * D * 128;
+  static constexpr uint32_t kV0 = kK0 + kDqKSlots * kSlotBytes;
+  static constexpr uint32_t kDS = kV0 + kDqVSlots * kSlotBytes;
   static constexpr uint32_t kDSBytes = kKB * kBoxBytes;
-  static constexpr uint32_t kBar = kDS0 + 2 * kDSBytes;
+  static constexpr uint32_t kBar = kDS + kDSBytes;
   static constexpr uint32_t kTotal = kBar + 256;
 };
 
@@ -78,15 +86,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* qd_full = bars + 0;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_free = bars + 7;
-  uint64_t* ds_full = bars + 9;
-  uint64_t* ds_free = bars + 11;
-  uint64_t* mma_done = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* k_full = bars + 1;   // [3]
+  uint64_t* k_empty = bars + 4;  // [3]
+  uint64_t* v_full = bars + 7;   // [2]
+  uint64_t* v_empty = bars + 9;  // [2]
+  uint64_t* s_full = bars + 11;  // [3]
+  uint64_t* s_free = bars + 14;  // [3]
+  uint64_t* ds_full = bars + 17;
+  uint64_t* ds_free = bars + 18;
+  uint64_t* mma_done = bars + 19;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
 
   const Geo& g = P.g;
   const int I = blockIdx.x, head = blockIdx.y;
@@ -102,14 +112,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   const int nsteps = (cnt + kKB - 1) / kKB;
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < kDqKSlots; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kDqVSlots; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < kDqSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kSoftWarps);
-      mbar_init(&ds_full[i], kSoftWarps);
-      mbar_init(&ds_free[i], 1);
     }
+    mbar_init(ds_full, kSoftWarps);
+    mbar_init(ds_free, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -122,7 +138,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tdQ = tbase + 256;
+  const uint32_t tdQ = tbase + 384;
 
   if (warp == 0) {
     if (lane == 0 && nsteps > 0) {
@@ -133,75 +149,96 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
         tma_load_5d(sm + L::kDO + dh * kBoxBytes, &P.mdo[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
       }
-      int issued = 0;
-      for (int j = 0; j < nsteps; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_abortable(&kv_empty[st], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
-        uint8_t* stage = sm + L::kStage0 + st * L::kStageBytes;
-        mbar_arrive_expect_tx(&kv_full[st], L::kStageBytes);
+      auto block_of = [&](int j, int slot) -> int {
+        int e = j * kKB + slot;
+        if (e >= cnt) e = j * kKB;
+        int J = P.idx[beg + e];
+        if (J < 0 || J >= g.n_blocks) {
+          atomicOr(status, kDevErrBounds);
+          J = 0;
+        }
+        return J;
+      };
+      auto load_step = [&](const CUtensorMap* maps, uint8_t* dst, uint64_t* bar, int j) {
+        mbar_arrive_expect_tx(bar, L::kSlotBytes);
         for (int slot = 0; slot < kKB; ++slot) {
-          int e = j * kKB + slot;
-          if (e >= cnt) e = j * kKB;
-          int J = P.idx[beg + e];
-          if (J < 0 || J >= g.n_blocks) {
-            atomicOr(status, kDevErrBounds);
-            J = 0;
-          }
+          const int J = block_of(j, slot);
           const int sJ = safe_shape(g, P.zone_shape, J, status);
           const BlockBox kb = block_box(g, sJ, J);
-          for (int dh = 0; dh < D / 64; ++dh) {
-            const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
-            tma_load_5d(stage + off, &P.mk[sJ], &kv_full[st], dh * 64, head, kb.w0, kb.h0, kb.t0);
-            tma_load_5d(stage + L::kHalf + off, &P.mv[sJ], &kv_full[st], dh * 64, head, kb.w0, kb.h0, kb.t0);
-          }
+          for (int dh = 0; dh < D / 64; ++dh)
+            tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &maps[sJ], bar, dh * 64, head, kb.w0, kb.h0,
+                        kb.t0);
         }
-        ++issued;
+      };
+      int kj = 0, vj = 0;
+      Watchdog wd;
+      wd.reset();
+      while (kj < nsteps || vj < nsteps) {
+        bool did = false;
+        if (kj < nsteps && mbar_test(&k_empty[kj % kDqKSlots], ((kj / kDqKSlots) & 1) ^ 1)) {
+          load_step(P.mk, sm + L::kK0 + (kj % kDqKSlots) * L::kSlotBytes, &k_full[kj % kDqKSlots], kj);
+          ++kj;
+          did = true;
+        }
+        if (vj < kj && mbar_test(&v_empty[vj & 1], ((vj >> 1) & 1) ^ 1)) {
+          load_step(P.mv, sm + L::kV0 + (vj & 1) * L::kSlotBytes, &v_full[vj & 1], vj);
+          ++vj;
+          did = true;
+        }
+        if (did) wd.reset();
+        else if (!wd.ok(status, abort_flag)) break;
       }
       mbar_wait(qd_full, 0, status);
-      for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, status);
+      for (int i = kj - kDqKSlots > 0 ? kj - kDqKSlots : 0; i < kj; ++i)
+        mbar_wait(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, status);
+      for (int i = vj - kDqVSlots > 0 ? vj - kDqVSlots : 0; i < vj; ++i)
+        mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
     }
   } else if (warp == 1) {
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
-      const uint32_t sQ = smem_u32(sm + L::kQ), sDO = smem_u32(sm + L::kDO);
+      const uint32_t sQ = smem_u32(sm + L::kQ), sDO = smem_u32(sm + L::kDO), sDS = smem_u32(sm + L::kDS);
       bool ok = mbar_wait_abortable(qd_full, 0, status, abort_flag);
-      auto issue_dq = [&](int i) -> bool {
-        const int pb = i & 1;
-        if (!mbar_wait_abortable(&ds_full[pb], (i >> 1) & 1, status, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t sDS = smem_u32(sm + L::kDS0 + pb * L::kDSBytes);
-        const uint32_t sK = smem_u32(sm + L::kStage0 + (i & 1) * L::kStageBytes);
+      int sj = 0, qj = 0;
+      Watchdog wd;
+      wd.reset();
+      while (ok && qj < nsteps) {
+        bool did = false;
+        if (qj < sj && mbar_test(ds_full, qj & 1)) {
+          tc_fence_after();
+          const uint32_t sK = smem_u32(sm + L::kK0 + (qj % kDqKSlots) * L::kSlotBytes);
 #pragma unroll
-        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-          mma_ws(tdQ, kmajor_desc(sDS, kk, kBoxBytes), mnmajor_desc(sK, kk, kBoxBytes, kKB * kBoxBytes), idQ,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&kv_empty[i & 1]);
-        mma_commit(&ds_free[pb]);
-        return true;
-      };
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const int st = j & 1, sb = j & 1;
-        if (!mbar_wait_abortable(&kv_full[st], (j >> 1) & 1, status, abort_flag)) break;
-        if (!mbar_wait_abortable(&s_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t sK = smem_u32(sm + L::kStage0 + st * L::kStageBytes);
-        const uint32_t sV = sK + L::kHalf;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws(tbase + sb * 64, kmajor_desc(sQ, kk, kBoxBytes), kmajor_desc(sK, kk, kKB * kBoxBytes), idS,
-                 kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws(tbase + 128 + sb * 64, kmajor_desc(sDO, kk, kBoxBytes), kmajor_desc(sV, kk, kKB * kBoxBytes), idS,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(&s_full[sb]);
-        if (j >= 1 && !issue_dq(j - 1)) {
-          ok = false;
-          break;
+          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+            mma_ws(tdQ, kmajor_desc(sDS, kk, kBoxBytes), mnmajor_desc(sK, kk, kBoxBytes, kKB * kBoxBytes), idQ,
+                   (qj > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&k_empty[qj % kDqKSlots]);
+          mma_commit(ds_free);
+          ++qj;
+          did = true;
         }
+        if (sj < nsteps && mbar_test(&k_full[sj % kDqKSlots], (sj / kDqKSlots) & 1) &&
+            mbar_test(&v_full[sj & 1], (sj >> 1) & 1) && mbar_test(&s_free[sj % kDqSBufs], ((sj / kDqSBufs) & 1) ^ 1)) {
+          tc_fence_after();
+          const uint32_t sK = smem_u32(sm + L::kK0 + (sj % kDqKSlots) * L::kSlotBytes);
+          const uint32_t sV = smem_u32(sm + L::kV0 + (sj & 1) * L::kSlotBytes);
+          const int sb = sj % kDqSBufs;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws(tbase + sb * 64, kmajor_desc(sQ, kk, kBoxBytes), kmajor_desc(sK, kk, kKB * kBoxBytes), idS,
+                   kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws(tbase + 192 + sb * 64, kmajor_desc(sDO, kk, kBoxBytes), kmajor_desc(sV, kk, kKB * kBoxBytes), idS,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(&s_full[sb]);
+          mma_commit(&v_empty[sj & 1]);
+          ++sj;
+          did = true;
+        }
+        if (did) wd.reset();
+        else if (!wd.ok(status, abort_flag)) break;
       }
-      if (ok) issue_dq(nsteps - 1);
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, status);
     }
@@ -213,12 +250,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     const float lse2 = P.lse2[size_t(row) * 64 + m];
     const float dm = P.dvec[size_t(row) * 64 + m];
     for (int j = 0; j < nsteps; ++j) {
-      const int sb = j & 1;
-      mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
+      const int sb = j % kDqSBufs;
+      mbar_wait_abortable(&s_full[sb], (j / kDqSBufs) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t rs[32], rp[32];
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
-      tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
+      tmem_ld32(tbase + lane_off + 192 + sb * 64 + ch * 32, rp);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -236,17 +273,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         }
         pk[i] = pack_bf16x2(d0, d1);
       }
-      if (j >= 2) mbar_wait_abortable(&ds_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag);
-      uint8_t* pt = sm + L::kDS0 + sb * L::kDSBytes + kh * kBoxBytes;
+      if (j >= 1) mbar_wait_abortable(ds_free, (j - 1) & 1, status, abort_flag);
+      uint8_t* pt = sm + L::kDS + kh * kBoxBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
             make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full[sb]);
+      if (lane == 0) mbar_arrive(ds_full);
     }
-    if (nsteps > 0) mbar_wait_abortable(&ds_free[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, status, abort_flag);
+    if (nsteps > 0) mbar_wait_abortable(ds_free, (nsteps - 1) & 1, status, abort_flag);
     tc_fence_after();
     const bool ok = *abort_flag == 0;
     constexpr int NC = D / 4;
@@ -272,6 +309,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
 }
 
 // --------------------------------------------------------------------- dkdv
+// Stages of (Q, dO, LSE, D) for two query blocks, 2 slots, each held until the
+// dV/dK products of its step complete; S^T/dP^T in TMEM (2 buffers each);
+// P^T and dS^T in one shared-memory buffer each. The issuer polls and starts
+// whichever of "scores of step s" / "dV, dK of step k" is ready.
 template <int D>
 struct DkvSmem {
   static constexpr uint32_t kK = 0;
@@ -386,45 +427,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       const uint32_t sK = smem_u32(sm + L::kK), sV = smem_u32(sm + L::kV);
       const uint32_t sPT = smem_u32(sm + L::kPT), sDST = smem_u32(sm + L::kDST);
       bool ok = mbar_wait_abortable(kv_full, 0, status, abort_flag);
-      auto issue_kv = [&](int i) -> bool {
-        if (!mbar_wait_abortable(ps_full, i & 1, status, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t sQ = smem_u32(sm + L::kStage0 + (i & 1) * L::kStageBytes);
-        const uint32_t sDO = sQ + L::kHalf;
+      int sj = 0, kj = 0;
+      Watchdog wd;
+      wd.reset();
+      while (ok && kj < nsteps) {
+        bool did = false;
+        if (kj < sj && mbar_test(ps_full, kj & 1)) {
+          tc_fence_after();
+          const uint32_t sQ = smem_u32(sm + L::kStage0 + (kj & 1) * L::kStageBytes);
+          const uint32_t sDO = sQ + L::kHalf;
 #pragma unroll
-        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-          mma_ws(tdV, kmajor_desc(sPT, kk, kBoxBytes), mnmajor_desc(sDO, kk, kBoxBytes, kKB * kBoxBytes), idO,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+            mma_ws(tdV, kmajor_desc(sPT, kk, kBoxBytes), mnmajor_desc(sDO, kk, kBoxBytes, kKB * kBoxBytes), idO,
+                   (kj > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-          mma_ws(tdK, kmajor_desc(sDST, kk, kBoxBytes), mnmajor_desc(sQ, kk, kBoxBytes, kKB * kBoxBytes), idO,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&st_empty[i & 1]);
-        mma_commit(ps_free);
-        return true;
-      };
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const int st = j & 1, sb = j & 1;
-        if (!mbar_wait_abortable(&st_full[st], (j >> 1) & 1, status, abort_flag)) break;
-        if (!mbar_wait_abortable(&s_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t sQ = smem_u32(sm + L::kStage0 + st * L::kStageBytes);
-        const uint32_t sDO = sQ + L::kHalf;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws(tbase + sb * 64, kmajor_desc(sK, kk, kBoxBytes), kmajor_desc(sQ, kk, kKB * kBoxBytes), idS,
-                 kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws(tbase + 128 + sb * 64, kmajor_desc(sV, kk, kBoxBytes), kmajor_desc(sDO, kk, kKB * kBoxBytes), idS,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(&s_full[sb]);
-        if (j >= 1 && !issue_kv(j - 1)) {
-          ok = false;
-          break;
+          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+            mma_ws(tdK, kmajor_desc(sDST, kk, kBoxBytes), mnmajor_desc(sQ, kk, kBoxBytes, kKB * kBoxBytes), idO,
+                   (kj > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&st_empty[kj & 1]);
+          mma_commit(ps_free);
+          ++kj;
+          did = true;
         }
+        if (sj < nsteps && mbar_test(&st_full[sj & 1], (sj >> 1) & 1) &&
+            mbar_test(&s_free[sj & 1], ((sj >> 1) & 1) ^ 1)) {
+          tc_fence_after();
+          const uint32_t sQ = smem_u32(sm + L::kStage0 + (sj & 1) * L::kStageBytes);
+          const uint32_t sDO = sQ + L::kHalf;
+          const int sb = sj & 1;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws(tbase + sb * 64, kmajor_desc(sK, kk, kBoxBytes), kmajor_desc(sQ, kk, kKB * kBoxBytes), idS,
+                   kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws(tbase + 128 + sb * 64, kmajor_desc(sV, kk, kBoxBytes), kmajor_desc(sDO, kk, kKB * kBoxBytes), idS,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(&s_full[sb]);
+          ++sj;
+          did = true;
+        }
+        if (did) wd.reset();
+        else if (!wd.ok(status, abort_flag)) break;
       }
-      if (ok) issue_kv(nsteps - 1);
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, status);
     }

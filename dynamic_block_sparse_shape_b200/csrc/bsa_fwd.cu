@@ -7,18 +7,20 @@
 // style), fp32 statistics and accumulators, bf16 operands.
 //
 // One CTA per (query block I, head). Warp roles:
-//   warp 0      TMA producer: Q once, then per step the K and V boxes of two
-//               selected key blocks (5-D tensor maps, one per block shape),
-//               double-buffered;
+//   warp 0      TMA producer: Q once; per step the K boxes (3-slot ring) and V
+//               boxes (2-slot ring) of two selected key blocks, through 5-D
+//               tensor maps (one per block shape);
 //   warp 1      TMEM owner and single-thread tcgen05 issuer:
-//               S_j = Q K_j^T   (.ws M=64, N=128, K=d)       -> TMEM, 2 buffers
-//               O  += P_j V_j   (.ws M=64, N=d,   K=128)     -> TMEM
-//               issued as S_0, S_1, PV_0, S_2, PV_1, ... so the tensor core
-//               computes S_{j+1} while the softmax works on S_j;
+//               S_j = Q K_j^T   (.ws M=64, N=128, K=d)   -> TMEM, 3 buffers
+//               O  += P_j V_j   (.ws M=64, N=d,   K=128) -> TMEM
 //   warps 2..9  softmax: 256 threads, four per query row (two TMEM lane halves
 //               x two column halves, 32 keys each); row maxima are exchanged
 //               through shared memory; P_j goes to shared memory as the bf16
 //               K-major A operand of the PV product (double-buffered).
+// The producer and the issuer never block on one barrier: each polls the
+// barriers of every operation it could start next (mbarrier.test_wait) and
+// starts whichever is ready, so a late K load does not hold back a ready PV
+// product and a K slot is refilled as soon as its S product completes.
 // The running max is only moved when it grows by more than 8 (log2 units);
 // the final division uses the same stale max, so the result is exact while
 // the rare O rescale (TMEM load/scale/store) stays off the common path.
@@ -34,7 +36,9 @@ namespace prism {
 namespace {
 
 constexpr int kKB = 2;  // key blocks per step
-constexpr int kStages = 2;
+constexpr int kKSlots = 3;
+constexpr int kVSlots = 2;
+constexpr int kSBufs = 3;
 constexpr int kSoftWarps = 8;
 constexpr int kFwdThreads = 64 + 32 * kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
@@ -59,16 +63,16 @@ template <int D>
 struct FwdSmem {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kQBytes = D * 128;
-  static constexpr uint32_t kStageK = kKB * D * 128;
-  static constexpr uint32_t kStageBytes = 2 * kStageK;
-  static constexpr uint32_t kStage0 = kQBytes;
+  static constexpr uint32_t kSlotBytes = kKB * D * 128;  // K (or V) of one step
+  static constexpr uint32_t kK0 = kQBytes;
+  static constexpr uint32_t kV0 = kK0 + kKSlots * kSlotBytes;
   static constexpr uint32_t kPBytes = kKB * kBoxBytes;
-  static constexpr uint32_t kP0 = kStage0 + kStages * kStageBytes;
+  static constexpr uint32_t kP0 = kV0 + kVSlots * kSlotBytes;
   static constexpr uint32_t kRed = kP0 + 2 * kPBytes;
   static constexpr uint32_t kRedBytes = (2 * 4 * 64 + 4 * 64) * 4;
   static constexpr uint32_t kBar = kRed + kRedBytes;
   static constexpr uint32_t kTotal = kBar + 256;
-  static constexpr uint32_t kTmemCols = 256;  // S: 2 x 64 columns, O: d/2 columns
+  static constexpr uint32_t kTmemCols = 256;  // S: 3 x 64 columns, O: d/2 columns at 192
 };
 
 template <int D>
@@ -78,15 +82,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_free = bars + 7;
-  uint64_t* p_full = bars + 9;
-  uint64_t* p_free = bars + 11;
-  uint64_t* mma_done = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* k_full = bars + 1;    // [3]
+  uint64_t* k_empty = bars + 4;   // [3]
+  uint64_t* v_full = bars + 7;    // [2]
+  uint64_t* v_empty = bars + 9;   // [2]
+  uint64_t* s_full = bars + 11;   // [3]
+  uint64_t* s_free = bars + 14;   // [3]
+  uint64_t* p_full = bars + 17;   // [2]
+  uint64_t* p_free = bars + 19;   // [2]
+  uint64_t* mma_done = bars + 21;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 23);
   float* red = reinterpret_cast<float*>(sm + L::kRed);
   float* redl = red + 2 * 4 * 64;
 
@@ -105,11 +111,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < kKSlots; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kSoftWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&p_full[i], kSoftWarps);
       mbar_init(&p_free[i], 1);
     }
@@ -125,7 +139,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tO = tbase + 128;
+  const uint32_t tO = tbase + 192;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -135,34 +149,60 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       mbar_arrive_expect_tx(q_full, L::kQBytes);
       for (int dh = 0; dh < D / 64; ++dh)
         tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], q_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
-      int issued = 0;
-      for (int j = 0; j < nsteps; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_abortable(&kv_empty[st], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
-        uint8_t* stage = sm + L::kStage0 + st * L::kStageBytes;
-        mbar_arrive_expect_tx(&kv_full[st], L::kStageBytes);
-        for (int slot = 0; slot < kKB; ++slot) {
-          int idx = j * kKB + slot;
-          if (idx >= cnt) idx = j * kKB;  // ragged tail: repeat a valid block, masked by the softmax
-          int J = P.col_idx[beg + idx];
-          if (J < 0 || J >= g.n_blocks) {
-            atomicOr(status, kDevErrBounds);
-            J = 0;
-          }
-          const int sJ = safe_shape(g, P.zone_shape, J, status);
-          const BlockBox kb = block_box(g, sJ, J);
-          for (int dh = 0; dh < D / 64; ++dh) {
-            tma_load_5d(stage + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &P.mk[sJ], &kv_full[st], dh * 64, head,
-                        kb.w0, kb.h0, kb.t0);
-            tma_load_5d(stage + L::kStageK + slot * (D * 128) + dh * kBoxBytes, &P.mv[sJ], &kv_full[st], dh * 64,
-                        head, kb.w0, kb.h0, kb.t0);
-          }
+      // block of slot `slot` of step j (a ragged tail repeats a valid block; the softmax masks it)
+      auto block_of = [&](int j, int slot) -> int {
+        int e = j * kKB + slot;
+        if (e >= cnt) e = j * kKB;
+        int J = P.col_idx[beg + e];
+        if (J < 0 || J >= g.n_blocks) {
+          atomicOr(status, kDevErrBounds);
+          J = 0;
         }
-        ++issued;
+        return J;
+      };
+      int kj = 0, vj = 0;
+      Watchdog wd;
+      wd.reset();
+      while (kj < nsteps || vj < nsteps) {
+        bool did = false;
+        if (kj < nsteps && mbar_test(&k_empty[kj % kKSlots], ((kj / kKSlots) & 1) ^ 1)) {
+          const int ks = kj % kKSlots;
+          uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
+          mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
+          for (int slot = 0; slot < kKB; ++slot) {
+            const int J = block_of(kj, slot);
+            const int sJ = safe_shape(g, P.zone_shape, J, status);
+            const BlockBox kb = block_box(g, sJ, J);
+            for (int dh = 0; dh < D / 64; ++dh)
+              tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &P.mk[sJ], &k_full[ks], dh * 64, head,
+                          kb.w0, kb.h0, kb.t0);
+          }
+          ++kj;
+          did = true;
+        }
+        if (vj < kj && mbar_test(&v_empty[vj & 1], ((vj >> 1) & 1) ^ 1)) {
+          const int vs = vj & 1;
+          uint8_t* dst = sm + L::kV0 + vs * L::kSlotBytes;
+          mbar_arrive_expect_tx(&v_full[vs], L::kSlotBytes);
+          for (int slot = 0; slot < kKB; ++slot) {
+            const int J = block_of(vj, slot);
+            const int sJ = safe_shape(g, P.zone_shape, J, status);
+            const BlockBox kb = block_box(g, sJ, J);
+            for (int dh = 0; dh < D / 64; ++dh)
+              tma_load_5d(dst + slot * (D * 128) + dh * kBoxBytes, &P.mv[sJ], &v_full[vs], dh * 64, head, kb.w0,
+                          kb.h0, kb.t0);
+          }
+          ++vj;
+          did = true;
+        }
+        if (did) wd.reset();
+        else if (!wd.ok(status, abort_flag)) break;
       }
       // drain: every issued copy has landed before the CTA may exit
       mbar_wait(q_full, 0, status);
-      for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, status);
+      for (int i = kj - kKSlots > 0 ? kj - kKSlots : 0; i < kj; ++i)
+        mbar_wait(&k_full[i % kKSlots], (i / kKSlots) & 1, status);
+      for (int i = vj - kVSlots > 0 ? vj - kVSlots : 0; i < vj; ++i) mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -171,36 +211,40 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       const uint32_t idO = idesc_bf16_f32(64, D, false, true);
       const uint32_t sQ = smem_u32(sm + L::kQ);
       bool ok = mbar_wait_abortable(q_full, 0, status, abort_flag);
-      auto issue_pv = [&](int i) -> bool {
-        const int pb = i & 1;
-        if (!mbar_wait_abortable(&p_full[pb], (i >> 1) & 1, status, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t sP = smem_u32(sm + L::kP0 + pb * L::kPBytes);
-        const uint32_t sV = smem_u32(sm + L::kStage0 + (i & 1) * L::kStageBytes + L::kStageK);
+      int sj = 0, pj = 0;
+      Watchdog wd;
+      wd.reset();
+      while (ok && pj < nsteps) {
+        bool did = false;
+        if (pj < sj && mbar_test(&p_full[pj & 1], (pj >> 1) & 1) && mbar_test(&v_full[pj & 1], (pj >> 1) & 1)) {
+          tc_fence_after();
+          const uint32_t sP = smem_u32(sm + L::kP0 + (pj & 1) * L::kPBytes);
+          const uint32_t sV = smem_u32(sm + L::kV0 + (pj & 1) * L::kSlotBytes);
 #pragma unroll
-        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-          mma_ws(tO, kmajor_desc(sP, kk, kBoxBytes), mnmajor_desc(sV, kk, D * 128, kBoxBytes), idO, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&kv_empty[i & 1]);
-        mma_commit(&p_free[pb]);
-        return true;
-      };
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const int st = j & 1, sb = j & 1;
-        if (!mbar_wait_abortable(&kv_full[st], (j >> 1) & 1, status, abort_flag)) break;
-        if (!mbar_wait_abortable(&s_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t sK = smem_u32(sm + L::kStage0 + st * L::kStageBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws(tbase + sb * 64, kmajor_desc(sQ, kk, kBoxBytes), kmajor_desc(sK, kk, kKB * kBoxBytes), idS,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(&s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
+          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+            mma_ws(tO, kmajor_desc(sP, kk, kBoxBytes), mnmajor_desc(sV, kk, D * 128, kBoxBytes), idO,
+                   (pj > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&v_empty[pj & 1]);
+          mma_commit(&p_free[pj & 1]);
+          ++pj;
+          did = true;
         }
+        if (sj < nsteps && mbar_test(&k_full[sj % kKSlots], (sj / kKSlots) & 1) &&
+            mbar_test(&s_free[sj % kSBufs], ((sj / kSBufs) & 1) ^ 1)) {
+          tc_fence_after();
+          const uint32_t sK = smem_u32(sm + L::kK0 + (sj % kKSlots) * L::kSlotBytes);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws(tbase + (sj % kSBufs) * 64, kmajor_desc(sQ, kk, kBoxBytes), kmajor_desc(sK, kk, kKB * kBoxBytes),
+                   idS, kk > 0 ? 1u : 0u);
+          mma_commit(&s_full[sj % kSBufs]);
+          mma_commit(&k_empty[sj % kKSlots]);
+          ++sj;
+          did = true;
+        }
+        if (did) wd.reset();
+        else if (!wd.ok(status, abort_flag)) break;
       }
-      if (ok) issue_pv(nsteps - 1);
       // every MMA this thread issued has completed before TMEM is released
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, status);
@@ -216,8 +260,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
     float m_run = -INFINITY, l_part = 0.f;
     for (int j = 0; j < nsteps; ++j) {
-      const int sb = j & 1;
-      mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
+      const int sb = j % kSBufs, pb = j & 1, rb = j & 1;
+      mbar_wait_abortable(&s_full[sb], (j / kSBufs) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t r[32];
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, r);
@@ -233,10 +277,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         x[i] = valid ? __uint_as_float(r[i]) * P.scale_log2 : -INFINITY;
         mx = fmaxf(mx, x[i]);
       }
-      red[(sb * 4 + q4) * 64 + m] = mx;
+      red[(rb * 4 + q4) * 64 + m] = mx;
       named_bar_sync(1, 32 * kSoftWarps);
-      const float mb = fmaxf(fmaxf(red[(sb * 4 + 0) * 64 + m], red[(sb * 4 + 1) * 64 + m]),
-                             fmaxf(red[(sb * 4 + 2) * 64 + m], red[(sb * 4 + 3) * 64 + m]));
+      const float mb = fmaxf(fmaxf(red[(rb * 4 + 0) * 64 + m], red[(rb * 4 + 1) * 64 + m]),
+                             fmaxf(red[(rb * 4 + 2) * 64 + m], red[(rb * 4 + 3) * 64 + m]));
       const float m_new = fmaxf(m_run, mb);
       const bool resc = m_new > m_run + kRescaleThreshold;
       if (__any_sync(0xffffffffu, resc)) {
@@ -279,15 +323,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         pk[i] = pack_bf16x2(p0, p1);
       }
       l_part += lsum;
-      if (j >= 2) mbar_wait_abortable(&p_free[sb], ((j >> 1) & 1) ^ 1, status, abort_flag);
-      uint8_t* pt = sm + L::kP0 + sb * L::kPBytes + kh * kBoxBytes;
+      if (j >= 2) mbar_wait_abortable(&p_free[pb], ((j >> 1) & 1) ^ 1, status, abort_flag);
+      uint8_t* pt = sm + L::kP0 + pb * L::kPBytes + kh * kBoxBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
             make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (lane == 0) mbar_arrive(&p_full[pb]);
     }
     // ---------------------------------------------------------- epilogue
     if (nsteps > 0) mbar_wait_abortable(&p_free[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, status, abort_flag);
@@ -304,28 +348,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     const int doff = kh * (D / 2) + ch * NC;
     float ov[NC];
     if (nsteps > 0) {
-      uint32_t o[NC];
-      if constexpr (NC == 32) tmem_ld32(tO + lane_off + ch * NC, o);
-      else tmem_ld16(tO + lane_off + ch * NC, o);
-      tmem_ld_wait();
+      tmem_ld_f<NC>(tO + lane_off + ch * NC, ov);
 #pragma unroll
-      for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : __uint_as_float(o[i]) * inv;
+      for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : ov[i] * inv;
     } else {
 #pragma unroll
       for (int i = 0; i < NC; ++i) ov[i] = 0.f;
     }
-    const int64_t obase = int64_t(tok) * P.tok_stride + int64_t(head) * D + doff;
-    if (P.out_fp32) {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(P.o) + obase);
-#pragma unroll
-      for (int i = 0; i < NC / 4; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
-    } else {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.o) + obase);
-#pragma unroll
-      for (int i = 0; i < NC / 8; ++i)
-        dst[i] = make_uint4(pack_bf16x2(ov[8 * i], ov[8 * i + 1]), pack_bf16x2(ov[8 * i + 2], ov[8 * i + 3]),
-                            pack_bf16x2(ov[8 * i + 4], ov[8 * i + 5]), pack_bf16x2(ov[8 * i + 6], ov[8 * i + 7]));
-    }
+    store_row<NC>(P.o, int64_t(tok) * P.tok_stride + int64_t(head) * D + doff, ov, P.out_fp32);
     if (q4 == 0) {
       const int N = g.T * g.H * g.W;
       P.lse[int64_t(head) * N + tok] = (l > 0.f && ok) ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;

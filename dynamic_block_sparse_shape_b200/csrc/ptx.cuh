@@ -52,6 +52,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Progress watchdog for polling loops that test several barriers: returns
+// false (and raises the CTA abort flag) once no progress was made for the
+// wait limit, or when another CTA already timed out.
+struct Watchdog {
+  uint64_t last;
+  uint32_t spins;
+  __device__ __forceinline__ void reset() {
+    last = global_timer_ns();
+    spins = 0;
+  }
+  __device__ __forceinline__ bool ok(int* status, volatile int* abort) {
+    if (++spins & 255u) return true;
+    if (*abort) return false;
+    if (*reinterpret_cast<volatile int*>(status) & kDevErrTimeout) {
+      *abort = 1;
+      return false;
+    }
+    if (global_timer_ns() - last > PRISM_WAIT_LIMIT_NS) {
+      atomicOr(status, kDevErrTimeout);
+      *abort = 1;
+      return false;
+    }
+    return true;
+  }
+};
+
 // Bounded wait for the phase with the given parity to complete. On timeout
 // it ORs kDevErrTimeout into *status and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
