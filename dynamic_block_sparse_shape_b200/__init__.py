@@ -68,6 +68,8 @@ _SIGNATURES = {
     "prism_check_device_status": (ctypes.c_int, [_P, _P]),
     "prism_zone_shapes": (ctypes.c_int, [_GEO, _P, _I64, _I32, ctypes.c_int, _P, _I64, _I32, ctypes.c_int,
                                          ctypes.POINTER(_ShapeParams), _P, _P, _P, _SZ, _P]),
+    "prism_zone_shapes_static": (ctypes.c_int, [_GEO, _P, _I64, _I32, ctypes.c_int, _P, _I64, _I32, ctypes.c_int,
+                                                ctypes.POINTER(_ShapeParams), _P, _P, _P]),
     "prism_block_pool": (ctypes.c_int, [_GEO, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _P, _P, _P, _SZ, _P]),
     "prism_block_select": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, _I32, _F32, _P, _P, _P, _P, _I64,
                                           ctypes.POINTER(_I64), _P, _SZ, _P]),

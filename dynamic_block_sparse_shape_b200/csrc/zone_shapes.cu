@@ -24,6 +24,7 @@
 #include <algorithm>
 #include <cfloat>
 #include <cmath>
+#include <mutex>
 
 #include "host.h"
 #include "ptx.cuh"
@@ -365,6 +366,119 @@ extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void*
     const size_t smem = size_t(kFeatStages) * g.Zt * g.Zh * g.Zw * 128 + 1024;
     const int n_tiles = g.n_zones * n_chunks;
     const int grid = std::min(n_tiles, sm_count());
+    if (fes == 2) {
+      cudaFuncSetAttribute(feat_stats_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      feat_stats_kernel<2><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
+    } else {
+      cudaFuncSetAttribute(feat_stats_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      feat_stats_kernel<4><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
+    }
+    if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
+  }
+  if (res) {
+    const int res_es = res_dtype == PRISM_FP32 ? 4 : 2;
+    if ((int64_t(res_c) * res_es) % 16) return PRISM_ERR_ARG;
+    const int blocks = (N + 7) / 8;
+    if (res_es == 2)
+      res_norm_kernel<2><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(res), res_ld * res_es,
+                                                res_c * res_es, N, r);
+    else
+      res_norm_kernel<4><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(res), res_ld * res_es,
+                                                res_c * res_es, N, r);
+    zone_res_kernel<<<g.n_zones, 256, 0, s>>>(g, r, zres);
+    if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
+  }
+  choose_kernel<<<1, 1024, 0, s>>>(g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio,
+                                   p.gamma, p.gate_max, zone_shape, zone_margin);
+  return cuda_status(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of prism_zone_shapes. The scratch (per-zone channel
+// partial sums, per-token residual norms, per-zone residual statistics and the
+// status word) lives in one file-scope device array instead of a caller
+// workspace. Host code only ever sees the array's host-side shadow, so the
+// device address is looked up once per device with cudaGetSymbolAddress.
+namespace prism {
+namespace {
+
+constexpr size_t kZoneStaticBytes = size_t(4) << 20;  // 4 MiB, held by every GPU that loads the library
+static __device__ __align__(256) uint8_t g_zone_scratch[kZoneStaticBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_zone_scratch on the current device (set up on first use).
+prism_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_zone_scratch) != cudaSuccess || !p) return PRISM_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return PRISM_OK;
+}
+
+}  // namespace
+}  // namespace prism
+
+extern "C" prism_status prism_zone_shapes_static(const prism_geometry* geo, const void* feat, int64_t feat_ld,
+                                                 int32_t feat_c, prism_dtype feat_dtype, const void* res,
+                                                 int64_t res_ld, int32_t res_c, prism_dtype res_dtype,
+                                                 const prism_shape_params* params, int32_t* zone_shape,
+                                                 float* zone_margin, void* stream) {
+  Geo g;
+  prism_status st = make_geo(geo, &g);
+  if (st != PRISM_OK) return st;
+  if (!zone_shape) return PRISM_ERR_ARG;
+  const prism_shape_params def = {1.0f, 0.25f, 4.0f};
+  const prism_shape_params p = params ? *params : def;
+  if (!(p.gamma >= 0.f) || !(p.w_audio >= 0.f) || !(p.gate_max >= 0.f)) return PRISM_ERR_ARG;
+  if (feat) {
+    if (feat_dtype != PRISM_BF16 && feat_dtype != PRISM_FP32) return PRISM_ERR_DTYPE;
+    if (feat_c <= 0 || feat_c % 64 || feat_ld < feat_c || feat_ld % 8) return PRISM_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(feat) % 16) return PRISM_ERR_ARG;
+  } else {
+    feat_c = 0;
+  }
+  if (res) {
+    if (res_dtype != PRISM_BF16 && res_dtype != PRISM_FP32) return PRISM_ERR_DTYPE;
+    if (res_c <= 0 || res_c % 8 || res_ld < res_c || res_ld % 8) return PRISM_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(res) % 16) return PRISM_ERR_ARG;
+  } else {
+    res_c = 0;
+  }
+  const int fes = feat_dtype == PRISM_FP32 ? 4 : 2;
+  const ZoneWs L = zone_ws_layout(g, feat_c, fes, res_c);
+  if (L.total > kZoneStaticBytes) return PRISM_ERR_UNSUPPORTED;  // grid too large for the static scratch
+  void* scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != PRISM_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w8 = static_cast<uint8_t*>(scratch);
+  float* partial = reinterpret_cast<float*>(w8 + L.partial);
+  float* r = reinterpret_cast<float*>(w8 + L.r);
+  double* zres = reinterpret_cast<double*>(w8 + L.zres);
+  int* status = ws_status(scratch);
+  // the status word is the only scratch a kernel reads before writing it
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return PRISM_ERR_CUDA;
+  const int N = g.T * g.H * g.W;
+  const int n_chunks = feat_c * fes / 128;
+  if (feat) {
+    CUtensorMap fmap;
+    const uint64_t dims[4] = {uint64_t(feat_c), uint64_t(g.W), uint64_t(g.H), uint64_t(g.T)};
+    const uint64_t strides[3] = {uint64_t(feat_ld) * fes, uint64_t(feat_ld) * fes * g.W,
+                                 uint64_t(feat_ld) * fes * g.W * g.H};
+    const uint32_t box[4] = {uint32_t(128 / fes), uint32_t(g.Zw), uint32_t(g.Zh), uint32_t(g.Zt)};
+    st = encode_tiled(&fmap, fes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, feat,
+                      dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != PRISM_OK) return st;
+    const size_t smem = size_t(kFeatStages) * g.Zt * g.Zh * g.Zw * 128 + 1024;
+    const int grid = std::min(g.n_zones * n_chunks, sm_count());
     if (fes == 2) {
       cudaFuncSetAttribute(feat_stats_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
       feat_stats_kernel<2><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);

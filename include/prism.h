@@ -155,6 +155,35 @@ PRISM_API prism_status prism_zone_shapes(const prism_geometry* geo, const void* 
                                float* zone_margin, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * prism_zone_shapes without a workspace (the Prism pages have no counterpart
+ * to this entry point; it is a deployment variant of a1 + a2).
+ *
+ * For callers that cannot allocate device memory: code that runs inside a
+ * host framework owning every device allocation (a serving runtime's fixed
+ * pool, a plugin interface that hands out no scratch buffer), or code that must
+ * not call cudaMalloc after start-up because it would synchronise the device
+ * in the middle of its work. Inputs, outputs and the result are exactly those
+ * of prism_zone_shapes; only the scratch differs: it lives in one static
+ * device array of 4 MiB inside the library, which every GPU that loads the
+ * library holds until the process exits. That bounds the grid: about 7 bytes
+ * per token plus 32 per zone with 3072 bf16 channels (the 2K grid of 294,912
+ * tokens needs 2.1 MB); a call that needs more returns PRISM_ERR_UNSUPPORTED.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine). The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress with that device current); make that first call before
+ * any stream capture. All calls share the array and it keeps the last call's
+ * contents, so calls that overlap on the GPU (different streams, or several
+ * host threads) race and must be serialised by the caller. Device-side wait
+ * timeouts are not reported by this variant (there is no workspace to hold
+ * the status word the caller could read back).
+ */
+PRISM_API prism_status prism_zone_shapes_static(const prism_geometry* geo, const void* feat, int64_t feat_ld,
+                                                int32_t feat_c, prism_dtype feat_dtype, const void* res,
+                                                int64_t res_ld, int32_t res_c, prism_dtype res_dtype,
+                                                const prism_shape_params* params, int32_t* zone_shape,
+                                                float* zone_margin, void* stream);
+
+/*
  * a3 — block partition and mean pooling ("block-level features", README
  * "Overview"): q_pool[h, b, :] = mean of the 64 rows Q[n, h, :] of block b,
  * likewise k_pool.
