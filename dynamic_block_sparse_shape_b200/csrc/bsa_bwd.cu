@@ -75,7 +75,8 @@ struct DqSmem {
   static constexpr uint32_t kV0 = kK0 + kDqKSlots * kSlotBytes;
   static constexpr uint32_t kDS = kV0 + kDqVSlots * kSlotBytes;
   static constexpr uint32_t kDSBytes = kKB * kBoxBytes;
-  static constexpr uint32_t kBar = kDS + kDSBytes;
+  static constexpr uint32_t kDesc = kDS + kDSBytes;  // block coordinate ring
+  static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
 };
 
@@ -141,58 +142,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   const uint32_t tdQ = tbase + 384;
 
   if (warp == 0) {
-    if (lane == 0 && nsteps > 0) {
-      const int sI = safe_shape(g, P.zone_shape, I, status);
-      const BlockBox qb = block_box(g, sI, I);
-      mbar_arrive_expect_tx(qd_full, 2 * D * 128);
-      for (int dh = 0; dh < D / 64; ++dh) {
-        tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
-        tma_load_5d(sm + L::kDO + dh * kBoxBytes, &P.mdo[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
-      }
-      auto block_of = [&](int j, int slot) -> int {
-        int e = j * kKB + slot;
-        if (e >= cnt) e = j * kKB;
-        int J = P.idx[beg + e];
-        if (J < 0 || J >= g.n_blocks) {
-          atomicOr(status, kDevErrBounds);
-          J = 0;
+    if (nsteps > 0) {
+      DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
+      if (lane == 0) {
+        const int sI = safe_shape(g, P.zone_shape, I, status);
+        const BlockBox qb = block_box(g, sI, I);
+        mbar_arrive_expect_tx(qd_full, 2 * D * 128);
+        for (int dh = 0; dh < D / 64; ++dh) {
+          tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+          tma_load_5d(sm + L::kDO + dh * kBoxBytes, &P.mdo[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
         }
-        return J;
-      };
+      }
       auto load_step = [&](const CUtensorMap* maps, uint8_t* dst, uint64_t* bar, int j) {
         mbar_arrive_expect_tx(bar, L::kSlotBytes);
         for (int slot = 0; slot < kKB; ++slot) {
-          const int J = block_of(j, slot);
-          const int sJ = safe_shape(g, P.zone_shape, J, status);
-          const BlockBox kb = block_box(g, sJ, J);
+          const int4 b = dc.get(kKB * j + slot);
           for (int dh = 0; dh < D / 64; ++dh)
-            tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &maps[sJ], bar, dh * 64, head, kb.w0, kb.h0,
-                        kb.t0);
+            tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &maps[b.x], bar, dh * 64, head, b.y, b.z,
+                        b.w);
         }
       };
       int kj = 0, vj = 0;
       Watchdog wd;
       wd.reset();
       while (kj < nsteps || vj < nsteps) {
-        bool did = false;
-        if (kj < nsteps && mbar_test(&k_empty[kj % kDqKSlots], ((kj / kDqKSlots) & 1) ^ 1)) {
-          load_step(P.mk, sm + L::kK0 + (kj % kDqKSlots) * L::kSlotBytes, &k_full[kj % kDqKSlots], kj);
-          ++kj;
-          did = true;
+        if (kj < nsteps) dc.ensure(kKB * kj + kKB - 1, g, P.idx, beg, cnt, P.zone_shape, status, lane);
+        int nk = kj, nv = vj, stop = 0;
+        if (lane == 0) {
+          bool did = false;
+          if (nk < nsteps && mbar_test(&k_empty[nk % kDqKSlots], ((nk / kDqKSlots) & 1) ^ 1)) {
+            load_step(P.mk, sm + L::kK0 + (nk % kDqKSlots) * L::kSlotBytes, &k_full[nk % kDqKSlots], nk);
+            ++nk;
+            did = true;
+          }
+          if (nv < nk && mbar_test(&v_empty[nv & 1], ((nv >> 1) & 1) ^ 1)) {
+            load_step(P.mv, sm + L::kV0 + (nv & 1) * L::kSlotBytes, &v_full[nv & 1], nv);
+            ++nv;
+            did = true;
+          }
+          if (did) wd.reset();
+          else if (!wd.ok(status, abort_flag)) stop = 1;
         }
-        if (vj < kj && mbar_test(&v_empty[vj & 1], ((vj >> 1) & 1) ^ 1)) {
-          load_step(P.mv, sm + L::kV0 + (vj & 1) * L::kSlotBytes, &v_full[vj & 1], vj);
-          ++vj;
-          did = true;
-        }
-        if (did) wd.reset();
-        else if (!wd.ok(status, abort_flag)) break;
+        kj = __shfl_sync(0xffffffffu, nk, 0);
+        vj = __shfl_sync(0xffffffffu, nv, 0);
+        if (__shfl_sync(0xffffffffu, stop, 0)) break;
       }
-      mbar_wait(qd_full, 0, status);
-      for (int i = kj - kDqKSlots > 0 ? kj - kDqKSlots : 0; i < kj; ++i)
-        mbar_wait(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, status);
-      for (int i = vj - kDqVSlots > 0 ? vj - kDqVSlots : 0; i < vj; ++i)
-        mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
+      if (lane == 0) {
+        mbar_wait(qd_full, 0, status);
+        for (int i = kj - kDqKSlots > 0 ? kj - kDqKSlots : 0; i < kj; ++i)
+          mbar_wait(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, status);
+        for (int i = vj - kDqVSlots > 0 ? vj - kDqVSlots : 0; i < vj; ++i)
+          mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && nsteps > 0) {
@@ -324,7 +325,8 @@ struct DkvSmem {
   static constexpr uint32_t kPT = kStage0 + 2 * kStageBytes;
   static constexpr uint32_t kPBytes = kKB * kBoxBytes;
   static constexpr uint32_t kDST = kPT + kPBytes;
-  static constexpr uint32_t kBar = kDST + kPBytes;
+  static constexpr uint32_t kDesc = kDST + kPBytes;  // block coordinate ring
+  static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
 };
 
@@ -382,43 +384,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   const uint32_t tdV = tbase + 256, tdK = tbase + 384;
 
   if (warp == 0) {
-    if (lane == 0 && nsteps > 0) {
-      const int sJ = safe_shape(g, P.zone_shape, J, status);
-      const BlockBox kb = block_box(g, sJ, J);
-      mbar_arrive_expect_tx(kv_full, 2 * D * 128);
-      for (int dh = 0; dh < D / 64; ++dh) {
-        tma_load_5d(sm + L::kK + dh * kBoxBytes, &P.mk[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
-        tma_load_5d(sm + L::kV + dh * kBoxBytes, &P.mv[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
+    if (nsteps > 0) {
+      DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
+      if (lane == 0) {
+        const int sJ = safe_shape(g, P.zone_shape, J, status);
+        const BlockBox kb = block_box(g, sJ, J);
+        mbar_arrive_expect_tx(kv_full, 2 * D * 128);
+        for (int dh = 0; dh < D / 64; ++dh) {
+          tma_load_5d(sm + L::kK + dh * kBoxBytes, &P.mk[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
+          tma_load_5d(sm + L::kV + dh * kBoxBytes, &P.mv[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
+        }
       }
       int issued = 0;
-      for (int j = 0; j < nsteps; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_abortable(&st_empty[st], ((j >> 1) & 1) ^ 1, status, abort_flag)) break;
-        uint8_t* stage = sm + L::kStage0 + st * L::kStageBytes;
-        mbar_arrive_expect_tx(&st_full[st], 2 * L::kHalf + kKB * 2 * 256);
-        for (int slot = 0; slot < kKB; ++slot) {
-          int e = j * kKB + slot;
-          if (e >= cnt) e = j * kKB;
-          int I = P.idx[beg + e];
-          if (I < 0 || I >= g.n_blocks) {
-            atomicOr(status, kDevErrBounds);
-            I = 0;
+      Watchdog wd;
+      wd.reset();
+      while (issued < nsteps) {
+        const int j = issued;
+        dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, P.zone_shape, status, lane);
+        int go = 0, stop = 0;
+        if (lane == 0) {
+          if (mbar_test(&st_empty[j & 1], ((j >> 1) & 1) ^ 1)) {
+            uint8_t* stage = sm + L::kStage0 + (j & 1) * L::kStageBytes;
+            uint64_t* bar = &st_full[j & 1];
+            mbar_arrive_expect_tx(bar, 2 * L::kHalf + kKB * 2 * 256);
+            for (int slot = 0; slot < kKB; ++slot) {
+              const int4 b = dc.get(kKB * j + slot);
+              for (int dh = 0; dh < D / 64; ++dh) {
+                const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
+                tma_load_5d(stage + off, &P.mq[b.x], bar, dh * 64, head, b.y, b.z, b.w);
+                tma_load_5d(stage + L::kHalf + off, &P.mdo[b.x], bar, dh * 64, head, b.y, b.z, b.w);
+              }
+              int e = kKB * j + slot;
+              if (e >= cnt) e = kKB * j;
+              int Iq = P.idx[beg + e];
+              if (Iq < 0 || Iq >= g.n_blocks) Iq = 0;  // reported by the coordinate cache
+              const size_t rowoff = (size_t(head) * g.n_blocks + Iq) * 64;
+              bulk_load(stage + L::kLD + slot * 256, P.lse2 + rowoff, 256, bar);
+              bulk_load(stage + L::kLD + 512 + slot * 256, P.dvec + rowoff, 256, bar);
+            }
+            go = 1;
+            wd.reset();
+          } else if (!wd.ok(status, abort_flag)) {
+            stop = 1;
           }
-          const int sI = safe_shape(g, P.zone_shape, I, status);
-          const BlockBox qb = block_box(g, sI, I);
-          for (int dh = 0; dh < D / 64; ++dh) {
-            const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
-            tma_load_5d(stage + off, &P.mq[sI], &st_full[st], dh * 64, head, qb.w0, qb.h0, qb.t0);
-            tma_load_5d(stage + L::kHalf + off, &P.mdo[sI], &st_full[st], dh * 64, head, qb.w0, qb.h0, qb.t0);
-          }
-          const size_t rowoff = (size_t(head) * g.n_blocks + I) * 64;
-          bulk_load(stage + L::kLD + slot * 256, P.lse2 + rowoff, 256, &st_full[st]);
-          bulk_load(stage + L::kLD + 512 + slot * 256, P.dvec + rowoff, 256, &st_full[st]);
         }
-        ++issued;
+        issued += __shfl_sync(0xffffffffu, go, 0);
+        if (__shfl_sync(0xffffffffu, stop, 0)) break;
       }
-      mbar_wait(kv_full, 0, status);
-      for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i) mbar_wait(&st_full[i & 1], (i >> 1) & 1, status);
+      if (lane == 0) {
+        mbar_wait(kv_full, 0, status);
+        for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
+          mbar_wait(&st_full[i & 1], (i >> 1) & 1, status);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0 && nsteps > 0) {

@@ -57,6 +57,39 @@ __device__ __forceinline__ int safe_shape(const Geo& g, const int32_t* zone_shap
   return s;
 }
 
+// TMA coordinates (shape, w0, h0, t0) of the blocks named by a CSR / CSC list,
+// computed 32 at a time by a whole warp (coalesced list reads, parallel
+// zone-shape lookups) into a shared-memory ring, so the thread that issues the
+// TMA copies never waits on a dependent global load. Entry e of a list of
+// `cnt` blocks processed two per step: e < cnt is the list's e-th block; a
+// ragged tail (e >= cnt in the last step) repeats the step's first block.
+constexpr int kDescRing = 64;
+
+struct DescCache {
+  int4* ring;  // shared memory, kDescRing entries
+  int filled;
+  // Makes entries [0, e] available; the whole warp must call it.
+  __device__ __forceinline__ void ensure(int e, const Geo& g, const int32_t* list, int beg, int cnt,
+                                         const int32_t* zone_shape, int* status, int lane) {
+    while (e >= filled) {
+      const int ee = filled + lane;
+      int idx = ee < cnt ? ee : (ee & ~1);
+      if (idx >= cnt) idx = 0;
+      int J = list[beg + idx];
+      if (J < 0 || J >= g.n_blocks) {
+        atomicOr(status, kDevErrBounds);
+        J = 0;
+      }
+      const int s = safe_shape(g, zone_shape, J, status);
+      const BlockBox bb = block_box(g, s, J);
+      ring[ee % kDescRing] = make_int4(s, bb.w0, bb.h0, bb.t0);
+      __syncwarp();
+      filled += 32;
+    }
+  }
+  __device__ __forceinline__ int4 get(int e) const { return ring[e % kDescRing]; }
+};
+
 // Store 32 (or 16) fp32 values as bf16 or fp32 at dst (16-byte aligned).
 template <int NC>
 __device__ __forceinline__ void store_row(void* dst, int64_t off, const float* v, bool fp32) {

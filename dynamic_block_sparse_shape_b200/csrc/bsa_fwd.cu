@@ -70,7 +70,8 @@ struct FwdSmem {
   static constexpr uint32_t kP0 = kV0 + kVSlots * kSlotBytes;
   static constexpr uint32_t kRed = kP0 + 2 * kPBytes;
   static constexpr uint32_t kRedBytes = (2 * 4 * 64 + 4 * 64) * 4;
-  static constexpr uint32_t kBar = kRed + kRedBytes;
+  static constexpr uint32_t kDesc = kRed + kRedBytes;  // block coordinate ring
+  static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
   static constexpr uint32_t kTmemCols = 256;  // S: 3 x 64 columns, O: d/2 columns at 192
 };
@@ -143,66 +144,64 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && nsteps > 0) {
-      const int sI = safe_shape(g, P.zone_shape, I, status);
-      const BlockBox qb = block_box(g, sI, I);
-      mbar_arrive_expect_tx(q_full, L::kQBytes);
-      for (int dh = 0; dh < D / 64; ++dh)
-        tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], q_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
-      // block of slot `slot` of step j (a ragged tail repeats a valid block; the softmax masks it)
-      auto block_of = [&](int j, int slot) -> int {
-        int e = j * kKB + slot;
-        if (e >= cnt) e = j * kKB;
-        int J = P.col_idx[beg + e];
-        if (J < 0 || J >= g.n_blocks) {
-          atomicOr(status, kDevErrBounds);
-          J = 0;
-        }
-        return J;
-      };
+    if (nsteps > 0) {
+      DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
+      if (lane == 0) {
+        const int sI = safe_shape(g, P.zone_shape, I, status);
+        const BlockBox qb = block_box(g, sI, I);
+        mbar_arrive_expect_tx(q_full, L::kQBytes);
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], q_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+      }
       int kj = 0, vj = 0;
       Watchdog wd;
       wd.reset();
       while (kj < nsteps || vj < nsteps) {
-        bool did = false;
-        if (kj < nsteps && mbar_test(&k_empty[kj % kKSlots], ((kj / kKSlots) & 1) ^ 1)) {
-          const int ks = kj % kKSlots;
-          uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
-          mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
-          for (int slot = 0; slot < kKB; ++slot) {
-            const int J = block_of(kj, slot);
-            const int sJ = safe_shape(g, P.zone_shape, J, status);
-            const BlockBox kb = block_box(g, sJ, J);
-            for (int dh = 0; dh < D / 64; ++dh)
-              tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &P.mk[sJ], &k_full[ks], dh * 64, head,
-                          kb.w0, kb.h0, kb.t0);
+        if (kj < nsteps) dc.ensure(kKB * kj + kKB - 1, g, P.col_idx, beg, cnt, P.zone_shape, status, lane);
+        int nk = kj, nv = vj, stop = 0;
+        if (lane == 0) {
+          bool did = false;
+          if (nk < nsteps && mbar_test(&k_empty[nk % kKSlots], ((nk / kKSlots) & 1) ^ 1)) {
+            const int ks = nk % kKSlots;
+            uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
+            mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
+            for (int slot = 0; slot < kKB; ++slot) {
+              const int4 b = dc.get(kKB * nk + slot);
+              for (int dh = 0; dh < D / 64; ++dh)
+                tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &P.mk[b.x], &k_full[ks], dh * 64, head,
+                            b.y, b.z, b.w);
+            }
+            ++nk;
+            did = true;
           }
-          ++kj;
-          did = true;
-        }
-        if (vj < kj && mbar_test(&v_empty[vj & 1], ((vj >> 1) & 1) ^ 1)) {
-          const int vs = vj & 1;
-          uint8_t* dst = sm + L::kV0 + vs * L::kSlotBytes;
-          mbar_arrive_expect_tx(&v_full[vs], L::kSlotBytes);
-          for (int slot = 0; slot < kKB; ++slot) {
-            const int J = block_of(vj, slot);
-            const int sJ = safe_shape(g, P.zone_shape, J, status);
-            const BlockBox kb = block_box(g, sJ, J);
-            for (int dh = 0; dh < D / 64; ++dh)
-              tma_load_5d(dst + slot * (D * 128) + dh * kBoxBytes, &P.mv[sJ], &v_full[vs], dh * 64, head, kb.w0,
-                          kb.h0, kb.t0);
+          if (nv < nk && mbar_test(&v_empty[nv & 1], ((nv >> 1) & 1) ^ 1)) {
+            const int vs = nv & 1;
+            uint8_t* dst = sm + L::kV0 + vs * L::kSlotBytes;
+            mbar_arrive_expect_tx(&v_full[vs], L::kSlotBytes);
+            for (int slot = 0; slot < kKB; ++slot) {
+              const int4 b = dc.get(kKB * nv + slot);
+              for (int dh = 0; dh < D / 64; ++dh)
+                tma_load_5d(dst + slot * (D * 128) + dh * kBoxBytes, &P.mv[b.x], &v_full[vs], dh * 64, head, b.y,
+                            b.z, b.w);
+            }
+            ++nv;
+            did = true;
           }
-          ++vj;
-          did = true;
+          if (did) wd.reset();
+          else if (!wd.ok(status, abort_flag)) stop = 1;
         }
-        if (did) wd.reset();
-        else if (!wd.ok(status, abort_flag)) break;
+        kj = __shfl_sync(0xffffffffu, nk, 0);
+        vj = __shfl_sync(0xffffffffu, nv, 0);
+        if (__shfl_sync(0xffffffffu, stop, 0)) break;
       }
-      // drain: every issued copy has landed before the CTA may exit
-      mbar_wait(q_full, 0, status);
-      for (int i = kj - kKSlots > 0 ? kj - kKSlots : 0; i < kj; ++i)
-        mbar_wait(&k_full[i % kKSlots], (i / kKSlots) & 1, status);
-      for (int i = vj - kVSlots > 0 ? vj - kVSlots : 0; i < vj; ++i) mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
+      if (lane == 0) {
+        // drain: every issued copy has landed before the CTA may exit
+        mbar_wait(q_full, 0, status);
+        for (int i = kj - kKSlots > 0 ? kj - kKSlots : 0; i < kj; ++i)
+          mbar_wait(&k_full[i % kKSlots], (i / kKSlots) & 1, status);
+        for (int i = vj - kVSlots > 0 ? vj - kVSlots : 0; i < vj; ++i)
+          mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

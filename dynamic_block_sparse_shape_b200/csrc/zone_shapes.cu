@@ -113,10 +113,16 @@ __global__ void __launch_bounds__(kFeatThreads, 1)
           step = 1;
         }
         float s0 = 0.f, s1 = 0.f;
-        for (int i = 0; i < La; ++i) {
-          const float2 x = load_word<ES>(base + (r0 + i * step) * 128);
-          s0 += x.x;
-          s1 += x.y;
+        for (int i0 = 0; i0 < La; i0 += 8) {
+          float2 x[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)  // eight independent shared loads in flight
+            x[i] = i0 + i < La ? load_word<ES>(base + (r0 + (i0 + i) * step) * 128) : make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            s0 += x[i].x;
+            s1 += x[i].y;
+          }
         }
         acc = fmaf(s0, s0, fmaf(s1, s1, acc));
       }
