@@ -96,6 +96,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def max_over_ranks(value: float, device="cpu") -> float:
+    """The largest per-rank value (timings are reported as the slowest rank);
+    a no-op without an initialised process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_ms_per_layer(ms_per_step_max: float, world: int) -> float:
+    """Replicas: every rank runs one layer per step, so the job finishes
+    `world` layers in the slowest rank's step time."""
+    return ms_per_step_max / world
+
+
 # ---------------------------------------------------------------------------- GPU arm
 def build_inputs(wl, device):
     import torch
@@ -346,11 +364,7 @@ def run_gpu(args):
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    ms_total = e0.elapsed_time(e1)
-    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = float(t.item()) / args.steps
+    ms_step = max_over_ranks(e0.elapsed_time(e1), device=dev) / args.steps
     stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) / len(v) for k, v in rec.items()}
     pipe.P.check_device_status(pipe.ws)
     # end to end through the public API with host buffers
@@ -362,7 +376,7 @@ def run_gpu(args):
     achieved = attn_flop / t_attn / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     out = {
-        "metric": METRIC, "value": round(ms_step / world, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": round(whole_job_ms_per_layer(ms_step, world), 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{wl.name}: grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]} ({wl.n_tokens} tokens), "
@@ -382,8 +396,8 @@ def run_gpu(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_sample(wl, x, feats, res, q_blocks=24, kv_blocks=4, sel_rows=1024,
-                                         users_per_kv=16)
+        out["cpu_baseline"] = cpu_sample(wl, x, feats, res, q_blocks=160, kv_blocks=8, sel_rows=4608,
+                                         users_per_kv=48)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -462,6 +476,53 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_sweep(args):
+    """The selection/sparsity sweep on the 2K grid: for amplitude x top_k x
+    cdf_threshold, kept-block statistics per row and fwd / bwd times."""
+    import numpy as np
+    import torch
+    from dynamic_block_sparse_shape_b200 import synth
+    from dynamic_block_sparse_shape_b200 import build as pbuild
+    pbuild.build()
+    dev = torch.device("cuda")
+    points = synth.sweep_workloads()
+    by_amp = {}
+    for wl in points:
+        by_amp.setdefault(wl.amplitude, []).append(wl)
+    for amp, wls in by_amp.items():
+        x, feats, res = build_inputs(wls[0], dev)
+        pipe = None
+        for wl in wls:
+            if pipe is None:
+                pipe = Pipeline(wl, x, feats, res)
+            pipe.wl = wl
+            sel = pipe.P.block_select(pipe.qp, pipe.kp, pipe.scale, wl.top_k, wl.cdf_threshold, ws=pipe.ws,
+                                      csr=False)
+            pipe.nnz = sel["total"]
+            pipe.col_idx = torch.empty(max(1, pipe.nnz), dtype=torch.int32, device=dev)
+            pipe.ws.ensure(pipe.P.workspace_size("bsa_bwd", pipe.geo, heads=wl.heads, head_dim=wl.head_dim,
+                                                 nnz=pipe.nnz))
+            kept = sel["kept"].cpu().numpy().ravel()
+            rec = {}
+            for rep in range(2):  # one warm-up, one timed
+                rec = {}
+                pipe.step(record=rec)
+                torch.cuda.synchronize()
+            ms = {k: v[0][0].elapsed_time(v[0][1]) for k, v in rec.items()}
+            t_attn = (ms["bsa_fwd"] + ms["bsa_bwd"]) * 1e-3
+            pipe.P.check_device_status(pipe.ws)
+            print(json.dumps({
+                "point": wl.name, "amplitude": amp, "top_k": wl.top_k, "cdf_threshold": wl.cdf_threshold,
+                "kept_mean": round(float(kept.mean()), 2), "kept_p50": float(np.percentile(kept, 50)),
+                "kept_p99": float(np.percentile(kept, 99)), "kept_max": int(kept.max()),
+                "density": round(pipe.nnz / (wl.heads * pipe.nb * pipe.nb), 5), "pairs": pipe.nnz,
+                "stage_ms": {k: round(v, 3) for k, v in ms.items()},
+                "tflops": round(pipe.nnz * (FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR) / t_attn / 1e12, 1)}),
+                flush=True)
+        del pipe, x, feats, res
+        torch.cuda.empty_cache()
+
+
 def _cpu_inputs(wl):
     from dynamic_block_sparse_shape_b200 import synth
     x = synth.qkv(wl)
@@ -481,10 +542,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="run the 45-point selection/sparsity sweep instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.sweep:
+        run_sweep(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

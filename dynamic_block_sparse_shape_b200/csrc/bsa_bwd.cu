@@ -64,7 +64,7 @@ struct BwdParams {
 // barrier they could act on and start whichever operation is ready.
 constexpr int kDqKSlots = 3;
 constexpr int kDqVSlots = 2;
-constexpr int kDqSBufs = 3;
+constexpr int kDqSBufs = 2;
 
 template <int D>
 struct DqSmem {
@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   uint64_t* mma_done = bars + 19;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
+  uint64_t* qa_full = bars + 22;  // Q and dO copied into TMEM by the softmax warps
 
   const Geo& g = P.g;
   const int I = blockIdx.x, head = blockIdx.y;
@@ -128,6 +129,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     mbar_init(ds_full, kSoftWarps);
     mbar_init(ds_free, 1);
     mbar_init(mma_done, 1);
+    mbar_init(qa_full, kSoftWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -139,7 +141,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tdQ = tbase + 384;
+  // TMEM columns: S [2 x 64] at 0, dP [2 x 64] at 128, dQ at 256, Q at 320, dO at 384
+  const uint32_t tdQ = tbase + 256, tQ = tbase + 320, tDO = tbase + 384;
 
   if (warp == 0) {
     if (nsteps > 0) {
@@ -199,8 +202,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
-      const uint32_t sQ = smem_u32(sm + L::kQ), sDO = smem_u32(sm + L::kDO), sDS = smem_u32(sm + L::kDS);
-      bool ok = mbar_wait_abortable(qd_full, 0, status, abort_flag);
+      const uint32_t sDS = smem_u32(sm + L::kDS);
+      bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
+      tc_fence_after();
       int sj = 0, qj = 0;
       Watchdog wd;
       wd.reset();
@@ -226,12 +230,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
           const int sb = sj % kDqSBufs;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws(tbase + sb * 64, kmajor_desc(sQ, kk, kBoxBytes), kmajor_desc(sK, kk, kKB * kBoxBytes), idS,
-                   kk > 0 ? 1u : 0u);
+            mma_ws_ts(tbase + sb * 64, tQ + kk * 8, kmajor_desc(sK, kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws(tbase + 192 + sb * 64, kmajor_desc(sDO, kk, kBoxBytes), kmajor_desc(sV, kk, kKB * kBoxBytes), idS,
-                   kk > 0 ? 1u : 0u);
+            mma_ws_ts(tbase + 128 + sb * 64, tDO + kk * 8, kmajor_desc(sV, kk, kKB * kBoxBytes), idS,
+                      kk > 0 ? 1u : 0u);
           mma_commit(&s_full[sb]);
           mma_commit(&v_empty[sj & 1]);
           ++sj;
@@ -250,13 +253,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
     const float lse2 = P.lse2[size_t(row) * 64 + m];
     const float dm = P.dvec[size_t(row) * 64 + m];
+    if (nsteps > 0) {
+      // Q and dO are the A operands of every S / dP product: one copy into TMEM
+      mbar_wait_abortable(qd_full, 0, status, abort_flag);
+      tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kDO, tDO + lane_off, m, ch);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qa_full);
+    }
     for (int j = 0; j < nsteps; ++j) {
       const int sb = j % kDqSBufs;
       mbar_wait_abortable(&s_full[sb], (j / kDqSBufs) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t rs[32], rp[32];
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
-      tmem_ld32(tbase + lane_off + 192 + sb * 64 + ch * 32, rp);
+      tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -346,6 +358,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   uint64_t* mma_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
+  uint64_t* ka_full = bars + 14;  // K and V copied into TMEM by the softmax warps
 
   const Geo& g = P.g;
   const int J = blockIdx.x, head = blockIdx.y;
@@ -370,6 +383,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     mbar_init(ps_full, kSoftWarps);
     mbar_init(ps_free, 1);
     mbar_init(mma_done, 1);
+    mbar_init(ka_full, kSoftWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -381,7 +395,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tdV = tbase + 256, tdK = tbase + 384;
+  // TMEM columns: S^T [2 x 64] at 0, dP^T [2 x 64] at 128, dV at 256, dK at 320, K at 384, V at 448
+  const uint32_t tdV = tbase + 256, tdK = tbase + 320, tK = tbase + 384, tV = tbase + 448;
 
   if (warp == 0) {
     if (nsteps > 0) {
@@ -441,9 +456,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idO = idesc_bf16_f32(64, D, false, true);
-      const uint32_t sK = smem_u32(sm + L::kK), sV = smem_u32(sm + L::kV);
       const uint32_t sPT = smem_u32(sm + L::kPT), sDST = smem_u32(sm + L::kDST);
-      bool ok = mbar_wait_abortable(kv_full, 0, status, abort_flag);
+      bool ok = mbar_wait_abortable(ka_full, 0, status, abort_flag);
+      tc_fence_after();
       int sj = 0, kj = 0;
       Watchdog wd;
       wd.reset();
@@ -474,12 +489,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
           const int sb = sj & 1;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws(tbase + sb * 64, kmajor_desc(sK, kk, kBoxBytes), kmajor_desc(sQ, kk, kKB * kBoxBytes), idS,
-                   kk > 0 ? 1u : 0u);
+            mma_ws_ts(tbase + sb * 64, tK + kk * 8, kmajor_desc(sQ, kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws(tbase + 128 + sb * 64, kmajor_desc(sV, kk, kBoxBytes), kmajor_desc(sDO, kk, kKB * kBoxBytes), idS,
-                   kk > 0 ? 1u : 0u);
+            mma_ws_ts(tbase + 128 + sb * 64, tV + kk * 8, kmajor_desc(sDO, kk, kKB * kBoxBytes), idS,
+                      kk > 0 ? 1u : 0u);
           mma_commit(&s_full[sb]);
           ++sj;
           did = true;
@@ -495,6 +509,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     const int Ln = sp * 32 + lane;
     const int m = Ln & 63, kh = Ln >> 6;
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
+    if (nsteps > 0) {
+      // K and V are the A operands of every S^T / dP^T product: one copy into TMEM
+      mbar_wait_abortable(kv_full, 0, status, abort_flag);
+      tile_to_tmem_a<D>(sm + L::kK, tK + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kV, tV + lane_off, m, ch);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ka_full);
+    }
     for (int j = 0; j < nsteps; ++j) {
       const int sb = j & 1;
       mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);

@@ -28,6 +28,48 @@ __device__ __forceinline__ void mma_ws(uint32_t d_tmem, uint64_t adesc, uint64_t
       : "memory");
 }
 
+// Same product with the A operand read from TMEM. For M = 64 the .ws datapath
+// reads row m of A from lane m and from lane m + 64, so A must be stored in
+// both lane halves; packed bf16 pairs, 8 columns per 16-element K step.
+__device__ __forceinline__ void mma_ws_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.ws.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Copies this thread's part of a resident 64-row operand tile ([D/64 boxes]
+// [64 rows][128 B], 128-byte swizzle, as TMA writes it) into TMEM as a .ws A
+// operand: the thread in TMEM lane L writes row L mod 64, column half `ch`
+// (D/4 packed columns) at t_addr = tile column base + lane offset. Tensor-core
+// reads of a resident tile then cost no shared-memory bandwidth.
+template <int D>
+__device__ __forceinline__ void tile_to_tmem_a(const uint8_t* tile, uint32_t t_addr, int m, int ch) {
+  constexpr int NW = D / 4;  // packed words per thread
+  uint32_t v[NW];
+  const int d0 = ch * (D / 2);
+  const uint8_t* box = tile + (d0 / 64) * kBoxBytes;
+  const int c0 = (d0 % 64) / 8;
+#pragma unroll
+  for (int c = 0; c < NW / 4; ++c) {
+    const uint4 u = *reinterpret_cast<const uint4*>(box + sw128_offset(m, c0 + c));
+    v[4 * c] = u.x;
+    v[4 * c + 1] = u.y;
+    v[4 * c + 2] = u.z;
+    v[4 * c + 3] = u.w;
+  }
+  if constexpr (NW == 32) {
+    tmem_st16(t_addr + ch * NW, v);
+    tmem_st16(t_addr + ch * NW + 16, v + 16);
+  } else {
+    tmem_st16(t_addr + ch * NW, v);
+  }
+  tmem_st_wait();
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

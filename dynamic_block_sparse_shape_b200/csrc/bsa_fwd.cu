@@ -73,7 +73,7 @@ struct FwdSmem {
   static constexpr uint32_t kDesc = kRed + kRedBytes;  // block coordinate ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
-  static constexpr uint32_t kTmemCols = 256;  // S: 3 x 64 columns, O: d/2 columns at 192
+  static constexpr uint32_t kTmemCols = 512;  // S: 3 x 64 columns, O at 192, Q (A operand) at 256
 };
 
 template <int D>
@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   uint64_t* mma_done = bars + 21;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 23);
+  uint64_t* qa_full = bars + 24;  // Q copied into TMEM by the softmax warps
   float* red = reinterpret_cast<float*>(sm + L::kRed);
   float* redl = red + 2 * 4 * 64;
 
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       mbar_init(&p_free[i], 1);
     }
     mbar_init(mma_done, 1);
+    mbar_init(qa_full, kSoftWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -141,6 +143,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t tO = tbase + 192;
+  const uint32_t tQ = tbase + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -208,8 +211,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idO = idesc_bf16_f32(64, D, false, true);
-      const uint32_t sQ = smem_u32(sm + L::kQ);
-      bool ok = mbar_wait_abortable(q_full, 0, status, abort_flag);
+      bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
+      tc_fence_after();
       int sj = 0, pj = 0;
       Watchdog wd;
       wd.reset();
@@ -234,8 +237,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
           const uint32_t sK = smem_u32(sm + L::kK0 + (sj % kKSlots) * L::kSlotBytes);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws(tbase + (sj % kSBufs) * 64, kmajor_desc(sQ, kk, kBoxBytes), kmajor_desc(sK, kk, kKB * kBoxBytes),
-                   idS, kk > 0 ? 1u : 0u);
+            mma_ws_ts(tbase + (sj % kSBufs) * 64, tQ + kk * 8, kmajor_desc(sK, kk, kKB * kBoxBytes), idS,
+                      kk > 0 ? 1u : 0u);
           mma_commit(&s_full[sj % kSBufs]);
           mma_commit(&k_empty[sj % kKSlots]);
           ++sj;
@@ -258,6 +261,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     const int q4 = kh * 2 + ch;
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
     float m_run = -INFINITY, l_part = 0.f;
+    if (nsteps > 0) {
+      // Q becomes the A operand of every S product: one copy into TMEM
+      mbar_wait_abortable(q_full, 0, status, abort_flag);
+      tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, ch);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qa_full);
+    }
     for (int j = 0; j < nsteps; ++j) {
       const int sb = j % kSBufs, pb = j & 1, rb = j & 1;
       mbar_wait_abortable(&s_full[sb], (j / kSBufs) & 1, status, abort_flag);

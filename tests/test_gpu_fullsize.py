@@ -1,0 +1,150 @@
+"""Full-size parity on the 720p, 1080p and 2K workloads, in the launch
+configuration bench.py times, on outputs the oracle can compute one by one:
+
+* zone shapes of every zone (bit-exact where the oracle's cost margin > 1e-3);
+* pooled features of sampled blocks of every head;
+* the selection of sampled query blocks of one head (bit-exact where the
+  oracle's margins are safe) and its CSR;
+* O and LSE of sampled query blocks and, on the 2K training step, dQ of those
+  blocks and dK / dV of sampled key blocks.
+
+The GPU stages after the zone shapes take the oracle's zone shapes as input
+(an oracle value may feed the CUDA path, never the reverse), so both sides use
+one block partition. Sampled attention rows are compared only where the GPU's
+selection equals the oracle's for every block they depend on.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dynamic_block_sparse_shape_b200 as P
+from dynamic_block_sparse_shape_b200 import synth
+from oracle import prism_oracle as O
+from tests.gpu_util import (CDF_MARGIN, LOGIT_GAP, assert_close, f64, mask_bits_to_bool, require_gpu)
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def _inputs(wl, dev):
+    x = synth.qkv(wl, device=dev)
+    feats = None
+    if wl.features == "synthetic":
+        feats = synth.video_features(wl, device=dev)
+    elif wl.features == "q":
+        feats = x["q"].view(wl.n_tokens, -1)
+    res = synth.a2v_residual(wl, device=dev)[0] if wl.residual else None
+    return x, feats, res
+
+
+def _oracle_zone_shapes(wl, cand, feats, res):
+    r = None
+    if res is not None:
+        r = np.concatenate([O.token_norms(res[i:i + 32768].to("cpu", torch.float64).numpy())
+                            for i in range(0, res.shape[0], 32768)])
+    Fh = None
+    if feats is not None:
+        Fh = feats.to("cpu")  # bf16 rows, upcast per zone by the oracle
+    nz = int(np.prod(O.zone_counts(wl.grid, wl.zone)))
+    idx = np.zeros(nz, dtype=np.int32)
+    margin = np.zeros(nz)
+
+    class _F:
+        def __getitem__(self, ids):
+            return Fh[torch.as_tensor(np.asarray(ids))].to(torch.float64).numpy()
+    for z0 in range(0, nz, 64):
+        zl = list(range(z0, min(nz, z0 + 64)))
+        st = O.zone_statistics(wl.grid, wl.zone, F=_F() if feats is not None else None, zones=zl, r=r)
+        i, m = O.choose_shapes(st, cand, have_features=feats is not None, have_residual=r is not None)
+        idx[zl] = i
+        margin[zl] = m
+    return idx, margin
+
+
+@pytest.mark.parametrize("name", ["720p", "1080p", "2k"])
+def test_full_size_workload(name):
+    require_gpu()
+    wl = synth.WORKLOADS[name]
+    dev = torch.device("cuda")
+    cand = tuple(synth.candidates_for(wl))
+    geo = P.Geometry(wl.grid, wl.zone, cand)
+    nz, nb = geo.counts()
+    x, feats, res = _inputs(wl, dev)
+    ws = P.Workspace(dev)
+    # ---- a2: every zone
+    zs_gpu, margin_gpu = P.zone_shapes(geo, feat=feats, res=res, ws=ws)
+    idx_r, margin_r = _oracle_zone_shapes(wl, cand, feats, res)
+    qual = margin_r > 1e-3
+    assert qual.mean() > 0.5
+    assert np.array_equal(zs_gpu.cpu().numpy()[qual], idx_r[qual])
+    # downstream stages run on the oracle's partition
+    zs = torch.tensor(idx_r, dtype=torch.int32, device=dev)
+    blocks = O.block_tokens(wl.grid, wl.zone, cand, idx_r)
+    H, d = wl.heads, wl.head_dim
+    sc = 1.0 / math.sqrt(d)
+    # ---- a3: sampled blocks, every head
+    qp, kp = P.block_pool(geo, zs, x["q"], x["k"], ws=ws)
+    rng = np.random.default_rng(0)
+    bs = rng.choice(nb, size=32, replace=False)
+    toks = torch.as_tensor(blocks[bs].reshape(-1), device=dev)
+    for t, pooled in ((x["q"], qp), (x["k"], kp)):
+        rows = t[toks].to("cpu", torch.float64).numpy().reshape(len(bs), 64, H, d)
+        ref = rows.mean(axis=1).transpose(1, 0, 2)
+        assert np.abs(f64(pooled[:, torch.as_tensor(bs, device=dev)]) - ref).max() < 2e-6
+    # ---- a4 + a5: one head, every row (the key-block columns need all of them)
+    h = 1 % H
+    sel = P.block_select(qp, kp, sc, wl.top_k, wl.cdf_threshold, ws=ws)
+    qh = x["q"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
+    kh = x["k"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
+    qpr, kpr = O.block_pool(qh, blocks), O.block_pool(kh, blocks)
+    ref = O.block_select(qpr, kpr, sc, wl.top_k, wl.cdf_threshold)
+    got = mask_bits_to_bool(sel["mask"][h:h + 1], nb)[0]
+    kept = sel["kept"][h].cpu().numpy()
+    sq = (ref["gap"][0] > LOGIT_GAP) & (ref["margin"][0] > CDF_MARGIN)
+    assert sq.sum() >= 0.05 * nb
+    assert np.array_equal(got[sq], ref["mask"][0][sq])
+    assert np.all(kept >= min(wl.top_k, nb)) and np.array_equal(got.sum(axis=1), kept)
+    rp = sel["row_ptr"].cpu().numpy()
+    ci = sel["col_idx"].cpu().numpy()
+    for I in rng.choice(nb, size=16, replace=False):
+        r = h * nb + I
+        assert ci[rp[r]:rp[r + 1]].tolist() == np.nonzero(got[I])[0].tolist()
+    # ---- a6 (+ a7): sampled rows with identical selections
+    o, lse = P.bsa_fwd(geo, zs, x["q"], x["k"], x["v"], sc, sel["row_ptr"], sel["col_idx"], ws=ws)
+    same_row = np.all(got == ref["mask"][0], axis=1)
+    rows = [int(I) for I in rng.permutation(np.nonzero(same_row)[0])[:12]]
+    assert len(rows) >= 6
+    vh = x["v"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
+    doh = x["do"][:, h].to("cpu", torch.float64).numpy()[:, None, :] if wl.backward else None
+    if wl.backward:
+        dq, dk, dv = P.bsa_bwd(geo, zs, x["q"], x["k"], x["v"], o, lse, x["do"], sc, sel["row_ptr"],
+                               sel["col_idx"], sel["total"], ws=ws)
+    torch.cuda.synchronize()
+    P.check_device_status(ws)
+    cache = {}
+    for I in rows:
+        rr = O.attention_block_rows(qh, kh, vh, blocks, np.nonzero(ref["mask"][0][I])[0], 0, I, sc, dO=doh)
+        cache[(0, I)] = rr
+        tk = torch.as_tensor(blocks[I], device=dev)
+        assert_close("O", f64(o[tk, h]), rr["O"])
+        assert_close("LSE", f64(lse[h, tk]), rr["lse"])
+        if wl.backward:
+            assert_close("dQ", f64(dq[tk, h]), rr["dQ"])
+    if wl.backward:
+        # key blocks all of whose users (query blocks that selected them) have
+        # exactly the oracle's selection, so their LSE and D agree too
+        cols = []
+        n_users = ref["mask"][0].sum(axis=0)
+        for J in np.argsort(n_users, kind="stable"):  # the cheapest columns first
+            users = np.nonzero(ref["mask"][0][:, J])[0]
+            if len(users) > 0 and np.array_equal(got[:, J], ref["mask"][0][:, J]) and same_row[users].all():
+                cols.append(int(J))
+            if len(cols) == 2:
+                break
+        assert cols
+        for J in cols:
+            gk, gv = O.attention_kv_block_grads(qh, kh, vh, doh, blocks, ref["mask"][0], 0, J, sc, row_cache=cache)
+            tk = torch.as_tensor(blocks[J], device=dev)
+            assert_close("dK", f64(dk[tk, h]), gk)
+            assert_close("dV", f64(dv[tk, h]), gv)
