@@ -202,7 +202,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
-      const uint32_t sDS = smem_u32(sm + L::kDS);
+      const uint64_t dDS = sdesc_sw128(smem_u32(sm + L::kDS), 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::kK0), 16, 1024);                 // K as B of S
+      const uint64_t dKmn0 = sdesc_sw128(smem_u32(sm + L::kK0), kKB * kBoxBytes, 1024);  // K as B of dQ
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), 16, 1024);
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
       tc_fence_after();
       int sj = 0, qj = 0;
@@ -212,10 +215,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         bool did = false;
         if (qj < sj && mbar_test(ds_full, qj & 1)) {
           tc_fence_after();
-          const uint32_t sK = smem_u32(sm + L::kK0 + (qj % kDqKSlots) * L::kSlotBytes);
+          const uint64_t dK = dKmn0 + uint64_t((qj % kDqKSlots) * (L::kSlotBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tdQ, kmajor_desc(sDS, kk, kBoxBytes), mnmajor_desc(sK, kk, kBoxBytes, kKB * kBoxBytes), idQ,
+            mma_ws(tdQ, dDS + kmajor_step(kk, kBoxBytes), dK + mnmajor_step(kk, kBoxBytes), idQ,
                    (qj > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&k_empty[qj % kDqKSlots]);
           mma_commit(ds_free);
@@ -225,15 +228,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         if (sj < nsteps && mbar_test(&k_full[sj % kDqKSlots], (sj / kDqKSlots) & 1) &&
             mbar_test(&v_full[sj & 1], (sj >> 1) & 1) && mbar_test(&s_free[sj % kDqSBufs], ((sj / kDqSBufs) & 1) ^ 1)) {
           tc_fence_after();
-          const uint32_t sK = smem_u32(sm + L::kK0 + (sj % kDqKSlots) * L::kSlotBytes);
-          const uint32_t sV = smem_u32(sm + L::kV0 + (sj & 1) * L::kSlotBytes);
+          const uint64_t dK = dK0 + uint64_t((sj % kDqKSlots) * (L::kSlotBytes >> 4));
+          const uint64_t dV = dV0 + uint64_t((sj & 1) * (L::kSlotBytes >> 4));
           const int sb = sj % kDqSBufs;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + sb * 64, tQ + kk * 8, kmajor_desc(sK, kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+            mma_ws_ts(tbase + sb * 64, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + 128 + sb * 64, tDO + kk * 8, kmajor_desc(sV, kk, kKB * kBoxBytes), idS,
+            mma_ws_ts(tbase + 128 + sb * 64, tDO + kk * 8, dV + kmajor_step(kk, kKB * kBoxBytes), idS,
                       kk > 0 ? 1u : 0u);
           mma_commit(&s_full[sb]);
           mma_commit(&v_empty[sj & 1]);
@@ -456,7 +459,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idO = idesc_bf16_f32(64, D, false, true);
-      const uint32_t sPT = smem_u32(sm + L::kPT), sDST = smem_u32(sm + L::kDST);
+      const uint64_t dPT = sdesc_sw128(smem_u32(sm + L::kPT), 16, 1024);
+      const uint64_t dDST = sdesc_sw128(smem_u32(sm + L::kDST), 16, 1024);
+      const uint32_t sQ0 = smem_u32(sm + L::kStage0);
+      const uint64_t dQ0 = sdesc_sw128(sQ0, 16, 1024);                                   // Q as B of S^T
+      const uint64_t dDO0 = sdesc_sw128(sQ0 + L::kHalf, 16, 1024);                       // dO as B of dP^T
+      const uint64_t dQmn0 = sdesc_sw128(sQ0, kKB * kBoxBytes, 1024);                    // Q as B of dK
+      const uint64_t dDOmn0 = sdesc_sw128(sQ0 + L::kHalf, kKB * kBoxBytes, 1024);        // dO as B of dV
+      constexpr uint64_t kStageStep = L::kStageBytes >> 4;
       bool ok = mbar_wait_abortable(ka_full, 0, status, abort_flag);
       tc_fence_after();
       int sj = 0, kj = 0;
@@ -466,15 +476,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
         bool did = false;
         if (kj < sj && mbar_test(ps_full, kj & 1)) {
           tc_fence_after();
-          const uint32_t sQ = smem_u32(sm + L::kStage0 + (kj & 1) * L::kStageBytes);
-          const uint32_t sDO = sQ + L::kHalf;
+          const uint64_t st = uint64_t(kj & 1) * kStageStep;
 #pragma unroll
           for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tdV, kmajor_desc(sPT, kk, kBoxBytes), mnmajor_desc(sDO, kk, kBoxBytes, kKB * kBoxBytes), idO,
+            mma_ws(tdV, dPT + kmajor_step(kk, kBoxBytes), dDOmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
                    (kj > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tdK, kmajor_desc(sDST, kk, kBoxBytes), mnmajor_desc(sQ, kk, kBoxBytes, kKB * kBoxBytes), idO,
+            mma_ws(tdK, dDST + kmajor_step(kk, kBoxBytes), dQmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
                    (kj > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&st_empty[kj & 1]);
           mma_commit(ps_free);
@@ -484,15 +493,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
         if (sj < nsteps && mbar_test(&st_full[sj & 1], (sj >> 1) & 1) &&
             mbar_test(&s_free[sj & 1], ((sj >> 1) & 1) ^ 1)) {
           tc_fence_after();
-          const uint32_t sQ = smem_u32(sm + L::kStage0 + (sj & 1) * L::kStageBytes);
-          const uint32_t sDO = sQ + L::kHalf;
+          const uint64_t st = uint64_t(sj & 1) * kStageStep;
           const int sb = sj & 1;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + sb * 64, tK + kk * 8, kmajor_desc(sQ, kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+            mma_ws_ts(tbase + sb * 64, tK + kk * 8, dQ0 + st + kmajor_step(kk, kKB * kBoxBytes), idS,
+                      kk > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + 128 + sb * 64, tV + kk * 8, kmajor_desc(sDO, kk, kKB * kBoxBytes), idS,
+            mma_ws_ts(tbase + 128 + sb * 64, tV + kk * 8, dDO0 + st + kmajor_step(kk, kKB * kBoxBytes), idS,
                       kk > 0 ? 1u : 0u);
           mma_commit(&s_full[sb]);
           ++sj;

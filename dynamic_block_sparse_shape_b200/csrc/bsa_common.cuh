@@ -90,6 +90,17 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kstep, uint3
   return sdesc_sw128(base + uint32_t(kstep >> 2) * slot_stride + uint32_t(kstep & 3) * 2048u, n_stride, 1024);
 }
 
+// The same K-step addressing as offsets (16-byte units) added to a base
+// descriptor's start-address field (bits 0..13; every address here is below
+// 256 KB, so the add never carries out of the field). Issuing threads build
+// one base descriptor per buffer and add a compile-time constant per step.
+__host__ __device__ constexpr uint64_t kmajor_step(int kstep, uint32_t box_stride) {
+  return uint64_t((uint32_t(kstep >> 2) * box_stride + uint32_t(kstep & 3) * 32u) >> 4);
+}
+__host__ __device__ constexpr uint64_t mnmajor_step(int kstep, uint32_t slot_stride) {
+  return uint64_t((uint32_t(kstep >> 2) * slot_stride + uint32_t(kstep & 3) * 2048u) >> 4);
+}
+
 __device__ __forceinline__ int safe_shape(const Geo& g, const int32_t* zone_shape, int b, int* status) {
   int s = zone_shape[b / g.bpz];
   if (s < 0 || s >= g.n_cand) {
