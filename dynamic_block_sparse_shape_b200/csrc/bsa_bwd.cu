@@ -65,6 +65,7 @@ struct BwdParams {
 constexpr int kDqKSlots = 3;
 constexpr int kDqVSlots = 2;
 constexpr int kDqSBufs = 2;
+static_assert(kDqVSlots == kDqSBufs, "V slot j is released by the score barrier of step j");
 
 template <int D>
 struct DqSmem {
@@ -89,8 +90,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   uint64_t* qd_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [3]
   uint64_t* k_empty = bars + 4;  // [3]
-  uint64_t* v_full = bars + 7;   // [2]
-  uint64_t* v_empty = bars + 9;  // [2]
+  uint64_t* v_full = bars + 7;   // [2] (a V slot is free once the dP product that read it completed: s_full)
   uint64_t* s_full = bars + 11;  // [3]
   uint64_t* s_free = bars + 14;  // [3]
   uint64_t* ds_full = bars + 17;
@@ -118,10 +118,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
     }
-    for (int i = 0; i < kDqVSlots; ++i) {
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
-    }
+    for (int i = 0; i < kDqVSlots; ++i) mbar_init(&v_full[i], 1);
     for (int i = 0; i < kDqSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kSoftWarps);
@@ -178,7 +175,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
             ++nk;
             did = true;
           }
-          if (nv < nk && mbar_test(&v_empty[nv & 1], ((nv >> 1) & 1) ^ 1)) {
+          if (nv < nk && mbar_test(&s_full[nv % kDqSBufs], ((nv / kDqSBufs) & 1) ^ 1)) {
             load_step(P.mv, sm + L::kV0 + (nv & 1) * L::kSlotBytes, &v_full[nv & 1], nv);
             ++nv;
             did = true;
@@ -239,7 +236,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
             mma_ws_ts(tbase + 128 + sb * 64, tDO + kk * 8, dV + kmajor_step(kk, kKB * kBoxBytes), idS,
                       kk > 0 ? 1u : 0u);
           mma_commit(&s_full[sb]);
-          mma_commit(&v_empty[sj & 1]);
           ++sj;
           did = true;
         }
@@ -276,18 +272,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
-      const bool valid = (j * kKB + kh) < cnt && lse2 > -INFINITY;
+      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
       uint32_t pk[16];
+      if (valid) {
+        const float c = P.scale_log2, nl = -lse2;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float d0 = 0.f, d1 = 0.f;
-        if (valid) {
-          const float p0 = fast_exp2(__uint_as_float(rs[2 * i]) * P.scale_log2 - lse2);
-          const float p1 = fast_exp2(__uint_as_float(rs[2 * i + 1]) * P.scale_log2 - lse2);
-          d0 = p0 * (__uint_as_float(rp[2 * i]) - dm);
-          d1 = p1 * (__uint_as_float(rp[2 * i + 1]) - dm);
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(rs[2 * i]), c, nl));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(rs[2 * i + 1]), c, nl));
+          pk[i] = pack_bf16x2(p0 * (__uint_as_float(rp[2 * i]) - dm), p1 * (__uint_as_float(rp[2 * i + 1]) - dm));
         }
-        pk[i] = pack_bf16x2(d0, d1);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = 0u;
       }
       if (j >= 1) mbar_wait_abortable(ds_free, (j - 1) & 1, status, abort_flag);
       uint8_t* pt = sm + L::kDS + kh * kBoxBytes;
@@ -542,21 +539,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       // the per-query LSE / D rows arrived by bulk copy on st_full: observe it
       mbar_wait_abortable(&st_full[sb], (j >> 1) & 1, status, abort_flag);
       const float* ld = reinterpret_cast<const float*>(sm + L::kStage0 + (j & 1) * L::kStageBytes + L::kLD);
-      const float* l2 = ld + kh * 64 + ch * 32;
-      const float* dd = ld + 128 + kh * 64 + ch * 32;
+      // the 32 queries of this thread's columns: LSE * log2(e) and D, same for the whole warp
+      const float4* l2 = reinterpret_cast<const float4*>(ld + kh * 64 + ch * 32);
+      const float4* dd = reinterpret_cast<const float4*>(ld + 128 + kh * 64 + ch * 32);
       uint32_t pp[16], pd[16];
+      if (valid) {
+        const float c = P.scale_log2;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-        if (valid) {
-          const float a0 = l2[2 * i], a1 = l2[2 * i + 1];
-          p0 = a0 > -INFINITY ? fast_exp2(__uint_as_float(rs[2 * i]) * P.scale_log2 - a0) : 0.f;
-          p1 = a1 > -INFINITY ? fast_exp2(__uint_as_float(rs[2 * i + 1]) * P.scale_log2 - a1) : 0.f;
-          d0 = p0 * (__uint_as_float(rp[2 * i]) - dd[2 * i]);
-          d1 = p1 * (__uint_as_float(rp[2 * i + 1]) - dd[2 * i + 1]);
+        for (int i = 0; i < 8; ++i) {
+          const float4 a = l2[i], e = dd[i];
+          const float p0 = fast_exp2(fmaf(__uint_as_float(rs[4 * i]), c, -a.x));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 1]), c, -a.y));
+          const float p2 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 2]), c, -a.z));
+          const float p3 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 3]), c, -a.w));
+          pp[2 * i] = pack_bf16x2(p0, p1);
+          pp[2 * i + 1] = pack_bf16x2(p2, p3);
+          pd[2 * i] = pack_bf16x2(p0 * (__uint_as_float(rp[4 * i]) - e.x), p1 * (__uint_as_float(rp[4 * i + 1]) - e.y));
+          pd[2 * i + 1] =
+              pack_bf16x2(p2 * (__uint_as_float(rp[4 * i + 2]) - e.z), p3 * (__uint_as_float(rp[4 * i + 3]) - e.w));
         }
-        pp[i] = pack_bf16x2(p0, p1);
-        pd[i] = pack_bf16x2(d0, d1);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pp[i] = pd[i] = 0u;
       }
       if (j >= 1) mbar_wait_abortable(ps_free, (j - 1) & 1, status, abort_flag);
       uint8_t* pt = sm + L::kPT + kh * kBoxBytes;
@@ -651,7 +655,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const Geo g, const int32_
     const size_t at = (size_t(head) * g.n_blocks + b) * 64 + r;
     d_blk[at] = acc;
     const int N = g.T * g.H * g.W;
-    lse2_blk[at] = lse[int64_t(head) * N + tok] * 1.4426950408889634f;
+    // A query with no keys has LSE = -inf and, by definition, P = 0 and no
+    // gradient. Storing +inf there makes exp2(s * c - lse2) = exp2(-inf) = 0 in
+    // both passes without a per-score test.
+    const float l = lse[int64_t(head) * N + tok];
+    lse2_blk[at] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
   }
 }
 

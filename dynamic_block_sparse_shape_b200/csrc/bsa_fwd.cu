@@ -39,6 +39,7 @@ constexpr int kKB = 2;  // key blocks per step
 constexpr int kKSlots = 3;
 constexpr int kVSlots = 2;
 constexpr int kSBufs = 3;
+constexpr int kPBufs = 3;
 constexpr int kSoftWarps = 8;
 constexpr int kFwdThreads = 64 + 32 * kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
@@ -68,7 +69,11 @@ struct FwdSmem {
   static constexpr uint32_t kV0 = kK0 + kKSlots * kSlotBytes;
   static constexpr uint32_t kPBytes = kKB * kBoxBytes;
   static constexpr uint32_t kP0 = kV0 + kVSlots * kSlotBytes;
-  static constexpr uint32_t kRed = kP0 + 2 * kPBytes;
+  // P buffers 0 and 1 follow the V ring; buffer 2 reuses the Q tile once Q
+  // has been copied into TMEM (d = 128: 16 KB), else its own region.
+  static constexpr bool kPInQ = kQBytes >= kPBytes;
+  static constexpr uint32_t kP2 = kPInQ ? kQ : kP0 + 2 * kPBytes;
+  static constexpr uint32_t kRed = kP0 + (kPInQ ? 2 : 3) * kPBytes;
   static constexpr uint32_t kRedBytes = (2 * 4 * 64 + 4 * 64) * 4;
   static constexpr uint32_t kDesc = kRed + kRedBytes;  // block coordinate ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 16;
@@ -83,18 +88,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* q_full = bars + 0;
+  // K and V slots have no "empty" barriers of their own: a K slot is free once
+  // the S product that read it has completed (s_full), a V slot once its PV
+  // product has (p_free).
   uint64_t* k_full = bars + 1;    // [3]
-  uint64_t* k_empty = bars + 4;   // [3]
   uint64_t* v_full = bars + 7;    // [2]
-  uint64_t* v_empty = bars + 9;   // [2]
   uint64_t* s_full = bars + 11;   // [3]
   uint64_t* s_free = bars + 14;   // [3]
-  uint64_t* p_full = bars + 17;   // [2]
-  uint64_t* p_free = bars + 19;   // [2]
-  uint64_t* mma_done = bars + 21;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 23);
-  uint64_t* qa_full = bars + 24;  // Q copied into TMEM by the softmax warps
+  uint64_t* p_full = bars + 17;   // [3]
+  uint64_t* p_free = bars + 20;   // [3]
+  uint64_t* mma_done = bars + 23;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 25);
+  uint64_t* qa_full = bars + 26;  // Q copied into TMEM by the softmax warps
   float* red = reinterpret_cast<float*>(sm + L::kRed);
   float* redl = red + 2 * 4 * 64;
 
@@ -115,17 +121,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     mbar_init(q_full, 1);
     for (int i = 0; i < kKSlots; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
     }
     for (int i = 0; i < kVSlots; ++i) {
       mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kSoftWarps);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPBufs; ++i) {
       mbar_init(&p_full[i], kSoftWarps);
       mbar_init(&p_free[i], 1);
     }
@@ -164,7 +168,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         int nk = kj, nv = vj, stop = 0;
         if (lane == 0) {
           bool did = false;
-          if (nk < nsteps && mbar_test(&k_empty[nk % kKSlots], ((nk / kKSlots) & 1) ^ 1)) {
+          // a K slot is free once the S product of three steps back is done (its s_full phase)
+          if (nk < nsteps && mbar_test(&s_full[nk % kKSlots], ((nk / kKSlots) & 1) ^ 1)) {
             const int ks = nk % kKSlots;
             uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
             mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
@@ -177,7 +182,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
             ++nk;
             did = true;
           }
-          if (nv < nk && mbar_test(&v_empty[nv & 1], ((nv >> 1) & 1) ^ 1)) {
+          // a V slot is free once the PV product of two steps back is done (its p_free phase)
+          if (nv < nk && (nv < kVSlots || mbar_test(&p_free[(nv - kVSlots) % kPBufs], ((nv - kVSlots) / kPBufs) & 1))) {
             const int vs = nv & 1;
             uint8_t* dst = sm + L::kV0 + vs * L::kSlotBytes;
             mbar_arrive_expect_tx(&v_full[vs], L::kSlotBytes);
@@ -211,6 +217,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idO = idesc_bf16_f32(64, D, false, true);
+      // base descriptors of slot 0 of each ring; slot i adds i * slot bytes / 16
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::kK0), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), kBoxBytes, 1024);
+      const uint64_t dP0 = sdesc_sw128(smem_u32(sm + L::kP0), 16, 1024);
+      const uint64_t dP2 = sdesc_sw128(smem_u32(sm + L::kP2), 16, 1024);
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
       tc_fence_after();
       int sj = 0, pj = 0;
@@ -218,29 +229,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       wd.reset();
       while (ok && pj < nsteps) {
         bool did = false;
-        if (pj < sj && mbar_test(&p_full[pj & 1], (pj >> 1) & 1) && mbar_test(&v_full[pj & 1], (pj >> 1) & 1)) {
+        if (pj < sj && mbar_test(&p_full[pj % kPBufs], (pj / kPBufs) & 1) &&
+            mbar_test(&v_full[pj & 1], (pj >> 1) & 1)) {
           tc_fence_after();
-          const uint32_t sP = smem_u32(sm + L::kP0 + (pj & 1) * L::kPBytes);
-          const uint32_t sV = smem_u32(sm + L::kV0 + (pj & 1) * L::kSlotBytes);
+          const int pb = pj % kPBufs;
+          const uint64_t dP = pb < 2 ? dP0 + uint64_t(pb * (L::kPBytes >> 4)) : dP2;
+          const uint64_t dV = dV0 + uint64_t((pj & 1) * (L::kSlotBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tO, kmajor_desc(sP, kk, kBoxBytes), mnmajor_desc(sV, kk, D * 128, kBoxBytes), idO,
+            mma_ws(tO, dP + kmajor_step(kk, kBoxBytes), dV + mnmajor_step(kk, D * 128), idO,
                    (pj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&v_empty[pj & 1]);
-          mma_commit(&p_free[pj & 1]);
+          mma_commit(&p_free[pb]);
           ++pj;
           did = true;
         }
         if (sj < nsteps && mbar_test(&k_full[sj % kKSlots], (sj / kKSlots) & 1) &&
             mbar_test(&s_free[sj % kSBufs], ((sj / kSBufs) & 1) ^ 1)) {
           tc_fence_after();
-          const uint32_t sK = smem_u32(sm + L::kK0 + (sj % kKSlots) * L::kSlotBytes);
+          const uint64_t dK = dK0 + uint64_t((sj % kKSlots) * (L::kSlotBytes >> 4));
+          const uint32_t tS = tbase + (sj % kSBufs) * 64;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + (sj % kSBufs) * 64, tQ + kk * 8, kmajor_desc(sK, kk, kKB * kBoxBytes), idS,
-                      kk > 0 ? 1u : 0u);
+            mma_ws_ts(tS, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
           mma_commit(&s_full[sj % kSBufs]);
-          mma_commit(&k_empty[sj % kKSlots]);
           ++sj;
           did = true;
         }
@@ -270,7 +281,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       if (lane == 0) mbar_arrive(qa_full);
     }
     for (int j = 0; j < nsteps; ++j) {
-      const int sb = j % kSBufs, pb = j & 1, rb = j & 1;
+      const int sb = j % kSBufs, pb = j % kPBufs, rb = j & 1;
       mbar_wait_abortable(&s_full[sb], (j / kSBufs) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t r[32];
@@ -279,13 +290,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
-      const bool valid = (j * kKB + kh) < cnt;
-      float x[32];
+      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform: kh is fixed per warp
       float mx = -INFINITY;
+      if (valid) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        x[i] = valid ? __uint_as_float(r[i]) * P.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[i]);
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
+        mx *= P.scale_log2;  // the scale is positive, so it commutes with the max
       }
       red[(rb * 4 + q4) * 64 + m] = mx;
       named_bar_sync(1, 32 * kSoftWarps);
@@ -301,7 +311,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         }
         if (j > 0) {
           // O holds PV_0 .. PV_{j-1}: wait for the last of them, then rescale
-          mbar_wait_abortable(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, status, abort_flag);
+          mbar_wait_abortable(&p_free[(j - 1) % kPBufs], ((j - 1) / kPBufs) & 1, status, abort_flag);
           tc_fence_after();
           uint32_t o[32];
           const uint32_t ta = tO + lane_off + ch * (D / 4);
@@ -324,17 +334,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         }
       }
       uint32_t pk[16];
-      float lsum = 0.f;
+      if (valid) {  // m_run is finite here: it includes this thread's finite maximum
+        const float c = P.scale_log2, nm = -m_run;
+        float lsum = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float p0 = x[2 * i] == -INFINITY ? 0.f : fast_exp2(x[2 * i] - m_run);
-        const float p1 = x[2 * i + 1] == -INFINITY ? 0.f : fast_exp2(x[2 * i + 1] - m_run);
-        lsum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(r[2 * i]), c, nm));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(r[2 * i + 1]), c, nm));
+          lsum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        l_part += lsum;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = 0u;
       }
-      l_part += lsum;
-      if (j >= 2) mbar_wait_abortable(&p_free[pb], ((j >> 1) & 1) ^ 1, status, abort_flag);
-      uint8_t* pt = sm + L::kP0 + pb * L::kPBytes + kh * kBoxBytes;
+      if (j >= kPBufs) mbar_wait_abortable(&p_free[pb], ((j / kPBufs) & 1) ^ 1, status, abort_flag);
+      uint8_t* pt = sm + (pb < 2 ? L::kP0 + pb * L::kPBytes : L::kP2) + kh * kBoxBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
@@ -344,7 +360,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       if (lane == 0) mbar_arrive(&p_full[pb]);
     }
     // ---------------------------------------------------------- epilogue
-    if (nsteps > 0) mbar_wait_abortable(&p_free[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, status, abort_flag);
+    if (nsteps > 0)
+      mbar_wait_abortable(&p_free[(nsteps - 1) % kPBufs], ((nsteps - 1) / kPBufs) & 1, status, abort_flag);
     tc_fence_after();
     redl[q4 * 64 + m] = l_part;
     named_bar_sync(1, 32 * kSoftWarps);
