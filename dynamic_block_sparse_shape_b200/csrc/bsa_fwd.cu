@@ -6,21 +6,34 @@
 // exact: an online softmax over the kept 64-token key blocks (FlashAttention
 // style), fp32 statistics and accumulators, bf16 operands.
 //
-// One CTA per (query block I, head). Warp roles:
-//   warp 0      TMA producer: Q once; per step the K boxes (3-slot ring) and V
-//               boxes (2-slot ring) of two selected key blocks, through 5-D
+// One CTA per (query block I, head); a step covers two selected key blocks.
+// Warp roles:
+//   warp 0      TMA producer: Q once; per step the K boxes and the V boxes of
+//               the step's two key blocks (3-slot rings each), through 5-D
 //               tensor maps (one per block shape);
 //   warp 1      TMEM owner and single-thread tcgen05 issuer:
-//               S_j = Q K_j^T   (.ws M=64, N=128, K=d)   -> TMEM, 3 buffers
-//               O  += P_j V_j   (.ws M=64, N=d,   K=128) -> TMEM
-//   warps 2..9  softmax: 256 threads, four per query row (two TMEM lane halves
-//               x two column halves, 32 keys each); row maxima are exchanged
-//               through shared memory; P_j goes to shared memory as the bf16
-//               K-major A operand of the PV product (double-buffered).
+//               S_j = Q [K_j0 K_j1]^T  (.ws M=64, N=128, K=d, Q from TMEM)
+//               O_h += P_jh V_jh       (.ws M=64, N=128, K=64, P from TMEM)
+//   warps 2..9  softmax: 256 threads, four per query row (two TMEM lane
+//               halves x two column halves, 32 keys each); row maxima are
+//               exchanged through shared memory.
+// TMEM holds every tensor-core A operand: Q, and P (3 buffers of its own, so
+// S_{j+3} may be issued while PV_j still reads P_j). The .ws datapath computes the accumulator
+// columns n < N/2 in lanes 0..63 from A rows in lanes 0..63 and the columns
+// n >= N/2 in lanes 64..127 from A rows in lanes 64..127. S_j of key block 0
+// lands in the low lanes and of key block 1 in the high lanes, so the P rows
+// each lane half holds belong to one key block. The PV product is therefore
+// issued with its B operand's two 64-column halves taken from V of key block
+// 0 (low half) and key block 1 (high half): lane m accumulates the block-0
+// part of O row m, lane m + 64 the block-1 part, each over all d channels
+// (d/64 products per K step). The two parts are added once, in the epilogue.
+// P never touches shared memory, so per step shared memory carries only the
+// K and V tiles (TMA writes, tensor-core reads).
 // The producer and the issuer never block on one barrier: each polls the
 // barriers of every operation it could start next (mbarrier.test_wait) and
-// starts whichever is ready, so a late K load does not hold back a ready PV
-// product and a K slot is refilled as soon as its S product completes.
+// starts whichever is ready. K slot j%3 is refilled once S_j has completed,
+// V slot j%3 and P buffer j%3 once PV_j has; S buffer j%3 once the softmax
+// warps have read S_j.
 // The running max is only moved when it grows by more than 8 (log2 units);
 // the final division uses the same stale max, so the result is exact while
 // the rare O rescale (TMEM load/scale/store) stays off the common path.
@@ -36,10 +49,7 @@ namespace prism {
 namespace {
 
 constexpr int kKB = 2;  // key blocks per step
-constexpr int kKSlots = 3;
-constexpr int kVSlots = 2;
-constexpr int kSBufs = 3;
-constexpr int kPBufs = 3;
+constexpr int kRing = 3;  // K slots = V slots = S buffers = P buffers
 constexpr int kSoftWarps = 8;
 constexpr int kFwdThreads = 64 + 32 * kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
@@ -65,20 +75,23 @@ struct FwdSmem {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kQBytes = D * 128;
   static constexpr uint32_t kSlotBytes = kKB * D * 128;  // K (or V) of one step
-  static constexpr uint32_t kK0 = kQBytes;
-  static constexpr uint32_t kV0 = kK0 + kKSlots * kSlotBytes;
-  static constexpr uint32_t kPBytes = kKB * kBoxBytes;
-  static constexpr uint32_t kP0 = kV0 + kVSlots * kSlotBytes;
-  // P buffers 0 and 1 follow the V ring; buffer 2 reuses the Q tile once Q
-  // has been copied into TMEM (d = 128: 16 KB), else its own region.
-  static constexpr bool kPInQ = kQBytes >= kPBytes;
-  static constexpr uint32_t kP2 = kPInQ ? kQ : kP0 + 2 * kPBytes;
-  static constexpr uint32_t kRed = kP0 + (kPInQ ? 2 : 3) * kPBytes;
+  static constexpr uint32_t kK0 = kQBytes;                // [slot][dh][block][64][128 B]
+  static constexpr uint32_t kV0 = kK0 + kRing * kSlotBytes;  // [slot][block][dh][64][128 B]
+  static constexpr uint32_t kRed = kV0 + kRing * kSlotBytes;
   static constexpr uint32_t kRedBytes = (2 * 4 * 64 + 4 * 64) * 4;
   static constexpr uint32_t kDesc = kRed + kRedBytes;  // block coordinate ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
-  static constexpr uint32_t kTmemCols = 512;  // S: 3 x 64 columns, O at 192, Q (A operand) at 256
+  // epilogue exchange of O parts: [kh][ch][64 rows][D/4 + 4 floats], in the K ring
+  static constexpr uint32_t kXPitch = D / 4 + 4;
+  static_assert(4 * 64 * kXPitch * 4 <= kRing * kSlotBytes, "exchange buffer fits the K ring");
+  // TMEM: S buffers at 0, 64, 128; O parts (D columns) at 192; Q (A operand,
+  // D/2 columns) after O; P buffers (32 columns each) after Q
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTO = 192;
+  static constexpr uint32_t kTQ = 192 + D;
+  static constexpr uint32_t kTP = kTQ + D / 2;
+  static_assert(kTP + kRing * 32 <= kTmemCols, "TMEM budget");
 };
 
 template <int D>
@@ -88,19 +101,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* q_full = bars + 0;
-  // K and V slots have no "empty" barriers of their own: a K slot is free once
-  // the S product that read it has completed (s_full), a V slot once its PV
-  // product has (p_free).
-  uint64_t* k_full = bars + 1;    // [3]
-  uint64_t* v_full = bars + 7;    // [2]
-  uint64_t* s_full = bars + 11;   // [3]
-  uint64_t* s_free = bars + 14;   // [3]
-  uint64_t* p_full = bars + 17;   // [3]
-  uint64_t* p_free = bars + 20;   // [3]
-  uint64_t* mma_done = bars + 23;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 25);
-  uint64_t* qa_full = bars + 26;  // Q copied into TMEM by the softmax warps
+  uint64_t* k_full = bars + 1;   // [3]
+  uint64_t* v_full = bars + 4;   // [3]
+  uint64_t* s_full = bars + 7;   // [3] S_j complete (also: K slot j%3 free)
+  uint64_t* s_free = bars + 10;  // [3] S_j read by the 8 softmax warps
+  uint64_t* p_full = bars + 13;  // [3] P_j written to TMEM by the 8 softmax warps
+  uint64_t* p_free = bars + 16;  // [3] PV_j complete (V slot and P buffer j%3 free)
+  uint64_t* mma_done = bars + 19;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
+  uint64_t* qa_full = bars + 22;  // Q copied into TMEM by the softmax warps
   float* red = reinterpret_cast<float*>(sm + L::kRed);
   float* redl = red + 2 * 4 * 64;
 
@@ -119,17 +129,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < kKSlots; ++i) {
+    for (int i = 0; i < kRing; ++i) {
       mbar_init(&k_full[i], 1);
-    }
-    for (int i = 0; i < kVSlots; ++i) {
       mbar_init(&v_full[i], 1);
-    }
-    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kSoftWarps);
-    }
-    for (int i = 0; i < kPBufs; ++i) {
       mbar_init(&p_full[i], kSoftWarps);
       mbar_init(&p_free[i], 1);
     }
@@ -146,8 +150,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tO = tbase + 192;
-  const uint32_t tQ = tbase + 256;
+  const uint32_t tO = tbase + L::kTO;
+  const uint32_t tQ = tbase + L::kTQ;
+  const uint32_t tP = tbase + L::kTP;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -168,9 +173,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         int nk = kj, nv = vj, stop = 0;
         if (lane == 0) {
           bool did = false;
-          // a K slot is free once the S product of three steps back is done (its s_full phase)
-          if (nk < nsteps && mbar_test(&s_full[nk % kKSlots], ((nk / kKSlots) & 1) ^ 1)) {
-            const int ks = nk % kKSlots;
+          // K slot nk%3 last held the K of step nk-3: free once S_{nk-3} completed
+          if (nk < nsteps && mbar_test(&s_full[nk % kRing], ((nk / kRing) & 1) ^ 1)) {
+            const int ks = nk % kRing;
             uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
             mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
             for (int slot = 0; slot < kKB; ++slot) {
@@ -182,9 +187,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
             ++nk;
             did = true;
           }
-          // a V slot is free once the PV product of two steps back is done (its p_free phase)
-          if (nv < nk && (nv < kVSlots || mbar_test(&p_free[(nv - kVSlots) % kPBufs], ((nv - kVSlots) / kPBufs) & 1))) {
-            const int vs = nv & 1;
+          // V slot nv%3 last held the V of step nv-3: free once PV_{nv-3} completed
+          if (nv < nk && mbar_test(&p_free[nv % kRing], ((nv / kRing) & 1) ^ 1)) {
+            const int vs = nv % kRing;
             uint8_t* dst = sm + L::kV0 + vs * L::kSlotBytes;
             mbar_arrive_expect_tx(&v_full[vs], L::kSlotBytes);
             for (int slot = 0; slot < kKB; ++slot) {
@@ -206,22 +211,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       if (lane == 0) {
         // drain: every issued copy has landed before the CTA may exit
         mbar_wait(q_full, 0, status);
-        for (int i = kj - kKSlots > 0 ? kj - kKSlots : 0; i < kj; ++i)
-          mbar_wait(&k_full[i % kKSlots], (i / kKSlots) & 1, status);
-        for (int i = vj - kVSlots > 0 ? vj - kVSlots : 0; i < vj; ++i)
-          mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
+        for (int i = kj - kRing > 0 ? kj - kRing : 0; i < kj; ++i)
+          mbar_wait(&k_full[i % kRing], (i / kRing) & 1, status);
+        for (int i = vj - kRing > 0 ? vj - kRing : 0; i < vj; ++i)
+          mbar_wait(&v_full[i % kRing], (i / kRing) & 1, status);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
-      const uint32_t idO = idesc_bf16_f32(64, D, false, true);
-      // base descriptors of slot 0 of each ring; slot i adds i * slot bytes / 16
+      const uint32_t idO = idesc_bf16_f32(64, 128, false, true);
+      // K: K-major B of S. V: MN-major B of PV whose two 64-column halves are
+      // the same 64 channels of V of key block 0 and of key block 1 (LBO = the
+      // block stride), so N = 128 covers one channel group for both blocks.
       const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::kK0), 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), kBoxBytes, 1024);
-      const uint64_t dP0 = sdesc_sw128(smem_u32(sm + L::kP0), 16, 1024);
-      const uint64_t dP2 = sdesc_sw128(smem_u32(sm + L::kP2), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), D * 128, 1024);
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
       tc_fence_after();
       int sj = 0, pj = 0;
@@ -229,29 +234,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       wd.reset();
       while (ok && pj < nsteps) {
         bool did = false;
-        if (pj < sj && mbar_test(&p_full[pj % kPBufs], (pj / kPBufs) & 1) &&
-            mbar_test(&v_full[pj & 1], (pj >> 1) & 1)) {
+        if (pj < sj && mbar_test(&p_full[pj % kRing], (pj / kRing) & 1) &&
+            mbar_test(&v_full[pj % kRing], (pj / kRing) & 1)) {
           tc_fence_after();
-          const int pb = pj % kPBufs;
-          const uint64_t dP = pb < 2 ? dP0 + uint64_t(pb * (L::kPBytes >> 4)) : dP2;
-          const uint64_t dV = dV0 + uint64_t((pj & 1) * (L::kSlotBytes >> 4));
+          const int b = pj % kRing;
+          const uint64_t dV = dV0 + uint64_t(b * (L::kSlotBytes >> 4));
 #pragma unroll
-          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tO, dP + kmajor_step(kk, kBoxBytes), dV + mnmajor_step(kk, D * 128), idO,
-                   (pj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&p_free[pb]);
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              mma_ws_ts(tO + c * 64, tP + b * 32 + kk * 8, dV + uint64_t((c * kBoxBytes + kk * 2048) >> 4), idO,
+                        (pj > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&p_free[b]);
           ++pj;
           did = true;
         }
-        if (sj < nsteps && mbar_test(&k_full[sj % kKSlots], (sj / kKSlots) & 1) &&
-            mbar_test(&s_free[sj % kSBufs], ((sj / kSBufs) & 1) ^ 1)) {
+        // S_sj overwrites buffer sj%3, which the softmax warps read S_{sj-3} from
+        if (sj < nsteps && mbar_test(&k_full[sj % kRing], (sj / kRing) & 1) &&
+            mbar_test(&s_free[sj % kRing], ((sj / kRing) & 1) ^ 1)) {
           tc_fence_after();
-          const uint64_t dK = dK0 + uint64_t((sj % kKSlots) * (L::kSlotBytes >> 4));
-          const uint32_t tS = tbase + (sj % kSBufs) * 64;
+          const int b = sj % kRing;
+          const uint64_t dK = dK0 + uint64_t(b * (L::kSlotBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tS, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
-          mma_commit(&s_full[sj % kSBufs]);
+            mma_ws_ts(tbase + b * 64, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+          mma_commit(&s_full[b]);
           ++sj;
           did = true;
         }
@@ -281,20 +288,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       if (lane == 0) mbar_arrive(qa_full);
     }
     for (int j = 0; j < nsteps; ++j) {
-      const int sb = j % kSBufs, pb = j % kPBufs, rb = j & 1;
-      mbar_wait_abortable(&s_full[sb], (j / kSBufs) & 1, status, abort_flag);
+      const int b = j % kRing, rb = j & 1;
+      mbar_wait_abortable(&s_full[b], (j / kRing) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t r[32];
-      tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, r);
+      tmem_ld32(tbase + lane_off + b * 64 + ch * 32, r);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
+      if (lane == 0) mbar_arrive(&s_free[b]);
       const bool valid = (j * kKB + kh) < cnt;  // warp-uniform: kh is fixed per warp
       float mx = -INFINITY;
       if (valid) {
+        // two chains of three-input maxima over r[0..29], then r[30], r[31]
+        float ca = fmax3(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+        float cb = fmax3(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
+        for (int i = 6; i < 30; i += 4) {
+          ca = fmax3(ca, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+          cb = fmax3(cb, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+        }
+        mx = fmaxf(fmax3(ca, cb, __uint_as_float(r[30])), __uint_as_float(r[31]));
         mx *= P.scale_log2;  // the scale is positive, so it commutes with the max
       }
       red[(rb * 4 + q4) * 64 + m] = mx;
@@ -310,27 +324,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
           m_run = m_new;
         }
         if (j > 0) {
-          // O holds PV_0 .. PV_{j-1}: wait for the last of them, then rescale
-          mbar_wait_abortable(&p_free[(j - 1) % kPBufs], ((j - 1) / kPBufs) & 1, status, abort_flag);
+          // this lane's O part holds PV_0 .. PV_{j-1}: wait for the last, then rescale
+          mbar_wait_abortable(&p_free[(j - 1) % kRing], ((j - 1) / kRing) & 1, status, abort_flag);
           tc_fence_after();
-          uint32_t o[32];
-          const uint32_t ta = tO + lane_off + ch * (D / 4);
-          if constexpr (D == 128) {
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            uint32_t o[32];
+            const uint32_t ta = tO + lane_off + ch * (D / 2) + h * 32;
             tmem_ld32(ta, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st16(ta, o);
             tmem_st16(ta + 16, o + 16);
-          } else {
-            tmem_ld16(ta, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st16(ta, o);
           }
           tmem_st_wait();
-          tc_fence_before();
         }
       }
       uint32_t pk[16];
@@ -349,19 +357,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = 0u;
       }
-      if (j >= kPBufs) mbar_wait_abortable(&p_free[pb], ((j / kPBufs) & 1) ^ 1, status, abort_flag);
-      uint8_t* pt = sm + (pb < 2 ? L::kP0 + pb * L::kPBytes : L::kP2) + kh * kBoxBytes;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
-            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-      fence_proxy_async_smem();
+      // P buffer b last held P_{j-3}: free once PV_{j-3} completed
+      if (j >= kRing) mbar_wait_abortable(&p_free[b], ((j / kRing) & 1) ^ 1, status, abort_flag);
+      tmem_st16(tP + lane_off + b * 32 + ch * 16, pk);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[pb]);
+      if (lane == 0) mbar_arrive(&p_full[b]);
     }
     // ---------------------------------------------------------- epilogue
-    if (nsteps > 0)
-      mbar_wait_abortable(&p_free[(nsteps - 1) % kPBufs], ((nsteps - 1) / kPBufs) & 1, status, abort_flag);
+    if (nsteps > 0) mbar_wait_abortable(&p_free[(nsteps - 1) % kRing], ((nsteps - 1) / kRing) & 1, status, abort_flag);
     tc_fence_after();
     redl[q4 * 64 + m] = l_part;
     named_bar_sync(1, 32 * kSoftWarps);
@@ -371,18 +376,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     const int sI = safe_shape(g, P.zone_shape, I, status);
     const BlockBox qb = block_box(g, sI, I);
     const int tok = block_token(g, qb, m);
+    // This lane holds the key-block-kh part of O row m over channels
+    // [ch*D/2, ch*D/2 + D/2). It keeps the quarter [.. + kh*D/4, + D/4) and
+    // hands the other quarter to the thread of the other lane half.
     constexpr int NC = D / 4;
-    const int doff = kh * (D / 2) + ch * NC;
+    const int keep = ch * (D / 2) + kh * NC, give = ch * (D / 2) + (kh ^ 1) * NC;
     float ov[NC];
-    if (nsteps > 0) {
-      tmem_ld_f<NC>(tO + lane_off + ch * NC, ov);
+    if (nsteps > 0) {  // uniform; on an abort the values are discarded below
+      float gv[NC];
+      tmem_ld_f<NC>(tO + lane_off + give, gv);
+      tmem_ld_f<NC>(tO + lane_off + keep, ov);
+      float* xo = reinterpret_cast<float*>(sm + L::kK0) + ((kh * 2 + ch) * 64 + m) * L::kXPitch;
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i)
+        reinterpret_cast<float4*>(xo)[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
+      named_bar_sync(1, 32 * kSoftWarps);
+      const float* xi = reinterpret_cast<const float*>(sm + L::kK0) + (((kh ^ 1) * 2 + ch) * 64 + m) * L::kXPitch;
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i) {
+        const float4 t = reinterpret_cast<const float4*>(xi)[i];
+        ov[4 * i] += t.x;
+        ov[4 * i + 1] += t.y;
+        ov[4 * i + 2] += t.z;
+        ov[4 * i + 3] += t.w;
+      }
 #pragma unroll
       for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : ov[i] * inv;
     } else {
 #pragma unroll
       for (int i = 0; i < NC; ++i) ov[i] = 0.f;
     }
-    store_row<NC>(P.o, int64_t(tok) * P.tok_stride + int64_t(head) * D + doff, ov, P.out_fp32);
+    store_row<NC>(P.o, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, ov, P.out_fp32);
     if (q4 == 0) {
       const int N = g.T * g.H * g.W;
       P.lse[int64_t(head) * N + tok] = (l > 0.f && ok) ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
