@@ -322,39 +322,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
 }
 
 // --------------------------------------------------------------------- dkdv
-// Stages of (Q, dO, LSE, D) for two query blocks, 2 slots, each held until the
-// dV/dK products of its step complete; S^T/dP^T in TMEM (2 buffers each);
-// P^T and dS^T in one shared-memory buffer each. The issuer polls and starts
-// whichever of "scores of step s" / "dV, dK of step k" is ready.
+// Three stages of (Q, dO) for two query blocks, each held from its load until
+// the dV/dK products of its step complete. S^T / dP^T in TMEM (2 buffers each).
+// The K/V tile is staged through shared memory once, copied into TMEM (the A
+// operand of every S^T / dP^T product) and its shared-memory space then holds
+// P^T and dS^T, the A operands of the dV / dK products. LSE and D of the
+// step's query rows come straight from global memory into registers, one
+// step ahead.
+// The issuer runs one fixed order, A_0, A_1, B_0, A_2, B_1, A_3, ... with
+// A_j = (S^T_j, dP^T_j) and B_j = (dV += P^T_j dO_j, dK += dS^T_j Q_j). It
+// waits once per group: for stage j landed before A_j, for P^T_j / dS^T_j
+// written before B_j. A_{j+2} reuses the score buffers of step j, which the
+// softmax warps read before writing P^T_j, so that reuse needs no barrier of
+// its own.
 template <int D>
 struct DkvSmem {
-  static constexpr uint32_t kK = 0;
-  static constexpr uint32_t kV = D * 128;
-  static constexpr uint32_t kHalf = kKB * D * 128;  // Q (or dO) of one stage
-  static constexpr uint32_t kLD = 2 * kHalf;        // lse2 [slot][64], D [slot][64]
-  static constexpr uint32_t kStageBytes = 2 * kHalf + 1024;
-  static constexpr uint32_t kStage0 = 2 * D * 128;
-  static constexpr uint32_t kPT = kStage0 + 2 * kStageBytes;
-  static constexpr uint32_t kPBytes = kKB * kBoxBytes;
-  static constexpr uint32_t kDST = kPT + kPBytes;
-  static constexpr uint32_t kDesc = kDST + kPBytes;  // block coordinate ring
+  static constexpr uint32_t kKV = 0;               // K, V staging [2][dh][64][128 B]; then P^T, dS^T
+  static constexpr uint32_t kKVBytes = 32768;      // max(2 * D * 128, P^T + dS^T)
+  static constexpr uint32_t kPT = 0;               // [query block][64 keys][128 B]
+  static constexpr uint32_t kDST = kBoxBytes * kKB;
+  static constexpr uint32_t kHalf = kKB * D * 128;  // Q (or dO) of one stage, [dh][query block][64][128 B]
+  static constexpr uint32_t kStageBytes = 2 * kHalf;
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kStage0 = kKVBytes;
+  static constexpr uint32_t kDesc = kStage0 + kStages * kStageBytes;  // block coordinate ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
+  static_assert(2 * D * 128 <= kKVBytes && kDST + kKB * kBoxBytes <= kKVBytes, "staging tile");
 };
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_constant__ BwdParams P) {
   using L = DkvSmem<D>;
+  constexpr int NS = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* kv_full = bars + 0;
-  uint64_t* st_full = bars + 1;
-  uint64_t* st_empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_free = bars + 7;
-  uint64_t* ps_full = bars + 9;
-  uint64_t* ps_free = bars + 10;
+  uint64_t* st_full = bars + 1;   // [3] stage landed
+  uint64_t* st_free = bars + 4;   // [3] B of the stage's step complete
+  uint64_t* s_full = bars + 7;    // [2] A_j complete
+  uint64_t* ps_full = bars + 9;   // P^T_j, dS^T_j written (8 softmax warps)
+  uint64_t* ps_free = bars + 10;  // B_j complete (P^T / dS^T buffer free)
   uint64_t* mma_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
@@ -374,12 +383,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   const int nsteps = (cnt + kKB - 1) / kKB;
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(&st_full[i], 1);
-      mbar_init(&st_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kSoftWarps);
+      mbar_init(&st_free[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
     mbar_init(ps_full, kSoftWarps);
     mbar_init(ps_free, 1);
     mbar_init(mma_done, 1);
@@ -399,6 +407,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   const uint32_t tdV = tbase + 256, tdK = tbase + 320, tK = tbase + 384, tV = tbase + 448;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     if (nsteps > 0) {
       DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
       if (lane == 0) {
@@ -406,123 +415,134 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
         const BlockBox kb = block_box(g, sJ, J);
         mbar_arrive_expect_tx(kv_full, 2 * D * 128);
         for (int dh = 0; dh < D / 64; ++dh) {
-          tma_load_5d(sm + L::kK + dh * kBoxBytes, &P.mk[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
-          tma_load_5d(sm + L::kV + dh * kBoxBytes, &P.mv[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
+          tma_load_5d(sm + L::kKV + dh * kBoxBytes, &P.mk[sJ], kv_full, dh * 64, head, kb.w0, kb.h0, kb.t0);
+          tma_load_5d(sm + L::kKV + D * 128 + dh * kBoxBytes, &P.mv[sJ], kv_full, dh * 64, head, kb.w0, kb.h0,
+                      kb.t0);
         }
       }
+      bool ok = true;
       int issued = 0;
-      Watchdog wd;
-      wd.reset();
-      while (issued < nsteps) {
-        const int j = issued;
+      for (int j = 0; j < nsteps && ok; ++j) {
         dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, P.zone_shape, status, lane);
-        int go = 0, stop = 0;
         if (lane == 0) {
-          if (mbar_test(&st_empty[j & 1], ((j >> 1) & 1) ^ 1)) {
-            uint8_t* stage = sm + L::kStage0 + (j & 1) * L::kStageBytes;
-            uint64_t* bar = &st_full[j & 1];
-            mbar_arrive_expect_tx(bar, 2 * L::kHalf + kKB * 2 * 256);
+          const int s = j % NS;
+          // stage s last held step j - 3: free once its dV / dK products completed
+          if (j >= NS) ok = mbar_wait_abortable(&st_free[s], ((j / NS) - 1) & 1, status, abort_flag);
+          if (ok) {
+            uint8_t* stage = sm + L::kStage0 + s * L::kStageBytes;
+            mbar_arrive_expect_tx(&st_full[s], L::kStageBytes);
             for (int slot = 0; slot < kKB; ++slot) {
               const int4 b = dc.get(kKB * j + slot);
               for (int dh = 0; dh < D / 64; ++dh) {
                 const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
-                tma_load_5d(stage + off, &P.mq[b.x], bar, dh * 64, head, b.y, b.z, b.w);
-                tma_load_5d(stage + L::kHalf + off, &P.mdo[b.x], bar, dh * 64, head, b.y, b.z, b.w);
+                tma_load_5d(stage + off, &P.mq[b.x], &st_full[s], dh * 64, head, b.y, b.z, b.w);
+                tma_load_5d(stage + L::kHalf + off, &P.mdo[b.x], &st_full[s], dh * 64, head, b.y, b.z, b.w);
               }
-              int e = kKB * j + slot;
-              if (e >= cnt) e = kKB * j;
-              int Iq = P.idx[beg + e];
-              if (Iq < 0 || Iq >= g.n_blocks) Iq = 0;  // reported by the coordinate cache
-              const size_t rowoff = (size_t(head) * g.n_blocks + Iq) * 64;
-              bulk_load(stage + L::kLD + slot * 256, P.lse2 + rowoff, 256, bar);
-              bulk_load(stage + L::kLD + 512 + slot * 256, P.dvec + rowoff, 256, bar);
             }
-            go = 1;
-            wd.reset();
-          } else if (!wd.ok(status, abort_flag)) {
-            stop = 1;
+            issued = j + 1;
           }
         }
-        issued += __shfl_sync(0xffffffffu, go, 0);
-        if (__shfl_sync(0xffffffffu, stop, 0)) break;
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
       if (lane == 0) {
+        // drain: every issued copy has landed before the CTA may exit
         mbar_wait(kv_full, 0, status);
-        for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
-          mbar_wait(&st_full[i & 1], (i >> 1) & 1, status);
+        for (int i = issued - NS > 0 ? issued - NS : 0; i < issued; ++i)
+          mbar_wait(&st_full[i % NS], (i / NS) & 1, status);
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idO = idesc_bf16_f32(64, D, false, true);
       const uint64_t dPT = sdesc_sw128(smem_u32(sm + L::kPT), 16, 1024);
       const uint64_t dDST = sdesc_sw128(smem_u32(sm + L::kDST), 16, 1024);
       const uint32_t sQ0 = smem_u32(sm + L::kStage0);
-      const uint64_t dQ0 = sdesc_sw128(sQ0, 16, 1024);                                   // Q as B of S^T
-      const uint64_t dDO0 = sdesc_sw128(sQ0 + L::kHalf, 16, 1024);                       // dO as B of dP^T
-      const uint64_t dQmn0 = sdesc_sw128(sQ0, kKB * kBoxBytes, 1024);                    // Q as B of dK
-      const uint64_t dDOmn0 = sdesc_sw128(sQ0 + L::kHalf, kKB * kBoxBytes, 1024);        // dO as B of dV
+      const uint64_t dQ0 = sdesc_sw128(sQ0, 16, 1024);                             // Q as B of S^T
+      const uint64_t dDO0 = sdesc_sw128(sQ0 + L::kHalf, 16, 1024);                 // dO as B of dP^T
+      const uint64_t dQmn0 = sdesc_sw128(sQ0, kKB * kBoxBytes, 1024);              // Q as B of dK
+      const uint64_t dDOmn0 = sdesc_sw128(sQ0 + L::kHalf, kKB * kBoxBytes, 1024);  // dO as B of dV
       constexpr uint64_t kStageStep = L::kStageBytes >> 4;
       bool ok = mbar_wait_abortable(ka_full, 0, status, abort_flag);
-      tc_fence_after();
-      int sj = 0, kj = 0;
-      Watchdog wd;
-      wd.reset();
-      while (ok && kj < nsteps) {
-        bool did = false;
-        if (kj < sj && mbar_test(ps_full, kj & 1)) {
-          tc_fence_after();
-          const uint64_t st = uint64_t(kj & 1) * kStageStep;
+      // A_j: S^T_j = K Q_j^T and dP^T_j = V dO_j^T into score buffer j % 2
+      auto issue_a = [&](int j) {
+        const uint64_t st = uint64_t(j % NS) * kStageStep;
+        const uint32_t tS = tbase + (j & 1) * 64;
 #pragma unroll
-          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tdV, dPT + kmajor_step(kk, kBoxBytes), dDOmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
-                   (kj > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws_ts(tS, tK + kk * 8, dQ0 + st + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tdK, dDST + kmajor_step(kk, kBoxBytes), dQmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
-                   (kj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&st_empty[kj & 1]);
-          mma_commit(ps_free);
-          ++kj;
-          did = true;
-        }
-        if (sj < nsteps && mbar_test(&st_full[sj & 1], (sj >> 1) & 1) &&
-            mbar_test(&s_free[sj & 1], ((sj >> 1) & 1) ^ 1)) {
-          tc_fence_after();
-          const uint64_t st = uint64_t(sj & 1) * kStageStep;
-          const int sb = sj & 1;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + sb * 64, tK + kk * 8, dQ0 + st + kmajor_step(kk, kKB * kBoxBytes), idS,
-                      kk > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + 128 + sb * 64, tV + kk * 8, dDO0 + st + kmajor_step(kk, kKB * kBoxBytes), idS,
-                      kk > 0 ? 1u : 0u);
-          mma_commit(&s_full[sb]);
-          ++sj;
-          did = true;
-        }
-        if (did) wd.reset();
-        else if (!wd.ok(status, abort_flag)) break;
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws_ts(tS + 128, tV + kk * 8, dDO0 + st + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+        mma_commit(&s_full[j & 1]);
+      };
+      for (int j = 0; j < 2 && j < nsteps && ok; ++j) {
+        ok = mbar_wait_abortable(&st_full[j % NS], (j / NS) & 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_a(j);
       }
+      for (int j = 0; j < nsteps && ok; ++j) {
+        ok = mbar_wait_abortable(ps_full, j & 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t st = uint64_t(j % NS) * kStageStep;
+#pragma unroll
+        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+          mma_ws(tdV, dPT + kmajor_step(kk, kBoxBytes), dDOmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+          mma_ws(tdK, dDST + kmajor_step(kk, kBoxBytes), dQmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&st_free[j % NS]);
+        mma_commit(ps_free);
+        if (j + 2 < nsteps) {
+          ok = mbar_wait_abortable(&st_full[(j + 2) % NS], ((j + 2) / NS) & 1, status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_a(j + 2);
+        }
+      }
+      // every MMA this thread issued has completed before TMEM is released
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, status);
     }
   } else {
+    // ------------------------------------------------------------ softmax
     const int sw = warp - 2, sp = warp & 3, ch = sw >> 2;
     const int Ln = sp * 32 + lane;
     const int m = Ln & 63, kh = Ln >> 6;
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
+    // LSE * log2(e) and D of the 32 query rows this thread scores in step j
+    // (query block kh of the step, rows ch*32 ..), loaded one step ahead
+    float4 l2[8], dd[8];
+    auto load_ld = [&](int j) {
+      int e = kKB * j + kh;
+      if (e >= cnt) e = kKB * j;
+      int Iq = P.idx[beg + e];
+      if (Iq < 0 || Iq >= g.n_blocks) Iq = 0;  // reported by the coordinate cache
+      const size_t rowoff = (size_t(head) * g.n_blocks + Iq) * 64 + ch * 32;
+      const float4* a = reinterpret_cast<const float4*>(P.lse2 + rowoff);
+      const float4* b = reinterpret_cast<const float4*>(P.dvec + rowoff);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        l2[i] = __ldg(a + i);
+        dd[i] = __ldg(b + i);
+      }
+    };
     if (nsteps > 0) {
+      load_ld(0);
       // K and V are the A operands of every S^T / dP^T product: one copy into TMEM
       mbar_wait_abortable(kv_full, 0, status, abort_flag);
-      tile_to_tmem_a<D>(sm + L::kK, tK + lane_off, m, ch);
-      tile_to_tmem_a<D>(sm + L::kV, tV + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kKV, tK + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kKV + D * 128, tV + lane_off, m, ch);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ka_full);
+      // the staging tile holds P^T / dS^T from now on: every softmax warp has read it
+      named_bar_sync(1, 32 * kSoftWarps);
     }
     for (int j = 0; j < nsteps; ++j) {
       const int sb = j & 1;
@@ -532,16 +552,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
       tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      const bool valid = (j * kKB + kh) < cnt;
-      // the per-query LSE / D rows arrived by bulk copy on st_full: observe it
-      mbar_wait_abortable(&st_full[sb], (j >> 1) & 1, status, abort_flag);
-      const float* ld = reinterpret_cast<const float*>(sm + L::kStage0 + (j & 1) * L::kStageBytes + L::kLD);
-      // the 32 queries of this thread's columns: LSE * log2(e) and D, same for the whole warp
-      const float4* l2 = reinterpret_cast<const float4*>(ld + kh * 64 + ch * 32);
-      const float4* dd = reinterpret_cast<const float4*>(ld + 128 + kh * 64 + ch * 32);
+      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
       uint32_t pp[16], pd[16];
       if (valid) {
         const float c = P.scale_log2;
@@ -562,6 +573,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
 #pragma unroll
         for (int i = 0; i < 16; ++i) pp[i] = pd[i] = 0u;
       }
+      if (j + 1 < nsteps) load_ld(j + 1);  // in flight while this step is stored
+      // the P^T / dS^T buffer last held step j - 1: free once B_{j-1} completed
       if (j >= 1) mbar_wait_abortable(ps_free, (j - 1) & 1, status, abort_flag);
       uint8_t* pt = sm + L::kPT + kh * kBoxBytes;
       uint8_t* dt = sm + L::kDST + kh * kBoxBytes;
@@ -573,6 +586,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
             make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
       }
       fence_proxy_async_smem();
+      // this step's score reads precede the arrival: the issuer then reuses the buffers for A_{j+2}
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ps_full);
     }

@@ -121,19 +121,21 @@ __device__ __forceinline__ int safe_shape(const Geo& g, const int32_t* zone_shap
 // computed 32 at a time by a whole warp (coalesced list reads, parallel
 // zone-shape lookups) into a shared-memory ring, so the thread that issues the
 // TMA copies never waits on a dependent global load. Entry e of a list of
-// `cnt` blocks processed two per step: e < cnt is the list's e-th block; a
-// ragged tail (e >= cnt in the last step) repeats the step's first block.
+// `cnt` blocks processed `step` (a power of two) per step: e < cnt is the
+// list's e-th block; a ragged tail (e >= cnt in the last step) repeats the
+// step's first block.
 constexpr int kDescRing = 64;
 
 struct DescCache {
   int4* ring;  // shared memory, kDescRing entries
   int filled;
+  int step = 2;
   // Makes entries [0, e] available; the whole warp must call it.
   __device__ __forceinline__ void ensure(int e, const Geo& g, const int32_t* list, int beg, int cnt,
                                          const int32_t* zone_shape, int* status, int lane) {
     while (e >= filled) {
       const int ee = filled + lane;
-      int idx = ee < cnt ? ee : (ee & ~1);
+      int idx = ee < cnt ? ee : (ee & ~(step - 1));
       if (idx >= cnt) idx = 0;
       int J = list[beg + idx];
       if (J < 0 || J >= g.n_blocks) {
