@@ -58,47 +58,50 @@ struct BwdParams {
 };
 
 // ----------------------------------------------------------------------- dq
-// Rings: K (3 slots, held until the dQ product of its step completes), V (2
-// slots, held until the dP product), score buffers S/dP (3 each, TMEM),
-// dS (one shared-memory buffer). The producer and the issuer poll every
-// barrier they could act on and start whichever operation is ready.
-constexpr int kDqKSlots = 3;
-constexpr int kDqVSlots = 2;
-constexpr int kDqSBufs = 2;
-static_assert(kDqVSlots == kDqSBufs, "V slot j is released by the score barrier of step j");
-
+// Three slots, each holding K and V of one step (two key blocks) from its load
+// until the dQ product of that step completes. S / dP in TMEM (2 buffers
+// each). Q and dO are staged through shared memory once and copied into TMEM
+// (the A operands of every S / dP product); that shared-memory space then
+// holds dS in two buffers, the A operand of the dQ products.
+// The issuer runs one fixed order, A_0, A_1, B_0, A_2, B_1, ... with
+// A_j = (S_j = Q K_j^T, dP_j = dO V_j^T) and B_j = (dQ += dS_j K_j), waiting
+// once per group: for slot j landed before A_j, for dS_j written before B_j.
+// A_{j+2} reuses the score buffers of step j, which the softmax warps read
+// before writing dS_j, so that reuse needs no barrier of its own. dS_j goes to
+// buffer j % 2 and has its own ready barrier per buffer, so a parity wait on
+// it can never be two phases behind.
 template <int D>
 struct DqSmem {
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kDO = D * 128;
-  static constexpr uint32_t kSlotBytes = kKB * D * 128;  // K (or V) of one step, [dh][block][64][128 B]
-  static constexpr uint32_t kK0 = 2 * D * 128;
-  static constexpr uint32_t kV0 = kK0 + kDqKSlots * kSlotBytes;
-  static constexpr uint32_t kDS = kV0 + kDqVSlots * kSlotBytes;
-  static constexpr uint32_t kDSBytes = kKB * kBoxBytes;
-  static constexpr uint32_t kDesc = kDS + kDSBytes;  // block coordinate ring
+  static constexpr uint32_t kQD = 0;                 // Q, dO staging [2][dh][64][128 B]; then dS [2]
+  static constexpr uint32_t kQDBytes = 32768;        // max(2 * D * 128, two dS buffers)
+  static constexpr uint32_t kDSBytes = kKB * kBoxBytes;  // [key block][64 rows][128 B]
+  static constexpr uint32_t kHalf = kKB * D * 128;   // K (or V) of one step, [dh][key block][64][128 B]
+  static constexpr uint32_t kSlotBytes = 2 * kHalf;  // K then V
+  static constexpr int kSlots = 3;
+  static constexpr uint32_t kSlot0 = kQDBytes;
+  static constexpr uint32_t kDesc = kSlot0 + kSlots * kSlotBytes;  // block coordinate ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
+  static_assert(2 * D * 128 <= kQDBytes && 2 * kDSBytes <= kQDBytes, "staging tile");
 };
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_constant__ BwdParams P) {
   using L = DqSmem<D>;
+  constexpr int NS = L::kSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* qd_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [3]
-  uint64_t* k_empty = bars + 4;  // [3]
-  uint64_t* v_full = bars + 7;   // [2] (a V slot is free once the dP product that read it completed: s_full)
-  uint64_t* s_full = bars + 11;  // [3]
-  uint64_t* s_free = bars + 14;  // [3]
-  uint64_t* ds_full = bars + 17;
-  uint64_t* ds_free = bars + 18;
-  uint64_t* mma_done = bars + 19;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
-  uint64_t* qa_full = bars + 22;  // Q and dO copied into TMEM by the softmax warps
+  uint64_t* kv_full = bars + 1;    // [3] K and V of the slot's step landed
+  uint64_t* kv_free = bars + 4;    // [3] dQ product of the slot's step complete
+  uint64_t* s_full = bars + 7;     // [2] A_j complete
+  uint64_t* ds_full = bars + 9;    // [2] dS_j written (8 softmax warps), index j % 2
+  uint64_t* ds_free = bars + 11;   // [2] B_j complete (dS buffer j % 2 free)
+  uint64_t* mma_done = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* qa_full = bars + 16;  // Q and dO copied into TMEM by the softmax warps
 
   const Geo& g = P.g;
   const int I = blockIdx.x, head = blockIdx.y;
@@ -114,17 +117,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   const int nsteps = (cnt + kKB - 1) / kKB;
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    for (int i = 0; i < kDqKSlots; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_free[i], 1);
     }
-    for (int i = 0; i < kDqVSlots; ++i) mbar_init(&v_full[i], 1);
-    for (int i = 0; i < kDqSBufs; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kSoftWarps);
+      mbar_init(&ds_full[i], kSoftWarps);
+      mbar_init(&ds_free[i], 1);
     }
-    mbar_init(ds_full, kSoftWarps);
-    mbar_init(ds_free, 1);
     mbar_init(mma_done, 1);
     mbar_init(qa_full, kSoftWarps);
     *abort_flag = 0;
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   const uint32_t tdQ = tbase + 256, tQ = tbase + 320, tDO = tbase + 384;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     if (nsteps > 0) {
       DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
       if (lane == 0) {
@@ -149,103 +151,98 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         const BlockBox qb = block_box(g, sI, I);
         mbar_arrive_expect_tx(qd_full, 2 * D * 128);
         for (int dh = 0; dh < D / 64; ++dh) {
-          tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
-          tma_load_5d(sm + L::kDO + dh * kBoxBytes, &P.mdo[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+          tma_load_5d(sm + L::kQD + dh * kBoxBytes, &P.mq[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+          tma_load_5d(sm + L::kQD + D * 128 + dh * kBoxBytes, &P.mdo[sI], qd_full, dh * 64, head, qb.w0, qb.h0,
+                      qb.t0);
         }
       }
-      auto load_step = [&](const CUtensorMap* maps, uint8_t* dst, uint64_t* bar, int j) {
-        mbar_arrive_expect_tx(bar, L::kSlotBytes);
-        for (int slot = 0; slot < kKB; ++slot) {
-          const int4 b = dc.get(kKB * j + slot);
-          for (int dh = 0; dh < D / 64; ++dh)
-            tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &maps[b.x], bar, dh * 64, head, b.y, b.z,
-                        b.w);
-        }
-      };
-      int kj = 0, vj = 0;
-      Watchdog wd;
-      wd.reset();
-      while (kj < nsteps || vj < nsteps) {
-        if (kj < nsteps) dc.ensure(kKB * kj + kKB - 1, g, P.idx, beg, cnt, P.zone_shape, status, lane);
-        int nk = kj, nv = vj, stop = 0;
+      bool ok = true;
+      int issued = 0;
+      for (int j = 0; j < nsteps && ok; ++j) {
+        dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, P.zone_shape, status, lane);
         if (lane == 0) {
-          bool did = false;
-          if (nk < nsteps && mbar_test(&k_empty[nk % kDqKSlots], ((nk / kDqKSlots) & 1) ^ 1)) {
-            load_step(P.mk, sm + L::kK0 + (nk % kDqKSlots) * L::kSlotBytes, &k_full[nk % kDqKSlots], nk);
-            ++nk;
-            did = true;
+          const int s = j % NS;
+          // slot s last held step j - 3: free once its dQ product completed
+          if (j >= NS) ok = mbar_wait_abortable(&kv_free[s], ((j / NS) - 1) & 1, status, abort_flag);
+          if (ok) {
+            uint8_t* dst = sm + L::kSlot0 + s * L::kSlotBytes;
+            mbar_arrive_expect_tx(&kv_full[s], L::kSlotBytes);
+            for (int slot = 0; slot < kKB; ++slot) {
+              const int4 b = dc.get(kKB * j + slot);
+              for (int dh = 0; dh < D / 64; ++dh) {
+                const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
+                tma_load_5d(dst + off, &P.mk[b.x], &kv_full[s], dh * 64, head, b.y, b.z, b.w);
+                tma_load_5d(dst + L::kHalf + off, &P.mv[b.x], &kv_full[s], dh * 64, head, b.y, b.z, b.w);
+              }
+            }
+            issued = j + 1;
           }
-          if (nv < nk && mbar_test(&s_full[nv % kDqSBufs], ((nv / kDqSBufs) & 1) ^ 1)) {
-            load_step(P.mv, sm + L::kV0 + (nv & 1) * L::kSlotBytes, &v_full[nv & 1], nv);
-            ++nv;
-            did = true;
-          }
-          if (did) wd.reset();
-          else if (!wd.ok(status, abort_flag)) stop = 1;
         }
-        kj = __shfl_sync(0xffffffffu, nk, 0);
-        vj = __shfl_sync(0xffffffffu, nv, 0);
-        if (__shfl_sync(0xffffffffu, stop, 0)) break;
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
       if (lane == 0) {
+        // drain: every issued copy has landed before the CTA may exit
         mbar_wait(qd_full, 0, status);
-        for (int i = kj - kDqKSlots > 0 ? kj - kDqKSlots : 0; i < kj; ++i)
-          mbar_wait(&k_full[i % kDqKSlots], (i / kDqKSlots) & 1, status);
-        for (int i = vj - kDqVSlots > 0 ? vj - kDqVSlots : 0; i < vj; ++i)
-          mbar_wait(&v_full[i & 1], (i >> 1) & 1, status);
+        for (int i = issued - NS > 0 ? issued - NS : 0; i < issued; ++i)
+          mbar_wait(&kv_full[i % NS], (i / NS) & 1, status);
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
       const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
-      const uint64_t dDS = sdesc_sw128(smem_u32(sm + L::kDS), 16, 1024);
-      const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::kK0), 16, 1024);                 // K as B of S
-      const uint64_t dKmn0 = sdesc_sw128(smem_u32(sm + L::kK0), kKB * kBoxBytes, 1024);  // K as B of dQ
-      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), 16, 1024);
+      const uint64_t dDS0 = sdesc_sw128(smem_u32(sm + L::kQD), 16, 1024);
+      const uint32_t sK0 = smem_u32(sm + L::kSlot0);
+      const uint64_t dK0 = sdesc_sw128(sK0, 16, 1024);                        // K as B of S
+      const uint64_t dKmn0 = sdesc_sw128(sK0, kKB * kBoxBytes, 1024);         // K as B of dQ
+      const uint64_t dV0 = sdesc_sw128(sK0 + L::kHalf, 16, 1024);             // V as B of dP
+      constexpr uint64_t kSlotStep = L::kSlotBytes >> 4;
+      constexpr uint64_t kDSStep = L::kDSBytes >> 4;
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
-      tc_fence_after();
-      int sj = 0, qj = 0;
-      Watchdog wd;
-      wd.reset();
-      while (ok && qj < nsteps) {
-        bool did = false;
-        if (qj < sj && mbar_test(ds_full, qj & 1)) {
-          tc_fence_after();
-          const uint64_t dK = dKmn0 + uint64_t((qj % kDqKSlots) * (L::kSlotBytes >> 4));
+      // A_j: S_j and dP_j into score buffer j % 2
+      auto issue_a = [&](int j) {
+        const uint64_t so = uint64_t(j % NS) * kSlotStep;
+        const uint32_t tS = tbase + (j & 1) * 64;
 #pragma unroll
-          for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-            mma_ws(tdQ, dDS + kmajor_step(kk, kBoxBytes), dK + mnmajor_step(kk, kBoxBytes), idQ,
-                   (qj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&k_empty[qj % kDqKSlots]);
-          mma_commit(ds_free);
-          ++qj;
-          did = true;
-        }
-        if (sj < nsteps && mbar_test(&k_full[sj % kDqKSlots], (sj / kDqKSlots) & 1) &&
-            mbar_test(&v_full[sj & 1], (sj >> 1) & 1) && mbar_test(&s_free[sj % kDqSBufs], ((sj / kDqSBufs) & 1) ^ 1)) {
-          tc_fence_after();
-          const uint64_t dK = dK0 + uint64_t((sj % kDqKSlots) * (L::kSlotBytes >> 4));
-          const uint64_t dV = dV0 + uint64_t((sj & 1) * (L::kSlotBytes >> 4));
-          const int sb = sj % kDqSBufs;
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws_ts(tS, tQ + kk * 8, dK0 + so + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + sb * 64, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + 128 + sb * 64, tDO + kk * 8, dV + kmajor_step(kk, kKB * kBoxBytes), idS,
-                      kk > 0 ? 1u : 0u);
-          mma_commit(&s_full[sb]);
-          ++sj;
-          did = true;
-        }
-        if (did) wd.reset();
-        else if (!wd.ok(status, abort_flag)) break;
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws_ts(tS + 128, tDO + kk * 8, dV0 + so + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+        mma_commit(&s_full[j & 1]);
+      };
+      for (int j = 0; j < 2 && j < nsteps && ok; ++j) {
+        ok = mbar_wait_abortable(&kv_full[j % NS], (j / NS) & 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_a(j);
       }
+      for (int j = 0; j < nsteps && ok; ++j) {
+        ok = mbar_wait_abortable(&ds_full[j & 1], (j >> 1) & 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t so = uint64_t(j % NS) * kSlotStep;
+        const uint64_t dDS = dDS0 + uint64_t(j & 1) * kDSStep;
+#pragma unroll
+        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
+          mma_ws(tdQ, dDS + kmajor_step(kk, kBoxBytes), dKmn0 + so + mnmajor_step(kk, kBoxBytes), idQ,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&kv_free[j % NS]);
+        mma_commit(&ds_free[j & 1]);
+        if (j + 2 < nsteps) {
+          ok = mbar_wait_abortable(&kv_full[(j + 2) % NS], ((j + 2) / NS) & 1, status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_a(j + 2);
+        }
+      }
+      // every MMA this thread issued has completed before TMEM is released
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, status);
     }
   } else {
+    // ------------------------------------------------------------ softmax
     const int sw = warp - 2, sp = warp & 3, ch = sw >> 2;
     const int Ln = sp * 32 + lane;
     const int m = Ln & 63, kh = Ln >> 6;
@@ -255,23 +252,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     if (nsteps > 0) {
       // Q and dO are the A operands of every S / dP product: one copy into TMEM
       mbar_wait_abortable(qd_full, 0, status, abort_flag);
-      tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, ch);
-      tile_to_tmem_a<D>(sm + L::kDO, tDO + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kQD, tQ + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kQD + D * 128, tDO + lane_off, m, ch);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(qa_full);
+      // the staging tile holds dS from now on: every softmax warp has read it
+      named_bar_sync(1, 32 * kSoftWarps);
     }
     for (int j = 0; j < nsteps; ++j) {
-      const int sb = j % kDqSBufs;
-      mbar_wait_abortable(&s_full[sb], (j / kDqSBufs) & 1, status, abort_flag);
+      const int sb = j & 1;
+      mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t rs[32], rp[32];
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
       tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
       const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
       uint32_t pk[16];
       if (valid) {
@@ -286,17 +282,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = 0u;
       }
-      if (j >= 1) mbar_wait_abortable(ds_free, (j - 1) & 1, status, abort_flag);
-      uint8_t* pt = sm + L::kDS + kh * kBoxBytes;
+      // dS buffer j % 2 last held dS_{j-2}: free once B_{j-2} completed
+      if (j >= 2) mbar_wait_abortable(&ds_free[sb], ((j - 2) >> 1) & 1, status, abort_flag);
+      uint8_t* pt = sm + L::kQD + sb * L::kDSBytes + kh * kBoxBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
             make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       fence_proxy_async_smem();
+      // this step's score reads precede the arrival: the issuer then reuses the buffers for A_{j+2}
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (lane == 0) mbar_arrive(&ds_full[sb]);
     }
-    if (nsteps > 0) mbar_wait_abortable(ds_free, (nsteps - 1) & 1, status, abort_flag);
+    if (nsteps > 0) mbar_wait_abortable(&ds_free[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, status, abort_flag);
     tc_fence_after();
     const bool ok = *abort_flag == 0;
     constexpr int NC = D / 4;
