@@ -2,8 +2,8 @@
 // "Overview"; mean pooling as the block feature).
 //
 // One CTA per (block, tensor): each thread owns 8 consecutive channels of the
-// token row [heads * head_dim] and walks the block's 64 tokens (bt rows of bh
-// runs of bw contiguous tokens), accumulating in fp32 with 16-byte loads.
+// token row [heads * head_dim] and walks the block's 64 tokens eight at a time
+// (eight independent 16-byte loads in flight), accumulating in fp32.
 // The output layout is [heads, n_blocks, head_dim] fp32.
 #include <cuda_bf16.h>
 
@@ -55,18 +55,23 @@ __global__ void __launch_bounds__(1024) pool_kernel(const Geo g, const int32_t* 
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int rt = 0; rt < bb.bt; ++rt) {
-    for (int rh = 0; rh < bb.bh; ++rh) {
-      const int64_t n0 = (int64_t(bb.t0 + rt) * g.H + bb.h0 + rh) * g.W + bb.w0;
-      const T* row = src + n0 * tok_stride + c0;
-#pragma unroll 4
-      for (int rw = 0; rw < bb.bw; ++rw) {
-        float x[8];
-        load8<T>(row + int64_t(rw) * tok_stride, x);
+  // Block extents divide 64, so they are powers of two: token r of the block
+  // (raster t, h, w) is found with shifts. Eight independent loads in flight.
+  const int lw = __ffs(bb.bw) - 1, lhw = lw + __ffs(bb.bh) - 1;
+  const T* base = src + c0;
+  for (int r0 = 0; r0 < kBlockTokens; r0 += 8) {
+    float x[8][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += x[i];
-      }
+    for (int i = 0; i < 8; ++i) {
+      const int r = r0 + i;
+      const int rt = r >> lhw, rh = (r >> lw) & (bb.bh - 1), rw = r & (bb.bw - 1);
+      const int64_t n = (int64_t(bb.t0 + rt) * g.H + bb.h0 + rh) * g.W + bb.w0 + rw;
+      load8<T>(base + n * tok_stride, x[i]);
     }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += x[i][c];
   }
   const float inv = 1.0f / 64.0f;
   reinterpret_cast<float4*>(out)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);

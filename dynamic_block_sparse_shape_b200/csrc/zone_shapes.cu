@@ -14,6 +14,9 @@
 //                slice into shared memory per stage; 8 warps each own one of
 //                {t, h, w line sums, plain sum of squares} x {even, odd
 //                lines}; lanes own one 4-byte word (2 bf16 / 1 fp32 channels).
+//   feat_stats8  the same statistics for 8 x 8 x 8 zones: 16 compute warps
+//                over t-slices and h-planes, 16-byte shared loads, fixed
+//                strides (the general kernel serves every other zone shape).
 //   res_norm     one warp per token: r(n) = ||res[n, :]||_2 in fp32.
 //   zone_res     one CTA per zone: line variances of r along t/h/w (fp64) and
 //                the zone sum of r.
@@ -134,6 +137,170 @@ __global__ void __launch_bounds__(kFeatThreads, 1)
       partial[size_t(tile) * 8 + warp] = acc;
       mbar_arrive(&empty_bar[s]);
     }
+  }
+}
+
+// The same statistics for 8 x 8 x 8 zones, with fixed strides and 16-byte
+// shared loads. 16 compute warps: warp k < 8 owns the t-slice t = k (sum of
+// squares, the line sums along w and along h of that slice), warp 8 + k the
+// h-plane h = k (line sums along t). A lane owns one 16-byte channel group
+// (cg = lane % 8) of rows w = q and w = q + 4 (q = lane / 8), so one load
+// instruction covers four rows. The 16 warps' sums are combined in a fixed
+// order by warp 0 (deterministic) into the per-tile layout {t, h, w, x^2}
+// (slots 2 * kind; slots 2 * kind + 1 are zero).
+constexpr int kFeat8Warps = 16;
+constexpr int kFeat8Threads = 32 * (kFeat8Warps + 1);
+
+template <int ES>
+__device__ __forceinline__ void unpack16(const uint4 u, float* x) {
+  if constexpr (ES == 2) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    x[0] = __uint_as_float(u.x);
+    x[1] = __uint_as_float(u.y);
+    x[2] = __uint_as_float(u.z);
+    x[3] = __uint_as_float(u.w);
+  }
+}
+
+template <int ES>
+__global__ void __launch_bounds__(kFeat8Threads, 1)
+    feat_stats8_kernel(const __grid_constant__ CUtensorMap fmap, const Geo g, int n_chunks, float* __restrict__ partial,
+                       int* status) {
+  constexpr int CPL = 16 / ES;        // channels per lane
+  constexpr uint32_t kTile = 512 * 128;  // one zone x 128-byte channel slice
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* red = reinterpret_cast<float*>(smem + kFeatStages * kTile);  // [stage][warp][4]
+  __shared__ uint64_t full_bar[kFeatStages], empty_bar[kFeatStages], red_bar[kFeatStages];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = g.n_zones * n_chunks;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFeatStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kFeat8Warps);
+      mbar_init(&red_bar[s], kFeat8Warps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == kFeat8Warps) {
+    if (lane == 0) {
+      tma_prefetch_desc(&fmap);
+      int k = 0;
+      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++k) {
+        const int s = k % kFeatStages;
+        if (!mbar_wait(&empty_bar[s], ((k / kFeatStages) & 1) ^ 1, status)) break;
+        const int z = tile / n_chunks, c = tile - z * n_chunks;
+        const int zt = z / (g.nzh * g.nzw), zr = z - zt * g.nzh * g.nzw;
+        const int zh = zr / g.nzw, zw = zr - zh * g.nzw;
+        mbar_arrive_expect_tx(&full_bar[s], kTile);
+        tma_load_4d(smem + size_t(s) * kTile, &fmap, &full_bar[s], c * (128 / ES), zw * 8, zh * 8, zt * 8);
+      }
+    }
+    return;
+  }
+  const int q = lane >> 3, cg = lane & 7;
+  const bool slice = warp < 8;  // t-slice (true) or h-plane (false)
+  const int k8 = warp & 7;
+  int k = 0;
+  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++k) {
+    const int s = k % kFeatStages;
+    if (!mbar_wait(&full_bar[s], (k / kFeatStages) & 1, status)) break;
+    const uint8_t* base = smem + size_t(s) * kTile + cg * 16;
+    float col[2][CPL];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) col[a][c] = 0.f;
+    float a_sq = 0.f, a_w = 0.f, a_col = 0.f;
+    if (slice) {
+      // rows t*64 + 4i + q: h = i / 2, w = 4 (i % 2) + q
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        float x0[CPL], x1[CPL], rp[CPL];
+        unpack16<ES>(*reinterpret_cast<const uint4*>(base + (k8 * 64 + 8 * h + q) * 128), x0);
+        unpack16<ES>(*reinterpret_cast<const uint4*>(base + (k8 * 64 + 8 * h + 4 + q) * 128), x1);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          a_sq = fmaf(x0[c], x0[c], fmaf(x1[c], x1[c], a_sq));
+          col[0][c] += x0[c];
+          col[1][c] += x1[c];
+          rp[c] = x0[c] + x1[c];
+        }
+        // line sum along w of (t, h): the four q-lanes of this channel group
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          rp[c] += __shfl_xor_sync(0xffffffffu, rp[c], 8);
+          rp[c] += __shfl_xor_sync(0xffffffffu, rp[c], 16);
+        }
+        if (q == 0) {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) a_w = fmaf(rp[c], rp[c], a_w);
+        }
+      }
+    } else {
+      // rows t*64 + h*8 + 4 (i % 2) + q with t = i / 2: the columns are the t-lines
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        float x0[CPL], x1[CPL];
+        unpack16<ES>(*reinterpret_cast<const uint4*>(base + (t * 64 + k8 * 8 + q) * 128), x0);
+        unpack16<ES>(*reinterpret_cast<const uint4*>(base + (t * 64 + k8 * 8 + 4 + q) * 128), x1);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          col[0][c] += x0[c];
+          col[1][c] += x1[c];
+        }
+      }
+    }
+    // column sums are complete line sums (along h for a t-slice, along t for an h-plane)
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) a_col = fmaf(col[a][c], col[a][c], a_col);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      a_sq += __shfl_xor_sync(0xffffffffu, a_sq, o);
+      a_w += __shfl_xor_sync(0xffffffffu, a_w, o);
+      a_col += __shfl_xor_sync(0xffffffffu, a_col, o);
+    }
+    float* rs = red + (s * kFeat8Warps + warp) * 4;
+    if (lane == 0) {
+      rs[0] = a_col;  // t-slice: h-lines; h-plane: t-lines
+      rs[1] = a_w;
+      rs[2] = a_sq;
+      mbar_arrive(&red_bar[s]);
+    }
+    if (warp == 0) {
+      // combine the 16 warps in a fixed order; the tile's stage is released after it
+      if (lane == 0) {
+        const bool ok = mbar_wait(&red_bar[s], (k / kFeatStages) & 1, status);
+        const float* r = red + s * kFeat8Warps * 4;
+        float st = 0.f, sh = 0.f, sw = 0.f, sq = 0.f;
+        for (int w = 0; w < 8; ++w) {
+          sh += r[w * 4 + 0];
+          sw += r[w * 4 + 1];
+          sq += r[w * 4 + 2];
+          st += r[(8 + w) * 4 + 0];
+        }
+        float* p = partial + size_t(tile) * 8;
+        p[0] = ok ? st : 0.f;
+        p[1] = 0.f;
+        p[2] = ok ? sh : 0.f;
+        p[3] = 0.f;
+        p[4] = ok ? sw : 0.f;
+        p[5] = 0.f;
+        p[6] = ok ? sq : 0.f;
+        p[7] = 0.f;
+      }
+      __syncwarp();
+    }
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
   }
 }
 
@@ -296,6 +463,44 @@ int sm_count() {
   return n;
 }
 
+// Channel line statistics of the features into `partial` ([tile][8], tile =
+// zone * n_chunks + 128-byte channel slice): the fixed-stride kernel for
+// 8 x 8 x 8 zones, the general one otherwise.
+prism_status launch_feat_stats(const Geo& g, const void* feat, int64_t feat_ld, int feat_c, int fes, int n_chunks,
+                               float* partial, int* status, cudaStream_t s) {
+  CUtensorMap fmap;
+  const uint64_t dims[4] = {uint64_t(feat_c), uint64_t(g.W), uint64_t(g.H), uint64_t(g.T)};
+  const uint64_t strides[3] = {uint64_t(feat_ld) * fes, uint64_t(feat_ld) * fes * g.W,
+                               uint64_t(feat_ld) * fes * g.W * g.H};
+  const uint32_t box[4] = {uint32_t(128 / fes), uint32_t(g.Zw), uint32_t(g.Zh), uint32_t(g.Zt)};
+  prism_status st = encode_tiled(&fmap, fes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                                 4, feat, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != PRISM_OK) return st;
+  const int n_tiles = g.n_zones * n_chunks;
+  const int grid = std::min(n_tiles, sm_count());
+  if (g.Zt == 8 && g.Zh == 8 && g.Zw == 8) {
+    const size_t smem = size_t(kFeatStages) * 512 * 128 + size_t(kFeatStages) * kFeat8Warps * 4 * sizeof(float) + 1024;
+    if (fes == 2) {
+      cudaFuncSetAttribute(feat_stats8_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      feat_stats8_kernel<2><<<grid, kFeat8Threads, smem, s>>>(fmap, g, n_chunks, partial, status);
+    } else {
+      cudaFuncSetAttribute(feat_stats8_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      feat_stats8_kernel<4><<<grid, kFeat8Threads, smem, s>>>(fmap, g, n_chunks, partial, status);
+    }
+  } else {
+    const size_t smem = size_t(kFeatStages) * g.Zt * g.Zh * g.Zw * 128 + 1024;
+    if (fes == 2) {
+      cudaFuncSetAttribute(feat_stats_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      feat_stats_kernel<2><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
+    } else {
+      cudaFuncSetAttribute(feat_stats_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      feat_stats_kernel<4><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
+    }
+  }
+  return cudaGetLastError() == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA;
+}
+
+
 struct ZoneWs {
   size_t partial, r, zres, total;
 };
@@ -361,25 +566,7 @@ extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void*
   const int N = g.T * g.H * g.W;
   const int n_chunks = feat_c * fes / 128;
   if (feat) {
-    CUtensorMap fmap;
-    const uint64_t dims[4] = {uint64_t(feat_c), uint64_t(g.W), uint64_t(g.H), uint64_t(g.T)};
-    const uint64_t strides[3] = {uint64_t(feat_ld) * fes, uint64_t(feat_ld) * fes * g.W,
-                                 uint64_t(feat_ld) * fes * g.W * g.H};
-    const uint32_t box[4] = {uint32_t(128 / fes), uint32_t(g.Zw), uint32_t(g.Zh), uint32_t(g.Zt)};
-    st = encode_tiled(&fmap, fes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, feat,
-                      dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != PRISM_OK) return st;
-    const size_t smem = size_t(kFeatStages) * g.Zt * g.Zh * g.Zw * 128 + 1024;
-    const int n_tiles = g.n_zones * n_chunks;
-    const int grid = std::min(n_tiles, sm_count());
-    if (fes == 2) {
-      cudaFuncSetAttribute(feat_stats_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      feat_stats_kernel<2><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
-    } else {
-      cudaFuncSetAttribute(feat_stats_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      feat_stats_kernel<4><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
-    }
-    if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
+    if ((st = launch_feat_stats(g, feat, feat_ld, feat_c, fes, n_chunks, partial, status, s)) != PRISM_OK) return st;
   }
   if (res) {
     const int res_es = res_dtype == PRISM_FP32 ? 4 : 2;
@@ -475,24 +662,7 @@ extern "C" prism_status prism_zone_shapes_static(const prism_geometry* geo, cons
   const int N = g.T * g.H * g.W;
   const int n_chunks = feat_c * fes / 128;
   if (feat) {
-    CUtensorMap fmap;
-    const uint64_t dims[4] = {uint64_t(feat_c), uint64_t(g.W), uint64_t(g.H), uint64_t(g.T)};
-    const uint64_t strides[3] = {uint64_t(feat_ld) * fes, uint64_t(feat_ld) * fes * g.W,
-                                 uint64_t(feat_ld) * fes * g.W * g.H};
-    const uint32_t box[4] = {uint32_t(128 / fes), uint32_t(g.Zw), uint32_t(g.Zh), uint32_t(g.Zt)};
-    st = encode_tiled(&fmap, fes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, feat,
-                      dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != PRISM_OK) return st;
-    const size_t smem = size_t(kFeatStages) * g.Zt * g.Zh * g.Zw * 128 + 1024;
-    const int grid = std::min(g.n_zones * n_chunks, sm_count());
-    if (fes == 2) {
-      cudaFuncSetAttribute(feat_stats_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      feat_stats_kernel<2><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
-    } else {
-      cudaFuncSetAttribute(feat_stats_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      feat_stats_kernel<4><<<grid, kFeatThreads, smem, s>>>(fmap, g, n_chunks, partial, status);
-    }
-    if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
+    if ((st = launch_feat_stats(g, feat, feat_ld, feat_c, fes, n_chunks, partial, status, s)) != PRISM_OK) return st;
   }
   if (res) {
     const int res_es = res_dtype == PRISM_FP32 ? 4 : 2;
