@@ -20,8 +20,9 @@
 //   res_norm     one warp per token: r(n) = ||res[n, :]||_2 in fp32.
 //   zone_res     one CTA per zone: line variances of r along t/h/w (fp64) and
 //                the zone sum of r.
-//   choose       one CTA: grid mean of r, then per zone the costs in fp64,
-//                argmin (ties to the lower index) and margin.
+//   choose       one warp per zone: grid mean of r (every CTA, same order),
+//                the zone's chunk partials, then the costs in fp64, argmin
+//                (ties to the lower index) and margin.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -383,14 +384,19 @@ __global__ void __launch_bounds__(256) zone_res_kernel(const Geo g, const float*
   }
 }
 
-__global__ void __launch_bounds__(1024) choose_kernel(const Geo g, const float* __restrict__ partial, int n_chunks,
-                                                      int feat_c, const double* __restrict__ zres, int have_feat,
-                                                      int have_res, float w_audio, float gamma, float gate_max,
-                                                      int32_t* __restrict__ zone_shape,
-                                                      float* __restrict__ zone_margin) {
-  __shared__ double red[1024];
-  __shared__ double mbar_s;
-  const int tid = threadIdx.x;
+// One warp per zone (8 zones per CTA). Every CTA first forms the grid mean of
+// r from the per-zone sums in the same fixed order (so all CTAs agree), then
+// each warp sums its zone's per-chunk partials (lanes over chunks, fp64) and
+// lane 0 evaluates the costs.
+constexpr int kChooseWarps = 8;
+__global__ void __launch_bounds__(32 * kChooseWarps) choose_kernel(const Geo g, const float* __restrict__ partial,
+                                                                   int n_chunks, int feat_c,
+                                                                   const double* __restrict__ zres, int have_feat,
+                                                                   int have_res, float w_audio, float gamma,
+                                                                   float gate_max, int32_t* __restrict__ zone_shape,
+                                                                   float* __restrict__ zone_margin) {
+  __shared__ double red[32 * kChooseWarps];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   double s = 0;
   if (have_res)
     for (int z = tid; z < g.n_zones; z += blockDim.x) s += zres[size_t(z) * 4 + 3];
@@ -400,56 +406,64 @@ __global__ void __launch_bounds__(1024) choose_kernel(const Geo g, const float* 
     if (tid < w) red[tid] += red[tid + w];
     __syncthreads();
   }
-  if (tid == 0) mbar_s = red[0] / (double(g.T) * g.H * g.W);
-  __syncthreads();
-  const double mbar = mbar_s;
+  const double mbar = red[0] / (double(g.T) * g.H * g.W);
+  const int z = blockIdx.x * kChooseWarps + warp;
+  if (z >= g.n_zones) return;
+  double q[4] = {0, 0, 0, 0};
+  if (have_feat) {
+    for (int c = lane; c < n_chunks; c += 32) {
+      const float4 a = *reinterpret_cast<const float4*>(partial + (size_t(z) * n_chunks + c) * 8);
+      const float4 b = *reinterpret_cast<const float4*>(partial + (size_t(z) * n_chunks + c) * 8 + 4);
+      q[0] += double(a.x) + double(a.y);
+      q[1] += double(a.z) + double(a.w);
+      q[2] += double(b.x) + double(b.y);
+      q[3] += double(b.z) + double(b.w);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int o = 16; o; o >>= 1) q[k] += __shfl_xor_sync(0xffffffffu, q[k], o);
+  }
+  if (lane != 0) return;
+  if (!have_feat && !have_res) {
+    zone_shape[z] = 0;
+    if (zone_margin) zone_margin[z] = INFINITY;
+    return;
+  }
   const double zvol = double(g.Zt) * g.Zh * g.Zw;
   const double Z[3] = {double(g.Zt), double(g.Zh), double(g.Zw)};
-  for (int z = tid; z < g.n_zones; z += blockDim.x) {
-    if (!have_feat && !have_res) {
-      zone_shape[z] = 0;
-      if (zone_margin) zone_margin[z] = INFINITY;
-      continue;
-    }
-    double V[3] = {0, 0, 0}, A[3] = {0, 0, 0};
-    if (have_feat) {
-      double q[4] = {0, 0, 0, 0};
-      for (int c = 0; c < n_chunks; ++c) {
-        const float* p = partial + (size_t(z) * n_chunks + c) * 8;
-        for (int k = 0; k < 4; ++k) q[k] += double(p[2 * k]) + double(p[2 * k + 1]);
-      }
-      for (int a = 0; a < 3; ++a) V[a] = (q[3] - q[a] / Z[a]) / (zvol * feat_c);
-    }
-    double gz = 0;
-    if (have_res && mbar > 0) {
-      for (int a = 0; a < 3; ++a) A[a] = zres[size_t(z) * 4 + a];
-      const double m = zres[size_t(z) * 4 + 3] / zvol;
-      gz = fmin(fmax(m / mbar - 1.0, 0.0), double(gate_max));
-    }
-    const double sv = V[0] + V[1] + V[2] + 1e-12, sa = A[0] + A[1] + A[2] + 1e-12;
-    double S[3];
-    for (int a = 0; a < 3; ++a) S[a] = 3.0 * V[a] / sv + double(w_audio) * gz * 3.0 * A[a] / sa;
-    const double tot = S[0] + S[1] + S[2];
-    for (int a = 0; a < 3; ++a) S[a] = tot > 0 ? 3.0 * S[a] / tot : 1.0;
-    double best = INFINITY, second = INFINITY;
-    int bi = 0;
-    for (int c = 0; c < g.n_cand; ++c) {
-      double cost = 0;
-      for (int a = 0; a < 3; ++a) {
-        const double e = log2(double(g.cand[c][a]));
-        cost += S[a] * e + double(gamma) * (e - 2.0) * (e - 2.0);
-      }
-      if (cost < best) {
-        second = best;
-        best = cost;
-        bi = c;
-      } else if (cost < second) {
-        second = cost;
-      }
-    }
-    zone_shape[z] = bi;
-    if (zone_margin) zone_margin[z] = float(second - best);
+  double V[3] = {0, 0, 0}, A[3] = {0, 0, 0};
+  if (have_feat)
+    for (int a = 0; a < 3; ++a) V[a] = (q[3] - q[a] / Z[a]) / (zvol * feat_c);
+  double gz = 0;
+  if (have_res && mbar > 0) {
+    for (int a = 0; a < 3; ++a) A[a] = zres[size_t(z) * 4 + a];
+    const double m = zres[size_t(z) * 4 + 3] / zvol;
+    gz = fmin(fmax(m / mbar - 1.0, 0.0), double(gate_max));
   }
+  const double sv = V[0] + V[1] + V[2] + 1e-12, sa = A[0] + A[1] + A[2] + 1e-12;
+  double S[3];
+  for (int a = 0; a < 3; ++a) S[a] = 3.0 * V[a] / sv + double(w_audio) * gz * 3.0 * A[a] / sa;
+  const double tot = S[0] + S[1] + S[2];
+  for (int a = 0; a < 3; ++a) S[a] = tot > 0 ? 3.0 * S[a] / tot : 1.0;
+  double best = INFINITY, second = INFINITY;
+  int bi = 0;
+  for (int c = 0; c < g.n_cand; ++c) {
+    double cost = 0;
+    for (int a = 0; a < 3; ++a) {
+      const double e = log2(double(g.cand[c][a]));
+      cost += S[a] * e + double(gamma) * (e - 2.0) * (e - 2.0);
+    }
+    if (cost < best) {
+      second = best;
+      best = cost;
+      bi = c;
+    } else if (cost < second) {
+      second = cost;
+    }
+  }
+  zone_shape[z] = bi;
+  if (zone_margin) zone_margin[z] = float(second - best);
 }
 
 int sm_count() {
@@ -581,7 +595,7 @@ extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void*
     zone_res_kernel<<<g.n_zones, 256, 0, s>>>(g, r, zres);
     if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
   }
-  choose_kernel<<<1, 1024, 0, s>>>(g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio,
+  choose_kernel<<<(g.n_zones + kChooseWarps - 1) / kChooseWarps, 32 * kChooseWarps, 0, s>>>(g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio,
                                    p.gamma, p.gate_max, zone_shape, zone_margin);
   return cuda_status(cudaGetLastError());
 }
@@ -677,7 +691,7 @@ extern "C" prism_status prism_zone_shapes_static(const prism_geometry* geo, cons
     zone_res_kernel<<<g.n_zones, 256, 0, s>>>(g, r, zres);
     if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
   }
-  choose_kernel<<<1, 1024, 0, s>>>(g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio,
+  choose_kernel<<<(g.n_zones + kChooseWarps - 1) / kChooseWarps, 32 * kChooseWarps, 0, s>>>(g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio,
                                    p.gamma, p.gate_max, zone_shape, zone_margin);
   return cuda_status(cudaGetLastError());
 }

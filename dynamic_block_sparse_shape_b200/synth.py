@@ -64,6 +64,11 @@ WORKLOADS = {
     # the 2K grid with 2 heads and Q as the feature input: every attention tensor (151 MB) is still
     # larger than L2, and the whole working set (~1.3 GB) is small enough for profiler captures
     "2k-2h": Workload("2k-2h", (32, 72, 128), 2, 128, "bf16", (8, 8, 8), 4, 0.20, True, "q", False, seed=3),
+    # the 2K grid with the full video features and a2v residual ([N, 3072] bf16 each, as in the 2K
+    # training step) but 2 heads: the zone statistics stream their full 2K inputs while the whole
+    # working set (~4.8 GB) stays small enough for profiler captures of the selection path
+    "2k-stats": Workload("2k-stats", (32, 72, 128), 2, 128, "bf16", (8, 8, 8), 4, 0.20, True, "synthetic", True,
+                         seed=3),
 }
 
 
