@@ -30,6 +30,11 @@ METRIC = "2K block-sparse attn fwd+bwd ms/layer; achieved TFLOP/s vs BF16 tensor
 UNIT = "ms/layer"
 FWD_FLOP_PER_PAIR = 4 * 64 * 64 * 128  # QK^T and PV over one (query block, key block) pair, d = 128
 BWD_FLOP_PER_PAIR = 2.5 * FWD_FLOP_PER_PAIR
+# DRAM bytes (read + write) per selected (query block, key block) pair of the three attention
+# kernels together (forward, dQ, dK/dV), from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum) of the 2-head 2K workload: 96.43 GB over 4,445,104 pairs. Scaled by the
+# selected pairs of the timed workload; the K/V re-reads that miss L2 grow with the pairs.
+ATTN_DRAM_BYTES_PER_PAIR = 96.43e9 / 4445104
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -330,6 +335,24 @@ def cpu_sample(wl, x, feats, res, q_blocks=4, kv_blocks=2, sel_rows=256, users_p
             "wall_s": round(time.time() - t_all, 1), "stage_ms": {k: round(1e3 * v, 1) for k, v in timings.items()}}
 
 
+def selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src):
+    """HBM roofline of the streaming stages: the zone statistics read the features and
+    the a2v residual once, the pooling reads Q and K once (algorithmic bytes)."""
+    hbm = float(peaks.get("hbm_gbs"))
+    q_bytes = wl.n_tokens * wl.heads * wl.head_dim * 2
+    stat_bytes = sum(t.numel() * t.element_size() for t in (feats, res) if t is not None)
+    out = {}
+    for name, nbytes in (("zone_shapes", stat_bytes), ("block_pool", 2 * q_bytes)):
+        ms = stage_ms.get(name)
+        if not ms or not nbytes:
+            continue
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
+                     "peak_source": f"{peak_src} copy bandwidth"}
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -388,9 +411,12 @@ def run_gpu(args):
         "selected_pairs": nnz, "density": round(nnz / (wl.heads * pipe.nb * pipe.nb), 4),
         "stage_ms": {k: round(v, 3) for k, v in stage_ms.items()},
         "roofline": {"bound": "tensor", "kernel": "bsa_fwd + bsa_bwd (dq, dkdv)", "achieved": round(achieved, 1),
-                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": round(nnz * ATTN_DRAM_BYTES_PER_PAIR),
+                     "traffic_source": "ncu dram bytes per selected pair (2-head 2K capture) x selected pairs",
                      "peak_source": f"{peak_src} bf16 sustained",
                      "flop_per_pair": FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR},
+        "roofline_selection_path": selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src),
         "e2e": e2e,
         "gpu_launches": pipe.launches_per_step() * args.steps,
         "clocks": clocks,
