@@ -158,6 +158,8 @@ class Pipeline:
         self.kept = torch.empty((H, self.nb), dtype=torch.int32, device=dev)
         self.row_ptr = torch.empty(H * self.nb + 1, dtype=torch.int32, device=dev)
         self.o = torch.empty_like(x["q"])
+        # rounding residual of the bf16 output, so that the backward's D = dO . O uses O to ~16 bits
+        self.o_lo = torch.empty_like(x["q"]) if x["q"].dtype == torch.bfloat16 else None
         self.lse = torch.empty((H, wl.n_tokens), dtype=torch.float32, device=dev)
         self.grads = tuple(torch.empty_like(x["q"]) for _ in range(3))
         self.zone_shape = torch.empty(self.nz, dtype=torch.int32, device=dev)
@@ -208,12 +210,12 @@ class Pipeline:
     def stage_fwd(self):
         x = self.x
         self.P.bsa_fwd(self.geo, self.zone_shape, x["q"], x["k"], x["v"], self.scale, self.row_ptr, self.col_idx,
-                       ws=self.ws, out=self.o, lse=self.lse)
+                       ws=self.ws, out=self.o, lse=self.lse, o_lo=self.o_lo)
 
     def stage_bwd(self):
         x = self.x
         self.P.bsa_bwd(self.geo, self.zone_shape, x["q"], x["k"], x["v"], self.o, self.lse, x["do"], self.scale,
-                       self.row_ptr, self.col_idx, self.nnz, ws=self.ws, grads=self.grads)
+                       self.row_ptr, self.col_idx, self.nnz, ws=self.ws, grads=self.grads, o_lo=self.o_lo)
 
     STAGES = ("zone_shapes", "block_pool", "block_select", "bsa_fwd", "bsa_bwd")
     # kernels each stage launches (prism kernels only; memsets excluded)

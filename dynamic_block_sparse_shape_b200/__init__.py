@@ -75,9 +75,9 @@ _SIGNATURES = {
                                           ctypes.POINTER(_I64), _P, _SZ, _P]),
     "prism_mask_to_csr": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _I64, _P, _SZ, _P]),
     "prism_bsa_fwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32, _P, _P, _P, _P,
-                                     _P, _SZ, _P]),
-    "prism_bsa_bwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32, _P,
-                                     _P, _I64, _P, _P, _P, _P, _SZ, _P]),
+                                     _P, _P, _SZ, _P]),
+    "prism_bsa_bwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32,
+                                     _P, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
 }
 
 
@@ -281,8 +281,12 @@ def mask_to_csr(mask: torch.Tensor, row_ptr: torch.Tensor, n_blocks: int, col_id
 
 
 def bsa_fwd(geo: Geometry, zone_shape, q, k, v, scale, row_ptr, col_idx, ws: Optional[Workspace] = None,
-            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None):
-    """a6: block-sparse attention forward. Returns (O like q, LSE fp32 [H, N])."""
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None,
+            o_lo: Optional[torch.Tensor] = None):
+    """a6: block-sparse attention forward. Returns (O like q, LSE fp32 [H, N]).
+
+    o_lo (optional, bf16 like a bf16 q): receives the rounding residual of O,
+    to be passed to bsa_bwd so that D = dO . O is formed from O to ~16 bits."""
     N, H, d = q.shape
     assert q.stride(2) == 1 and q.stride(1) == d and k.stride() == q.stride() and v.stride() == q.stride()
     need = workspace_size("bsa_fwd", geo, heads=H, head_dim=d, dtype=q.dtype)
@@ -290,16 +294,21 @@ def bsa_fwd(geo: Geometry, zone_shape, q, k, v, scale, row_ptr, col_idx, ws: Opt
     o = out if out is not None else torch.empty_like(q)
     assert o.stride() == q.stride()
     lse_t = lse if lse is not None else torch.empty((H, N), dtype=torch.float32, device=q.device)
+    if o_lo is not None:
+        assert o_lo.dtype == torch.bfloat16 and o_lo.stride() == q.stride()
     g = geo.c()
     _check(lib().prism_bsa_fwd(ctypes.byref(g), _ptr(zone_shape), _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), H, d,
-                               q.stride(0), float(scale), _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(lse_t), ws.ptr,
-                               ws.nbytes, _stream(stream)), "prism_bsa_fwd")
+                               q.stride(0), float(scale), _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(lse_t),
+                               _ptr(o_lo), ws.ptr, ws.nbytes, _stream(stream)), "prism_bsa_fwd")
     return o, lse_t
 
 
 def bsa_bwd(geo: Geometry, zone_shape, q, k, v, o, lse, do, scale, row_ptr, col_idx, nnz: int,
-            ws: Optional[Workspace] = None, grads: Optional[Sequence[torch.Tensor]] = None, stream=None):
-    """a7: block-sparse attention backward. Returns (dQ, dK, dV) like q."""
+            ws: Optional[Workspace] = None, grads: Optional[Sequence[torch.Tensor]] = None, stream=None,
+            o_lo: Optional[torch.Tensor] = None):
+    """a7: block-sparse attention backward. Returns (dQ, dK, dV) like q.
+
+    o_lo: the forward's rounding residual of O (bsa_fwd's o_lo), or None."""
     N, H, d = q.shape
     for t in (k, v, o, do):
         assert t.stride() == q.stride()
@@ -307,8 +316,10 @@ def bsa_bwd(geo: Geometry, zone_shape, q, k, v, o, lse, do, scale, row_ptr, col_
     ws = (ws or Workspace(q.device)).ensure(need)
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q))
     g = geo.c()
-    _check(lib().prism_bsa_bwd(ctypes.byref(g), _ptr(zone_shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                               _ptr(do), _dtype_code(q), H, d, q.stride(0), float(scale), _ptr(row_ptr),
+    if o_lo is not None:
+        assert o_lo.dtype == torch.bfloat16 and o_lo.stride() == q.stride()
+    _check(lib().prism_bsa_bwd(ctypes.byref(g), _ptr(zone_shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o_lo),
+                               _ptr(lse), _ptr(do), _dtype_code(q), H, d, q.stride(0), float(scale), _ptr(row_ptr),
                                _ptr(col_idx), int(nnz), _ptr(dq), _ptr(dk), _ptr(dv), ws.ptr, ws.nbytes,
                                _stream(stream)), "prism_bsa_bwd")
     return dq, dk, dv

@@ -26,6 +26,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <type_traits>
 
 #include "bsa_common.cuh"
 #include "host.h"
@@ -624,6 +625,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
 // --------------------------------------------------------------------- prep
 template <typename T>
 __device__ __forceinline__ float dot_chunk(const T* a, const T* b, int n);
+
 template <>
 __device__ __forceinline__ float dot_chunk<__nv_bfloat16>(const __nv_bfloat16* a, const __nv_bfloat16* b, int n) {
   float s = 0.f;
@@ -652,7 +654,9 @@ __device__ __forceinline__ float dot_chunk<float>(const float* a, const float* b
 
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const Geo g, const int32_t* __restrict__ zone_shape,
-                                                       const T* __restrict__ o, const T* __restrict__ dout,
+                                                       const T* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ o_lo,
+                                                       const T* __restrict__ dout,
                                                        int64_t tok_stride, int head_dim, const float* __restrict__ lse,
                                                        float* __restrict__ lse2_blk, float* __restrict__ d_blk,
                                                        int* status) {
@@ -663,6 +667,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const Geo g, const int32_
   const int n = head_dim / 4;
   const int64_t off = int64_t(tok) * tok_stride + int64_t(head) * head_dim + part * n;
   float acc = dot_chunk<T>(o + off, dout + off, n);
+  // the forward's rounding residual restores O to about 16 bits before the dot
+  if constexpr (std::is_same_v<T, __nv_bfloat16>) {
+    if (o_lo) acc += dot_chunk<T>(o_lo + off, dout + off, n);
+  }
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   if (part == 0) {
@@ -746,8 +754,9 @@ size_t bsa_bwd_ws_bytes(const Geo& g, int heads, int head_dim, prism_dtype dtype
 using namespace prism;
 
 extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q,
-                                      const void* k, const void* v, const void* o, const float* lse,
-                                      const void* dout, prism_dtype dtype, int32_t heads, int32_t head_dim,
+                                      const void* k, const void* v, const void* o, const void* o_lo,
+                                      const float* lse, const void* dout, prism_dtype dtype, int32_t heads,
+                                      int32_t head_dim,
                                       int64_t tok_stride, float scale, const int32_t* row_ptr,
                                       const int32_t* col_idx, int64_t nnz, void* dq, void* dk, void* dv, void* ws,
                                       size_t ws_bytes, void* stream) {
@@ -762,7 +771,7 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   if (tok_stride < int64_t(heads) * head_dim || tok_stride % 8) return PRISM_ERR_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return PRISM_ERR_ARG;
   if (nnz < 0 || nnz > int64_t(heads) * g.n_blocks * g.n_blocks) return PRISM_ERR_ARG;
-  for (const void* p : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+  for (const void* p : {q, k, v, o, o_lo, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
                         static_cast<const void*>(dv)})
     if (reinterpret_cast<uintptr_t>(p) % 16) return PRISM_ERR_ARG;
   const BwdWs W = bwd_ws_layout(g, heads, head_dim, dtype, nnz);
@@ -795,10 +804,11 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   const dim3 grid(g.n_blocks, heads);
   if (dtype == PRISM_BF16)
     bwd_prep_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g, zone_shape, static_cast<const __nv_bfloat16*>(o),
+                                                        static_cast<const __nv_bfloat16*>(o_lo),
                                                         static_cast<const __nv_bfloat16*>(dout), tok_stride, head_dim,
                                                         lse, lse2, dvec, status);
   else
-    bwd_prep_kernel<float><<<grid, 256, 0, s>>>(g, zone_shape, static_cast<const float*>(o),
+    bwd_prep_kernel<float><<<grid, 256, 0, s>>>(g, zone_shape, static_cast<const float*>(o), nullptr,
                                                 static_cast<const float*>(dout), tok_stride, head_dim, lse, lse2,
                                                 dvec, status);
   const int rows = heads * g.n_blocks;

@@ -64,6 +64,7 @@ struct FwdParams {
   const int32_t* col_idx;
   void* o;
   float* lse;
+  __nv_bfloat16* o_lo;  // rounding residual of a bf16 o, or null
   int* status;
   int64_t tok_stride;  // of o, elements
   float scale_log2;
@@ -407,6 +408,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       for (int i = 0; i < NC; ++i) ov[i] = 0.f;
     }
     store_row<NC>(P.o, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, ov, P.out_fp32);
+    if (P.o_lo) {
+      // what the bf16 store of O dropped: O = o + o_lo to about 16 bits
+      float lo[NC];
+#pragma unroll
+      for (int i = 0; i < NC; ++i) lo[i] = ov[i] - __bfloat162float(__float2bfloat16_rn(ov[i]));
+      store_row<NC>(P.o_lo, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, lo, false);
+    }
     if (q4 == 0) {
       const int N = g.T * g.H * g.W;
       P.lse[int64_t(head) * N + tok] = (l > 0.f && ok) ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -458,8 +466,8 @@ using namespace prism;
 extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q,
                                       const void* k, const void* v, prism_dtype dtype, int32_t heads,
                                       int32_t head_dim, int64_t tok_stride, float scale, const int32_t* row_ptr,
-                                      const int32_t* col_idx, void* o, float* lse, void* ws, size_t ws_bytes,
-                                      void* stream) {
+                                      const int32_t* col_idx, void* o, float* lse, void* o_lo, void* ws,
+                                      size_t ws_bytes, void* stream) {
   Geo g;
   prism_status st = make_geo(geo, &g);
   if (st != PRISM_OK) return st;
@@ -469,7 +477,7 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
   if (heads < 1 || heads > 65535) return PRISM_ERR_UNSUPPORTED;
   if (tok_stride < int64_t(heads) * head_dim || tok_stride % 8) return PRISM_ERR_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return PRISM_ERR_ARG;
-  for (const void* p : {q, k, v, static_cast<const void*>(o)})
+  for (const void* p : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(o_lo)})
     if (reinterpret_cast<uintptr_t>(p) % 16) return PRISM_ERR_ARG;
   const size_t need = bsa_fwd_ws_bytes(g, heads, head_dim, dtype);
   if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < need) return PRISM_ERR_WORKSPACE;
@@ -506,6 +514,7 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
   P.col_idx = col_idx;
   P.o = o;
   P.lse = lse;
+  P.o_lo = dtype == PRISM_BF16 ? static_cast<__nv_bfloat16*>(o_lo) : nullptr;
   P.status = ws_status(ws);
   P.tok_stride = tok_stride;
   P.scale_log2 = scale * 1.4426950408889634f;

@@ -258,11 +258,18 @@ PRISM_API prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* ro
  *       give O = 0 and lse = -inf).
  * o: device [N, heads, head_dim] out, same dtype as q, token stride tok_stride.
  * lse: device float [heads, N] out.
+ * o_lo: optional device bf16 [N, heads, head_dim] out (token stride
+ *       tok_stride), or NULL: the rounding residual of the bf16 output,
+ *       O_fp32 - bf16(O_fp32), so that O_fp32 = o + o_lo to about 16 bits.
+ *       Passing it to prism_bsa_bwd makes D_i = dO_i . O_i exact to that
+ *       precision; with a nearly one-hot softmax, dS = P (dP - D) cancels
+ *       and bf16 rounding of O alone would dominate dQ and dK. Ignored (may be
+ *       NULL) for fp32 outputs, which carry no rounding.
  */
 PRISM_API prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
                            const void* v, prism_dtype dtype, int32_t heads, int32_t head_dim, int64_t tok_stride,
                            float scale, const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
-                           void* ws, size_t ws_bytes, void* stream);
+                           void* o_lo, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * a7 — block-sparse attention backward (Prism trains natively with the
@@ -270,12 +277,14 @@ PRISM_API prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* z
  * D_i = sum_c dO_ic O_ic; P_ij = exp(scale q_i.k_j - lse_i) on the selected
  * blocks; dV_j = sum_i P_ij dO_i; dS_ij = P_ij (dO_i . v_j - D_i);
  * dQ_i = scale sum_j dS_ij k_j; dK_j = scale sum_i dS_ij q_i.
- * Arguments as prism_bsa_fwd; o and lse are the forward's outputs; dout is
- * device [N, heads, head_dim]; dq, dk, dv are device outs like q. nnz =
+ * Arguments as prism_bsa_fwd; o, o_lo (or NULL) and lse are the forward's
+ * outputs (with o_lo, D_i = dO_i . (O_i + O_lo_i)); dout is device
+ * [N, heads, head_dim]; dq, dk, dv are device outs like q. nnz =
  * row_ptr[heads*n_blocks] (for workspace sizing; checked against ws_bytes).
  */
 PRISM_API prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
-                           const void* v, const void* o, const float* lse, const void* dout, prism_dtype dtype,
+                           const void* v, const void* o, const void* o_lo, const float* lse, const void* dout,
+                           prism_dtype dtype,
                            int32_t heads, int32_t head_dim, int64_t tok_stride, float scale, const int32_t* row_ptr,
                            const int32_t* col_idx, int64_t nnz, void* dq, void* dk, void* dv, void* ws,
                            size_t ws_bytes, void* stream);

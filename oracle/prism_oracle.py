@@ -339,8 +339,20 @@ def masked_attention_bwd(Q, K, V, O, lse, dO, allowed, scale):
 # Sampled rows for large grids: the same sums restricted to the unmasked
 # columns (masked terms are exactly zero, so this equals the masked form).
 # --------------------------------------------------------------------------
-def attention_block_rows(Q, K, V, blocks, kept_blocks, h, I, scale, dO=None):
-    """O, LSE (and dQ, D when dO is given) for the 64 query tokens of block I of head h."""
+# Unit roundoff of bf16 (8 significant bits, round to nearest).
+BF16_U = 2.0 ** -8
+
+
+def attention_block_rows(Q, K, V, blocks, kept_blocks, h, I, scale, dO=None, bf16_bound=False):
+    """O, LSE (and dQ, D when dO is given) for the 64 query tokens of block I of head h.
+
+    With ``bf16_bound``, also the elementwise worst-case effect of the bf16
+    roundings a bf16 tensor-core implementation performs on top of exact
+    arithmetic: P rounded for the P V product and O rounded when stored
+    (``O_bound``); D formed from that computed O (``D_bound``), which enters
+    dS = P (dP - D); dS rounded for the dS K product and dQ rounded when
+    stored (``dQ_bound``). First order in the unit roundoff; a tolerance
+    model, not a reference value."""
     qi = blocks[I]
     kj = blocks[np.asarray(kept_blocks)].reshape(-1)
     q = np.asarray(Q[qi, h], np.float64)
@@ -353,6 +365,8 @@ def attention_block_rows(Q, K, V, blocks, kept_blocks, h, I, scale, dO=None):
     O = (P / l) @ v
     lse = (mx + np.log(l))[:, 0]
     out = {"O": O, "lse": lse, "tokens": qi}
+    if bf16_bound:
+        out["O_bound"] = BF16_U * ((P / l) @ np.abs(v) + np.abs(O))
     if dO is not None:
         do = np.asarray(dO[qi, h], np.float64)
         Pn = P / l
@@ -361,21 +375,32 @@ def attention_block_rows(Q, K, V, blocks, kept_blocks, h, I, scale, dO=None):
         dS = Pn * (dP - D[:, None])
         out["dQ"] = scale * dS @ k
         out["D"] = D
+        if bf16_bound:
+            bD = BF16_U * (np.abs(do) * (Pn @ np.abs(v))).sum(axis=1)
+            out["D_bound"] = bD
+            out["dQ_bound"] = (BF16_U * (scale * np.abs(dS) @ np.abs(k) + np.abs(out["dQ"])) +
+                               scale * bD[:, None] * (Pn @ np.abs(k)))
     return out
 
 
-def attention_kv_block_grads(Q, K, V, dO, blocks, sel_mask_h, h, J, scale, row_cache=None):
+def attention_kv_block_grads(Q, K, V, dO, blocks, sel_mask_h, h, J, scale, row_cache=None, bf16_bound=False):
     """dK, dV for the 64 key tokens of block J of head h.
 
     ``sel_mask_h`` [nb, nb] is the head's block mask; every query block I that
     selected J contributes, with its own LSE and D = rowsum(dO * O) computed
-    from its full selected set.
+    from its full selected set. With ``bf16_bound`` the result is
+    (dK, dV, dK_bound, dV_bound): the worst-case effect of rounding P^T and
+    dS^T to bf16 for the products and dK, dV when stored (see
+    attention_block_rows).
     """
     kj = blocks[J]
     k = np.asarray(K[kj, h], np.float64)
     v = np.asarray(V[kj, h], np.float64)
     dK = np.zeros_like(k)
     dV = np.zeros_like(v)
+    bK = np.zeros_like(k)
+    bV = np.zeros_like(v)
+    bKD = np.zeros_like(k)  # through D formed from the computed O (already carries the unit roundoff)
     for I in np.nonzero(sel_mask_h[:, J])[0]:
         key = (h, int(I))
         if row_cache is not None and key in row_cache:
@@ -393,4 +418,15 @@ def attention_kv_block_grads(Q, K, V, dO, blocks, sel_mask_h, h, J, scale, row_c
         dP = do @ v.T
         dS = P * (dP - rr["D"][:, None])
         dK += scale * dS.T @ q
+        if bf16_bound:
+            bD = rr["D_bound"] if "D_bound" in rr else BF16_U * (
+                np.abs(do) * ((np.exp(scale * q @ np.asarray(K[blocks[np.nonzero(sel_mask_h[I])[0]].reshape(-1), h],
+                                                               np.float64).T - rr["lse"][:, None]))
+                              @ np.abs(np.asarray(V[blocks[np.nonzero(sel_mask_h[I])[0]].reshape(-1), h],
+                                                  np.float64)))).sum(axis=1)
+            bV += P.T @ np.abs(do)
+            bK += scale * np.abs(dS).T @ np.abs(q)
+            bKD += scale * P.T @ (bD[:, None] * np.abs(q))
+    if bf16_bound:
+        return dK, dV, BF16_U * (bK + np.abs(dK)) + bKD, BF16_U * (bV + np.abs(dV))
     return dK, dV

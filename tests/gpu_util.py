@@ -43,16 +43,31 @@ def csr_from_mask(mask: np.ndarray, device):
             torch.tensor(col if col.size else np.zeros(1), dtype=torch.int32, device=device), int(row_ptr[-1]))
 
 
-def assert_close(name, got, ref, atol_max=ATOL_MAX, atol_mean=ATOL_MEAN):
+def assert_close(name, got, ref, atol_max=ATOL_MAX, atol_mean=ATOL_MEAN, bound=None):
+    """Max-abs and mean-abs error against the fp64 oracle. With ``bound`` (the
+    oracle's elementwise worst-case effect of the bf16 roundings a bf16
+    tensor-core implementation performs), an element may exceed atol_max up to
+    its bound: at unit data scale the bound stays below atol_max, at larger
+    scales (gradients of order 1-10) bf16 rounding alone can exceed it."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
     fin = np.isfinite(ref)
     assert np.array_equal(np.isfinite(got), fin), f"{name}: finiteness differs"
     err = np.abs(got[fin] - ref[fin])
+    if bound is not None and err.size:
+        allowed = np.maximum(atol_max, np.asarray(bound, dtype=np.float64)[fin])
+        worst = float((err / allowed).max())
+        mean = float(err.mean())
+        assert worst <= 1.0 and mean <= atol_mean, (
+            f"{name}: error / max({atol_max}, bf16 bound) {worst:.3f}, mean-abs {mean:.3e}, max-abs {err.max():.3e}")
+        return float(err.max()), mean
     mx = float(err.max()) if err.size else 0.0
     mean = float(err.mean()) if err.size else 0.0
-    assert mx <= atol_max and mean <= atol_mean, f"{name}: max-abs {mx:.3e} mean-abs {mean:.3e}"
+    ref_max = float(np.abs(ref[fin]).max()) if err.size else 0.0
+    ref_rms = float(np.sqrt(np.mean(ref[fin] ** 2))) if err.size else 0.0
+    assert mx <= atol_max and mean <= atol_mean, (
+        f"{name}: max-abs {mx:.3e} mean-abs {mean:.3e} (reference max-abs {ref_max:.3e}, rms {ref_rms:.3e})")
     return mx, mean
 
 

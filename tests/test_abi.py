@@ -92,17 +92,22 @@ def test_host_validation_codes(lib):
     assert pool(ctypes.byref(g), fake, fake, fake, 0, 24, 128, 3000, fake, fake, ws, 256, None) == 1
     # attention: null pointers, bad scale, small workspace
     fwd = lib.prism_bsa_fwd
-    assert fwd(ctypes.byref(g), fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, fake, fake, ws, 256,
-               None) == 1
-    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, -1.0, fake, fake, fake, fake, ws, 256,
-               None) == 1
-    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 1, 24, 128, 3072, 0.088, fake, fake, fake, fake, ws, 256,
-               None) == 4  # fp32 inputs need staging space
+    assert fwd(ctypes.byref(g), fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, fake, fake, None, ws,
+               256, None) == 1
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, -1.0, fake, fake, fake, fake, None, ws,
+               256, None) == 1
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 1, 24, 128, 3072, 0.088, fake, fake, fake, fake, None, ws,
+               256, None) == 4  # fp32 inputs need staging space
+    # the optional output residual must be 16-byte aligned like o
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, fake, fake,
+               ctypes.c_void_p((1 << 20) + 2), ws, 1 << 40, None) == 1
     bwd = lib.prism_bsa_bwd
-    assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, 1000,
-               fake, fake, fake, ws, 256, None) == 4
-    assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, -5,
-               fake, fake, fake, ws, 1 << 40, None) == 1
+    assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake,
+               1000, fake, fake, fake, ws, 256, None) == 4
+    assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake,
+               -5, fake, fake, fake, ws, 1 << 40, None) == 1
+    assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, ctypes.c_void_p((1 << 20) + 2), fake, fake, 0, 24, 128,
+               3072, 0.088, fake, fake, 1000, fake, fake, fake, ws, 1 << 40, None) == 1
     # zone shapes: channels not a multiple of 64, misaligned workspace
     zs = lib.prism_zone_shapes
     assert zs(ctypes.byref(g), fake, 3072, 3000, 0, None, 0, 0, 0, None, fake, None, ws, 1 << 30, None) == 1

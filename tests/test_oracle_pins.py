@@ -374,3 +374,64 @@ def test_empty_selection_row_is_zero_with_no_gradient():
     O2, l2 = O.masked_attention_fwd(Q[keep], K, V, allowed[:, keep], 0.5)
     _, dK2, dV2 = O.masked_attention_bwd(Q[keep], K, V, O2, l2, dO[keep], allowed[:, keep], 0.5)
     assert np.allclose(dK, dK2) and np.allclose(dV, dV2)
+
+
+def test_bf16_rounding_bound_covers_emulated_rounding():
+    """The oracle's bf16 rounding bound holds for an explicit emulation of the
+    roundings (P and dS rounded to bf16 as product operands, O / dQ / dK / dV
+    rounded when stored) on peaked softmax rows, and it is tight enough that
+    dropping one key block of a row breaks it."""
+    import torch
+
+    def bf16(x):
+        return torch.tensor(x, dtype=torch.float64).to(torch.bfloat16).to(torch.float64).numpy()
+
+    rng = np.random.default_rng(23)
+    grid, zone, cand = (4, 8, 8), (4, 8, 8), ((4, 4, 4),)
+    blocks = O.block_tokens(grid, zone, cand, np.zeros(1, dtype=np.int32))
+    nb, N, H, d = blocks.shape[0], 256, 1, 64
+    q = bf16(4.0 * rng.standard_normal((N, H, d)))
+    k = bf16(4.0 * rng.standard_normal((N, H, d)))
+    v = bf16(rng.standard_normal((N, H, d)))
+    do = bf16(rng.standard_normal((N, H, d)))
+    sc = 1.0 / np.sqrt(d)
+    mask = np.ones((nb, nb), dtype=bool)
+    I = 1
+    rr = O.attention_block_rows(q, k, v, blocks, np.arange(nb), 0, I, sc, dO=do, bf16_bound=True)
+    # emulation of the roundings, everything else exact
+    qi, kj = blocks[I], blocks.reshape(-1)
+    S = sc * q[qi, 0] @ k[kj, 0].T
+    P = np.exp(S - S.max(axis=1, keepdims=True))
+    l = P.sum(axis=1, keepdims=True)
+    O_fp = (bf16(P) / l) @ v[kj, 0]  # O with P rounded for the product, before its storage rounding
+    O_em = bf16(O_fp)
+    dP = do[qi, 0] @ v[kj, 0].T
+    D_em = (do[qi, 0] * O_fp).sum(axis=1)  # D from the computed O (stored with its rounding residual)
+    dS = (P / l) * (dP - D_em[:, None])
+    dQ_em = bf16(sc * bf16(dS) @ k[kj, 0])
+    assert (P / l).max(axis=1).mean() > 0.5  # peaked rows
+    for name, em, ref, bound in (("O", O_em, rr["O"], rr["O_bound"]), ("dQ", dQ_em, rr["dQ"], rr["dQ_bound"])):
+        err = np.abs(em - ref)
+        assert np.all(err <= 1.001 * bound + 1e-12), name
+        assert bound.max() < 0.05 * np.abs(ref).max(), name  # not vacuous
+    # a planted error: the same row with its last key block dropped
+    bad = O.attention_block_rows(q, k, v, blocks, np.arange(nb - 1), 0, I, sc, dO=do)
+    assert np.any(np.abs(bad["dQ"] - rr["dQ"]) > rr["dQ_bound"])
+    # dK, dV of one key block over all query blocks
+    J = 2
+    dK, dV, bK, bV = O.attention_kv_block_grads(q, k, v, do, blocks, mask, 0, J, sc, bf16_bound=True)
+    kb = blocks[J]
+    dK_em = np.zeros_like(dK)
+    dV_em = np.zeros_like(dV)
+    for Iq in range(nb):
+        r2 = O.attention_block_rows(q, k, v, blocks, np.arange(nb), 0, Iq, sc, dO=do)
+        qq, dd = q[blocks[Iq], 0], do[blocks[Iq], 0]
+        Sq = sc * qq @ k[kj, 0].T
+        Pr = np.exp(Sq - Sq.max(axis=1, keepdims=True))
+        D_q = (dd * ((bf16(Pr) / Pr.sum(axis=1, keepdims=True)) @ v[kj, 0])).sum(axis=1)
+        Pq = np.exp(sc * qq @ k[kb, 0].T - r2["lse"][:, None])
+        dSq = Pq * (dd @ v[kb, 0].T - D_q[:, None])
+        dV_em += bf16(Pq).T @ dd
+        dK_em += sc * bf16(dSq).T @ qq
+    for name, em, ref, bound in (("dK", bf16(dK_em), dK, bK), ("dV", bf16(dV_em), dV, bV)):
+        assert np.all(np.abs(em - ref) <= 1.001 * bound + 1e-12), name
