@@ -29,7 +29,7 @@ Sources (the method is described in prose only; no formula is printed):
   (thelatestinai.com/papers/2610.05416): dynamic sparse attention computes
   only selected key/value blocks, ranked by a block proxy score.
 
-Where the pages leave a step open, the readings taken here are (R1..R16 in the
+Where the pages leave a step open, the readings taken here are (R1..R21 in the
 design notes):
 
 * zones tile the grid in raster (zt, zh, zw) order; a shape is (bt, bh, bw);
@@ -48,7 +48,10 @@ design notes):
 * m = max(k, min{m : C_m >= tau}), C_m the cumulative softmax mass of the top
   m; k >= n_blocks or tau >= 1 keeps every block (R8, R9);
 * attention is exact softmax attention restricted to the selected blocks,
-  scale 1/sqrt(d); gradients hold the selection fixed.
+  scale 1/sqrt(d); gradients hold the selection fixed;
+* optional scoring bias b_J = beta * mean_J r / mean_grid r added to every
+  logit of key block J (R20); per-head k and tau, and a top-k sparsity ratio
+  rho giving k = max(1, n_b - floor(rho n_b)) (R21).
 
 Parity of the shape rule and of the candidate set with Prism's own code is
 unpinned (the pages print neither); what is pinned is this documented rule.
@@ -259,8 +262,13 @@ def select_row(s, top_k, tau):
     return kept, m, m_star, gap, margin
 
 
-def block_select(qp, kp, scale, top_k, tau, rows=None):
+def block_select(qp, kp, scale, top_k, tau, rows=None, key_bias=None):
     """Selection for every (head, query block) or for ``rows`` = list of (h, I).
+
+    ``top_k`` and ``tau`` are scalars or per-head sequences of length heads
+    (R21: each head keeps its own floor and mass threshold). ``key_bias`` is
+    None or [nb]: b_J added to every head's logit of key block J before the
+    ranking and the softmax (R20, the audio-norm scoring bias).
 
     Returns dict: mask bool [heads, nb, nb] (only selected rows filled when
     ``rows`` is given), kept [heads, nb] (-1 where not computed), gap and
@@ -269,6 +277,9 @@ def block_select(qp, kp, scale, top_k, tau, rows=None):
     qp = np.asarray(qp, np.float64)
     kp = np.asarray(kp, np.float64)
     H, nb, _ = qp.shape
+    ks = np.broadcast_to(np.asarray(top_k, dtype=np.int64), (H,))
+    taus = np.broadcast_to(np.asarray(tau, dtype=np.float64), (H,))
+    bias = np.zeros(nb) if key_bias is None else np.asarray(key_bias, np.float64).reshape(nb)
     mask = np.zeros((H, nb, nb), dtype=bool)
     kept = np.full((H, nb), -1, dtype=np.int64)
     gap = np.full((H, nb), np.nan)
@@ -276,13 +287,48 @@ def block_select(qp, kp, scale, top_k, tau, rows=None):
     if rows is None:
         rows = [(h, i) for h in range(H) for i in range(nb)]
     for h, i in rows:
-        s = scale * (kp[h] @ qp[h, i])
-        idx, m, _, g, mg = select_row(s, top_k, tau)
+        s = scale * (kp[h] @ qp[h, i]) + bias
+        idx, m, _, g, mg = select_row(s, int(ks[h]), float(taus[h]))
         mask[h, i, idx] = True
         kept[h, i] = m
         gap[h, i] = g
         margin[h, i] = mg
     return {"mask": mask, "kept": kept, "gap": gap, "margin": margin}
+
+
+def topk_from_sparsity(rho, n_blocks):
+    """Top-k floor from a top-k sparsity ratio [WT-step, section "实际案例与上手参考":
+    ``BSA_SPARSITY`` switches the block-sparse attention on and sets its top-k
+    sparsity ratio].
+
+    Reading R21: the ratio is the fraction of key blocks the top-k part drops,
+    so k = n_blocks - floor(rho * n_blocks), at least 1. rho is taken as a
+    float32 (the precision the library's argument has) and the product is
+    formed in fp64. 0 <= rho < 1.
+    """
+    rho = float(np.float32(rho))
+    if not (0.0 <= rho < 1.0):
+        raise ValueError("sparsity ratio must lie in [0, 1)")
+    return max(1, int(n_blocks) - int(math.floor(rho * int(n_blocks))))
+
+
+def block_key_bias(R, blocks, beta):
+    """Audio-norm bias of every key block [WT-bridge: the per-token L2 norm of
+    the unscaled a2v residual is the proxy of audio influence, and the walkthrough
+    says it is taken "during BSA scoring"; sounding regions keep more attention].
+
+    Reading R20: b_J = beta * (mean over the 64 tokens n of block J of r(n)) /
+    (mean over all tokens of r(n)), r(n) = ||R[n, :]||_2. The ratio makes the
+    bias independent of the residual's scale; adding b_J to the logits raises
+    the proxy probability of key blocks with a strong audio coupling. A zero
+    residual gives b = 0.
+    """
+    r = token_norms(R)
+    blocks = np.asarray(blocks)
+    mean_grid = r.mean()
+    if mean_grid == 0.0:
+        return np.zeros(blocks.shape[0])
+    return beta * r[blocks].mean(axis=1) / mean_grid
 
 
 # --------------------------------------------------------------------------

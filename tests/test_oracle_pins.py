@@ -261,6 +261,87 @@ def test_default_cdf_threshold_from_the_pages():
     assert float(g["cdf_threshold_default"]) == 0.20
 
 
+def test_topk_from_sparsity_is_the_smallest_count_keeping_the_fraction():
+    """k = the least count >= 1 whose share of the blocks is at least 1 - rho,
+    checked in exact rational arithmetic on the float32 value of rho."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    cases = [(0.0, 10), (0.5, 10), (0.9, 4608), (0.75, 4608), (0.999, 10), (0.1, 10), (0.3, 10)]
+    cases += [(float(rng.uniform(0, 1)), int(rng.integers(1, 6000))) for _ in range(200)]
+    for rho, nb in cases:
+        r32 = Fraction(float(np.float32(rho)))
+        want = next(k for k in range(1, nb + 1) if Fraction(k, nb) >= 1 - r32)
+        assert O.topk_from_sparsity(rho, nb) == want, (rho, nb)
+    assert O.topk_from_sparsity(0.9, 4608) == 461
+    assert O.topk_from_sparsity(0.0, 7) == 7
+    for bad in (-0.1, 1.0, float("nan")):
+        with pytest.raises(ValueError):
+            O.topk_from_sparsity(bad, 10)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_per_head_selection_matches_subset_brute_force(seed):
+    rng = np.random.default_rng(100 + seed)
+    H, nb, d = 3, 8, 4
+    qp, kp = rng.normal(size=(H, nb, d)), rng.normal(0, 1.5, size=(H, nb, d))
+    ks, taus = [1, 3, 2], [0.6, 0.05, 0.35]
+    bias = rng.normal(0, 1.0, nb)
+    for kb in (None, bias):
+        r = O.block_select(qp, kp, 0.5, ks, taus, key_bias=kb)
+        for h in range(H):
+            for i in range(nb):
+                s = 0.5 * np.array([qp[h, i] @ kp[h, j] for j in range(nb)])
+                if kb is not None:
+                    s = s + kb
+                p = np.exp(s - s.max())
+                p /= p.sum()
+                want = _brute_force_selection(p, ks[h], taus[h])
+                assert set(np.nonzero(r["mask"][h, i])[0].tolist()) == want
+
+
+def test_key_bias_closed_form_on_two_blocks():
+    """Grid 4x4x8 in one zone, shape (4,4,4): block 0 holds w < 4, block 1
+    w >= 4. Residual rows c_n e_0 with |c| = 1 in block 0 and 3 in block 1
+    (signs mixed): block means 1 and 3, grid mean 2."""
+    grid, zone = (4, 4, 8), (4, 4, 8)
+    blocks = O.block_tokens(grid, zone, [(4, 4, 4)], [0])
+    N = 128
+    R = np.zeros((N, 5))
+    for n in range(N):
+        w = n % 8
+        R[n, 0] = (1.0 if w < 4 else 3.0) * (-1.0 if n % 3 == 0 else 1.0)
+    b = O.block_key_bias(R, blocks, beta=2.0)
+    assert np.allclose(b, [2.0 * 1 / 2, 2.0 * 3 / 2], rtol=0, atol=1e-15)
+    # norms, not values: spreading the same norm over other channels leaves b unchanged
+    R2 = np.zeros((N, 5))
+    R2[:, 1] = R[:, 0] * 0.6
+    R2[:, 3] = R[:, 0] * 0.8
+    assert np.allclose(O.block_key_bias(R2, blocks, 2.0), b, atol=1e-14)
+    # scale invariance and the zero residual
+    assert np.allclose(O.block_key_bias(7.5 * R, blocks, 2.0), b, atol=1e-14)
+    assert (O.block_key_bias(np.zeros((N, 5)), blocks, 2.0) == 0).all()
+
+
+def test_key_bias_invariants_in_selection():
+    rng = np.random.default_rng(11)
+    H, nb, d = 2, 12, 8
+    qp, kp = rng.normal(size=(H, nb, d)), rng.normal(size=(H, nb, d))
+    sc = 1 / math.sqrt(d)
+    base = O.block_select(qp, kp, sc, 2, 0.3)
+    # a constant bias shifts every logit of a row equally: selection unchanged
+    same = O.block_select(qp, kp, sc, 2, 0.3, key_bias=np.full(nb, 0.8))
+    assert (same["mask"] == base["mask"]).all()
+    # beta = 0: unchanged
+    zero = O.block_select(qp, kp, sc, 2, 0.3, key_bias=np.zeros(nb))
+    assert (zero["mask"] == base["mask"]).all()
+    # one loud block with a large bias is kept by every row
+    kb = np.zeros(nb)
+    kb[5] = 40.0
+    loud = O.block_select(qp, kp, sc, 1, 0.2, key_bias=kb)
+    assert loud["mask"][:, :, 5].all()
+    assert (loud["kept"] == 1).all()
+
+
 # ----------------------------------------------------------------- attention
 def _tiny_problem(seed=0, N=128, H=2, d=16, nblocks=None):
     rng = np.random.default_rng(seed)
