@@ -17,8 +17,8 @@ import torch
 
 __all__ = [
     "PrismError", "Geometry", "ShapeParams", "lib", "library_path", "workspace_size", "Workspace", "zone_shapes",
-    "block_pool", "block_select", "mask_to_csr", "bsa_fwd", "bsa_bwd", "check_device_status", "STATUS", "OP",
-    "DEFAULT_CDF_THRESHOLD",
+    "block_pool", "block_select", "block_select_ex", "topk_from_sparsity", "block_audio_bias", "mask_to_csr",
+    "bsa_fwd", "bsa_bwd", "check_device_status", "STATUS", "OP", "DEFAULT_CDF_THRESHOLD",
 ]
 
 DEFAULT_CDF_THRESHOLD = 0.20
@@ -55,6 +55,12 @@ class _ShapeParams(ctypes.Structure):
     _fields_ = [("w_audio", ctypes.c_float), ("gamma", ctypes.c_float), ("gate_max", ctypes.c_float)]
 
 
+class _SelectParams(ctypes.Structure):
+    _fields_ = [("top_k", ctypes.c_int32), ("cdf_threshold", ctypes.c_float),
+                ("head_top_k", ctypes.POINTER(ctypes.c_int32)), ("head_cdf_threshold", ctypes.POINTER(ctypes.c_float)),
+                ("key_bias", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I32, _I64, _F32, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 _GEO = ctypes.POINTER(_Geometry)
@@ -73,6 +79,10 @@ _SIGNATURES = {
     "prism_block_pool": (ctypes.c_int, [_GEO, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _P, _P, _P, _SZ, _P]),
     "prism_block_select": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, _I32, _F32, _P, _P, _P, _P, _I64,
                                           ctypes.POINTER(_I64), _P, _SZ, _P]),
+    "prism_block_select_ex": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, ctypes.POINTER(_SelectParams), _P, _P,
+                                             _P, _P, _I64, ctypes.POINTER(_I64), _P, _SZ, _P]),
+    "prism_topk_from_sparsity": (ctypes.c_int, [_F32, _I32, ctypes.POINTER(_I32)]),
+    "prism_block_audio_bias": (ctypes.c_int, [_GEO, _P, _P, _I64, _I32, ctypes.c_int, _F32, _P, _P, _SZ, _P]),
     "prism_mask_to_csr": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _I64, _P, _SZ, _P]),
     "prism_bsa_fwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32, _P, _P, _P, _P,
                                      _P, _P, _SZ, _P]),
@@ -267,6 +277,73 @@ def block_select(qp: torch.Tensor, kp: torch.Tensor, scale: float, top_k: int,
         col = torch.empty(max(1, total.value), dtype=torch.int32, device=dev)
         mask_to_csr(mask, row_ptr, nb, col, ws=ws, stream=stream)
         out["col_idx"] = col[:total.value]
+    return out
+
+
+def block_select_ex(qp: torch.Tensor, kp: torch.Tensor, scale: float, top_k,
+                    cdf_threshold=DEFAULT_CDF_THRESHOLD, key_bias: Optional[torch.Tensor] = None,
+                    ws: Optional[Workspace] = None, csr: bool = True, stream=None):
+    """a4+a5 with per-head settings: ``top_k`` and ``cdf_threshold`` are scalars
+    or sequences of one value per head; ``key_bias`` is None or a device fp32
+    [n_blocks] added to every head's logit of each key block (for example from
+    ``block_audio_bias``). Returns the same dict as ``block_select``."""
+    H, nb, d = qp.shape
+    words = (nb + 31) // 32
+    dev = qp.device
+    ws = (ws or Workspace(dev)).ensure(256)
+    cp = _SelectParams()
+    keep = []
+    if isinstance(top_k, (int,)) or (torch.is_tensor(top_k) and top_k.dim() == 0):
+        cp.top_k = int(top_k)
+    else:
+        arr = (ctypes.c_int32 * H)(*[int(x) for x in top_k])
+        keep.append(arr)
+        cp.top_k = int(arr[0]) if H else 1
+        cp.head_top_k = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+    if isinstance(cdf_threshold, (int, float)) or (torch.is_tensor(cdf_threshold) and cdf_threshold.dim() == 0):
+        cp.cdf_threshold = float(cdf_threshold)
+    else:
+        arr = (ctypes.c_float * H)(*[float(x) for x in cdf_threshold])
+        keep.append(arr)
+        cp.cdf_threshold = float(arr[0]) if H else 0.0
+        cp.head_cdf_threshold = ctypes.cast(arr, ctypes.POINTER(ctypes.c_float))
+    if key_bias is not None:
+        assert key_bias.dtype == torch.float32 and key_bias.numel() == nb and key_bias.is_contiguous()
+        cp.key_bias = key_bias.data_ptr()
+    mask = torch.empty((H, nb, words), dtype=torch.int32, device=dev)
+    kept = torch.empty((H, nb), dtype=torch.int32, device=dev)
+    row_ptr = torch.empty(H * nb + 1, dtype=torch.int32, device=dev)
+    total = _I64()
+    _check(lib().prism_block_select_ex(_ptr(qp), _ptr(kp), H, nb, d, float(scale), ctypes.byref(cp), _ptr(mask),
+                                       _ptr(kept), _ptr(row_ptr), None, 0, ctypes.byref(total), ws.ptr, ws.nbytes,
+                                       _stream(stream)), "prism_block_select_ex")
+    out = {"mask": mask, "kept": kept, "row_ptr": row_ptr, "total": int(total.value), "col_idx": None}
+    if csr:
+        col = torch.empty(max(1, total.value), dtype=torch.int32, device=dev)
+        mask_to_csr(mask, row_ptr, nb, col, ws=ws, stream=stream)
+        out["col_idx"] = col[:total.value]
+    return out
+
+
+def topk_from_sparsity(sparsity: float, n_blocks: int) -> int:
+    """Top-k floor for a top-k sparsity ratio: n_blocks - floor(sparsity * n_blocks), at least 1."""
+    k = _I32()
+    _check(lib().prism_topk_from_sparsity(float(sparsity), int(n_blocks), ctypes.byref(k)), "prism_topk_from_sparsity")
+    return int(k.value)
+
+
+def block_audio_bias(geo: Geometry, zone_shape: torch.Tensor, res: torch.Tensor, beta: float,
+                     ws: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """Audio-norm bias of every key block, device fp32 [n_blocks]:
+    beta * (block mean of ||res[n]||) / (grid mean of ||res[n]||)."""
+    _, nb = geo.counts()
+    assert res.dim() == 2 and res.stride(1) == 1
+    ws = (ws or Workspace(res.device)).ensure(256)
+    out = torch.empty(nb, dtype=torch.float32, device=res.device)
+    g = geo.c()
+    _check(lib().prism_block_audio_bias(ctypes.byref(g), _ptr(zone_shape), _ptr(res), res.stride(0), res.shape[1],
+                                        _dtype_code(res), float(beta), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)),
+           "prism_block_audio_bias")
     return out
 
 

@@ -8,18 +8,22 @@
 // overhead, so the scores here live only in shared memory.
 //
 // select_kernel: one CTA = 8 query blocks of one head (one warp each).
-//   1. logits s_J = scale * qbar_I . kbar_J for all J, fp32 FFMA, with the
-//      key features staged transposed in shared memory (2 keys x 4 rows per
-//      thread per channel);
+//   1. logits s_J = scale * qbar_I . kbar_J (+ b_J, the optional key-block
+//      bias, walkthrough section "桥接残差反哺稀疏注意力") for all J, fp32 FFMA,
+//      with the key features staged transposed in shared memory (2 keys x 4
+//      rows per thread per channel);
 //   2. per row: max, p_J = exp(s_J - max) in place, Z = sum p (fp64);
 //   3. the mass threshold: bisection on the float bits of p for
 //      u* = max{u : sum_{key_J >= u} p_J >= tau * Z}; ties at u* are taken in
 //      ascending J until the mass is reached -> m*;
 //   4. m = max(k, m*); if m > m*, a bisection on counts finds the m-th key;
+//      k and tau are the row's head's (per-head settings, walkthrough section
+//      "实际案例与上手参考": the top-k part of the selection is a tunable ratio);
 //   5. the kept set (ranked by p descending, ties to the lower J) is written
 //      as a bitmask row with warp ballots, and kept[row] = m.
 // scan_kernel: exclusive scan of kept into the CSR row_ptr (one CTA).
 // fill_kernel: one warp per row expands the bitmask into ascending col_idx.
+#include <algorithm>
 #include <cfloat>
 #include <cmath>
 
@@ -34,6 +38,16 @@ constexpr int kKeyTile = 256;
 constexpr int kDChunk = 32;
 constexpr int kKtPitch = kKeyTile + 2;
 constexpr int kSelMaxBlocks = 5120;
+constexpr int kSelMaxHeads = 128;  // per-head settings passed as a kernel parameter
+
+// Per-head floor k and mass threshold tau (uniform when per_head == 0).
+struct SelHeads {
+  int per_head;
+  int k0;
+  float tau0;
+  int k[kSelMaxHeads];
+  float tau[kSelMaxHeads];
+};
 
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
@@ -62,8 +76,9 @@ __device__ __forceinline__ int count_at_least(const float* p, int nb, uint32_t u
 }
 
 __global__ void __launch_bounds__(kSelThreads, 1)
-    select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int nb, int d, float scale, int top_k,
-                  float tau, uint32_t* __restrict__ mask, int32_t* __restrict__ kept) {
+    select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int nb, int d, float scale,
+                  const __grid_constant__ SelHeads hp, const float* __restrict__ kbias, uint32_t* __restrict__ mask,
+                  int32_t* __restrict__ kept) {
   extern __shared__ __align__(16) float sm[];
   float* srow = sm;                                  // [kSelRows][nb]
   float* kT = srow + size_t(kSelRows) * nb;          // [kDChunk][kKtPitch]
@@ -109,13 +124,15 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int key = key0 + 2 * kpair + j;
-        if (key < nb) srow[size_t(4 * rh + i) * nb + key] = acc[i][j] * scale;
+        if (key < nb) srow[size_t(4 * rh + i) * nb + key] = acc[i][j] * scale + (kbias ? __ldg(kbias + key) : 0.f);
       }
   }
   __syncthreads();
   // ---- 2..5. one warp per query block
   const int I = I0 + warp;
   if (I >= nb) return;
+  const int top_k = hp.per_head ? hp.k[head] : hp.k0;
+  const float tau = hp.per_head ? hp.tau[head] : hp.tau0;
   float* p = srow + size_t(warp) * nb;
   const int words = (nb + 31) >> 5;
   uint32_t* mrow = mask + (size_t(head) * nb + I) * words;
@@ -288,18 +305,20 @@ cudaError_t launch_mask_to_lists(const uint32_t* mask, const int32_t* row_ptr, i
 
 using namespace prism;
 
-extern "C" prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
-                                           int32_t head_dim, float scale, int32_t top_k, float cdf_threshold,
-                                           uint32_t* mask, int32_t* kept, int32_t* row_ptr, int32_t* col_idx,
-                                           int64_t col_cap, int64_t* total_kept, void* ws, size_t ws_bytes,
-                                           void* stream) {
+namespace {
+
+prism_status block_select_impl(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
+                               int32_t head_dim, float scale, const SelHeads& hp, const float* key_bias,
+                               uint32_t* mask, int32_t* kept, int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
+                               int64_t* total_kept, void* ws, size_t ws_bytes, void* stream) {
   if (!q_pool || !k_pool || !mask || !kept || !row_ptr) return PRISM_ERR_ARG;
-  if (heads < 1 || n_blocks < 1 || top_k < 1) return PRISM_ERR_ARG;
-  if (!(cdf_threshold >= 0.f) || !(scale > 0.f) || !std::isfinite(scale)) return PRISM_ERR_ARG;
+  if (heads < 1 || n_blocks < 1) return PRISM_ERR_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return PRISM_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return PRISM_ERR_UNSUPPORTED;
   if (n_blocks > kSelMaxBlocks) return PRISM_ERR_UNSUPPORTED;
   if (int64_t(heads) * n_blocks * n_blocks >= (int64_t(1) << 31)) return PRISM_ERR_UNSUPPORTED;
   if (reinterpret_cast<uintptr_t>(q_pool) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16) return PRISM_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(key_bias) % 4) return PRISM_ERR_ARG;
   if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
   if (col_idx && col_cap < 0) return PRISM_ERR_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -307,8 +326,7 @@ extern "C" prism_status prism_block_select(const float* q_pool, const float* k_p
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return PRISM_ERR_CUDA;
   const dim3 grid((n_blocks + kSelRows - 1) / kSelRows, heads);
-  select_kernel<<<grid, kSelThreads, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, top_k, cdf_threshold, mask,
-                                                kept);
+  select_kernel<<<grid, kSelThreads, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, hp, key_bias, mask, kept);
   const int rows = heads * n_blocks;
   if (launch_exclusive_scan(kept, rows, row_ptr, s) != cudaSuccess) return PRISM_ERR_CUDA;
   if (total_kept) {
@@ -324,6 +342,54 @@ extern "C" prism_status prism_block_select(const float* q_pool, const float* k_p
       return PRISM_ERR_CUDA;
   }
   return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
+                                           int32_t head_dim, float scale, int32_t top_k, float cdf_threshold,
+                                           uint32_t* mask, int32_t* kept, int32_t* row_ptr, int32_t* col_idx,
+                                           int64_t col_cap, int64_t* total_kept, void* ws, size_t ws_bytes,
+                                           void* stream) {
+  if (top_k < 1 || !(cdf_threshold >= 0.f)) return PRISM_ERR_ARG;
+  SelHeads hp{};
+  hp.per_head = 0;
+  hp.k0 = top_k;
+  hp.tau0 = cdf_threshold;
+  return block_select_impl(q_pool, k_pool, heads, n_blocks, head_dim, scale, hp, nullptr, mask, kept, row_ptr,
+                           col_idx, col_cap, total_kept, ws, ws_bytes, stream);
+}
+
+extern "C" prism_status prism_block_select_ex(const float* q_pool, const float* k_pool, int32_t heads,
+                                              int32_t n_blocks, int32_t head_dim, float scale,
+                                              const prism_select_params* params, uint32_t* mask, int32_t* kept,
+                                              int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
+                                              int64_t* total_kept, void* ws, size_t ws_bytes, void* stream) {
+  if (!params || heads < 1) return PRISM_ERR_ARG;
+  SelHeads hp{};
+  hp.k0 = params->top_k;
+  hp.tau0 = params->cdf_threshold;
+  const bool per_head = params->head_top_k || params->head_cdf_threshold;
+  if (per_head) {
+    if (heads > kSelMaxHeads) return PRISM_ERR_UNSUPPORTED;
+    hp.per_head = 1;
+    for (int h = 0; h < heads; ++h) {
+      hp.k[h] = params->head_top_k ? params->head_top_k[h] : params->top_k;
+      hp.tau[h] = params->head_cdf_threshold ? params->head_cdf_threshold[h] : params->cdf_threshold;
+      if (hp.k[h] < 1 || !(hp.tau[h] >= 0.f)) return PRISM_ERR_ARG;
+    }
+  } else if (hp.k0 < 1 || !(hp.tau0 >= 0.f)) {
+    return PRISM_ERR_ARG;
+  }
+  return block_select_impl(q_pool, k_pool, heads, n_blocks, head_dim, scale, hp, params->key_bias, mask, kept,
+                           row_ptr, col_idx, col_cap, total_kept, ws, ws_bytes, stream);
+}
+
+extern "C" prism_status prism_topk_from_sparsity(float sparsity, int32_t n_blocks, int32_t* top_k) {
+  if (!top_k || n_blocks < 1 || !(sparsity >= 0.f) || !(sparsity < 1.f)) return PRISM_ERR_ARG;
+  const int64_t dropped = int64_t(std::floor(double(sparsity) * double(n_blocks)));
+  *top_k = int32_t(std::max<int64_t>(1, int64_t(n_blocks) - dropped));
+  return PRISM_OK;
 }
 
 extern "C" prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* row_ptr, int32_t rows,

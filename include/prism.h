@@ -232,6 +232,76 @@ PRISM_API prism_status prism_block_select(const float* q_pool, const float* k_po
                                 int32_t* kept, int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
                                 int64_t* total_kept, void* ws, size_t ws_bytes, void* stream);
 
+/* Per-call selection settings of prism_block_select_ex. */
+typedef struct {
+  int32_t top_k;                   /* k of every head when head_top_k is NULL (>= 1) */
+  float cdf_threshold;             /* tau of every head when head_cdf_threshold is NULL (>= 0) */
+  const int32_t* head_top_k;       /* host int32 [heads] (each >= 1), or NULL */
+  const float* head_cdf_threshold; /* host float [heads] (each >= 0), or NULL */
+  const float* key_bias;           /* device float [n_blocks], or NULL: b_J added to s_J */
+} prism_select_params;
+
+/*
+ * a4 + a5 with per-head settings and an optional key-block scoring bias.
+ *
+ * Per-head k and tau: the walkthrough (wmrh.cn/news/72296) section
+ * "实际案例与上手参考" exposes the selection as a tunable knob
+ * (BSA_SPARSITY, a top-k sparsity ratio); this entry point lets every head
+ * carry its own floor k_h and mass threshold tau_h. Scoring bias: the same
+ * walkthrough, section "桥接残差反哺稀疏注意力", says the per-token norm of the
+ * a2v residual is read when BSA scores blocks and that sounding regions keep
+ * more attention; with key_bias (e.g. from prism_block_audio_bias) the logits
+ * become s_J = scale * q_pool[h,I] . k_pool[h,J] + b_J for every head before
+ * the ranking and the softmax. Otherwise the rule, outputs and their layout
+ * are those of prism_block_select, with k = k_h and tau = tau_h in row (h, I).
+ * With head_top_k = head_cdf_threshold = key_bias = NULL the result is
+ * identical to prism_block_select(top_k, cdf_threshold).
+ *
+ * params: host, required. Per-head arrays need heads <= 128
+ *       (PRISM_ERR_UNSUPPORTED above); any k < 1 or tau < 0 (or NaN) returns
+ *       PRISM_ERR_ARG before any work is enqueued. key_bias must be 4-byte
+ *       aligned; a NaN entry gives its key block no mass.
+ */
+PRISM_API prism_status prism_block_select_ex(const float* q_pool, const float* k_pool, int32_t heads,
+                                             int32_t n_blocks, int32_t head_dim, float scale,
+                                             const prism_select_params* params, uint32_t* mask, int32_t* kept,
+                                             int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
+                                             int64_t* total_kept, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Top-k floor from a top-k sparsity ratio (walkthrough section
+ * "实际案例与上手参考": BSA_SPARSITY sets the top-k sparsity ratio). The library's
+ * reading: the ratio is the fraction of key blocks the top-k part drops, so
+ * k = n_blocks - floor(sparsity * n_blocks) with the product formed in double
+ * from the float argument, at least 1; that is the smallest count that keeps
+ * at least the fraction 1 - sparsity of the blocks. Host only.
+ * sparsity in [0, 1), n_blocks >= 1, top_k: host out. PRISM_ERR_ARG otherwise.
+ */
+PRISM_API prism_status prism_topk_from_sparsity(float sparsity, int32_t n_blocks, int32_t* top_k);
+
+/*
+ * Audio-norm bias of every key block, for prism_block_select_ex (walkthrough
+ * section "桥接残差反哺稀疏注意力": the per-token L2 norm of the unscaled a2v
+ * residual is the proxy of how strongly audio drives a visual region, read
+ * when BSA scores blocks; sounding regions keep more attention). The library's
+ * reading: b_J = beta * mean_{n in block J} r(n) / mean_{all n} r(n),
+ * r(n) = ||res[n, :]||_2 (fp32 per token, fp64 grid mean). The ratio makes
+ * the bias independent of the residual's scale; a zero residual gives b = 0.
+ *
+ * zone_shape: device int32 [n_zones] (from prism_zone_shapes); the blocks are
+ *       those of prism_block_pool.
+ * res: device [N, res_c] (bf16 or fp32), row stride res_ld elements (a
+ *       multiple of 8), res_c a positive multiple of 8, 16-byte aligned.
+ * beta: finite scale of the bias (0 gives b = 0).
+ * key_bias: device float [n_blocks] out.
+ * ws: at least prism_workspace_size(PRISM_OP_BLOCK_SELECT, ...) bytes; only
+ *       its status word is used (an out-of-range zone_shape entry leaves the
+ *       whole bias NaN and reports PRISM_ERR_DEVICE).
+ */
+PRISM_API prism_status prism_block_audio_bias(const prism_geometry* geo, const int32_t* zone_shape, const void* res,
+                                              int64_t res_ld, int32_t res_c, prism_dtype res_dtype, float beta,
+                                              float* key_bias, void* ws, size_t ws_bytes, void* stream);
+
 /*
  * Expands a selection bitmask (as written by prism_block_select) into the
  * CSR column lists: col_idx[row_ptr[r] .. row_ptr[r+1]) = the set bits of row

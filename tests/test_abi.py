@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import dynamic_block_sparse_shape_b200 as P
@@ -115,6 +116,54 @@ def test_host_validation_codes(lib):
               1 << 30, None) == 4
     # mask_to_csr
     assert lib.prism_mask_to_csr(fake, fake, 0, 10, fake, 10, ws, 256, None) == 1
+
+
+def test_select_ex_and_audio_bias_validation(lib):
+    g = _geo().c()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    ws = ctypes.c_void_p(1 << 24)
+    SP = P._SelectParams
+    sel = lib.prism_block_select_ex
+
+    def call(params, heads=24, nb=4608, d=128, w=ws):
+        return sel(fake, fake, heads, nb, d, 0.088, params, fake, fake, fake, None, 0, None, w, 256, None)
+
+    assert call(None) == 1
+    assert call(ctypes.byref(SP(0, 0.2))) == 1                       # k < 1
+    assert call(ctypes.byref(SP(4, float("nan")))) == 1              # tau NaN
+    ks = (ctypes.c_int32 * 24)(*([4] * 23 + [0]))                    # one head with k = 0
+    assert call(ctypes.byref(SP(4, 0.2, ctypes.cast(ks, ctypes.POINTER(ctypes.c_int32))))) == 1
+    taus = (ctypes.c_float * 24)(*([0.2] * 23 + [-1.0]))             # one head with tau < 0
+    assert call(ctypes.byref(SP(4, 0.2, None, ctypes.cast(taus, ctypes.POINTER(ctypes.c_float))))) == 1
+    many = (ctypes.c_int32 * 129)(*([4] * 129))                      # per-head arrays need heads <= 128
+    assert call(ctypes.byref(SP(4, 0.2, ctypes.cast(many, ctypes.POINTER(ctypes.c_int32)))), heads=129, nb=64) == 9
+    good = SP(4, 0.2, ctypes.cast(ks, ctypes.POINTER(ctypes.c_int32)))
+    ks[23] = 4
+    assert call(ctypes.byref(good), d=96) == 9
+    assert call(ctypes.byref(good), w=None) == 4
+    assert call(ctypes.byref(SP(4, 0.2, None, None, (1 << 20) + 2))) == 1  # misaligned key_bias
+    bias = lib.prism_block_audio_bias
+    assert bias(ctypes.byref(g), fake, None, 3072, 3072, 0, 1.0, fake, ws, 256, None) == 1
+    assert bias(ctypes.byref(g), fake, fake, 3072, 3072, 5, 1.0, fake, ws, 256, None) == 3
+    assert bias(ctypes.byref(g), fake, fake, 3072, 3070, 0, 1.0, fake, ws, 256, None) == 1
+    assert bias(ctypes.byref(g), fake, fake, 3000, 3072, 0, 1.0, fake, ws, 256, None) == 1
+    assert bias(ctypes.byref(g), fake, fake, 3072, 3072, 0, float("inf"), fake, ws, 256, None) == 1
+    assert bias(ctypes.byref(g), fake, fake, 3072, 3072, 0, 1.0, fake, None, 256, None) == 4
+
+
+def test_topk_from_sparsity_matches_oracle(lib):
+    """Host logic of the ratio form of top-k, against the oracle's rule."""
+    from oracle import prism_oracle as O
+    rng = np.random.default_rng(7)
+    cases = [(0.0, 1), (0.0, 4608), (0.9, 4608), (0.75, 4608), (0.5, 10), (0.3, 10), (0.999, 3)]
+    cases += [(float(rng.uniform(0, 1)), int(rng.integers(1, 6000))) for _ in range(500)]
+    k = ctypes.c_int32()
+    for rho, nb in cases:
+        assert lib.prism_topk_from_sparsity(rho, nb, ctypes.byref(k)) == 0
+        assert k.value == O.topk_from_sparsity(rho, nb), (rho, nb)
+    for rho, nb in ((-0.1, 10), (1.0, 10), (float("nan"), 10), (0.5, 0)):
+        assert lib.prism_topk_from_sparsity(rho, nb, ctypes.byref(k)) == 1
+    assert lib.prism_topk_from_sparsity(0.5, 10, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

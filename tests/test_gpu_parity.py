@@ -217,20 +217,30 @@ def test_block_pool_all_shapes(dtype):
 
 
 # --------------------------------------------------------------------------- selection
-def _selection_parity(qp, kp, sc, top_k, tau):
-    sel = P.block_select(qp, kp, sc, top_k, tau)
+def _selection_parity(qp, kp, sc, top_k, tau, qpr, kpr, key_bias=None, key_bias_r=None):
+    """GPU selection on (qp, kp[, key_bias]) against the oracle's selection on
+    its own fp64 inputs (qpr, kpr[, key_bias_r]). top_k / tau are scalars (the
+    plain entry point) or per-head lists (the _ex entry point)."""
     H, nb, _ = qp.shape
-    ref = O.block_select(f64(qp), f64(kp), sc, top_k, tau)
+    per_head = not np.isscalar(top_k) or not np.isscalar(tau)
+    if per_head or key_bias is not None:
+        sel = P.block_select_ex(qp, kp, sc, top_k, tau, key_bias=key_bias)
+    else:
+        sel = P.block_select(qp, kp, sc, top_k, tau)
+    ref = O.block_select(qpr, kpr, sc, top_k, tau, key_bias=key_bias_r)
     got = mask_bits_to_bool(sel["mask"], nb)
     kept = sel["kept"].cpu().numpy()
     qual = (ref["gap"] > LOGIT_GAP) & (ref["margin"] > CDF_MARGIN)
     assert np.array_equal(got[qual], ref["mask"][qual])
     assert np.array_equal(kept[qual], ref["kept"][qual])
-    # every row: kept >= k, popcount == kept, and any difference from the
-    # oracle lies among blocks whose logits are within LOGIT_GAP of the boundary
-    assert np.all(kept >= min(top_k, nb))
+    # every row: kept >= its head's k, popcount == kept, and any difference from
+    # the oracle lies among blocks whose logits are within 5e-2 of the boundary
+    ks = np.broadcast_to(np.asarray(top_k), (H,))
+    assert np.all(kept >= np.minimum(ks, nb)[:, None])
     assert np.array_equal(got.sum(axis=2), kept)
-    s = O.block_logits(f64(qp), f64(kp), sc)
+    s = O.block_logits(qpr, kpr, sc)
+    if key_bias_r is not None:
+        s = s + np.asarray(key_bias_r)[None, None, :]
     for h, i in zip(*np.nonzero(~qual)):
         diff = got[h, i] ^ ref["mask"][h, i]
         if diff.any():
@@ -240,23 +250,52 @@ def _selection_parity(qp, kp, sc, top_k, tau):
     # CSR matches the mask
     rp = sel["row_ptr"].cpu().numpy()
     assert rp[-1] == kept.sum() and sel["total"] == kept.sum()
+    ci = sel["col_idx"].cpu().numpy()
+    for r in range(0, H * nb, max(1, H * nb // 64)):
+        assert ci[rp[r]:rp[r + 1]].tolist() == np.nonzero(got.reshape(H * nb, nb)[r])[0].tolist()
     return int(qual.sum()), qual.size
 
 
-@pytest.mark.parametrize("top_k,tau", [(1, 0.05), (4, 0.2), (16, 0.5), (4, 1.0), (4, 0.0), (2000, 0.2)])
-def test_block_select_synthetic_720p_heads(top_k, tau):
-    wl = synth.WORKLOADS["720p"]
+def _pooled_720p(heads=2, seed=None):
+    """720p grid, Q/K from the workload's generator. The zone shapes are the
+    oracle's rule applied to Q viewed as the feature input (as the 720p workload
+    does), or with ``seed`` a seeded draw over all candidates; either way they
+    are an input to both sides. Returns the GPU pooled features and the oracle's
+    own fp64 pooling of the same Q/K."""
     import dataclasses
-    wl = dataclasses.replace(wl, heads=2)
+    wl = dataclasses.replace(synth.WORKLOADS["720p"], heads=heads)
     x = synth.qkv(wl)
     geo = P.Geometry(wl.grid, wl.zone, CAND)
+    nz, _ = geo.counts()
+    if seed is None:
+        zone_shape, _, _ = O.zone_shapes(wl.grid, wl.zone, CAND, F=f64(x["q"].reshape(wl.n_tokens, -1)))
+    else:
+        zone_shape = np.random.default_rng(seed).integers(0, len(CAND), nz)
     dev = torch.device("cuda")
     q, k = x["q"].to(dev), x["k"].to(dev)
-    N = wl.n_tokens
-    zs, _ = P.zone_shapes(geo, feat=q.view(N, -1))
+    zs = torch.tensor(zone_shape, dtype=torch.int32, device=dev)
     qp, kp = P.block_pool(geo, zs, q, k)
-    n_q, n = _selection_parity(qp, kp, scale_for(wl.head_dim), top_k, tau)
+    blocks = O.block_tokens(wl.grid, wl.zone, CAND, zone_shape)
+    return wl, geo, zs, zone_shape, blocks, qp, kp, O.block_pool(f64(x["q"]), blocks), O.block_pool(f64(x["k"]), blocks)
+
+
+@pytest.fixture(scope="module")
+def pooled_720p():
+    return _pooled_720p()
+
+
+@pytest.mark.parametrize("top_k,tau", [(1, 0.05), (4, 0.2), (16, 0.5), (4, 1.0), (4, 0.0), (2000, 0.2)])
+def test_block_select_synthetic_720p_heads(top_k, tau, pooled_720p):
+    wl, _, _, _, _, qp, kp, qpr, kpr = pooled_720p
+    n_q, n = _selection_parity(qp, kp, scale_for(wl.head_dim), top_k, tau, qpr, kpr)
     assert n_q > 0.2 * n
+
+
+def test_block_select_random_zone_shapes():
+    """Pooled features over a seeded mix of all candidate shapes."""
+    wl, _, _, _, _, qp, kp, qpr, kpr = _pooled_720p(heads=2, seed=21)
+    _selection_parity(qp, kp, scale_for(wl.head_dim), 4, 0.2, qpr, kpr)
+    _selection_parity(qp, kp, scale_for(wl.head_dim), [2, 8], [0.5, 0.1], qpr, kpr)
 
 
 def test_block_select_ragged_block_count():
@@ -264,9 +303,72 @@ def test_block_select_ragged_block_count():
     gen = torch.Generator().manual_seed(9)
     dev = torch.device("cuda")
     for nb in (37, 1, 65, 200):
-        qp = torch.randn((3, nb, 64), generator=gen).to(dev)
-        kp = torch.randn((3, nb, 64), generator=gen).to(dev)
-        _selection_parity(qp, kp, 0.125, 3, 0.3)
+        qp = torch.randn((3, nb, 64), generator=gen)
+        kp = torch.randn((3, nb, 64), generator=gen)
+        _selection_parity(qp.to(dev), kp.to(dev), 0.125, 3, 0.3, f64(qp), f64(kp))
+
+
+def test_block_select_per_head_k_and_tau():
+    """Per-head floors and thresholds (the ratio form gives the floors of two heads)."""
+    wl, _, _, _, _, qp, kp, qpr, kpr = _pooled_720p(heads=4)
+    nb = qp.shape[1]
+    ks = [1, P.topk_from_sparsity(0.99, nb), P.topk_from_sparsity(0.9, nb), 4]
+    assert ks[1:3] == [O.topk_from_sparsity(0.99, nb), O.topk_from_sparsity(0.9, nb)]
+    taus = [0.05, 0.2, 0.5, 1.0]
+    n_q, n = _selection_parity(qp, kp, scale_for(wl.head_dim), ks, taus, qpr, kpr)
+    assert n_q > 0.2 * n
+    # per-head arrays equal to the scalars reproduce the plain entry point bit for bit
+    a = P.block_select(qp, kp, scale_for(wl.head_dim), 4, 0.2)
+    b = P.block_select_ex(qp, kp, scale_for(wl.head_dim), [4] * 4, [0.2] * 4)
+    assert torch.equal(a["mask"], b["mask"]) and torch.equal(a["col_idx"], b["col_idx"])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_block_audio_bias_matches_oracle(dtype):
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["1080p"], grid=(16, 32, 48))
+    dev = torch.device("cuda")
+    R, _ = synth.a2v_residual(wl, device=dev)
+    R = R.to(dtype)
+    geo = P.Geometry(wl.grid, wl.zone, CAND)
+    nz, nb = geo.counts()
+    zone_shape = np.random.default_rng(23).integers(0, len(CAND), nz)
+    zs = torch.tensor(zone_shape, dtype=torch.int32, device=dev)
+    ws = P.Workspace(dev)
+    blocks = O.block_tokens(wl.grid, wl.zone, CAND, zone_shape)
+    for beta in (0.0, 2.0, -0.5):
+        b = P.block_audio_bias(geo, zs, R, beta, ws=ws)
+        ref = O.block_key_bias(f64(R), blocks, beta)
+        assert np.allclose(f64(b), ref, rtol=1e-5, atol=1e-6), np.abs(f64(b) - ref).max()
+    # strided residual rows (row stride 3072 + 64) and the zero residual
+    Rs = torch.zeros((geo.n_tokens, 3136), dtype=dtype, device=dev)
+    Rs[:, :3072] = R
+    b = P.block_audio_bias(geo, zs, Rs[:, :3072], 2.0, ws=ws)
+    assert np.allclose(f64(b), O.block_key_bias(f64(R), blocks, 2.0), rtol=1e-5, atol=1e-6)
+    assert (P.block_audio_bias(geo, zs, torch.zeros_like(R), 2.0, ws=ws) == 0).all()
+    P.check_device_status(ws)
+
+
+def test_block_select_with_audio_bias_end_to_end():
+    """720p Q/K with a synthetic a2v residual: bias from the residual norms on
+    both sides, then the biased hybrid selection; the bias raises the loud
+    blocks' share of the kept sets."""
+    wl, geo, zs, zone_shape, blocks, qp, kp, qpr, kpr = _pooled_720p(heads=2)
+    dev = torch.device("cuda")
+    R, _ = synth.a2v_residual(wl, channels=768, device=dev)
+    sc = scale_for(wl.head_dim)
+    beta = 3.0
+    b = P.block_audio_bias(geo, zs, R, beta)
+    br = O.block_key_bias(f64(R), blocks, beta)
+    n_q, n = _selection_parity(qp, kp, sc, 4, 0.2, qpr, kpr, key_bias=b, key_bias_r=br)
+    assert n_q > 0.2 * n
+    plain = mask_bits_to_bool(P.block_select(qp, kp, sc, 4, 0.2)["mask"], qp.shape[1])
+    biased = mask_bits_to_bool(P.block_select_ex(qp, kp, sc, 4, 0.2, key_bias=b)["mask"], qp.shape[1])
+    loud = br > np.quantile(br, 0.9)
+    # the loud blocks' share of what the rows keep rises (the rows also keep
+    # fewer blocks: the softmax mass concentrates on them)
+    share = lambda m: m[:, :, loud].sum() / m.sum()
+    assert share(biased) > share(plain) and biased.sum() <= plain.sum()
 
 
 # --------------------------------------------------------------------------- zone shapes
