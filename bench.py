@@ -355,6 +355,63 @@ def selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src):
     return out
 
 
+def measure_selection_variants(pipe, res, peaks, peak_src, reps=5):
+    """Per-call times of the selection variants outside the timed step (CUDA events,
+    same stream, after the step's warm-up): the audio-norm key-block bias over the
+    a2v residual (an HBM stream: algorithmic bytes = the residual read once), and
+    the selection with per-head k / tau and that bias next to the plain selection."""
+    import ctypes
+    import torch
+    P, wl = pipe.P, pipe.wl
+    H, nb, d = pipe.qp.shape
+    g = pipe.geo.c()
+    bias = torch.empty(nb, dtype=torch.float32, device=pipe.qp.device)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    out = {}
+    if res is not None:
+        def run_bias():
+            P._check(P.lib().prism_block_audio_bias(ctypes.byref(g), P._ptr(pipe.zone_shape), P._ptr(res),
+                                                    res.stride(0), res.shape[1], P.BF16, 1.0, P._ptr(bias),
+                                                    pipe.ws.ptr, pipe.ws.nbytes, P._stream()), "audio_bias")
+        ms = timed(run_bias)
+        nbytes = res.numel() * res.element_size()
+        hbm = float(peaks.get("hbm_gbs"))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out["block_audio_bias"] = {"ms": round(ms, 4), "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                   "unit": "GB/s", "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
+                                   "peak_source": f"{peak_src} copy bandwidth"}
+    else:
+        bias.zero_()
+    ks = (ctypes.c_int32 * H)(*[max(1, wl.top_k >> (h % 3)) for h in range(H)])
+    taus = (ctypes.c_float * H)(*[wl.cdf_threshold * (1 + (h % 2)) for h in range(H)])
+    cp = P._SelectParams(wl.top_k, wl.cdf_threshold, ctypes.cast(ks, ctypes.POINTER(ctypes.c_int32)),
+                         ctypes.cast(taus, ctypes.POINTER(ctypes.c_float)), bias.data_ptr())
+    mask = torch.empty_like(pipe.mask)
+    kept = torch.empty_like(pipe.kept)
+    row_ptr = torch.empty_like(pipe.row_ptr)
+
+    def run_ex():
+        P._check(P.lib().prism_block_select_ex(P._ptr(pipe.qp), P._ptr(pipe.kp), H, nb, d, pipe.scale,
+                                               ctypes.byref(cp), P._ptr(mask), P._ptr(kept), P._ptr(row_ptr), None,
+                                               0, None, pipe.ws.ptr, pipe.ws.nbytes, P._stream()), "select_ex")
+    out["block_select_ex"] = {"ms": round(timed(run_ex), 4),
+                              "settings": "per-head k in {k, k/2, k/4}, tau in {tau, 2 tau}, audio-norm bias beta 1",
+                              "plain_block_select_ms": round(timed(pipe.stage_select), 4)}
+    P.check_device_status(pipe.ws)
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -395,6 +452,7 @@ def run_gpu(args):
     # end to end through the public API with host buffers
     e2e = None if args.no_e2e else run_e2e(pipe, wl, x, feats, res, steps=min(args.steps, args.e2e_steps))
     peaks, peak_src = _peaks()
+    variants = measure_selection_variants(pipe, res, peaks, peak_src)
     nnz = pipe.nnz
     attn_flop = nnz * (FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR)
     t_attn = (stage_ms["bsa_fwd"] + stage_ms["bsa_bwd"]) * 1e-3
@@ -419,6 +477,7 @@ def run_gpu(args):
                      "peak_source": f"{peak_src} bf16 sustained",
                      "flop_per_pair": FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR},
         "roofline_selection_path": selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src),
+        "selection_variants": variants,
         "e2e": e2e,
         "gpu_launches": pipe.launches_per_step() * args.steps,
         "clocks": clocks,
