@@ -33,6 +33,10 @@ Where the pages leave a step open, the readings taken here are (R1..R21 in the
 design notes):
 
 * zones tile the grid in raster (zt, zh, zw) order; a shape is (bt, bh, bw);
+  a grid that is not a whole number of zones is tiled as if rounded up, and
+  zones and block boxes are clipped to it: statistics, pooling and attention
+  use the member tokens only, and a box with no member is an empty block that
+  takes no part in the selection (R16);
 * V_a = mean over channels and over the lines parallel to axis a of the
   population variance of the feature channel along the line (R3);
 * r(n) = ||R[n, :]||_2; A_a = mean over lines parallel to a of the population
@@ -72,24 +76,25 @@ DEFAULT_GATE_MAX = 4.0
 # a1: macro-zone tiling  [README "Overview"]
 # --------------------------------------------------------------------------
 def zone_counts(grid, zone):
-    """Number of zones along (t, h, w); the grid must be a whole number of zones."""
+    """Number of zones along (t, h, w). Zones tile the grid rounded up to whole
+    zones; where an extent is not a multiple of the zone, the last zone along that
+    axis is clipped to the grid (reading R16)."""
     T, H, W = grid
     Zt, Zh, Zw = zone
-    if T % Zt or H % Zh or W % Zw:
-        raise ValueError("grid is not a whole number of zones")
-    return T // Zt, H // Zh, W // Zw
+    return -(-T // Zt), -(-H // Zh), -(-W // Zw)
 
 
 def zone_token_ids(grid, zone, z):
-    """Token ids of zone z as a [Zt, Zh, Zw] array (raster token order n = (t*H+h)*W+w)."""
+    """Token ids of zone z as a [zt', zh', zw'] array (raster token order
+    n = (t*H+h)*W+w); the extents are the zone's, clipped to the grid."""
     T, H, W = grid
     Zt, Zh, Zw = zone
     nt, nh, nw = zone_counts(grid, zone)
     zt, rem = divmod(z, nh * nw)
     zh, zw = divmod(rem, nw)
-    t = zt * Zt + np.arange(Zt)
-    h = zh * Zh + np.arange(Zh)
-    w = zw * Zw + np.arange(Zw)
+    t = np.arange(zt * Zt, min(T, zt * Zt + Zt))
+    h = np.arange(zh * Zh, min(H, zh * Zh + Zh))
+    w = np.arange(zw * Zw, min(W, zw * Zw + Zw))
     return (t[:, None, None] * H + h[None, :, None]) * W + w[None, None, :]
 
 
@@ -196,13 +201,18 @@ def blocks_per_zone(zone):
 
 
 def block_tokens(grid, zone, cand, shape_idx):
-    """Token ids [n_blocks, 64] of every block (tokens raster (t,h,w) inside)."""
+    """Token ids [n_blocks, 64] of every block (tokens raster (t,h,w) inside the
+    block's box). Blocks tile the zones of the rounded-up grid; a box position
+    outside the grid holds -1, so an edge block has fewer than 64 members and a
+    box wholly outside the grid is an empty block (reading R16)."""
+    T, H, W = grid
     nt, nh, nw = zone_counts(grid, zone)
     nz = nt * nh * nw
     bpz = blocks_per_zone(zone)
-    out = np.zeros((nz * bpz, 64), dtype=np.int64)
+    out = np.full((nz * bpz, 64), -1, dtype=np.int64)
     for z in range(nz):
-        ids = zone_token_ids(grid, zone, z)  # [Zt, Zh, Zw]
+        zt, rem = divmod(z, nh * nw)
+        zh, zw = divmod(rem, nw)
         bt, bh, bw = cand[int(shape_idx[z])]
         if bt * bh * bw != 64 or zone[0] % bt or zone[1] % bh or zone[2] % bw:
             raise ValueError("candidate does not tile the zone with 64-token blocks")
@@ -211,15 +221,33 @@ def block_tokens(grid, zone, cand, shape_idx):
             for lh in range(gh):
                 for lw in range(gw):
                     local = (lt * gh + lh) * gw + lw
-                    box = ids[lt * bt:(lt + 1) * bt, lh * bh:(lh + 1) * bh, lw * bw:(lw + 1) * bw]
-                    out[z * bpz + local] = box.reshape(-1)
+                    t = zt * zone[0] + lt * bt + np.arange(bt)
+                    h = zh * zone[1] + lh * bh + np.arange(bh)
+                    w = zw * zone[2] + lw * bw + np.arange(bw)
+                    tt, hh, ww = np.meshgrid(t, h, w, indexing="ij")
+                    ids = (tt * H + hh) * W + ww
+                    ids[(tt >= T) | (hh >= H) | (ww >= W)] = -1
+                    out[z * bpz + local] = ids.reshape(-1)
     return out
 
 
+def block_members(blocks, b):
+    """Token ids of block b that lie in the grid (raster order kept)."""
+    row = np.asarray(blocks[b])
+    return row[row >= 0]
+
+
 def block_pool(X, blocks):
-    """Mean of the 64 token rows of every block: X [N, heads, d] -> [heads, n_blocks, d]."""
+    """Mean of the member token rows of every block: X [N, heads, d] ->
+    [heads, n_blocks, d]. An empty block has no feature: NaN (R16)."""
     X = np.asarray(X, dtype=np.float64)
-    return X[blocks].mean(axis=1).transpose(1, 0, 2).copy()
+    blocks = np.asarray(blocks)
+    out = np.full((X.shape[1], blocks.shape[0], X.shape[2]), np.nan)
+    for b in range(blocks.shape[0]):
+        m = block_members(blocks, b)
+        if m.size:
+            out[:, b] = X[m].mean(axis=0)
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -270,6 +298,11 @@ def block_select(qp, kp, scale, top_k, tau, rows=None, key_bias=None):
     None or [nb]: b_J added to every head's logit of key block J before the
     ranking and the softmax (R20, the audio-norm scoring bias).
 
+    A block whose pooled feature is NaN (an empty block, R16) takes no part: as
+    a key it is never kept and carries no mass; as a query its row is empty
+    (kept 0). The rule then runs over the other key blocks, so "k >= n_blocks"
+    and "tau >= 1" keep every non-empty block.
+
     Returns dict: mask bool [heads, nb, nb] (only selected rows filled when
     ``rows`` is given), kept [heads, nb] (-1 where not computed), gap and
     margin arrays (nan where not computed).
@@ -287,8 +320,14 @@ def block_select(qp, kp, scale, top_k, tau, rows=None, key_bias=None):
     if rows is None:
         rows = [(h, i) for h in range(H) for i in range(nb)]
     for h, i in rows:
-        s = scale * (kp[h] @ qp[h, i]) + bias
+        if np.isnan(qp[h, i]).any():
+            kept[h, i] = 0
+            gap[h, i] = margin[h, i] = math.inf
+            continue
+        valid = np.nonzero(~np.isnan(kp[h]).any(axis=1))[0]
+        s = scale * (kp[h, valid] @ qp[h, i]) + bias[valid]
         idx, m, _, g, mg = select_row(s, int(ks[h]), float(taus[h]))
+        idx = valid[idx]
         mask[h, i, idx] = True
         kept[h, i] = m
         gap[h, i] = g
@@ -326,9 +365,14 @@ def block_key_bias(R, blocks, beta):
     r = token_norms(R)
     blocks = np.asarray(blocks)
     mean_grid = r.mean()
+    out = np.zeros(blocks.shape[0])
     if mean_grid == 0.0:
-        return np.zeros(blocks.shape[0])
-    return beta * r[blocks].mean(axis=1) / mean_grid
+        return out
+    for b in range(blocks.shape[0]):
+        m = block_members(blocks, b)
+        if m.size:  # an empty block keeps 0 (it is never selected)
+            out[b] = beta * r[m].mean() / mean_grid
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -336,9 +380,10 @@ def block_key_bias(R, blocks, beta):
 # --------------------------------------------------------------------------
 def token_block_index(blocks, n_tokens):
     """Block id of every token."""
-    b = np.empty(n_tokens, dtype=np.int64)
+    b = np.full(n_tokens, -1, dtype=np.int64)
     for i, row in enumerate(blocks):
-        b[row] = i
+        row = np.asarray(row)
+        b[row[row >= 0]] = i
     return b
 
 
@@ -399,8 +444,9 @@ def attention_block_rows(Q, K, V, blocks, kept_blocks, h, I, scale, dO=None, bf1
     dS = P (dP - D); dS rounded for the dS K product and dQ rounded when
     stored (``dQ_bound``). First order in the unit roundoff; a tolerance
     model, not a reference value."""
-    qi = blocks[I]
-    kj = blocks[np.asarray(kept_blocks)].reshape(-1)
+    qi = block_members(blocks, I)
+    kj = np.asarray(blocks)[np.asarray(kept_blocks, dtype=np.int64)].reshape(-1)
+    kj = kj[kj >= 0]
     q = np.asarray(Q[qi, h], np.float64)
     k = np.asarray(K[kj, h], np.float64)
     v = np.asarray(V[kj, h], np.float64)
@@ -439,7 +485,7 @@ def attention_kv_block_grads(Q, K, V, dO, blocks, sel_mask_h, h, J, scale, row_c
     dS^T to bf16 for the products and dK, dV when stored (see
     attention_block_rows).
     """
-    kj = blocks[J]
+    kj = block_members(blocks, J)
     k = np.asarray(K[kj, h], np.float64)
     v = np.asarray(V[kj, h], np.float64)
     dK = np.zeros_like(k)
@@ -455,7 +501,7 @@ def attention_kv_block_grads(Q, K, V, dO, blocks, sel_mask_h, h, J, scale, row_c
             rr = attention_block_rows(Q, K, V, blocks, np.nonzero(sel_mask_h[I])[0], h, int(I), scale, dO=dO)
             if row_cache is not None:
                 row_cache[key] = rr
-        qi = blocks[I]
+        qi = block_members(blocks, I)
         q = np.asarray(Q[qi, h], np.float64)
         do = np.asarray(dO[qi, h], np.float64)
         S = scale * q @ k.T
@@ -465,11 +511,13 @@ def attention_kv_block_grads(Q, K, V, dO, blocks, sel_mask_h, h, J, scale, row_c
         dS = P * (dP - rr["D"][:, None])
         dK += scale * dS.T @ q
         if bf16_bound:
-            bD = rr["D_bound"] if "D_bound" in rr else BF16_U * (
-                np.abs(do) * ((np.exp(scale * q @ np.asarray(K[blocks[np.nonzero(sel_mask_h[I])[0]].reshape(-1), h],
-                                                               np.float64).T - rr["lse"][:, None]))
-                              @ np.abs(np.asarray(V[blocks[np.nonzero(sel_mask_h[I])[0]].reshape(-1), h],
-                                                  np.float64)))).sum(axis=1)
+            if "D_bound" in rr:
+                bD = rr["D_bound"]
+            else:
+                ks_ = np.asarray(blocks)[np.nonzero(sel_mask_h[I])[0]].reshape(-1)
+                ks_ = ks_[ks_ >= 0]
+                Pn_ = np.exp(scale * q @ np.asarray(K[ks_, h], np.float64).T - rr["lse"][:, None])
+                bD = BF16_U * (np.abs(do) * (Pn_ @ np.abs(np.asarray(V[ks_, h], np.float64)))).sum(axis=1)
             bV += P.T @ np.abs(do)
             bK += scale * np.abs(dS).T @ np.abs(q)
             bKD += scale * P.T @ (bD[:, None] * np.abs(q))

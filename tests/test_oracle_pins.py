@@ -196,6 +196,167 @@ def test_pooling_of_a_linear_field_is_its_value_at_the_block_centre():
         assert np.allclose(pooled[0, b], expect, atol=1e-12)
 
 
+# ----------------------------------------------------------------- grids that are not whole zones
+PARTIAL_GRID, PARTIAL_ZONE = (10, 13, 9), (8, 8, 8)
+
+
+def test_partial_grid_blocks_from_coordinates():
+    """Every token of a 10x13x9 grid (zones 8x8x8, clipped at the far edges),
+    placed by direct coordinate arithmetic, sits at its raster slot of its
+    block's box; every token appears once and nothing else is a member."""
+    T, H, W = PARTIAL_GRID
+    nt, nh, nw = O.zone_counts(PARTIAL_GRID, PARTIAL_ZONE)
+    assert (nt, nh, nw) == (2, 2, 2)
+    rng = np.random.default_rng(4)
+    idx = rng.integers(0, len(CAND), nt * nh * nw)
+    blocks = O.block_tokens(PARTIAL_GRID, PARTIAL_ZONE, CAND, idx)
+    assert blocks.shape == (8 * 8, 64)
+    for t in range(T):
+        for h in range(H):
+            for w in range(W):
+                z = ((t // 8) * nh + h // 8) * nw + w // 8
+                bt, bh, bw = CAND[idx[z]]
+                lt, lh, lw = (t % 8) // bt, (h % 8) // bh, (w % 8) // bw
+                b = z * 8 + (lt * (8 // bh) + lh) * (8 // bw) + lw
+                r = (((t % 8) % bt) * bh + (h % 8) % bh) * bw + (w % 8) % bw
+                assert blocks[b, r] == (t * H + h) * W + w
+    assert (blocks >= 0).sum() == T * H * W
+    assert np.array_equal(np.sort(blocks[blocks >= 0]), np.arange(T * H * W))
+
+
+def test_clipped_zone_line_variance_closed_forms():
+    """Grid 8x8x11: the second zone along w holds columns 8..10. A feature
+    equal to w gives V_w = (L^2 - 1)/12 with L the clipped line length (63/12
+    in the full zone, 8/12 in the clipped one) and V_t = V_h = 0."""
+    grid = (8, 8, 11)
+    N = 8 * 8 * 11
+    w = np.arange(N) % 11
+    F = np.stack([w, 2.0 * w], axis=1).astype(np.float64)
+    st = O.zone_statistics(grid, (8, 8, 8), F=F)
+    assert st["V"].shape == (2, 3)
+    assert np.allclose(st["V"][0], [0, 0, 2.5 * 63 / 12], atol=1e-12)  # channel mean of 1 and 4
+    assert np.allclose(st["V"][1], [0, 0, 2.5 * 8 / 12], atol=1e-12)
+    # zone mean of the residual norm over the member tokens only
+    r = np.where(w >= 8, 3.0, 1.0)
+    st = O.zone_statistics(grid, (8, 8, 8), r=r)
+    assert np.allclose(st["m"], [1.0, 3.0]) and np.isclose(st["mbar"], (8 * 1 + 3 * 3) / 11)
+
+
+def test_partial_block_pooling_is_the_field_at_the_member_centroid():
+    T, H, W = PARTIAL_GRID
+    tt, hh, ww = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    coef = np.array([[0.5, -1.0, 0.25, 2.0], [1.5, 0.5, -0.75, 0.0]])
+    X = (coef[:, 0] * tt.reshape(-1, 1) + coef[:, 1] * hh.reshape(-1, 1) + coef[:, 2] * ww.reshape(-1, 1)
+         + coef[:, 3])[:, None, :]  # [N, 1 head, 2 channels]
+    idx = np.random.default_rng(8).integers(0, len(CAND), 8)
+    blocks = O.block_tokens(PARTIAL_GRID, PARTIAL_ZONE, CAND, idx)
+    pooled = O.block_pool(X, blocks)
+    n_empty = 0
+    for b in range(blocks.shape[0]):
+        m = blocks[b][blocks[b] >= 0]
+        if not m.size:
+            assert np.isnan(pooled[0, b]).all()
+            n_empty += 1
+            continue
+        t, h, w = m // (H * W), (m // W) % H, m % W
+        c = np.array([t.mean(), h.mean(), w.mean()])
+        assert np.allclose(pooled[0, b], coef[:, :3] @ c + coef[:, 3], atol=1e-12)
+    assert n_empty > 0  # the draw leaves some boxes wholly outside the grid
+
+
+def test_selection_skips_empty_blocks():
+    """Grid 8x8x10, zones 8x8x8; the second zone takes (8,8,1), whose boxes at
+    w >= 10 are empty: they are never kept and their rows are empty; on the
+    other blocks the rule equals subset brute force."""
+    grid, zone = (8, 8, 10), (8, 8, 8)
+    cand = [(4, 4, 4), (8, 8, 1)]
+    blocks = O.block_tokens(grid, zone, cand, [0, 1])
+    empty = (blocks < 0).all(axis=1)
+    assert empty.sum() == 6
+    rng = np.random.default_rng(6)
+    X = rng.normal(size=(8 * 8 * 10, 2, 6))
+    Y = rng.normal(size=(8 * 8 * 10, 2, 6))
+    qp, kp = O.block_pool(X, blocks), O.block_pool(Y, blocks)
+    sc = 0.9
+    for k, tau in ((1, 0.3), (3, 0.05), (20, 0.2), (2, 1.0)):
+        r = O.block_select(qp, kp, sc, k, tau)
+        assert not r["mask"][:, :, empty].any()
+        assert (r["kept"][:, empty] == 0).all() and not r["mask"][:, empty].any()
+        valid = np.nonzero(~empty)[0]
+        for h in range(2):
+            for i in valid:
+                s = sc * kp[h, valid] @ qp[h, i]
+                p = np.exp(s - s.max())
+                p /= p.sum()
+                want = {int(valid[j]) for j in _brute_force_selection_fast(p, k, tau)}
+                assert set(np.nonzero(r["mask"][h, i])[0].tolist()) == want
+        if tau >= 1.0:
+            assert (r["kept"][:, valid] == valid.size).all()
+
+
+def _brute_force_selection_fast(p, k, tau):
+    """The subset rule on many blocks: the best subset of each size is the top
+    of the sorted masses (ties to the lower index), so only prefixes are tried."""
+    n = len(p)
+    if k >= n or tau >= 1.0:
+        return set(range(n))
+    order = sorted(range(n), key=lambda j: (-p[j], j))
+    c, m_min = 0.0, n
+    for m in range(1, n + 1):
+        c += p[order[m - 1]]
+        if c >= tau:
+            m_min = m
+            break
+    return set(order[:max(k, m_min)])
+
+
+def test_partial_grid_dense_selection_is_full_attention():
+    """Keeping every non-empty block of a 6x8x10 grid (zones 4x8x8, clipped)
+    gives full softmax attention over all tokens (torch SDPA, fp64), through
+    both the masked form and the row-gathered form."""
+    grid, zone = (6, 8, 10), (4, 8, 8)
+    cand = [(4, 4, 4), (2, 4, 8), (4, 8, 2), (1, 8, 8)]
+    nz = int(np.prod(O.zone_counts(grid, zone)))
+    idx = np.random.default_rng(2).integers(0, len(cand), nz)
+    blocks = O.block_tokens(grid, zone, cand, idx)
+    N, H, d = 6 * 8 * 10, 2, 8
+    rng = np.random.default_rng(3)
+    Q, K, V, dO = (rng.normal(size=(N, H, d)) for _ in range(4))
+    qp, kp = O.block_pool(Q, blocks), O.block_pool(K, blocks)
+    sc = 1 / math.sqrt(d)
+    sel = O.block_select(qp, kp, sc, 1, 1.0)
+    allowed = O.token_mask(sel["mask"], blocks, N)
+    assert allowed.all()
+    Oo, lse = O.masked_attention_fwd(Q, K, V, allowed, sc)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(Q).permute(1, 0, 2), torch.tensor(K).permute(1, 0, 2), torch.tensor(V).permute(1, 0, 2),
+        scale=sc).permute(1, 0, 2).numpy()
+    assert np.allclose(Oo, ref, atol=1e-12)
+    dQ, dK, dV = O.masked_attention_bwd(Q, K, V, Oo, lse, dO, allowed, sc)
+    nonempty = np.nonzero((blocks >= 0).any(axis=1))[0]
+    cache = {}
+    for b in nonempty[:: max(1, len(nonempty) // 6)]:
+        m = O.block_members(blocks, b)
+        rr = O.attention_block_rows(Q, K, V, blocks, np.nonzero(sel["mask"][1, b])[0], 1, b, sc, dO=dO)
+        assert np.array_equal(rr["tokens"], m)
+        assert np.allclose(rr["O"], Oo[m, 1], atol=1e-12) and np.allclose(rr["dQ"], dQ[m, 1], atol=1e-12)
+        gk, gv = O.attention_kv_block_grads(Q, K, V, dO, blocks, sel["mask"][1], 1, b, sc, row_cache=cache)
+        assert np.allclose(gk, dK[m, 1], atol=1e-12) and np.allclose(gv, dV[m, 1], atol=1e-12)
+
+
+def test_partial_grid_audio_bias_uses_member_tokens():
+    grid, zone = (8, 8, 10), (8, 8, 8)
+    blocks = O.block_tokens(grid, zone, [(4, 4, 4), (8, 8, 1)], [0, 1])
+    N = 640
+    w = np.arange(N) % 10
+    R = np.zeros((N, 3))
+    R[:, 2] = np.where(w >= 8, 4.0, 1.0)  # the two clipped columns are loud
+    b = O.block_key_bias(R, blocks, 1.0)
+    mbar = (8 * 1 + 2 * 4) / 10
+    assert np.allclose(b[:8], 1.0 / mbar)
+    assert np.allclose(b[8:10], 4.0 / mbar) and (b[10:] == 0).all()
+
+
 # ----------------------------------------------------------------- selection
 def _brute_force_selection(p, k, tau):
     """Smallest m such that SOME subset of size m carries mass >= tau (the
