@@ -6,13 +6,15 @@
 // and sounding regions keep more attention. The library's reading:
 //   b_J = beta * mean_{n in J} r(n) / mean_{all n} r(n),  r(n) = ||res[n, :]||_2.
 //
-// block_norm_kernel: one CTA per block, one warp per 8 of its 64 tokens. A
+// block_norm_kernel: one CTA per block, one warp per 8 of its 64 slots. A
 //   token's sum of squares is a strided lane sum of 16-byte loads (fp32),
-//   reduced by a fixed butterfly; the block mean adds the 64 norms in a fixed
-//   order. Every residual row is read once: the kernel is an HBM stream.
-// bias_normalize_kernel: one CTA. The grid mean of r is the mean of the block
-//   means (every block holds 64 tokens), summed in fp64 in a fixed order;
-//   then b_J = beta * mean_J / grid mean in place (0 for a zero residual).
+//   reduced by a fixed butterfly; the block sum adds the member tokens' norms
+//   in a fixed order (a block clipped by the grid's edge has fewer than 64
+//   members). Every residual row is read once: the kernel is an HBM stream.
+// bias_normalize_kernel: one CTA. The grid mean of r is the sum of the block
+//   sums over the token count, summed in fp64 in a fixed order; then
+//   b_J = beta * (sum_J / members_J) / grid mean in place (0 for a zero
+//   residual and for an empty block, which the selection never keeps).
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -71,9 +73,11 @@ __global__ void __launch_bounds__(kNormWarps * 32) block_norm_kernel(const Geo g
   // (raster t, h, w) is found with shifts.
   const int lw = __ffs(bb.bw) - 1, lhw = lw + __ffs(bb.bh) - 1;
   const int n16 = row_bytes / 16;
+  const uint64_t members = g.partial ? block_slot_mask(g, bb) : ~uint64_t(0);
   float sum = 0.f;
   for (int i = 0; i < kNormTokensPerWarp; ++i) {
     const int r = warp * kNormTokensPerWarp + i;
+    if (!((members >> r) & 1)) continue;  // warp-uniform
     const int rt = r >> lhw, rh = (r >> lw) & (bb.bh - 1), rw = r & (bb.bw - 1);
     const int64_t n = (int64_t(bb.t0 + rt) * g.H + bb.h0 + rh) * g.W + bb.w0 + rw;
     sum += sqrtf(row_sum_squares<ES>(res + n * ld_bytes, n16, lane));
@@ -84,14 +88,15 @@ __global__ void __launch_bounds__(kNormWarps * 32) block_norm_kernel(const Geo g
     float t = 0.f;
 #pragma unroll
     for (int w = 0; w < kNormWarps; ++w) t += part[w];
-    out[b] = t * (1.0f / kBlockTokens);
+    out[b] = t;  // the block's sum of r over its members
   }
 }
 
-__global__ void __launch_bounds__(kNormalizeThreads) bias_normalize_kernel(float* __restrict__ bias, int nb,
-                                                                           float beta) {
+__global__ void __launch_bounds__(kNormalizeThreads) bias_normalize_kernel(const Geo g,
+                                                                           const int32_t* __restrict__ zone_shape,
+                                                                           float* __restrict__ bias, float beta) {
   __shared__ double red[kNormalizeThreads];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, nb = g.n_blocks;
   double s = 0.0;
   for (int j = tid; j < nb; j += kNormalizeThreads) s += double(bias[j]);
   red[tid] = s;
@@ -100,10 +105,19 @@ __global__ void __launch_bounds__(kNormalizeThreads) bias_normalize_kernel(float
     if (tid < half) red[tid] += red[tid + half];
     __syncthreads();
   }
-  const double mean = red[0] / double(nb);
-  for (int j = tid; j < nb; j += kNormalizeThreads)
-    bias[j] = mean > 0.0 ? float(double(beta) * double(bias[j]) / mean)
-                         : (mean == 0.0 ? 0.f : __int_as_float(0x7fc00000));  // NaN: a block reported an error
+  const double mean = red[0] / (double(g.T) * g.H * g.W);
+  for (int j = tid; j < nb; j += kNormalizeThreads) {
+    int members = kBlockTokens;
+    if (g.partial) {
+      const int sh = zone_shape[zone_of_block(g, j)];
+      members = (sh >= 0 && sh < g.n_cand) ? __popcll(block_slot_mask(g, block_box(g, sh, j))) : 0;
+    }
+    float v;
+    if (!(mean >= 0.0)) v = __int_as_float(0x7fc00000);  // NaN: a block reported an error
+    else if (mean == 0.0 || members == 0) v = 0.f;
+    else v = float(double(beta) * (double(bias[j]) / members) / mean);
+    bias[j] = v;
+  }
 }
 
 }  // namespace
@@ -134,6 +148,6 @@ extern "C" prism_status prism_block_audio_bias(const prism_geometry* geo, const 
   else
     block_norm_kernel<4><<<g.n_blocks, kNormWarps * 32, 0, s>>>(g, zone_shape, r, ld_bytes, row_bytes, key_bias,
                                                                 ws_status(ws));
-  bias_normalize_kernel<<<1, kNormalizeThreads, 0, s>>>(key_bias, g.n_blocks, beta);
+  bias_normalize_kernel<<<1, kNormalizeThreads, 0, s>>>(g, zone_shape, key_bias, beta);
   return cuda_status(cudaGetLastError());
 }

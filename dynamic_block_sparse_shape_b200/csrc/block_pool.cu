@@ -3,7 +3,8 @@
 //
 // One CTA per (block, tensor): each thread owns 8 consecutive channels of the
 // token row [heads * head_dim] and walks the block's 64 tokens eight at a time
-// (eight independent 16-byte loads in flight), accumulating in fp32.
+// (eight independent 16-byte loads in flight), accumulating in fp32. A block
+// clipped by the grid's edge averages its member tokens; an empty one is NaN.
 // The output layout is [heads, n_blocks, head_dim] fp32.
 #include <cuda_bf16.h>
 
@@ -33,6 +34,35 @@ __device__ __forceinline__ void load8<float>(const float* p, float* x) {
   x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
+// Sum of the block's member rows over this thread's 8 channels. GUARD is false
+// for a block wholly inside the grid: eight unconditional loads in flight.
+template <typename T, bool GUARD>
+__device__ __forceinline__ void sum_block_rows(const Geo& g, const BlockBox& bb, const T* base, int64_t tok_stride,
+                                               uint64_t members, float* acc) {
+  // Block extents divide 64, so they are powers of two: token r of the block
+  // (raster t, h, w) is found with shifts.
+  const int lw = __ffs(bb.bw) - 1, lhw = lw + __ffs(bb.bh) - 1;
+  for (int r0 = 0; r0 < kBlockTokens; r0 += 8) {
+    float x[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = r0 + i;
+      const int rt = r >> lhw, rh = (r >> lw) & (bb.bh - 1), rw = r & (bb.bw - 1);
+      const int64_t n = (int64_t(bb.t0 + rt) * g.H + bb.h0 + rh) * g.W + bb.w0 + rw;
+      if (!GUARD || ((members >> r) & 1)) {
+        load8<T>(base + n * tok_stride, x[i]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) x[i][c] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += x[i][c];
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(1024) pool_kernel(const Geo g, const int32_t* __restrict__ zone_shape,
                                                     const T* __restrict__ q, const T* __restrict__ k,
@@ -52,28 +82,19 @@ __global__ void __launch_bounds__(1024) pool_kernel(const Geo g, const int32_t* 
     return;
   }
   const BlockBox bb = block_box(g, shape, b);
+  // members: the box's slots inside the grid (all 64 unless the zone is clipped)
+  const uint64_t members = g.partial ? block_slot_mask(g, bb) : ~uint64_t(0);
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  // Block extents divide 64, so they are powers of two: token r of the block
-  // (raster t, h, w) is found with shifts. Eight independent loads in flight.
-  const int lw = __ffs(bb.bw) - 1, lhw = lw + __ffs(bb.bh) - 1;
   const T* base = src + c0;
-  for (int r0 = 0; r0 < kBlockTokens; r0 += 8) {
-    float x[8][8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + i;
-      const int rt = r >> lhw, rh = (r >> lw) & (bb.bh - 1), rw = r & (bb.bw - 1);
-      const int64_t n = (int64_t(bb.t0 + rt) * g.H + bb.h0 + rh) * g.W + bb.w0 + rw;
-      load8<T>(base + n * tok_stride, x[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] += x[i][c];
-  }
-  const float inv = 1.0f / 64.0f;
+  if (members == ~uint64_t(0))
+    sum_block_rows<T, false>(g, bb, base, tok_stride, members, acc);
+  else
+    sum_block_rows<T, true>(g, bb, base, tok_stride, members, acc);
+  // an empty block has no feature: NaN, which the selection reads as "absent"
+  const int cnt = __popcll(members);
+  const float inv = cnt ? 1.0f / float(cnt) : __int_as_float(0x7fc00000);
   reinterpret_cast<float4*>(out)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
   reinterpret_cast<float4*>(out)[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
 }

@@ -7,13 +7,16 @@
 // paper page: computing and materialising the proxy scores is the routing
 // overhead, so the scores here live only in shared memory.
 //
-// select_kernel: one CTA = 8 query blocks of one head (one warp each).
+// select_kernel: one CTA = 8 query blocks of one head (one warp each); 4 when
+// more than 5120 key blocks' logits must fit in shared memory.
 //   1. logits s_J = scale * qbar_I . kbar_J (+ b_J, the optional key-block
 //      bias, walkthrough section "桥接残差反哺稀疏注意力") for all J, fp32 FFMA,
 //      with the key features staged transposed in shared memory (2 keys x 4
 //      rows per thread per channel);
-//   2. per row: max, p_J = exp(s_J - max) in place, Z = sum p (fp64);
-//   3. the mass threshold: bisection on the float bits of p for
+//   2. per row: max, p_J = exp(s_J - max) in place as a ranking key (float
+//      bits + 1; 0 for a NaN logit, which marks an absent block: an empty
+//      block of a grid clipped at its edge), Z = sum p (fp64);
+//   3. the mass threshold: bisection on the keys for
 //      u* = max{u : sum_{key_J >= u} p_J >= tau * Z}; ties at u* are taken in
 //      ascending J until the mass is reached -> m*;
 //   4. m = max(k, m*); if m > m*, a bisection on counts finds the m-th key;
@@ -32,12 +35,13 @@
 namespace prism {
 namespace {
 
-constexpr int kSelRows = 8;
-constexpr int kSelThreads = 256;
 constexpr int kKeyTile = 256;
 constexpr int kDChunk = 32;
 constexpr int kKtPitch = kKeyTile + 2;
-constexpr int kSelMaxBlocks = 5120;
+// Rows of logits per CTA live in shared memory: 8 rows up to 5120 key blocks,
+// 4 rows (half the threads) up to 10240 (the 2K latent grid has 7680).
+constexpr int kSelMaxBlocks8 = 5120;
+constexpr int kSelMaxBlocks = 10240;
 constexpr int kSelMaxHeads = 128;  // per-head settings passed as a kernel parameter
 
 // Per-head floor k and mass threshold tau (uniform when per_head == 0).
@@ -60,37 +64,45 @@ __device__ __forceinline__ int warp_sum_i(int v) {
   return v;
 }
 
-// Mass of the entries whose key is >= u (fp64, warp-reduced).
-__device__ __forceinline__ double mass_at_least(const float* p, int nb, uint32_t u, int lane) {
+// Row entries are kept as ranking keys: key = (float bits of p) + 1 for a
+// present key block and 0 for an absent one (NaN logit: an empty block, or a
+// NaN input). For p >= 0 the float bits order like the values, so keys order
+// like p with every absent block below every present one.
+__device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float(key - 1u); }
+
+// Mass of the entries whose key is >= u >= 1 (fp64, warp-reduced).
+__device__ __forceinline__ double mass_at_least(const uint32_t* p, int nb, uint32_t u, int lane) {
   double acc = 0;
   for (int j = lane; j < nb; j += 32) {
-    const float v = p[j];
-    if (__float_as_uint(v) >= u) acc += double(v);
+    const uint32_t k = p[j];
+    if (k >= u) acc += double(key_value(k));
   }
   return warp_sum_d(acc);
 }
-__device__ __forceinline__ int count_at_least(const float* p, int nb, uint32_t u, int lane) {
+__device__ __forceinline__ int count_at_least(const uint32_t* p, int nb, uint32_t u, int lane) {
   int c = 0;
-  for (int j = lane; j < nb; j += 32) c += __float_as_uint(p[j]) >= u;
+  for (int j = lane; j < nb; j += 32) c += p[j] >= u;
   return warp_sum_i(c);
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1)
+template <int ROWS>
+__global__ void __launch_bounds__(ROWS * 32, 1)
     select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int nb, int d, float scale,
                   const __grid_constant__ SelHeads hp, const float* __restrict__ kbias, uint32_t* __restrict__ mask,
                   int32_t* __restrict__ kept) {
+  constexpr int kThreads = ROWS * 32;
   extern __shared__ __align__(16) float sm[];
-  float* srow = sm;                                  // [kSelRows][nb]
-  float* kT = srow + size_t(kSelRows) * nb;          // [kDChunk][kKtPitch]
-  float* qT = kT + kDChunk * kKtPitch;               // [d][kSelRows]
+  float* srow = sm;                                  // [ROWS][nb]
+  float* kT = srow + size_t(ROWS) * nb;              // [kDChunk][kKtPitch]
+  float* qT = kT + kDChunk * kKtPitch;               // [d][ROWS]
   const int head = blockIdx.y;
-  const int I0 = blockIdx.x * kSelRows;
+  const int I0 = blockIdx.x * ROWS;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* qh = qp + size_t(head) * nb * d;
   const float* kh = kp + size_t(head) * nb * d;
-  for (int i = tid; i < kSelRows * d; i += kSelThreads) {
+  for (int i = tid; i < ROWS * d; i += kThreads) {
     const int r = i / d, c = i - r * d;
-    qT[c * kSelRows + r] = (I0 + r < nb) ? qh[size_t(I0 + r) * d + c] : 0.f;
+    qT[c * ROWS + r] = (I0 + r < nb) ? qh[size_t(I0 + r) * d + c] : 0.f;
   }
   // ---- 1. logits
   const int kpair = tid & 127, rh = tid >> 7;
@@ -99,7 +111,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     for (int c0 = 0; c0 < d; c0 += kDChunk) {
       __syncthreads();
       // stage kT[c][j] = kbar[key0 + j][c0 + c], 256 keys x 32 channels
-      for (int i = tid; i < kKeyTile * (kDChunk / 4); i += kSelThreads) {
+      for (int i = tid; i < kKeyTile * (kDChunk / 4); i += kThreads) {
         const int j = i >> 3, q4 = i & 7;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (key0 + j < nb) v = __ldg(reinterpret_cast<const float4*>(kh + size_t(key0 + j) * d + c0) + q4);
@@ -112,7 +124,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 #pragma unroll 8
       for (int c = 0; c < kDChunk; ++c) {
         const float2 kv = *reinterpret_cast<const float2*>(kT + c * kKtPitch + 2 * kpair);
-        const float4 qv = *reinterpret_cast<const float4*>(qT + (c0 + c) * kSelRows + 4 * rh);
+        const float4 qv = *reinterpret_cast<const float4*>(qT + (c0 + c) * ROWS + 4 * rh);
         acc[0][0] = fmaf(qv.x, kv.x, acc[0][0]); acc[0][1] = fmaf(qv.x, kv.y, acc[0][1]);
         acc[1][0] = fmaf(qv.y, kv.x, acc[1][0]); acc[1][1] = fmaf(qv.y, kv.y, acc[1][1]);
         acc[2][0] = fmaf(qv.z, kv.x, acc[2][0]); acc[2][1] = fmaf(qv.z, kv.y, acc[2][1]);
@@ -133,28 +145,46 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (I >= nb) return;
   const int top_k = hp.per_head ? hp.k[head] : hp.k0;
   const float tau = hp.per_head ? hp.tau[head] : hp.tau0;
-  float* p = srow + size_t(warp) * nb;
+  uint32_t* p = reinterpret_cast<uint32_t*>(srow + size_t(warp) * nb);
+  const float* sl = srow + size_t(warp) * nb;
   const int words = (nb + 31) >> 5;
   uint32_t* mrow = mask + (size_t(head) * nb + I) * words;
   float mx = -INFINITY;
-  for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, p[j]);
+  for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, sl[j]);  // fmaxf skips NaN
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   double zacc = 0;
-  for (int j = lane; j < nb; j += 32) {
-    float e = expf(p[j] - mx);
-    if (!(e >= 0.f)) e = 0.f;  // NaN logits carry no mass
-    p[j] = e;
-    zacc += double(e);
+  int n_present = 0;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    uint32_t key = 0u;
+    if (j < nb) {
+      const float s = sl[j];
+      if (s == s) {  // present: NaN logits mark absent blocks
+        float e = expf(s - mx);
+        if (!(e >= 0.f)) e = 0.f;  // every present logit -inf: no mass
+        key = __float_as_uint(e) + 1u;
+        zacc += double(e);
+      }
+      p[j] = key;
+    }
+    n_present += __popc(__ballot_sync(0xffffffffu, key != 0u));
   }
   const double Z = warp_sum_d(zacc);
   __syncwarp();
-  if (top_k >= nb || tau >= 1.0f) {
-    for (int w = lane; w < words; w += 32) {
-      const int rem = nb - 32 * w;
-      mrow[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+  if (n_present == 0) {  // an empty query block (or no present key): empty row
+    for (int w = lane; w < words; w += 32) mrow[w] = 0u;
+    if (lane == 0) kept[size_t(head) * nb + I] = 0;
+    return;
+  }
+  if (top_k >= n_present || tau >= 1.0f) {
+    // every present block
+    for (int w = 0; w < words; ++w) {
+      const int j = 32 * w + lane;
+      const uint32_t kb = __ballot_sync(0xffffffffu, j < nb && p[j] != 0u);
+      if (lane == 0) mrow[w] = kb;
     }
-    if (lane == 0) kept[size_t(head) * nb + I] = nb;
+    if (lane == 0) kept[size_t(head) * nb + I] = n_present;
     return;
   }
   const double target = double(tau) * Z;
@@ -164,13 +194,13 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   if (target <= 0.0) {
     // C_1 >= tau already: the single largest entry (ties -> lowest J).
     uint32_t best = 0;
-    for (int j = lane; j < nb; j += 32) best = max(best, __float_as_uint(p[j]));
+    for (int j = lane; j < nb; j += 32) best = max(best, p[j]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
     u_star = best;
     m_star = count_at_least(p, nb, u_star + 1, lane) + 1;
   } else {
-    uint32_t lo = 0, hi = 0x3F800001u;  // mass(>= lo) >= target, mass(>= hi) < target
+    uint32_t lo = 1, hi = 0x3F800002u;  // mass(>= lo) >= target, mass(>= hi) < target
     while (hi - lo > 1) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
       if (mass_at_least(p, nb, mid, lane) >= target) lo = mid; else hi = mid;
@@ -184,13 +214,11 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     bool found = false;
     for (int base = 0; base < nb && !found; base += 32) {
       const int j = base + lane;
-      const bool tie = j < nb && __float_as_uint(p[j]) == u_star;
+      const bool tie = j < nb && p[j] == u_star;
       uint32_t bal = __ballot_sync(0xffffffffu, tie);
       while (bal) {
-        const int src = __ffs(bal) - 1;
         bal &= bal - 1;
-        (void)src;
-        run += double(__uint_as_float(u_star));  // every tied entry has p = u_star
+        run += double(key_value(u_star));  // every tied entry has p = value of u_star
         ++rank;
         if (run >= target) { found = true; break; }
       }
@@ -198,14 +226,14 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     if (!found) rank = max(rank, 1);
     m_star = above_cnt + rank;
   }
-  const int m = max(min(top_k, nb), m_star);
+  const int m = max(min(top_k, n_present), m_star);
   uint32_t u_final;
   int keep_ties;  // number of entries tied at u_final to keep, lowest J first
   if (m == m_star) {
     u_final = u_star;
     keep_ties = m - count_at_least(p, nb, u_star + 1, lane);
   } else {
-    uint32_t lo = 0, hi = 0x7F800001u;  // count(>= lo) >= m, count(>= hi) < m
+    uint32_t lo = 1, hi = 0x7F800002u;  // count(>= lo) >= m, count(>= hi) < m
     while (hi - lo > 1) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
       if (count_at_least(p, nb, mid, lane) >= m) lo = mid; else hi = mid;
@@ -216,7 +244,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
   int tie_run = 0;
   for (int w = 0; w < words; ++w) {
     const int j = 32 * w + lane;
-    const uint32_t key = j < nb ? __float_as_uint(p[j]) : 0u;
+    const uint32_t key = j < nb ? p[j] : 0u;
     const bool tie = j < nb && key == u_final;
     const uint32_t tb = __ballot_sync(0xffffffffu, tie);
     const int my_rank = tie_run + __popc(tb & ((1u << lane) - 1u));
@@ -322,11 +350,19 @@ prism_status block_select_impl(const float* q_pool, const float* k_pool, int32_t
   if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
   if (col_idx && col_cap < 0) return PRISM_ERR_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const size_t smem = (size_t(kSelRows) * n_blocks + kDChunk * kKtPitch + size_t(head_dim) * kSelRows) * sizeof(float);
-  if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return PRISM_ERR_CUDA;
-  const dim3 grid((n_blocks + kSelRows - 1) / kSelRows, heads);
-  select_kernel<<<grid, kSelThreads, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, hp, key_bias, mask, kept);
+  const int rows_per_cta = n_blocks <= kSelMaxBlocks8 ? 8 : 4;
+  const size_t smem =
+      (size_t(rows_per_cta) * n_blocks + kDChunk * kKtPitch + size_t(head_dim) * rows_per_cta) * sizeof(float);
+  const dim3 grid((n_blocks + rows_per_cta - 1) / rows_per_cta, heads);
+  if (rows_per_cta == 8) {
+    if (cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+    select_kernel<8><<<grid, 256, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, hp, key_bias, mask, kept);
+  } else {
+    if (cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+      return PRISM_ERR_CUDA;
+    select_kernel<4><<<grid, 128, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, hp, key_bias, mask, kept);
+  }
   const int rows = heads * n_blocks;
   if (launch_exclusive_scan(kept, rows, row_ptr, s) != cudaSuccess) return PRISM_ERR_CUDA;
   if (total_kept) {

@@ -263,13 +263,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     }
     for (int j = 0; j < nsteps; ++j) {
       const int sb = j & 1;
+      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
+      // keys of a key block clipped by the grid's edge (read before the wait)
+      uint32_t members = 0xffffffffu;
+      if (g.partial && valid)
+        members = uint32_t(key_block_members(g, P.zone_shape, __ldg(P.idx + beg + j * kKB + kh)) >> (ch * 32));
       mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t rs[32], rp[32];
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
       tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
       tmem_ld_wait();
-      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
+      mask_scores32(rs, members);  // P = exp2(-inf) = 0 there, hence dS = 0
       uint32_t pk[16];
       if (valid) {
         const float c = P.scale_log2, nl = -lse2;
@@ -310,8 +315,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       for (int i = 0; i < NC; ++i) v[i] = 0.f;
     }
     const int sI = safe_shape(g, P.zone_shape, I, status);
-    const int tok = block_token(g, block_box(g, sI, I), m);
-    store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * (D / 2) + ch * NC, v, P.out_fp32);
+    const BlockBox qb = block_box(g, sI, I);
+    const int tok = block_token(g, qb, m);
+    if (!g.partial || block_slot_in_grid(g, qb, m))  // a slot outside the grid has no row
+      store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * (D / 2) + ch * NC, v,
+                    P.out_fp32);
   }
   tc_fence_before();
   __syncthreads();
@@ -609,10 +617,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       for (int i = 0; i < NC; ++i) vv[i] = vk[i] = 0.f;
     }
     const int sJ = safe_shape(g, P.zone_shape, J, status);
-    const int tok = block_token(g, block_box(g, sJ, J), m);
+    const BlockBox kb = block_box(g, sJ, J);
+    const int tok = block_token(g, kb, m);
     const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * (D / 2) + ch * NC;
-    store_row<NC>(P.out0, off, vk, P.out_fp32);
-    store_row<NC>(P.out1, off, vv, P.out_fp32);
+    // a key slot outside the grid (a block clipped by the edge) has no row; the
+    // query slots outside the grid carry P = 0 (LSE = +inf from the prep pass)
+    if (!g.partial || block_slot_in_grid(g, kb, m)) {
+      store_row<NC>(P.out0, off, vk, P.out_fp32);
+      store_row<NC>(P.out1, off, vv, P.out_fp32);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -663,13 +676,19 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const Geo g, const int32_
   const int b = blockIdx.x, head = blockIdx.y;
   const int r = threadIdx.x >> 2, part = threadIdx.x & 3;
   const int s = safe_shape(g, zone_shape, b, status);
-  const int tok = block_token(g, block_box(g, s, b), r);
+  const BlockBox bb = block_box(g, s, b);
+  const int tok = block_token(g, bb, r);
+  // a slot outside the grid (a block clipped by the edge) has no token
+  const bool in_grid = !g.partial || block_slot_in_grid(g, bb, r);
   const int n = head_dim / 4;
   const int64_t off = int64_t(tok) * tok_stride + int64_t(head) * head_dim + part * n;
-  float acc = dot_chunk<T>(o + off, dout + off, n);
-  // the forward's rounding residual restores O to about 16 bits before the dot
-  if constexpr (std::is_same_v<T, __nv_bfloat16>) {
-    if (o_lo) acc += dot_chunk<T>(o_lo + off, dout + off, n);
+  float acc = 0.f;
+  if (in_grid) {
+    acc = dot_chunk<T>(o + off, dout + off, n);
+    // the forward's rounding residual restores O to about 16 bits before the dot
+    if constexpr (std::is_same_v<T, __nv_bfloat16>) {
+      if (o_lo) acc += dot_chunk<T>(o_lo + off, dout + off, n);
+    }
   }
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
@@ -679,8 +698,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const Geo g, const int32_
     const int N = g.T * g.H * g.W;
     // A query with no keys has LSE = -inf and, by definition, P = 0 and no
     // gradient. Storing +inf there makes exp2(s * c - lse2) = exp2(-inf) = 0 in
-    // both passes without a per-score test.
-    const float l = lse[int64_t(head) * N + tok];
+    // both passes without a per-score test; so does a slot outside the grid.
+    const float l = in_grid ? lse[int64_t(head) * N + tok] : -INFINITY;
     lse2_blk[at] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
   }
 }

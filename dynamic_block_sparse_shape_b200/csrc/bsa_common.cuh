@@ -117,6 +117,29 @@ __device__ __forceinline__ int safe_shape(const Geo& g, const int32_t* zone_shap
   return s;
 }
 
+// Slots of key block b that lie in the grid, as a 64-bit mask over the raster
+// slots of its box: all ones unless b's zone is clipped by the grid's edge.
+// The TMA copy of a clipped box fills its outside slots with zeros; the
+// softmax warps give those keys a score of -inf. A block id out of range
+// (reported by the coordinate cache) counts as whole.
+__device__ __forceinline__ uint64_t key_block_members(const Geo& g, const int32_t* zone_shape, int b) {
+  if (b < 0 || b >= g.n_blocks) return ~uint64_t(0);
+  const int z = zone_of_block(g, b);
+  if (zone_is_whole(g, z)) return ~uint64_t(0);
+  int s = __ldg(zone_shape + z);
+  if (s < 0 || s >= g.n_cand) s = 0;
+  return block_slot_mask(g, block_box(g, s, b));
+}
+
+// Scores of keys outside the grid become -inf: r[i] holds key ch*32 + i.
+__device__ __forceinline__ void mask_scores32(uint32_t* r, uint32_t members) {
+  if (members != 0xffffffffu) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (!((members >> i) & 1u)) r[i] = 0xff800000u;  // -inf
+  }
+}
+
 // TMA coordinates (shape, w0, h0, t0) of the blocks named by a CSR / CSC list,
 // computed 32 at a time by a whole warp (coalesced list reads, parallel
 // zone-shape lookups) into a shared-memory ring, so the thread that issues the

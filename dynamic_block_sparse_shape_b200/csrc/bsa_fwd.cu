@@ -290,6 +290,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     }
     for (int j = 0; j < nsteps; ++j) {
       const int b = j % kRing, rb = j & 1;
+      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform: kh is fixed per warp
+      // keys of a key block clipped by the grid's edge (read before the wait)
+      uint32_t members = 0xffffffffu;
+      if (g.partial && valid)
+        members = uint32_t(key_block_members(g, P.zone_shape, __ldg(P.col_idx + beg + j * kKB + kh)) >> (ch * 32));
       mbar_wait_abortable(&s_full[b], (j / kRing) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t r[32];
@@ -298,7 +303,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);
-      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform: kh is fixed per warp
+      mask_scores32(r, members);
       float mx = -INFINITY;
       if (valid) {
         // two chains of three-input maxima over r[0..29], then r[30], r[31]
@@ -343,8 +348,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         }
       }
       uint32_t pk[16];
-      if (valid) {  // m_run is finite here: it includes this thread's finite maximum
-        const float c = P.scale_log2, nm = -m_run;
+      if (valid) {
+        // m_run is finite unless every key so far lay outside the grid (then every p is 0)
+        const float c = P.scale_log2, nm = m_run == -INFINITY ? 0.f : -m_run;
         float lsum = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -377,6 +383,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     const int sI = safe_shape(g, P.zone_shape, I, status);
     const BlockBox qb = block_box(g, sI, I);
     const int tok = block_token(g, qb, m);
+    // a query slot outside the grid (a block clipped by the edge) has no output
+    const bool row_in = !g.partial || block_slot_in_grid(g, qb, m);
     // This lane holds the key-block-kh part of O row m over channels
     // [ch*D/2, ch*D/2 + D/2). It keeps the quarter [.. + kh*D/4, + D/4) and
     // hands the other quarter to the thread of the other lane half.
@@ -407,15 +415,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
 #pragma unroll
       for (int i = 0; i < NC; ++i) ov[i] = 0.f;
     }
-    store_row<NC>(P.o, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, ov, P.out_fp32);
-    if (P.o_lo) {
+    if (row_in) store_row<NC>(P.o, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, ov, P.out_fp32);
+    if (P.o_lo && row_in) {
       // what the bf16 store of O dropped: O = o + o_lo to about 16 bits
       float lo[NC];
 #pragma unroll
       for (int i = 0; i < NC; ++i) lo[i] = ov[i] - __bfloat162float(__float2bfloat16_rn(ov[i]));
       store_row<NC>(P.o_lo, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, lo, false);
     }
-    if (q4 == 0) {
+    if (q4 == 0 && row_in) {
       const int N = g.T * g.H * g.W;
       P.lse[int64_t(head) * N + tok] = (l > 0.f && ok) ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }

@@ -6,6 +6,11 @@
 // block id is z * blocks_per_zone + local id. Tokens inside a block are
 // raster (t, h, w), token id n = (t * H + h) * W + w. (Prism README,
 // "Overview": spatiotemporal macro-zones with a tailored block shape each.)
+//
+// A grid that is not a whole number of zones is tiled as if rounded up: the
+// last zone along such an axis, and the block boxes in it, are clipped to the
+// grid. A block's members are the slots of its box inside the grid; a box with
+// none is an empty block. `partial` is set when any axis is clipped.
 #pragma once
 #include <cstdint>
 
@@ -27,6 +32,7 @@ struct Geo {
   int Zt, Zh, Zw;
   int nzt, nzh, nzw;
   int n_zones, bpz, n_blocks;
+  int partial;  // some extent is not a multiple of the zone
   int n_cand;
   int cand[kMaxCand][3];
 };
@@ -70,5 +76,43 @@ __host__ __device__ __forceinline__ int block_token(const Geo& g, const BlockBox
 }
 
 __host__ __device__ __forceinline__ int zone_of_block(const Geo& g, int b) { return b / g.bpz; }
+
+// True when the r-th slot (raster inside the box) of a block lies in the grid.
+__host__ __device__ __forceinline__ bool block_slot_in_grid(const Geo& g, const BlockBox& bb, int r) {
+  const int rt = r / (bb.bh * bb.bw);
+  const int rr = r - rt * bb.bh * bb.bw;
+  const int rh = rr / bb.bw;
+  const int rw = rr - rh * bb.bw;
+  return bb.t0 + rt < g.T && bb.h0 + rh < g.H && bb.w0 + rw < g.W;
+}
+
+// The box's slots inside the grid as a 64-bit mask (bit r = slot r).
+__host__ __device__ __forceinline__ uint64_t block_slot_mask(const Geo& g, const BlockBox& bb) {
+  const int vt = g.T - bb.t0 < bb.bt ? (g.T - bb.t0 > 0 ? g.T - bb.t0 : 0) : bb.bt;
+  const int vh = g.H - bb.h0 < bb.bh ? (g.H - bb.h0 > 0 ? g.H - bb.h0 : 0) : bb.bh;
+  const int vw = g.W - bb.w0 < bb.bw ? (g.W - bb.w0 > 0 ? g.W - bb.w0 : 0) : bb.bw;
+  if (vt == bb.bt && vh == bb.bh && vw == bb.bw) return ~uint64_t(0);
+  const uint64_t row = vw >= 64 ? ~uint64_t(0) : ((uint64_t(1) << vw) - 1);
+  uint64_t m = 0;
+  for (int rt = 0; rt < vt; ++rt)
+    for (int rh = 0; rh < vh; ++rh) m |= row << ((rt * bb.bh + rh) * bb.bw);
+  return m;
+}
+
+// Extents of zone z clipped to the grid.
+__host__ __device__ __forceinline__ void zone_extents(const Geo& g, int z, int* et, int* eh, int* ew) {
+  const int zt = z / (g.nzh * g.nzw), zr = z - zt * g.nzh * g.nzw;
+  const int zh = zr / g.nzw, zw = zr - zh * g.nzw;
+  *et = g.T - zt * g.Zt < g.Zt ? g.T - zt * g.Zt : g.Zt;
+  *eh = g.H - zh * g.Zh < g.Zh ? g.H - zh * g.Zh : g.Zh;
+  *ew = g.W - zw * g.Zw < g.Zw ? g.W - zw * g.Zw : g.Zw;
+}
+
+// True when zone z lies wholly inside the grid.
+__host__ __device__ __forceinline__ bool zone_is_whole(const Geo& g, int z) {
+  int et, eh, ew;
+  zone_extents(g, z, &et, &eh, &ew);
+  return et == g.Zt && eh == g.Zh && ew == g.Zw;
+}
 
 }  // namespace prism

@@ -13,7 +13,6 @@ prism_status make_geo(const prism_geometry* geo, Geo* out) {
   if (!geo || !out || !geo->cand) return PRISM_ERR_ARG;
   const prism_dim3 g = geo->grid, z = geo->zone;
   if (g.t <= 0 || g.h <= 0 || g.w <= 0 || z.t <= 0 || z.h <= 0 || z.w <= 0) return PRISM_ERR_SHAPE;
-  if (g.t % z.t || g.h % z.h || g.w % z.w) return PRISM_ERR_SHAPE;
   const int64_t zvol = int64_t(z.t) * z.h * z.w;
   if (zvol % kBlockTokens) return PRISM_ERR_SHAPE;
   if (zvol > kMaxZoneTokens) return PRISM_ERR_UNSUPPORTED;
@@ -24,8 +23,12 @@ prism_status make_geo(const prism_geometry* geo, Geo* out) {
   std::memset(&r, 0, sizeof(r));
   r.T = g.t; r.H = g.h; r.W = g.w;
   r.Zt = z.t; r.Zh = z.h; r.Zw = z.w;
-  r.nzt = g.t / z.t; r.nzh = g.h / z.h; r.nzw = g.w / z.w;
-  r.n_zones = r.nzt * r.nzh * r.nzw;
+  // zones tile the grid rounded up to whole zones; the last along an axis may be clipped
+  r.nzt = (g.t + z.t - 1) / z.t; r.nzh = (g.h + z.h - 1) / z.h; r.nzw = (g.w + z.w - 1) / z.w;
+  r.partial = (g.t % z.t) || (g.h % z.h) || (g.w % z.w);
+  const int64_t nz = int64_t(r.nzt) * r.nzh * r.nzw;
+  if (nz * (zvol / kBlockTokens) >= (int64_t(1) << 31)) return PRISM_ERR_UNSUPPORTED;
+  r.n_zones = int(nz);
   r.bpz = int(zvol / kBlockTokens);
   r.n_blocks = r.n_zones * r.bpz;
   r.n_cand = geo->n_cand;

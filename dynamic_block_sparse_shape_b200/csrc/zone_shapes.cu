@@ -343,21 +343,24 @@ __global__ void __launch_bounds__(256) zone_res_kernel(const Geo g, const float*
   const int z = blockIdx.x;
   const int zt = z / (g.nzh * g.nzw), zr = z - zt * g.nzh * g.nzw;
   const int zh = zr / g.nzw, zw = zr - zh * g.nzw;
-  const int zvol = g.Zt * g.Zh * g.Zw, HW = g.Zh * g.Zw;
+  // the zone's extents clipped to the grid (whole zones: Zt, Zh, Zw)
+  int Et, Eh, Ew;
+  zone_extents(g, z, &Et, &Eh, &Ew);
+  const int zvol = Et * Eh * Ew, HW = Eh * Ew;
   for (int i = threadIdx.x; i < zvol; i += blockDim.x) {
-    const int t = i / HW, h = (i / g.Zw) % g.Zh, w = i % g.Zw;
+    const int t = i / HW, h = (i / Ew) % Eh, w = i % Ew;
     rz[i] = r[((zt * g.Zt + t) * g.H + zh * g.Zh + h) * g.W + zw * g.Zw + w];
   }
   __syncthreads();
   double acc[4] = {0, 0, 0, 0};
   for (int a = 0; a < 3; ++a) {
-    const int La = a == 0 ? g.Zt : (a == 1 ? g.Zh : g.Zw);
+    const int La = a == 0 ? Et : (a == 1 ? Eh : Ew);
     const int nlines = zvol / La;
     for (int line = threadIdx.x; line < nlines; line += blockDim.x) {
       int r0, step;
       if (a == 0) { r0 = line; step = HW; }
-      else if (a == 1) { const int t = line / g.Zw; r0 = t * HW + (line - t * g.Zw); step = g.Zw; }
-      else { r0 = line * g.Zw; step = 1; }
+      else if (a == 1) { const int t = line / Ew; r0 = t * HW + (line - t * Ew); step = Ew; }
+      else { r0 = line * Ew; step = 1; }
       double mean = 0;
       for (int i = 0; i < La; ++i) mean += rz[r0 + i * step];
       mean /= La;
@@ -430,8 +433,12 @@ __global__ void __launch_bounds__(32 * kChooseWarps) choose_kernel(const Geo g, 
     if (zone_margin) zone_margin[z] = INFINITY;
     return;
   }
-  const double zvol = double(g.Zt) * g.Zh * g.Zw;
-  const double Z[3] = {double(g.Zt), double(g.Zh), double(g.Zw)};
+  // line lengths and member count of the zone clipped to the grid; the channel
+  // partial sums count only member tokens (the TMA copy fills the rest with 0)
+  int Et, Eh, Ew;
+  zone_extents(g, z, &Et, &Eh, &Ew);
+  const double zvol = double(Et) * Eh * Ew;
+  const double Z[3] = {double(Et), double(Eh), double(Ew)};
   double V[3] = {0, 0, 0}, A[3] = {0, 0, 0};
   if (have_feat)
     for (int a = 0; a < 3; ++a) V[a] = (q[3] - q[a] / Z[a]) / (zvol * feat_c);

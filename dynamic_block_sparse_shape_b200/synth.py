@@ -19,6 +19,9 @@ training, 24 heads of width 128, 3072-wide hidden states):
 * ``720p``: grid 16x48x80, 24 heads, d=128, bf16, Q/K = 8 sinusoids + noise.
 * ``1080p``: grid 16x72x128, plus video features and an a2v residual.
 * ``2k``: grid 32x72x128, the 1080p recipe on the 2K latent grid.
+* ``720p-latent`` / ``2k-latent``: grids 16x45x80 and 32x90x160, the real
+  latent sizes of 720p and 2K frames, whose 45 / 90 rows are not a whole
+  number of 8-token zones; the 1080p recipe otherwise.
 """
 from __future__ import annotations
 
@@ -69,6 +72,12 @@ WORKLOADS = {
     # working set (~4.8 GB) stays small enough for profiler captures of the selection path
     "2k-stats": Workload("2k-stats", (32, 72, 128), 2, 128, "bf16", (8, 8, 8), 4, 0.20, True, "synthetic", True,
                          seed=3),
+    # the real VAE latent grids (16x spatial, 4x temporal downsampling): 720p gives 45 x 80 tokens per frame,
+    # 2K (2560 x 1440) 90 x 160; 45 and 90 are not multiples of the 8-token zone, so the last zone row is clipped
+    "720p-latent": Workload("720p-latent", (16, 45, 80), 24, 128, "bf16", (8, 8, 8), 4, 0.20, True, "synthetic",
+                            True, seed=5),
+    "2k-latent": Workload("2k-latent", (32, 90, 160), 24, 128, "bf16", (8, 8, 8), 4, 0.20, True, "synthetic", True,
+                          seed=6),
 }
 
 
@@ -159,7 +168,8 @@ def video_features(wl: Workload, channels=3072, device="cpu", base_amplitude=0.5
     gen = make_generator(1000 + wl.seed, device)
     T, H, W = wl.grid
     Zt, Zh, Zw = wl.zone
-    nt, nh, nw = T // Zt, H // Zh, W // Zw
+    # zones tile the grid rounded up (the last one per axis may be clipped)
+    nt, nh, nw = -(-T // Zt), -(-H // Zh), -(-W // Zw)
     nz = nt * nh * nw
     x = sinusoid_field(wl.grid, channels, 8, 1.0, 4, gen, device)  # fp32 [N, C]
     dom = torch.randint(0, 3, (nz,), generator=gen, device=device)

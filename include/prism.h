@@ -22,6 +22,17 @@
  *   (Zt/bt, Zh/bh, Zw/bw) sub-grid; global block id = z * blocks_per_zone +
  *   local id, blocks_per_zone = Zt*Zh*Zw/64. Tokens inside a block are raster
  *   (t, h, w). Query and key blocks use the same partition.
+ * - Grids that are not a whole number of zones (real video latents, e.g. 45
+ *   latent rows at 720p; the Prism pages train at 720p, 1080p and 2K and do
+ *   not say how edges are tiled; this is the library's reading): zones tile
+ *   the grid rounded up to whole zones, so n_zones = prod ceil(extent/zone),
+ *   and the last zone along a clipped axis covers only the grid's remainder.
+ *   Block boxes tile the unclipped zone as above and keep their ids; a block's
+ *   members are the slots of its box inside the grid (fewer than 64 at the
+ *   edge), and a box with no member is an empty block. Zone statistics use the
+ *   member tokens (lines clipped), pooling averages the members (an empty
+ *   block's pooled row is NaN), the selection never keeps an empty block and
+ *   leaves its row empty, and attention runs over member tokens only.
  * - Q, K, V, O, dO, dQ, dK, dV are token-major [N, heads, head_dim] with a
  *   token stride of `tok_stride` elements (>= heads*head_dim, a multiple of 8)
  *   and contiguous heads and channels.
@@ -74,8 +85,9 @@ typedef struct {
 } prism_dim3;
 
 /* Token-grid geometry shared by the block-level entry points.
- * grid: latent token grid (T, H, W); zone: macro-zone extents (Zt, Zh, Zw),
- * dividing the grid, with Zt*Zh*Zw a multiple of 64 and at most 512;
+ * grid: latent token grid (T, H, W); zone: macro-zone extents (Zt, Zh, Zw)
+ * (need not divide the grid, see above), with Zt*Zh*Zw a multiple of 64 and
+ * at most 512;
  * cand: host array of n_cand (1..16) candidate block shapes. */
 typedef struct {
   prism_dim3 grid;
@@ -212,7 +224,10 @@ PRISM_API prism_status prism_block_pool(const prism_geometry* geo, const int32_t
  * top_k >= n_blocks or cdf_threshold >= 1 keeps every block. Scores are never
  * written to memory.
  *
- * q_pool, k_pool: device float [heads, n_blocks, head_dim].
+ * q_pool, k_pool: device float [heads, n_blocks, head_dim]; n_blocks at most
+ *       10240 and heads * n_blocks^2 below 2^31 (PRISM_ERR_UNSUPPORTED
+ *       otherwise). A NaN pooled row marks an empty block (see the
+ *       conventions): never kept as a key; as a query its row is empty.
  * top_k >= 1; cdf_threshold >= 0.
  * mask: device uint32 [heads, n_blocks, ceil(n_blocks/32)] out; bit (J % 32)
  *       of word J / 32 of row (h, I) is set when J is kept.

@@ -49,8 +49,12 @@ def _geo(grid=(32, 72, 128), zone=(8, 8, 8), cand=DEFAULT_CANDIDATES):
 def test_geometry_counts_and_errors(lib):
     assert _geo().counts() == (576, 4608)
     assert _geo((4, 8, 8), (4, 8, 8), [(4, 4, 4)]).counts() == (1, 4)
+    # grids that are not whole zones: zones tile the grid rounded up
+    from oracle import prism_oracle as O
+    for grid in ((32, 72, 127), (16, 45, 80), (32, 90, 160), (1, 1, 1), (9, 17, 8)):
+        nz = int(np.prod(O.zone_counts(grid, (8, 8, 8))))
+        assert _geo(grid, (8, 8, 8), DEFAULT_CANDIDATES).counts() == (nz, 8 * nz), grid
     bad = [
-        ((32, 72, 127), (8, 8, 8), DEFAULT_CANDIDATES, 2),  # grid not divisible by the zone
         ((32, 72, 128), (8, 8, 8), [(4, 4, 2)], 2),  # candidate volume != 64
         ((32, 72, 128), (8, 8, 8), [(16, 2, 2)], 2),  # candidate does not divide the zone
         ((32, 64, 128), (16, 16, 16), [(4, 4, 4)], 9),  # zone larger than 512 tokens
@@ -83,7 +87,7 @@ def test_host_validation_codes(lib):
     assert sel(fake, fake, 24, 4608, 128, 0.088, 0, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 1
     assert sel(fake, fake, 24, 4608, 128, 0.088, 4, -0.1, fake, fake, fake, None, 0, None, ws, 256, None) == 1
     assert sel(fake, fake, 24, 4608, 96, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 9
-    assert sel(fake, fake, 24, 9000, 128, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 9
+    assert sel(fake, fake, 24, 10241, 128, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 9
     assert sel(fake, fake, 24, 4608, 128, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, None, 256, None) == 4
     assert sel(None, fake, 24, 4608, 128, 0.088, 4, 0.2, fake, fake, fake, None, 0, None, ws, 256, None) == 1
     # block_pool: dtype, head_dim, token stride

@@ -235,17 +235,22 @@ def _selection_parity(qp, kp, sc, top_k, tau, qpr, kpr, key_bias=None, key_bias_
     assert np.array_equal(kept[qual], ref["kept"][qual])
     # every row: kept >= its head's k, popcount == kept, and any difference from
     # the oracle lies among blocks whose logits are within 5e-2 of the boundary
+    # empty blocks (NaN pooled features, grids clipped at an edge) take no part
+    present = ~np.isnan(kpr).any(axis=2)
+    empty_row = np.isnan(qpr).any(axis=2)
     ks = np.broadcast_to(np.asarray(top_k), (H,))
-    assert np.all(kept >= np.minimum(ks, nb)[:, None])
+    floor = np.where(empty_row, 0, np.minimum(ks, present.sum(axis=1))[:, None])
+    assert np.all(kept >= floor) and np.all(kept[empty_row] == 0)
+    assert not (got & ~present[:, None, :]).any()
     assert np.array_equal(got.sum(axis=2), kept)
-    s = O.block_logits(qpr, kpr, sc)
+    s = O.block_logits(np.nan_to_num(qpr), np.nan_to_num(kpr), sc)
     if key_bias_r is not None:
         s = s + np.asarray(key_bias_r)[None, None, :]
     for h, i in zip(*np.nonzero(~qual)):
         diff = got[h, i] ^ ref["mask"][h, i]
         if diff.any():
-            order = np.sort(s[h, i])[::-1]
-            bound = order[min(ref["kept"][h, i], nb) - 1]
+            order = np.sort(s[h, i][present[h]])[::-1]
+            bound = order[min(ref["kept"][h, i], present[h].sum()) - 1]
             assert np.all(np.abs(s[h, i][diff] - bound) < 5e-2)
     # CSR matches the mask
     rp = sel["row_ptr"].cpu().numpy()
@@ -369,6 +374,103 @@ def test_block_select_with_audio_bias_end_to_end():
     # fewer blocks: the softmax mass concentrates on them)
     share = lambda m: m[:, :, loud].sum() / m.sum()
     assert share(biased) > share(plain) and biased.sum() <= plain.sum()
+
+
+# --------------------------------------------------------------------------- grids that are not whole zones
+PARTIAL_GRID, PARTIAL_ZONE = (10, 13, 9), (8, 8, 8)  # every zone axis clipped
+
+
+def _partial_geometry(seed):
+    geo = P.Geometry(PARTIAL_GRID, PARTIAL_ZONE, CAND)
+    nz, nb = geo.counts()
+    zone_shape = np.random.default_rng(seed).integers(0, len(CAND), nz)
+    blocks = O.block_tokens(PARTIAL_GRID, PARTIAL_ZONE, CAND, zone_shape)
+    return geo, nz, nb, zone_shape, blocks
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_attention_partial_grid(d):
+    """Blocks clipped by the grid's edge (fewer than 64 member tokens) as queries
+    and keys, empty blocks inside the selected sets, a row whose only selected
+    block is empty (no keys: O = 0, LSE = -inf), forward and backward."""
+    geo, nz, nb, zone_shape, blocks = _partial_geometry(31 + d)
+    members = (blocks >= 0).sum(axis=1)
+    assert (members == 0).any() and ((members > 0) & (members < 64)).any()
+    rng = np.random.default_rng(d)
+    H = 2
+    mask = rng.random((H, nb, nb)) < 0.3
+    mask[:, np.arange(nb), np.arange(nb)] = True
+    e = int(np.nonzero(members == 0)[0][0])
+    r = int(np.nonzero(members > 0)[0][1])
+    mask[0, r, :] = False
+    mask[0, r, e] = True  # only an empty block
+    gen = torch.Generator().manual_seed(41 + d)
+    N = geo.n_tokens
+    dev = torch.device("cuda")
+    q, k, v, do = (torch.randn((N, H, d), generator=gen).to(torch.bfloat16).to(dev) for _ in range(4))
+    _check_attention(geo, zone_shape, q, k, v, do, mask)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_block_pool_partial_grid(dtype):
+    geo, nz, nb, zone_shape, blocks = _partial_geometry(5)
+    H, d = 4, 128
+    gen = torch.Generator().manual_seed(6)
+    dev = torch.device("cuda")
+    q = torch.randn((geo.n_tokens, H, d), generator=gen).to(dtype)
+    k = torch.randn((geo.n_tokens, H, d), generator=gen).to(dtype)
+    zs = torch.tensor(zone_shape, dtype=torch.int32, device=dev)
+    qp, kp = P.block_pool(geo, zs, q.to(dev), k.to(dev))
+    for got, x in ((qp, q), (kp, k)):
+        ref = O.block_pool(f64(x), blocks)
+        g = f64(got)
+        assert np.array_equal(np.isnan(g), np.isnan(ref))
+        fin = ~np.isnan(ref)
+        assert np.abs(g[fin] - ref[fin]).max() < 2e-6
+
+
+def test_block_select_partial_grid():
+    """Empty blocks are never kept and their rows are empty; clipped blocks
+    take part like whole ones; per-head settings and the bias as well."""
+    geo, nz, nb, zone_shape, blocks = _partial_geometry(7)
+    H, d = 3, 64
+    gen = torch.Generator().manual_seed(8)
+    dev = torch.device("cuda")
+    q = torch.randn((geo.n_tokens, H, d), generator=gen) + 1.5 * torch.randn((1, H, d), generator=gen)
+    k = torch.randn((geo.n_tokens, H, d), generator=gen)
+    zs = torch.tensor(zone_shape, dtype=torch.int32, device=dev)
+    qp, kp = P.block_pool(geo, zs, q.to(dev), k.to(dev))
+    qpr, kpr = O.block_pool(f64(q), blocks), O.block_pool(f64(k), blocks)
+    sc = scale_for(d)
+    for top_k, tau in ((1, 0.2), (3, 0.5), (100, 0.2), (2, 1.0)):
+        _selection_parity(qp, kp, sc, top_k, tau, qpr, kpr)
+    _selection_parity(qp, kp, sc, [1, 4, 2], [0.1, 0.3, 1.0], qpr, kpr)
+    R = torch.randn((geo.n_tokens, 64), generator=gen) * torch.rand((geo.n_tokens, 1), generator=gen)
+    b = P.block_audio_bias(geo, zs, R.to(dev), 2.0)
+    br = O.block_key_bias(f64(R), blocks, 2.0)
+    assert np.allclose(f64(b), br, rtol=1e-5, atol=1e-6)
+    _selection_parity(qp, kp, sc, 2, 0.2, qpr, kpr, key_bias=b, key_bias_r=br)
+
+
+def test_zone_shapes_partial_grid():
+    """The real 720p latent rows (45 = 5 zones + 5) and a clipped t axis."""
+    import dataclasses
+    wl = dataclasses.replace(synth.WORKLOADS["720p-latent"], grid=(12, 45, 32))
+    dev = torch.device("cuda")
+    F = synth.video_features(wl, device=dev)
+    R, _ = synth.a2v_residual(wl, device=dev)
+    geo = P.Geometry(wl.grid, wl.zone, CAND)
+    nz, _ = geo.counts()
+    assert nz == 2 * 6 * 4
+    for feat, res in ((F, R), (F, None), (None, R)):
+        zs, margin = P.zone_shapes(geo, feat=feat, res=res)
+        idx_r, margin_r, st = O.zone_shapes(wl.grid, wl.zone, CAND, F=None if feat is None else f64(feat),
+                                            R=None if res is None else f64(res))
+        got = zs.cpu().numpy()
+        qual = margin_r > 1e-3
+        assert qual.mean() > 0.5
+        assert np.array_equal(got[qual], idx_r[qual])
+        assert np.allclose(margin.cpu().numpy()[qual], margin_r[qual], rtol=1e-3, atol=1e-4)
 
 
 # --------------------------------------------------------------------------- zone shapes
