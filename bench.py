@@ -9,7 +9,12 @@ larger than L2, so no flush is needed between steps.
 
 Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle on a
 bounded sample of the same workload instead. Multi-GPU runs are independent
-replicas (the path has no exchange step); ``value`` is whole-job ms per layer.
+replicas by default (the path has no exchange step; ``value`` is whole-job ms
+per layer, weak scaling). ``--shard heads`` splits one layer's heads across the
+ranks instead (every stage after the zone shapes is per head; each rank
+computes the zone shapes from the replicated features): ``value`` is the
+slowest rank's time for its shard, i.e. ms per layer, strong scaling.
+``--head-slice a:b`` times one such shard alone on one GPU (per-GPU timing).
 """
 from __future__ import annotations
 
@@ -113,10 +118,11 @@ def max_over_ranks(value: float, device="cpu") -> float:
     return float(t.item())
 
 
-def whole_job_ms_per_layer(ms_per_step_max: float, world: int) -> float:
+def whole_job_ms_per_layer(ms_per_step_max: float, world: int, shard: str = "replicas") -> float:
     """Replicas: every rank runs one layer per step, so the job finishes
-    `world` layers in the slowest rank's step time."""
-    return ms_per_step_max / world
+    `world` layers in the slowest rank's step time. Head shards: the ranks
+    together run one layer per step, finished when the slowest rank is."""
+    return ms_per_step_max / world if shard == "replicas" else ms_per_step_max
 
 
 # ---------------------------------------------------------------------------- GPU arm
@@ -425,6 +431,17 @@ def run_gpu(args):
     wl = synth.WORKLOADS[args.config]
     dev = torch.device("cuda", local)
     x, feats, res = build_inputs(wl, dev)
+    full_heads = wl.heads
+    h0, h1 = 0, wl.heads
+    if args.shard == "heads" or args.head_slice:
+        import dataclasses
+        from dynamic_block_sparse_shape_b200.shard import head_shard, parse_head_slice
+        h0, h1 = parse_head_slice(args.head_slice, wl.heads) if args.head_slice else head_shard(wl.heads, world, rank)
+        # this rank's heads of Q, K, V, dO; the features and the residual stay whole (zone shapes on every rank)
+        x = {k: v[:, h0:h1].contiguous() for k, v in x.items()}
+        torch.cuda.empty_cache()
+        wl = dataclasses.replace(wl, heads=h1 - h0)
+    shard = "heads" if (args.shard == "heads" or args.head_slice) else "replicas"
     pipe = Pipeline(wl, x, feats, res)
     for _ in range(args.warmup):
         pipe.step()
@@ -459,13 +476,18 @@ def run_gpu(args):
     achieved = attn_flop / t_attn / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     out = {
-        "metric": METRIC, "value": round(whole_job_ms_per_layer(ms_step, world), 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False, "scaling": "weak",
+        "metric": METRIC, "value": round(whole_job_ms_per_layer(ms_step, world, shard), 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False,
+        "scaling": "strong" if shard == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{wl.name}: grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]} ({wl.n_tokens} tokens), "
                                f"{wl.heads} heads x d{wl.head_dim}, zones {wl.zone}, top_k {wl.top_k}, "
                                f"cdf_threshold {wl.cdf_threshold}, fwd+bwd",
-                   "parallelism": "replicas" if world > 1 else "single",
+                   "parallelism": (f"one shard alone: heads {h0}:{h1} of {full_heads} (per-GPU timing)"
+                                   if args.head_slice else
+                                   f"heads sharded over {world} ranks (rank 0: {h0}:{h1})" if shard == "heads" else
+                                   "replicas" if world > 1 else "single"),
                    "l2": "inputs larger than L2 (each 1.8 GB), no flush"},
         "tflops": round(achieved, 1),
         "selected_pairs": nnz, "density": round(nnz / (wl.heads * pipe.nb * pipe.nb), 4),
@@ -630,6 +652,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="run the 45-point selection/sparsity sweep instead")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="multi-GPU layout: independent replicas, or one layer's heads split across ranks")
+    ap.add_argument("--head-slice", default="", help="a:b, time heads a..b-1 of the layer alone (one shard)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
