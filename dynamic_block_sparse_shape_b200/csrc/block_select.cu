@@ -8,11 +8,11 @@
 // overhead, so the scores here live only in shared memory.
 //
 // select_kernel: one CTA = 8 query blocks of one head (one warp each); 4 when
-// more than 5120 key blocks' logits must fit in shared memory.
+// more than 6912 key blocks' logits must fit in shared memory.
 //   1. logits s_J = scale * qbar_I . kbar_J (+ b_J, the optional key-block
-//      bias, walkthrough section "桥接残差反哺稀疏注意力") for all J, fp32 FFMA,
-//      with the key features staged transposed in shared memory (2 keys x 4
-//      rows per thread per channel);
+//      bias, walkthrough section "桥接残差反哺稀疏注意力") for all J, fp32 FFMA:
+//      a thread streams two keys' pooled features from global memory and
+//      forms their logits against the CTA's rows (shared-memory broadcasts);
 //   2. per row: max, p_J = exp(s_J - max) in place as a ranking key (float
 //      bits + 1; 0 for a NaN logit, which marks an absent block: an empty
 //      block of a grid clipped at its edge), Z = sum p (fp64);
@@ -35,12 +35,9 @@
 namespace prism {
 namespace {
 
-constexpr int kKeyTile = 256;
-constexpr int kDChunk = 32;
-constexpr int kKtPitch = kKeyTile + 2;
-// Rows of logits per CTA live in shared memory: 8 rows up to 5120 key blocks,
+// Rows of logits per CTA live in shared memory: 8 rows up to 6912 key blocks,
 // 4 rows (half the threads) up to 10240 (the 2K latent grid has 7680).
-constexpr int kSelMaxBlocks8 = 5120;
+constexpr int kSelMaxBlocks8 = 6912;
 constexpr int kSelMaxBlocks = 10240;
 constexpr int kSelMaxHeads = 128;  // per-head settings passed as a kernel parameter
 
@@ -70,14 +67,26 @@ __device__ __forceinline__ int warp_sum_i(int v) {
 // like p with every absent block below every present one.
 __device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float(key - 1u); }
 
-// Mass of the entries whose key is >= u >= 1 (fp64, warp-reduced).
+// Mass of the entries whose key is >= u >= 1: four independent fp32 chains per
+// lane (at most nb/128 terms each, relative error below 2e-6 of the row's
+// mass for 10240 entries), combined in fp64 and warp-reduced in a fixed order.
+// The row total Z is this function at u = 1, so the bisection's invariant
+// mass(>= 1) = Z >= tau Z holds exactly.
 __device__ __forceinline__ double mass_at_least(const uint32_t* p, int nb, uint32_t u, int lane) {
-  double acc = 0;
-  for (int j = lane; j < nb; j += 32) {
-    const uint32_t k = p[j];
-    if (k >= u) acc += double(key_value(k));
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int j = lane;
+  for (; j + 96 < nb; j += 128) {
+    const uint32_t k0 = p[j], k1 = p[j + 32], k2 = p[j + 64], k3 = p[j + 96];
+    a0 += k0 >= u ? key_value(k0) : 0.f;
+    a1 += k1 >= u ? key_value(k1) : 0.f;
+    a2 += k2 >= u ? key_value(k2) : 0.f;
+    a3 += k3 >= u ? key_value(k3) : 0.f;
   }
-  return warp_sum_d(acc);
+  for (; j < nb; j += 32) {
+    const uint32_t k = p[j];
+    a0 += k >= u ? key_value(k) : 0.f;
+  }
+  return warp_sum_d((double(a0) + double(a1)) + (double(a2) + double(a3)));
 }
 __device__ __forceinline__ int count_at_least(const uint32_t* p, int nb, uint32_t u, int lane) {
   int c = 0;
@@ -92,9 +101,8 @@ __global__ void __launch_bounds__(ROWS * 32, 1)
                   int32_t* __restrict__ kept) {
   constexpr int kThreads = ROWS * 32;
   extern __shared__ __align__(16) float sm[];
-  float* srow = sm;                                  // [ROWS][nb]
-  float* kT = srow + size_t(ROWS) * nb;              // [kDChunk][kKtPitch]
-  float* qT = kT + kDChunk * kKtPitch;               // [d][ROWS]
+  float* srow = sm;                      // [ROWS][nb]
+  float* qT = srow + size_t(ROWS) * nb;  // [d][ROWS]: one float4 = one channel of 4 rows
   const int head = blockIdx.y;
   const int I0 = blockIdx.x * ROWS;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -104,40 +112,48 @@ __global__ void __launch_bounds__(ROWS * 32, 1)
     const int r = i / d, c = i - r * d;
     qT[c * ROWS + r] = (I0 + r < nb) ? qh[size_t(I0 + r) * d + c] : 0.f;
   }
-  // ---- 1. logits
-  const int kpair = tid & 127, rh = tid >> 7;
-  for (int key0 = 0; key0 < nb; key0 += kKeyTile) {
-    float acc[4][2] = {{0, 0}, {0, 0}, {0, 0}, {0, 0}};
-    for (int c0 = 0; c0 < d; c0 += kDChunk) {
-      __syncthreads();
-      // stage kT[c][j] = kbar[key0 + j][c0 + c], 256 keys x 32 channels
-      for (int i = tid; i < kKeyTile * (kDChunk / 4); i += kThreads) {
-        const int j = i >> 3, q4 = i & 7;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (key0 + j < nb) v = __ldg(reinterpret_cast<const float4*>(kh + size_t(key0 + j) * d + c0) + q4);
-        kT[(q4 * 4 + 0) * kKtPitch + j] = v.x;
-        kT[(q4 * 4 + 1) * kKtPitch + j] = v.y;
-        kT[(q4 * 4 + 2) * kKtPitch + j] = v.z;
-        kT[(q4 * 4 + 3) * kKtPitch + j] = v.w;
-      }
-      __syncthreads();
-#pragma unroll 8
-      for (int c = 0; c < kDChunk; ++c) {
-        const float2 kv = *reinterpret_cast<const float2*>(kT + c * kKtPitch + 2 * kpair);
-        const float4 qv = *reinterpret_cast<const float4*>(qT + (c0 + c) * ROWS + 4 * rh);
-        acc[0][0] = fmaf(qv.x, kv.x, acc[0][0]); acc[0][1] = fmaf(qv.x, kv.y, acc[0][1]);
-        acc[1][0] = fmaf(qv.y, kv.x, acc[1][0]); acc[1][1] = fmaf(qv.y, kv.y, acc[1][1]);
-        acc[2][0] = fmaf(qv.z, kv.x, acc[2][0]); acc[2][1] = fmaf(qv.z, kv.y, acc[2][1]);
-        acc[3][0] = fmaf(qv.w, kv.x, acc[3][0]); acc[3][1] = fmaf(qv.w, kv.y, acc[3][1]);
+  __syncthreads();
+  // ---- 1. logits. A thread owns key pairs (k0, k0 + 1), k0 = 2 * (tid + i * kThreads), and streams their
+  // pooled features straight from global memory (no reuse across threads, so no staging): two 16-byte
+  // loads per key cover a whole 32-byte sector, with four steps of them in flight; the CTA's query rows
+  // are shared-memory broadcasts. Channels accumulate in ascending order, one chain per (row, key).
+  for (int k0 = 2 * tid; k0 < nb; k0 += 2 * kThreads) {
+    const int k1 = k0 + 1 < nb ? k0 + 1 : k0;  // a ragged tail recomputes k0, and stores nothing for it
+    const float4* r0 = reinterpret_cast<const float4*>(kh + size_t(k0) * d);
+    const float4* r1 = reinterpret_cast<const float4*>(kh + size_t(k1) * d);
+    float a0[ROWS], a1[ROWS];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) a0[r] = a1[r] = 0.f;
+#pragma unroll 4
+    for (int c8 = 0; c8 < d / 8; ++c8) {
+      const float4 x0 = __ldg(r0 + 2 * c8), x1 = __ldg(r0 + 2 * c8 + 1);
+      const float4 y0 = __ldg(r1 + 2 * c8), y1 = __ldg(r1 + 2 * c8 + 1);
+      const float xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const float ya[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float* qc = qT + (8 * c8 + i) * ROWS;
+#pragma unroll
+        for (int r4 = 0; r4 < ROWS / 4; ++r4) {
+          const float4 qv = *reinterpret_cast<const float4*>(qc + 4 * r4);
+          a0[4 * r4 + 0] = fmaf(qv.x, xa[i], a0[4 * r4 + 0]);
+          a0[4 * r4 + 1] = fmaf(qv.y, xa[i], a0[4 * r4 + 1]);
+          a0[4 * r4 + 2] = fmaf(qv.z, xa[i], a0[4 * r4 + 2]);
+          a0[4 * r4 + 3] = fmaf(qv.w, xa[i], a0[4 * r4 + 3]);
+          a1[4 * r4 + 0] = fmaf(qv.x, ya[i], a1[4 * r4 + 0]);
+          a1[4 * r4 + 1] = fmaf(qv.y, ya[i], a1[4 * r4 + 1]);
+          a1[4 * r4 + 2] = fmaf(qv.z, ya[i], a1[4 * r4 + 2]);
+          a1[4 * r4 + 3] = fmaf(qv.w, ya[i], a1[4 * r4 + 3]);
+        }
       }
     }
+    const float b0 = kbias ? __ldg(kbias + k0) : 0.f;
+    const float b1 = kbias ? __ldg(kbias + k1) : 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int key = key0 + 2 * kpair + j;
-        if (key < nb) srow[size_t(4 * rh + i) * nb + key] = acc[i][j] * scale + (kbias ? __ldg(kbias + key) : 0.f);
-      }
+    for (int r = 0; r < ROWS; ++r) {
+      srow[size_t(r) * nb + k0] = a0[r] * scale + b0;
+      if (k1 != k0) srow[size_t(r) * nb + k1] = a1[r] * scale + b1;
+    }
   }
   __syncthreads();
   // ---- 2..5. one warp per query block
@@ -153,7 +169,6 @@ __global__ void __launch_bounds__(ROWS * 32, 1)
   for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, sl[j]);  // fmaxf skips NaN
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  double zacc = 0;
   int n_present = 0;
   for (int j0 = 0; j0 < nb; j0 += 32) {
     const int j = j0 + lane;
@@ -164,14 +179,13 @@ __global__ void __launch_bounds__(ROWS * 32, 1)
         float e = expf(s - mx);
         if (!(e >= 0.f)) e = 0.f;  // every present logit -inf: no mass
         key = __float_as_uint(e) + 1u;
-        zacc += double(e);
       }
       p[j] = key;
     }
     n_present += __popc(__ballot_sync(0xffffffffu, key != 0u));
   }
-  const double Z = warp_sum_d(zacc);
   __syncwarp();
+  const double Z = mass_at_least(p, nb, 1u, lane);
   if (n_present == 0) {  // an empty query block (or no present key): empty row
     for (int w = lane; w < words; w += 32) mrow[w] = 0u;
     if (lane == 0) kept[size_t(head) * nb + I] = 0;
@@ -351,8 +365,7 @@ prism_status block_select_impl(const float* q_pool, const float* k_pool, int32_t
   if (col_idx && col_cap < 0) return PRISM_ERR_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int rows_per_cta = n_blocks <= kSelMaxBlocks8 ? 8 : 4;
-  const size_t smem =
-      (size_t(rows_per_cta) * n_blocks + kDChunk * kKtPitch + size_t(head_dim) * rows_per_cta) * sizeof(float);
+  const size_t smem = (size_t(rows_per_cta) * n_blocks + size_t(head_dim) * rows_per_cta) * sizeof(float);
   const dim3 grid((n_blocks + rows_per_cta - 1) / rows_per_cta, heads);
   if (rows_per_cta == 8) {
     if (cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
