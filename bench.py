@@ -172,6 +172,7 @@ class Pipeline:
         self.zone_margin = torch.empty(self.nz, dtype=torch.float32, device=dev)
         self.ws.ensure(P.workspace_size("zone_shapes", self.geo, feat_c=feats.shape[1] if feats is not None else 0,
                                         res_c=res.shape[1] if res is not None else 0))
+        self.ws.ensure(P.workspace_size("block_select", self.geo, heads=H, head_dim=d))
         # size the CSR and the workspaces from one selection pass
         self.stage_zone()
         self.stage_pool()
@@ -180,6 +181,7 @@ class Pipeline:
         self.col_idx = torch.empty(max(1, self.nnz), dtype=torch.int32, device=dev)
         need = max(P.workspace_size("zone_shapes", self.geo, feat_c=feats.shape[1] if feats is not None else 0,
                                     res_c=res.shape[1] if res is not None else 0),
+                   P.workspace_size("block_select", self.geo, heads=H, head_dim=d),
                    P.workspace_size("bsa_fwd", self.geo, heads=H, head_dim=d),
                    P.workspace_size("bsa_bwd", self.geo, heads=H, head_dim=d, nnz=self.nnz))
         self.ws.ensure(need)

@@ -17,7 +17,8 @@ import torch
 
 __all__ = [
     "PrismError", "Geometry", "ShapeParams", "lib", "library_path", "workspace_size", "Workspace", "zone_shapes",
-    "block_pool", "block_select", "block_select_ex", "topk_from_sparsity", "block_audio_bias", "mask_to_csr",
+    "block_pool", "block_select", "block_select_ex", "select_workspace_size", "topk_from_sparsity",
+    "block_audio_bias", "mask_to_csr",
     "bsa_fwd", "bsa_bwd", "check_device_status", "STATUS", "OP", "DEFAULT_CDF_THRESHOLD",
 ]
 
@@ -82,6 +83,7 @@ _SIGNATURES = {
     "prism_block_select_ex": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _F32, ctypes.POINTER(_SelectParams), _P, _P,
                                              _P, _P, _I64, ctypes.POINTER(_I64), _P, _SZ, _P]),
     "prism_topk_from_sparsity": (ctypes.c_int, [_F32, _I32, ctypes.POINTER(_I32)]),
+    "prism_block_select_workspace_size": (ctypes.c_int, [_I32, _I32, _I32, ctypes.POINTER(_SZ)]),
     "prism_block_audio_bias": (ctypes.c_int, [_GEO, _P, _P, _I64, _I32, ctypes.c_int, _F32, _P, _P, _SZ, _P]),
     "prism_mask_to_csr": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _I64, _P, _SZ, _P]),
     "prism_bsa_fwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32, _P, _P, _P, _P,
@@ -255,6 +257,14 @@ def block_pool(geo: Geometry, zone_shape: torch.Tensor, q: torch.Tensor, k: torc
     return qp, kp
 
 
+def select_workspace_size(heads: int, n_blocks: int, head_dim: int) -> int:
+    """Workspace bytes of block_select / block_select_ex for these pooled shapes."""
+    b = _SZ()
+    _check(lib().prism_block_select_workspace_size(int(heads), int(n_blocks), int(head_dim), ctypes.byref(b)),
+           "prism_block_select_workspace_size")
+    return int(b.value)
+
+
 def block_select(qp: torch.Tensor, kp: torch.Tensor, scale: float, top_k: int,
                  cdf_threshold: float = DEFAULT_CDF_THRESHOLD, ws: Optional[Workspace] = None, csr: bool = True,
                  stream=None):
@@ -264,7 +274,7 @@ def block_select(qp: torch.Tensor, kp: torch.Tensor, scale: float, top_k: int,
     H, nb, d = qp.shape
     words = (nb + 31) // 32
     dev = qp.device
-    ws = (ws or Workspace(dev)).ensure(256)
+    ws = (ws or Workspace(dev)).ensure(select_workspace_size(H, nb, d))
     mask = torch.empty((H, nb, words), dtype=torch.int32, device=dev)
     kept = torch.empty((H, nb), dtype=torch.int32, device=dev)
     row_ptr = torch.empty(H * nb + 1, dtype=torch.int32, device=dev)
@@ -290,7 +300,7 @@ def block_select_ex(qp: torch.Tensor, kp: torch.Tensor, scale: float, top_k,
     H, nb, d = qp.shape
     words = (nb + 31) // 32
     dev = qp.device
-    ws = (ws or Workspace(dev)).ensure(256)
+    ws = (ws or Workspace(dev)).ensure(select_workspace_size(H, nb, d))
     cp = _SelectParams()
     keep = []
     if isinstance(top_k, (int,)) or (torch.is_tensor(top_k) and top_k.dim() == 0):

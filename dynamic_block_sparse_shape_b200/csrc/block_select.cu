@@ -7,12 +7,14 @@
 // paper page: computing and materialising the proxy scores is the routing
 // overhead, so the scores here live only in shared memory.
 //
-// select_kernel: one CTA = 8 query blocks of one head (one warp each); 4 when
-// more than 6912 key blocks' logits must fit in shared memory.
+// select_kernel: one CTA = 8 query blocks of one head; 4 when more than 6912
+// key blocks' logits must fit in shared memory. Two warps per row compute the
+// logits; then one warp per row selects.
 //   1. logits s_J = scale * qbar_I . kbar_J (+ b_J, the optional key-block
 //      bias, walkthrough section "桥接残差反哺稀疏注意力") for all J, fp32 FFMA:
-//      a thread streams two keys' pooled features from global memory and
-//      forms their logits against the CTA's rows (shared-memory broadcasts);
+//      a thread streams four keys of the workspace's transposed pooled keys
+//      (coalesced 512-byte warp reads per channel) and forms their logits
+//      against the CTA's rows (shared-memory broadcasts);
 //   2. per row: max, p_J = exp(s_J - max) in place as a ranking key (float
 //      bits + 1; 0 for a NaN logit, which marks an absent block: an empty
 //      block of a grid clipped at its edge), Z = sum p (fp64);
@@ -24,6 +26,7 @@
 //      "实际案例与上手参考": the top-k part of the selection is a tunable ratio);
 //   5. the kept set (ranked by p descending, ties to the lower J) is written
 //      as a bitmask row with warp ballots, and kept[row] = m.
+// transpose_keys_kernel: k_pool per head into key-major order in the workspace.
 // scan_kernel: exclusive scan of kept into the CSR row_ptr (one CTA).
 // fill_kernel: one warp per row expands the bitmask into ascending col_idx.
 #include <algorithm>
@@ -95,11 +98,12 @@ __device__ __forceinline__ int count_at_least(const uint32_t* p, int nb, uint32_
 }
 
 template <int ROWS>
-__global__ void __launch_bounds__(ROWS * 32, 1)
-    select_kernel(const float* __restrict__ qp, const float* __restrict__ kp, int nb, int d, float scale,
+__global__ void __launch_bounds__(ROWS * 64, 1)
+    select_kernel(const float* __restrict__ qp, const float* __restrict__ kT, int nb, int nbp, int d, float scale,
                   const __grid_constant__ SelHeads hp, const float* __restrict__ kbias, uint32_t* __restrict__ mask,
                   int32_t* __restrict__ kept) {
-  constexpr int kThreads = ROWS * 32;
+  // two warps per row: all of them stream logits (more loads in flight), one per row selects
+  constexpr int kThreads = ROWS * 64;
   extern __shared__ __align__(16) float sm[];
   float* srow = sm;                      // [ROWS][nb]
   float* qT = srow + size_t(ROWS) * nb;  // [d][ROWS]: one float4 = one channel of 4 rows
@@ -107,58 +111,51 @@ __global__ void __launch_bounds__(ROWS * 32, 1)
   const int I0 = blockIdx.x * ROWS;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* qh = qp + size_t(head) * nb * d;
-  const float* kh = kp + size_t(head) * nb * d;
   for (int i = tid; i < ROWS * d; i += kThreads) {
     const int r = i / d, c = i - r * d;
     qT[c * ROWS + r] = (I0 + r < nb) ? qh[size_t(I0 + r) * d + c] : 0.f;
   }
   __syncthreads();
-  // ---- 1. logits. A thread owns key pairs (k0, k0 + 1), k0 = 2 * (tid + i * kThreads), and streams their
-  // pooled features straight from global memory (no reuse across threads, so no staging): two 16-byte
-  // loads per key cover a whole 32-byte sector, with four steps of them in flight; the CTA's query rows
-  // are shared-memory broadcasts. Channels accumulate in ascending order, one chain per (row, key).
-  for (int k0 = 2 * tid; k0 < nb; k0 += 2 * kThreads) {
-    const int k1 = k0 + 1 < nb ? k0 + 1 : k0;  // a ragged tail recomputes k0, and stores nothing for it
-    const float4* r0 = reinterpret_cast<const float4*>(kh + size_t(k0) * d);
-    const float4* r1 = reinterpret_cast<const float4*>(kh + size_t(k1) * d);
-    float a0[ROWS], a1[ROWS];
+  // ---- 1. logits. kT is the head's pooled keys transposed, [d][nbp]: for channel c a warp reads 32 x 4
+  // consecutive keys (512 contiguous bytes). A thread owns keys k0 .. k0+3, k0 = 4 * (tid + i * kThreads),
+  // and forms their logits against the CTA's rows (shared-memory broadcasts). Channels accumulate in
+  // ascending order, one chain per (row, key).
+  const float* kTh = kT + size_t(head) * d * nbp;
+  for (int k0 = 4 * tid; k0 < nb; k0 += 4 * kThreads) {
+    float a[ROWS][4];
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) a0[r] = a1[r] = 0.f;
-#pragma unroll 4
-    for (int c8 = 0; c8 < d / 8; ++c8) {
-      const float4 x0 = __ldg(r0 + 2 * c8), x1 = __ldg(r0 + 2 * c8 + 1);
-      const float4 y0 = __ldg(r1 + 2 * c8), y1 = __ldg(r1 + 2 * c8 + 1);
-      const float xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      const float ya[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+    for (int r = 0; r < ROWS; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < d; ++c) {
+      const float4 kv = __ldg(reinterpret_cast<const float4*>(kTh + size_t(c) * nbp + k0));
+      const float* qc = qT + c * ROWS;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float* qc = qT + (8 * c8 + i) * ROWS;
+      for (int r4 = 0; r4 < ROWS / 4; ++r4) {
+        const float4 qv = *reinterpret_cast<const float4*>(qc + 4 * r4);
+        const float qs[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-        for (int r4 = 0; r4 < ROWS / 4; ++r4) {
-          const float4 qv = *reinterpret_cast<const float4*>(qc + 4 * r4);
-          a0[4 * r4 + 0] = fmaf(qv.x, xa[i], a0[4 * r4 + 0]);
-          a0[4 * r4 + 1] = fmaf(qv.y, xa[i], a0[4 * r4 + 1]);
-          a0[4 * r4 + 2] = fmaf(qv.z, xa[i], a0[4 * r4 + 2]);
-          a0[4 * r4 + 3] = fmaf(qv.w, xa[i], a0[4 * r4 + 3]);
-          a1[4 * r4 + 0] = fmaf(qv.x, ya[i], a1[4 * r4 + 0]);
-          a1[4 * r4 + 1] = fmaf(qv.y, ya[i], a1[4 * r4 + 1]);
-          a1[4 * r4 + 2] = fmaf(qv.z, ya[i], a1[4 * r4 + 2]);
-          a1[4 * r4 + 3] = fmaf(qv.w, ya[i], a1[4 * r4 + 3]);
+        for (int i = 0; i < 4; ++i) {
+          a[4 * r4 + i][0] = fmaf(qs[i], kv.x, a[4 * r4 + i][0]);
+          a[4 * r4 + i][1] = fmaf(qs[i], kv.y, a[4 * r4 + i][1]);
+          a[4 * r4 + i][2] = fmaf(qs[i], kv.z, a[4 * r4 + i][2]);
+          a[4 * r4 + i][3] = fmaf(qs[i], kv.w, a[4 * r4 + i][3]);
         }
       }
     }
-    const float b0 = kbias ? __ldg(kbias + k0) : 0.f;
-    const float b1 = kbias ? __ldg(kbias + k1) : 0.f;
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-      srow[size_t(r) * nb + k0] = a0[r] * scale + b0;
-      if (k1 != k0) srow[size_t(r) * nb + k1] = a1[r] * scale + b1;
+    for (int jk = 0; jk < 4; ++jk) {
+      const int key = k0 + jk;
+      if (key < nb) {
+        const float bj = kbias ? __ldg(kbias + key) : 0.f;
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) srow[size_t(r) * nb + key] = a[r][jk] * scale + bj;
+      }
     }
   }
   __syncthreads();
   // ---- 2..5. one warp per query block
   const int I = I0 + warp;
-  if (I >= nb) return;
+  if (warp >= ROWS || I >= nb) return;
   const int top_k = hp.per_head ? hp.k[head] : hp.k0;
   const float tau = hp.per_head ? hp.tau[head] : hp.tau0;
   uint32_t* p = reinterpret_cast<uint32_t*>(srow + size_t(warp) * nb);
@@ -270,6 +267,25 @@ __global__ void __launch_bounds__(ROWS * 32, 1)
   if (lane == 0) kept[size_t(head) * nb + I] = m;
 }
 
+// kT[h][c][j] = kp[h][j][c] for j < nb, 0 for nb <= j < nbp (32 x 32 tiles through shared memory).
+__global__ void __launch_bounds__(256) transpose_keys_kernel(const float* __restrict__ kp, int nb, int nbp, int d,
+                                                             float* __restrict__ kT) {
+  __shared__ float tile[32][33];
+  const int h = blockIdx.z, j0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const float* src = kp + size_t(h) * nb * d;
+  float* dst = kT + size_t(h) * d * nbp;
+  for (int r = ty; r < 32; r += 8) {
+    const int j = j0 + r, c = c0 + tx;
+    tile[r][tx] = (j < nb && c < d) ? src[size_t(j) * d + c] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int c = c0 + r, j = j0 + tx;
+    if (c < d && j < nbp) dst[size_t(c) * nbp + j] = tile[tx][r];
+  }
+}
+
 // Exclusive scan of n ints into out[0..n] (out[n] = total), one CTA.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ in, int n, int32_t* __restrict__ out) {
   __shared__ int64_t part[1024];
@@ -330,7 +346,11 @@ __global__ void __launch_bounds__(256) fill_kernel(const uint32_t* __restrict__ 
 
 }  // namespace
 
-size_t block_select_ws_bytes() { return kWsHeader; }
+// The status word, then the pooled keys transposed per head, [heads][d][nbp], nbp = nb rounded up to 4.
+size_t block_select_ws_bytes(int heads, int nb, int d) {
+  const size_t nbp = (size_t(nb) + 3) & ~size_t(3);
+  return kWsHeader + align_up(size_t(heads) * d * nbp * sizeof(float), 256);
+}
 
 cudaError_t launch_exclusive_scan(const int32_t* in, int n, int32_t* out, cudaStream_t s) {
   scan_kernel<<<1, 1024, 0, s>>>(in, n, out);
@@ -361,20 +381,25 @@ prism_status block_select_impl(const float* q_pool, const float* k_pool, int32_t
   if (int64_t(heads) * n_blocks * n_blocks >= (int64_t(1) << 31)) return PRISM_ERR_UNSUPPORTED;
   if (reinterpret_cast<uintptr_t>(q_pool) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16) return PRISM_ERR_ARG;
   if (reinterpret_cast<uintptr_t>(key_bias) % 4) return PRISM_ERR_ARG;
-  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < block_select_ws_bytes(heads, n_blocks, head_dim))
+    return PRISM_ERR_WORKSPACE;
   if (col_idx && col_cap < 0) return PRISM_ERR_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int nbp = (n_blocks + 3) & ~3;
+  float* kT = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kWsHeader);
+  transpose_keys_kernel<<<dim3((nbp + 31) / 32, (head_dim + 31) / 32, heads), 256, 0, s>>>(k_pool, n_blocks, nbp,
+                                                                                        head_dim, kT);
   const int rows_per_cta = n_blocks <= kSelMaxBlocks8 ? 8 : 4;
   const size_t smem = (size_t(rows_per_cta) * n_blocks + size_t(head_dim) * rows_per_cta) * sizeof(float);
   const dim3 grid((n_blocks + rows_per_cta - 1) / rows_per_cta, heads);
   if (rows_per_cta == 8) {
     if (cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
       return PRISM_ERR_CUDA;
-    select_kernel<8><<<grid, 256, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, hp, key_bias, mask, kept);
+    select_kernel<8><<<grid, 512, smem, s>>>(q_pool, kT, n_blocks, nbp, head_dim, scale, hp, key_bias, mask, kept);
   } else {
     if (cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
       return PRISM_ERR_CUDA;
-    select_kernel<4><<<grid, 128, smem, s>>>(q_pool, k_pool, n_blocks, head_dim, scale, hp, key_bias, mask, kept);
+    select_kernel<4><<<grid, 256, smem, s>>>(q_pool, kT, n_blocks, nbp, head_dim, scale, hp, key_bias, mask, kept);
   }
   const int rows = heads * n_blocks;
   if (launch_exclusive_scan(kept, rows, row_ptr, s) != cudaSuccess) return PRISM_ERR_CUDA;
@@ -432,6 +457,13 @@ extern "C" prism_status prism_block_select_ex(const float* q_pool, const float* 
   }
   return block_select_impl(q_pool, k_pool, heads, n_blocks, head_dim, scale, hp, params->key_bias, mask, kept,
                            row_ptr, col_idx, col_cap, total_kept, ws, ws_bytes, stream);
+}
+
+extern "C" prism_status prism_block_select_workspace_size(int32_t heads, int32_t n_blocks, int32_t head_dim,
+                                                          size_t* bytes) {
+  if (!bytes || heads < 1 || n_blocks < 1 || head_dim < 1) return PRISM_ERR_ARG;
+  *bytes = block_select_ws_bytes(heads, n_blocks, head_dim);
+  return PRISM_OK;
 }
 
 extern "C" prism_status prism_topk_from_sparsity(float sparsity, int32_t n_blocks, int32_t* top_k) {

@@ -139,7 +139,8 @@ extern "C" prism_status prism_workspace_size(prism_op op, const prism_geometry* 
       *bytes = zone_shapes_ws_bytes(g, feat_c, in_dtype, res_c);
       return PRISM_OK;
     case PRISM_OP_BLOCK_SELECT:
-      *bytes = block_select_ws_bytes();
+      if (heads < 1 || head_dim < 1) return PRISM_ERR_ARG;
+      *bytes = block_select_ws_bytes(heads, g.n_blocks, head_dim);
       return PRISM_OK;
     case PRISM_OP_BSA_FWD:
       if (heads < 1 || (head_dim != 64 && head_dim != 128)) return PRISM_ERR_ARG;

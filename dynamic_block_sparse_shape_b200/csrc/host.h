@@ -56,7 +56,7 @@ int device_sm_count();
 
 // Workspace bytes of each entry point (header included).
 size_t zone_shapes_ws_bytes(const Geo& g, int feat_c, prism_dtype feat_dtype, int res_c);
-size_t block_select_ws_bytes();
+size_t block_select_ws_bytes(int heads, int nb, int d);
 size_t bsa_fwd_ws_bytes(const Geo& g, int heads, int head_dim, prism_dtype dtype);
 size_t bsa_bwd_ws_bytes(const Geo& g, int heads, int head_dim, prism_dtype dtype, int64_t nnz);
 

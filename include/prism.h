@@ -241,6 +241,10 @@ PRISM_API prism_status prism_block_pool(const prism_geometry* geo, const int32_t
  *       PRISM_ERR_CAPACITY after the sync, with col_idx untouched (this check
  *       needs total_kept != NULL; without it the fill clips at col_cap and
  *       reports PRISM_ERR_DEVICE through prism_check_device_status).
+ * ws: at least prism_workspace_size(PRISM_OP_BLOCK_SELECT, geo, heads,
+ *       head_dim, ...) bytes (equivalently prism_block_select_workspace_size):
+ *       the status word and a key-major copy of k_pool, heads * head_dim *
+ *       ceil4(n_blocks) floats, from which the scores are formed.
  */
 PRISM_API prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
                                 int32_t head_dim, float scale, int32_t top_k, float cdf_threshold, uint32_t* mask,
@@ -282,6 +286,13 @@ PRISM_API prism_status prism_block_select_ex(const float* q_pool, const float* k
                                              const prism_select_params* params, uint32_t* mask, int32_t* kept,
                                              int32_t* row_ptr, int32_t* col_idx, int64_t col_cap,
                                              int64_t* total_kept, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of prism_block_select / prism_block_select_ex for pooled
+ * features of `heads` x `n_blocks` x `head_dim` (the same value as
+ * prism_workspace_size(PRISM_OP_BLOCK_SELECT, ...) for that geometry's block
+ * count), for callers that hold only the pooled shapes. Host only. */
+PRISM_API prism_status prism_block_select_workspace_size(int32_t heads, int32_t n_blocks, int32_t head_dim,
+                                                         size_t* bytes);
 
 /*
  * Top-k floor from a top-k sparsity ratio (walkthrough section

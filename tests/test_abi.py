@@ -68,7 +68,10 @@ def test_geometry_counts_and_errors(lib):
 
 def test_workspace_sizes(lib):
     g = _geo()
-    assert P.workspace_size("block_select", g) == 256
+    # the status word and a key-major copy of the pooled keys (heads x head_dim x n_blocks rounded up to 4)
+    assert P.workspace_size("block_select", g) == 256 + 4608 * 128 * 4
+    assert P.workspace_size("block_select", g, heads=24, head_dim=128) == P.select_workspace_size(24, 4608, 128)
+    assert P.select_workspace_size(3, 37, 64) == 256 + (3 * 64 * 40 * 4 + 255) // 256 * 256
     z = P.workspace_size("zone_shapes", g, feat_c=3072, res_c=3072)
     assert z >= 576 * 48 * 8 * 4 + 294912 * 4
     b = P.workspace_size("bsa_bwd", g, heads=24, head_dim=128, nnz=1000)
