@@ -36,7 +36,8 @@ namespace {
 
 constexpr int kKB = 2;
 constexpr int kSoftWarps = 8;
-constexpr int kBwdThreads = 64 + 32 * kSoftWarps;
+constexpr int kBwdThreads = 64 + 32 * kSoftWarps + 32;
+constexpr int kIssuerB = 2 + kSoftWarps;  // warp of the second MMA issuer
 
 struct BwdParams {
   CUtensorMap mq[kMaxCand];
@@ -64,13 +65,13 @@ struct BwdParams {
 // each). Q and dO are staged through shared memory once and copied into TMEM
 // (the A operands of every S / dP product); that shared-memory space then
 // holds dS in two buffers, the A operand of the dQ products.
-// The issuer runs one fixed order, A_0, A_1, B_0, A_2, B_1, ... with
-// A_j = (S_j = Q K_j^T, dP_j = dO V_j^T) and B_j = (dQ += dS_j K_j), waiting
-// once per group: for slot j landed before A_j, for dS_j written before B_j.
-// A_{j+2} reuses the score buffers of step j, which the softmax warps read
-// before writing dS_j, so that reuse needs no barrier of its own. dS_j goes to
-// buffer j % 2 and has its own ready barrier per buffer, so a parity wait on
-// it can never be two phases behind.
+// Two threads issue the products, each in step order: warp 1 issues
+// A_j = (S_j = Q K_j^T, dP_j = dO V_j^T) once slot j has landed and the
+// softmax warps have read the score buffers of step j - 2; warp 10 issues
+// B_j = (dQ += dS_j K_j) once dS_j is written. While one waits on a barrier
+// the other's products keep the tensor pipe busy. dS_j goes to buffer j % 2
+// and has its own ready barrier per buffer, so a parity wait on it can never
+// be two phases behind.
 template <int D>
 struct DqSmem {
   static constexpr uint32_t kQD = 0;                 // Q, dO staging [2][dh][64][128 B]; then dS [2]
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
   uint64_t* qa_full = bars + 16;  // Q and dO copied into TMEM by the softmax warps
+  uint64_t* s_free = bars + 17;   // [2] S_j, dP_j read by the softmax warps, index j % 2
+  uint64_t* b_done = bars + 19;   // every B product complete
 
   const Geo& g = P.g;
   const int I = blockIdx.x, head = blockIdx.y;
@@ -126,8 +129,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       mbar_init(&s_full[i], 1);
       mbar_init(&ds_full[i], kSoftWarps);
       mbar_init(&ds_free[i], 1);
+      mbar_init(&s_free[i], kSoftWarps);
     }
     mbar_init(mma_done, 1);
+    mbar_init(b_done, 1);
     mbar_init(qa_full, kSoftWarps);
     *abort_flag = 0;
     fence_barrier_init();
@@ -189,20 +194,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ A issuer
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
-      const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
-      const uint64_t dDS0 = sdesc_sw128(smem_u32(sm + L::kQD), 16, 1024);
       const uint32_t sK0 = smem_u32(sm + L::kSlot0);
-      const uint64_t dK0 = sdesc_sw128(sK0, 16, 1024);                        // K as B of S
-      const uint64_t dKmn0 = sdesc_sw128(sK0, kKB * kBoxBytes, 1024);         // K as B of dQ
-      const uint64_t dV0 = sdesc_sw128(sK0 + L::kHalf, 16, 1024);             // V as B of dP
+      const uint64_t dK0 = sdesc_sw128(sK0, 16, 1024);             // K as B of S
+      const uint64_t dV0 = sdesc_sw128(sK0 + L::kHalf, 16, 1024);  // V as B of dP
       constexpr uint64_t kSlotStep = L::kSlotBytes >> 4;
-      constexpr uint64_t kDSStep = L::kDSBytes >> 4;
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
-      // A_j: S_j and dP_j into score buffer j % 2
-      auto issue_a = [&](int j) {
+      // A_j: S_j and dP_j into score buffer j % 2, once slot j has landed and
+      // the softmax warps have read that buffer's step j - 2
+      for (int j = 0; j < nsteps && ok; ++j) {
+        ok = mbar_wait_abortable(&kv_full[j % NS], (j / NS) & 1, status, abort_flag) &&
+             mbar_wait_abortable(&s_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
         const uint64_t so = uint64_t(j % NS) * kSlotStep;
         const uint32_t tS = tbase + (j & 1) * 64;
 #pragma unroll
@@ -212,13 +218,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ws_ts(tS + 128, tDO + kk * 8, dV0 + so + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
         mma_commit(&s_full[j & 1]);
-      };
-      for (int j = 0; j < 2 && j < nsteps && ok; ++j) {
-        ok = mbar_wait_abortable(&kv_full[j % NS], (j / NS) & 1, status, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_a(j);
       }
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, status);
+    }
+  } else if (warp == kIssuerB) {
+    // ------------------------------------------------------------ B issuer
+    if (lane == 0 && nsteps > 0) {
+      const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
+      const uint64_t dDS0 = sdesc_sw128(smem_u32(sm + L::kQD), 16, 1024);
+      const uint64_t dKmn0 = sdesc_sw128(smem_u32(sm + L::kSlot0), kKB * kBoxBytes, 1024);  // K as B of dQ
+      constexpr uint64_t kSlotStep = L::kSlotBytes >> 4;
+      constexpr uint64_t kDSStep = L::kDSBytes >> 4;
+      bool ok = true;
+      // B_j once dS_j is written (which implies A_j, hence slot j, complete)
       for (int j = 0; j < nsteps && ok; ++j) {
         ok = mbar_wait_abortable(&ds_full[j & 1], (j >> 1) & 1, status, abort_flag);
         if (!ok) break;
@@ -231,16 +245,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&kv_free[j % NS]);
         mma_commit(&ds_free[j & 1]);
-        if (j + 2 < nsteps) {
-          ok = mbar_wait_abortable(&kv_full[(j + 2) % NS], ((j + 2) / NS) & 1, status, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_a(j + 2);
-        }
       }
-      // every MMA this thread issued has completed before TMEM is released
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0, status);
+      mma_commit(b_done);
+      mbar_wait(b_done, 0, status);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -274,6 +281,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
       tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
       tmem_ld_wait();
+      // the score buffers are free for A_{j+2}
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
       mask_scores32(rs, members);  // P = exp2(-inf) = 0 there, hence dS = 0
       uint32_t pk[16];
       if (valid) {
@@ -296,8 +307,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
             make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       fence_proxy_async_smem();
-      // this step's score reads precede the arrival: the issuer then reuses the buffers for A_{j+2}
-      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full[sb]);
     }
@@ -337,12 +346,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
 // P^T and dS^T, the A operands of the dV / dK products. LSE and D of the
 // step's query rows come straight from global memory into registers, one
 // step ahead.
-// The issuer runs one fixed order, A_0, A_1, B_0, A_2, B_1, A_3, ... with
-// A_j = (S^T_j, dP^T_j) and B_j = (dV += P^T_j dO_j, dK += dS^T_j Q_j). It
-// waits once per group: for stage j landed before A_j, for P^T_j / dS^T_j
-// written before B_j. A_{j+2} reuses the score buffers of step j, which the
-// softmax warps read before writing P^T_j, so that reuse needs no barrier of
-// its own.
+// Two threads issue the products, each in step order: warp 1 issues
+// A_j = (S^T_j, dP^T_j) once stage j has landed and the softmax warps have
+// read the score buffers of step j - 2; warp 10 issues
+// B_j = (dV += P^T_j dO_j, dK += dS^T_j Q_j) once P^T_j / dS^T_j are written.
+// While one waits on a barrier the other's products keep the tensor pipe
+// busy.
 template <int D>
 struct DkvSmem {
   static constexpr uint32_t kKV = 0;               // K, V staging [2][dh][64][128 B]; then P^T, dS^T
@@ -376,6 +385,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
   uint64_t* ka_full = bars + 14;  // K and V copied into TMEM by the softmax warps
+  uint64_t* s_free = bars + 15;   // [2] S^T_j, dP^T_j read by the softmax warps, index j % 2
+  uint64_t* b_done = bars + 17;   // every B product complete
 
   const Geo& g = P.g;
   const int J = blockIdx.x, head = blockIdx.y;
@@ -395,7 +406,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       mbar_init(&st_full[i], 1);
       mbar_init(&st_free[i], 1);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kSoftWarps);
+    }
+    mbar_init(b_done, 1);
     mbar_init(ps_full, kSoftWarps);
     mbar_init(ps_free, 1);
     mbar_init(mma_done, 1);
@@ -460,21 +475,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ A issuer
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
-      const uint32_t idO = idesc_bf16_f32(64, D, false, true);
-      const uint64_t dPT = sdesc_sw128(smem_u32(sm + L::kPT), 16, 1024);
-      const uint64_t dDST = sdesc_sw128(smem_u32(sm + L::kDST), 16, 1024);
       const uint32_t sQ0 = smem_u32(sm + L::kStage0);
-      const uint64_t dQ0 = sdesc_sw128(sQ0, 16, 1024);                             // Q as B of S^T
-      const uint64_t dDO0 = sdesc_sw128(sQ0 + L::kHalf, 16, 1024);                 // dO as B of dP^T
-      const uint64_t dQmn0 = sdesc_sw128(sQ0, kKB * kBoxBytes, 1024);              // Q as B of dK
-      const uint64_t dDOmn0 = sdesc_sw128(sQ0 + L::kHalf, kKB * kBoxBytes, 1024);  // dO as B of dV
+      const uint64_t dQ0 = sdesc_sw128(sQ0, 16, 1024);              // Q as B of S^T
+      const uint64_t dDO0 = sdesc_sw128(sQ0 + L::kHalf, 16, 1024);  // dO as B of dP^T
       constexpr uint64_t kStageStep = L::kStageBytes >> 4;
       bool ok = mbar_wait_abortable(ka_full, 0, status, abort_flag);
-      // A_j: S^T_j = K Q_j^T and dP^T_j = V dO_j^T into score buffer j % 2
-      auto issue_a = [&](int j) {
+      // A_j: S^T_j = K Q_j^T and dP^T_j = V dO_j^T into score buffer j % 2, once
+      // stage j has landed and the softmax warps have read that buffer's step j - 2
+      for (int j = 0; j < nsteps && ok; ++j) {
+        ok = mbar_wait_abortable(&st_full[j % NS], (j / NS) & 1, status, abort_flag) &&
+             mbar_wait_abortable(&s_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
         const uint64_t st = uint64_t(j % NS) * kStageStep;
         const uint32_t tS = tbase + (j & 1) * 64;
 #pragma unroll
@@ -484,13 +499,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ws_ts(tS + 128, tV + kk * 8, dDO0 + st + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
         mma_commit(&s_full[j & 1]);
-      };
-      for (int j = 0; j < 2 && j < nsteps && ok; ++j) {
-        ok = mbar_wait_abortable(&st_full[j % NS], (j / NS) & 1, status, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        issue_a(j);
       }
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, status);
+    }
+  } else if (warp == kIssuerB) {
+    // ------------------------------------------------------------ B issuer
+    if (lane == 0 && nsteps > 0) {
+      const uint32_t idO = idesc_bf16_f32(64, D, false, true);
+      const uint64_t dPT = sdesc_sw128(smem_u32(sm + L::kPT), 16, 1024);
+      const uint64_t dDST = sdesc_sw128(smem_u32(sm + L::kDST), 16, 1024);
+      const uint32_t sQ0 = smem_u32(sm + L::kStage0);
+      const uint64_t dQmn0 = sdesc_sw128(sQ0, kKB * kBoxBytes, 1024);              // Q as B of dK
+      const uint64_t dDOmn0 = sdesc_sw128(sQ0 + L::kHalf, kKB * kBoxBytes, 1024);  // dO as B of dV
+      constexpr uint64_t kStageStep = L::kStageBytes >> 4;
+      bool ok = true;
+      // B_j once P^T_j / dS^T_j are written (which implies A_j, hence stage j, complete)
       for (int j = 0; j < nsteps && ok; ++j) {
         ok = mbar_wait_abortable(ps_full, j & 1, status, abort_flag);
         if (!ok) break;
@@ -506,16 +531,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&st_free[j % NS]);
         mma_commit(ps_free);
-        if (j + 2 < nsteps) {
-          ok = mbar_wait_abortable(&st_full[(j + 2) % NS], ((j + 2) / NS) & 1, status, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_a(j + 2);
-        }
       }
-      // every MMA this thread issued has completed before TMEM is released
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0, status);
+      mma_commit(b_done);
+      mbar_wait(b_done, 0, status);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -560,6 +578,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
       tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
       tmem_ld_wait();
+      // the score buffers are free for A_{j+2}
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[sb]);
       const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
       uint32_t pp[16], pd[16];
       if (valid) {
@@ -594,8 +616,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
             make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
       }
       fence_proxy_async_smem();
-      // this step's score reads precede the arrival: the issuer then reuses the buffers for A_{j+2}
-      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ps_full);
     }

@@ -11,12 +11,17 @@
 //   warp 0      TMA producer: Q once; per step the K boxes and the V boxes of
 //               the step's two key blocks (3-slot rings each), through 5-D
 //               tensor maps (one per block shape);
-//   warp 1      TMEM owner and single-thread tcgen05 issuer:
-//               S_j = Q [K_j0 K_j1]^T  (.ws M=64, N=128, K=d, Q from TMEM)
-//               O_h += P_jh V_jh       (.ws M=64, N=128, K=64, P from TMEM)
+//   warp 1      TMEM owner and issuer of the score products
+//               S_j = Q [K_j0 K_j1]^T  (.ws M=64, N=128, K=d, Q from TMEM);
 //   warps 2..9  softmax: 256 threads, four per query row (two TMEM lane
 //               halves x two column halves, 32 keys each); row maxima are
-//               exchanged through shared memory.
+//               exchanged through shared memory;
+//   warp 10     issuer of the value products
+//               O_h += P_jh V_jh       (.ws M=64, N=128, K=64, P from TMEM).
+// Two issuing threads feed the one tensor pipe: while one waits on a
+// barrier the other's products keep the pipe busy (a single issuer leaves
+// the pipe idle for every barrier test it makes). Each commits and drains
+// its own products.
 // TMEM holds every tensor-core A operand: Q, and P (3 buffers of its own, so
 // S_{j+3} may be issued while PV_j still reads P_j). The .ws datapath computes the accumulator
 // columns n < N/2 in lanes 0..63 from A rows in lanes 0..63 and the columns
@@ -29,11 +34,11 @@
 // (d/64 products per K step). The two parts are added once, in the epilogue.
 // P never touches shared memory, so per step shared memory carries only the
 // K and V tiles (TMA writes, tensor-core reads).
-// The producer and the issuer never block on one barrier: each polls the
-// barriers of every operation it could start next (mbarrier.test_wait) and
-// starts whichever is ready. K slot j%3 is refilled once S_j has completed,
-// V slot j%3 and P buffer j%3 once PV_j has; S buffer j%3 once the softmax
-// warps have read S_j.
+// The producer never blocks on one barrier: it polls the barriers of every
+// copy it could start next (mbarrier.test_wait) and starts whichever is
+// ready. Each issuer waits for its own operands in step order. K slot j%3 is
+// refilled once S_j has completed, V slot j%3 and P buffer j%3 once PV_j
+// has; S buffer j%3 once the softmax warps have read S_j.
 // The running max is only moved when it grows by more than 8 (log2 units);
 // the final division uses the same stale max, so the result is exact while
 // the rare O rescale (TMEM load/scale/store) stays off the common path.
@@ -51,7 +56,8 @@ namespace {
 constexpr int kKB = 2;  // key blocks per step
 constexpr int kRing = 3;  // K slots = V slots = S buffers = P buffers
 constexpr int kSoftWarps = 8;
-constexpr int kFwdThreads = 64 + 32 * kSoftWarps;
+constexpr int kFwdThreads = 64 + 32 * kSoftWarps + 32;
+constexpr int kPvWarp = 2 + kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct FwdParams {
@@ -112,6 +118,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
   uint64_t* qa_full = bars + 22;  // Q copied into TMEM by the softmax warps
+  uint64_t* pv_done = bars + 23;  // every value product complete
   float* red = reinterpret_cast<float*>(sm + L::kRed);
   float* redl = red + 2 * 4 * 64;
 
@@ -140,6 +147,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     }
     mbar_init(mma_done, 1);
     mbar_init(qa_full, kSoftWarps);
+    mbar_init(pv_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -219,56 +227,54 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ score issuer
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
-      const uint32_t idO = idesc_bf16_f32(64, 128, false, true);
-      // K: K-major B of S. V: MN-major B of PV whose two 64-column halves are
-      // the same 64 channels of V of key block 0 and of key block 1 (LBO = the
-      // block stride), so N = 128 covers one channel group for both blocks.
       const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::kK0), 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), D * 128, 1024);
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
-      tc_fence_after();
-      int sj = 0, pj = 0;
-      Watchdog wd;
-      wd.reset();
-      while (ok && pj < nsteps) {
-        bool did = false;
-        if (pj < sj && mbar_test(&p_full[pj % kRing], (pj / kRing) & 1) &&
-            mbar_test(&v_full[pj % kRing], (pj / kRing) & 1)) {
-          tc_fence_after();
-          const int b = pj % kRing;
-          const uint64_t dV = dV0 + uint64_t(b * (L::kSlotBytes >> 4));
+      for (int sj = 0; sj < nsteps && ok; ++sj) {
+        const int b = sj % kRing;
+        // K of step sj landed; S buffer b read by the softmax warps (S_{sj-3})
+        ok = mbar_wait_abortable(&k_full[b], (sj / kRing) & 1, status, abort_flag) &&
+             mbar_wait_abortable(&s_free[b], ((sj / kRing) & 1) ^ 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dK = dK0 + uint64_t(b * (L::kSlotBytes >> 4));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              mma_ws_ts(tO + c * 64, tP + b * 32 + kk * 8, dV + uint64_t((c * kBoxBytes + kk * 2048) >> 4), idO,
-                        (pj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&p_free[b]);
-          ++pj;
-          did = true;
-        }
-        // S_sj overwrites buffer sj%3, which the softmax warps read S_{sj-3} from
-        if (sj < nsteps && mbar_test(&k_full[sj % kRing], (sj / kRing) & 1) &&
-            mbar_test(&s_free[sj % kRing], ((sj / kRing) & 1) ^ 1)) {
-          tc_fence_after();
-          const int b = sj % kRing;
-          const uint64_t dK = dK0 + uint64_t(b * (L::kSlotBytes >> 4));
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ws_ts(tbase + b * 64, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
-          mma_commit(&s_full[b]);
-          ++sj;
-          did = true;
-        }
-        if (did) wd.reset();
-        else if (!wd.ok(status, abort_flag)) break;
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ws_ts(tbase + b * 64, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+        mma_commit(&s_full[b]);
       }
-      // every MMA this thread issued has completed before TMEM is released
+      // every product this thread issued has completed before TMEM is released
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, status);
+    }
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ value issuer
+    if (lane == 0 && nsteps > 0) {
+      const uint32_t idO = idesc_bf16_f32(64, 128, false, true);
+      // V: MN-major B of PV whose two 64-column halves are the same 64
+      // channels of V of key block 0 and of key block 1 (LBO = the block
+      // stride), so N = 128 covers one channel group for both blocks.
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), D * 128, 1024);
+      bool ok = true;
+      for (int pj = 0; pj < nsteps && ok; ++pj) {
+        const int b = pj % kRing;
+        ok = mbar_wait_abortable(&p_full[b], (pj / kRing) & 1, status, abort_flag) &&
+             mbar_wait_abortable(&v_full[b], (pj / kRing) & 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dV = dV0 + uint64_t(b * (L::kSlotBytes >> 4));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            mma_ws_ts(tO + c * 64, tP + b * 32 + kk * 8, dV + uint64_t((c * kBoxBytes + kk * 2048) >> 4), idO,
+                      (pj > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&p_free[b]);
+      }
+      mma_commit(pv_done);
+      mbar_wait(pv_done, 0, status);
     }
   } else {
     // ------------------------------------------------------------ softmax
