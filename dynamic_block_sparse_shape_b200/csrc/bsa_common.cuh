@@ -175,6 +175,42 @@ struct DescCache {
   __device__ __forceinline__ int4 get(int e) const { return ring[e % kDescRing]; }
 };
 
+// Block ids named by a CSR / CSC list, read 32 at a time by a whole warp
+// (coalesced list reads) into a shared-memory ring, so the thread that issues
+// the copies never waits on a dependent global load. Entry e of a list of
+// `cnt` blocks processed `step` (a power of two) per step: e < cnt is the
+// list's e-th block; a ragged tail (e >= cnt in the last step) repeats the
+// step's first block. An id out of range is reported and replaced by 0.
+struct IdCache {
+  int* ring;  // shared memory, kDescRing entries
+  int filled;
+  int step = 2;
+  // Makes entries [0, e] available; the whole warp must call it.
+  __device__ __forceinline__ void ensure(int e, const Geo& g, const int32_t* list, int beg, int cnt, int* status,
+                                         int lane) {
+    while (e >= filled) {
+      const int ee = filled + lane;
+      int idx = ee < cnt ? ee : (ee & ~(step - 1));
+      if (idx >= cnt) idx = 0;
+      int J = list[beg + idx];
+      if (J < 0 || J >= g.n_blocks) {
+        atomicOr(status, kDevErrBounds);
+        J = 0;
+      }
+      ring[ee % kDescRing] = J;
+      __syncwarp();
+      filled += 32;
+    }
+  }
+  __device__ __forceinline__ int get(int e) const { return ring[e % kDescRing]; }
+};
+
+// Byte offset of the operand image of (head, block) in a block-major image
+// buffer (one D * 128-byte image per block and head, head-major).
+__device__ __forceinline__ size_t image_offset(const Geo& g, int head, int b, int D) {
+  return (size_t(head) * g.n_blocks + b) * size_t(D) * 128u;
+}
+
 // Store 32 (or 16) fp32 values as bf16 or fp32 at dst (16-byte aligned).
 template <int NC>
 __device__ __forceinline__ void store_row(void* dst, int64_t off, const float* v, bool fp32) {

@@ -8,9 +8,10 @@
 //
 // One CTA per (query block I, head); a step covers two selected key blocks.
 // Warp roles:
-//   warp 0      TMA producer: Q once; per step the K boxes and the V boxes of
-//               the step's two key blocks (3-slot rings each), through 5-D
-//               tensor maps (one per block shape);
+//   warp 0      copy producer: Q once, through a 5-D tensor map (one per
+//               block shape); per step K and V of the step's two key blocks
+//               (3-slot rings each) as bulk copies of their block images
+//               (written by block_images_kernel before the attention kernel);
 //   warp 1      TMEM owner and issuer of the score products
 //               S_j = Q [K_j0 K_j1]^T  (.ws M=64, N=128, K=d, Q from TMEM);
 //   warps 2..9  softmax: 256 threads, four per query row (two TMEM lane
@@ -62,8 +63,8 @@ constexpr float kRescaleThreshold = 8.0f;
 
 struct FwdParams {
   CUtensorMap mq[kMaxCand];
-  CUtensorMap mk[kMaxCand];
-  CUtensorMap mv[kMaxCand];
+  const uint8_t* kimg;  // block images of K and V (layout in host.h)
+  const uint8_t* vimg;
   Geo g;
   const int32_t* zone_shape;
   const int32_t* row_ptr;
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (nsteps > 0) {
-      DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
+      IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
       if (lane == 0) {
         const int sI = safe_shape(g, P.zone_shape, I, status);
         const BlockBox qb = block_box(g, sI, I);
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       Watchdog wd;
       wd.reset();
       while (kj < nsteps || vj < nsteps) {
-        if (kj < nsteps) dc.ensure(kKB * kj + kKB - 1, g, P.col_idx, beg, cnt, P.zone_shape, status, lane);
+        if (kj < nsteps) dc.ensure(kKB * kj + kKB - 1, g, P.col_idx, beg, cnt, status, lane);
         int nk = kj, nv = vj, stop = 0;
         if (lane == 0) {
           bool did = false;
@@ -188,10 +189,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
             uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
             mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
             for (int slot = 0; slot < kKB; ++slot) {
-              const int4 b = dc.get(kKB * nk + slot);
+              const uint8_t* src = P.kimg + image_offset(g, head, dc.get(kKB * nk + slot), D);
               for (int dh = 0; dh < D / 64; ++dh)
-                tma_load_5d(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &P.mk[b.x], &k_full[ks], dh * 64, head,
-                            b.y, b.z, b.w);
+                bulk_load(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, src + dh * kBoxBytes, kBoxBytes,
+                          &k_full[ks]);
             }
             ++nk;
             did = true;
@@ -201,12 +202,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
             const int vs = nv % kRing;
             uint8_t* dst = sm + L::kV0 + vs * L::kSlotBytes;
             mbar_arrive_expect_tx(&v_full[vs], L::kSlotBytes);
-            for (int slot = 0; slot < kKB; ++slot) {
-              const int4 b = dc.get(kKB * nv + slot);
-              for (int dh = 0; dh < D / 64; ++dh)
-                tma_load_5d(dst + slot * (D * 128) + dh * kBoxBytes, &P.mv[b.x], &v_full[vs], dh * 64, head, b.y,
-                            b.z, b.w);
-            }
+            for (int slot = 0; slot < kKB; ++slot)
+              bulk_load(dst + slot * (D * 128), P.vimg + image_offset(g, head, dc.get(kKB * nv + slot), D), D * 128,
+                        &v_full[vs]);
             ++nv;
             did = true;
           }
@@ -453,7 +451,57 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, int64_t tok_stride
   *reinterpret_cast<uint2*>(dst + i) = out;
 }
 
+// Block-major operand images (layout in host.h): one CTA per (block, head),
+// 128 threads, D/16 independent 16-byte loads per thread; sixteen consecutive
+// threads (D = 128) read one token's 256-byte head slice.
+template <int D>
+__global__ void __launch_bounds__(128) block_images_kernel(const Geo g, const int32_t* __restrict__ zone_shape,
+                                                           const __nv_bfloat16* __restrict__ src, int64_t tok_stride,
+                                                           uint8_t* __restrict__ dst, int* status) {
+  constexpr int CPR = D / 8;            // 16-byte chunks per row
+  constexpr int PER = 64 * CPR / 128;   // chunks per thread
+  const int b = blockIdx.x, head = blockIdx.y;
+  const int s = safe_shape(g, zone_shape, b, status);
+  const BlockBox bb = block_box(g, s, b);
+  uint8_t* img = dst + image_offset(g, head, b, D);
+  uint4 v[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + 128 * k;
+    const int r = i / CPR, c = i % CPR;
+    v[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (!g.partial || block_slot_in_grid(g, bb, r)) {
+      const int tok = block_token(g, bb, r);
+      v[k] = __ldg(reinterpret_cast<const uint4*>(src + int64_t(tok) * tok_stride + int64_t(head) * D + c * 8));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + 128 * k;
+    const int r = i / CPR, c = i % CPR;
+    *reinterpret_cast<uint4*>(img + (c / 8) * kBoxBytes + sw128_offset(r, c % 8)) = v[k];
+  }
+}
+
 }  // namespace
+
+size_t block_images_bytes(const Geo& g, int heads, int head_dim) {
+  return size_t(heads) * g.n_blocks * size_t(head_dim) * 128u;
+}
+
+prism_status launch_block_images(const Geo& g, const int32_t* zone_shape, const void* src, int64_t tok_stride,
+                                 int heads, int head_dim, void* dst, int* status, cudaStream_t s) {
+  const dim3 grid(g.n_blocks, heads);
+  const auto* sp = static_cast<const __nv_bfloat16*>(src);
+  auto* dp = static_cast<uint8_t*>(dst);
+  if (head_dim == 128)
+    block_images_kernel<128><<<grid, 128, 0, s>>>(g, zone_shape, sp, tok_stride, dp, status);
+  else if (head_dim == 64)
+    block_images_kernel<64><<<grid, 128, 0, s>>>(g, zone_shape, sp, tok_stride, dp, status);
+  else
+    return PRISM_ERR_UNSUPPORTED;
+  return cuda_status(cudaGetLastError());
+}
 
 prism_status stage_bf16(const void* src, prism_dtype dtype, int64_t tok_stride, int C, int64_t n_tokens,
                         __nv_bfloat16* dst, cudaStream_t s) {
@@ -464,12 +512,15 @@ prism_status stage_bf16(const void* src, prism_dtype dtype, int64_t tok_stride, 
   return cuda_status(cudaGetLastError());
 }
 
+// Workspace: [fp32 input only: bf16 copies of q, k, v] + block images of k and v.
 size_t bsa_fwd_ws_bytes(const Geo& g, int heads, int head_dim, prism_dtype dtype) {
   WsCarver c;
   if (dtype == PRISM_FP32) {
     const size_t t = size_t(g.T) * g.H * g.W * heads * head_dim * 2;
     c.take(t); c.take(t); c.take(t);
   }
+  c.take(block_images_bytes(g, heads, head_dim));
+  c.take(block_images_bytes(g, heads, head_dim));
   return c.off;
 }
 
@@ -500,10 +551,10 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
   const void* kb = k;
   const void* vb = v;
   int64_t in_stride = tok_stride;
+  WsCarver c;
   if (dtype == PRISM_FP32) {
     const int64_t N = int64_t(g.T) * g.H * g.W;
     const int C = heads * head_dim;
-    WsCarver c;
     const size_t t = size_t(N) * C * 2;
     __nv_bfloat16* sq = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + c.take(t));
     __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + c.take(t));
@@ -514,14 +565,22 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
     qb = sq; kb = sk; vb = sv;
     in_stride = C;
   }
+  // K and V as block images: every key block the kernel gathers is then one
+  // contiguous bulk copy per 64 channels instead of 64 scattered token rows
+  uint8_t* kimg = static_cast<uint8_t*>(ws) + c.take(block_images_bytes(g, heads, head_dim));
+  uint8_t* vimg = static_cast<uint8_t*>(ws) + c.take(block_images_bytes(g, heads, head_dim));
+  if ((st = launch_block_images(g, zone_shape, kb, in_stride, heads, head_dim, kimg, ws_status(ws), s)) != PRISM_OK)
+    return st;
+  if ((st = launch_block_images(g, zone_shape, vb, in_stride, heads, head_dim, vimg, ws_status(ws), s)) != PRISM_OK)
+    return st;
   FwdParams P;
   std::memset(&P, 0, sizeof(P));
-  for (int c = 0; c < g.n_cand; ++c) {
-    const int bt = g.cand[c][0], bh = g.cand[c][1], bw = g.cand[c][2];
-    if ((st = encode_block_map(&P.mq[c], qb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
-    if ((st = encode_block_map(&P.mk[c], kb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
-    if ((st = encode_block_map(&P.mv[c], vb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+  for (int ci = 0; ci < g.n_cand; ++ci) {
+    const int bt = g.cand[ci][0], bh = g.cand[ci][1], bw = g.cand[ci][2];
+    if ((st = encode_block_map(&P.mq[ci], qb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
   }
+  P.kimg = kimg;
+  P.vimg = vimg;
   P.g = g;
   P.zone_shape = zone_shape;
   P.row_ptr = row_ptr;

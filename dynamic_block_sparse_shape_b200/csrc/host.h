@@ -45,6 +45,16 @@ prism_status encode_block_map(CUtensorMap* map, const void* base, const Geo& g, 
 
 inline int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
 
+// Block-major operand images of a token-major [N, heads, d] bf16 tensor: for
+// every (head, block) the block's 64 rows of that head laid out exactly as a
+// shared-memory operand tile, [d/64][64 rows][128 B] with the 128-byte
+// swizzle, slots outside the grid zero. One image is d * 128 bytes; images
+// are head-major, block-minor. A plain bulk copy of an image into a
+// 1024-byte-aligned shared-memory tile gives the tile the tensor cores read.
+size_t block_images_bytes(const Geo& g, int heads, int head_dim);
+prism_status launch_block_images(const Geo& g, const int32_t* zone_shape, const void* src, int64_t tok_stride,
+                                 int heads, int head_dim, void* dst, int* status, cudaStream_t s);
+
 // Exclusive scan of n ints: out[0..n] with out[n] = total (one CTA).
 cudaError_t launch_exclusive_scan(const int32_t* in, int n, int32_t* out, cudaStream_t s);
 // Expands bitmask rows (ceil(nb/32) words each) into ascending index lists at

@@ -361,6 +361,11 @@ PRISM_API prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* ro
  *       precision; with a nearly one-hot softmax, dS = P (dP - D) cancels
  *       and bf16 rounding of O alone would dominate dQ and dK. Ignored (may be
  *       NULL) for fp32 outputs, which carry no rounding.
+ * ws: at least prism_workspace_size(PRISM_OP_BSA_FWD, ...) bytes. It holds
+ *       block-major copies of K and V (2 * heads * n_blocks * head_dim * 128
+ *       bytes: each 64-token block of each head as one contiguous, already
+ *       swizzled operand tile, so the kernel gathers a key block with one bulk
+ *       copy) and, for fp32 inputs, the bf16 copies of Q, K and V.
  */
 PRISM_API prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
                            const void* v, prism_dtype dtype, int32_t heads, int32_t head_dim, int64_t tok_stride,
