@@ -21,7 +21,9 @@
 //               P^T, dS^T in the softmax warps, then dV += P^T dO and
 //               dK += dS^T Q (.ws M=64, N=d); dK, dV live in TMEM.
 // Splitting dQ from dK/dV costs one recomputation of S and dP but needs no
-// atomics and is deterministic.
+// atomics and is deterministic. Each pass streams its two operands (K and V,
+// or Q and dO) as bulk copies of block images made just before it; the
+// single-use Q / dO (dq) and K / V (dkdv) tiles come through 5-D tensor maps.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -44,6 +46,10 @@ struct BwdParams {
   CUtensorMap mk[kMaxCand];
   CUtensorMap mv[kMaxCand];
   CUtensorMap mdo[kMaxCand];
+  // block images (layout in host.h) of the two operands a kernel streams:
+  // K and V for dq, Q and dO for dkdv
+  const uint8_t* img0;
+  const uint8_t* img1;
   Geo g;
   const int32_t* zone_shape;
   const int32_t* ptr;  // CSR row_ptr (dq) or CSC col_ptr (dkdv), over (head, block)
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (nsteps > 0) {
-      DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
+      IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
       if (lane == 0) {
         const int sI = safe_shape(g, P.zone_shape, I, status);
         const BlockBox qb = block_box(g, sI, I);
@@ -165,7 +171,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < nsteps && ok; ++j) {
-        dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, P.zone_shape, status, lane);
+        dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, status, lane);
         if (lane == 0) {
           const int s = j % NS;
           // slot s last held step j - 3: free once its dQ product completed
@@ -174,11 +180,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
             uint8_t* dst = sm + L::kSlot0 + s * L::kSlotBytes;
             mbar_arrive_expect_tx(&kv_full[s], L::kSlotBytes);
             for (int slot = 0; slot < kKB; ++slot) {
-              const int4 b = dc.get(kKB * j + slot);
+              const size_t io = image_offset(g, head, dc.get(kKB * j + slot), D);
               for (int dh = 0; dh < D / 64; ++dh) {
                 const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
-                tma_load_5d(dst + off, &P.mk[b.x], &kv_full[s], dh * 64, head, b.y, b.z, b.w);
-                tma_load_5d(dst + L::kHalf + off, &P.mv[b.x], &kv_full[s], dh * 64, head, b.y, b.z, b.w);
+                bulk_load(dst + off, P.img0 + io + dh * kBoxBytes, kBoxBytes, &kv_full[s]);
+                bulk_load(dst + L::kHalf + off, P.img1 + io + dh * kBoxBytes, kBoxBytes, &kv_full[s]);
               }
             }
             issued = j + 1;
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (nsteps > 0) {
-      DescCache dc{reinterpret_cast<int4*>(sm + L::kDesc), 0};
+      IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
       if (lane == 0) {
         const int sJ = safe_shape(g, P.zone_shape, J, status);
         const BlockBox kb = block_box(g, sJ, J);
@@ -446,7 +452,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < nsteps && ok; ++j) {
-        dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, P.zone_shape, status, lane);
+        dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, status, lane);
         if (lane == 0) {
           const int s = j % NS;
           // stage s last held step j - 3: free once its dV / dK products completed
@@ -455,11 +461,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
             uint8_t* stage = sm + L::kStage0 + s * L::kStageBytes;
             mbar_arrive_expect_tx(&st_full[s], L::kStageBytes);
             for (int slot = 0; slot < kKB; ++slot) {
-              const int4 b = dc.get(kKB * j + slot);
+              const size_t io = image_offset(g, head, dc.get(kKB * j + slot), D);
               for (int dh = 0; dh < D / 64; ++dh) {
                 const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
-                tma_load_5d(stage + off, &P.mq[b.x], &st_full[s], dh * 64, head, b.y, b.z, b.w);
-                tma_load_5d(stage + L::kHalf + off, &P.mdo[b.x], &st_full[s], dh * 64, head, b.y, b.z, b.w);
+                bulk_load(stage + off, P.img0 + io + dh * kBoxBytes, kBoxBytes, &st_full[s]);
+                bulk_load(stage + L::kHalf + off, P.img1 + io + dh * kBoxBytes, kBoxBytes, &st_full[s]);
               }
             }
             issued = j + 1;
@@ -755,7 +761,7 @@ __global__ void __launch_bounds__(256) popc_rows_kernel(const uint32_t* __restri
 }
 
 struct BwdWs {
-  size_t stage_q, stage_k, stage_v, stage_do, lse2, dvec, tmask, ccnt, cptr, ridx, total;
+  size_t stage_q, stage_k, stage_v, stage_do, lse2, dvec, tmask, ccnt, cptr, ridx, img0, img1, total;
 };
 
 BwdWs bwd_ws_layout(const Geo& g, int heads, int head_dim, prism_dtype dtype, int64_t nnz) {
@@ -775,6 +781,9 @@ BwdWs bwd_ws_layout(const Geo& g, int heads, int head_dim, prism_dtype dtype, in
   w.ccnt = c.take(rows * 4);
   w.cptr = c.take((rows + 1) * 4);
   w.ridx = c.take(size_t(nnz > 0 ? nnz : 1) * 4);
+  // block images of K and V for the dq pass, then of Q and dO for the dkdv pass
+  w.img0 = c.take(block_images_bytes(g, heads, head_dim));
+  w.img1 = c.take(block_images_bytes(g, heads, head_dim));
   w.total = c.off;
   return w;
 }
@@ -877,7 +886,13 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   P.scale_log2 = scale * 1.4426950408889634f;
   P.scale = scale;
   P.out_fp32 = dtype == PRISM_FP32;
-  // dQ: q-stationary over the CSR
+  uint8_t* img0 = w8 + W.img0;
+  uint8_t* img1 = w8 + W.img1;
+  // dQ: q-stationary over the CSR, streaming K and V
+  if ((st = launch_block_images(g, zone_shape, kb, in_stride, heads, head_dim, img0, status, s)) != PRISM_OK) return st;
+  if ((st = launch_block_images(g, zone_shape, vb, in_stride, heads, head_dim, img1, status, s)) != PRISM_OK) return st;
+  P.img0 = img0;
+  P.img1 = img1;
   P.ptr = row_ptr;
   P.idx = col_idx;
   P.out0 = dq;
@@ -894,7 +909,11 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
     bsa_dq_kernel<64><<<grid, kBwdThreads, smem, s>>>(P);
   }
   if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
-  // dK, dV: kv-stationary over the CSC
+  // dK, dV: kv-stationary over the CSC, streaming Q and dO (the images
+  // overwrite those of K and V once the dq pass is done: same stream)
+  if ((st = launch_block_images(g, zone_shape, qb, in_stride, heads, head_dim, img0, status, s)) != PRISM_OK) return st;
+  if ((st = launch_block_images(g, zone_shape, dob, in_stride, heads, head_dim, img1, status, s)) != PRISM_OK)
+    return st;
   P.ptr = cptr;
   P.idx = ridx;
   P.out0 = dk;

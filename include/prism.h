@@ -382,6 +382,11 @@ PRISM_API prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* z
  * outputs (with o_lo, D_i = dO_i . (O_i + O_lo_i)); dout is device
  * [N, heads, head_dim]; dq, dk, dv are device outs like q. nnz =
  * row_ptr[heads*n_blocks] (for workspace sizing; checked against ws_bytes).
+ * ws: at least prism_workspace_size(PRISM_OP_BSA_BWD, ...) bytes: D and the
+ *       LSE in block order, the CSC of the selection (4 bytes per selected
+ *       pair), two block-major operand copies (2 * heads * n_blocks *
+ *       head_dim * 128 bytes; K and V for the dQ pass, then Q and dO for the
+ *       dK/dV pass) and, for fp32 inputs, bf16 copies of Q, K, V and dO.
  */
 PRISM_API prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
                            const void* v, const void* o, const void* o_lo, const float* lse, const void* dout,
