@@ -227,7 +227,8 @@ class Pipeline:
 
     STAGES = ("zone_shapes", "block_pool", "block_select", "bsa_fwd", "bsa_bwd")
     # kernels each stage launches (prism kernels only; memsets excluded)
-    LAUNCHES = {"zone_shapes": 4, "block_pool": 1, "block_select": 3, "bsa_fwd": 1, "bsa_bwd": 7}
+    # (bsa_fwd: K and V block images + attention; bsa_bwd: prep, CSC (3), K/V images, dQ, Q/dO images, dK/dV)
+    LAUNCHES = {"zone_shapes": 4, "block_pool": 1, "block_select": 3, "bsa_fwd": 3, "bsa_bwd": 11}
 
     def step(self, record=None):
         fns = (self.stage_zone, self.stage_pool, self.stage_select, self.stage_fwd, self.stage_bwd)

@@ -14,35 +14,38 @@
 //               (written by block_images_kernel before the attention kernel);
 //   warp 1      TMEM owner and issuer of the score products
 //               S_j = Q [K_j0 K_j1]^T  (.ws M=64, N=128, K=d, Q from TMEM);
-//   warps 2..9  softmax: 256 threads, four per query row (two TMEM lane
-//               halves x two column halves, 32 keys each); row maxima are
-//               exchanged through shared memory;
+//   warps 2..9  softmax, two groups of four warps taking alternate steps
+//               (group j % 2 takes step j), one thread per TMEM lane: a
+//               thread holds the 64 scores of one query row against one key
+//               block of the step;
 //   warp 10     issuer of the value products
-//               O_h += P_jh V_jh       (.ws M=64, N=128, K=64, P from TMEM).
-// Two issuing threads feed the one tensor pipe: while one waits on a
-// barrier the other's products keep the pipe busy (a single issuer leaves
-// the pipe idle for every barrier test it makes). Each commits and drains
-// its own products.
-// TMEM holds every tensor-core A operand: Q, and P (3 buffers of its own, so
-// S_{j+3} may be issued while PV_j still reads P_j). The .ws datapath computes the accumulator
-// columns n < N/2 in lanes 0..63 from A rows in lanes 0..63 and the columns
-// n >= N/2 in lanes 64..127 from A rows in lanes 64..127. S_j of key block 0
-// lands in the low lanes and of key block 1 in the high lanes, so the P rows
-// each lane half holds belong to one key block. The PV product is therefore
-// issued with its B operand's two 64-column halves taken from V of key block
-// 0 (low half) and key block 1 (high half): lane m accumulates the block-0
-// part of O row m, lane m + 64 the block-1 part, each over all d channels
-// (d/64 products per K step). The two parts are added once, in the epilogue.
-// P never touches shared memory, so per step shared memory carries only the
-// K and V tiles (TMA writes, tensor-core reads).
+//               O_g += P_j [V_j0 | V_j1]  (.ws M=64, N=2d, K=64, P from TMEM).
+// Two issuing threads feed the one tensor pipe: while one waits on a barrier
+// the other's products keep the pipe busy. Two softmax groups keep each SM
+// sub-partition busy: while one group waits (barriers, tensor-memory loads),
+// the other computes exponentials.
+// TMEM holds every tensor-core A operand: Q, and P (one buffer per group).
+// The .ws datapath computes the accumulator columns n < N/2 in lanes 0..63
+// from A rows in lanes 0..63 and the columns n >= N/2 in lanes 64..127 from
+// A rows in lanes 64..127. S_j of key block 0 lands in the low lanes and of
+// key block 1 in the high lanes, so the P rows each lane half holds belong to
+// one key block, and the value product takes its B operand's first d columns
+// from V of key block 0 and the next d from V of key block 1: lane m
+// accumulates the block-0 part of O row m, lane m + 64 the block-1 part, over
+// all d channels. Each group has its own O parts, so every (group, lane half)
+// part keeps its own running max and sum: no thread exchanges a row maximum
+// with another while the row is streamed. The four parts of a row are merged
+// once, in the epilogue. P never touches shared memory, so per step shared
+// memory carries only the K and V tiles (bulk-copy writes, tensor-core reads).
 // The producer never blocks on one barrier: it polls the barriers of every
 // copy it could start next (mbarrier.test_wait) and starts whichever is
 // ready. Each issuer waits for its own operands in step order. K slot j%3 is
-// refilled once S_j has completed, V slot j%3 and P buffer j%3 once PV_j
-// has; S buffer j%3 once the softmax warps have read S_j.
-// The running max is only moved when it grows by more than 8 (log2 units);
-// the final division uses the same stale max, so the result is exact while
-// the rare O rescale (TMEM load/scale/store) stays off the common path.
+// refilled once S_j has completed, V slot j%3 once PV_j has; a group's S
+// buffer once its warps have read it, its P buffer once its last PV has
+// completed.
+// A part's running max is only moved when it grows by more than 8 (log2
+// units); the final merge uses the same stale maxima, so the result is exact
+// while the rare O rescale (TMEM load/scale/store) stays off the common path.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -54,9 +57,11 @@
 namespace prism {
 namespace {
 
-constexpr int kKB = 2;  // key blocks per step
-constexpr int kRing = 3;  // K slots = V slots = S buffers = P buffers
-constexpr int kSoftWarps = 8;
+constexpr int kKB = 2;      // key blocks per step
+constexpr int kRing = 3;    // K slots = V slots
+constexpr int kGroups = 2;  // softmax warp groups, alternate steps
+constexpr int kGroupWarps = 4;
+constexpr int kSoftWarps = kGroups * kGroupWarps;
 constexpr int kFwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kPvWarp = 2 + kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
@@ -82,25 +87,37 @@ template <int D>
 struct FwdSmem {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kQBytes = D * 128;
-  static constexpr uint32_t kSlotBytes = kKB * D * 128;  // K (or V) of one step
-  static constexpr uint32_t kK0 = kQBytes;                // [slot][dh][block][64][128 B]
+  static constexpr uint32_t kSlotBytes = kKB * D * 128;      // K (or V) of one step
+  static constexpr uint32_t kK0 = kQBytes;                   // [slot][dh][block][64][128 B]
   static constexpr uint32_t kV0 = kK0 + kRing * kSlotBytes;  // [slot][block][dh][64][128 B]
-  static constexpr uint32_t kRed = kV0 + kRing * kSlotBytes;
-  static constexpr uint32_t kRedBytes = (2 * 4 * 64 + 4 * 64) * 4;
-  static constexpr uint32_t kDesc = kRed + kRedBytes;  // block coordinate ring
+  static constexpr uint32_t kRed = kV0 + kRing * kSlotBytes; // per part: running max, sum [4][64] each
+  static constexpr uint32_t kRedBytes = 2 * 4 * 64 * 4;
+  static constexpr uint32_t kDesc = kRed + kRedBytes;  // block-id ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 16;
   static constexpr uint32_t kTotal = kBar + 256;
-  // epilogue exchange of O parts: [kh][ch][64 rows][D/4 + 4 floats], in the K ring
+  // epilogue exchange of scaled O parts: [src part][dst quarter][64 rows][D/4 + 4 floats], over the K/V rings
   static constexpr uint32_t kXPitch = D / 4 + 4;
-  static_assert(4 * 64 * kXPitch * 4 <= kRing * kSlotBytes, "exchange buffer fits the K ring");
-  // TMEM: S buffers at 0, 64, 128; O parts (D columns) at 192; Q (A operand,
-  // D/2 columns) after O; P buffers (32 columns each) after Q
+  static_assert(16 * 64 * kXPitch * 4 <= 2 * kRing * kSlotBytes, "exchange buffer fits the K/V rings");
+  // TMEM: S buffers (64 columns per group) at 0; O parts (D columns per
+  // group) at 128; Q (A operand, D/2 columns); P buffers (32 columns per group)
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTO = 192;
-  static constexpr uint32_t kTQ = 192 + D;
+  static constexpr uint32_t kTO = 64 * kGroups;
+  static constexpr uint32_t kTQ = kTO + kGroups * D;
   static constexpr uint32_t kTP = kTQ + D / 2;
-  static_assert(kTP + kRing * 32 <= kTmemCols, "TMEM budget");
+  static_assert(kTP + kGroups * 32 <= kTmemCols, "TMEM budget");
 };
+
+// Maximum of 64 scores (raw bits of fp32 values).
+__device__ __forceinline__ float max64(const uint32_t* r) {
+  float ca = fmax3(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
+  float cb = fmax3(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
+#pragma unroll
+  for (int i = 6; i < 62; i += 4) {
+    ca = fmax3(ca, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+    cb = fmax3(cb, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+  }
+  return fmax3(fmaxf(ca, cb), __uint_as_float(r[62]), __uint_as_float(r[63]));
+}
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_constant__ FwdParams P) {
@@ -109,19 +126,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [3]
-  uint64_t* v_full = bars + 4;   // [3]
-  uint64_t* s_full = bars + 7;   // [3] S_j complete (also: K slot j%3 free)
-  uint64_t* s_free = bars + 10;  // [3] S_j read by the 8 softmax warps
-  uint64_t* p_full = bars + 13;  // [3] P_j written to TMEM by the 8 softmax warps
-  uint64_t* p_free = bars + 16;  // [3] PV_j complete (V slot and P buffer j%3 free)
-  uint64_t* mma_done = bars + 19;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
-  uint64_t* qa_full = bars + 22;  // Q copied into TMEM by the softmax warps
-  uint64_t* pv_done = bars + 23;  // every value product complete
-  float* red = reinterpret_cast<float*>(sm + L::kRed);
-  float* redl = red + 2 * 4 * 64;
+  uint64_t* k_full = bars + 1;    // [3] K of the slot's step landed
+  uint64_t* v_full = bars + 4;    // [3] V of the slot's step landed
+  uint64_t* k_free = bars + 7;    // [3] S of the slot's step complete
+  uint64_t* v_free = bars + 10;   // [3] PV of the slot's step complete
+  uint64_t* s_full = bars + 13;   // [2] per group: its current S complete
+  uint64_t* s_free = bars + 15;   // [2] per group: its S read by its 4 warps
+  uint64_t* p_full = bars + 17;   // [2] per group: its P written to TMEM by its 4 warps
+  uint64_t* p_free = bars + 19;   // [2] per group: its PV complete (P buffer and O parts quiescent)
+  uint64_t* mma_done = bars + 21;
+  uint64_t* pv_done = bars + 22;
+  uint64_t* qa_full = bars + 23;  // Q copied into TMEM by the softmax warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 25);
+  float* redm = reinterpret_cast<float*>(sm + L::kRed);
+  float* redl = redm + 4 * 64;
 
   const Geo& g = P.g;
   const int I = blockIdx.x, head = blockIdx.y;
@@ -141,14 +160,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
+      mbar_init(&k_free[i], 1);
+      mbar_init(&v_free[i], 1);
+    }
+    for (int i = 0; i < kGroups; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kSoftWarps);
-      mbar_init(&p_full[i], kSoftWarps);
+      mbar_init(&s_free[i], kGroupWarps);
+      mbar_init(&p_full[i], kGroupWarps);
       mbar_init(&p_free[i], 1);
     }
     mbar_init(mma_done, 1);
-    mbar_init(qa_full, kSoftWarps);
     mbar_init(pv_done, 1);
+    mbar_init(qa_full, kSoftWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -184,7 +207,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         if (lane == 0) {
           bool did = false;
           // K slot nk%3 last held the K of step nk-3: free once S_{nk-3} completed
-          if (nk < nsteps && mbar_test(&s_full[nk % kRing], ((nk / kRing) & 1) ^ 1)) {
+          if (nk < nsteps && mbar_test(&k_free[nk % kRing], ((nk / kRing) & 1) ^ 1)) {
             const int ks = nk % kRing;
             uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
             mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
@@ -198,7 +221,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
             did = true;
           }
           // V slot nv%3 last held the V of step nv-3: free once PV_{nv-3} completed
-          if (nv < nk && mbar_test(&p_free[nv % kRing], ((nv / kRing) & 1) ^ 1)) {
+          if (nv < nk && mbar_test(&v_free[nv % kRing], ((nv / kRing) & 1) ^ 1)) {
             const int vs = nv % kRing;
             uint8_t* dst = sm + L::kV0 + vs * L::kSlotBytes;
             mbar_arrive_expect_tx(&v_full[vs], L::kSlotBytes);
@@ -231,17 +254,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::kK0), 16, 1024);
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
       for (int sj = 0; sj < nsteps && ok; ++sj) {
-        const int b = sj % kRing;
-        // K of step sj landed; S buffer b read by the softmax warps (S_{sj-3})
+        const int b = sj % kRing, gs = sj & 1;
+        // K of step sj landed; the group's S buffer read by its warps (its previous step)
         ok = mbar_wait_abortable(&k_full[b], (sj / kRing) & 1, status, abort_flag) &&
-             mbar_wait_abortable(&s_free[b], ((sj / kRing) & 1) ^ 1, status, abort_flag);
+             mbar_wait_abortable(&s_free[gs], ((sj >> 1) & 1) ^ 1, status, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dK = dK0 + uint64_t(b * (L::kSlotBytes >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws_ts(tbase + b * 64, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
-        mma_commit(&s_full[b]);
+          mma_ws_ts(tbase + gs * 64, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+        mma_commit(&s_full[gs]);
+        mma_commit(&k_free[b]);
       }
       // every product this thread issued has completed before TMEM is released
       mma_commit(mma_done);
@@ -250,26 +274,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   } else if (warp == kPvWarp) {
     // ------------------------------------------------------------ value issuer
     if (lane == 0 && nsteps > 0) {
-      const uint32_t idO = idesc_bf16_f32(64, 128, false, true);
-      // V: MN-major B of PV whose two 64-column halves are the same 64
-      // channels of V of key block 0 and of key block 1 (LBO = the block
-      // stride), so N = 128 covers one channel group for both blocks.
-      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), D * 128, 1024);
+      // B = V of the step, MN-major, N = 2d: the d channels of key block 0
+      // (64-column chunks kBoxBytes apart, as the slot holds [block][dh]),
+      // then those of key block 1. One product per 16-key step.
+      const uint32_t idO = idesc_bf16_f32(64, 2 * D, false, true);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::kV0), kBoxBytes, 1024);
       bool ok = true;
       for (int pj = 0; pj < nsteps && ok; ++pj) {
-        const int b = pj % kRing;
-        ok = mbar_wait_abortable(&p_full[b], (pj / kRing) & 1, status, abort_flag) &&
+        const int b = pj % kRing, gp = pj & 1;
+        ok = mbar_wait_abortable(&p_full[gp], (pj >> 1) & 1, status, abort_flag) &&
              mbar_wait_abortable(&v_full[b], (pj / kRing) & 1, status, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dV = dV0 + uint64_t(b * (L::kSlotBytes >> 4));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            mma_ws_ts(tO + c * 64, tP + b * 32 + kk * 8, dV + uint64_t((c * kBoxBytes + kk * 2048) >> 4), idO,
-                      (pj > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&p_free[b]);
+          mma_ws_ts(tO + gp * D, tP + gp * 32 + kk * 8, dV + uint64_t((kk * 2048) >> 4), idO,
+                    (pj >= kGroups || kk > 0) ? 1u : 0u);
+        mma_commit(&p_free[gp]);
+        mma_commit(&v_free[b]);
       }
       mma_commit(pv_done);
       mbar_wait(pv_done, 0, status);
@@ -277,55 +300,42 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   } else {
     // ------------------------------------------------------------ softmax
     const int sw = warp - 2;
-    const int sp = warp & 3;
-    const int ch = sw >> 2;
+    const int grp = sw / kGroupWarps;
+    const int sp = warp & 3;  // TMEM lane quarter of this warp
     const int Ln = sp * 32 + lane;
     const int m = Ln & 63, kh = Ln >> 6;
-    const int q4 = kh * 2 + ch;
+    const int part = grp * 2 + kh;  // warp-uniform
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
     float m_run = -INFINITY, l_part = 0.f;
     if (nsteps > 0) {
       // Q becomes the A operand of every S product: one copy into TMEM
+      // (the two groups copy the two column halves)
       mbar_wait_abortable(q_full, 0, status, abort_flag);
-      tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, grp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(qa_full);
     }
-    for (int j = 0; j < nsteps; ++j) {
-      const int b = j % kRing, rb = j & 1;
+    int k = 0;  // this group's step count
+    for (int j = grp; j < nsteps; j += kGroups, ++k) {
       const bool valid = (j * kKB + kh) < cnt;  // warp-uniform: kh is fixed per warp
       // keys of a key block clipped by the grid's edge (read before the wait)
-      uint32_t members = 0xffffffffu;
-      if (g.partial && valid)
-        members = uint32_t(key_block_members(g, P.zone_shape, __ldg(P.col_idx + beg + j * kKB + kh)) >> (ch * 32));
-      mbar_wait_abortable(&s_full[b], (j / kRing) & 1, status, abort_flag);
+      uint64_t members = ~uint64_t(0);
+      if (g.partial && valid) members = key_block_members(g, P.zone_shape, __ldg(P.col_idx + beg + j * kKB + kh));
+      mbar_wait_abortable(&s_full[grp], k & 1, status, abort_flag);
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tbase + lane_off + b * 64 + ch * 32, r);
+      uint32_t r[64];
+      tmem_ld32(tbase + lane_off + grp * 64, r);
+      tmem_ld32(tbase + lane_off + grp * 64 + 32, r + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
-      mask_scores32(r, members);
-      float mx = -INFINITY;
-      if (valid) {
-        // two chains of three-input maxima over r[0..29], then r[30], r[31]
-        float ca = fmax3(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]));
-        float cb = fmax3(__uint_as_float(r[3]), __uint_as_float(r[4]), __uint_as_float(r[5]));
-#pragma unroll
-        for (int i = 6; i < 30; i += 4) {
-          ca = fmax3(ca, __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-          cb = fmax3(cb, __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-        }
-        mx = fmaxf(fmax3(ca, cb, __uint_as_float(r[30])), __uint_as_float(r[31]));
-        mx *= P.scale_log2;  // the scale is positive, so it commutes with the max
-      }
-      red[(rb * 4 + q4) * 64 + m] = mx;
-      named_bar_sync(1, 32 * kSoftWarps);
-      const float mb = fmaxf(fmaxf(red[(rb * 4 + 0) * 64 + m], red[(rb * 4 + 1) * 64 + m]),
-                             fmaxf(red[(rb * 4 + 2) * 64 + m], red[(rb * 4 + 3) * 64 + m]));
-      const float m_new = fmaxf(m_run, mb);
+      if (lane == 0) mbar_arrive(&s_free[grp]);
+      mask_scores32(r, uint32_t(members));
+      mask_scores32(r + 32, uint32_t(members >> 32));
+      // the scale is positive, so it commutes with the max
+      const float mx = valid ? max64(r) * P.scale_log2 : -INFINITY;
+      const float m_new = fmaxf(m_run, mx);
       const bool resc = m_new > m_run + kRescaleThreshold;
       if (__any_sync(0xffffffffu, resc)) {
         const float alpha = resc ? fast_exp2(m_run - m_new) : 1.f;
@@ -333,14 +343,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
           l_part *= alpha;
           m_run = m_new;
         }
-        if (j > 0) {
-          // this lane's O part holds PV_0 .. PV_{j-1}: wait for the last, then rescale
-          mbar_wait_abortable(&p_free[(j - 1) % kRing], ((j - 1) / kRing) & 1, status, abort_flag);
+        if (k > 0) {
+          // this lane's O part holds the group's earlier PVs: wait for the last, then rescale
+          mbar_wait_abortable(&p_free[grp], (k - 1) & 1, status, abort_flag);
           tc_fence_after();
 #pragma unroll
-          for (int h = 0; h < D / 64; ++h) {
+          for (int h = 0; h < D / 32; ++h) {
             uint32_t o[32];
-            const uint32_t ta = tO + lane_off + ch * (D / 2) + h * 32;
+            const uint32_t ta = tO + grp * D + lane_off + h * 32;
             tmem_ld32(ta, o);
             tmem_ld_wait();
 #pragma unroll
@@ -351,60 +361,91 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
           tmem_st_wait();
         }
       }
-      uint32_t pk[16];
+      uint32_t pk[32];
       if (valid) {
         // m_run is finite unless every key so far lay outside the grid (then every p is 0)
         const float c = P.scale_log2, nm = m_run == -INFINITY ? 0.f : -m_run;
-        float lsum = 0.f;
+        float la = 0.f, lb = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 32; ++i) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(r[2 * i]), c, nm));
           const float p1 = fast_exp2(fmaf(__uint_as_float(r[2 * i + 1]), c, nm));
-          lsum += p0 + p1;
+          la += p0;
+          lb += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        l_part += lsum;
+        l_part += la + lb;
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = 0u;
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
       }
-      // P buffer b last held P_{j-3}: free once PV_{j-3} completed
-      if (j >= kRing) mbar_wait_abortable(&p_free[b], ((j / kRing) & 1) ^ 1, status, abort_flag);
-      tmem_st16(tP + lane_off + b * 32 + ch * 16, pk);
+      // the group's P buffer: free once its previous PV completed
+      if (k > 0) mbar_wait_abortable(&p_free[grp], (k - 1) & 1, status, abort_flag);
+      tmem_st16(tP + lane_off + grp * 32, pk);
+      tmem_st16(tP + lane_off + grp * 32 + 16, pk + 16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[b]);
+      if (lane == 0) mbar_arrive(&p_full[grp]);
     }
     // ---------------------------------------------------------- epilogue
-    if (nsteps > 0) mbar_wait_abortable(&p_free[(nsteps - 1) % kRing], ((nsteps - 1) / kRing) & 1, status, abort_flag);
+    // k = this group's step count; its last PV complete before O is read
+    if (k > 0) mbar_wait_abortable(&p_free[grp], (k - 1) & 1, status, abort_flag);
     tc_fence_after();
-    redl[q4 * 64 + m] = l_part;
+    redm[part * 64 + m] = m_run;
+    redl[part * 64 + m] = l_part;
     named_bar_sync(1, 32 * kSoftWarps);
     const bool ok = *abort_flag == 0;  // uniform: read after the barrier
-    const float l = redl[m] + redl[64 + m] + redl[128 + m] + redl[192 + m];
-    const float inv = (l > 0.f && ok) ? 1.f / l : 0.f;
+    // merge the row's four parts: max M, sum L = sum_p l_p 2^(m_p - M)
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) M = fmaxf(M, redm[q * 64 + m]);
+    float Lsum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lq = redl[q * 64 + m];
+      if (lq > 0.f) Lsum += lq * fast_exp2(redm[q * 64 + m] - M);
+    }
+    const float inv = (Lsum > 0.f && ok) ? 1.f / Lsum : 0.f;
+    const float w = (l_part > 0.f) ? fast_exp2(m_run - M) * inv : 0.f;
     const int sI = safe_shape(g, P.zone_shape, I, status);
     const BlockBox qb = block_box(g, sI, I);
     const int tok = block_token(g, qb, m);
     // a query slot outside the grid (a block clipped by the edge) has no output
     const bool row_in = !g.partial || block_slot_in_grid(g, qb, m);
-    // This lane holds the key-block-kh part of O row m over channels
-    // [ch*D/2, ch*D/2 + D/2). It keeps the quarter [.. + kh*D/4, + D/4) and
-    // hands the other quarter to the thread of the other lane half.
+    // This thread keeps channel quarter `part` of row m and hands the other
+    // three quarters of its scaled part to the threads that keep them.
     constexpr int NC = D / 4;
-    const int keep = ch * (D / 2) + kh * NC, give = ch * (D / 2) + (kh ^ 1) * NC;
+    float* X = reinterpret_cast<float*>(sm + L::kK0);
     float ov[NC];
-    if (nsteps > 0) {  // uniform; on an abort the values are discarded below
-      float gv[NC];
-      tmem_ld_f<NC>(tO + lane_off + give, gv);
-      tmem_ld_f<NC>(tO + lane_off + keep, ov);
-      float* xo = reinterpret_cast<float*>(sm + L::kK0) + ((kh * 2 + ch) * 64 + m) * L::kXPitch;
 #pragma unroll
-      for (int i = 0; i < NC / 4; ++i)
-        reinterpret_cast<float4*>(xo)[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
-      named_bar_sync(1, 32 * kSoftWarps);
-      const float* xi = reinterpret_cast<const float*>(sm + L::kK0) + (((kh ^ 1) * 2 + ch) * 64 + m) * L::kXPitch;
+    for (int i = 0; i < NC; ++i) ov[i] = 0.f;
+#pragma unroll
+    for (int qd = 0; qd < 4; ++qd) {
+      float v[NC];
+      if (k > 0) {  // warp-uniform; a group with no step has no O part
+        tmem_ld_f<NC>(tO + grp * D + lane_off + qd * NC, v);
+#pragma unroll
+        for (int i = 0; i < NC; ++i) v[i] = w == 0.f ? 0.f : v[i] * w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < NC; ++i) v[i] = 0.f;
+      }
+      if (qd == part) {
+#pragma unroll
+        for (int i = 0; i < NC; ++i) ov[i] = v[i];
+      } else {
+        float* xo = X + ((part * 4 + qd) * 64 + m) * L::kXPitch;
+#pragma unroll
+        for (int i = 0; i < NC / 4; ++i)
+          reinterpret_cast<float4*>(xo)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    }
+    named_bar_sync(1, 32 * kSoftWarps);
+#pragma unroll
+    for (int src = 0; src < 4; ++src) {
+      if (src == part) continue;
+      const float* xi = X + ((src * 4 + part) * 64 + m) * L::kXPitch;
 #pragma unroll
       for (int i = 0; i < NC / 4; ++i) {
         const float4 t = reinterpret_cast<const float4*>(xi)[i];
@@ -413,23 +454,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
         ov[4 * i + 2] += t.z;
         ov[4 * i + 3] += t.w;
       }
-#pragma unroll
-      for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : ov[i] * inv;
-    } else {
-#pragma unroll
-      for (int i = 0; i < NC; ++i) ov[i] = 0.f;
     }
-    if (row_in) store_row<NC>(P.o, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, ov, P.out_fp32);
+    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + part * NC;
+    if (row_in) store_row<NC>(P.o, off, ov, P.out_fp32);
     if (P.o_lo && row_in) {
       // what the bf16 store of O dropped: O = o + o_lo to about 16 bits
       float lo[NC];
 #pragma unroll
       for (int i = 0; i < NC; ++i) lo[i] = ov[i] - __bfloat162float(__float2bfloat16_rn(ov[i]));
-      store_row<NC>(P.o_lo, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, lo, false);
+      store_row<NC>(P.o_lo, off, lo, false);
     }
-    if (q4 == 0 && row_in) {
+    if (part == 0 && row_in) {
       const int N = g.T * g.H * g.W;
-      P.lse[int64_t(head) * N + tok] = (l > 0.f && ok) ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      P.lse[int64_t(head) * N + tok] = (Lsum > 0.f && ok) ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
     }
   }
   tc_fence_before();
