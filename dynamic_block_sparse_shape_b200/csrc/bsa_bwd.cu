@@ -38,6 +38,7 @@ namespace {
 
 constexpr int kKB = 2;
 constexpr int kSoftWarps = 8;
+constexpr int kGroupWarps = 4;  // dq: the softmax warps form two groups taking alternate steps
 constexpr int kBwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kIssuerB = 2 + kSoftWarps;  // warp of the second MMA issuer
 
@@ -67,30 +68,37 @@ struct BwdParams {
 
 // ----------------------------------------------------------------------- dq
 // Three slots, each holding K and V of one step (two key blocks) from its load
-// until the dQ product of that step completes. S / dP in TMEM (2 buffers
-// each). Q and dO are staged through shared memory once and copied into TMEM
-// (the A operands of every S / dP product); that shared-memory space then
-// holds dS in two buffers, the A operand of the dQ products.
+// until the dQ product of that step completes. Q and dO are staged through
+// shared memory once and copied into TMEM (the A operands of every S / dP
+// product).
+// The softmax warps form two groups of four taking alternate steps (group
+// j % 2 takes step j), one thread per TMEM lane: the thread in lane m + 64 kh
+// holds row m of S_j and dP_j against key block kh of the step (64 values
+// each) and writes dS (bf16) back over the first 32 columns of its group's S
+// buffer. dS is thus the TMEM A operand of the dQ product, and the .ws lane
+// split makes lane half kh accumulate the key-block-kh part of dQ: the B
+// operand's two 64-column halves are the same 64 channels of K of key block 0
+// and of key block 1. The two parts are added once, in the epilogue.
 // Two threads issue the products, each in step order: warp 1 issues
-// A_j = (S_j = Q K_j^T, dP_j = dO V_j^T) once slot j has landed and the
-// softmax warps have read the score buffers of step j - 2; warp 10 issues
-// B_j = (dQ += dS_j K_j) once dS_j is written. While one waits on a barrier
-// the other's products keep the tensor pipe busy. dS_j goes to buffer j % 2
-// and has its own ready barrier per buffer, so a parity wait on it can never
-// be two phases behind.
+// A_j = (S_j = Q K_j^T, dP_j = dO V_j^T) into group (j % 2)'s buffers once
+// slot j has landed and that group's previous dQ product (which read dS from
+// the same buffer) has completed; warp 10 issues B_j = (dQ_parts += dS_j K_j)
+// once dS_j is written. While one waits on a barrier the other's products keep
+// the tensor pipe busy.
 template <int D>
 struct DqSmem {
-  static constexpr uint32_t kQD = 0;                 // Q, dO staging [2][dh][64][128 B]; then dS [2]
-  static constexpr uint32_t kQDBytes = 32768;        // max(2 * D * 128, two dS buffers)
-  static constexpr uint32_t kDSBytes = kKB * kBoxBytes;  // [key block][64 rows][128 B]
+  static constexpr uint32_t kQD = 0;               // Q, dO staging [2][dh][64][128 B]
+  static constexpr uint32_t kQDBytes = 2 * D * 128;
   static constexpr uint32_t kHalf = kKB * D * 128;   // K (or V) of one step, [dh][key block][64][128 B]
   static constexpr uint32_t kSlotBytes = 2 * kHalf;  // K then V
   static constexpr int kSlots = 3;
   static constexpr uint32_t kSlot0 = kQDBytes;
-  static constexpr uint32_t kDesc = kSlot0 + kSlots * kSlotBytes;  // block coordinate ring
-  static constexpr uint32_t kBar = kDesc + kDescRing * 16;
+  static constexpr uint32_t kDesc = kSlot0 + kSlots * kSlotBytes;  // block-id ring
+  static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 256;
-  static_assert(2 * D * 128 <= kQDBytes && 2 * kDSBytes <= kQDBytes, "staging tile");
+  // epilogue exchange of dQ part quarters: [kh][group][64 rows][D/4 + 4 floats], over the slots
+  static constexpr uint32_t kXPitch = D / 4 + 4;
+  static_assert(4 * 64 * kXPitch * 4 <= kSlots * kSlotBytes, "exchange buffer fits the slots");
 };
 
 template <int D>
@@ -103,15 +111,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   uint64_t* qd_full = bars + 0;
   uint64_t* kv_full = bars + 1;    // [3] K and V of the slot's step landed
   uint64_t* kv_free = bars + 4;    // [3] dQ product of the slot's step complete
-  uint64_t* s_full = bars + 7;     // [2] A_j complete
-  uint64_t* ds_full = bars + 9;    // [2] dS_j written (8 softmax warps), index j % 2
-  uint64_t* ds_free = bars + 11;   // [2] B_j complete (dS buffer j % 2 free)
+  uint64_t* s_full = bars + 7;     // [2] per group: its A complete
+  uint64_t* ds_full = bars + 9;    // [2] per group: its dS written to TMEM (4 warps)
+  uint64_t* ds_free = bars + 11;   // [2] per group: its B complete (its S / dP buffers free)
   uint64_t* mma_done = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
   uint64_t* qa_full = bars + 16;  // Q and dO copied into TMEM by the softmax warps
-  uint64_t* s_free = bars + 17;   // [2] S_j, dP_j read by the softmax warps, index j % 2
-  uint64_t* b_done = bars + 19;   // every B product complete
+  uint64_t* b_done = bars + 17;   // every B product complete
 
   const Geo& g = P.g;
   const int I = blockIdx.x, head = blockIdx.y;
@@ -133,9 +140,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&ds_full[i], kSoftWarps);
+      mbar_init(&ds_full[i], kGroupWarps);
       mbar_init(&ds_free[i], 1);
-      mbar_init(&s_free[i], kSoftWarps);
     }
     mbar_init(mma_done, 1);
     mbar_init(b_done, 1);
@@ -151,8 +157,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  // TMEM columns: S [2 x 64] at 0, dP [2 x 64] at 128, dQ at 256, Q at 320, dO at 384
-  const uint32_t tdQ = tbase + 256, tQ = tbase + 320, tDO = tbase + 384;
+  // TMEM columns: S [2 groups x 64] at 0 (dS over its first 32), dP [2 x 64]
+  // at 128, dQ parts at 256 (D columns), Q at 384, dO at 448
+  const uint32_t tdQ = tbase + 256, tQ = tbase + 384, tDO = tbase + 448;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -208,11 +215,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
       const uint64_t dV0 = sdesc_sw128(sK0 + L::kHalf, 16, 1024);  // V as B of dP
       constexpr uint64_t kSlotStep = L::kSlotBytes >> 4;
       bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
-      // A_j: S_j and dP_j into score buffer j % 2, once slot j has landed and
-      // the softmax warps have read that buffer's step j - 2
+      // A_j: S_j and dP_j into group (j % 2)'s buffers, once slot j has landed
+      // and that group's previous B (which read dS from the S buffer) completed
       for (int j = 0; j < nsteps && ok; ++j) {
         ok = mbar_wait_abortable(&kv_full[j % NS], (j / NS) & 1, status, abort_flag) &&
-             mbar_wait_abortable(&s_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
+             mbar_wait_abortable(&ds_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = uint64_t(j % NS) * kSlotStep;
@@ -232,11 +239,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   } else if (warp == kIssuerB) {
     // ------------------------------------------------------------ B issuer
     if (lane == 0 && nsteps > 0) {
-      const uint32_t idQ = idesc_bf16_f32(64, D, false, true);
-      const uint64_t dDS0 = sdesc_sw128(smem_u32(sm + L::kQD), 16, 1024);
-      const uint64_t dKmn0 = sdesc_sw128(smem_u32(sm + L::kSlot0), kKB * kBoxBytes, 1024);  // K as B of dQ
+      // B = K of the step, MN-major, N = 128: 64 channels of key block 0
+      // then the same channels of key block 1 (LBO = the block stride)
+      const uint32_t idQ = idesc_bf16_f32(64, 128, false, true);
+      const uint64_t dKmn0 = sdesc_sw128(smem_u32(sm + L::kSlot0), kBoxBytes, 1024);
       constexpr uint64_t kSlotStep = L::kSlotBytes >> 4;
-      constexpr uint64_t kDSStep = L::kDSBytes >> 4;
       bool ok = true;
       // B_j once dS_j is written (which implies A_j, hence slot j, complete)
       for (int j = 0; j < nsteps && ok; ++j) {
@@ -244,11 +251,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = uint64_t(j % NS) * kSlotStep;
-        const uint64_t dDS = dDS0 + uint64_t(j & 1) * kDSStep;
+        const uint32_t tDS = tbase + (j & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-          mma_ws(tdQ, dDS + kmajor_step(kk, kBoxBytes), dKmn0 + so + mnmajor_step(kk, kBoxBytes), idQ,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            mma_ws_ts(tdQ + c * 64, tDS + kk * 8, dKmn0 + so + uint64_t((c * kKB * kBoxBytes + kk * 2048) >> 4), idQ,
+                      (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&kv_free[j % NS]);
         mma_commit(&ds_free[j & 1]);
       }
@@ -257,72 +266,92 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int sw = warp - 2, sp = warp & 3, ch = sw >> 2;
+    const int sw = warp - 2, grp = sw / kGroupWarps, sp = warp & 3;
     const int Ln = sp * 32 + lane;
     const int m = Ln & 63, kh = Ln >> 6;
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
     const float lse2 = P.lse2[size_t(row) * 64 + m];
     const float dm = P.dvec[size_t(row) * 64 + m];
     if (nsteps > 0) {
-      // Q and dO are the A operands of every S / dP product: one copy into TMEM
+      // Q and dO are the A operands of every S / dP product: one copy into
+      // TMEM (the two groups copy the two column halves)
       mbar_wait_abortable(qd_full, 0, status, abort_flag);
-      tile_to_tmem_a<D>(sm + L::kQD, tQ + lane_off, m, ch);
-      tile_to_tmem_a<D>(sm + L::kQD + D * 128, tDO + lane_off, m, ch);
+      tile_to_tmem_a<D>(sm + L::kQD, tQ + lane_off, m, grp);
+      tile_to_tmem_a<D>(sm + L::kQD + D * 128, tDO + lane_off, m, grp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(qa_full);
-      // the staging tile holds dS from now on: every softmax warp has read it
-      named_bar_sync(1, 32 * kSoftWarps);
     }
-    for (int j = 0; j < nsteps; ++j) {
-      const int sb = j & 1;
+    int k = 0;  // this group's step count
+    for (int j = grp; j < nsteps; j += 2, ++k) {
       const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
       // keys of a key block clipped by the grid's edge (read before the wait)
-      uint32_t members = 0xffffffffu;
-      if (g.partial && valid)
-        members = uint32_t(key_block_members(g, P.zone_shape, __ldg(P.idx + beg + j * kKB + kh)) >> (ch * 32));
-      mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
+      uint64_t members = ~uint64_t(0);
+      if (g.partial && valid) members = key_block_members(g, P.zone_shape, __ldg(P.idx + beg + j * kKB + kh));
+      mbar_wait_abortable(&s_full[grp], k & 1, status, abort_flag);
       tc_fence_after();
-      uint32_t rs[32], rp[32];
-      tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
-      tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
-      tmem_ld_wait();
-      // the score buffers are free for A_{j+2}
+      uint32_t pk[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32(tbase + lane_off + grp * 64 + h * 32, rs);
+        tmem_ld32(tbase + lane_off + 128 + grp * 64 + h * 32, rp);
+        tmem_ld_wait();
+        mask_scores32(rs, uint32_t(members >> (32 * h)));  // P = exp2(-inf) = 0 there, hence dS = 0
+        if (valid) {
+          const float c = P.scale_log2, nl = -lse2;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(rs[2 * i]), c, nl));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(rs[2 * i + 1]), c, nl));
+            pk[16 * h + i] =
+                pack_bf16x2(p0 * (__uint_as_float(rp[2 * i]) - dm), p1 * (__uint_as_float(rp[2 * i + 1]) - dm));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[16 * h + i] = 0u;
+        }
+      }
+      // dS over the first 32 columns of the S buffer (every S / dP value of
+      // this lane was read above)
+      tmem_st16(tbase + lane_off + grp * 64, pk);
+      tmem_st16(tbase + lane_off + grp * 64 + 16, pk + 16);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      mask_scores32(rs, members);  // P = exp2(-inf) = 0 there, hence dS = 0
-      uint32_t pk[16];
-      if (valid) {
-        const float c = P.scale_log2, nl = -lse2;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(rs[2 * i]), c, nl));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(rs[2 * i + 1]), c, nl));
-          pk[i] = pack_bf16x2(p0 * (__uint_as_float(rp[2 * i]) - dm), p1 * (__uint_as_float(rp[2 * i + 1]) - dm));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = 0u;
-      }
-      // dS buffer j % 2 last held dS_{j-2}: free once B_{j-2} completed
-      if (j >= 2) mbar_wait_abortable(&ds_free[sb], ((j - 2) >> 1) & 1, status, abort_flag);
-      uint8_t* pt = sm + L::kQD + sb * L::kDSBytes + kh * kBoxBytes;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
-            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full[sb]);
+      if (lane == 0) mbar_arrive(&ds_full[grp]);
     }
-    if (nsteps > 0) mbar_wait_abortable(&ds_free[(nsteps - 1) & 1], ((nsteps - 1) >> 1) & 1, status, abort_flag);
+    // ---------------------------------------------------------- epilogue
+    // this group's last B complete; once both groups are here every product
+    // is complete and the slots hold the exchange buffer
+    if (k > 0) mbar_wait_abortable(&ds_free[grp], (k - 1) & 1, status, abort_flag);
     tc_fence_after();
+    named_bar_sync(1, 32 * kSoftWarps);
     const bool ok = *abort_flag == 0;
+    // This thread holds the key-block-kh part of dQ row m; it keeps channel
+    // quarter grp * 2 + kh and hands quarter grp * 2 + (kh ^ 1) to the thread
+    // of the other lane half.
     constexpr int NC = D / 4;
+    const int keep = grp * (D / 2) + kh * NC, give = grp * (D / 2) + (kh ^ 1) * NC;
     float v[NC];
-    if (nsteps > 0) {
-      tmem_ld_f<NC>(tdQ + lane_off + ch * NC, v);
+    if (nsteps > 0) {  // uniform; on an abort the values are discarded below
+      float gv[NC];
+      tmem_ld_f<NC>(tdQ + lane_off + give, gv);
+      tmem_ld_f<NC>(tdQ + lane_off + keep, v);
+      float* xo = reinterpret_cast<float*>(sm + L::kSlot0) + ((kh * 2 + grp) * 64 + m) * L::kXPitch;
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i)
+        reinterpret_cast<float4*>(xo)[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
+      named_bar_sync(1, 32 * kSoftWarps);
+      const float* xi = reinterpret_cast<const float*>(sm + L::kSlot0) + (((kh ^ 1) * 2 + grp) * 64 + m) * L::kXPitch;
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i) {
+        const float4 t = reinterpret_cast<const float4*>(xi)[i];
+        v[4 * i] += t.x;
+        v[4 * i + 1] += t.y;
+        v[4 * i + 2] += t.z;
+        v[4 * i + 3] += t.w;
+      }
 #pragma unroll
       for (int i = 0; i < NC; ++i) v[i] = ok ? v[i] * P.scale : 0.f;
     } else {
@@ -333,8 +362,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     const BlockBox qb = block_box(g, sI, I);
     const int tok = block_token(g, qb, m);
     if (!g.partial || block_slot_in_grid(g, qb, m))  // a slot outside the grid has no row
-      store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * (D / 2) + ch * NC, v,
-                    P.out_fp32);
+      store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, v, P.out_fp32);
   }
   tc_fence_before();
   __syncthreads();
