@@ -378,8 +378,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
 // The K/V tile is staged through shared memory once, copied into TMEM (the A
 // operand of every S^T / dP^T product) and its shared-memory space then holds
 // P^T and dS^T, the A operands of the dV / dK products. LSE and D of the
-// step's query rows come straight from global memory into registers, one
-// step ahead.
+// step's two query blocks are copied with the stage (bulk copies counted on
+// the stage's barrier) into one of two small buffers, released by the
+// softmax warps once read: no global load sits on the softmax warps' path.
 // Two threads issue the products, each in step order: warp 1 issues
 // A_j = (S^T_j, dP^T_j) once stage j has landed and the softmax warps have
 // read the score buffers of step j - 2; warp 10 issues
@@ -396,10 +397,16 @@ struct DkvSmem {
   static constexpr uint32_t kStageBytes = 2 * kHalf;
   static constexpr int kStages = 3;
   static constexpr uint32_t kStage0 = kKVBytes;
-  static constexpr uint32_t kDesc = kStage0 + kStages * kStageBytes;  // block coordinate ring
-  static constexpr uint32_t kBar = kDesc + kDescRing * 16;
+  // LSE * log2(e) and D of the step's query blocks, [2 buffers][query block][lse2 64 | D 64] floats
+  static constexpr uint32_t kLD0 = kStage0 + kStages * kStageBytes;
+  static constexpr uint32_t kLDBytes = kKB * 2 * 64 * 4;
+  static constexpr uint32_t kDesc = kLD0 + 2 * kLDBytes;  // block-id ring
+  static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 256;
   static_assert(2 * D * 128 <= kKVBytes && kDST + kKB * kBoxBytes <= kKVBytes, "staging tile");
+  // allocated without alignment slack: the kernel checks that the dynamic
+  // shared memory starts on a 1024-byte boundary
+  static_assert(kTotal <= 227 * 1024, "shared-memory budget");
 };
 
 template <int D>
@@ -407,7 +414,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   using L = DkvSmem<D>;
   constexpr int NS = L::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // the 128-byte-swizzled tiles need 1024-byte alignment and there is no
+  // slack to align up: refuse (reported, no access) if the start is off
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(P.status, kDevErrBounds);
+    return;
+  }
+  uint8_t* sm = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* st_full = bars + 1;   // [3] stage landed
@@ -421,6 +434,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   uint64_t* ka_full = bars + 14;  // K and V copied into TMEM by the softmax warps
   uint64_t* s_free = bars + 15;   // [2] S^T_j, dP^T_j read by the softmax warps, index j % 2
   uint64_t* b_done = bars + 17;   // every B product complete
+  uint64_t* ld_free = bars + 18;  // [2] LSE / D buffer read by the 8 softmax warps
 
   const Geo& g = P.g;
   const int J = blockIdx.x, head = blockIdx.y;
@@ -445,6 +459,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       mbar_init(&s_free[i], kSoftWarps);
     }
     mbar_init(b_done, 1);
+    mbar_init(&ld_free[0], kSoftWarps);
+    mbar_init(&ld_free[1], kSoftWarps);
     mbar_init(ps_full, kSoftWarps);
     mbar_init(ps_free, 1);
     mbar_init(mma_done, 1);
@@ -487,7 +503,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
           if (j >= NS) ok = mbar_wait_abortable(&st_free[s], ((j / NS) - 1) & 1, status, abort_flag);
           if (ok) {
             uint8_t* stage = sm + L::kStage0 + s * L::kStageBytes;
-            mbar_arrive_expect_tx(&st_full[s], L::kStageBytes);
+            mbar_arrive_expect_tx(&st_full[s], L::kStageBytes + L::kLDBytes);
             for (int slot = 0; slot < kKB; ++slot) {
               const size_t io = image_offset(g, head, dc.get(kKB * j + slot), D);
               for (int dh = 0; dh < D / 64; ++dh) {
@@ -497,6 +513,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
               }
             }
             issued = j + 1;
+            // LSE / D buffer j % 2 last held step j - 2: free once the softmax
+            // warps read it. The copies are issued even after a failed wait
+            // (an abort, results discarded) so that the stage's barrier completes.
+            ok = mbar_wait_abortable(&ld_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
+            uint8_t* ldb = sm + L::kLD0 + (j & 1) * L::kLDBytes;
+            for (int slot = 0; slot < kKB; ++slot) {
+              const size_t ro = (size_t(head) * g.n_blocks + dc.get(kKB * j + slot)) * 64;
+              bulk_load(ldb + slot * 512, P.lse2 + ro, 256, &st_full[s]);
+              bulk_load(ldb + slot * 512 + 256, P.dvec + ro, 256, &st_full[s]);
+            }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -575,25 +601,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     const int Ln = sp * 32 + lane;
     const int m = Ln & 63, kh = Ln >> 6;
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
-    // LSE * log2(e) and D of the 32 query rows this thread scores in step j
-    // (query block kh of the step, rows ch*32 ..), loaded one step ahead
-    float4 l2[8], dd[8];
-    auto load_ld = [&](int j) {
-      int e = kKB * j + kh;
-      if (e >= cnt) e = kKB * j;
-      int Iq = P.idx[beg + e];
-      if (Iq < 0 || Iq >= g.n_blocks) Iq = 0;  // reported by the coordinate cache
-      const size_t rowoff = (size_t(head) * g.n_blocks + Iq) * 64 + ch * 32;
-      const float4* a = reinterpret_cast<const float4*>(P.lse2 + rowoff);
-      const float4* b = reinterpret_cast<const float4*>(P.dvec + rowoff);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        l2[i] = __ldg(a + i);
-        dd[i] = __ldg(b + i);
-      }
-    };
     if (nsteps > 0) {
-      load_ld(0);
       // K and V are the A operands of every S^T / dP^T product: one copy into TMEM
       mbar_wait_abortable(kv_full, 0, status, abort_flag);
       tile_to_tmem_a<D>(sm + L::kKV, tK + lane_off, m, ch);
@@ -607,6 +615,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     for (int j = 0; j < nsteps; ++j) {
       const int sb = j & 1;
       mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
+      // the stage's copies (LSE / D included) have landed: A_j read the stage,
+      // and the wait makes the copied LSE / D visible to this warp
+      mbar_wait_abortable(&st_full[j % NS], (j / NS) & 1, status, abort_flag);
       tc_fence_after();
       uint32_t rs[32], rp[32];
       tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
@@ -617,6 +628,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[sb]);
       const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
+      // LSE * log2(e) and D of the 32 query rows this thread scores (query
+      // block kh of the step, rows ch*32 ..)
+      const float4* ldp = reinterpret_cast<const float4*>(sm + L::kLD0 + (j & 1) * L::kLDBytes + kh * 512) + ch * 8;
+      float4 l2[8], dd[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        l2[i] = ldp[i];
+        dd[i] = ldp[16 + i];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ld_free[j & 1]);
       uint32_t pp[16], pd[16];
       if (valid) {
         const float c = P.scale_log2;
@@ -637,7 +659,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
 #pragma unroll
         for (int i = 0; i < 16; ++i) pp[i] = pd[i] = 0u;
       }
-      if (j + 1 < nsteps) load_ld(j + 1);  // in flight while this step is stored
       // the P^T / dS^T buffer last held step j - 1: free once B_{j-1} completed
       if (j >= 1) mbar_wait_abortable(ps_free, (j - 1) & 1, status, abort_flag);
       uint8_t* pt = sm + L::kPT + kh * kBoxBytes;
@@ -947,13 +968,13 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   P.out0 = dk;
   P.out1 = dv;
   if (head_dim == 128) {
-    const size_t smem = DkvSmem<128>::kTotal + 1024;
+    const size_t smem = DkvSmem<128>::kTotal;
     if (cudaFuncSetAttribute(bsa_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
         cudaSuccess)
       return PRISM_ERR_CUDA;
     bsa_dkdv_kernel<128><<<grid, kBwdThreads, smem, s>>>(P);
   } else {
-    const size_t smem = DkvSmem<64>::kTotal + 1024;
+    const size_t smem = DkvSmem<64>::kTotal;
     if (cudaFuncSetAttribute(bsa_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
         cudaSuccess)
       return PRISM_ERR_CUDA;
