@@ -38,7 +38,7 @@ namespace {
 
 constexpr int kKB = 2;
 constexpr int kSoftWarps = 8;
-constexpr int kGroupWarps = 4;  // dq: the softmax warps form two groups taking alternate steps
+constexpr int kGroupWarps = 4;  // the softmax warps form two groups taking alternate steps
 constexpr int kBwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kIssuerB = 2 + kSoftWarps;  // warp of the second MMA issuer
 
@@ -373,26 +373,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
 }
 
 // --------------------------------------------------------------------- dkdv
-// Three stages of (Q, dO) for two query blocks, each held from its load until
-// the dV/dK products of its step complete. S^T / dP^T in TMEM (2 buffers each).
-// The K/V tile is staged through shared memory once, copied into TMEM (the A
-// operand of every S^T / dP^T product) and its shared-memory space then holds
-// P^T and dS^T, the A operands of the dV / dK products. LSE and D of the
-// step's two query blocks are copied with the stage (bulk copies counted on
-// the stage's barrier) into one of two small buffers, released by the
+// K and V of the key block stay in shared memory (the A operands of every
+// S^T / dP^T product). Three stages of (Q, dO) for two query blocks, each held
+// from its load until the dV/dK products of its step complete. LSE and D of
+// the step's two query blocks are copied with the stage (bulk copies counted
+// on the stage's barrier) into one of two small buffers, released by the
 // softmax warps once read: no global load sits on the softmax warps' path.
+// The softmax warps form two groups of four taking alternate steps (group
+// j % 2 takes step j), one thread per TMEM lane: the thread in lane m + 64 kh
+// holds key row m of S^T_j and dP^T_j against query block kh of the step (64
+// values each) and writes P^T and dS^T (bf16) back over the first 32 columns
+// of its group's S^T and dP^T buffers. They are the TMEM A operands of the
+// dV and dK products, and the .ws lane split makes lane half kh accumulate
+// the query-block-kh part of dV and dK: the B operand's two 64-column halves
+// are the same 64 channels of dO (or Q) of query block 0 and of query block
+// 1. The two parts are added once, in the epilogue.
 // Two threads issue the products, each in step order: warp 1 issues
-// A_j = (S^T_j, dP^T_j) once stage j has landed and the softmax warps have
-// read the score buffers of step j - 2; warp 10 issues
-// B_j = (dV += P^T_j dO_j, dK += dS^T_j Q_j) once P^T_j / dS^T_j are written.
-// While one waits on a barrier the other's products keep the tensor pipe
-// busy.
+// A_j = (S^T_j = K Q_j^T, dP^T_j = V dO_j^T) into group (j % 2)'s buffers once
+// stage j has landed and that group's previous dV/dK products (which read
+// P^T / dS^T from the same buffers) have completed; warp 10 issues
+// B_j = (dV_parts += P^T_j dO_j, dK_parts += dS^T_j Q_j) once P^T_j / dS^T_j
+// are written. While one waits on a barrier the other's products keep the
+// tensor pipe busy.
 template <int D>
 struct DkvSmem {
-  static constexpr uint32_t kKV = 0;               // K, V staging [2][dh][64][128 B]; then P^T, dS^T
-  static constexpr uint32_t kKVBytes = 32768;      // max(2 * D * 128, P^T + dS^T)
-  static constexpr uint32_t kPT = 0;               // [query block][64 keys][128 B]
-  static constexpr uint32_t kDST = kBoxBytes * kKB;
+  static constexpr uint32_t kKV = 0;  // K, V [2][dh][64][128 B], resident
+  static constexpr uint32_t kKVBytes = 2 * D * 128;
   static constexpr uint32_t kHalf = kKB * D * 128;  // Q (or dO) of one stage, [dh][query block][64][128 B]
   static constexpr uint32_t kStageBytes = 2 * kHalf;
   static constexpr int kStages = 3;
@@ -403,7 +409,9 @@ struct DkvSmem {
   static constexpr uint32_t kDesc = kLD0 + 2 * kLDBytes;  // block-id ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 256;
-  static_assert(2 * D * 128 <= kKVBytes && kDST + kKB * kBoxBytes <= kKVBytes, "staging tile");
+  // epilogue exchange of dV / dK part quarters: [dV, dK][kh][group][64 rows][D/4 + 4 floats], over the stages
+  static constexpr uint32_t kXPitch = D / 4 + 4;
+  static_assert(2 * 4 * 64 * kXPitch * 4 <= kStages * kStageBytes, "exchange buffer fits the stages");
   // allocated without alignment slack: the kernel checks that the dynamic
   // shared memory starts on a 1024-byte boundary
   static_assert(kTotal <= 227 * 1024, "shared-memory budget");
@@ -423,18 +431,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   uint8_t* sm = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
   uint64_t* kv_full = bars + 0;
-  uint64_t* st_full = bars + 1;   // [3] stage landed
+  uint64_t* st_full = bars + 1;   // [3] stage landed (Q, dO, LSE, D)
   uint64_t* st_free = bars + 4;   // [3] B of the stage's step complete
-  uint64_t* s_full = bars + 7;    // [2] A_j complete
-  uint64_t* ps_full = bars + 9;   // P^T_j, dS^T_j written (8 softmax warps)
-  uint64_t* ps_free = bars + 10;  // B_j complete (P^T / dS^T buffer free)
-  uint64_t* mma_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
-  uint64_t* ka_full = bars + 14;  // K and V copied into TMEM by the softmax warps
-  uint64_t* s_free = bars + 15;   // [2] S^T_j, dP^T_j read by the softmax warps, index j % 2
-  uint64_t* b_done = bars + 17;   // every B product complete
-  uint64_t* ld_free = bars + 18;  // [2] LSE / D buffer read by the 8 softmax warps
+  uint64_t* s_full = bars + 7;    // [2] per group: its A complete
+  uint64_t* ps_full = bars + 9;   // [2] per group: its P^T, dS^T written to TMEM (4 warps)
+  uint64_t* ps_free = bars + 11;  // [2] per group: its B complete (its S^T / dP^T buffers free)
+  uint64_t* ld_free = bars + 13;  // [2] LSE / D buffer read by its group (4 warps)
+  uint64_t* mma_done = bars + 15;
+  uint64_t* b_done = bars + 16;   // every B product complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 18);
 
   const Geo& g = P.g;
   const int J = blockIdx.x, head = blockIdx.y;
@@ -456,15 +462,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kSoftWarps);
+      mbar_init(&ps_full[i], kGroupWarps);
+      mbar_init(&ps_free[i], 1);
+      mbar_init(&ld_free[i], kGroupWarps);
     }
-    mbar_init(b_done, 1);
-    mbar_init(&ld_free[0], kSoftWarps);
-    mbar_init(&ld_free[1], kSoftWarps);
-    mbar_init(ps_full, kSoftWarps);
-    mbar_init(ps_free, 1);
     mbar_init(mma_done, 1);
-    mbar_init(ka_full, kSoftWarps);
+    mbar_init(b_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -476,8 +479,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  // TMEM columns: S^T [2 x 64] at 0, dP^T [2 x 64] at 128, dV at 256, dK at 320, K at 384, V at 448
-  const uint32_t tdV = tbase + 256, tdK = tbase + 320, tK = tbase + 384, tV = tbase + 448;
+  // TMEM columns: S^T [2 groups x 64] at 0 (P^T over its first 32), dP^T
+  // [2 x 64] at 128 (dS^T over its first 32), dV parts at 256, dK parts at
+  // 256 + D (D columns each)
+  const uint32_t tdV = tbase + 256, tdK = tbase + 256 + D;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -513,9 +518,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
               }
             }
             issued = j + 1;
-            // LSE / D buffer j % 2 last held step j - 2: free once the softmax
-            // warps read it. The copies are issued even after a failed wait
-            // (an abort, results discarded) so that the stage's barrier completes.
+            // LSE / D buffer j % 2 last held step j - 2: free once its group read it.
+            // The copies are issued even after a failed wait (an abort, results
+            // discarded) so that the stage's barrier completes.
             ok = mbar_wait_abortable(&ld_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
             uint8_t* ldb = sm + L::kLD0 + (j & 1) * L::kLDBytes;
             for (int slot = 0; slot < kKB; ++slot) {
@@ -538,26 +543,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     // ------------------------------------------------------------ A issuer
     if (lane == 0 && nsteps > 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
+      const uint64_t dKa = sdesc_sw128(smem_u32(sm + L::kKV), 16, 1024);            // K as A of S^T
+      const uint64_t dVa = sdesc_sw128(smem_u32(sm + L::kKV + D * 128), 16, 1024);  // V as A of dP^T
       const uint32_t sQ0 = smem_u32(sm + L::kStage0);
       const uint64_t dQ0 = sdesc_sw128(sQ0, 16, 1024);              // Q as B of S^T
       const uint64_t dDO0 = sdesc_sw128(sQ0 + L::kHalf, 16, 1024);  // dO as B of dP^T
       constexpr uint64_t kStageStep = L::kStageBytes >> 4;
-      bool ok = mbar_wait_abortable(ka_full, 0, status, abort_flag);
-      // A_j: S^T_j = K Q_j^T and dP^T_j = V dO_j^T into score buffer j % 2, once
-      // stage j has landed and the softmax warps have read that buffer's step j - 2
+      bool ok = mbar_wait_abortable(kv_full, 0, status, abort_flag);
+      // A_j into group (j % 2)'s buffers once stage j has landed and that
+      // group's previous B (which read P^T / dS^T from them) completed
       for (int j = 0; j < nsteps && ok; ++j) {
         ok = mbar_wait_abortable(&st_full[j % NS], (j / NS) & 1, status, abort_flag) &&
-             mbar_wait_abortable(&s_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
+             mbar_wait_abortable(&ps_free[j & 1], ((j >> 1) & 1) ^ 1, status, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint64_t st = uint64_t(j % NS) * kStageStep;
         const uint32_t tS = tbase + (j & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws_ts(tS, tK + kk * 8, dQ0 + st + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+          mma_ws(tS, dKa + kmajor_step(kk, kBoxBytes), dQ0 + st + kmajor_step(kk, kKB * kBoxBytes), idS,
+                 kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ws_ts(tS + 128, tV + kk * 8, dDO0 + st + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+          mma_ws(tS + 128, dVa + kmajor_step(kk, kBoxBytes), dDO0 + st + kmajor_step(kk, kKB * kBoxBytes), idS,
+                 kk > 0 ? 1u : 0u);
         mma_commit(&s_full[j & 1]);
       }
       // every MMA this thread issued has completed before TMEM is released
@@ -567,121 +576,140 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
   } else if (warp == kIssuerB) {
     // ------------------------------------------------------------ B issuer
     if (lane == 0 && nsteps > 0) {
-      const uint32_t idO = idesc_bf16_f32(64, D, false, true);
-      const uint64_t dPT = sdesc_sw128(smem_u32(sm + L::kPT), 16, 1024);
-      const uint64_t dDST = sdesc_sw128(smem_u32(sm + L::kDST), 16, 1024);
+      // B = dO (or Q) of the step, MN-major, N = 128: 64 channels of query
+      // block 0 then the same channels of query block 1 (LBO = the block stride)
+      const uint32_t idO = idesc_bf16_f32(64, 128, false, true);
       const uint32_t sQ0 = smem_u32(sm + L::kStage0);
-      const uint64_t dQmn0 = sdesc_sw128(sQ0, kKB * kBoxBytes, 1024);              // Q as B of dK
-      const uint64_t dDOmn0 = sdesc_sw128(sQ0 + L::kHalf, kKB * kBoxBytes, 1024);  // dO as B of dV
+      const uint64_t dQmn0 = sdesc_sw128(sQ0, kBoxBytes, 1024);              // Q as B of dK
+      const uint64_t dDOmn0 = sdesc_sw128(sQ0 + L::kHalf, kBoxBytes, 1024);  // dO as B of dV
       constexpr uint64_t kStageStep = L::kStageBytes >> 4;
       bool ok = true;
       // B_j once P^T_j / dS^T_j are written (which implies A_j, hence stage j, complete)
       for (int j = 0; j < nsteps && ok; ++j) {
-        ok = mbar_wait_abortable(ps_full, j & 1, status, abort_flag);
+        ok = mbar_wait_abortable(&ps_full[j & 1], (j >> 1) & 1, status, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint64_t st = uint64_t(j % NS) * kStageStep;
+        const uint32_t tPT = tbase + (j & 1) * 64, tDST = tPT + 128;
 #pragma unroll
-        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-          mma_ws(tdV, dPT + kmajor_step(kk, kBoxBytes), dDOmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-        for (int kk = 0; kk < 64 * kKB / 16; ++kk)
-          mma_ws(tdK, dDST + kmajor_step(kk, kBoxBytes), dQmn0 + st + mnmajor_step(kk, kBoxBytes), idO,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+          for (int c = 0; c < D / 64; ++c)
+            mma_ws_ts(tdV + c * 64, tPT + kk * 8, dDOmn0 + st + uint64_t((c * kKB * kBoxBytes + kk * 2048) >> 4),
+                      idO, (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            mma_ws_ts(tdK + c * 64, tDST + kk * 8, dQmn0 + st + uint64_t((c * kKB * kBoxBytes + kk * 2048) >> 4),
+                      idO, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&st_free[j % NS]);
-        mma_commit(ps_free);
+        mma_commit(&ps_free[j & 1]);
       }
       mma_commit(b_done);
       mbar_wait(b_done, 0, status);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int sw = warp - 2, sp = warp & 3, ch = sw >> 2;
+    const int sw = warp - 2, grp = sw / kGroupWarps, sp = warp & 3;
     const int Ln = sp * 32 + lane;
     const int m = Ln & 63, kh = Ln >> 6;
     const uint32_t lane_off = uint32_t(sp * 32) << 16;
-    if (nsteps > 0) {
-      // K and V are the A operands of every S^T / dP^T product: one copy into TMEM
-      mbar_wait_abortable(kv_full, 0, status, abort_flag);
-      tile_to_tmem_a<D>(sm + L::kKV, tK + lane_off, m, ch);
-      tile_to_tmem_a<D>(sm + L::kKV + D * 128, tV + lane_off, m, ch);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ka_full);
-      // the staging tile holds P^T / dS^T from now on: every softmax warp has read it
-      named_bar_sync(1, 32 * kSoftWarps);
-    }
-    for (int j = 0; j < nsteps; ++j) {
-      const int sb = j & 1;
-      mbar_wait_abortable(&s_full[sb], (j >> 1) & 1, status, abort_flag);
+    int k = 0;  // this group's step count
+    for (int j = grp; j < nsteps; j += 2, ++k) {
+      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
+      mbar_wait_abortable(&s_full[grp], k & 1, status, abort_flag);
       // the stage's copies (LSE / D included) have landed: A_j read the stage,
       // and the wait makes the copied LSE / D visible to this warp
       mbar_wait_abortable(&st_full[j % NS], (j / NS) & 1, status, abort_flag);
       tc_fence_after();
-      uint32_t rs[32], rp[32];
-      tmem_ld32(tbase + lane_off + sb * 64 + ch * 32, rs);
-      tmem_ld32(tbase + lane_off + 128 + sb * 64 + ch * 32, rp);
-      tmem_ld_wait();
-      // the score buffers are free for A_{j+2}
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
-      // LSE * log2(e) and D of the 32 query rows this thread scores (query
-      // block kh of the step, rows ch*32 ..)
-      const float4* ldp = reinterpret_cast<const float4*>(sm + L::kLD0 + (j & 1) * L::kLDBytes + kh * 512) + ch * 8;
-      float4 l2[8], dd[8];
+      // LSE * log2(e) and D of the 64 query rows of query block kh of the step
+      const float4* ldp = reinterpret_cast<const float4*>(sm + L::kLD0 + (j & 1) * L::kLDBytes + kh * 512);
+      uint32_t pp[32], pd[32];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        l2[i] = ldp[i];
-        dd[i] = ldp[16 + i];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32(tbase + lane_off + grp * 64 + h * 32, rs);
+        tmem_ld32(tbase + lane_off + 128 + grp * 64 + h * 32, rp);
+        tmem_ld_wait();
+        if (valid) {
+          const float c = P.scale_log2;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 a = ldp[h * 8 + i], e = ldp[16 + h * 8 + i];
+            const float p0 = fast_exp2(fmaf(__uint_as_float(rs[4 * i]), c, -a.x));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 1]), c, -a.y));
+            const float p2 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 2]), c, -a.z));
+            const float p3 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 3]), c, -a.w));
+            pp[16 * h + 2 * i] = pack_bf16x2(p0, p1);
+            pp[16 * h + 2 * i + 1] = pack_bf16x2(p2, p3);
+            pd[16 * h + 2 * i] =
+                pack_bf16x2(p0 * (__uint_as_float(rp[4 * i]) - e.x), p1 * (__uint_as_float(rp[4 * i + 1]) - e.y));
+            pd[16 * h + 2 * i + 1] =
+                pack_bf16x2(p2 * (__uint_as_float(rp[4 * i + 2]) - e.z), p3 * (__uint_as_float(rp[4 * i + 3]) - e.w));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pp[16 * h + i] = pd[16 * h + i] = 0u;
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ld_free[j & 1]);
-      uint32_t pp[16], pd[16];
-      if (valid) {
-        const float c = P.scale_log2;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 a = l2[i], e = dd[i];
-          const float p0 = fast_exp2(fmaf(__uint_as_float(rs[4 * i]), c, -a.x));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 1]), c, -a.y));
-          const float p2 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 2]), c, -a.z));
-          const float p3 = fast_exp2(fmaf(__uint_as_float(rs[4 * i + 3]), c, -a.w));
-          pp[2 * i] = pack_bf16x2(p0, p1);
-          pp[2 * i + 1] = pack_bf16x2(p2, p3);
-          pd[2 * i] = pack_bf16x2(p0 * (__uint_as_float(rp[4 * i]) - e.x), p1 * (__uint_as_float(rp[4 * i + 1]) - e.y));
-          pd[2 * i + 1] =
-              pack_bf16x2(p2 * (__uint_as_float(rp[4 * i + 2]) - e.z), p3 * (__uint_as_float(rp[4 * i + 3]) - e.w));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pp[i] = pd[i] = 0u;
-      }
-      // the P^T / dS^T buffer last held step j - 1: free once B_{j-1} completed
-      if (j >= 1) mbar_wait_abortable(ps_free, (j - 1) & 1, status, abort_flag);
-      uint8_t* pt = sm + L::kPT + kh * kBoxBytes;
-      uint8_t* dt = sm + L::kDST + kh * kBoxBytes;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        *reinterpret_cast<uint4*>(pt + sw128_offset(m, ch * 4 + q)) =
-            make_uint4(pp[4 * q], pp[4 * q + 1], pp[4 * q + 2], pp[4 * q + 3]);
-        *reinterpret_cast<uint4*>(dt + sw128_offset(m, ch * 4 + q)) =
-            make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
-      }
-      fence_proxy_async_smem();
+      // P^T and dS^T over the first 32 columns of the group's S^T and dP^T
+      // buffers (every S^T / dP^T value of this lane was read above)
+      tmem_st16(tbase + lane_off + grp * 64, pp);
+      tmem_st16(tbase + lane_off + grp * 64 + 16, pp + 16);
+      tmem_st16(tbase + lane_off + 128 + grp * 64, pd);
+      tmem_st16(tbase + lane_off + 128 + grp * 64 + 16, pd + 16);
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ps_full);
+      if (lane == 0) mbar_arrive(&ps_full[grp]);
     }
-    if (nsteps > 0) mbar_wait_abortable(ps_free, (nsteps - 1) & 1, status, abort_flag);
+    // ---------------------------------------------------------- epilogue
+    // this group's last B complete; once both groups are here every product
+    // is complete and every copy consumed: the stages hold the exchange buffer
+    if (k > 0) mbar_wait_abortable(&ps_free[grp], (k - 1) & 1, status, abort_flag);
     tc_fence_after();
+    named_bar_sync(1, 32 * kSoftWarps);
     const bool ok = *abort_flag == 0;
+    // This thread holds the query-block-kh parts of dV and dK row m; it keeps
+    // channel quarter grp * 2 + kh of each and hands quarter grp * 2 + (kh ^ 1)
+    // to the thread of the other lane half.
     constexpr int NC = D / 4;
+    const int keep = grp * (D / 2) + kh * NC, give = grp * (D / 2) + (kh ^ 1) * NC;
     float vv[NC], vk[NC];
-    if (nsteps > 0) {
-      tmem_ld_f<NC>(tdV + lane_off + ch * NC, vv);
-      tmem_ld_f<NC>(tdK + lane_off + ch * NC, vk);
+    float* X = reinterpret_cast<float*>(sm + L::kStage0);
+    if (nsteps > 0) {  // uniform; on an abort the values are discarded below
+      float gv[NC];
+      tmem_ld_f<NC>(tdV + lane_off + give, gv);
+      float* xo = X + ((0 * 4 + kh * 2 + grp) * 64 + m) * L::kXPitch;
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i)
+        reinterpret_cast<float4*>(xo)[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
+      tmem_ld_f<NC>(tdK + lane_off + give, gv);
+      xo = X + ((1 * 4 + kh * 2 + grp) * 64 + m) * L::kXPitch;
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i)
+        reinterpret_cast<float4*>(xo)[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
+      tmem_ld_f<NC>(tdV + lane_off + keep, vv);
+      tmem_ld_f<NC>(tdK + lane_off + keep, vk);
+      named_bar_sync(1, 32 * kSoftWarps);
+      const float* xv = X + ((0 * 4 + (kh ^ 1) * 2 + grp) * 64 + m) * L::kXPitch;
+      const float* xk = X + ((1 * 4 + (kh ^ 1) * 2 + grp) * 64 + m) * L::kXPitch;
+#pragma unroll
+      for (int i = 0; i < NC / 4; ++i) {
+        const float4 tv = reinterpret_cast<const float4*>(xv)[i];
+        const float4 tk = reinterpret_cast<const float4*>(xk)[i];
+        vv[4 * i] += tv.x;
+        vv[4 * i + 1] += tv.y;
+        vv[4 * i + 2] += tv.z;
+        vv[4 * i + 3] += tv.w;
+        vk[4 * i] += tk.x;
+        vk[4 * i + 1] += tk.y;
+        vk[4 * i + 2] += tk.z;
+        vk[4 * i + 3] += tk.w;
+      }
 #pragma unroll
       for (int i = 0; i < NC; ++i) {
         vv[i] = ok ? vv[i] : 0.f;
@@ -694,7 +722,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     const int sJ = safe_shape(g, P.zone_shape, J, status);
     const BlockBox kb = block_box(g, sJ, J);
     const int tok = block_token(g, kb, m);
-    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * (D / 2) + ch * NC;
+    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + keep;
     // a key slot outside the grid (a block clipped by the edge) has no row; the
     // query slots outside the grid carry P = 0 (LSE = +inf from the prep pass)
     if (!g.partial || block_slot_in_grid(g, kb, m)) {
