@@ -14,16 +14,20 @@
 //               csc_count + scan + list fill give the CSC (ascending I);
 //   dq          one CTA per (query block, head), q-stationary: per step of two
 //               selected key blocks, S = Q K^T and dP = dO V^T (.ws M=64,
-//               N=128), then dS in the softmax warps, then dQ += dS K (.ws
-//               M=64, N=d); dQ lives in TMEM for the whole row;
+//               N=128), then dS in the softmax warps (written back into
+//               TMEM), then dQ += dS K (.ws M=64, dS as the TMEM A operand);
+//               dQ lives in TMEM for the whole row;
 //   dkdv        one CTA per (key block, head), kv-stationary over the query
 //               blocks that selected it: S^T = K Q^T, dP^T = V dO^T, then
-//               P^T, dS^T in the softmax warps, then dV += P^T dO and
-//               dK += dS^T Q (.ws M=64, N=d); dK, dV live in TMEM.
-// Splitting dQ from dK/dV costs one recomputation of S and dP but needs no
-// atomics and is deterministic. Each pass streams its two operands (K and V,
-// or Q and dO) as bulk copies of block images made just before it; the
-// single-use Q / dO (dq) and K / V (dkdv) tiles come through 5-D tensor maps.
+//               P^T, dS^T in the softmax warps (written back into TMEM), then
+//               dV += P^T dO and dK += dS^T Q (.ws M=64, P^T / dS^T as TMEM A
+//               operands); dK, dV live in TMEM.
+// Both passes issue their products from two threads and run the softmax in
+// two warp groups on alternate steps. Splitting dQ from dK/dV costs one
+// recomputation of S and dP but needs no atomics and is deterministic. Each
+// pass streams its two operands (K and V, or Q and dO) as bulk copies of
+// block images made just before it; the tiles a CTA keeps for its whole life
+// (Q / dO in dq, K / V in dkdv) come through 5-D tensor maps.
 #include <cuda_bf16.h>
 
 #include <cmath>
