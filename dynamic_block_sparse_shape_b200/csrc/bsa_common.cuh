@@ -83,29 +83,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// K-major descriptor for the k-th 16-element step of a [n_box][rows][128 B]
-// operand whose boxes sit box_stride bytes apart (64 channels per box).
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int kstep, uint32_t box_stride) {
-  return sdesc_sw128(base + uint32_t(kstep >> 2) * box_stride + uint32_t(kstep & 3) * 32u, 16, 1024);
-}
-
-// MN-major descriptor for the k-th 16-row step of an operand made of 64-row
-// x 128-byte boxes whose rows run along the contraction index: box
-// (slot, n_box) sits at base + slot * slot_stride + n_box * n_stride, where a
-// slot covers 64 contraction rows and n_box the 64-column slices along N.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kstep, uint32_t slot_stride, uint32_t n_stride) {
-  return sdesc_sw128(base + uint32_t(kstep >> 2) * slot_stride + uint32_t(kstep & 3) * 2048u, n_stride, 1024);
-}
-
-// The same K-step addressing as offsets (16-byte units) added to a base
-// descriptor's start-address field (bits 0..13; every address here is below
-// 256 KB, so the add never carries out of the field). Issuing threads build
-// one base descriptor per buffer and add a compile-time constant per step.
+// K-step addressing as offsets (16-byte units) added to a base descriptor's
+// start-address field (bits 0..13; every address here is below 256 KB, so the
+// add never carries out of the field). Issuing threads build one base
+// descriptor per buffer and add a compile-time constant per step: the k-th
+// 16-element step of a K-major [n_box][rows][128 B] operand whose 64-channel
+// boxes sit box_stride bytes apart.
 __host__ __device__ constexpr uint64_t kmajor_step(int kstep, uint32_t box_stride) {
   return uint64_t((uint32_t(kstep >> 2) * box_stride + uint32_t(kstep & 3) * 32u) >> 4);
-}
-__host__ __device__ constexpr uint64_t mnmajor_step(int kstep, uint32_t slot_stride) {
-  return uint64_t((uint32_t(kstep >> 2) * slot_stride + uint32_t(kstep & 3) * 2048u) >> 4);
 }
 
 __device__ __forceinline__ int safe_shape(const Geo& g, const int32_t* zone_shape, int b, int* status) {
@@ -140,40 +125,8 @@ __device__ __forceinline__ void mask_scores32(uint32_t* r, uint32_t members) {
   }
 }
 
-// TMA coordinates (shape, w0, h0, t0) of the blocks named by a CSR / CSC list,
-// computed 32 at a time by a whole warp (coalesced list reads, parallel
-// zone-shape lookups) into a shared-memory ring, so the thread that issues the
-// TMA copies never waits on a dependent global load. Entry e of a list of
-// `cnt` blocks processed `step` (a power of two) per step: e < cnt is the
-// list's e-th block; a ragged tail (e >= cnt in the last step) repeats the
-// step's first block.
+// Entries of the block-id ring below.
 constexpr int kDescRing = 64;
-
-struct DescCache {
-  int4* ring;  // shared memory, kDescRing entries
-  int filled;
-  int step = 2;
-  // Makes entries [0, e] available; the whole warp must call it.
-  __device__ __forceinline__ void ensure(int e, const Geo& g, const int32_t* list, int beg, int cnt,
-                                         const int32_t* zone_shape, int* status, int lane) {
-    while (e >= filled) {
-      const int ee = filled + lane;
-      int idx = ee < cnt ? ee : (ee & ~(step - 1));
-      if (idx >= cnt) idx = 0;
-      int J = list[beg + idx];
-      if (J < 0 || J >= g.n_blocks) {
-        atomicOr(status, kDevErrBounds);
-        J = 0;
-      }
-      const int s = safe_shape(g, zone_shape, J, status);
-      const BlockBox bb = block_box(g, s, J);
-      ring[ee % kDescRing] = make_int4(s, bb.w0, bb.h0, bb.t0);
-      __syncwarp();
-      filled += 32;
-    }
-  }
-  __device__ __forceinline__ int4 get(int e) const { return ring[e % kDescRing]; }
-};
 
 // Block ids named by a CSR / CSC list, read 32 at a time by a whole warp
 // (coalesced list reads) into a shared-memory ring, so the thread that issues

@@ -93,7 +93,7 @@ struct FwdSmem {
   static constexpr uint32_t kRed = kV0 + kRing * kSlotBytes; // per part: running max, sum [4][64] each
   static constexpr uint32_t kRedBytes = 2 * 4 * 64 * 4;
   static constexpr uint32_t kDesc = kRed + kRedBytes;  // block-id ring
-  static constexpr uint32_t kBar = kDesc + kDescRing * 16;
+  static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 256;
   // epilogue exchange of scaled O parts: [src part][dst quarter][64 rows][D/4 + 4 floats], over the K/V rings
   static constexpr uint32_t kXPitch = D / 4 + 4;
