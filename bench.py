@@ -169,7 +169,9 @@ class Pipeline:
         # rounding residual of the bf16 output, so that the backward's D = dO . O uses O to ~16 bits
         self.o_lo = torch.empty_like(x["q"]) if x["q"].dtype == torch.bfloat16 else None
         self.lse = torch.empty((H, wl.n_tokens), dtype=torch.float32, device=dev)
-        self.grads = tuple(torch.empty_like(x["q"]) for _ in range(3))
+        # forward-only workloads (720p, 1080p) have no dO and no backward stage
+        self.backward = "do" in x
+        self.grads = tuple(torch.empty_like(x["q"]) for _ in range(3)) if self.backward else ()
         self.zone_shape = torch.empty(self.nz, dtype=torch.int32, device=dev)
         self.zone_margin = torch.empty(self.nz, dtype=torch.float32, device=dev)
         self.ws.ensure(P.workspace_size("zone_shapes", self.geo, feat_c=feats.shape[1] if feats is not None else 0,
@@ -235,6 +237,8 @@ class Pipeline:
     def step(self, record=None):
         fns = (self.stage_zone, self.stage_pool, self.stage_select, self.stage_fwd, self.stage_bwd)
         for name, fn in zip(self.STAGES, fns):
+            if name == "bsa_bwd" and not self.backward:
+                continue
             if record is not None:
                 e0 = self.torch.cuda.Event(enable_timing=True)
                 e1 = self.torch.cuda.Event(enable_timing=True)
@@ -247,6 +251,8 @@ class Pipeline:
 
     def launches_per_step(self):
         n = sum(self.LAUNCHES.values())
+        if not self.backward:
+            n -= self.LAUNCHES["bsa_bwd"]
         if self.feats is None:
             n -= 1
         if self.res is None:
@@ -476,8 +482,9 @@ def run_gpu(args):
     peaks, peak_src = _peaks()
     variants = measure_selection_variants(pipe, res, peaks, peak_src)
     nnz = pipe.nnz
-    attn_flop = nnz * (FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR)
-    t_attn = (stage_ms["bsa_fwd"] + stage_ms["bsa_bwd"]) * 1e-3
+    flop_per_pair = FWD_FLOP_PER_PAIR + (BWD_FLOP_PER_PAIR if pipe.backward else 0)
+    attn_flop = nnz * flop_per_pair
+    t_attn = (stage_ms["bsa_fwd"] + stage_ms.get("bsa_bwd", 0.0)) * 1e-3
     achieved = attn_flop / t_attn / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     out = {
@@ -488,7 +495,7 @@ def run_gpu(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{wl.name}: grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]} ({wl.n_tokens} tokens), "
                                f"{wl.heads} heads x d{wl.head_dim}, zones {wl.zone}, top_k {wl.top_k}, "
-                               f"cdf_threshold {wl.cdf_threshold}, fwd+bwd",
+                               f"cdf_threshold {wl.cdf_threshold}, {'fwd+bwd' if pipe.backward else 'fwd only'}",
                    "parallelism": (f"one shard alone: heads {h0}:{h1} of {full_heads} (per-GPU timing)"
                                    if args.head_slice else
                                    f"heads sharded over {world} ranks (rank 0: {h0}:{h1})" if shard == "heads" else
@@ -497,12 +504,13 @@ def run_gpu(args):
         "tflops": round(achieved, 1),
         "selected_pairs": nnz, "density": round(nnz / (wl.heads * pipe.nb * pipe.nb), 4),
         "stage_ms": {k: round(v, 3) for k, v in stage_ms.items()},
-        "roofline": {"bound": "tensor", "kernel": "bsa_fwd + bsa_bwd (dq, dkdv)", "achieved": round(achieved, 1),
+        "roofline": {"bound": "tensor", "kernel": "bsa_fwd + bsa_bwd (dq, dkdv)" if pipe.backward else "bsa_fwd",
+                     "achieved": round(achieved, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": round(nnz * ATTN_DRAM_BYTES_PER_PAIR),
+                     "traffic": round(nnz * ATTN_DRAM_BYTES_PER_PAIR) if pipe.backward else None,
                      "traffic_source": "ncu dram bytes per selected pair (2-head 2K capture) x selected pairs",
                      "peak_source": f"{peak_src} bf16 sustained",
-                     "flop_per_pair": FWD_FLOP_PER_PAIR + BWD_FLOP_PER_PAIR},
+                     "flop_per_pair": flop_per_pair},
         "roofline_selection_path": selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src),
         "selection_variants": variants,
         "e2e": e2e,
