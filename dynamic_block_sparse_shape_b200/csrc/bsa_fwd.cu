@@ -95,9 +95,9 @@ struct FwdSmem {
   static constexpr uint32_t kDesc = kRed + kRedBytes;  // block-id ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 256;
-  // epilogue exchange of scaled O parts: [src part][dst quarter][64 rows][D/4 + 4 floats], over the K/V rings
+  // epilogue exchange of merged O quarters: [lane half][group][64 rows][D/4 + 4 floats], over the K ring
   static constexpr uint32_t kXPitch = D / 4 + 4;
-  static_assert(16 * 64 * kXPitch * 4 <= 2 * kRing * kSlotBytes, "exchange buffer fits the K/V rings");
+  static_assert(4 * 64 * kXPitch * 4 <= kRing * kSlotBytes, "exchange buffer fits the K ring");
   // TMEM: S buffers (64 columns per group) at 0; O parts (D columns per
   // group) at 128; Q (A operand, D/2 columns); P buffers (32 columns per group)
   static constexpr uint32_t kTmemCols = 512;
@@ -407,55 +407,60 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
       if (lq > 0.f) Lsum += lq * fast_exp2(redm[q * 64 + m] - M);
     }
     const float inv = (Lsum > 0.f && ok) ? 1.f / Lsum : 0.f;
-    const float w = (l_part > 0.f) ? fast_exp2(m_run - M) * inv : 0.f;
+    // weights of the two groups' parts held in this thread's TMEM lane (the
+    // key-block-kh half of row m); a group that took no step has no O part
+    float wg[kGroups];
+#pragma unroll
+    for (int gq = 0; gq < kGroups; ++gq) {
+      const int q = gq * 2 + kh;
+      wg[gq] = redl[q * 64 + m] > 0.f ? fast_exp2(redm[q * 64 + m] - M) * inv : 0.f;
+    }
     const int sI = safe_shape(g, P.zone_shape, I, status);
     const BlockBox qb = block_box(g, sI, I);
     const int tok = block_token(g, qb, m);
     // a query slot outside the grid (a block clipped by the edge) has no output
     const bool row_in = !g.partial || block_slot_in_grid(g, qb, m);
-    // This thread keeps channel quarter `part` of row m and hands the other
-    // three quarters of its scaled part to the threads that keep them.
+    // This thread merges both groups' parts of its lane over channel half grp,
+    // keeps quarter grp * 2 + kh of the row and hands quarter grp * 2 + (kh ^ 1)
+    // to the thread of the other lane half (same group, same row).
     constexpr int NC = D / 4;
+    const int keep = grp * (D / 2) + kh * NC, give = grp * (D / 2) + (kh ^ 1) * NC;
     float* X = reinterpret_cast<float*>(sm + L::kK0);
-    float ov[NC];
+    float ov[NC], gv[NC];
 #pragma unroll
-    for (int i = 0; i < NC; ++i) ov[i] = 0.f;
+    for (int i = 0; i < NC; ++i) ov[i] = gv[i] = 0.f;
 #pragma unroll
-    for (int qd = 0; qd < 4; ++qd) {
-      float v[NC];
-      if (k > 0) {  // warp-uniform; a group with no step has no O part
-        tmem_ld_f<NC>(tO + grp * D + lane_off + qd * NC, v);
+    for (int gq = 0; gq < kGroups; ++gq) {
+      if (nsteps > gq) {  // CTA-uniform: group gq took at least one step
+        float a[NC], b[NC];
+        tmem_ld_f<NC>(tO + gq * D + lane_off + keep, a);
+        tmem_ld_f<NC>(tO + gq * D + lane_off + give, b);
+        const float w = wg[gq];
 #pragma unroll
-        for (int i = 0; i < NC; ++i) v[i] = w == 0.f ? 0.f : v[i] * w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < NC; ++i) v[i] = 0.f;
-      }
-      if (qd == part) {
-#pragma unroll
-        for (int i = 0; i < NC; ++i) ov[i] = v[i];
-      } else {
-        float* xo = X + ((part * 4 + qd) * 64 + m) * L::kXPitch;
-#pragma unroll
-        for (int i = 0; i < NC / 4; ++i)
-          reinterpret_cast<float4*>(xo)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        for (int i = 0; i < NC; ++i) {
+          ov[i] = fmaf(a[i], w, ov[i]);
+          gv[i] = fmaf(b[i], w, gv[i]);
+        }
       }
     }
+    float* xo = X + ((kh * 2 + grp) * 64 + m) * L::kXPitch;
+#pragma unroll
+    for (int i = 0; i < NC / 4; ++i)
+      reinterpret_cast<float4*>(xo)[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
     named_bar_sync(1, 32 * kSoftWarps);
+    const float* xi = X + (((kh ^ 1) * 2 + grp) * 64 + m) * L::kXPitch;
 #pragma unroll
-    for (int src = 0; src < 4; ++src) {
-      if (src == part) continue;
-      const float* xi = X + ((src * 4 + part) * 64 + m) * L::kXPitch;
-#pragma unroll
-      for (int i = 0; i < NC / 4; ++i) {
-        const float4 t = reinterpret_cast<const float4*>(xi)[i];
-        ov[4 * i] += t.x;
-        ov[4 * i + 1] += t.y;
-        ov[4 * i + 2] += t.z;
-        ov[4 * i + 3] += t.w;
-      }
+    for (int i = 0; i < NC / 4; ++i) {
+      const float4 t = reinterpret_cast<const float4*>(xi)[i];
+      ov[4 * i] += t.x;
+      ov[4 * i + 1] += t.y;
+      ov[4 * i + 2] += t.z;
+      ov[4 * i + 3] += t.w;
     }
-    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + part * NC;
+    // o[i] keeps 0 where every weight is 0 (no key, or an abort)
+#pragma unroll
+    for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : ov[i];
+    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + keep;
     if (row_in) store_row<NC>(P.o, off, ov, P.out_fp32);
     if (P.o_lo && row_in) {
       // what the bf16 store of O dropped: O = o + o_lo to about 16 bits
