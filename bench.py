@@ -127,6 +127,15 @@ def whole_job_ms_per_layer(ms_per_step_max: float, world: int, shard: str = "rep
     return ms_per_step_max / world if shard == "replicas" else ms_per_step_max
 
 
+def workload_config(wl, parallelism):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": f"{wl.name}: grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]} ({wl.n_tokens} tokens), "
+                        f"{wl.heads} heads x d{wl.head_dim}, zones {wl.zone}, top_k {wl.top_k}, "
+                        f"cdf_threshold {wl.cdf_threshold}, {'fwd+bwd' if wl.backward else 'fwd only'}",
+            "parallelism": parallelism,
+            "l2": "inputs larger than L2 (each 1.8 GB), no flush"}
+
+
 # ---------------------------------------------------------------------------- GPU arm
 def build_inputs(wl, device):
     import torch
@@ -493,14 +502,10 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False,
         "scaling": "strong" if shard == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{wl.name}: grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]} ({wl.n_tokens} tokens), "
-                               f"{wl.heads} heads x d{wl.head_dim}, zones {wl.zone}, top_k {wl.top_k}, "
-                               f"cdf_threshold {wl.cdf_threshold}, {'fwd+bwd' if pipe.backward else 'fwd only'}",
-                   "parallelism": (f"one shard alone: heads {h0}:{h1} of {full_heads} (per-GPU timing)"
-                                   if args.head_slice else
-                                   f"heads sharded over {world} ranks (rank 0: {h0}:{h1})" if shard == "heads" else
-                                   "replicas" if world > 1 else "single"),
-                   "l2": "inputs larger than L2 (each 1.8 GB), no flush"},
+        "config": workload_config(wl, (f"one shard alone: heads {h0}:{h1} of {full_heads} (per-GPU timing)"
+                                       if args.head_slice else
+                                       f"heads sharded over {world} ranks (rank 0: {h0}:{h1})" if shard == "heads"
+                                       else "replicas" if world > 1 else "single")),
         "tflops": round(achieved, 1),
         "selected_pairs": nnz, "density": round(nnz / (wl.heads * pipe.nb * pipe.nb), 4),
         "stage_ms": {k: round(v, 3) for k, v in stage_ms.items()},
@@ -629,7 +634,7 @@ def run_reference(args):
     out = {"metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
            "dtype": "f64", "data": "synthetic", "impl": "reference",
-           "config": {"workload": f"{wl.name} (oracle on host cores, bounded sample per step)"},
+           "config": workload_config(wl, "single"),
            "cpu_baseline": cpu,
            "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
