@@ -68,6 +68,8 @@ constexpr float kRescaleThreshold = 8.0f;
 
 struct FwdParams {
   CUtensorMap mq[kMaxCand];
+  CUtensorMap mo[kMaxCand];   // O and its rounding residual, for bf16 outputs:
+  CUtensorMap mol[kMaxCand];  // the epilogue stores a block's rows with 5-D box copies
   const uint8_t* kimg;  // block images of K and V (layout in host.h)
   const uint8_t* vimg;
   Geo g;
@@ -81,6 +83,7 @@ struct FwdParams {
   int64_t tok_stride;  // of o, elements
   float scale_log2;
   int out_fp32;
+  int tma_out;  // bf16 output: stores through the O / o_lo tensor maps
 };
 
 template <int D>
@@ -460,14 +463,47 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     // o[i] keeps 0 where every weight is 0 (no key, or an abort)
 #pragma unroll
     for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : ov[i];
-    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + keep;
-    if (row_in) store_row<NC>(P.o, off, ov, P.out_fp32);
-    if (P.o_lo && row_in) {
-      // what the bf16 store of O dropped: O = o + o_lo to about 16 bits
-      float lo[NC];
+    if (P.tma_out) {
+      // bf16 rows of the block into two swizzled [d/64][64][128 B] tiles in
+      // the V ring (free: every product is complete), then one box store per
+      // 64 channels; rows outside the grid fall outside the tensor and are
+      // not written
+      uint8_t* to = sm + L::kV0;
+      uint8_t* tl = to + D * 128;
+      const int dh = keep / 64, c0 = (keep % 64) / 8;
 #pragma unroll
-      for (int i = 0; i < NC; ++i) lo[i] = ov[i] - __bfloat162float(__float2bfloat16_rn(ov[i]));
-      store_row<NC>(P.o_lo, off, lo, false);
+      for (int q = 0; q < NC / 8; ++q) {
+        float lo[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lo[i] = ov[8 * q + i] - __bfloat162float(__float2bfloat16_rn(ov[8 * q + i]));
+        const uint32_t so = dh * kBoxBytes + sw128_offset(m, c0 + q);
+        *reinterpret_cast<uint4*>(to + so) =
+            make_uint4(pack_bf16x2(ov[8 * q], ov[8 * q + 1]), pack_bf16x2(ov[8 * q + 2], ov[8 * q + 3]),
+                       pack_bf16x2(ov[8 * q + 4], ov[8 * q + 5]), pack_bf16x2(ov[8 * q + 6], ov[8 * q + 7]));
+        *reinterpret_cast<uint4*>(tl + so) =
+            make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]), pack_bf16x2(lo[4], lo[5]),
+                       pack_bf16x2(lo[6], lo[7]));
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 32 * kSoftWarps);
+      if (warp == 2 && lane == 0) {
+        for (int h = 0; h < D / 64; ++h) {
+          tma_store_5d(&P.mo[sI], to + h * kBoxBytes, h * 64, head, qb.w0, qb.h0, qb.t0);
+          if (P.o_lo) tma_store_5d(&P.mol[sI], tl + h * kBoxBytes, h * 64, head, qb.w0, qb.h0, qb.t0);
+        }
+        bulk_commit_group();
+        bulk_wait_group_read0();  // the tiles stay valid until read
+      }
+    } else {
+      const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + keep;
+      if (row_in) store_row<NC>(P.o, off, ov, P.out_fp32);
+      if (P.o_lo && row_in) {
+        // what the bf16 store of O dropped: O = o + o_lo to about 16 bits
+        float lo[NC];
+#pragma unroll
+        for (int i = 0; i < NC; ++i) lo[i] = ov[i] - __bfloat162float(__float2bfloat16_rn(ov[i]));
+        store_row<NC>(P.o_lo, off, lo, false);
+      }
     }
     if (part == 0 && row_in) {
       const int N = g.T * g.H * g.W;
@@ -617,10 +653,17 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
     return st;
   FwdParams P;
   std::memset(&P, 0, sizeof(P));
+  const bool tma_out = dtype == PRISM_BF16;
   for (int ci = 0; ci < g.n_cand; ++ci) {
     const int bt = g.cand[ci][0], bh = g.cand[ci][1], bw = g.cand[ci][2];
     if ((st = encode_block_map(&P.mq[ci], qb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+    if (tma_out) {
+      if ((st = encode_block_map(&P.mo[ci], o, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK) return st;
+      if (o_lo && (st = encode_block_map(&P.mol[ci], o_lo, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK)
+        return st;
+    }
   }
+  P.tma_out = tma_out ? 1 : 0;
   P.kimg = kimg;
   P.vimg = vimg;
   P.g = g;
