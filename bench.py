@@ -37,11 +37,11 @@ FWD_FLOP_PER_PAIR = 4 * 64 * 64 * 128  # QK^T and PV over one (query block, key 
 BWD_FLOP_PER_PAIR = 2.5 * FWD_FLOP_PER_PAIR
 # DRAM bytes (read + write) per selected (query block, key block) pair of the three attention
 # kernels together (forward, dQ, dK/dV), from one ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum) of the 2-head 2K workload: 91.23 GB over 4,445,104 pairs (forward
-# 27.00, dQ 25.56, dK/dV 38.67 GB). Scaled by the selected pairs of the timed workload; the operand
+# dram__bytes_write.sum) of the 2-head 2K workload: 91.72 GB over 4,445,104 pairs (forward
+# 26.98, dQ 25.90, dK/dV 38.84 GB). Scaled by the selected pairs of the timed workload; the operand
 # re-reads that miss L2 grow with the pairs. The block-image passes before each kernel (one read
 # and one write of the streamed operands) are not included.
-ATTN_DRAM_BYTES_PER_PAIR = 91.23e9 / 4445104
+ATTN_DRAM_BYTES_PER_PAIR = 91.72e9 / 4445104
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
