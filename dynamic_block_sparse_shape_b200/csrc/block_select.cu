@@ -9,7 +9,8 @@
 //
 // select_kernel: one CTA = 8 query blocks of one head; 4 when more than 6912
 // key blocks' logits must fit in shared memory. Two warps per row compute the
-// logits; then one warp per row selects.
+// logits, then select: each takes one half of the row, and the row's sums,
+// counts and maxima combine through shared memory at a 64-thread barrier.
 //   1. logits s_J = scale * qbar_I . kbar_J (+ b_J, the optional key-block
 //      bias, walkthrough section "桥接残差反哺稀疏注意力") for all J, fp32 FFMA:
 //      a thread streams four keys of the workspace's transposed pooled keys
@@ -34,6 +35,7 @@
 #include <cmath>
 
 #include "host.h"
+#include "ptx.cuh"
 
 namespace prism {
 namespace {
@@ -75,9 +77,9 @@ __device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_floa
 // mass for 10240 entries), combined in fp64 and warp-reduced in a fixed order.
 // The row total Z is this function at u = 1, so the bisection's invariant
 // mass(>= 1) = Z >= tau Z holds exactly.
-__device__ __forceinline__ double mass_at_least(const uint32_t* p, int nb, uint32_t u, int lane) {
+__device__ __forceinline__ double mass_at_least(const uint32_t* p, int jb, int nb, uint32_t u, int lane) {
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  int j = lane;
+  int j = jb + lane;
   for (; j + 96 < nb; j += 128) {
     const uint32_t k0 = p[j], k1 = p[j + 32], k2 = p[j + 64], k3 = p[j + 96];
     a0 += k0 >= u ? key_value(k0) : 0.f;
@@ -91,11 +93,64 @@ __device__ __forceinline__ double mass_at_least(const uint32_t* p, int nb, uint3
   }
   return warp_sum_d((double(a0) + double(a1)) + (double(a2) + double(a3)));
 }
-__device__ __forceinline__ int count_at_least(const uint32_t* p, int nb, uint32_t u, int lane) {
+__device__ __forceinline__ int count_at_least(const uint32_t* p, int jb, int nb, uint32_t u, int lane) {
   int c = 0;
-  for (int j = lane; j < nb; j += 32) c += p[j] >= u;
+  for (int j = jb + lane; j < nb; j += 32) c += p[j] >= u;
   return warp_sum_i(c);
 }
+__device__ __forceinline__ int count_equal(const uint32_t* p, int jb, int nb, uint32_t u, int lane) {
+  int c = 0;
+  for (int j = jb + lane; j < nb; j += 32) c += p[j] == u;
+  return warp_sum_i(c);
+}
+
+// The two warps of a row each reduce their half of the row; a pair value is
+// published in shared memory and combined after a 64-thread named barrier
+// (one per row). Values alternate between two slots, so a slot is rewritten
+// only after a later barrier that both warps passed after reading it. Both
+// warps combine in the same order (half 0 + half 1): their decisions agree.
+struct RowPair {
+  double* xd;  // [2 slots][2 halves]
+  int* xi;     // [2 slots][2 halves]
+  int bar, h, lane, slot;
+  __device__ __forceinline__ void sync() { named_bar_sync(bar, 64); }
+  __device__ __forceinline__ double sum_d(double v) {
+    if (lane == 0) xd[2 * slot + h] = v;
+    sync();
+    const double r = xd[2 * slot] + xd[2 * slot + 1];
+    slot ^= 1;
+    return r;
+  }
+  __device__ __forceinline__ int sum_i(int v) {
+    if (lane == 0) xi[2 * slot + h] = v;
+    sync();
+    const int r = xi[2 * slot] + xi[2 * slot + 1];
+    slot ^= 1;
+    return r;
+  }
+  __device__ __forceinline__ float max_f(float v) {
+    if (lane == 0) xd[2 * slot + h] = double(v);
+    sync();
+    const float r = fmaxf(float(xd[2 * slot]), float(xd[2 * slot + 1]));
+    slot ^= 1;
+    return r;
+  }
+  __device__ __forceinline__ uint32_t max_u(uint32_t v) {
+    if (lane == 0) xi[2 * slot + h] = int(v);
+    sync();
+    const uint32_t r = max(uint32_t(xi[2 * slot]), uint32_t(xi[2 * slot + 1]));
+    slot ^= 1;
+    return r;
+  }
+  // half 0's value, for both warps
+  __device__ __forceinline__ int first_i(int v) {
+    if (lane == 0) xi[2 * slot + h] = v;
+    sync();
+    const int r = xi[2 * slot];
+    slot ^= 1;
+    return r;
+  }
+};
 
 template <int ROWS>
 __global__ void __launch_bounds__(ROWS * 64, 1)
@@ -153,49 +208,58 @@ __global__ void __launch_bounds__(ROWS * 64, 1)
     }
   }
   __syncthreads();
-  // ---- 2..5. one warp per query block
-  const int I = I0 + warp;
-  if (warp >= ROWS || I >= nb) return;
+  // ---- 2..5. two warps per query block, each over one half of the row
+  // (split at a multiple of 32 entries, so each bitmask word has one owner)
+  const int r = warp >> 1, h = warp & 1;
+  const int I = I0 + r;
+  if (I >= nb) return;  // both warps of the row
+  RowPair pr{reinterpret_cast<double*>(qT + d * ROWS) + 4 * r, reinterpret_cast<int*>(
+                 reinterpret_cast<double*>(qT + d * ROWS) + 4 * ROWS) + 4 * r, 1 + r, h, lane, 0};
   const int top_k = hp.per_head ? hp.k[head] : hp.k0;
   const float tau = hp.per_head ? hp.tau[head] : hp.tau0;
-  uint32_t* p = reinterpret_cast<uint32_t*>(srow + size_t(warp) * nb);
-  const float* sl = srow + size_t(warp) * nb;
+  uint32_t* p = reinterpret_cast<uint32_t*>(srow + size_t(r) * nb);
+  const float* sl = srow + size_t(r) * nb;
   const int words = (nb + 31) >> 5;
   uint32_t* mrow = mask + (size_t(head) * nb + I) * words;
+  const int half = ((nb + 63) >> 6) << 5;
+  const int jb = h * half, je = max(jb, min(nb, jb + half));
+  const int wb = jb >> 5, we = (je + 31) >> 5;  // this warp's bitmask words
   float mx = -INFINITY;
-  for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, sl[j]);  // fmaxf skips NaN
+  for (int j = jb + lane; j < je; j += 32) mx = fmaxf(mx, sl[j]);  // fmaxf skips NaN
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  int n_present = 0;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
+  mx = pr.max_f(mx);
+  int np = 0;
+  for (int j0 = jb; j0 < je; j0 += 32) {
     const int j = j0 + lane;
     uint32_t key = 0u;
-    if (j < nb) {
-      const float s = sl[j];
-      if (s == s) {  // present: NaN logits mark absent blocks
-        float e = expf(s - mx);
+    if (j < je) {
+      const float sv = sl[j];
+      if (sv == sv) {  // present: NaN logits mark absent blocks
+        float e = expf(sv - mx);
         if (!(e >= 0.f)) e = 0.f;  // every present logit -inf: no mass
         key = __float_as_uint(e) + 1u;
       }
       p[j] = key;
     }
-    n_present += __popc(__ballot_sync(0xffffffffu, key != 0u));
+    np += __popc(__ballot_sync(0xffffffffu, key != 0u));
   }
   __syncwarp();
-  const double Z = mass_at_least(p, nb, 1u, lane);
+  const int n_present = pr.sum_i(np);
+  const double Z = pr.sum_d(mass_at_least(p, jb, je, 1u, lane));
   if (n_present == 0) {  // an empty query block (or no present key): empty row
-    for (int w = lane; w < words; w += 32) mrow[w] = 0u;
-    if (lane == 0) kept[size_t(head) * nb + I] = 0;
+    for (int w = wb + lane; w < we; w += 32) mrow[w] = 0u;
+    if (h == 0 && lane == 0) kept[size_t(head) * nb + I] = 0;
     return;
   }
   if (top_k >= n_present || tau >= 1.0f) {
     // every present block
-    for (int w = 0; w < words; ++w) {
+    for (int w = wb; w < we; ++w) {
       const int j = 32 * w + lane;
-      const uint32_t kb = __ballot_sync(0xffffffffu, j < nb && p[j] != 0u);
+      const uint32_t kb = __ballot_sync(0xffffffffu, j < je && p[j] != 0u);
       if (lane == 0) mrow[w] = kb;
     }
-    if (lane == 0) kept[size_t(head) * nb + I] = n_present;
+    if (h == 0 && lane == 0) kept[size_t(head) * nb + I] = n_present;
     return;
   }
   const double target = double(tau) * Z;
@@ -205,34 +269,29 @@ __global__ void __launch_bounds__(ROWS * 64, 1)
   if (target <= 0.0) {
     // C_1 >= tau already: the single largest entry (ties -> lowest J).
     uint32_t best = 0;
-    for (int j = lane; j < nb; j += 32) best = max(best, p[j]);
+    for (int j = jb + lane; j < je; j += 32) best = max(best, p[j]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-    u_star = best;
-    m_star = count_at_least(p, nb, u_star + 1, lane) + 1;
+    u_star = pr.max_u(best);
+    m_star = pr.sum_i(count_at_least(p, jb, je, u_star + 1, lane)) + 1;
   } else {
     uint32_t lo = 1, hi = 0x3F800002u;  // mass(>= lo) >= target, mass(>= hi) < target
     while (hi - lo > 1) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (mass_at_least(p, nb, mid, lane) >= target) lo = mid; else hi = mid;
+      if (pr.sum_d(mass_at_least(p, jb, je, mid, lane)) >= target) lo = mid; else hi = mid;
     }
     u_star = lo;
-    const double above = mass_at_least(p, nb, u_star + 1, lane);
-    const int above_cnt = count_at_least(p, nb, u_star + 1, lane);
-    // walk the entries tied at u_star in ascending J
+    const double above = pr.sum_d(mass_at_least(p, jb, je, u_star + 1, lane));
+    const int above_cnt = pr.sum_i(count_at_least(p, jb, je, u_star + 1, lane));
+    // take the entries tied at u_star in ascending J: each adds the same value
+    const int ties = pr.sum_i(count_equal(p, jb, je, u_star, lane));
     double run = above;
     int rank = 0;
     bool found = false;
-    for (int base = 0; base < nb && !found; base += 32) {
-      const int j = base + lane;
-      const bool tie = j < nb && p[j] == u_star;
-      uint32_t bal = __ballot_sync(0xffffffffu, tie);
-      while (bal) {
-        bal &= bal - 1;
-        run += double(key_value(u_star));  // every tied entry has p = value of u_star
-        ++rank;
-        if (run >= target) { found = true; break; }
-      }
+    for (int t = 0; t < ties && !found; ++t) {
+      run += double(key_value(u_star));
+      ++rank;
+      found = run >= target;
     }
     if (!found) rank = max(rank, 1);
     m_star = above_cnt + rank;
@@ -242,29 +301,31 @@ __global__ void __launch_bounds__(ROWS * 64, 1)
   int keep_ties;  // number of entries tied at u_final to keep, lowest J first
   if (m == m_star) {
     u_final = u_star;
-    keep_ties = m - count_at_least(p, nb, u_star + 1, lane);
+    keep_ties = m - pr.sum_i(count_at_least(p, jb, je, u_star + 1, lane));
   } else {
     uint32_t lo = 1, hi = 0x7F800002u;  // count(>= lo) >= m, count(>= hi) < m
     while (hi - lo > 1) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (count_at_least(p, nb, mid, lane) >= m) lo = mid; else hi = mid;
+      if (pr.sum_i(count_at_least(p, jb, je, mid, lane)) >= m) lo = mid; else hi = mid;
     }
     u_final = lo;
-    keep_ties = m - count_at_least(p, nb, u_final + 1, lane);
+    keep_ties = m - pr.sum_i(count_at_least(p, jb, je, u_final + 1, lane));
   }
-  int tie_run = 0;
-  for (int w = 0; w < words; ++w) {
+  // ties at u_final in the first half precede those of the second
+  const int ties_first = pr.first_i(count_equal(p, jb, je, u_final, lane));
+  int tie_run = h == 0 ? 0 : ties_first;
+  for (int w = wb; w < we; ++w) {
     const int j = 32 * w + lane;
-    const uint32_t key = j < nb ? p[j] : 0u;
-    const bool tie = j < nb && key == u_final;
+    const uint32_t key = j < je ? p[j] : 0u;
+    const bool tie = j < je && key == u_final;
     const uint32_t tb = __ballot_sync(0xffffffffu, tie);
     const int my_rank = tie_run + __popc(tb & ((1u << lane) - 1u));
-    const bool keep = j < nb && (key > u_final || (tie && my_rank < keep_ties));
+    const bool keep = j < je && (key > u_final || (tie && my_rank < keep_ties));
     const uint32_t kb = __ballot_sync(0xffffffffu, keep);
     tie_run += __popc(tb);
     if (lane == 0) mrow[w] = kb;
   }
-  if (lane == 0) kept[size_t(head) * nb + I] = m;
+  if (h == 0 && lane == 0) kept[size_t(head) * nb + I] = m;
 }
 
 // kT[h][c][j] = kp[h][j][c] for j < nb, 0 for nb <= j < nbp (32 x 32 tiles through shared memory).
@@ -390,7 +451,9 @@ prism_status block_select_impl(const float* q_pool, const float* k_pool, int32_t
   transpose_keys_kernel<<<dim3((nbp + 31) / 32, (head_dim + 31) / 32, heads), 256, 0, s>>>(k_pool, n_blocks, nbp,
                                                                                         head_dim, kT);
   const int rows_per_cta = n_blocks <= kSelMaxBlocks8 ? 8 : 4;
-  const size_t smem = (size_t(rows_per_cta) * n_blocks + size_t(head_dim) * rows_per_cta) * sizeof(float);
+  // logits [rows][nb], query rows [d][rows], then the row pairs' exchange slots (4 doubles + 4 ints per row)
+  const size_t smem = (size_t(rows_per_cta) * n_blocks + size_t(head_dim) * rows_per_cta) * sizeof(float) +
+                      size_t(rows_per_cta) * (4 * sizeof(double) + 4 * sizeof(int));
   const dim3 grid((n_blocks + rows_per_cta - 1) / rows_per_cta, heads);
   if (rows_per_cta == 8) {
     if (cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
