@@ -79,6 +79,14 @@ def test_workspace_sizes(lib):
     assert b2 - b == 4096 or b2 - b == 3840 or b2 > b
     f32 = P.workspace_size("bsa_fwd", g, heads=24, head_dim=128, dtype=__import__("torch").float32)
     assert f32 >= 3 * 294912 * 24 * 128 * 2
+    # bf16 forward: the status word and the block images of K and V, one d x 128-byte tile per
+    # (head, block) each
+    image = 24 * 4608 * 128 * 128
+    assert P.workspace_size("bsa_fwd", g, heads=24, head_dim=128) == 256 + 2 * image
+    assert P.workspace_size("bsa_fwd", g, heads=2, head_dim=64) == 256 + 2 * (2 * 4608 * 64 * 128)
+    assert f32 == 256 + 3 * 294912 * 24 * 128 * 2 + 2 * image
+    # backward: two image buffers (K and V, then Q and dO) on top of the block-order LSE / D and the CSC
+    assert b > 2 * image and b - 2 * image < 2 ** 28
 
 
 def test_host_validation_codes(lib):
