@@ -50,6 +50,12 @@ def _check_attention(geo, zone_shape_np, q, k, v, do, mask, with_bwd=True):
     qd, kd, vd, dod = (f64(t) for t in (q, k, v, do))
     Or, lser, dqr, dkr, dvr = _oracle_attention(qd, kd, vd, dod, blocks, mask, sc)
     res = {"O": assert_close("O", f64(o), Or)}
+    if o_lo is not None:
+        # the rounding residual: below half a bf16 ulp of o (bf16-rounded itself), and o + o_lo
+        # closer to the fp64 result than o alone
+        ob, ol = f64(o), f64(o_lo)
+        assert np.all(np.abs(ol) <= np.abs(ob) * 2.0 ** -8 * 1.01 + 1e-30)
+        assert np.mean(np.abs(ob + ol - Or)) <= np.mean(np.abs(ob - Or)) + 1e-7
     lse_g = f64(lse)
     fin = np.isfinite(lser)
     assert np.array_equal(np.isfinite(lse_g), fin)
