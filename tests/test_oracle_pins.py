@@ -177,6 +177,99 @@ def test_zone_statistics_end_to_end_on_planted_zones():
     assert np.all(idx0 == 0)
 
 
+# ----------------------------------------------------------------- shape rule, by value
+# Cost vectors worked out by hand from the documented reading of the rule
+# (README "Overview": finer partitioning along axes of rapid visual change and
+# strong audio-visual coupling; walkthrough section "桥接残差反哺稀疏注意力":
+# the a2v residual's per-token norm marks sounding regions, which get finer
+# blocks). The reading: V^_a = 3 V_a / sum V, A^_a = 3 A_a / sum A, gate
+# g = clip(m / mbar - 1, 0, 4), S = V^ + 1 * g * A^ renormalised to sum 3,
+# cost(c) = sum_a S_a log2(ext_a) + 0.25 sum_a (log2(ext_a) - 2)^2.
+# Every extent is a power of two, so each cost is an exact fraction; the
+# derivations are written beside each case, and no value is computed by code.
+# For the ten default candidates, in order, e = log2(ext) is
+#   (2,2,2) (3,1,2) (3,2,1) (2,3,1) (1,3,2) (1,2,3) (2,1,3) (0,3,3) (3,0,3) (3,3,0)
+# and the isotropy penalty 0.25 * sum (e-2)^2 is
+#   0       0.5     0.5     0.5     0.5     0.5     0.5     1.5     1.5     1.5
+SHAPE_COST_CASES = [
+    # (a) features only, anisotropic: V = (1, 2, 5), sum 8 -> S = (3/8, 6/8, 15/8) (already sum 3).
+    #     e.g. (8,8,1): 3*3/8 + 3*6/8 + 0 = 27/8, + 1.5 = 4.875; (8,4,2): 9/8 + 12/8 + 15/8 = 36/8, + 0.5 = 5.0
+    dict(V=(1, 2, 5), A=(0, 0, 0), m=0.0, mbar=0.0, use_audio=False,
+         cost=(6.0, 6.125, 5.0, 5.375, 6.875, 8.0, 7.625, 9.375, 8.25, 4.875), best=9, margin=0.125),
+    # (b) isotropic features, sounding zone below the gate cap: V = (1,1,1) -> (1,1,1);
+    #     A = (0, 3, 1) -> A^ = (0, 9/4, 3/4); m/mbar = 2 -> g = 1;
+    #     S = (1, 13/4, 7/4), sum 6 -> renormalised (1/2, 13/8, 7/8).
+    #     e.g. (8,2,4): 3/2 + 13/8 + 14/8 = 39/8, + 0.5 = 5.375; (8,1,8): 3/2 + 0 + 21/8 = 33/8, + 1.5 = 5.625
+    dict(V=(1, 1, 1), A=(0, 3, 1), m=2.0, mbar=1.0, use_audio=True,
+         cost=(6.0, 5.375, 6.125, 7.25, 7.625, 6.875, 5.75, 9.0, 5.625, 7.875), best=1, margin=0.25),
+    # (c) as (b) but m/mbar = 7: m/mbar - 1 = 6 is capped at 4 -> S = (1, 1 + 9, 1 + 3) = (1, 10, 4),
+    #     sum 15 -> renormalised (1/5, 2, 4/5).
+    #     e.g. (8,1,8): 3/5 + 0 + 12/5 = 3, + 1.5 = 4.5; (8,2,4): 3/5 + 2 + 8/5 = 4.2, + 0.5 = 4.7
+    dict(V=(1, 1, 1), A=(0, 3, 1), m=7.0, mbar=1.0, use_audio=True,
+         cost=(6.0, 4.7, 5.9, 7.7, 8.3, 7.1, 5.3, 9.9, 4.5, 8.1), best=8, margin=0.2),
+    # (d) anisotropic features and audio: V^ = (3/8, 6/8, 15/8); A = (2, 1, 1) -> A^ = (3/2, 3/4, 3/4);
+    #     m/mbar = 3 -> g = 2; S = (27/8, 18/8, 27/8), sum 9 -> renormalised (9/8, 6/8, 9/8).
+    #     The isotropic candidate wins: (4,4,4) 6.0 against (4,8,2) and (2,8,4) at 45/8 + 0.5 = 6.125
+    dict(V=(1, 2, 5), A=(2, 1, 1), m=3.0, mbar=1.0, use_audio=True,
+         cost=(6.0, 6.875, 6.5, 6.125, 6.125, 6.5, 6.875, 7.125, 8.25, 7.125), best=0, margin=0.125),
+]
+
+
+def _shape_cost_mismatches(cost_fn):
+    """Differences between cost_fn and the hand-worked costs, argmins and margins."""
+    bad = []
+    for i, c in enumerate(SHAPE_COST_CASES):
+        got = np.asarray(cost_fn(np.array(c["V"], float), np.array(c["A"], float), c["m"], c["mbar"], CAND,
+                                 use_audio=c["use_audio"]), dtype=np.float64)
+        if got.shape != (len(CAND),) or not np.allclose(got, c["cost"], rtol=0, atol=1e-9):
+            bad.append((i, "cost", got.tolist()))
+            continue
+        if int(np.argmin(got)) != c["best"]:
+            bad.append((i, "argmin", int(np.argmin(got))))
+        if abs(float(np.sort(got)[1] - got.min()) - c["margin"]) > 1e-9:
+            bad.append((i, "margin", float(np.sort(got)[1] - got.min())))
+    return bad
+
+
+def test_shape_cost_equals_hand_worked_values():
+    assert _shape_cost_mismatches(O.shape_cost) == []
+
+
+def test_choose_shapes_margin_equals_hand_worked_values():
+    for c in SHAPE_COST_CASES:
+        st = {"V": np.array([c["V"]], float), "A": np.array([c["A"]], float), "m": np.array([c["m"]]),
+              "mbar": c["mbar"]}
+        idx, margin = O.choose_shapes(st, CAND, have_features=True, have_residual=c["use_audio"])
+        assert int(idx[0]) == c["best"] and abs(margin[0] - c["margin"]) < 1e-9
+
+
+# Plausible slips in the cost: each must change at least one hand-worked value.
+SHAPE_COST_MUTANTS = {
+    "natural log for log2": ("np.log2(", "np.log("),
+    "|e - 2| for (e - 2)^2": ("((e - 2.0) ** 2)", "np.abs(e - 2.0)"),
+    "audio gate without its cap": ("min(max(m / mbar - 1.0, 0.0), gate_max)", "max(m / mbar - 1.0, 0.0)"),
+    "no renormalisation to sum 3": ("S = 3.0 * S / tot if tot > 0 else np.ones(3)", "S = S"),
+    "gate without the -1": ("m / mbar - 1.0", "m / mbar"),
+    "gamma 1 for 0.25": ("gamma * ((e - 2.0)", "1.0 * ((e - 2.0)"),
+    "audio term unweighted by the gate": ("S = Vh + w_audio * g * Ah", "S = Vh + w_audio * Ah"),
+    "unnormalised feature variances": ("Vh = 3.0 * V / (V.sum() + EPS)", "Vh = V"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SHAPE_COST_MUTANTS))
+def test_shape_cost_pins_catch_planted_mistakes(name):
+    """Plants one slip into a copy of the oracle's cost (on the CPU) and checks
+    that the hand-worked values reject it."""
+    import inspect
+    import textwrap
+    src = textwrap.dedent(inspect.getsource(O.shape_cost))
+    old, new = SHAPE_COST_MUTANTS[name]
+    assert src.count(old) >= 1, f"mutation site not found: {old}"
+    ns = dict(vars(O))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    assert _shape_cost_mismatches(ns["shape_cost"]) != [], name
+
+
 # ----------------------------------------------------------------- pooling
 def test_pooling_of_a_linear_field_is_its_value_at_the_block_centre():
     grid, zone = (8, 8, 16), (8, 8, 8)
