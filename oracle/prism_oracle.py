@@ -319,13 +319,17 @@ def block_select(qp, kp, scale, top_k, tau, rows=None, key_bias=None):
     margin = np.full((H, nb), np.nan)
     if rows is None:
         rows = [(h, i) for h in range(H) for i in range(nb)]
+    present = {}  # per head: the key blocks that take part, and their pooled features and biases
     for h, i in rows:
         if np.isnan(qp[h, i]).any():
             kept[h, i] = 0
             gap[h, i] = margin[h, i] = math.inf
             continue
-        valid = np.nonzero(~np.isnan(kp[h]).any(axis=1))[0]
-        s = scale * (kp[h, valid] @ qp[h, i]) + bias[valid]
+        if h not in present:
+            v = np.nonzero(~np.isnan(kp[h]).any(axis=1))[0]
+            present[h] = (v, kp[h, v], bias[v])
+        valid, kv, bv = present[h]
+        s = scale * (kv @ qp[h, i]) + bv
         idx, m, _, g, mg = select_row(s, int(ks[h]), float(taus[h]))
         idx = valid[idx]
         mask[h, i, idx] = True

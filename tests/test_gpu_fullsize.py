@@ -1,16 +1,22 @@
 """Full-size parity on the 720p, 1080p and 2K workloads, on the real 720p latent
-grid (16 x 45 x 80, whose last zone row is clipped), and on two corners of
-the 2K selection/sparsity sweep (the sparsest: structure amplitude 4, k = 1,
+grid (16 x 45 x 80, whose last zone row is clipped), and on six points of the
+2K selection/sparsity sweep (the sparsest: structure amplitude 4, k = 1,
 tau = 0.05; the densest: amplitude 0.25, k = 16, tau = 1, every key block
-kept), in the launch configuration bench.py times, on outputs the oracle can
-compute one by one:
+kept; the floor deciding m: amplitude 4 with k = 4, tau = 0.2 and k = 16,
+tau = 0.4; the mass deciding m: amplitude 1, k = 1, tau = 0.4 and amplitude
+0.25, k = 1, tau = 0.05), in the launch configuration bench.py times, on
+outputs the oracle can compute one by one:
 
 * zone shapes of every zone (bit-exact where the oracle's cost margin > 1e-3);
 * pooled features of sampled blocks of every head;
-* the selection of sampled query blocks of one head (bit-exact where the
-  oracle's margins are safe) and its CSR;
+* the selection of every query block of four heads: bit-exact where the
+  oracle's margins are safe, and elsewhere one of the selections the rule
+  admits within the stated rounding (tests/selection_check.py), with the
+  bit-exact fraction printed and held at 95 % or more; sampled CSR rows;
 * O and LSE of sampled query blocks and, on the 2K training step, dQ of those
-  blocks and dK / dV of sampled key blocks.
+  blocks and dK / dV of sampled key blocks, within max-abs 2e-2 and mean-abs
+  2e-3 (the amplitude-4 sweep points admit elements above 2e-2 up to the
+  oracle's bf16 rounding bound, and print how many).
 
 The GPU stages after the zone shapes take the oracle's zone shapes as input
 (an oracle value may feed the CUDA path, never the reverse), so both sides use
@@ -26,7 +32,8 @@ import torch
 import dynamic_block_sparse_shape_b200 as P
 from dynamic_block_sparse_shape_b200 import synth
 from oracle import prism_oracle as O
-from tests.gpu_util import (CDF_MARGIN, LOGIT_GAP, assert_close, f64, mask_bits_to_bool, require_gpu)
+from tests.gpu_util import assert_close, f64, mask_bits_to_bool, require_gpu
+from tests.selection_check import check_head_selection
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -66,7 +73,10 @@ def _oracle_zone_shapes(wl, cand, feats, res):
     return idx, margin
 
 
-SWEEP_POINTS = ["2k-sweep-a4.0-k1-t0.05", "2k-sweep-a0.25-k16-t1.0"]
+# sweep points spanning the rule's regimes: the sparsest and the densest corner, the floor k deciding m
+# (amplitude 4, k 4 and 16), the mass deciding m at tau 0.4 and at tau 0.05 (amplitudes 1 and 0.25)
+SWEEP_POINTS = ["2k-sweep-a4.0-k1-t0.05", "2k-sweep-a0.25-k16-t1.0", "2k-sweep-a4.0-k4-t0.2",
+                "2k-sweep-a1.0-k1-t0.4", "2k-sweep-a0.25-k1-t0.05", "2k-sweep-a4.0-k16-t0.4"]
 
 
 def _workload(name):
@@ -113,26 +123,36 @@ def test_full_size_workload(name):
                 continue
             ref = t[torch.as_tensor(m, device=dev)].to("cpu", torch.float64).numpy().mean(axis=0)
             assert np.abs(got[:, i] - ref).max() < 2e-6
-    # ---- a4 + a5: one head, every row (the key-block columns need all of them)
-    h = 1 % H
+    # ---- a4 + a5: every row of four heads, checked by the oracle's rule (tests/selection_check.py)
     sel = P.block_select(qp, kp, sc, wl.top_k, wl.cdf_threshold, ws=ws)
-    qh = x["q"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
-    kh = x["k"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
-    qpr, kpr = O.block_pool(qh, blocks), O.block_pool(kh, blocks)
-    ref = O.block_select(qpr, kpr, sc, wl.top_k, wl.cdf_threshold)
-    got = mask_bits_to_bool(sel["mask"][h:h + 1], nb)[0]
-    kept = sel["kept"][h].cpu().numpy()
-    sq = (ref["gap"][0] > LOGIT_GAP) & (ref["margin"][0] > CDF_MARGIN)
-    assert sq.sum() >= 0.05 * nb
-    assert np.array_equal(got[sq], ref["mask"][0][sq])
+    heads = sorted({0, 1 % H, H // 2, H - 1})
+    masks = {hh: mask_bits_to_bool(sel["mask"][hh:hh + 1], nb)[0] for hh in heads}
+    kept_all = sel["kept"].cpu().numpy()
     empty = members == 0
-    assert np.all(kept[~empty] >= min(wl.top_k, int((~empty).sum()))) and np.all(kept[empty] == 0)
-    assert np.array_equal(got.sum(axis=1), kept) and not got[:, empty].any()
+    h = 1 % H  # the head whose attention rows are sampled below
+    for hh in heads:
+        qh_ = x["q"][:, hh].to("cpu", torch.float64).numpy()[:, None, :]
+        kh_ = x["k"][:, hh].to("cpu", torch.float64).numpy()[:, None, :]
+        qpr_h, kpr_h = O.block_pool(qh_, blocks)[0], O.block_pool(kh_, blocks)[0]
+        st = check_head_selection(masks[hh], kept_all[hh], qpr_h, kpr_h, sc, wl.top_k, wl.cdf_threshold)
+        print(f"{name} head {hh}: {st['exact']}/{st['rows']} rows bit-exact ({st['exact'] / st['rows']:.4f}), "
+              f"{st['qualified']} margin-qualified, {st['m_range']} with m inside [m(tau-d), m(tau+d)], "
+              f"{st['swaps']} with swaps inside the boundary band")
+        assert st["exact"] >= 0.95 * st["rows"], st
+        assert np.all(kept_all[hh][empty] == 0) and not masks[hh][:, empty].any()
+        if hh == h:
+            ref_mask_h = O.block_select(qpr_h[None], kpr_h[None], sc, wl.top_k, wl.cdf_threshold)["mask"][0]
+    got = masks[h]
+    ref = {"mask": ref_mask_h[None]}
     rp = sel["row_ptr"].cpu().numpy()
     ci = sel["col_idx"].cpu().numpy()
-    for I in rng.choice(nb, size=16, replace=False):
-        r = h * nb + I
-        assert ci[rp[r]:rp[r + 1]].tolist() == np.nonzero(got[I])[0].tolist()
+    assert rp[-1] == kept_all.sum() == sel["total"]
+    for hh in heads:
+        for I in rng.choice(nb, size=16, replace=False):
+            r = hh * nb + I
+            assert ci[rp[r]:rp[r + 1]].tolist() == np.nonzero(masks[hh][I])[0].tolist()
+    qh = x["q"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
+    kh = x["k"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
     # ---- a6 (+ a7): sampled rows with identical selections
     o_lo = torch.empty_like(x["q"])  # bf16 workloads: the forward's rounding residual of O for D
     o, lse = P.bsa_fwd(geo, zs, x["q"], x["k"], x["v"], sc, sel["row_ptr"], sel["col_idx"], ws=ws, o_lo=o_lo)
@@ -150,16 +170,19 @@ def test_full_size_workload(name):
                                sel["col_idx"], sel["total"], ws=ws, o_lo=o_lo)
     torch.cuda.synchronize()
     P.check_device_status(ws)
+    # max-abs 2e-2 as stated; only the amplitude-4 sweep points, whose gradients reach several units,
+    # admit an element beyond it up to the oracle's bound of the bf16 roundings (reading R18)
+    wide = wl.amplitude > 1.0
     cache = {}
     for I in rows:
         rr = O.attention_block_rows(qh, kh, vh, blocks, np.nonzero(ref["mask"][0][I])[0], 0, I, sc, dO=doh,
                                     bf16_bound=True)
         cache[(0, I)] = rr
         tk = torch.as_tensor(O.block_members(blocks, I), device=dev)
-        assert_close("O", f64(o[tk, h]), rr["O"], bound=rr["O_bound"])
+        assert_close("O", f64(o[tk, h]), rr["O"], bound=rr["O_bound"] if wide else None)
         assert_close("LSE", f64(lse[h, tk]), rr["lse"])
         if wl.backward:
-            assert_close("dQ", f64(dq[tk, h]), rr["dQ"], bound=rr["dQ_bound"])
+            assert_close("dQ", f64(dq[tk, h]), rr["dQ"], bound=rr["dQ_bound"] if wide else None)
     if wl.backward and not dense:
         # key blocks all of whose users (query blocks that selected them) have
         # exactly the oracle's selection, so their LSE and D agree too (with
@@ -187,5 +210,5 @@ def test_full_size_workload(name):
             gk, gv, bk, bv = O.attention_kv_block_grads(qh, kh, vh, doh, blocks, ref["mask"][0], 0, J, sc,
                                                         row_cache=cache, bf16_bound=True)
             tk = torch.as_tensor(O.block_members(blocks, J), device=dev)
-            assert_close("dK", f64(dk[tk, h]), gk, bound=bk)
-            assert_close("dV", f64(dv[tk, h]), gv, bound=bv)
+            assert_close("dK", f64(dk[tk, h]), gk, bound=bk if wide else None)
+            assert_close("dV", f64(dv[tk, h]), gv, bound=bv if wide else None)
