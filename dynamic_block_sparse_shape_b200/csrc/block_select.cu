@@ -4,30 +4,40 @@
 // step keeps the k highest-scoring blocks, then extends along the CDF of the
 // block scores until cdf_threshold (default 0.20). Prism README "Overview":
 // the hybrid rule sets each query's sparsity. Sol-Attn abstract on the Prism
-// paper page: computing and materialising the proxy scores is the routing
-// overhead, so the scores here live only in shared memory.
+// paper page: blocks are ranked by a block proxy score.
 //
-// select_kernel: one CTA = 8 query blocks of one head; 4 when more than 6912
-// key blocks' logits must fit in shared memory. Two warps per row compute the
-// logits, then select: each takes one half of the row, and the row's sums,
-// counts and maxima combine through shared memory at a 64-thread barrier.
-//   1. logits s_J = scale * qbar_I . kbar_J (+ b_J, the optional key-block
-//      bias, walkthrough section "桥接残差反哺稀疏注意力") for all J, fp32 FFMA:
-//      a thread streams four keys of the workspace's transposed pooled keys
-//      (coalesced 512-byte warp reads per channel) and forms their logits
-//      against the CTA's rows (shared-memory broadcasts);
-//   2. per row: max, p_J = exp(s_J - max) in place as a ranking key (float
-//      bits + 1; 0 for a NaN logit, which marks an absent block: an empty
-//      block of a grid clipped at its edge), Z = sum p (fp64);
-//   3. the mass threshold: bisection on the keys for
-//      u* = max{u : sum_{key_J >= u} p_J >= tau * Z}; ties at u* are taken in
-//      ascending J until the mass is reached -> m*;
-//   4. m = max(k, m*); if m > m*, a bisection on counts finds the m-th key;
-//      k and tau are the row's head's (per-head settings, walkthrough section
-//      "实际案例与上手参考": the top-k part of the selection is a tunable ratio);
-//   5. the kept set (ranked by p descending, ties to the lower J) is written
-//      as a bitmask row with warp ballots, and kept[row] = m.
-// transpose_keys_kernel: k_pool per head into key-major order in the workspace.
+// Three kernels per call, the last two once per chunk of heads:
+//   split_tf32_kernel: q_pool and k_pool into tf32-exact halves, x = hi + lo
+//     (hi keeps the top 10 mantissa bits of x, lo = x - hi is exact in fp32).
+//   score_kernel: the logits s_IJ = scale * qbar_I . kbar_J (+ b_J, the
+//     optional key-block bias, walkthrough section "桥接残差反哺稀疏注意力") of
+//     a chunk of heads as a tcgen05 kind::tf32 GEMM in split precision:
+//     hi.hi + hi.lo + lo.hi accumulated in fp32 in tensor memory (relative
+//     error about 2^-20 of sum_c |q_c k_c|, against 2^-8 for one bf16 product).
+//     A persistent CTA per SM takes 128 x 256 tiles in turn: the 32-channel
+//     slices of the four operand halves come by TMA (128-byte swizzle) into a
+//     two-stage ring, two TMEM accumulators let the epilogue of one tile
+//     overlap the products of the next, and the logits leave as 32 x 32 TMA
+//     box stores (128-byte rows). The chunk's
+//     logits go to the workspace (one head of the 2K grid is 85 MB, which
+//     stays in the 126 MB L2 until the selection reads it).
+//   select_rows_kernel: one 128-thread CTA per (head, query block), the row's
+//     entries in registers (thread t holds J = t + 128 i):
+//     1. max of the present logits (a NaN logit marks an absent block: an
+//        empty block of a grid clipped at its edge), p_J = exp(s_J - max),
+//        Z = sum p (fp32 chains of at most VPT terms per thread, combined in
+//        fp64 in a fixed order);
+//     2. the mass threshold u* = max{u : sum_{p_J >= u} p_J >= tau Z}: a
+//        bisection on the float bits of p inside the row's [min, max] bracket
+//        until at most 32 entries remain in the bracket (or one value); those
+//        are sorted in one warp and their masses added in rank order in fp64;
+//        the count m* follows, ties at u* taken in ascending J;
+//     3. m = max(k, m*); when k decides, the same bracketed search on counts
+//        finds the k-th largest entry;
+//     4. the kept set (p descending, ties to the lower J) written as bitmask
+//        words by warp ballots, and kept[row] = m.
+//   k and tau are the row's head's (per-head settings, walkthrough section
+//   "实际案例与上手参考": the top-k part of the selection is a tunable ratio).
 // scan_kernel: exclusive scan of kept into the CSR row_ptr (one CTA).
 // fill_kernel: one warp per row expands the bitmask into ascending col_idx.
 #include <algorithm>
@@ -40,9 +50,6 @@
 namespace prism {
 namespace {
 
-// Rows of logits per CTA live in shared memory: 8 rows up to 6912 key blocks,
-// 4 rows (half the threads) up to 10240 (the 2K latent grid has 7680).
-constexpr int kSelMaxBlocks8 = 6912;
 constexpr int kSelMaxBlocks = 10240;
 constexpr int kSelMaxHeads = 128;  // per-head settings passed as a kernel parameter
 
@@ -53,6 +60,283 @@ struct SelHeads {
   float tau0;
   int k[kSelMaxHeads];
   float tau[kSelMaxHeads];
+};
+
+// ------------------------------------------------------------------ split
+// hi = x with the low 13 mantissa bits cleared (exactly a tf32 value, so the
+// tensor core reads it unchanged); lo = x - hi, exact in fp32, of which the
+// tensor core keeps the top 10 mantissa bits. NaN stays NaN in both.
+__global__ void __launch_bounds__(256) split_tf32_kernel(const float4* __restrict__ x, size_t n4,
+                                                         float4* __restrict__ hi, float4* __restrict__ lo) {
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n4; i += size_t(gridDim.x) * blockDim.x) {
+    const float4 v = x[i];
+    float4 h, l;
+    h.x = __uint_as_float(__float_as_uint(v.x) & 0xFFFFE000u);
+    h.y = __uint_as_float(__float_as_uint(v.y) & 0xFFFFE000u);
+    h.z = __uint_as_float(__float_as_uint(v.z) & 0xFFFFE000u);
+    h.w = __uint_as_float(__float_as_uint(v.w) & 0xFFFFE000u);
+    l.x = v.x - h.x;
+    l.y = v.y - h.y;
+    l.z = v.z - h.z;
+    l.w = v.w - h.w;
+    hi[i] = h;
+    lo[i] = l;
+  }
+}
+
+// ------------------------------------------------------------------ scores
+constexpr int kScM = 128;                      // query blocks per tile (TMEM lanes)
+constexpr int kScN = 256;                      // key blocks per tile (TMEM columns)
+constexpr int kScAtomBytes = 128;              // 32 fp32 channels: one 128-byte swizzle row
+constexpr int kScABytes = kScM * kScAtomBytes;  // 16 KB
+constexpr int kScBBytes = kScN * kScAtomBytes;  // 32 KB
+constexpr int kScStageBytes = 2 * kScABytes + 2 * kScBBytes;  // A hi, A lo, B hi, B lo
+constexpr int kScStages = 2;
+constexpr int kScEpiWarps = 4;
+constexpr int kScStageOut = 32 * 128;  // one epilogue store tile: 32 rows x 32 logits
+constexpr int kScOutOff = kScStages * kScStageBytes;
+constexpr int kScBarOff = kScOutOff + kScEpiWarps * 2 * kScStageOut;
+constexpr int kScSmem = kScBarOff + 256 + 1024;  // + barriers, + alignment slack
+constexpr int kScThreads = 64 + 32 * kScEpiWarps;
+
+struct ScoreParams {
+  CUtensorMap q_hi, q_lo, k_hi, k_lo;  // 3-D fp32 (d, n_blocks, heads), box (32, 128 | 256, 1)
+  CUtensorMap out;                     // logits, 3-D fp32 (nbp, n_blocks, round heads), box (32, 32, 1)
+  const float* kbias;                  // [nb] or null
+  int nb, d, head0, heads;             // heads: in this round
+  float scale;
+  int* status;
+};
+
+// Instruction descriptor for kind::tf32 with fp32 accumulation, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 3-D tiled store from this CTA's shared memory (bulk-group completion); box
+// elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+// Waits until at most one committed bulk store of this thread still reads its source.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// Waits until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Persistent: CTA b takes tiles b, b + grid, ... of the round; tile t is
+// (head t / (rows * cols), query tile, key tile) in raster order.
+//   warp 0      copies: per 32-channel slice, A hi/lo (128 query blocks) and
+//               B hi/lo (256 key blocks) into a two-stage ring;
+//   warp 1      TMEM owner and MMA issuer: per slice 4 x (lo.hi, hi.lo, hi.hi)
+//               products into one of two 256-column accumulators;
+//   warps 2..5  epilogue: a thread per TMEM lane (query block), 32 logits per
+//               load, scaled (+ bias), through a swizzled shared-memory tile
+//               into one 32 x 32 TMA box store (128-byte rows);
+// the epilogue of tile i overlaps the products of tile i + 1.
+__global__ void __launch_bounds__(kScThreads, 1) score_kernel(const __grid_constant__ ScoreParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kScBarOff);
+  uint64_t* full = bars;            // [2] slice landed
+  uint64_t* empty = bars + 2;       // [2] slice's products complete
+  uint64_t* acc_full = bars + 4;    // [2] accumulator's products complete
+  uint64_t* acc_empty = bars + 6;   // [2] accumulator read by the epilogue warps
+  uint64_t* mma_done = bars + 8;    // every product complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int atoms = P.d / 32;
+  const int n_it = (P.nb + kScM - 1) / kScM, n_jt = (P.nb + kScN - 1) / kScN;
+  const int total = P.heads * n_it * n_jt;
+  int* status = P.status;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kScStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kScEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * kScN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&P.q_hi);
+      tma_prefetch_desc(&P.q_lo);
+      tma_prefetch_desc(&P.k_hi);
+      tma_prefetch_desc(&P.k_lo);
+      bool ok = true;
+      int it = 0;  // slices issued
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int hz = t / (n_it * n_jt), r = t - hz * n_it * n_jt;
+        const int I0 = (r / n_jt) * kScM, J0 = (r % n_jt) * kScN, head = P.head0 + hz;
+        for (int a = 0; a < atoms; ++a) {
+          const int st = it % kScStages;
+          // stage st last held slice it - 2: free once its products completed
+          if (it >= kScStages) ok = mbar_wait_abortable(&empty[st], ((it / kScStages) - 1) & 1, status, abort_flag);
+          if (!ok) break;
+          uint8_t* sb = sm + st * kScStageBytes;
+          mbar_arrive_expect_tx(&full[st], kScStageBytes);
+          tma_load_3d(sb, &P.q_hi, &full[st], 32 * a, I0, head);
+          tma_load_3d(sb + kScABytes, &P.q_lo, &full[st], 32 * a, I0, head);
+          tma_load_3d(sb + 2 * kScABytes, &P.k_hi, &full[st], 32 * a, J0, head);
+          tma_load_3d(sb + 2 * kScABytes + kScBBytes, &P.k_lo, &full[st], 32 * a, J0, head);
+          ++it;
+        }
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      for (int i = it - kScStages > 0 ? it - kScStages : 0; i < it; ++i)
+        mbar_wait(&full[i % kScStages], (i / kScStages) & 1, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_tf32_f32(kScM, kScN);
+      bool ok = true;
+      int it = 0, lt = 0;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+        const int acc = lt & 1;
+        // accumulator acc last held tile lt - 2: free once the epilogue read it
+        if (lt >= 2) ok = mbar_wait_abortable(&acc_empty[acc], ((lt >> 1) - 1) & 1, status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d = tbase + acc * kScN;
+        for (int a = 0; a < atoms && ok; ++a) {
+          const int st = it % kScStages;
+          ok = mbar_wait_abortable(&full[st], (it / kScStages) & 1, status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sb = smem_u32(sm + st * kScStageBytes);
+          const uint64_t ahi = sdesc_sw128(sb, 16, 1024), alo = sdesc_sw128(sb + kScABytes, 16, 1024);
+          const uint64_t bhi = sdesc_sw128(sb + 2 * kScABytes, 16, 1024);
+          const uint64_t blo = sdesc_sw128(sb + 2 * kScABytes + kScBBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 8 tf32 channels (32 bytes) per product
+            const uint64_t o = uint64_t(kk * 2);
+            mma_tf32(d, alo + o, bhi + o, idesc, (a > 0 || kk > 0) ? 1u : 0u);
+            mma_tf32(d, ahi + o, blo + o, idesc, 1u);
+            mma_tf32(d, ahi + o, bhi + o, idesc, 1u);
+          }
+          mma_commit(&empty[st]);
+          ++it;
+        }
+        if (ok) mma_commit(&acc_full[acc]);
+      }
+      // every product this thread issued has completed before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter
+    const uint32_t lane_off = uint32_t(q * 32) << 16;
+    uint8_t* outb = sm + kScOutOff + (warp - 2) * 2 * kScStageOut;
+    int sbuf = 0, lt = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+      const int hz = t / (n_it * n_jt), r = t - hz * n_it * n_jt;
+      const int I0 = (r / n_jt) * kScM, J0 = (r % n_jt) * kScN;
+      const int acc = lt & 1;
+      if (!mbar_wait_abortable(&acc_full[acc], (lt >> 1) & 1, status, abort_flag)) break;
+      tc_fence_after();
+      const bool rows_in = I0 + 32 * q < P.nb;  // some of this warp's query blocks exist
+#pragma unroll 1
+      for (int c = 0; c < kScN / 32; ++c) {
+        const int Jc = J0 + 32 * c;
+        if (Jc >= P.nb || !rows_in) break;  // warp-uniform
+        uint32_t rr[32];
+        tmem_ld32(tbase + acc * kScN + lane_off + 32 * c, rr);
+        tmem_ld_wait();
+        // the store tile written two stores ago has been read
+        if (lane == 0) bulk_wait_group_read1();
+        __syncwarp();
+        uint8_t* tile = outb + sbuf * kScStageOut;
+#pragma unroll
+        for (int qq = 0; qq < 8; ++qq) {
+          float v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int J = Jc + 4 * qq + e;
+            const float b = (P.kbias && J < P.nb) ? __ldg(P.kbias + J) : 0.f;
+            v[e] = __uint_as_float(rr[4 * qq + e]) * P.scale + b;
+          }
+          *reinterpret_cast<float4*>(tile + sw128_offset(lane, qq)) = make_float4(v[0], v[1], v[2], v[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&P.out, tile, Jc, I0 + 32 * q, hz);
+          bulk_commit_group();
+        }
+        sbuf ^= 1;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+    if (lane == 0) bulk_wait_group0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 2 * kScN);
+  }
+}
+
+// ------------------------------------------------------------------ selection
+constexpr int kSelThreads = 128;  // threads per row
+constexpr int kSelWarps = kSelThreads / 32;
+
+// Per-warp partial results in shared memory; two slots alternate, so a slot
+// is rewritten only after a later barrier that every warp passed after reading it.
+struct SelShared {
+  double d[2][kSelWarps];
+  int i[2][kSelWarps];
+  uint32_t u[2][kSelWarps][2];
+  float f[2][kSelWarps];
+  float lp[32];      // the entries of a final bracket (at most 32), in no order
+  float sorted[32];  // the same, descending
+  int lcount;
+  int res_i[4];
+  uint32_t res_u[2];
 };
 
 __device__ __forceinline__ double warp_sum_d(double v) {
@@ -66,285 +350,281 @@ __device__ __forceinline__ int warp_sum_i(int v) {
   return v;
 }
 
-// Row entries are kept as ranking keys: key = (float bits of p) + 1 for a
-// present key block and 0 for an absent one (NaN logit: an empty block, or a
-// NaN input). For p >= 0 the float bits order like the values, so keys order
-// like p with every absent block below every present one.
-__device__ __forceinline__ float key_value(uint32_t key) { return __uint_as_float(key - 1u); }
-
-// Mass of the entries whose key is >= u >= 1: four independent fp32 chains per
-// lane (at most nb/128 terms each, relative error below 2e-6 of the row's
-// mass for 10240 entries), combined in fp64 and warp-reduced in a fixed order.
-// The row total Z is this function at u = 1, so the bisection's invariant
-// mass(>= 1) = Z >= tau Z holds exactly.
-__device__ __forceinline__ double mass_at_least(const uint32_t* p, int jb, int nb, uint32_t u, int lane) {
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  int j = jb + lane;
-  for (; j + 96 < nb; j += 128) {
-    const uint32_t k0 = p[j], k1 = p[j + 32], k2 = p[j + 64], k3 = p[j + 96];
-    a0 += k0 >= u ? key_value(k0) : 0.f;
-    a1 += k1 >= u ? key_value(k1) : 0.f;
-    a2 += k2 >= u ? key_value(k2) : 0.f;
-    a3 += k3 >= u ? key_value(k3) : 0.f;
+// Sum over the CTA of (fp64 mass, int count); every thread gets the same
+// result (partials combined in warp order).
+__device__ __forceinline__ void cta_sum(double& m, int& c, SelShared& S, int& slot, int warp, int lane) {
+  m = warp_sum_d(m);
+  c = warp_sum_i(c);
+  if (lane == 0) {
+    S.d[slot][warp] = m;
+    S.i[slot][warp] = c;
   }
-  for (; j < nb; j += 32) {
-    const uint32_t k = p[j];
-    a0 += k >= u ? key_value(k) : 0.f;
-  }
-  return warp_sum_d((double(a0) + double(a1)) + (double(a2) + double(a3)));
-}
-__device__ __forceinline__ int count_at_least(const uint32_t* p, int jb, int nb, uint32_t u, int lane) {
-  int c = 0;
-  for (int j = jb + lane; j < nb; j += 32) c += p[j] >= u;
-  return warp_sum_i(c);
-}
-__device__ __forceinline__ int count_equal(const uint32_t* p, int jb, int nb, uint32_t u, int lane) {
-  int c = 0;
-  for (int j = jb + lane; j < nb; j += 32) c += p[j] == u;
-  return warp_sum_i(c);
+  __syncthreads();
+  m = (S.d[slot][0] + S.d[slot][1]) + (S.d[slot][2] + S.d[slot][3]);
+  c = (S.i[slot][0] + S.i[slot][1]) + (S.i[slot][2] + S.i[slot][3]);
+  slot ^= 1;
 }
 
-// The two warps of a row each reduce their half of the row; a pair value is
-// published in shared memory and combined after a 64-thread named barrier
-// (one per row). Values alternate between two slots, so a slot is rewritten
-// only after a later barrier that both warps passed after reading it. Both
-// warps combine in the same order (half 0 + half 1): their decisions agree.
-struct RowPair {
-  double* xd;  // [2 slots][2 halves]
-  int* xi;     // [2 slots][2 halves]
-  int bar, h, lane, slot;
-  __device__ __forceinline__ void sync() { named_bar_sync(bar, 64); }
-  __device__ __forceinline__ double sum_d(double v) {
-    if (lane == 0) xd[2 * slot + h] = v;
-    sync();
-    const double r = xd[2 * slot] + xd[2 * slot + 1];
-    slot ^= 1;
-    return r;
+// Mass (fp32 chain per thread, fp64 across threads) and count of the entries >= pm.
+template <int VPT>
+__device__ __forceinline__ void mass_count_at_least(const float (&p)[VPT], float pm, double& m, int& c) {
+  float a = 0.f;
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const bool ge = p[i] >= pm;  // false for NaN (absent)
+    a += ge ? p[i] : 0.f;
+    n += ge;
   }
-  __device__ __forceinline__ int sum_i(int v) {
-    if (lane == 0) xi[2 * slot + h] = v;
-    sync();
-    const int r = xi[2 * slot] + xi[2 * slot + 1];
-    slot ^= 1;
-    return r;
-  }
-  __device__ __forceinline__ float max_f(float v) {
-    if (lane == 0) xd[2 * slot + h] = double(v);
-    sync();
-    const float r = fmaxf(float(xd[2 * slot]), float(xd[2 * slot + 1]));
-    slot ^= 1;
-    return r;
-  }
-  __device__ __forceinline__ uint32_t max_u(uint32_t v) {
-    if (lane == 0) xi[2 * slot + h] = int(v);
-    sync();
-    const uint32_t r = max(uint32_t(xi[2 * slot]), uint32_t(xi[2 * slot + 1]));
-    slot ^= 1;
-    return r;
-  }
-  // half 0's value, for both warps
-  __device__ __forceinline__ int first_i(int v) {
-    if (lane == 0) xi[2 * slot + h] = v;
-    sync();
-    const int r = xi[2 * slot];
-    slot ^= 1;
-    return r;
-  }
-};
+  m = a;
+  c = n;
+}
 
-template <int ROWS>
-__global__ void __launch_bounds__(ROWS * 64, 1)
-    select_kernel(const float* __restrict__ qp, const float* __restrict__ kT, int nb, int nbp, int d, float scale,
-                  const __grid_constant__ SelHeads hp, const float* __restrict__ kbias, uint32_t* __restrict__ mask,
-                  int32_t* __restrict__ kept) {
-  // two warps per row: all of them stream logits (more loads in flight), one per row selects
-  constexpr int kThreads = ROWS * 64;
-  extern __shared__ __align__(16) float sm[];
-  float* srow = sm;                      // [ROWS][nb]
-  float* qT = srow + size_t(ROWS) * nb;  // [d][ROWS]: one float4 = one channel of 4 rows
-  const int head = blockIdx.y;
-  const int I0 = blockIdx.x * ROWS;
+// Gathers the entries of [lo, hi) (at most 32) into S.lp, then warp 0 sorts
+// them descending and picks the entry that decides the search: in mass mode
+// the first, in rank order, whose running mass (from mass_hi, fp64) reaches
+// the target; in count mode the one of rank need - cnt_hi - 1. Publishes its
+// value, the count of entries above it and the count of entries equal to it.
+template <int VPT>
+__device__ __forceinline__ void resolve_bracket(const float (&p)[VPT], uint32_t lo, uint32_t hi, int cnt_hi,
+                                             double mass_hi, bool mass_mode, double target, int need,
+                                             SelShared& S) {
+  if (threadIdx.x == 0) S.lcount = 0;
+  __syncthreads();
+  const float plo = __uint_as_float(lo), phi = __uint_as_float(hi);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    if (p[i] >= plo && p[i] < phi) {
+      const int at = atomicAdd(&S.lcount, 1);
+      if (at < 32) S.lp[at] = p[i];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int c = min(S.lcount, 32);
+    const float v = lane < c ? S.lp[lane] : -1.f;
+    int rank = 0;  // descending; equal values take consecutive ranks in list order
+    for (int o = 0; o < c; ++o) {
+      const float w = S.lp[o];
+      rank += (w > v) || (w == v && o < lane);
+    }
+    if (lane < c) S.sorted[rank] = v;
+    __syncwarp();
+    const float vr = lane < c ? S.sorted[lane] : -1.f;
+    int pick;
+    if (mass_mode) {
+      double cum = lane < c ? double(vr) : 0.0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xffffffffu, cum, o);
+        if (lane >= o) cum += t;
+      }
+      cum += mass_hi;
+      const uint32_t reach = __ballot_sync(0xffffffffu, lane < c && cum >= target);
+      pick = reach ? __ffs(reach) - 1 : c - 1;
+      if (lane == 0) S.res_i[1] = cnt_hi + pick + 1;  // the count up to the decisive entry
+    } else {
+      pick = need - cnt_hi - 1;
+    }
+    const float u = __shfl_sync(0xffffffffu, vr, pick);
+    const uint32_t above = __ballot_sync(0xffffffffu, lane < c && vr > u);
+    const uint32_t equal = __ballot_sync(0xffffffffu, lane < c && vr == u);
+    if (lane == 0) {
+      S.res_u[0] = __float_as_uint(u);
+      S.res_i[0] = cnt_hi + __popc(above);
+      S.res_i[2] = __popc(equal);
+    }
+  }
+  __syncthreads();
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const float* __restrict__ logits, int nb, int nbp,
+                                                                  int head0, const __grid_constant__ SelHeads hp,
+                                                                  uint32_t* __restrict__ mask,
+                                                                  int32_t* __restrict__ kept) {
+  __shared__ SelShared S;
+  __shared__ int tie_cnt[VPT][kSelWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const float* qh = qp + size_t(head) * nb * d;
-  for (int i = tid; i < ROWS * d; i += kThreads) {
-    const int r = i / d, c = i - r * d;
-    qT[c * ROWS + r] = (I0 + r < nb) ? qh[size_t(I0 + r) * d + c] : 0.f;
-  }
-  __syncthreads();
-  // ---- 1. logits. kT is the head's pooled keys transposed, [d][nbp]: for channel c a warp reads 32 x 4
-  // consecutive keys (512 contiguous bytes). A thread owns keys k0 .. k0+3, k0 = 4 * (tid + i * kThreads),
-  // and forms their logits against the CTA's rows (shared-memory broadcasts). Channels accumulate in
-  // ascending order, one chain per (row, key).
-  const float* kTh = kT + size_t(head) * d * nbp;
-  for (int k0 = 4 * tid; k0 < nb; k0 += 4 * kThreads) {
-    float a[ROWS][4];
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < d; ++c) {
-      const float4 kv = __ldg(reinterpret_cast<const float4*>(kTh + size_t(c) * nbp + k0));
-      const float* qc = qT + c * ROWS;
-#pragma unroll
-      for (int r4 = 0; r4 < ROWS / 4; ++r4) {
-        const float4 qv = *reinterpret_cast<const float4*>(qc + 4 * r4);
-        const float qs[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          a[4 * r4 + i][0] = fmaf(qs[i], kv.x, a[4 * r4 + i][0]);
-          a[4 * r4 + i][1] = fmaf(qs[i], kv.y, a[4 * r4 + i][1]);
-          a[4 * r4 + i][2] = fmaf(qs[i], kv.z, a[4 * r4 + i][2]);
-          a[4 * r4 + i][3] = fmaf(qs[i], kv.w, a[4 * r4 + i][3]);
-        }
-      }
-    }
-#pragma unroll
-    for (int jk = 0; jk < 4; ++jk) {
-      const int key = k0 + jk;
-      if (key < nb) {
-        const float bj = kbias ? __ldg(kbias + key) : 0.f;
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) srow[size_t(r) * nb + key] = a[r][jk] * scale + bj;
-      }
-    }
-  }
-  __syncthreads();
-  // ---- 2..5. two warps per query block, each over one half of the row
-  // (split at a multiple of 32 entries, so each bitmask word has one owner)
-  const int r = warp >> 1, h = warp & 1;
-  const int I = I0 + r;
-  if (I >= nb) return;  // both warps of the row
-  RowPair pr{reinterpret_cast<double*>(qT + d * ROWS) + 4 * r, reinterpret_cast<int*>(
-                 reinterpret_cast<double*>(qT + d * ROWS) + 4 * ROWS) + 4 * r, 1 + r, h, lane, 0};
-  const int top_k = hp.per_head ? hp.k[head] : hp.k0;
-  const float tau = hp.per_head ? hp.tau[head] : hp.tau0;
-  uint32_t* p = reinterpret_cast<uint32_t*>(srow + size_t(r) * nb);
-  const float* sl = srow + size_t(r) * nb;
+  const int hz = blockIdx.x / nb, I = blockIdx.x - hz * nb;
+  const int head = head0 + hz;
   const int words = (nb + 31) >> 5;
   uint32_t* mrow = mask + (size_t(head) * nb + I) * words;
-  const int half = ((nb + 63) >> 6) << 5;
-  const int jb = h * half, je = max(jb, min(nb, jb + half));
-  const int wb = jb >> 5, we = (je + 31) >> 5;  // this warp's bitmask words
+  int32_t* krow = kept + size_t(head) * nb + I;
+  const float* srow = logits + size_t(blockIdx.x) * nbp;
+  int slot = 0;
+  // ---- 1. logits, maximum, p = exp(s - max) (as 2^((s - max) log2 e))
+  float p[VPT];
   float mx = -INFINITY;
-  for (int j = jb + lane; j < je; j += 32) mx = fmaxf(mx, sl[j]);  // fmaxf skips NaN
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int J = tid + kSelThreads * i;
+    p[i] = J < nb ? __ldg(srow + J) : __uint_as_float(0x7fc00000u);
+    mx = fmaxf(mx, p[i]);  // fmaxf skips NaN
+  }
 #pragma unroll
   for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  mx = pr.max_f(mx);
+  if (lane == 0) S.f[slot][warp] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(S.f[slot][0], S.f[slot][1]), fmaxf(S.f[slot][2], S.f[slot][3]));
+  slot ^= 1;
+  const float mx2 = mx * 1.44269504088896341f;
+  uint32_t umin = 0xFFFFFFFFu, umax = 0u;
   int np = 0;
-  for (int j0 = jb; j0 < je; j0 += 32) {
-    const int j = j0 + lane;
-    uint32_t key = 0u;
-    if (j < je) {
-      const float sv = sl[j];
-      if (sv == sv) {  // present: NaN logits mark absent blocks
-        float e = expf(sv - mx);
-        if (!(e >= 0.f)) e = 0.f;  // every present logit -inf: no mass
-        key = __float_as_uint(e) + 1u;
-      }
-      p[j] = key;
+  float zs = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    if (p[i] == p[i]) {  // present
+      float e = exp2f(fmaf(p[i], 1.44269504088896341f, -mx2));
+      if (!(e >= 0.f)) e = 0.f;  // every present logit -inf: no mass
+      e = fminf(e, 1.f);
+      p[i] = e;
+      umin = min(umin, __float_as_uint(e));
+      umax = max(umax, __float_as_uint(e));
+      zs += e;
+      ++np;
     }
-    np += __popc(__ballot_sync(0xffffffffu, key != 0u));
   }
-  __syncwarp();
-  const int n_present = pr.sum_i(np);
-  const double Z = pr.sum_d(mass_at_least(p, jb, je, 1u, lane));
-  if (n_present == 0) {  // an empty query block (or no present key): empty row
-    for (int w = wb + lane; w < we; w += 32) mrow[w] = 0u;
-    if (h == 0 && lane == 0) kept[size_t(head) * nb + I] = 0;
-    return;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    umin = min(umin, __shfl_xor_sync(0xffffffffu, umin, o));
+    umax = max(umax, __shfl_xor_sync(0xffffffffu, umax, o));
   }
-  if (top_k >= n_present || tau >= 1.0f) {
-    // every present block
-    for (int w = wb; w < we; ++w) {
-      const int j = 32 * w + lane;
-      const uint32_t kb = __ballot_sync(0xffffffffu, j < je && p[j] != 0u);
-      if (lane == 0) mrow[w] = kb;
+  if (lane == 0) {
+    S.u[slot][warp][0] = umin;
+    S.u[slot][warp][1] = umax;
+  }
+  double Z = zs;
+  cta_sum(Z, np, S, slot, warp, lane);  // its barrier also publishes the minima and maxima
+  const int sl = slot ^ 1;
+  umin = min(min(S.u[sl][0][0], S.u[sl][1][0]), min(S.u[sl][2][0], S.u[sl][3][0]));
+  umax = max(max(S.u[sl][0][1], S.u[sl][1][1]), max(S.u[sl][2][1], S.u[sl][3][1]));
+  const int top_k = hp.per_head ? hp.k[head] : hp.k0;
+  const float tau = hp.per_head ? hp.tau[head] : hp.tau0;
+  if (np == 0 || top_k >= np || tau >= 1.0f) {
+    // an empty query block (or no present key): empty row; else every present block
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const uint32_t b = __ballot_sync(0xffffffffu, np > 0 && p[i] == p[i]);
+      const int w = i * kSelWarps + warp;
+      if (lane == 0 && w < words) mrow[w] = b;
     }
-    if (h == 0 && lane == 0) kept[size_t(head) * nb + I] = n_present;
+    if (tid == 0) *krow = np;
     return;
   }
   const double target = double(tau) * Z;
-  // u*: largest key with mass(key >= u) >= target.
-  uint32_t u_star;
-  int m_star;
-  if (target <= 0.0) {
-    // C_1 >= tau already: the single largest entry (ties -> lowest J).
-    uint32_t best = 0;
-    for (int j = jb + lane; j < je; j += 32) best = max(best, p[j]);
+  // ---- 2. the mass threshold, then 3. the floor k, with one bracketed search:
+  // mass mode keeps mass(>= lo) >= target > mass(>= hi); count mode keeps
+  // count(>= lo) >= m > count(>= hi). Each pass halves [lo, hi) in float bits;
+  // the search ends at one value or at most 32 entries in the bracket.
+  uint32_t lo = umin, hi = umax + 1u;
+  int cnt_lo = np, cnt_hi = 0;
+  double mass_hi = 0.0;
+  bool mass_mode = true;
+  int need = 0, m = 0;
+  uint32_t u_final = 0;
+  int cnt_gt = 0, ties_total = 0;  // entries above u_final, entries equal to it
+  if (target <= 0.0) lo = umax;  // the first entry in rank order reaches the target already
+#pragma unroll 1
+  for (int round = 0; round < 2; ++round) {
+    if (round == 1) {
+      // the floor decides: the m-th largest entry lies at or below u*
+      mass_mode = false;
+      need = m;
+      lo = umin;
+      hi = u_final + 1u;
+      cnt_lo = np;
+      cnt_hi = cnt_gt;
+    } else if (target <= 0.0) {
+      double ms;
+      int c;
+      mass_count_at_least(p, __uint_as_float(lo), ms, c);
+      cta_sum(ms, c, S, slot, warp, lane);
+      cnt_lo = c;
+    }
+#pragma unroll 1
+    while (cnt_lo - cnt_hi > 32 && hi - lo > 1u) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      double ms;
+      int c;
+      mass_count_at_least(p, __uint_as_float(mid), ms, c);
+      cta_sum(ms, c, S, slot, warp, lane);
+      if (mass_mode ? (ms >= target) : (c >= need)) {
+        lo = mid;
+        cnt_lo = c;
+      } else {
+        hi = mid;
+        cnt_hi = c;
+        mass_hi = ms;
+      }
+    }
+    int m_here;
+    if (hi - lo == 1u) {
+      // one value left: tied entries, each adding the same mass
+      u_final = lo;
+      cnt_gt = cnt_hi;
+      ties_total = cnt_lo - cnt_hi;
+      if (mass_mode) {
+        const double pv = double(__uint_as_float(lo));
+        double run = mass_hi;
+        int r = 0;
+        while (r < ties_total) {
+          run += pv;
+          ++r;
+          if (run >= target) break;
+        }
+        m_here = cnt_hi + max(r, 1);
+      } else {
+        m_here = need;
+      }
+    } else {
+      resolve_bracket(p, lo, hi, cnt_hi, mass_hi, mass_mode, target, need, S);
+      u_final = S.res_u[0];
+      cnt_gt = S.res_i[0];
+      ties_total = S.res_i[2];
+      m_here = mass_mode ? S.res_i[1] : need;
+    }
+    if (round == 0) {
+      m = max(min(top_k, np), m_here);
+      if (m == m_here) break;  // the mass decides
+    }
+  }
+  const int keep_ties = m - cnt_gt;
+  // ---- 4. bitmask: p > u_final, and the first keep_ties entries equal to u_final in ascending J
+  // (J = 128 i + 32 warp + lane: slot-major, then warp, then lane)
+  const float uf = __uint_as_float(u_final);
+  if (keep_ties >= ties_total) {
+    // every entry equal to u_final is kept
 #pragma unroll
-    for (int o = 16; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-    u_star = pr.max_u(best);
-    m_star = pr.sum_i(count_at_least(p, jb, je, u_star + 1, lane)) + 1;
+    for (int i = 0; i < VPT; ++i) {
+      const uint32_t kb = __ballot_sync(0xffffffffu, p[i] >= uf);
+      const int w = i * kSelWarps + warp;
+      if (lane == 0 && w < words) mrow[w] = kb;
+    }
   } else {
-    uint32_t lo = 1, hi = 0x3F800002u;  // mass(>= lo) >= target, mass(>= hi) < target
-    while (hi - lo > 1) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (pr.sum_d(mass_at_least(p, jb, je, mid, lane)) >= target) lo = mid; else hi = mid;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const uint32_t tb = __ballot_sync(0xffffffffu, p[i] == uf);
+      if (lane == 0) tie_cnt[i][warp] = __popc(tb);
     }
-    u_star = lo;
-    const double above = pr.sum_d(mass_at_least(p, jb, je, u_star + 1, lane));
-    const int above_cnt = pr.sum_i(count_at_least(p, jb, je, u_star + 1, lane));
-    // take the entries tied at u_star in ascending J: each adds the same value
-    const int ties = pr.sum_i(count_equal(p, jb, je, u_star, lane));
-    double run = above;
-    int rank = 0;
-    bool found = false;
-    for (int t = 0; t < ties && !found; ++t) {
-      run += double(key_value(u_star));
-      ++rank;
-      found = run >= target;
+    __syncthreads();
+    int run = 0;  // ties before the current slot
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      int before = run;
+      for (int w = 0; w < warp; ++w) before += tie_cnt[i][w];
+      run += (tie_cnt[i][0] + tie_cnt[i][1]) + (tie_cnt[i][2] + tie_cnt[i][3]);
+      const bool tie = p[i] == uf;
+      const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+      const int my_rank = before + __popc(tb & ((1u << lane) - 1u));
+      const bool keep = p[i] > uf || (tie && my_rank < keep_ties);
+      const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+      const int w = i * kSelWarps + warp;
+      if (lane == 0 && w < words) mrow[w] = kb;
     }
-    if (!found) rank = max(rank, 1);
-    m_star = above_cnt + rank;
   }
-  const int m = max(min(top_k, n_present), m_star);
-  uint32_t u_final;
-  int keep_ties;  // number of entries tied at u_final to keep, lowest J first
-  if (m == m_star) {
-    u_final = u_star;
-    keep_ties = m - pr.sum_i(count_at_least(p, jb, je, u_star + 1, lane));
-  } else {
-    uint32_t lo = 1, hi = 0x7F800002u;  // count(>= lo) >= m, count(>= hi) < m
-    while (hi - lo > 1) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      if (pr.sum_i(count_at_least(p, jb, je, mid, lane)) >= m) lo = mid; else hi = mid;
-    }
-    u_final = lo;
-    keep_ties = m - pr.sum_i(count_at_least(p, jb, je, u_final + 1, lane));
-  }
-  // ties at u_final in the first half precede those of the second
-  const int ties_first = pr.first_i(count_equal(p, jb, je, u_final, lane));
-  int tie_run = h == 0 ? 0 : ties_first;
-  for (int w = wb; w < we; ++w) {
-    const int j = 32 * w + lane;
-    const uint32_t key = j < je ? p[j] : 0u;
-    const bool tie = j < je && key == u_final;
-    const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-    const int my_rank = tie_run + __popc(tb & ((1u << lane) - 1u));
-    const bool keep = j < je && (key > u_final || (tie && my_rank < keep_ties));
-    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-    tie_run += __popc(tb);
-    if (lane == 0) mrow[w] = kb;
-  }
-  if (h == 0 && lane == 0) kept[size_t(head) * nb + I] = m;
-}
-
-// kT[h][c][j] = kp[h][j][c] for j < nb, 0 for nb <= j < nbp (32 x 32 tiles through shared memory).
-__global__ void __launch_bounds__(256) transpose_keys_kernel(const float* __restrict__ kp, int nb, int nbp, int d,
-                                                             float* __restrict__ kT) {
-  __shared__ float tile[32][33];
-  const int h = blockIdx.z, j0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const float* src = kp + size_t(h) * nb * d;
-  float* dst = kT + size_t(h) * d * nbp;
-  for (int r = ty; r < 32; r += 8) {
-    const int j = j0 + r, c = c0 + tx;
-    tile[r][tx] = (j < nb && c < d) ? src[size_t(j) * d + c] : 0.f;
-  }
-  __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int c = c0 + r, j = j0 + tx;
-    if (c < d && j < nbp) dst[size_t(c) * nbp + j] = tile[tx][r];
-  }
+  if (tid == 0) *krow = m;
 }
 
 // Exclusive scan of n ints into out[0..n] (out[n] = total), one CTA.
@@ -405,12 +685,53 @@ __global__ void __launch_bounds__(256) fill_kernel(const uint32_t* __restrict__ 
   }
 }
 
+// Entries per thread of select_rows_kernel: n_blocks / 128 rounded up to an instantiated size.
+constexpr int kVpts[] = {1, 2, 4, 8, 12, 16, 24, 32, 36, 40, 48, 64, 80};
+
+int select_vpt(int nb) {
+  const int need = (nb + kSelThreads - 1) / kSelThreads;
+  for (int v : kVpts)
+    if (v >= need) return v;
+  return 0;
+}
+
+template <int V>
+cudaError_t launch_rows_v(const float* logits, int nb, int nbp, int h0, int g, const SelHeads& hp, uint32_t* mask,
+                          int32_t* kept, cudaStream_t s) {
+  select_rows_kernel<V><<<unsigned(g) * unsigned(nb), kSelThreads, 0, s>>>(logits, nb, nbp, h0, hp, mask, kept);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_rows(int vpt, const float* logits, int nb, int nbp, int h0, int g, const SelHeads& hp,
+                               uint32_t* mask, int32_t* kept, cudaStream_t s) {
+  switch (vpt) {
+#define PRISM_ROWS_CASE(V) \
+  case V: return launch_rows_v<V>(logits, nb, nbp, h0, g, hp, mask, kept, s);
+    PRISM_ROWS_CASE(1) PRISM_ROWS_CASE(2) PRISM_ROWS_CASE(4) PRISM_ROWS_CASE(8) PRISM_ROWS_CASE(12)
+    PRISM_ROWS_CASE(16) PRISM_ROWS_CASE(24) PRISM_ROWS_CASE(32) PRISM_ROWS_CASE(36) PRISM_ROWS_CASE(40)
+    PRISM_ROWS_CASE(48) PRISM_ROWS_CASE(64) PRISM_ROWS_CASE(80)
+#undef PRISM_ROWS_CASE
+  }
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
-// The status word, then the pooled keys transposed per head, [heads][d][nbp], nbp = nb rounded up to 4.
+// Heads whose logits one score/selection round holds: as many as fit in 96 MB (the logits of a
+// round stay in the 126 MB L2 between the two kernels), at least one.
+int select_chunk_heads(int heads, int nb) {
+  const size_t nbp = (size_t(nb) + 3) & ~size_t(3);
+  const size_t per_head = size_t(nb) * nbp * sizeof(float);
+  const size_t budget = size_t(96) << 20;
+  return int(std::max<size_t>(1, std::min<size_t>(size_t(heads), budget / per_head)));
+}
+
+// The status word, then the tf32 halves of the pooled features (q hi, q lo, k hi, k lo, each
+// [heads][nb][d] fp32), then one round's logits [chunk heads][nb][nbp], nbp = nb rounded up to 4.
 size_t block_select_ws_bytes(int heads, int nb, int d) {
   const size_t nbp = (size_t(nb) + 3) & ~size_t(3);
-  return kWsHeader + align_up(size_t(heads) * d * nbp * sizeof(float), 256);
+  const size_t half = align_up(size_t(heads) * nb * d * sizeof(float), 256);
+  return kWsHeader + 4 * half + align_up(size_t(select_chunk_heads(heads, nb)) * nb * nbp * sizeof(float), 256);
 }
 
 cudaError_t launch_exclusive_scan(const int32_t* in, int n, int32_t* out, cudaStream_t s) {
@@ -447,22 +768,61 @@ prism_status block_select_impl(const float* q_pool, const float* k_pool, int32_t
   if (col_idx && col_cap < 0) return PRISM_ERR_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int nbp = (n_blocks + 3) & ~3;
-  float* kT = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kWsHeader);
-  transpose_keys_kernel<<<dim3((nbp + 31) / 32, (head_dim + 31) / 32, heads), 256, 0, s>>>(k_pool, n_blocks, nbp,
-                                                                                        head_dim, kT);
-  const int rows_per_cta = n_blocks <= kSelMaxBlocks8 ? 8 : 4;
-  // logits [rows][nb], query rows [d][rows], then the row pairs' exchange slots (4 doubles + 4 ints per row)
-  const size_t smem = (size_t(rows_per_cta) * n_blocks + size_t(head_dim) * rows_per_cta) * sizeof(float) +
-                      size_t(rows_per_cta) * (4 * sizeof(double) + 4 * sizeof(int));
-  const dim3 grid((n_blocks + rows_per_cta - 1) / rows_per_cta, heads);
-  if (rows_per_cta == 8) {
-    if (cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+  const size_t n_el = size_t(heads) * n_blocks * head_dim;
+  const size_t half = align_up(n_el * sizeof(float), 256);
+  uint8_t* base = static_cast<uint8_t*>(ws) + kWsHeader;
+  float* q_hi = reinterpret_cast<float*>(base);
+  float* q_lo = reinterpret_cast<float*>(base + half);
+  float* k_hi = reinterpret_cast<float*>(base + 2 * half);
+  float* k_lo = reinterpret_cast<float*>(base + 3 * half);
+  float* logits = reinterpret_cast<float*>(base + 4 * half);
+  {
+    const size_t n4 = n_el / 4;
+    const unsigned blocks = unsigned(std::min<size_t>((n4 + 255) / 256, size_t(device_sm_count()) * 16));
+    split_tf32_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(q_pool), n4,
+                                             reinterpret_cast<float4*>(q_hi), reinterpret_cast<float4*>(q_lo));
+    split_tf32_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(k_pool), n4,
+                                             reinterpret_cast<float4*>(k_hi), reinterpret_cast<float4*>(k_lo));
+  }
+  const int chunk = select_chunk_heads(heads, n_blocks);
+  ScoreParams sp;
+  {
+    const uint64_t dims[3] = {uint64_t(head_dim), uint64_t(n_blocks), uint64_t(heads)};
+    const uint64_t strides[2] = {uint64_t(head_dim) * 4, uint64_t(n_blocks) * head_dim * 4};
+    const uint32_t box_a[3] = {32, kScM, 1}, box_b[3] = {32, kScN, 1};
+    const uint64_t odims[3] = {uint64_t(nbp), uint64_t(n_blocks), uint64_t(chunk)};
+    const uint64_t ostrides[2] = {uint64_t(nbp) * 4, uint64_t(n_blocks) * nbp * 4};
+    const uint32_t box_o[3] = {32, 32, 1};
+    prism_status st = PRISM_OK;
+    if ((st = encode_tiled(&sp.q_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, q_hi, dims, strides, box_a,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != PRISM_OK ||
+        (st = encode_tiled(&sp.q_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, q_lo, dims, strides, box_a,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != PRISM_OK ||
+        (st = encode_tiled(&sp.k_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, k_hi, dims, strides, box_b,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != PRISM_OK ||
+        (st = encode_tiled(&sp.k_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, k_lo, dims, strides, box_b,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != PRISM_OK ||
+        (st = encode_tiled(&sp.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, logits, odims, ostrides, box_o,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != PRISM_OK)
+      return st;
+  }
+  sp.kbias = key_bias;
+  sp.nb = n_blocks;
+  sp.d = head_dim;
+  sp.scale = scale;
+  sp.status = ws_status(ws);
+  if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScSmem) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  const int vpt = select_vpt(n_blocks);
+  const int tiles_per_head = ((n_blocks + kScM - 1) / kScM) * ((n_blocks + kScN - 1) / kScN);
+  for (int h0 = 0; h0 < heads; h0 += chunk) {
+    const int g = std::min(chunk, heads - h0);
+    sp.head0 = h0;
+    sp.heads = g;
+    const int grid = std::min(g * tiles_per_head, device_sm_count());
+    score_kernel<<<grid, kScThreads, kScSmem, s>>>(sp);
+    if (launch_select_rows(vpt, logits, n_blocks, nbp, h0, g, hp, mask, kept, s) != cudaSuccess)
       return PRISM_ERR_CUDA;
-    select_kernel<8><<<grid, 512, smem, s>>>(q_pool, kT, n_blocks, nbp, head_dim, scale, hp, key_bias, mask, kept);
-  } else {
-    if (cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-      return PRISM_ERR_CUDA;
-    select_kernel<4><<<grid, 256, smem, s>>>(q_pool, kT, n_blocks, nbp, head_dim, scale, hp, key_bias, mask, kept);
   }
   const int rows = heads * n_blocks;
   if (launch_exclusive_scan(kept, rows, row_ptr, s) != cudaSuccess) return PRISM_ERR_CUDA;

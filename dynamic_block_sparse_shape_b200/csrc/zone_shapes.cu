@@ -397,7 +397,8 @@ __global__ void __launch_bounds__(32 * kChooseWarps) choose_kernel(const Geo g, 
                                                                    const double* __restrict__ zres, int have_feat,
                                                                    int have_res, float w_audio, float gamma,
                                                                    float gate_max, int32_t* __restrict__ zone_shape,
-                                                                   float* __restrict__ zone_margin) {
+                                                                   float* __restrict__ zone_margin,
+                                                                   const int* __restrict__ status) {
   __shared__ double red[32 * kChooseWarps];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   double s = 0;
@@ -428,6 +429,12 @@ __global__ void __launch_bounds__(32 * kChooseWarps) choose_kernel(const Geo g, 
       for (int o = 16; o; o >>= 1) q[k] += __shfl_xor_sync(0xffffffffu, q[k], o);
   }
   if (lane != 0) return;
+  if (*reinterpret_cast<const volatile int*>(status) & kDevErrTimeout) {
+    // a statistics kernel gave up waiting for its copies: its sums are incomplete
+    zone_shape[z] = -1;
+    if (zone_margin) zone_margin[z] = __int_as_float(0x7fc00000);
+    return;
+  }
   if (!have_feat && !have_res) {
     zone_shape[z] = 0;
     if (zone_margin) zone_margin[z] = INFINITY;
@@ -549,11 +556,73 @@ int device_sm_count() { return sm_count(); }
 
 using namespace prism;
 
-extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void* feat, int64_t feat_ld, int32_t feat_c,
-                                          prism_dtype feat_dtype, const void* res, int64_t res_ld, int32_t res_c,
-                                          prism_dtype res_dtype, const prism_shape_params* params,
-                                          int32_t* zone_shape, float* zone_margin, void* ws, size_t ws_bytes,
-                                          void* stream) {
+// ---------------------------------------------------------------------------
+// Allocation-free variant of prism_zone_shapes. The scratch (per-zone channel
+// partial sums, per-token residual norms, per-zone residual statistics and the
+// status word) lives in one file-scope device array instead of a caller
+// workspace. Host code only ever sees the array's host-side shadow, so the
+// device address is looked up with cudaGetSymbolAddress, once per device and
+// context: a new primary context (after cudaDeviceReset) reloads the module,
+// which may place the array elsewhere, so the address is looked up again.
+namespace prism {
+namespace {
+
+constexpr size_t kZoneStaticBytes = size_t(4) << 20;  // 4 MiB, held by every GPU that loads the library
+static __device__ __align__(256) uint8_t g_zone_scratch[kZoneStaticBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn g_ctx_get = nullptr;
+std::once_flag g_ctx_once;
+
+void load_ctx_get() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get = reinterpret_cast<CtxGetCurrentFn>(fn);
+}
+
+// Device address of g_zone_scratch in the current device's current context.
+prism_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_UNSUPPORTED;
+  std::call_once(g_ctx_once, load_ctx_get);
+  CUcontext ctx = nullptr;
+  if (g_ctx_get && g_ctx_get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
+    // (no context known yet, or a new one: the lookup itself makes the primary context current)
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_zone_scratch) != cudaSuccess || !p) return PRISM_ERR_CUDA;
+    if (g_ctx_get && g_ctx_get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+    g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
+  }
+  *out = g_scratch_ptr[dev];
+  return PRISM_OK;
+}
+
+}  // namespace
+}  // namespace prism
+
+namespace {
+
+// Where the scratch of a zone-shape call lives: the caller's workspace, or the
+// library's static device array (prism_zone_shapes_static).
+enum class ZoneScratch { kWorkspace, kStatic };
+
+// Validation and the launch sequence shared by prism_zone_shapes and
+// prism_zone_shapes_static; they differ only in where the scratch lives.
+prism_status zone_shapes_run(const prism_geometry* geo, const void* feat, int64_t feat_ld, int32_t feat_c,
+                             prism_dtype feat_dtype, const void* res, int64_t res_ld, int32_t res_c,
+                             prism_dtype res_dtype, const prism_shape_params* params, int32_t* zone_shape,
+                             float* zone_margin, ZoneScratch where, void* ws, size_t ws_bytes, void* stream) {
   Geo g;
   prism_status st = make_geo(geo, &g);
   if (st != PRISM_OK) return st;
@@ -568,17 +637,26 @@ extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void*
   } else {
     feat_c = 0;
   }
+  const int res_es = res_dtype == PRISM_FP32 ? 4 : 2;
   if (res) {
     if (res_dtype != PRISM_BF16 && res_dtype != PRISM_FP32) return PRISM_ERR_DTYPE;
     if (res_c <= 0 || res_c % 8 || res_ld < res_c || res_ld % 8) return PRISM_ERR_ARG;
     if (reinterpret_cast<uintptr_t>(res) % 16) return PRISM_ERR_ARG;
+    if ((int64_t(res_c) * res_es) % 16) return PRISM_ERR_ARG;
   } else {
     res_c = 0;
   }
   const int fes = feat_dtype == PRISM_FP32 ? 4 : 2;
   const ZoneWs L = zone_ws_layout(g, feat_c, fes, res_c);
-  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < L.total) return PRISM_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (where == ZoneScratch::kWorkspace) {
+    if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < L.total) return PRISM_ERR_WORKSPACE;
+  } else {
+    if (L.total > kZoneStaticBytes) return PRISM_ERR_UNSUPPORTED;  // grid too large for the static scratch
+    if ((st = static_scratch(&ws)) != PRISM_OK) return st;
+    // the status word is the only scratch a kernel reads before writing it
+    if (cudaMemsetAsync(ws_status(ws), 0, sizeof(int), s) != cudaSuccess) return PRISM_ERR_CUDA;
+  }
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
   float* partial = reinterpret_cast<float*>(w8 + L.partial);
   float* r = reinterpret_cast<float*>(w8 + L.r);
@@ -590,8 +668,6 @@ extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void*
     if ((st = launch_feat_stats(g, feat, feat_ld, feat_c, fes, n_chunks, partial, status, s)) != PRISM_OK) return st;
   }
   if (res) {
-    const int res_es = res_dtype == PRISM_FP32 ? 4 : 2;
-    if ((int64_t(res_c) * res_es) % 16) return PRISM_ERR_ARG;
     const int blocks = (N + 7) / 8;
     if (res_es == 2)
       res_norm_kernel<2><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(res), res_ld * res_es,
@@ -602,103 +678,28 @@ extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void*
     zone_res_kernel<<<g.n_zones, 256, 0, s>>>(g, r, zres);
     if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
   }
-  choose_kernel<<<(g.n_zones + kChooseWarps - 1) / kChooseWarps, 32 * kChooseWarps, 0, s>>>(g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio,
-                                   p.gamma, p.gate_max, zone_shape, zone_margin);
+  choose_kernel<<<(g.n_zones + kChooseWarps - 1) / kChooseWarps, 32 * kChooseWarps, 0, s>>>(
+      g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio, p.gamma, p.gate_max,
+      zone_shape, zone_margin, status);
   return cuda_status(cudaGetLastError());
 }
 
-// ---------------------------------------------------------------------------
-// Allocation-free variant of prism_zone_shapes. The scratch (per-zone channel
-// partial sums, per-token residual norms, per-zone residual statistics and the
-// status word) lives in one file-scope device array instead of a caller
-// workspace. Host code only ever sees the array's host-side shadow, so the
-// device address is looked up once per device with cudaGetSymbolAddress.
-namespace prism {
-namespace {
-
-constexpr size_t kZoneStaticBytes = size_t(4) << 20;  // 4 MiB, held by every GPU that loads the library
-static __device__ __align__(256) uint8_t g_zone_scratch[kZoneStaticBytes];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_zone_scratch on the current device (set up on first use).
-prism_status static_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_zone_scratch) != cudaSuccess || !p) return PRISM_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
-  return PRISM_OK;
-}
-
 }  // namespace
-}  // namespace prism
+
+extern "C" prism_status prism_zone_shapes(const prism_geometry* geo, const void* feat, int64_t feat_ld, int32_t feat_c,
+                                          prism_dtype feat_dtype, const void* res, int64_t res_ld, int32_t res_c,
+                                          prism_dtype res_dtype, const prism_shape_params* params,
+                                          int32_t* zone_shape, float* zone_margin, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  return zone_shapes_run(geo, feat, feat_ld, feat_c, feat_dtype, res, res_ld, res_c, res_dtype, params, zone_shape,
+                         zone_margin, ZoneScratch::kWorkspace, ws, ws_bytes, stream);
+}
 
 extern "C" prism_status prism_zone_shapes_static(const prism_geometry* geo, const void* feat, int64_t feat_ld,
                                                  int32_t feat_c, prism_dtype feat_dtype, const void* res,
                                                  int64_t res_ld, int32_t res_c, prism_dtype res_dtype,
                                                  const prism_shape_params* params, int32_t* zone_shape,
                                                  float* zone_margin, void* stream) {
-  Geo g;
-  prism_status st = make_geo(geo, &g);
-  if (st != PRISM_OK) return st;
-  if (!zone_shape) return PRISM_ERR_ARG;
-  const prism_shape_params def = {1.0f, 0.25f, 4.0f};
-  const prism_shape_params p = params ? *params : def;
-  if (!(p.gamma >= 0.f) || !(p.w_audio >= 0.f) || !(p.gate_max >= 0.f)) return PRISM_ERR_ARG;
-  if (feat) {
-    if (feat_dtype != PRISM_BF16 && feat_dtype != PRISM_FP32) return PRISM_ERR_DTYPE;
-    if (feat_c <= 0 || feat_c % 64 || feat_ld < feat_c || feat_ld % 8) return PRISM_ERR_ARG;
-    if (reinterpret_cast<uintptr_t>(feat) % 16) return PRISM_ERR_ARG;
-  } else {
-    feat_c = 0;
-  }
-  if (res) {
-    if (res_dtype != PRISM_BF16 && res_dtype != PRISM_FP32) return PRISM_ERR_DTYPE;
-    if (res_c <= 0 || res_c % 8 || res_ld < res_c || res_ld % 8) return PRISM_ERR_ARG;
-    if (reinterpret_cast<uintptr_t>(res) % 16) return PRISM_ERR_ARG;
-  } else {
-    res_c = 0;
-  }
-  const int fes = feat_dtype == PRISM_FP32 ? 4 : 2;
-  const ZoneWs L = zone_ws_layout(g, feat_c, fes, res_c);
-  if (L.total > kZoneStaticBytes) return PRISM_ERR_UNSUPPORTED;  // grid too large for the static scratch
-  void* scratch = nullptr;
-  if ((st = static_scratch(&scratch)) != PRISM_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* w8 = static_cast<uint8_t*>(scratch);
-  float* partial = reinterpret_cast<float*>(w8 + L.partial);
-  float* r = reinterpret_cast<float*>(w8 + L.r);
-  double* zres = reinterpret_cast<double*>(w8 + L.zres);
-  int* status = ws_status(scratch);
-  // the status word is the only scratch a kernel reads before writing it
-  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return PRISM_ERR_CUDA;
-  const int N = g.T * g.H * g.W;
-  const int n_chunks = feat_c * fes / 128;
-  if (feat) {
-    if ((st = launch_feat_stats(g, feat, feat_ld, feat_c, fes, n_chunks, partial, status, s)) != PRISM_OK) return st;
-  }
-  if (res) {
-    const int res_es = res_dtype == PRISM_FP32 ? 4 : 2;
-    if ((int64_t(res_c) * res_es) % 16) return PRISM_ERR_ARG;
-    const int blocks = (N + 7) / 8;
-    if (res_es == 2)
-      res_norm_kernel<2><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(res), res_ld * res_es,
-                                                res_c * res_es, N, r);
-    else
-      res_norm_kernel<4><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint8_t*>(res), res_ld * res_es,
-                                                res_c * res_es, N, r);
-    zone_res_kernel<<<g.n_zones, 256, 0, s>>>(g, r, zres);
-    if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
-  }
-  choose_kernel<<<(g.n_zones + kChooseWarps - 1) / kChooseWarps, 32 * kChooseWarps, 0, s>>>(g, partial, n_chunks, feat_c, zres, feat != nullptr, res != nullptr, p.w_audio,
-                                   p.gamma, p.gate_max, zone_shape, zone_margin);
-  return cuda_status(cudaGetLastError());
+  return zone_shapes_run(geo, feat, feat_ld, feat_c, feat_dtype, res, res_ld, res_c, res_dtype, params, zone_shape,
+                         zone_margin, ZoneScratch::kStatic, nullptr, 0, stream);
 }

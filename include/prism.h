@@ -160,6 +160,9 @@ PRISM_API prism_status prism_check_device_status(void* ws, void* stream);
  * zone_shape: device int32 [n_zones] out (candidate index per zone).
  * zone_margin: device float [n_zones] out (second-best minus best cost), or
  *       NULL.
+ * A statistics kernel whose bounded wait for its copies ran out leaves every
+ * zone_shape entry -1 (and every margin NaN) besides setting PRISM_ERR_TIMEOUT
+ * in the workspace status word.
  */
 PRISM_API prism_status prism_zone_shapes(const prism_geometry* geo, const void* feat, int64_t feat_ld, int32_t feat_c,
                                prism_dtype feat_dtype, const void* res, int64_t res_ld, int32_t res_c,
@@ -182,12 +185,14 @@ PRISM_API prism_status prism_zone_shapes(const prism_geometry* geo, const void* 
  * tokens needs 2.1 MB); a call that needs more returns PRISM_ERR_UNSUPPORTED.
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  * routine). The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress with that device current); make that first call before
- * any stream capture. All calls share the array and it keeps the last call's
- * contents, so calls that overlap on the GPU (different streams, or several
- * host threads) race and must be serialised by the caller. Device-side wait
- * timeouts are not reported by this variant (there is no workspace to hold
- * the status word the caller could read back).
+ * (cudaGetSymbolAddress with that device current), and looks it up again when
+ * the device's context has changed (after cudaDeviceReset the module is
+ * reloaded and the array may move); make that first call before any stream
+ * capture. All calls share the array and it keeps the last call's contents, so
+ * calls that overlap on the GPU (different streams, or several host threads)
+ * race and must be serialised by the caller. There is no workspace status word
+ * to read back: a device-side wait that ran out shows as zone_shape entries of
+ * -1 (margins NaN), which the downstream entry points reject as out of range.
  */
 PRISM_API prism_status prism_zone_shapes_static(const prism_geometry* geo, const void* feat, int64_t feat_ld,
                                                 int32_t feat_c, prism_dtype feat_dtype, const void* res,
@@ -221,8 +226,11 @@ PRISM_API prism_status prism_block_pool(const prism_geometry* geo, const int32_t
  * For head h and query block I: s_J = scale * q_pool[h,I] . k_pool[h,J] over
  * all key blocks J; p = softmax(s); blocks ranked by p descending, ties to the
  * lower J; m = max(top_k, min{m : p_(1) + ... + p_(m) >= cdf_threshold});
- * top_k >= n_blocks or cdf_threshold >= 1 keeps every block. Scores are never
- * written to memory.
+ * top_k >= n_blocks or cdf_threshold >= 1 keeps every block. The logits are
+ * formed on the tensor cores in split tf32 precision (hi.hi + hi.lo + lo.hi,
+ * relative error about 2^-20) for a round of heads at a time and held in the
+ * workspace (up to 96 MiB, sized to stay in L2) until that round's selection
+ * has read them; they are not an output.
  *
  * q_pool, k_pool: device float [heads, n_blocks, head_dim]; n_blocks at most
  *       10240 and heads * n_blocks^2 below 2^31 (PRISM_ERR_UNSUPPORTED
@@ -243,8 +251,10 @@ PRISM_API prism_status prism_block_pool(const prism_geometry* geo, const int32_t
  *       reports PRISM_ERR_DEVICE through prism_check_device_status).
  * ws: at least prism_workspace_size(PRISM_OP_BLOCK_SELECT, geo, heads,
  *       head_dim, ...) bytes (equivalently prism_block_select_workspace_size):
- *       the status word and a key-major copy of k_pool, heads * head_dim *
- *       ceil4(n_blocks) floats, from which the scores are formed.
+ *       the status word, the tf32 halves of q_pool and k_pool (4 * heads *
+ *       n_blocks * head_dim floats) and one round's logits (R * n_blocks *
+ *       ceil4(n_blocks) floats, R = the heads whose logits fit in 96 MiB, at
+ *       least 1).
  */
 PRISM_API prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,
                                 int32_t head_dim, float scale, int32_t top_k, float cdf_threshold, uint32_t* mask,
