@@ -371,14 +371,26 @@ def cpu_sample(wl, x, feats, res, q_blocks=4, kv_blocks=2, sel_rows=256, users_p
             "wall_s": round(time.time() - t_all, 1), "stage_ms": {k: round(1e3 * v, 1) for k, v in timings.items()}}
 
 
-def selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src):
-    """HBM roofline of the streaming stages: the zone statistics read the features and
-    the a2v residual once, the pooling reads Q and K once (algorithmic bytes)."""
+def selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src, nb):
+    """Rooflines of the selection path.
+
+    zone_shapes and block_pool are HBM streams: the zone statistics read the
+    features and the a2v residual once, the pooling reads Q and K once
+    (algorithmic bytes). block_select is not bound by HBM: its dominant work is
+    the block scoring, 2 * heads * nb^2 * d FLOP of dot products, executed on
+    the tensor cores as three tf32 products (hi.hi + hi.lo + lo.hi); it is
+    reported against the tf32 dense peak (the measured bf16 peak x 1/2, the
+    nominal tf32 / bf16 ratio) over the whole stage time (scores, threshold
+    search and bitmask), with its HBM bytes (pooled q and k read, bitmask and
+    counts written) for completeness. "path" sums the algorithmic bytes of all
+    three stages over their summed time against the HBM copy bandwidth."""
     hbm = float(peaks.get("hbm_gbs"))
     q_bytes = wl.n_tokens * wl.heads * wl.head_dim * 2
     stat_bytes = sum(t.numel() * t.element_size() for t in (feats, res) if t is not None)
+    pooled_bytes = 2 * wl.heads * nb * wl.head_dim * 4
+    sel_bytes = pooled_bytes + wl.heads * nb * ((nb + 31) // 32) * 4 + wl.heads * nb * 4 * 2
     out = {}
-    for name, nbytes in (("zone_shapes", stat_bytes), ("block_pool", 2 * q_bytes)):
+    for name, nbytes in (("zone_shapes", stat_bytes), ("block_pool", 2 * q_bytes + pooled_bytes)):
         ms = stage_ms.get(name)
         if not ms or not nbytes:
             continue
@@ -386,6 +398,24 @@ def selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src):
         out[name] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
                      "peak_source": f"{peak_src} copy bandwidth"}
+    ms = stage_ms.get("block_select")
+    if ms:
+        flop = 2.0 * wl.heads * nb * nb * wl.head_dim
+        tf32_peak = float(peaks.get("bf16_tflops")) / 2.0
+        executed = 3.0 * flop / (ms * 1e-3) / 1e12
+        out["block_select"] = {"bound": "tensor", "achieved": round(executed, 1), "peak": round(tf32_peak, 1),
+                               "unit": "TFLOP/s", "frac": round(executed / tf32_peak, 4),
+                               "scoring_flop": flop, "executed_tf32_flop": 3.0 * flop,
+                               "peak_source": f"{peak_src} bf16 burst x 1/2 (nominal tf32/bf16)",
+                               "hbm_gbs": round(sel_bytes / (ms * 1e-3) / 1e9, 1), "algorithmic_bytes": sel_bytes}
+    names = [n for n in ("zone_shapes", "block_pool", "block_select") if stage_ms.get(n)]
+    if names:
+        tot_ms = sum(stage_ms[n] for n in names)
+        tot_b = stat_bytes + 2 * q_bytes + pooled_bytes + sel_bytes
+        gbs = tot_b / (tot_ms * 1e-3) / 1e9
+        out["path"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                       "frac": round(gbs / hbm, 4), "algorithmic_bytes": tot_b, "ms": round(tot_ms, 3),
+                       "stages": names, "peak_source": f"{peak_src} copy bandwidth"}
     return out
 
 
@@ -523,8 +553,10 @@ def run_gpu(args):
                      "traffic": round(nnz * ATTN_DRAM_BYTES_PER_PAIR) if pipe.backward else None,
                      "traffic_source": "ncu dram bytes per selected pair (2-head 2K capture) x selected pairs",
                      "peak_source": f"{peak_src} bf16 sustained",
+                     "peak_burst": float(peaks.get("bf16_tflops")),
+                     "frac_burst": round(achieved / float(peaks.get("bf16_tflops")), 4),
                      "flop_per_pair": flop_per_pair},
-        "roofline_selection_path": selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src),
+        "roofline_selection_path": selection_path_roofline(wl, stage_ms, feats, res, peaks, peak_src, pipe.nb),
         "selection_variants": variants,
         "e2e": e2e,
         "gpu_launches": pipe.launches_per_step() * args.steps,

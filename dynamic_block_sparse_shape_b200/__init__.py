@@ -25,7 +25,8 @@ __all__ = [
 DEFAULT_CDF_THRESHOLD = 0.20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libprism.so")
+# PRISM_LIBRARY names another build of the library (a test variant) to load instead
+_LIB_PATH = os.environ.get("PRISM_LIBRARY") or os.path.join(_HERE, "libprism.so")
 
 STATUS = {
     0: "PRISM_OK", 1: "PRISM_ERR_ARG", 2: "PRISM_ERR_SHAPE", 3: "PRISM_ERR_DTYPE", 4: "PRISM_ERR_WORKSPACE",

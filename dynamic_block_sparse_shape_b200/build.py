@@ -48,16 +48,35 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
+# Test-only variant: device waits give up after 50 ms instead of about 2 s, and the
+# forward's copy producer can be told (through a workspace word) to skip one step's
+# copies, so that a test can make a bounded wait run out and check the reported status.
+FAULT_INJECTION_FLAGS = ["-DPRISM_FAULT_INJECTION", "-DPRISM_WAIT_LIMIT_NS=50000000ull"]
+
+
+def variant_path(tag: str) -> str:
+    return os.path.join(HERE, f"libprism_{tag}.so")
+
+
+def build_variant(tag: str, flags, verbose: bool = False) -> str:
+    """Builds a separately named copy of the library with extra compile flags
+    (objects in _build_<tag>/, library libprism_<tag>.so); returns its path."""
+    return build(verbose=verbose, extra_flags=flags, obj_dir=os.path.join(HERE, f"_build_{tag}"),
+                 out=variant_path(tag))
+
+
+def build(verbose: bool = False, force: bool = False, extra_flags=None, obj_dir=None, out=None) -> str:
     """Compile every .cu for sm_100a and link libprism.so; returns its path."""
-    os.makedirs(OBJ_DIR, exist_ok=True)
+    obj_dir = obj_dir or OBJ_DIR
+    out = out or OUT
+    os.makedirs(obj_dir, exist_ok=True)
     srcs = _sources()
     hdrs = _headers()
     flags = FLAGS + list(extra_flags or [])
     objs = []
     jobs = []
     for s in srcs:
-        o = os.path.join(OBJ_DIR, os.path.splitext(os.path.basename(s))[0] + ".o")
+        o = os.path.join(obj_dir, os.path.splitext(os.path.basename(s))[0] + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs + [__file__]):
             jobs.append([nvcc(), *ARCH, *flags, "-c", s, "-o", o])
@@ -71,11 +90,11 @@ def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
         list(ex.map(run, jobs))
-    if force or jobs or _stale(OUT, objs):
-        tmp = OUT + ".tmp"
+    if force or jobs or _stale(out, objs):
+        tmp = out + ".tmp"
         run([nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs])
-        os.replace(tmp, OUT)
-    return OUT
+        os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

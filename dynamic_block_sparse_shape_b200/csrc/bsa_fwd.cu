@@ -202,6 +202,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
           tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], q_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
       }
       int kj = 0, vj = 0;
+#ifdef PRISM_FAULT_INJECTION
+      // test builds only: when the workspace word after the status word is set, the CTA of
+      // (query block 0, head 0) never issues the K copies of its second step, so the score
+      // issuer's bounded wait for them runs out (the timeout path under test)
+      const int skip_k = (blockIdx.x == 0 && blockIdx.y == 0 &&
+                          *reinterpret_cast<volatile int*>(status + 1) != 0) ? 1 : -1;
+#endif
       Watchdog wd;
       wd.reset();
       while (kj < nsteps || vj < nsteps) {
@@ -212,13 +219,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
           // K slot nk%3 last held the K of step nk-3: free once S_{nk-3} completed
           if (nk < nsteps && mbar_test(&k_free[nk % kRing], ((nk / kRing) & 1) ^ 1)) {
             const int ks = nk % kRing;
-            uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
-            mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
-            for (int slot = 0; slot < kKB; ++slot) {
-              const uint8_t* src = P.kimg + image_offset(g, head, dc.get(kKB * nk + slot), D);
-              for (int dh = 0; dh < D / 64; ++dh)
-                bulk_load(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, src + dh * kBoxBytes, kBoxBytes,
-                          &k_full[ks]);
+            bool issue = true;
+#ifdef PRISM_FAULT_INJECTION
+            issue = nk != skip_k;
+#endif
+            if (issue) {
+              uint8_t* dst = sm + L::kK0 + ks * L::kSlotBytes;
+              mbar_arrive_expect_tx(&k_full[ks], L::kSlotBytes);
+              for (int slot = 0; slot < kKB; ++slot) {
+                const uint8_t* src = P.kimg + image_offset(g, head, dc.get(kKB * nk + slot), D);
+                for (int dh = 0; dh < D / 64; ++dh)
+                  bulk_load(dst + dh * (kKB * kBoxBytes) + slot * kBoxBytes, src + dh * kBoxBytes, kBoxBytes,
+                            &k_full[ks]);
+              }
             }
             ++nk;
             did = true;
