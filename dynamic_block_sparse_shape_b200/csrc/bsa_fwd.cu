@@ -48,6 +48,7 @@
 // while the rare O rescale (TMEM load/scale/store) stays off the common path.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -65,6 +66,7 @@ constexpr int kSoftWarps = kGroups * kGroupWarps;
 constexpr int kFwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kPvWarp = 2 + kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kSmallSteps = 4;  // rows of up to 8 key blocks go to bsa_fwd_small_kernel
 
 struct FwdParams {
   CUtensorMap mq[kMaxCand];
@@ -84,6 +86,7 @@ struct FwdParams {
   float scale_log2;
   int out_fp32;
   int tma_out;  // bf16 output: stores through the O / o_lo tensor maps
+  int heads;
 };
 
 template <int D>
@@ -157,6 +160,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
     cnt = 0;
   }
   const int nsteps = (cnt + kKB - 1) / kKB;
+  if (nsteps <= kSmallSteps) return;  // short and empty rows: bsa_fwd_small_kernel's
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -531,6 +535,352 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
   }
 }
 
+// ---------------------------------------------------------------- short rows
+// Rows of at most kSmallSteps steps (and empty rows) go to a second kernel
+// whose CTA needs a quarter of the tensor memory and 83 KB of shared memory,
+// so two CTAs share an SM and each one's fixed latencies (launch, the Q and
+// first K/V copies, the epilogue) overlap the other's work. A row of a few
+// key blocks is mostly fixed cost: on the 2K grid one CTA of bsa_fwd_kernel
+// spends about 7 us per row before and after its 0.5 us steps. Long rows stay
+// with bsa_fwd_kernel, which returns at once for the short ones.
+//   warp 0      copies: Q once (5-D TMA), per step K and V of the step's two
+//               key blocks into one K and one V slot (bulk copies of images);
+//   warp 1      TMEM owner, issues S_j = Q [K_j0 K_j1]^T and then
+//               O += P_j [V_j0 | V_j1] (.ws M=64; Q and P from TMEM), one
+//               step at a time: P_j is written over S_j's first 32 columns,
+//               so S_{j+1} waits for PV_j;
+//   warps 2..5  softmax, one thread per TMEM lane (row m of the block,
+//               key-block half kh of the step), running max and sum per
+//               lane half, merged in the epilogue.
+constexpr int kSmallThreads = 64 + 128;
+
+template <int D>
+struct FwdSmallSmem {
+  static constexpr uint32_t kQ = 0;                      // [dh][64][128 B]
+  static constexpr uint32_t kQBytes = D * 128;
+  static constexpr uint32_t kSlotBytes = kKB * D * 128;  // K (or V) of one step
+  static constexpr uint32_t kK = kQBytes;                // [dh][block][64][128 B]
+  static constexpr uint32_t kV = kK + kSlotBytes;        // [block][dh][64][128 B]
+  static constexpr uint32_t kRed = kV + kSlotBytes;      // per lane half: running max, sum [2][64] each
+  static constexpr uint32_t kRedBytes = 2 * 2 * 64 * 4;
+  static constexpr uint32_t kDesc = kRed + kRedBytes;  // block-id ring
+  static constexpr uint32_t kBar = kDesc + kDescRing * 4;
+  static constexpr uint32_t kTotal = kBar + 128;
+  // epilogue exchange of half rows: [lane half][64 rows][D/2 + 4 floats], over the K and V slots
+  static constexpr uint32_t kXPitch = D / 2 + 4;
+  static_assert(2 * 64 * kXPitch * 4 <= 2 * kSlotBytes, "exchange buffer fits the slots");
+  // TMEM: S (P over its first 32 columns) at 0, the O parts at 64 (D columns), Q at 64 + D (D/2)
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kTO = 64;
+  static constexpr uint32_t kTQ = 64 + D;
+  static_assert(kTQ + D / 2 <= kTmemCols, "TMEM budget");
+};
+
+// Output rows of an empty query block: O = 0 (and its residual), LSE = -inf.
+template <int D>
+__device__ __forceinline__ void write_empty_row(const FwdParams& P, int I, int head, int tid) {
+  const Geo& g = P.g;
+  if (tid >= 128) return;
+  const int m = tid & 63, half = tid >> 6;
+  int* status = P.status;
+  const int sI = safe_shape(g, P.zone_shape, I, status);
+  const BlockBox qb = block_box(g, sI, I);
+  if (g.partial && !block_slot_in_grid(g, qb, m)) return;
+  const int tok = block_token(g, qb, m);
+  constexpr int NC = D / 2;
+  float z[NC];
+#pragma unroll
+  for (int i = 0; i < NC; ++i) z[i] = 0.f;
+  const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + half * NC;
+  store_row<NC>(P.o, off, z, P.out_fp32);
+  if (P.o_lo) store_row<NC>(P.o_lo, off, z, false);
+  if (half == 0) P.lse[int64_t(head) * g.T * g.H * g.W + tok] = -INFINITY;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const __grid_constant__ FwdParams P) {
+  using L = FwdSmallSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* qa_full = bars + 1;   // Q copied into TMEM by the softmax warps
+  uint64_t* k_full = bars + 2;    // K of the step landed
+  uint64_t* k_free = bars + 3;    // S of the step complete (K slot free)
+  uint64_t* v_full = bars + 4;    // V of the step landed
+  uint64_t* s_full = bars + 5;    // S of the step complete
+  uint64_t* p_full = bars + 6;    // P of the step written (4 warps)
+  uint64_t* pv_done = bars + 7;   // PV of the step complete (V slot and S / P columns free)
+  uint64_t* mma_done = bars + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
+  float* redm = reinterpret_cast<float*>(sm + L::kRed);
+  float* redl = redm + 2 * 64;
+  const Geo& g = P.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = P.status;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tO = tbase + L::kTO, tQ = tbase + L::kTQ;
+  bool first = true;
+  // CTA b takes rows b, b + grid, ... (row = head * n_blocks + query block), the short and empty ones
+  for (int row = blockIdx.x; row < P.heads * g.n_blocks; row += gridDim.x) {
+    const int I = row % g.n_blocks, head = row / g.n_blocks;
+    const int beg = P.row_ptr[row];
+    int cnt = P.row_ptr[row + 1] - beg;
+    if (cnt < 0 || cnt > g.n_blocks) {
+      if (threadIdx.x == 0) atomicOr(status, kDevErrBounds);
+      cnt = 0;
+    }
+    const int nsteps = (cnt + kKB - 1) / kKB;
+    if (nsteps > kSmallSteps) continue;  // a long row: bsa_fwd_kernel's (uniform)
+    if (nsteps == 0) {
+      write_empty_row<D>(P, I, head, threadIdx.x);
+      continue;
+    }
+    if (threadIdx.x == 0) {
+      // the previous row left no copy, product or arrival pending on any barrier
+      if (!first)
+        for (int i = 0; i < 9; ++i) mbar_inval(&bars[i]);
+      for (int i = 0; i < 9; ++i) mbar_init(&bars[i], (i == 1 || i == 6) ? 4 : 1);
+      *abort_flag = 0;
+      fence_barrier_init();
+    }
+    first = false;
+    __syncthreads();
+
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
+      if (lane == 0) {
+        const int sI = safe_shape(g, P.zone_shape, I, status);
+        const BlockBox qb = block_box(g, sI, I);
+        mbar_arrive_expect_tx(q_full, L::kQBytes);
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], q_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+      }
+      bool ok = true;
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < nsteps && ok; ++j) {
+        dc.ensure(kKB * j + kKB - 1, g, P.col_idx, beg, cnt, status, lane);
+        if (lane == 0) {
+          // the K slot last held step j - 1: free once S_{j-1} completed
+          if (j > 0) ok = mbar_wait_abortable(k_free, (j - 1) & 1, status, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(k_full, L::kSlotBytes);
+            for (int slot = 0; slot < kKB; ++slot) {
+              const uint8_t* src = P.kimg + image_offset(g, head, dc.get(kKB * j + slot), D);
+              for (int dh = 0; dh < D / 64; ++dh)
+                bulk_load(sm + L::kK + dh * (kKB * kBoxBytes) + slot * kBoxBytes, src + dh * kBoxBytes, kBoxBytes,
+                          k_full);
+            }
+            k_issued = j + 1;
+          }
+          // the V slot last held step j - 1: free once PV_{j-1} completed
+          if (ok && j > 0) ok = mbar_wait_abortable(pv_done, (j - 1) & 1, status, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(v_full, L::kSlotBytes);
+            for (int slot = 0; slot < kKB; ++slot)
+              bulk_load(sm + L::kV + slot * (D * 128), P.vimg + image_offset(g, head, dc.get(kKB * j + slot), D),
+                        D * 128, v_full);
+            v_issued = j + 1;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      if (lane == 0) {
+        // drain: every issued copy has landed before the CTA may exit (one slot each: the last)
+        mbar_wait(q_full, 0, status);
+        if (k_issued > 0) mbar_wait(k_full, (k_issued - 1) & 1, status);
+        if (v_issued > 0) mbar_wait(v_full, (v_issued - 1) & 1, status);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ issuer
+      if (lane == 0) {
+        const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
+        const uint64_t dK = sdesc_sw128(smem_u32(sm + L::kK), 16, 1024);
+        // B = V of the step, MN-major, N = 2d: the d channels of key block 0, then those of key block 1
+        const uint32_t idO = idesc_bf16_f32(64, 2 * D, false, true);
+        const uint64_t dV = sdesc_sw128(smem_u32(sm + L::kV), kBoxBytes, 1024);
+        bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
+        for (int j = 0; j < nsteps && ok; ++j) {
+          // K of step j landed; PV_{j-1} (which read P from the S columns) complete
+          ok = mbar_wait_abortable(k_full, j & 1, status, abort_flag) &&
+               (j == 0 || mbar_wait_abortable(pv_done, (j - 1) & 1, status, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws_ts(tbase, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+          mma_commit(s_full);
+          mma_commit(k_free);
+          ok = mbar_wait_abortable(p_full, j & 1, status, abort_flag) &&
+               mbar_wait_abortable(v_full, j & 1, status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ws_ts(tO, tbase + kk * 8, dV + uint64_t((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(pv_done);
+        }
+        // every product this thread issued has completed before TMEM is released
+        mma_commit(mma_done);
+        mbar_wait(mma_done, 0, status);
+      }
+    } else {
+      // ------------------------------------------------------------ softmax
+      const int sp = warp & 3;  // TMEM lane quarter of this warp
+      const int Ln = sp * 32 + lane;
+      const int m = Ln & 63, kh = Ln >> 6;
+      const uint32_t lane_off = uint32_t(sp * 32) << 16;
+      float m_run = -INFINITY, l_run = 0.f;
+      // Q becomes the A operand of every S product: both column halves of this lane's row
+      mbar_wait_abortable(q_full, 0, status, abort_flag);
+      tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, 0);
+      tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, 1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qa_full);
+      for (int j = 0; j < nsteps; ++j) {
+        const bool valid = (j * kKB + kh) < cnt;  // warp-uniform: kh is fixed per warp
+        uint64_t members = ~uint64_t(0);
+        if (g.partial && valid) members = key_block_members(g, P.zone_shape, __ldg(P.col_idx + beg + j * kKB + kh));
+        mbar_wait_abortable(s_full, j & 1, status, abort_flag);
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld32(tbase + lane_off, r);
+        tmem_ld32(tbase + lane_off + 32, r + 32);
+        tmem_ld_wait();
+        mask_scores32(r, uint32_t(members));
+        mask_scores32(r + 32, uint32_t(members >> 32));
+        const float mx = valid ? max64(r) * P.scale_log2 : -INFINITY;
+        const float m_new = fmaxf(m_run, mx);
+        const bool resc = m_new > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, resc)) {
+          const float alpha = resc ? fast_exp2(m_run - m_new) : 1.f;
+          if (resc) {
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          if (j > 0) {
+            // O holds PV_{j-1}, complete: S_j was issued after it
+  #pragma unroll
+            for (int h = 0; h < D / 32; ++h) {
+              uint32_t o[32];
+              const uint32_t ta = tO + lane_off + h * 32;
+              tmem_ld32(ta, o);
+              tmem_ld_wait();
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st16(ta, o);
+              tmem_st16(ta + 16, o + 16);
+            }
+            tmem_st_wait();
+          }
+        }
+        uint32_t pk[32];
+        if (valid) {
+          const float c = P.scale_log2, nm = m_run == -INFINITY ? 0.f : -m_run;
+          float la = 0.f, lb = 0.f;
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(r[2 * i]), c, nm));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(r[2 * i + 1]), c, nm));
+            la += p0;
+            lb += p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          l_run += la + lb;
+        } else {
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        }
+        // P over the first 32 columns of S (every S value of this lane was read above)
+        tmem_st16(tbase + lane_off, pk);
+        tmem_st16(tbase + lane_off + 16, pk + 16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      // ---------------------------------------------------------- epilogue
+      mbar_wait_abortable(pv_done, (nsteps - 1) & 1, status, abort_flag);
+      tc_fence_after();
+      redm[kh * 64 + m] = m_run;
+      redl[kh * 64 + m] = l_run;
+      named_bar_sync(1, 128);
+      const bool ok = *abort_flag == 0;  // uniform: read after the barrier
+      const float M = fmaxf(redm[m], redm[64 + m]);
+      float Lsum = 0.f;
+  #pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float lq = redl[q * 64 + m];
+        if (lq > 0.f) Lsum += lq * fast_exp2(redm[q * 64 + m] - M);
+      }
+      const float inv = (Lsum > 0.f && ok) ? 1.f / Lsum : 0.f;
+      const float w = l_run > 0.f ? fast_exp2(m_run - M) * inv : 0.f;  // weight of this lane's part
+      // this thread keeps channel half kh of row m and hands half kh ^ 1 to the other lane half
+      constexpr int NC = D / 2;
+      float* X = reinterpret_cast<float*>(sm + L::kK);
+      float ov[NC];
+      {
+        float gv[32];
+  #pragma unroll
+        for (int h = 0; h < NC / 32; ++h) {
+          tmem_ld_f<32>(tO + lane_off + (kh ^ 1) * NC + h * 32, gv);
+          float* xo = X + ((kh ^ 1) * 64 + m) * L::kXPitch + h * 32;
+  #pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(xo)[i] =
+                make_float4(gv[4 * i] * w, gv[4 * i + 1] * w, gv[4 * i + 2] * w, gv[4 * i + 3] * w);
+          tmem_ld_f<32>(tO + lane_off + kh * NC + h * 32, ov + h * 32);
+        }
+      }
+      named_bar_sync(1, 128);
+      const float* xi = X + (kh * 64 + m) * L::kXPitch;
+  #pragma unroll
+      for (int i = 0; i < NC / 4; ++i) {
+        const float4 t = reinterpret_cast<const float4*>(xi)[i];
+        ov[4 * i] = fmaf(ov[4 * i], w, t.x);
+        ov[4 * i + 1] = fmaf(ov[4 * i + 1], w, t.y);
+        ov[4 * i + 2] = fmaf(ov[4 * i + 2], w, t.z);
+        ov[4 * i + 3] = fmaf(ov[4 * i + 3], w, t.w);
+      }
+  #pragma unroll
+      for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : ov[i];
+      const int sI = safe_shape(g, P.zone_shape, I, status);
+      const BlockBox qb = block_box(g, sI, I);
+      const int tok = block_token(g, qb, m);
+      const bool row_in = !g.partial || block_slot_in_grid(g, qb, m);
+      if (row_in) {
+        const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * NC;
+        store_row<NC>(P.o, off, ov, P.out_fp32);
+        if (P.o_lo) {
+          float lo[NC];
+  #pragma unroll
+          for (int i = 0; i < NC; ++i) lo[i] = ov[i] - __bfloat162float(__float2bfloat16_rn(ov[i]));
+          store_row<NC>(P.o_lo, off, lo, false);
+        }
+        if (kh == 0) {
+          const int N = g.T * g.H * g.W;
+          P.lse[int64_t(head) * N + tok] = (Lsum > 0.f && ok) ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+        }
+      }
+    }
+    // the row is complete (copies drained, products complete) before the next one
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (warp == 1) tmem_dealloc(tbase, L::kTmemCols);
+}
+
 // fp32 -> bf16 staging copy of a token-major tensor (contiguous output).
 __global__ void to_bf16_kernel(const float* __restrict__ src, int64_t tok_stride, int C, int64_t n_tokens,
                                __nv_bfloat16* __restrict__ dst) {
@@ -690,7 +1040,25 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
   P.tok_stride = tok_stride;
   P.scale_log2 = scale * 1.4426950408889634f;
   P.out_fp32 = dtype == PRISM_FP32;
+  P.heads = heads;
+  // long rows: one CTA per row, launched in row order (neighbouring rows share key blocks in L2);
+  // short and empty rows: two CTAs per SM, each looping over its rows
   const dim3 grid(g.n_blocks, heads);
+  const dim3 grid_small(std::min(heads * g.n_blocks, 2 * device_sm_count()));
+  // short and empty rows first (two CTAs per SM), then the long rows
+  if (head_dim == 128) {
+    const size_t smem = FwdSmallSmem<128>::kTotal + 1024;
+    if (cudaFuncSetAttribute(bsa_fwd_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return PRISM_ERR_CUDA;
+    bsa_fwd_small_kernel<128><<<grid_small, kSmallThreads, smem, s>>>(P);
+  } else {
+    const size_t smem = FwdSmallSmem<64>::kTotal + 1024;
+    if (cudaFuncSetAttribute(bsa_fwd_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return PRISM_ERR_CUDA;
+    bsa_fwd_small_kernel<64><<<grid_small, kSmallThreads, smem, s>>>(P);
+  }
   if (head_dim == 128) {
     const size_t smem = FwdSmem<128>::kTotal + 1024;
     if (cudaFuncSetAttribute(bsa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=

@@ -25,7 +25,7 @@ def main():
     zone_shape = rng.integers(0, len(cand), nz)
     mask = rng.random((H, nb, nb)) < 0.25
     mask[:, np.arange(nb), np.arange(nb)] = True
-    mask[0, 0, :8] = True  # query block 0 of head 0 takes at least four steps
+    mask[0, 0, :16] = True  # query block 0 of head 0 takes eight steps or more (the long-row kernel)
     counts = mask.reshape(H * nb, nb).sum(axis=1)
     row_ptr = np.zeros(H * nb + 1, dtype=np.int64)
     row_ptr[1:] = np.cumsum(counts)
