@@ -37,11 +37,12 @@ FWD_FLOP_PER_PAIR = 4 * 64 * 64 * 128  # QK^T and PV over one (query block, key 
 BWD_FLOP_PER_PAIR = 2.5 * FWD_FLOP_PER_PAIR
 # DRAM bytes (read + write) per selected (query block, key block) pair of the three attention
 # kernels together (forward, dQ, dK/dV), from one ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum) of the 2-head 2K workload: 91.72 GB over 4,445,104 pairs (forward
-# 26.98, dQ 25.90, dK/dV 38.84 GB). Scaled by the selected pairs of the timed workload; the operand
-# re-reads that miss L2 grow with the pairs. The block-image passes before each kernel (one read
-# and one write of the streamed operands) are not included.
-ATTN_DRAM_BYTES_PER_PAIR = 91.72e9 / 4445104
+# dram__bytes_write.sum) of the 2-head 2K workload taken after the last change to each kernel:
+# 92.42 GB over 4,445,106 pairs (forward 27.35, dQ 26.35, dK/dV 38.73 GB). Scaled by the selected
+# pairs of the timed workload; the operand re-reads that miss L2 grow with the pairs. The
+# block-image passes before each kernel (one read and one write of the streamed operands) are not
+# included.
+ATTN_DRAM_BYTES_PER_PAIR = 92.42e9 / 4445106
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -690,6 +691,9 @@ def run_sweep(args):
     pbuild.build()
     dev = torch.device("cuda")
     points = synth.sweep_workloads()
+    if args.sweep_filter:
+        import re
+        points = [w for w in points if re.search(args.sweep_filter, w.name)]
     by_amp = {}
     for wl in points:
         by_amp.setdefault(wl.amplitude, []).append(wl)
@@ -747,6 +751,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="run the 45-point selection/sparsity sweep instead")
+    ap.add_argument("--sweep-filter", default="", help="with --sweep: only the points whose name matches this regex")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="multi-GPU layout: independent replicas, or one layer's heads split across ranks")
     ap.add_argument("--head-slice", default="", help="a:b, time heads a..b-1 of the layer alone (one shard)")
