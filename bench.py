@@ -242,7 +242,7 @@ class Pipeline:
     STAGES = ("zone_shapes", "block_pool", "block_select", "bsa_fwd", "bsa_bwd")
     # kernels each stage launches (prism kernels only; memsets excluded)
     # (bsa_fwd: K and V block images + attention; bsa_bwd: prep, CSC (3), K/V images, dQ, Q/dO images, dK/dV)
-    # (block_select: the tf32 split of q and k, then per round of heads whose logits fit in 96 MiB a score
+    # (block_select: the tf32 split of q and k, then per round of heads whose logits fit in 1 GiB a score
     # GEMM and a selection launch, then the CSR scan; the rounds are counted in launches_per_step)
     LAUNCHES = {"zone_shapes": 4, "block_pool": 1, "block_select": 3, "bsa_fwd": 3, "bsa_bwd": 11}
 
@@ -264,7 +264,7 @@ class Pipeline:
     def select_rounds(self):
         nb = self.geo.counts()[1]
         nbp = (nb + 3) // 4 * 4
-        per_round = max(1, min(self.wl.heads, (96 << 20) // (nb * nbp * 4)))
+        per_round = max(1, min(self.wl.heads, (1024 << 20) // (nb * nbp * 4)))
         return -(-self.wl.heads // per_round)
 
     def launches_per_step(self):

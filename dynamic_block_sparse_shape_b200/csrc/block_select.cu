@@ -18,9 +18,8 @@
 //     slices of the four operand halves come by TMA (128-byte swizzle) into a
 //     two-stage ring, two TMEM accumulators let the epilogue of one tile
 //     overlap the products of the next, and the logits leave as 32 x 32 TMA
-//     box stores (128-byte rows). The chunk's
-//     logits go to the workspace (one head of the 2K grid is 85 MB, which
-//     stays in the 126 MB L2 until the selection reads it).
+//     box stores (128-byte rows) into the workspace, a round of heads at a
+//     time (up to 1 GiB of logits; one head of the 2K grid is 85 MB).
 //   select_rows_kernel: one 128-thread CTA per (head, query block), the row's
 //     entries in registers (thread t holds J = t + 128 i):
 //     1. max of the present logits (a NaN logit marks an absent block: an
@@ -717,12 +716,16 @@ cudaError_t launch_select_rows(int vpt, const float* logits, int nb, int nbp, in
 
 }  // namespace
 
-// Heads whose logits one score/selection round holds: as many as fit in 96 MB (the logits of a
-// round stay in the 126 MB L2 between the two kernels), at least one.
+// Heads whose logits one score/selection round holds: as many as fit in 1 GiB, at least one. A round
+// is one persistent score launch and one row launch over all its heads; at 2K (85 MB of logits per
+// head) rounds of one head cost 0.6 ms more over 24 heads in launch gaps and tails than rounds of 12.
+#ifndef PRISM_SELECT_ROUND_MIB
+#define PRISM_SELECT_ROUND_MIB 1024
+#endif
 int select_chunk_heads(int heads, int nb) {
   const size_t nbp = (size_t(nb) + 3) & ~size_t(3);
   const size_t per_head = size_t(nb) * nbp * sizeof(float);
-  const size_t budget = size_t(96) << 20;
+  const size_t budget = size_t(PRISM_SELECT_ROUND_MIB) << 20;
   return int(std::max<size_t>(1, std::min<size_t>(size_t(heads), budget / per_head)));
 }
 

@@ -229,8 +229,8 @@ PRISM_API prism_status prism_block_pool(const prism_geometry* geo, const int32_t
  * top_k >= n_blocks or cdf_threshold >= 1 keeps every block. The logits are
  * formed on the tensor cores in split tf32 precision (hi.hi + hi.lo + lo.hi,
  * relative error about 2^-20) for a round of heads at a time and held in the
- * workspace (up to 96 MiB, sized to stay in L2) until that round's selection
- * has read them; they are not an output.
+ * workspace (a round of heads whose logits fit in 1 GiB) until that round's
+ * selection has read them; they are not an output.
  *
  * q_pool, k_pool: device float [heads, n_blocks, head_dim]; n_blocks at most
  *       10240 and heads * n_blocks^2 below 2^31 (PRISM_ERR_UNSUPPORTED
@@ -253,7 +253,7 @@ PRISM_API prism_status prism_block_pool(const prism_geometry* geo, const int32_t
  *       head_dim, ...) bytes (equivalently prism_block_select_workspace_size):
  *       the status word, the tf32 halves of q_pool and k_pool (4 * heads *
  *       n_blocks * head_dim floats) and one round's logits (R * n_blocks *
- *       ceil4(n_blocks) floats, R = the heads whose logits fit in 96 MiB, at
+ *       ceil4(n_blocks) floats, R = the heads whose logits fit in 1 GiB, at
  *       least 1).
  */
 PRISM_API prism_status prism_block_select(const float* q_pool, const float* k_pool, int32_t heads, int32_t n_blocks,

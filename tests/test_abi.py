@@ -69,17 +69,17 @@ def test_geometry_counts_and_errors(lib):
 def test_workspace_sizes(lib):
     g = _geo()
     # the status word, the tf32 halves of the pooled q and k (4 x heads x n_blocks x head_dim floats), and the
-    # logits of one round of heads: as many heads as fit in 96 MiB (n_blocks x n_blocks rounded up to 4 floats
+    # logits of one round of heads: as many heads as fit in 1 GiB (n_blocks x n_blocks rounded up to 4 floats
     # each), at least one
     def sel_bytes(heads, nb, d):
         up = lambda x: (x + 255) // 256 * 256
         nbp = (nb + 3) // 4 * 4
         per_head = nb * nbp * 4
-        rounds = max(1, min(heads, (96 << 20) // per_head))
+        rounds = max(1, min(heads, (1024 << 20) // per_head))
         return 256 + 4 * up(heads * nb * d * 4) + up(rounds * nb * nbp * 4)
     assert P.workspace_size("block_select", g) == sel_bytes(1, 4608, 128)
     assert P.workspace_size("block_select", g, heads=24, head_dim=128) == P.select_workspace_size(24, 4608, 128)
-    assert P.select_workspace_size(24, 4608, 128) == sel_bytes(24, 4608, 128)  # one head per round at 2K
+    assert P.select_workspace_size(24, 4608, 128) == sel_bytes(24, 4608, 128)  # 12 heads per round at 2K
     assert P.select_workspace_size(24, 960, 128) == sel_bytes(24, 960, 128)  # every head in one round at 720p
     assert P.select_workspace_size(3, 37, 64) == sel_bytes(3, 37, 64)
     z = P.workspace_size("zone_shapes", g, feat_c=3072, res_c=3072)
