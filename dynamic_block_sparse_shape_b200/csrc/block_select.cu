@@ -629,14 +629,23 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const float* _
   if (tid == 0) *krow = m;
 }
 
-// Exclusive scan of n ints into out[0..n] (out[n] = total), one CTA.
+// Exclusive scan of n ints into out[0..n] (out[n] = total), one CTA: thread t owns a contiguous chunk
+// (a multiple of four entries), summed and rewritten with 16-byte accesses when both buffers are
+// 16-byte aligned, so its loads are in flight together instead of one dependent load per entry.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ in, int n, int32_t* __restrict__ out) {
   __shared__ int64_t part[1024];
   const int tid = threadIdx.x;
-  const int per = (n + 1023) / 1024;
-  const int b = tid * per, e = min(n, b + per);
+  const int per = (((n + 1023) / 1024) + 3) & ~3;
+  const int b = min(n, tid * per), e = min(n, b + per);
+  const bool vec = ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 15u) == 0;
+  const int ev = vec ? b + ((e - b) & ~3) : b;  // [b, ev) in int4 steps, then [ev, e) one by one
   int64_t s = 0;
-  for (int i = b; i < e; ++i) s += in[i];
+#pragma unroll 4
+  for (int i = b; i < ev; i += 4) {
+    const int4 v = *reinterpret_cast<const int4*>(in + i);
+    s += int64_t(v.x) + v.y + v.z + v.w;
+  }
+  for (int i = ev; i < e; ++i) s += in[i];
   part[tid] = s;
   __syncthreads();
   for (int off = 1; off < 1024; off <<= 1) {
@@ -646,7 +655,21 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     __syncthreads();
   }
   int64_t run = part[tid] - s;
-  for (int i = b; i < e; ++i) {
+#pragma unroll 2
+  for (int i = b; i < ev; i += 4) {
+    const int4 v = *reinterpret_cast<const int4*>(in + i);
+    int4 o;
+    o.x = int32_t(run);
+    run += v.x;
+    o.y = int32_t(run);
+    run += v.y;
+    o.z = int32_t(run);
+    run += v.z;
+    o.w = int32_t(run);
+    run += v.w;
+    *reinterpret_cast<int4*>(out + i) = o;
+  }
+  for (int i = ev; i < e; ++i) {
     out[i] = int32_t(run);
     run += in[i];
   }
