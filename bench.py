@@ -747,7 +747,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
     ap.add_argument("--config", default="2k")
-    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--e2e-steps", type=int, default=10,
+                    help="steps streamed through the e2e measurement (the first step's input copy and the last "
+                         "step's result copy are not overlapped with compute)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="run the 45-point selection/sparsity sweep instead")

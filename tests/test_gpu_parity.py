@@ -125,6 +125,30 @@ def test_attention_random_masks_all_shapes(d, density):
     _check_attention(geo, zone_shape, q, k, v, do, mask)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_attention_row_lengths_across_the_short_row_kernel(d):
+    """Rows of every length from 0 to 12 key blocks: the forward sends rows of at
+    most eight blocks (four steps) to its short-row kernel and longer ones to the
+    main kernel, so both run on the same data; the lengths cross the boundary,
+    and odd lengths leave a half step."""
+    grid, zone = (8, 16, 24), (8, 8, 8)
+    geo = P.Geometry(grid, zone, CAND)
+    nz, nb = geo.counts()
+    rng = np.random.default_rng(40 + d)
+    zone_shape = rng.integers(0, len(CAND), nz)
+    H = 2
+    mask = np.zeros((H, nb, nb), dtype=bool)
+    for h in range(H):
+        for i in range(nb):
+            n = (i + 5 * h) % 13  # 0 .. 12 blocks
+            mask[h, i, rng.choice(nb, size=n, replace=False)] = True
+    gen = torch.Generator().manual_seed(70 + d)
+    N = geo.n_tokens
+    dev = torch.device("cuda")
+    q, k, v, do = (torch.randn((N, H, d), generator=gen).to(torch.bfloat16).to(dev) for _ in range(4))
+    _check_attention(geo, zone_shape, q, k, v, do, mask)
+
+
 def test_attention_strided_tokens():
     """Q/K/V/O as views with a token stride larger than heads*head_dim."""
     grid, zone = (8, 8, 16), (8, 8, 8)
