@@ -339,6 +339,23 @@ def test_block_select_ragged_block_count():
         _selection_parity(qp.to(dev), kp.to(dev), 0.125, 3, 0.3, f64(qp), f64(kp))
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("nb,top_k,tau,amp", [(6000, 4, 0.2, 1.0), (7200, 16, 0.05, 3.0), (10240, 1, 0.5, 2.0)])
+def test_block_select_large_block_counts(nb, top_k, tau, amp):
+    """Block counts of the largest grids (7,200 blocks on the 2K latent grid),
+    where each selection thread holds 48, 64 or 80 logits of its row; the last
+    case also has empty blocks (NaN pooled features) spread over the row."""
+    gen = torch.Generator().manual_seed(nb)
+    dev = torch.device("cuda")
+    qp = amp * torch.randn((1, nb, 128), generator=gen)
+    kp = torch.randn((1, nb, 128), generator=gen)
+    if nb == 10240:
+        empty = torch.randperm(nb, generator=gen)[:97]
+        qp[0, empty[:40]] = float("nan")
+        kp[0, empty] = float("nan")
+    _selection_parity(qp.to(dev), kp.to(dev), 1.0 / math.sqrt(128), top_k, tau, f64(qp), f64(kp))
+
+
 def test_block_select_per_head_k_and_tau():
     """Per-head floors and thresholds (the ratio form gives the floors of two heads)."""
     wl, _, _, _, _, qp, kp, qpr, kpr = _pooled_720p(heads=4)
