@@ -87,8 +87,8 @@ _SIGNATURES = {
     "prism_block_select_workspace_size": (ctypes.c_int, [_I32, _I32, _I32, ctypes.POINTER(_SZ)]),
     "prism_block_audio_bias": (ctypes.c_int, [_GEO, _P, _P, _I64, _I32, ctypes.c_int, _F32, _P, _P, _SZ, _P]),
     "prism_mask_to_csr": (ctypes.c_int, [_P, _P, _I32, _I32, _P, _I64, _P, _SZ, _P]),
-    "prism_bsa_fwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32, _P, _P, _P, _P,
-                                     _P, _P, _SZ, _P]),
+    "prism_bsa_fwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32, _P, _P, _I64, _P,
+                                     _P, _P, _P, _SZ, _P]),
     "prism_bsa_bwd": (ctypes.c_int, [_GEO, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I64, _F32,
                                      _P, _P, _I64, _P, _P, _P, _P, _SZ, _P]),
 }
@@ -370,11 +370,13 @@ def mask_to_csr(mask: torch.Tensor, row_ptr: torch.Tensor, n_blocks: int, col_id
 
 def bsa_fwd(geo: Geometry, zone_shape, q, k, v, scale, row_ptr, col_idx, ws: Optional[Workspace] = None,
             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, stream=None,
-            o_lo: Optional[torch.Tensor] = None):
+            o_lo: Optional[torch.Tensor] = None, nnz: Optional[int] = None):
     """a6: block-sparse attention forward. Returns (O like q, LSE fp32 [H, N]).
 
     o_lo (optional, bf16 like a bf16 q): receives the rounding residual of O,
-    to be passed to bsa_bwd so that D = dO . O is formed from O to ~16 bits."""
+    to be passed to bsa_bwd so that D = dO . O is formed from O to ~16 bits.
+    nnz (optional): the selection's total kept pairs; it chooses the kernels'
+    plan (rows short on average: no block images), not the result."""
     N, H, d = q.shape
     assert q.stride(2) == 1 and q.stride(1) == d and k.stride() == q.stride() and v.stride() == q.stride()
     need = workspace_size("bsa_fwd", geo, heads=H, head_dim=d, dtype=q.dtype)
@@ -386,7 +388,8 @@ def bsa_fwd(geo: Geometry, zone_shape, q, k, v, scale, row_ptr, col_idx, ws: Opt
         assert o_lo.dtype == torch.bfloat16 and o_lo.stride() == q.stride()
     g = geo.c()
     _check(lib().prism_bsa_fwd(ctypes.byref(g), _ptr(zone_shape), _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), H, d,
-                               q.stride(0), float(scale), _ptr(row_ptr), _ptr(col_idx), _ptr(o), _ptr(lse_t),
+                               q.stride(0), float(scale), _ptr(row_ptr), _ptr(col_idx),
+                               -1 if nnz is None else int(nnz), _ptr(o), _ptr(lse_t),
                                _ptr(o_lo), ws.ptr, ws.nbytes, _stream(stream)), "prism_bsa_fwd")
     return o, lse_t
 

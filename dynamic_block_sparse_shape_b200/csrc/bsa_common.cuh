@@ -128,16 +128,34 @@ __device__ __forceinline__ void mask_scores32(uint32_t* r, uint32_t members) {
 // Entries of the block-id ring below.
 constexpr int kDescRing = 64;
 
+// Where a block's 5-D tensor-map box starts, with its candidate shape:
+// {shape, t0, h0, w0}.
+__device__ __forceinline__ int4 block_box_coords(const Geo& g, const int32_t* zone_shape, int b, int* status) {
+  int s = __ldg(zone_shape + b / g.bpz);
+  if (s < 0 || s >= g.n_cand) {
+    atomicOr(status, kDevErrBounds);
+    s = 0;
+  }
+  const BlockBox bb = block_box(g, s, b);
+  return make_int4(s, bb.t0, bb.h0, bb.w0);
+}
+
 // Block ids named by a CSR / CSC list, read 32 at a time by a whole warp
 // (coalesced list reads) into a shared-memory ring, so the thread that issues
 // the copies never waits on a dependent global load. Entry e of a list of
 // `cnt` blocks processed `step` (a power of two) per step: e < cnt is the
 // list's e-th block; a ragged tail (e >= cnt in the last step) repeats the
-// step's first block. An id out of range is reported and replaced by 0.
+// step's first block. An id out of range is reported and replaced by 0. With
+// `boxes` set, the same warp-wide pass also looks up each block's zone shape
+// and box origin (block_box_coords), so the thread that issues tensor-map
+// copies of the blocks has neither a dependent load nor the box arithmetic on
+// its path.
 struct IdCache {
   int* ring;  // shared memory, kDescRing entries
   int filled;
   int step = 2;
+  int4* boxes = nullptr;                // shared memory, kDescRing entries, or null
+  const int32_t* zone_shape = nullptr;  // with boxes
   // Makes entries [0, e] available; the whole warp must call it.
   __device__ __forceinline__ void ensure(int e, const Geo& g, const int32_t* list, int beg, int cnt, int* status,
                                          int lane) {
@@ -151,11 +169,13 @@ struct IdCache {
         J = 0;
       }
       ring[ee % kDescRing] = J;
+      if (boxes) boxes[ee % kDescRing] = block_box_coords(g, zone_shape, J, status);
       __syncwarp();
       filled += 32;
     }
   }
   __device__ __forceinline__ int get(int e) const { return ring[e % kDescRing]; }
+  __device__ __forceinline__ int4 box(int e) const { return boxes[e % kDescRing]; }
 };
 
 // Byte offset of the operand image of (head, block) in a block-major image

@@ -67,11 +67,16 @@ constexpr int kFwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kPvWarp = 2 + kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kSmallSteps = 4;  // rows of up to 8 key blocks go to bsa_fwd_small_kernel
+// With at most this many selected key blocks per row on average the short-row
+// kernel takes every row (the sparse plan)
+constexpr int kSparseBlocksPerRow = 8;
 
 struct FwdParams {
   CUtensorMap mq[kMaxCand];
   CUtensorMap mo[kMaxCand];   // O and its rounding residual, for bf16 outputs:
   CUtensorMap mol[kMaxCand];  // the epilogue stores a block's rows with 5-D box copies
+  CUtensorMap mk[kMaxCand];   // K and V, for the short-row kernel when it takes every row
+  CUtensorMap mv[kMaxCand];
   const uint8_t* kimg;  // block images of K and V (layout in host.h)
   const uint8_t* vimg;
   Geo g;
@@ -87,6 +92,7 @@ struct FwdParams {
   int out_fp32;
   int tma_out;  // bf16 output: stores through the O / o_lo tensor maps
   int heads;
+  int all_rows;  // the short-row kernel takes every row, K and V through mk / mv (no block images)
 };
 
 template <int D>
@@ -537,21 +543,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1) bsa_fwd_kernel(const __grid_co
 
 // ---------------------------------------------------------------- short rows
 // Rows of at most kSmallSteps steps (and empty rows) go to a second kernel
-// whose CTA needs a quarter of the tensor memory and 83 KB of shared memory,
-// so two CTAs share an SM and each one's fixed latencies (launch, the Q and
-// first K/V copies, the epilogue) overlap the other's work. A row of a few
-// key blocks is mostly fixed cost: on the 2K grid one CTA of bsa_fwd_kernel
-// spends about 7 us per row before and after its 0.5 us steps. Long rows stay
-// with bsa_fwd_kernel, which returns at once for the short ones.
-//   warp 0      copies: Q once (5-D TMA), per step K and V of the step's two
-//               key blocks into one K and one V slot (bulk copies of images);
+// whose CTA needs half of the tensor memory and about 100 KB of shared
+// memory, so two CTAs share an SM. A row of a few key blocks is mostly fixed
+// cost: copy latencies and the epilogue. Each CTA loops over the rows of its
+// stride and pipelines them: the copies of the next row (its Q, then its first
+// K and V) start as soon as the current row frees their buffers, and the next
+// row's first score product runs while the softmax warps finish the current
+// row's epilogue. Long rows stay with bsa_fwd_kernel, which returns at once
+// for the short ones. With `all_rows` set (the host's plan when the rows are
+// short on average) this kernel takes every row and gathers K and V through
+// 5-D tensor maps: no block images are made and bsa_fwd_kernel is not
+// launched.
+//   warp 0      copies: per row Q (5-D TMA) into one staging tile, free again
+//               once the softmax warps have moved Q into TMEM; per step K and
+//               V of the step's two key blocks into one K and one V slot;
 //   warp 1      TMEM owner, issues S_j = Q [K_j0 K_j1]^T and then
 //               O += P_j [V_j0 | V_j1] (.ws M=64; Q and P from TMEM), one
 //               step at a time: P_j is written over S_j's first 32 columns,
-//               so S_{j+1} waits for PV_j;
+//               so S_{j+1} waits for PV_j, and a row's first PV waits until
+//               the epilogue has read the previous row's O;
 //   warps 2..5  softmax, one thread per TMEM lane (row m of the block,
 //               key-block half kh of the step), running max and sum per
-//               lane half, merged in the epilogue.
+//               lane half, merged in the epilogue; between a row's last step
+//               and its epilogue they move the next row's Q into TMEM.
+// Barrier phases run on across rows: the copies, products and arrivals of the
+// CTA's s-th step complete phase s of their barriers, and the row barriers
+// (Q staged, Q in TMEM, O read) count the CTA's rows with work. Every wait is
+// placed so that the phase after the awaited one needs a step the waiter has
+// not yet enabled.
 constexpr int kSmallThreads = 64 + 128;
 
 template <int D>
@@ -563,12 +582,18 @@ struct FwdSmallSmem {
   static constexpr uint32_t kV = kK + kSlotBytes;        // [block][dh][64][128 B]
   static constexpr uint32_t kRed = kV + kSlotBytes;      // per lane half: running max, sum [2][64] each
   static constexpr uint32_t kRedBytes = 2 * 2 * 64 * 4;
-  static constexpr uint32_t kDesc = kRed + kRedBytes;  // block-id ring
+  // epilogue exchange of half rows in rounds of kXC channels, [lane half][64 rows][kXC + 4 floats];
+  // then the staging tile of a bf16 output block ([dh][64][128 B], swizzled) for its box stores
+  static constexpr int kXC = 32;
+  static constexpr uint32_t kXPitch = kXC + 4;
+  static constexpr uint32_t kX = kRed + kRedBytes;
+  static constexpr uint32_t kXBytes = 2 * 64 * kXPitch * 4;
+  static_assert(kX % 1024 == 0 && kXBytes >= D * 128, "the exchange buffer holds one swizzled output tile");
+  static constexpr uint32_t kBox = kX + kXBytes;  // box origins of the ring's blocks (5-D copies)
+  static constexpr uint32_t kDesc = kBox + kDescRing * 16;  // block-id ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 128;
-  // epilogue exchange of half rows: [lane half][64 rows][D/2 + 4 floats], over the K and V slots
-  static constexpr uint32_t kXPitch = D / 2 + 4;
-  static_assert(2 * 64 * kXPitch * 4 <= 2 * kSlotBytes, "exchange buffer fits the slots");
+  static_assert(2 * (kTotal + 2048) <= 228 * 1024, "two CTAs per SM");
   // TMEM: S (P over its first 32 columns) at 0, the O parts at 64 (D columns), Q at 64 + D (D/2)
   static constexpr uint32_t kTmemCols = 256;
   static constexpr uint32_t kTO = 64;
@@ -577,10 +602,10 @@ struct FwdSmallSmem {
 };
 
 // Output rows of an empty query block: O = 0 (and its residual), LSE = -inf.
+// tid: 0..127.
 template <int D>
 __device__ __forceinline__ void write_empty_row(const FwdParams& P, int I, int head, int tid) {
   const Geo& g = P.g;
-  if (tid >= 128) return;
   const int m = tid & 63, half = tid >> 6;
   int* status = P.status;
   const int sI = safe_shape(g, P.zone_shape, I, status);
@@ -597,28 +622,80 @@ __device__ __forceinline__ void write_empty_row(const FwdParams& P, int I, int h
   if (half == 0) P.lse[int64_t(head) * g.T * g.H * g.W + tok] = -INFINITY;
 }
 
+// List of row `row`: its first entry and its length (a malformed length is
+// reported and read as 0).
+__device__ __forceinline__ int row_list(const FwdParams& P, int row, int* beg) {
+  const int b = __ldg(P.row_ptr + row);
+  int cnt = __ldg(P.row_ptr + row + 1) - b;
+  if (cnt < 0 || cnt > P.g.n_blocks) {
+    atomicOr(P.status, kDevErrBounds);
+    cnt = 0;
+  }
+  *beg = b;
+  return cnt;
+}
+
+// Whether the short-row kernel computes a row of `nsteps` > 0 steps.
+__device__ __forceinline__ bool small_takes(const FwdParams& P, int nsteps) {
+  return P.all_rows || nsteps <= kSmallSteps;
+}
+
+// Copies one key block's K (or V) tile for the short-row kernel: from its block
+// image, or (all_rows) through the 5-D tensor map of its shape, from the box
+// origin {shape, t0, h0, w0} cached with its id. K tiles are laid out
+// [dh][block][64][128 B] (dst = slot base), V tiles [block][dh][64][128 B].
+template <int D>
+__device__ __forceinline__ void small_load_kv(const FwdParams& P, bool is_v, uint8_t* slot, int kb_slot, int head,
+                                              int J, int4 box, uint64_t* bar) {
+  const Geo& g = P.g;
+  if (P.all_rows) {
+    const CUtensorMap* map = is_v ? &P.mv[box.x] : &P.mk[box.x];
+    for (int dh = 0; dh < D / 64; ++dh) {
+      const uint32_t off = is_v ? kb_slot * (D * 128) + dh * kBoxBytes : dh * (kKB * kBoxBytes) + kb_slot * kBoxBytes;
+      tma_load_5d(slot + off, map, bar, dh * 64, head, box.w, box.z, box.y);
+    }
+  } else {
+    const uint8_t* src = (is_v ? P.vimg : P.kimg) + image_offset(g, head, J, D);
+    if (is_v) {
+      bulk_load(slot + kb_slot * (D * 128), src, D * 128, bar);
+    } else {
+      for (int dh = 0; dh < D / 64; ++dh)
+        bulk_load(slot + dh * (kKB * kBoxBytes) + kb_slot * kBoxBytes, src + dh * kBoxBytes, kBoxBytes, bar);
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const __grid_constant__ FwdParams P) {
   using L = FwdSmallSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
-  uint64_t* q_full = bars + 0;
-  uint64_t* qa_full = bars + 1;   // Q copied into TMEM by the softmax warps
-  uint64_t* k_full = bars + 2;    // K of the step landed
-  uint64_t* k_free = bars + 3;    // S of the step complete (K slot free)
-  uint64_t* v_full = bars + 4;    // V of the step landed
-  uint64_t* s_full = bars + 5;    // S of the step complete
-  uint64_t* p_full = bars + 6;    // P of the step written (4 warps)
-  uint64_t* pv_done = bars + 7;   // PV of the step complete (V slot and S / P columns free)
-  uint64_t* mma_done = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
+  uint64_t* q_full = bars + 0;   // Q of the row staged
+  uint64_t* qa_full = bars + 1;  // Q of the row in TMEM, staging tile free (4 warps)
+  uint64_t* k_full = bars + 2;   // K of the step landed
+  uint64_t* k_free = bars + 3;   // S of the step complete (K slot free)
+  uint64_t* v_full = bars + 4;   // V of the step landed
+  uint64_t* s_full = bars + 5;   // S of the step complete
+  uint64_t* p_full = bars + 6;   // P of the step written (4 warps)
+  uint64_t* pv_done = bars + 7;  // PV of the step complete (V slot and S / P columns free)
+  uint64_t* o_free = bars + 8;   // O of the row read by the epilogue (4 warps)
+  uint64_t* mma_done = bars + 9;
+  uint64_t* stage_free = bars + 10;  // the rounding-residual tile of the row, staged over Q, read
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
   float* redm = reinterpret_cast<float*>(sm + L::kRed);
   float* redl = redm + 2 * 64;
+  float* X = reinterpret_cast<float*>(sm + L::kX);
   const Geo& g = P.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* status = P.status;
+  const int rows = P.heads * g.n_blocks;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 1 || i == 6 || i == 8) ? 4 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
@@ -628,130 +705,181 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t tO = tbase + L::kTO, tQ = tbase + L::kTQ;
-  bool first = true;
-  // CTA b takes rows b, b + grid, ... (row = head * n_blocks + query block), the short and empty ones
-  for (int row = blockIdx.x; row < P.heads * g.n_blocks; row += gridDim.x) {
-    const int I = row % g.n_blocks, head = row / g.n_blocks;
-    const int beg = P.row_ptr[row];
-    int cnt = P.row_ptr[row + 1] - beg;
-    if (cnt < 0 || cnt > g.n_blocks) {
-      if (threadIdx.x == 0) atomicOr(status, kDevErrBounds);
-      cnt = 0;
-    }
-    const int nsteps = (cnt + kKB - 1) / kKB;
-    if (nsteps > kSmallSteps) continue;  // a long row: bsa_fwd_kernel's (uniform)
-    if (nsteps == 0) {
-      write_empty_row<D>(P, I, head, threadIdx.x);
-      continue;
-    }
-    if (threadIdx.x == 0) {
-      // the previous row left no copy, product or arrival pending on any barrier
-      if (!first)
-        for (int i = 0; i < 9; ++i) mbar_inval(&bars[i]);
-      for (int i = 0; i < 9; ++i) mbar_init(&bars[i], (i == 1 || i == 6) ? 4 : 1);
-      *abort_flag = 0;
-      fence_barrier_init();
-    }
-    first = false;
-    __syncthreads();
 
-    if (warp == 0) {
-      // ------------------------------------------------------------ producer
-      IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
+  // CTA b takes rows b, b + grid, ... (row = head * n_blocks + query block);
+  // every role walks the same sequence and skips the same rows
+  // bf16 output with a rounding residual: the residual tile is staged over the Q tile
+  const bool stage_lo = P.tma_out && P.o_lo;
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
+    if (P.all_rows) {
+      dc.boxes = reinterpret_cast<int4*>(sm + L::kBox);
+      dc.zone_shape = P.zone_shape;
+    }
+    bool ok = true;
+    int lq = 0, gs = 0, q_iss = 0, k_iss = 0, v_iss = 0;
+    for (int row = blockIdx.x; row < rows && ok; row += gridDim.x) {
+      int beg;
+      const int cnt = row_list(P, row, &beg);
+      const int nsteps = (cnt + kKB - 1) / kKB;
+      if (nsteps == 0 || !small_takes(P, nsteps)) continue;
+      const int I = row % g.n_blocks, head = row / g.n_blocks;
       if (lane == 0) {
-        const int sI = safe_shape(g, P.zone_shape, I, status);
-        const BlockBox qb = block_box(g, sI, I);
-        mbar_arrive_expect_tx(q_full, L::kQBytes);
-        for (int dh = 0; dh < D / 64; ++dh)
-          tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], q_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+        // the staging tile held the previous row's Q until it reached TMEM,
+        // then (bf16 output with a residual) the rounding residual of row lq - 2
+        // until its box stores read it
+        if (lq > 0) ok = mbar_wait_abortable(qa_full, (lq - 1) & 1, status, abort_flag);
+        if (ok && lq > 1 && stage_lo)
+          ok = mbar_wait_abortable(stage_free, (lq - 2) & 1, status, abort_flag);
+        if (ok) {
+          const int sI = safe_shape(g, P.zone_shape, I, status);
+          const BlockBox qb = block_box(g, sI, I);
+          mbar_arrive_expect_tx(q_full, L::kQBytes);
+          for (int dh = 0; dh < D / 64; ++dh)
+            tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], q_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+          q_iss = lq + 1;
+        }
       }
-      bool ok = true;
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < nsteps && ok; ++j) {
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      dc.filled = 0;
+      for (int j = 0; j < nsteps && ok; ++j, ++gs) {
         dc.ensure(kKB * j + kKB - 1, g, P.col_idx, beg, cnt, status, lane);
         if (lane == 0) {
-          // the K slot last held step j - 1: free once S_{j-1} completed
-          if (j > 0) ok = mbar_wait_abortable(k_free, (j - 1) & 1, status, abort_flag);
+          // the K slot last held step gs - 1: free once its S completed
+          if (gs > 0) ok = mbar_wait_abortable(k_free, (gs - 1) & 1, status, abort_flag);
           if (ok) {
             mbar_arrive_expect_tx(k_full, L::kSlotBytes);
-            for (int slot = 0; slot < kKB; ++slot) {
-              const uint8_t* src = P.kimg + image_offset(g, head, dc.get(kKB * j + slot), D);
-              for (int dh = 0; dh < D / 64; ++dh)
-                bulk_load(sm + L::kK + dh * (kKB * kBoxBytes) + slot * kBoxBytes, src + dh * kBoxBytes, kBoxBytes,
-                          k_full);
-            }
-            k_issued = j + 1;
+            for (int slot = 0; slot < kKB; ++slot)
+              small_load_kv<D>(P, false, sm + L::kK, slot, head, dc.get(kKB * j + slot),
+                               P.all_rows ? dc.box(kKB * j + slot) : int4{}, k_full);
+            k_iss = gs + 1;
           }
-          // the V slot last held step j - 1: free once PV_{j-1} completed
-          if (ok && j > 0) ok = mbar_wait_abortable(pv_done, (j - 1) & 1, status, abort_flag);
+          // the V slot last held step gs - 1: free once its PV completed
+          if (ok && gs > 0) ok = mbar_wait_abortable(pv_done, (gs - 1) & 1, status, abort_flag);
           if (ok) {
             mbar_arrive_expect_tx(v_full, L::kSlotBytes);
             for (int slot = 0; slot < kKB; ++slot)
-              bulk_load(sm + L::kV + slot * (D * 128), P.vimg + image_offset(g, head, dc.get(kKB * j + slot), D),
-                        D * 128, v_full);
-            v_issued = j + 1;
+              small_load_kv<D>(P, true, sm + L::kV, slot, head, dc.get(kKB * j + slot),
+                               P.all_rows ? dc.box(kKB * j + slot) : int4{}, v_full);
+            v_iss = gs + 1;
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       }
-      if (lane == 0) {
-        // drain: every issued copy has landed before the CTA may exit (one slot each: the last)
-        mbar_wait(q_full, 0, status);
-        if (k_issued > 0) mbar_wait(k_full, (k_issued - 1) & 1, status);
-        if (v_issued > 0) mbar_wait(v_full, (v_issued - 1) & 1, status);
-      }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ issuer
-      if (lane == 0) {
-        const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
-        const uint64_t dK = sdesc_sw128(smem_u32(sm + L::kK), 16, 1024);
-        // B = V of the step, MN-major, N = 2d: the d channels of key block 0, then those of key block 1
-        const uint32_t idO = idesc_bf16_f32(64, 2 * D, false, true);
-        const uint64_t dV = sdesc_sw128(smem_u32(sm + L::kV), kBoxBytes, 1024);
-        bool ok = mbar_wait_abortable(qa_full, 0, status, abort_flag);
-        for (int j = 0; j < nsteps && ok; ++j) {
-          // K of step j landed; PV_{j-1} (which read P from the S columns) complete
-          ok = mbar_wait_abortable(k_full, j & 1, status, abort_flag) &&
-               (j == 0 || mbar_wait_abortable(pv_done, (j - 1) & 1, status, abort_flag));
+      ++lq;
+    }
+    if (lane == 0) {
+      // drain: every issued copy has landed before the CTA may exit (one buffer each: the last)
+      if (q_iss > 0) mbar_wait(q_full, (q_iss - 1) & 1, status);
+      if (k_iss > 0) mbar_wait(k_full, (k_iss - 1) & 1, status);
+      if (v_iss > 0) mbar_wait(v_full, (v_iss - 1) & 1, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
+      const uint64_t dK = sdesc_sw128(smem_u32(sm + L::kK), 16, 1024);
+      // B = V of the step, MN-major, N = 2d: the d channels of key block 0, then those of key block 1
+      const uint32_t idO = idesc_bf16_f32(64, 2 * D, false, true);
+      const uint64_t dV = sdesc_sw128(smem_u32(sm + L::kV), kBoxBytes, 1024);
+      bool ok = true;
+      int lq = 0, gs = 0;
+      for (int row = blockIdx.x; row < rows && ok; row += gridDim.x) {
+        int beg;
+        const int cnt = row_list(P, row, &beg);
+        const int nsteps = (cnt + kKB - 1) / kKB;
+        if (nsteps == 0 || !small_takes(P, nsteps)) continue;
+        // Q of the row in TMEM
+        ok = mbar_wait_abortable(qa_full, lq & 1, status, abort_flag);
+        for (int j = 0; j < nsteps && ok; ++j, ++gs) {
+          // K of the step landed; PV of the previous step (which read P from the S columns) complete
+          ok = mbar_wait_abortable(k_full, gs & 1, status, abort_flag) &&
+               (gs == 0 || mbar_wait_abortable(pv_done, (gs - 1) & 1, status, abort_flag));
           if (!ok) break;
           tc_fence_after();
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ws_ts(tbase, tQ + kk * 8, dK + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
           mma_commit(s_full);
           mma_commit(k_free);
-          ok = mbar_wait_abortable(p_full, j & 1, status, abort_flag) &&
-               mbar_wait_abortable(v_full, j & 1, status, abort_flag);
+          // P written, V landed, and before a row's first PV the previous row's O read
+          ok = mbar_wait_abortable(p_full, gs & 1, status, abort_flag) &&
+               mbar_wait_abortable(v_full, gs & 1, status, abort_flag) &&
+               (j > 0 || lq == 0 || mbar_wait_abortable(o_free, (lq - 1) & 1, status, abort_flag));
           if (!ok) break;
           tc_fence_after();
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ws_ts(tO, tbase + kk * 8, dV + uint64_t((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(pv_done);
         }
-        // every product this thread issued has completed before TMEM is released
-        mma_commit(mma_done);
-        mbar_wait(mma_done, 0, status);
+        ++lq;
       }
-    } else {
-      // ------------------------------------------------------------ softmax
-      const int sp = warp & 3;  // TMEM lane quarter of this warp
-      const int Ln = sp * 32 + lane;
-      const int m = Ln & 63, kh = Ln >> 6;
-      const uint32_t lane_off = uint32_t(sp * 32) << 16;
-      float m_run = -INFINITY, l_run = 0.f;
-      // Q becomes the A operand of every S product: both column halves of this lane's row
-      mbar_wait_abortable(q_full, 0, status, abort_flag);
+      // every product this thread issued has completed before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, status);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    // The four warps run the same control flow whatever their waits return
+    // (after a timeout the waits give up at once and the values are
+    // discarded), so their named barriers always match.
+    const int sp = warp & 3;  // TMEM lane quarter of this warp
+    const int Ln = sp * 32 + lane;
+    const int m = Ln & 63, kh = Ln >> 6;
+    const uint32_t lane_off = uint32_t(sp * 32) << 16;
+    const int tid = threadIdx.x - 64;
+    // the next row of the stride with work from `r` on; empty rows on the way
+    // get their outputs. (b0, b1): row_ptr[r], row_ptr[r + 1], read in advance
+    auto seek = [&](int r, int b0, int b1, int& beg, int& cnt, int& nsteps) -> int {
+      for (bool first = true; r < rows; r += gridDim.x, first = false) {
+        if (first) {
+          beg = b0;
+          cnt = b1 - b0;
+          if (cnt < 0 || cnt > g.n_blocks) {
+            atomicOr(status, kDevErrBounds);
+            cnt = 0;
+          }
+        } else {
+          cnt = row_list(P, r, &beg);
+        }
+        nsteps = (cnt + kKB - 1) / kKB;
+        if (nsteps == 0) {
+          write_empty_row<D>(P, r % g.n_blocks, r / g.n_blocks, tid);
+          continue;
+        }
+        if (small_takes(P, nsteps)) return r;
+      }
+      return rows;
+    };
+    // Q becomes the A operand of every S product of its row: both column halves of this lane's row
+    auto q_to_tmem = [&](int lq) {
+      mbar_wait_abortable(q_full, lq & 1, status, abort_flag);
       tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, 0);
       tile_to_tmem_a<D>(sm + L::kQ, tQ + lane_off, m, 1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(qa_full);
-      for (int j = 0; j < nsteps; ++j) {
+    };
+    int beg = 0, cnt = 0, nsteps = 0;
+    int row = blockIdx.x < rows ? seek(blockIdx.x, __ldg(P.row_ptr + blockIdx.x), __ldg(P.row_ptr + blockIdx.x + 1),
+                                       beg, cnt, nsteps)
+                                : rows;
+    if (row < rows) q_to_tmem(0);
+    int lq = 0, gs = 0;
+    while (row < rows) {
+      const int I = row % g.n_blocks, head = row / g.n_blocks;
+      const int sI = safe_shape(g, P.zone_shape, I, status);  // read now, used in the epilogue
+      // the list bounds of the next row of the stride, read now, used after the steps
+      const int pr = row + gridDim.x;
+      const int pb0 = pr < rows ? __ldg(P.row_ptr + pr) : 0, pb1 = pr < rows ? __ldg(P.row_ptr + pr + 1) : 0;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < nsteps; ++j, ++gs) {
         const bool valid = (j * kKB + kh) < cnt;  // warp-uniform: kh is fixed per warp
         uint64_t members = ~uint64_t(0);
         if (g.partial && valid) members = key_block_members(g, P.zone_shape, __ldg(P.col_idx + beg + j * kKB + kh));
-        mbar_wait_abortable(s_full, j & 1, status, abort_flag);
+        mbar_wait_abortable(s_full, gs & 1, status, abort_flag);
         tc_fence_after();
         uint32_t r[64];
         tmem_ld32(tbase + lane_off, r);
@@ -769,14 +897,14 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
             m_run = m_new;
           }
           if (j > 0) {
-            // O holds PV_{j-1}, complete: S_j was issued after it
-  #pragma unroll
+            // O holds the row's PV of the previous step, complete: this S was issued after it
+#pragma unroll
             for (int h = 0; h < D / 32; ++h) {
               uint32_t o[32];
               const uint32_t ta = tO + lane_off + h * 32;
               tmem_ld32(ta, o);
               tmem_ld_wait();
-  #pragma unroll
+#pragma unroll
               for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
               tmem_st16(ta, o);
               tmem_st16(ta + 16, o + 16);
@@ -788,7 +916,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
         if (valid) {
           const float c = P.scale_log2, nm = m_run == -INFINITY ? 0.f : -m_run;
           float la = 0.f, lb = 0.f;
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float p0 = fast_exp2(fmaf(__uint_as_float(r[2 * i]), c, nm));
             const float p1 = fast_exp2(fmaf(__uint_as_float(r[2 * i + 1]), c, nm));
@@ -798,7 +926,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
           }
           l_run += la + lb;
         } else {
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 32; ++i) pk[i] = 0u;
         }
         // P over the first 32 columns of S (every S value of this lane was read above)
@@ -809,76 +937,133 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
       }
+      // every S product of this row has completed: the next row's Q may take the Q columns
+      int nbeg = 0, ncnt = 0, nns = 0;
+      const int nrow = seek(pr, pb0, pb1, nbeg, ncnt, nns);
+      if (nrow < rows) q_to_tmem(lq + 1);
       // ---------------------------------------------------------- epilogue
-      mbar_wait_abortable(pv_done, (nsteps - 1) & 1, status, abort_flag);
+      mbar_wait_abortable(pv_done, (gs - 1) & 1, status, abort_flag);
       tc_fence_after();
       redm[kh * 64 + m] = m_run;
       redl[kh * 64 + m] = l_run;
+      // the previous row's output tile has left the exchange buffer
+      if (P.tma_out && tid == 0) bulk_wait_group_read0();
       named_bar_sync(1, 128);
-      const bool ok = *abort_flag == 0;  // uniform: read after the barrier
+      const bool ok = *abort_flag == 0;
       const float M = fmaxf(redm[m], redm[64 + m]);
       float Lsum = 0.f;
-  #pragma unroll
+#pragma unroll
       for (int q = 0; q < 2; ++q) {
-        const float lq = redl[q * 64 + m];
-        if (lq > 0.f) Lsum += lq * fast_exp2(redm[q * 64 + m] - M);
+        const float lq2 = redl[q * 64 + m];
+        if (lq2 > 0.f) Lsum += lq2 * fast_exp2(redm[q * 64 + m] - M);
       }
       const float inv = (Lsum > 0.f && ok) ? 1.f / Lsum : 0.f;
       const float w = l_run > 0.f ? fast_exp2(m_run - M) * inv : 0.f;  // weight of this lane's part
-      // this thread keeps channel half kh of row m and hands half kh ^ 1 to the other lane half
+      // this thread keeps channel half kh of row m and hands half kh ^ 1 to the
+      // other lane half, kXC channels per round
       constexpr int NC = D / 2;
-      float* X = reinterpret_cast<float*>(sm + L::kK);
       float ov[NC];
-      {
-        float gv[32];
-  #pragma unroll
-        for (int h = 0; h < NC / 32; ++h) {
-          tmem_ld_f<32>(tO + lane_off + (kh ^ 1) * NC + h * 32, gv);
-          float* xo = X + ((kh ^ 1) * 64 + m) * L::kXPitch + h * 32;
-  #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(xo)[i] =
-                make_float4(gv[4 * i] * w, gv[4 * i + 1] * w, gv[4 * i + 2] * w, gv[4 * i + 3] * w);
-          tmem_ld_f<32>(tO + lane_off + kh * NC + h * 32, ov + h * 32);
+#pragma unroll
+      for (int c0 = 0; c0 < NC; c0 += L::kXC) {
+        float gv[L::kXC];
+        tmem_ld_f<L::kXC>(tO + lane_off + (kh ^ 1) * NC + c0, gv);
+        tmem_ld_f<L::kXC>(tO + lane_off + kh * NC + c0, ov + c0);
+        if (c0 + L::kXC == NC) {
+          // this warp's last read of O: the next row's first PV may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
         }
+        float* xo = X + ((kh ^ 1) * 64 + m) * L::kXPitch;
+#pragma unroll
+        for (int i = 0; i < L::kXC / 4; ++i)
+          reinterpret_cast<float4*>(xo)[i] =
+              make_float4(gv[4 * i] * w, gv[4 * i + 1] * w, gv[4 * i + 2] * w, gv[4 * i + 3] * w);
+        named_bar_sync(1, 128);
+        const float* xi = X + (kh * 64 + m) * L::kXPitch;
+#pragma unroll
+        for (int i = 0; i < L::kXC / 4; ++i) {
+          const float4 t = reinterpret_cast<const float4*>(xi)[i];
+          ov[c0 + 4 * i] = fmaf(ov[c0 + 4 * i], w, t.x);
+          ov[c0 + 4 * i + 1] = fmaf(ov[c0 + 4 * i + 1], w, t.y);
+          ov[c0 + 4 * i + 2] = fmaf(ov[c0 + 4 * i + 2], w, t.z);
+          ov[c0 + 4 * i + 3] = fmaf(ov[c0 + 4 * i + 3], w, t.w);
+        }
+        named_bar_sync(1, 128);  // the exchange buffer is free for the next round (and row)
       }
-      named_bar_sync(1, 128);
-      const float* xi = X + (kh * 64 + m) * L::kXPitch;
-  #pragma unroll
-      for (int i = 0; i < NC / 4; ++i) {
-        const float4 t = reinterpret_cast<const float4*>(xi)[i];
-        ov[4 * i] = fmaf(ov[4 * i], w, t.x);
-        ov[4 * i + 1] = fmaf(ov[4 * i + 1], w, t.y);
-        ov[4 * i + 2] = fmaf(ov[4 * i + 2], w, t.z);
-        ov[4 * i + 3] = fmaf(ov[4 * i + 3], w, t.w);
-      }
-  #pragma unroll
+#pragma unroll
       for (int i = 0; i < NC; ++i) ov[i] = inv == 0.f ? 0.f : ov[i];
-      const int sI = safe_shape(g, P.zone_shape, I, status);
       const BlockBox qb = block_box(g, sI, I);
       const int tok = block_token(g, qb, m);
       const bool row_in = !g.partial || block_slot_in_grid(g, qb, m);
-      if (row_in) {
+      if (P.tma_out) {
+        // bf16 rows of the block into swizzled [dh][64][128 B] tiles, O over
+        // the exchange buffer and its rounding residual over the Q tile (free:
+        // the next row's Q is in TMEM, and the copy warp stages the row after
+        // it only once these box stores have read the tile), then one box
+        // store per 64 channels and tile (rows outside the grid fall outside
+        // the tensor and are not written)
+        const int dh = (kh * NC) / 64, c0 = ((kh * NC) % 64) / 8;
+#pragma unroll
+        for (int q = 0; q < NC / 8; ++q) {
+          const uint32_t so = dh * kBoxBytes + sw128_offset(m, c0 + q);
+          const float* x = ov + 8 * q;
+          *reinterpret_cast<uint4*>(sm + L::kX + so) =
+              make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                         pack_bf16x2(x[6], x[7]));
+          if (stage_lo) {
+            float t[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t[i] = x[i] - __bfloat162float(__float2bfloat16_rn(x[i]));
+            *reinterpret_cast<uint4*>(sm + L::kQ + so) =
+                make_uint4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]), pack_bf16x2(t[4], t[5]),
+                           pack_bf16x2(t[6], t[7]));
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (tid == 0) {
+          for (int h = 0; h < D / 64; ++h) {
+            tma_store_5d(&P.mo[sI], sm + L::kX + h * kBoxBytes, h * 64, head, qb.w0, qb.h0, qb.t0);
+            if (stage_lo) tma_store_5d(&P.mol[sI], sm + L::kQ + h * kBoxBytes, h * 64, head, qb.w0, qb.h0, qb.t0);
+          }
+          bulk_commit_group();
+          if (stage_lo) {
+            bulk_wait_group_read0();
+            mbar_arrive(stage_free);
+          }
+        }
+      } else if (row_in) {
         const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + kh * NC;
         store_row<NC>(P.o, off, ov, P.out_fp32);
         if (P.o_lo) {
           float lo[NC];
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < NC; ++i) lo[i] = ov[i] - __bfloat162float(__float2bfloat16_rn(ov[i]));
           store_row<NC>(P.o_lo, off, lo, false);
         }
+      }
+      if (row_in) {
         if (kh == 0) {
           const int N = g.T * g.H * g.W;
           P.lse[int64_t(head) * N + tok] = (Lsum > 0.f && ok) ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
         }
       }
+      ++lq;
+      row = nrow;
+      beg = nbeg;
+      cnt = ncnt;
+      nsteps = nns;
     }
-    // the row is complete (copies drained, products complete) before the next one
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    // the last output tile has been read before the CTA's shared memory goes
+    if (P.tma_out && tid == 0) bulk_wait_group_read0();
   }
-  if (warp == 1) tmem_dealloc(tbase, L::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, L::kTmemCols);
+  }
 }
 
 // fp32 -> bf16 staging copy of a token-major tensor (contiguous output).
@@ -972,8 +1157,8 @@ using namespace prism;
 extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q,
                                       const void* k, const void* v, prism_dtype dtype, int32_t heads,
                                       int32_t head_dim, int64_t tok_stride, float scale, const int32_t* row_ptr,
-                                      const int32_t* col_idx, void* o, float* lse, void* o_lo, void* ws,
-                                      size_t ws_bytes, void* stream) {
+                                      const int32_t* col_idx, int64_t nnz, void* o, float* lse, void* o_lo,
+                                      void* ws, size_t ws_bytes, void* stream) {
   Geo g;
   prism_status st = make_geo(geo, &g);
   if (st != PRISM_OK) return st;
@@ -983,6 +1168,7 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
   if (heads < 1 || heads > 65535) return PRISM_ERR_UNSUPPORTED;
   if (tok_stride < int64_t(heads) * head_dim || tok_stride % 8) return PRISM_ERR_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return PRISM_ERR_ARG;
+  if (nnz < -1) return PRISM_ERR_ARG;
   for (const void* p : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(o_lo)})
     if (reinterpret_cast<uintptr_t>(p) % 16) return PRISM_ERR_ARG;
   const size_t need = bsa_fwd_ws_bytes(g, heads, head_dim, dtype);
@@ -1006,20 +1192,34 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
     qb = sq; kb = sk; vb = sv;
     in_stride = C;
   }
-  // K and V as block images: every key block the kernel gathers is then one
-  // contiguous bulk copy per 64 channels instead of 64 scattered token rows
+  // The plan. Sparse (a known nnz of at most kSparseBlocksPerRow key blocks
+  // per row on average): the short-row kernel takes every row and gathers K
+  // and V through 5-D tensor maps; each key block is read by few rows, so
+  // making block images would cost more than it saves. Otherwise K and V are
+  // made block images first: every key block the kernels gather is then one
+  // contiguous bulk copy per 64 channels instead of 64 scattered token rows;
+  // the short rows go to the short-row kernel and the long ones to
+  // bsa_fwd_kernel. Both plans compute the same result.
+  const int64_t rows = int64_t(heads) * g.n_blocks;
+  const bool all_rows = nnz >= 0 && nnz <= kSparseBlocksPerRow * rows;
   uint8_t* kimg = static_cast<uint8_t*>(ws) + c.take(block_images_bytes(g, heads, head_dim));
   uint8_t* vimg = static_cast<uint8_t*>(ws) + c.take(block_images_bytes(g, heads, head_dim));
-  if ((st = launch_block_images(g, zone_shape, kb, in_stride, heads, head_dim, kimg, ws_status(ws), s)) != PRISM_OK)
-    return st;
-  if ((st = launch_block_images(g, zone_shape, vb, in_stride, heads, head_dim, vimg, ws_status(ws), s)) != PRISM_OK)
-    return st;
+  if (!all_rows) {
+    if ((st = launch_block_images(g, zone_shape, kb, in_stride, heads, head_dim, kimg, ws_status(ws), s)) != PRISM_OK)
+      return st;
+    if ((st = launch_block_images(g, zone_shape, vb, in_stride, heads, head_dim, vimg, ws_status(ws), s)) != PRISM_OK)
+      return st;
+  }
   FwdParams P;
   std::memset(&P, 0, sizeof(P));
   const bool tma_out = dtype == PRISM_BF16;
   for (int ci = 0; ci < g.n_cand; ++ci) {
     const int bt = g.cand[ci][0], bh = g.cand[ci][1], bw = g.cand[ci][2];
     if ((st = encode_block_map(&P.mq[ci], qb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+    if (all_rows) {
+      if ((st = encode_block_map(&P.mk[ci], kb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+      if ((st = encode_block_map(&P.mv[ci], vb, g, heads, head_dim, in_stride, bt, bh, bw)) != PRISM_OK) return st;
+    }
     if (tma_out) {
       if ((st = encode_block_map(&P.mo[ci], o, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK) return st;
       if (o_lo && (st = encode_block_map(&P.mol[ci], o_lo, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK)
@@ -1041,10 +1241,11 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
   P.scale_log2 = scale * 1.4426950408889634f;
   P.out_fp32 = dtype == PRISM_FP32;
   P.heads = heads;
+  P.all_rows = all_rows ? 1 : 0;
   // long rows: one CTA per row, launched in row order (neighbouring rows share key blocks in L2);
   // short and empty rows: two CTAs per SM, each looping over its rows
   const dim3 grid(g.n_blocks, heads);
-  const dim3 grid_small(std::min(heads * g.n_blocks, 2 * device_sm_count()));
+  const dim3 grid_small(unsigned(std::min<int64_t>(rows, 2 * device_sm_count())));
   // short and empty rows first (two CTAs per SM), then the long rows
   if (head_dim == 128) {
     const size_t smem = FwdSmallSmem<128>::kTotal + 1024;
@@ -1059,6 +1260,7 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
       return PRISM_ERR_CUDA;
     bsa_fwd_small_kernel<64><<<grid_small, kSmallThreads, smem, s>>>(P);
   }
+  if (all_rows) return cuda_status(cudaGetLastError());
   if (head_dim == 128) {
     const size_t smem = FwdSmem<128>::kTotal + 1024;
     if (cudaFuncSetAttribute(bsa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=

@@ -362,6 +362,13 @@ PRISM_API prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* ro
  *       in the workspace), token stride tok_stride. head_dim 64 or 128.
  * row_ptr, col_idx: device CSR from prism_block_select (rows with no block
  *       give O = 0 and lse = -inf).
+ * nnz: row_ptr[heads*n_blocks] (the total_kept of prism_block_select), or -1
+ *       when the caller does not know it. It only chooses how the work is
+ *       laid out: with at most 8 selected key blocks per row on average the
+ *       kernel gathers K and V straight from k and v, row after row, and the
+ *       workspace's block images go unused; otherwise (and for -1) K and V
+ *       are first made block images. Any value >= -1 gives the same result;
+ *       below -1 is PRISM_ERR_ARG.
  * o: device [N, heads, head_dim] out, same dtype as q, token stride tok_stride.
  * lse: device float [heads, N] out.
  * o_lo: optional device bf16 [N, heads, head_dim] out (token stride
@@ -379,8 +386,8 @@ PRISM_API prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* ro
  */
 PRISM_API prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q, const void* k,
                            const void* v, prism_dtype dtype, int32_t heads, int32_t head_dim, int64_t tok_stride,
-                           float scale, const int32_t* row_ptr, const int32_t* col_idx, void* o, float* lse,
-                           void* o_lo, void* ws, size_t ws_bytes, void* stream);
+                           float scale, const int32_t* row_ptr, const int32_t* col_idx, int64_t nnz, void* o,
+                           float* lse, void* o_lo, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * a7 — block-sparse attention backward (Prism trains natively with the

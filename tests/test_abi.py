@@ -118,15 +118,18 @@ def test_host_validation_codes(lib):
     assert pool(ctypes.byref(g), fake, fake, fake, 0, 24, 128, 3000, fake, fake, ws, 256, None) == 1
     # attention: null pointers, bad scale, small workspace
     fwd = lib.prism_bsa_fwd
-    assert fwd(ctypes.byref(g), fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, fake, fake, None, ws,
+    assert fwd(ctypes.byref(g), fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, -1, fake, fake, None, ws,
                256, None) == 1
-    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, -1.0, fake, fake, fake, fake, None, ws,
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, -1.0, fake, fake, -1, fake, fake, None, ws,
                256, None) == 1
-    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 1, 24, 128, 3072, 0.088, fake, fake, fake, fake, None, ws,
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 1, 24, 128, 3072, 0.088, fake, fake, -1, fake, fake, None, ws,
                256, None) == 4  # fp32 inputs need staging space
     # the optional output residual must be 16-byte aligned like o
-    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, fake, fake,
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, -1, fake, fake,
                ctypes.c_void_p((1 << 20) + 2), ws, 1 << 40, None) == 1
+    # nnz below -1
+    assert fwd(ctypes.byref(g), fake, fake, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake, -2, fake, fake, None,
+               ws, 1 << 40, None) == 1
     bwd = lib.prism_bsa_bwd
     assert bwd(ctypes.byref(g), fake, fake, fake, fake, fake, None, fake, fake, 0, 24, 128, 3072, 0.088, fake, fake,
                1000, fake, fake, fake, ws, 256, None) == 4

@@ -155,7 +155,8 @@ def test_full_size_workload(name):
     kh = x["k"][:, h].to("cpu", torch.float64).numpy()[:, None, :]
     # ---- a6 (+ a7): sampled rows with identical selections
     o_lo = torch.empty_like(x["q"])  # bf16 workloads: the forward's rounding residual of O for D
-    o, lse = P.bsa_fwd(geo, zs, x["q"], x["k"], x["v"], sc, sel["row_ptr"], sel["col_idx"], ws=ws, o_lo=o_lo)
+    o, lse = P.bsa_fwd(geo, zs, x["q"], x["k"], x["v"], sc, sel["row_ptr"], sel["col_idx"], ws=ws, o_lo=o_lo,
+                       nnz=sel["total"])
     same_row = np.all(got == ref["mask"][0], axis=1) & ~empty
     n_rows = 4 if dense else 12  # a dense row attends to all 294912 keys
     clipped = (members > 0) & (members < 64)

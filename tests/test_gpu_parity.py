@@ -37,7 +37,13 @@ def _oracle_attention(q, k, v, do, blocks, mask, scale):
     return Oo, lse, dq, dk, dv
 
 
-def _check_attention(geo, zone_shape_np, q, k, v, do, mask, with_bwd=True):
+# The forward's two plans: "dense" (block images, long rows in the main kernel, the hint
+# nnz unknown) and "sparse" (every row in the short-row kernel, K / V gathered through
+# tensor maps; a hint of 0 kept pairs asks for it whatever the rows hold)
+FWD_NNZ = {"dense": None, "sparse": 0}
+
+
+def _check_attention(geo, zone_shape_np, q, k, v, do, mask, with_bwd=True, plan="dense"):
     """Run bsa_fwd / bsa_bwd on the CSR of `mask` and compare with the oracle."""
     dev = q.device
     H, d = q.shape[1], q.shape[2]
@@ -47,7 +53,7 @@ def _check_attention(geo, zone_shape_np, q, k, v, do, mask, with_bwd=True):
     row_ptr, col_idx, nnz = csr_from_mask(mask, dev)
     ws = P.Workspace(dev)
     o_lo = torch.empty_like(q) if q.dtype == torch.bfloat16 else None
-    o, lse = P.bsa_fwd(geo, zs, q, k, v, sc, row_ptr, col_idx, ws=ws, o_lo=o_lo)
+    o, lse = P.bsa_fwd(geo, zs, q, k, v, sc, row_ptr, col_idx, ws=ws, o_lo=o_lo, nnz=FWD_NNZ[plan])
     qd, kd, vd, dod = (f64(t) for t in (q, k, v, do))
     Or, lser, dqr, dkr, dvr = _oracle_attention(qd, kd, vd, dod, blocks, mask, sc)
     res = {"O": assert_close("O", f64(o), Or)}
@@ -99,12 +105,14 @@ def test_tiny_end_to_end():
     for r in range(H * nb):
         assert ci[rp[r]:rp[r + 1]].tolist() == np.nonzero(ref["mask"].reshape(H * nb, nb)[r])[0].tolist()
     _check_attention(geo, idx_r, q, k, v, do, ref["mask"])
+    _check_attention(geo, idx_r, q, k, v, do, ref["mask"], with_bwd=False, plan="sparse")
 
 
 # --------------------------------------------------------------------------- attention
+@pytest.mark.parametrize("plan", ["dense", "sparse"])
 @pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("density", [0.12, 0.5, 1.0])
-def test_attention_random_masks_all_shapes(d, density):
+def test_attention_random_masks_all_shapes(d, density, plan):
     """Every candidate shape in use, ragged rows (odd counts, one empty row)."""
     grid, zone = (8, 16, 24), (8, 8, 8)
     geo = P.Geometry(grid, zone, CAND)
@@ -122,15 +130,17 @@ def test_attention_random_masks_all_shapes(d, density):
     N = geo.n_tokens
     dev = torch.device("cuda")
     q, k, v, do = (torch.randn((N, H, d), generator=gen).to(torch.bfloat16).to(dev) for _ in range(4))
-    _check_attention(geo, zone_shape, q, k, v, do, mask)
+    _check_attention(geo, zone_shape, q, k, v, do, mask, plan=plan)
 
 
+@pytest.mark.parametrize("plan", ["dense", "sparse"])
 @pytest.mark.parametrize("d", [128, 64])
-def test_attention_row_lengths_across_the_short_row_kernel(d):
-    """Rows of every length from 0 to 12 key blocks: the forward sends rows of at
-    most eight blocks (four steps) to its short-row kernel and longer ones to the
-    main kernel, so both run on the same data; the lengths cross the boundary,
-    and odd lengths leave a half step."""
+def test_attention_row_lengths_across_the_short_row_kernel(d, plan):
+    """Rows of every length from 0 to 12 key blocks: in the dense plan the forward
+    sends rows of at most eight blocks (four steps) to its short-row kernel and
+    longer ones to the main kernel, so both run on the same data; the lengths
+    cross the boundary, and odd lengths leave a half step. In the sparse plan the
+    short-row kernel pipelines every row, empty ones in between."""
     grid, zone = (8, 16, 24), (8, 8, 8)
     geo = P.Geometry(grid, zone, CAND)
     nz, nb = geo.counts()
@@ -146,10 +156,11 @@ def test_attention_row_lengths_across_the_short_row_kernel(d):
     N = geo.n_tokens
     dev = torch.device("cuda")
     q, k, v, do = (torch.randn((N, H, d), generator=gen).to(torch.bfloat16).to(dev) for _ in range(4))
-    _check_attention(geo, zone_shape, q, k, v, do, mask)
+    _check_attention(geo, zone_shape, q, k, v, do, mask, plan=plan)
 
 
-def test_attention_strided_tokens():
+@pytest.mark.parametrize("plan", ["dense", "sparse"])
+def test_attention_strided_tokens(plan):
     """Q/K/V/O as views with a token stride larger than heads*head_dim."""
     grid, zone = (8, 8, 16), (8, 8, 8)
     geo = P.Geometry(grid, zone, CAND)
@@ -169,7 +180,7 @@ def test_attention_strided_tokens():
     row_ptr, col_idx, nnz = csr_from_mask(mask, dev)
     sc = scale_for(d)
     o = torch.empty((N, 4, H, d), dtype=torch.bfloat16, device=dev)[:, 1]
-    o, lse = P.bsa_fwd(geo, zs, q, k, v, sc, row_ptr, col_idx, out=o)
+    o, lse = P.bsa_fwd(geo, zs, q, k, v, sc, row_ptr, col_idx, out=o, nnz=FWD_NNZ[plan])
     Or, lser, _, _, _ = _oracle_attention(f64(q), f64(k), f64(v), f64(do), blocks, mask, sc)
     assert_close("O strided", f64(o), Or)
 
@@ -431,8 +442,9 @@ def _partial_geometry(seed):
     return geo, nz, nb, zone_shape, blocks
 
 
+@pytest.mark.parametrize("plan", ["dense", "sparse"])
 @pytest.mark.parametrize("d", [128, 64])
-def test_attention_partial_grid(d):
+def test_attention_partial_grid(d, plan):
     """Blocks clipped by the grid's edge (fewer than 64 member tokens) as queries
     and keys, empty blocks inside the selected sets, a row whose only selected
     block is empty (no keys: O = 0, LSE = -inf), forward and backward."""
@@ -451,7 +463,7 @@ def test_attention_partial_grid(d):
     N = geo.n_tokens
     dev = torch.device("cuda")
     q, k, v, do = (torch.randn((N, H, d), generator=gen).to(torch.bfloat16).to(dev) for _ in range(4))
-    _check_attention(geo, zone_shape, q, k, v, do, mask)
+    _check_attention(geo, zone_shape, q, k, v, do, mask, plan=plan)
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
