@@ -34,9 +34,10 @@ sys.path.insert(0, ROOT)
 METRIC = "2K block-sparse attn fwd+bwd ms/layer; achieved TFLOP/s vs BF16 tensor peak"
 UNIT = "ms/layer"
 FWD_FLOP_PER_PAIR = 4 * 64 * 64 * 128  # QK^T and PV over one (query block, key block) pair, d = 128
-# the forward takes its sparse plan (one short-row kernel, no block images) up to this many kept key
-# blocks per row on average (the library's threshold, restated for the launch count)
-FWD_SPARSE_BLOCKS_PER_ROW = 8
+# the attention takes its sparse plan (the forward's short-row kernel alone, no block images in the
+# forward or the backward) up to this many kept key blocks per row on average (the library's
+# threshold, restated for the launch count)
+SPARSE_BLOCKS_PER_ROW = 32
 BWD_FLOP_PER_PAIR = 2.5 * FWD_FLOP_PER_PAIR
 # DRAM bytes (read + write) per selected (query block, key block) pair of the three attention
 # kernels together (forward, dQ, dK/dV), from one ncu capture (dram__bytes_read.sum +
@@ -245,8 +246,8 @@ class Pipeline:
     STAGES = ("zone_shapes", "block_pool", "block_select", "bsa_fwd", "bsa_bwd")
     # kernels each stage launches (prism kernels only; memsets excluded)
     # (bsa_fwd: K and V block images + the short-row and main attention kernels, or the short-row kernel
-    # alone when the rows hold at most 8 key blocks on average; bsa_bwd: prep, CSC (3), K/V images, dQ,
-    # Q/dO images, dK/dV)
+    # alone when the rows hold at most 32 key blocks on average; bsa_bwd: prep, CSC (3), K/V images, dQ,
+    # Q/dO images, dK/dV, without the images in that case)
     # (block_select: the tf32 split of q and k, then per round of heads whose logits fit in 1 GiB a score
     # GEMM and a selection launch, then the CSR scan; the rounds are counted in launches_per_step)
     LAUNCHES = {"zone_shapes": 4, "block_pool": 1, "block_select": 3, "bsa_fwd": 4, "bsa_bwd": 11}
@@ -274,8 +275,8 @@ class Pipeline:
 
     def launches_per_step(self):
         n = sum(self.LAUNCHES.values()) + 2 * self.select_rounds()
-        if self.nnz <= FWD_SPARSE_BLOCKS_PER_ROW * self.wl.heads * self.geo.counts()[1]:
-            n -= 3  # the forward's sparse plan: no block images, no main-kernel launch
+        if self.nnz <= SPARSE_BLOCKS_PER_ROW * self.wl.heads * self.geo.counts()[1]:
+            n -= 3 + 4  # the sparse plan: no block images (2 + 4), no main forward kernel
         if not self.backward:
             n -= self.LAUNCHES["bsa_bwd"]
         if self.feats is None:

@@ -45,12 +45,18 @@ constexpr int kSoftWarps = 8;
 constexpr int kGroupWarps = 4;  // the softmax warps form two groups taking alternate steps
 constexpr int kBwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kIssuerB = 2 + kSoftWarps;  // warp of the second MMA issuer
+// With at most this many kept key blocks per row on average the passes gather
+// their streamed tiles through the tensor maps (no block images)
+constexpr int kSparseBlocksPerRow = 32;
 
 struct BwdParams {
   CUtensorMap mq[kMaxCand];
   CUtensorMap mk[kMaxCand];
   CUtensorMap mv[kMaxCand];
   CUtensorMap mdo[kMaxCand];
+  // bf16 outputs: dq (dq pass) or dk and dv (dkdv pass), stored as 5-D boxes
+  CUtensorMap mo0[kMaxCand];
+  CUtensorMap mo1[kMaxCand];
   // block images (layout in host.h) of the two operands a kernel streams:
   // K and V for dq, Q and dO for dkdv
   const uint8_t* img0;
@@ -68,7 +74,49 @@ struct BwdParams {
   float scale_log2;
   float scale;
   int out_fp32;
+  int gather;  // the streamed tiles come through the 5-D tensor maps (no block images)
 };
+
+// The rows of an output block leave as box stores for bf16 outputs: each
+// thread writes its NC channels (from `c`) of row m, rounded to bf16, into a
+// swizzled [D/64][64][128 B] tile; once every thread has written, one thread
+// stores the tile with one box per 64 channels (slots outside the grid fall
+// outside the tensor and are not written).
+template <int NC>
+__device__ __forceinline__ void tile_put_row(uint8_t* tile, int m, int c, const float* v) {
+  const int dh = c / 64, c0 = (c % 64) / 8;
+#pragma unroll
+  for (int q = 0; q < NC / 8; ++q) {
+    const float* x = v + 8 * q;
+    *reinterpret_cast<uint4*>(tile + dh * kBoxBytes + sw128_offset(m, c0 + q)) =
+        make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                   pack_bf16x2(x[6], x[7]));
+  }
+}
+
+// One step slot of the two streamed operands (K and V for dq, Q and dO for
+// dkdv) of block b, each laid out [dh][block][64][128 B] from dst0 / dst1:
+// bulk copies of the block images, or (gather) 5-D tensor-map copies from the
+// box origin {shape, t0, h0, w0} cached with the block id.
+template <int D>
+__device__ __forceinline__ void stream_pair(const BwdParams& P, const CUtensorMap* map0, const CUtensorMap* map1,
+                                            uint8_t* dst0, uint8_t* dst1, int slot, int head, int b, int4 box,
+                                            uint64_t* bar) {
+  if (P.gather) {
+    for (int dh = 0; dh < D / 64; ++dh) {
+      const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
+      tma_load_5d(dst0 + off, &map0[box.x], bar, dh * 64, head, box.w, box.z, box.y);
+      tma_load_5d(dst1 + off, &map1[box.x], bar, dh * 64, head, box.w, box.z, box.y);
+    }
+  } else {
+    const size_t io = image_offset(P.g, head, b, D);
+    for (int dh = 0; dh < D / 64; ++dh) {
+      const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
+      bulk_load(dst0 + off, P.img0 + io + dh * kBoxBytes, kBoxBytes, bar);
+      bulk_load(dst1 + off, P.img1 + io + dh * kBoxBytes, kBoxBytes, bar);
+    }
+  }
+}
 
 // ----------------------------------------------------------------------- dq
 // Three slots, each holding K and V of one step (two key blocks) from its load
@@ -100,9 +148,11 @@ struct DqSmem {
   static constexpr uint32_t kDesc = kSlot0 + kSlots * kSlotBytes;  // block-id ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 256;
-  // epilogue exchange of dQ part quarters: [kh][group][64 rows][D/4 + 4 floats], over the slots
+  // epilogue exchange of dQ part quarters: [kh][group][64 rows][D/4 + 4 floats], over the slots,
+  // then the bf16 dQ tile
   static constexpr uint32_t kXPitch = D / 4 + 4;
-  static_assert(4 * 64 * kXPitch * 4 <= kSlots * kSlotBytes, "exchange buffer fits the slots");
+  static constexpr uint32_t kXTile = (4 * 64 * kXPitch * 4 + 1023) / 1024 * 1024;
+  static_assert(kXTile + D * 128 <= kSlots * kSlotBytes, "exchange buffer and tile fit the slots");
 };
 
 template <int D>
@@ -179,10 +229,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
                       qb.t0);
         }
       }
+      if (P.gather) dc.zone_shape = P.zone_shape;
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < nsteps && ok; ++j) {
         dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, status, lane);
+        int4 bx[kKB] = {};
+        if (P.gather)
+          for (int slot = 0; slot < kKB; ++slot) bx[slot] = dc.box(kKB * j + slot);
         if (lane == 0) {
           const int s = j % NS;
           // slot s last held step j - 3: free once its dQ product completed
@@ -190,14 +244,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
           if (ok) {
             uint8_t* dst = sm + L::kSlot0 + s * L::kSlotBytes;
             mbar_arrive_expect_tx(&kv_full[s], L::kSlotBytes);
-            for (int slot = 0; slot < kKB; ++slot) {
-              const size_t io = image_offset(g, head, dc.get(kKB * j + slot), D);
-              for (int dh = 0; dh < D / 64; ++dh) {
-                const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
-                bulk_load(dst + off, P.img0 + io + dh * kBoxBytes, kBoxBytes, &kv_full[s]);
-                bulk_load(dst + L::kHalf + off, P.img1 + io + dh * kBoxBytes, kBoxBytes, &kv_full[s]);
-              }
-            }
+            for (int slot = 0; slot < kKB; ++slot)
+              stream_pair<D>(P, P.mk, P.mv, dst, dst + L::kHalf, slot, head, dc.get(kKB * j + slot), bx[slot],
+                             &kv_full[s]);
             issued = j + 1;
           }
         }
@@ -364,9 +413,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     }
     const int sI = safe_shape(g, P.zone_shape, I, status);
     const BlockBox qb = block_box(g, sI, I);
-    const int tok = block_token(g, qb, m);
-    if (!g.partial || block_slot_in_grid(g, qb, m))  // a slot outside the grid has no row
-      store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, v, P.out_fp32);
+    if (!P.out_fp32) {
+      // the dQ tile after the exchange buffer (both in the slots)
+      uint8_t* tile = sm + L::kSlot0 + L::kXTile;
+      tile_put_row<NC>(tile, m, keep, v);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 32 * kSoftWarps);
+      if (warp == 2 && lane == 0) {
+        for (int h = 0; h < D / 64; ++h) tma_store_5d(&P.mo0[sI], tile + h * kBoxBytes, h * 64, head, qb.w0, qb.h0, qb.t0);
+        bulk_commit_group();
+        bulk_wait_group_read0();  // the tile stays valid until read
+      }
+    } else {
+      const int tok = block_token(g, qb, m);
+      if (!g.partial || block_slot_in_grid(g, qb, m))  // a slot outside the grid has no row
+        store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, v, true);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -413,9 +475,11 @@ struct DkvSmem {
   static constexpr uint32_t kDesc = kLD0 + 2 * kLDBytes;  // block-id ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 256;
-  // epilogue exchange of dV / dK part quarters: [dV, dK][kh][group][64 rows][D/4 + 4 floats], over the stages
+  // epilogue exchange of dV / dK part quarters: [dV, dK][kh][group][64 rows][D/4 + 4 floats], over the
+  // stages, then the bf16 dK and dV tiles
   static constexpr uint32_t kXPitch = D / 4 + 4;
-  static_assert(2 * 4 * 64 * kXPitch * 4 <= kStages * kStageBytes, "exchange buffer fits the stages");
+  static constexpr uint32_t kXTile = (2 * 4 * 64 * kXPitch * 4 + 1023) / 1024 * 1024;
+  static_assert(kXTile + 2 * D * 128 <= kStages * kStageBytes, "exchange buffer and tiles fit the stages");
   // allocated without alignment slack: the kernel checks that the dynamic
   // shared memory starts on a 1024-byte boundary
   static_assert(kTotal <= 227 * 1024, "shared-memory budget");
@@ -502,10 +566,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
                       kb.t0);
         }
       }
+      if (P.gather) dc.zone_shape = P.zone_shape;
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < nsteps && ok; ++j) {
         dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, status, lane);
+        int4 bx[kKB] = {};
+        if (P.gather)
+          for (int slot = 0; slot < kKB; ++slot) bx[slot] = dc.box(kKB * j + slot);
         if (lane == 0) {
           const int s = j % NS;
           // stage s last held step j - 3: free once its dV / dK products completed
@@ -513,14 +581,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
           if (ok) {
             uint8_t* stage = sm + L::kStage0 + s * L::kStageBytes;
             mbar_arrive_expect_tx(&st_full[s], L::kStageBytes + L::kLDBytes);
-            for (int slot = 0; slot < kKB; ++slot) {
-              const size_t io = image_offset(g, head, dc.get(kKB * j + slot), D);
-              for (int dh = 0; dh < D / 64; ++dh) {
-                const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
-                bulk_load(stage + off, P.img0 + io + dh * kBoxBytes, kBoxBytes, &st_full[s]);
-                bulk_load(stage + L::kHalf + off, P.img1 + io + dh * kBoxBytes, kBoxBytes, &st_full[s]);
-              }
-            }
+            for (int slot = 0; slot < kKB; ++slot)
+              stream_pair<D>(P, P.mq, P.mdo, stage, stage + L::kHalf, slot, head, dc.get(kKB * j + slot), bx[slot],
+                             &st_full[s]);
             issued = j + 1;
             // LSE / D buffer j % 2 last held step j - 2: free once its group read it.
             // The copies are issued even after a failed wait (an abort, results
@@ -725,13 +788,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     }
     const int sJ = safe_shape(g, P.zone_shape, J, status);
     const BlockBox kb = block_box(g, sJ, J);
-    const int tok = block_token(g, kb, m);
-    const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + keep;
     // a key slot outside the grid (a block clipped by the edge) has no row; the
     // query slots outside the grid carry P = 0 (LSE = +inf from the prep pass)
-    if (!g.partial || block_slot_in_grid(g, kb, m)) {
-      store_row<NC>(P.out0, off, vk, P.out_fp32);
-      store_row<NC>(P.out1, off, vv, P.out_fp32);
+    if (!P.out_fp32) {
+      // the dK and dV tiles after the exchange buffer (all in the stages)
+      uint8_t* tk = sm + L::kStage0 + L::kXTile;
+      uint8_t* tv = tk + D * 128;
+      tile_put_row<NC>(tk, m, keep, vk);
+      tile_put_row<NC>(tv, m, keep, vv);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 32 * kSoftWarps);
+      if (warp == 2 && lane == 0) {
+        for (int h = 0; h < D / 64; ++h) {
+          tma_store_5d(&P.mo0[sJ], tk + h * kBoxBytes, h * 64, head, kb.w0, kb.h0, kb.t0);
+          tma_store_5d(&P.mo1[sJ], tv + h * kBoxBytes, h * 64, head, kb.w0, kb.h0, kb.t0);
+        }
+        bulk_commit_group();
+        bulk_wait_group_read0();  // the tiles stay valid until read
+      }
+    } else if (!g.partial || block_slot_in_grid(g, kb, m)) {
+      const int tok = block_token(g, kb, m);
+      const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + keep;
+      store_row<NC>(P.out0, off, vk, true);
+      store_row<NC>(P.out1, off, vv, true);
     }
   }
   tc_fence_before();
@@ -969,15 +1048,30 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   P.out_fp32 = dtype == PRISM_FP32;
   uint8_t* img0 = w8 + W.img0;
   uint8_t* img1 = w8 + W.img1;
+  // The plan: with at most kSparseBlocksPerRow kept key blocks per row on
+  // average each streamed block is read by few rows (or columns), so the
+  // passes gather them through the tensor maps instead of making block
+  // images of K, V, Q and dO first. Both plans compute the same result.
+  const bool gather = nnz <= int64_t(kSparseBlocksPerRow) * rows;
+  P.gather = gather ? 1 : 0;
   // dQ: q-stationary over the CSR, streaming K and V
-  if ((st = launch_block_images(g, zone_shape, kb, in_stride, heads, head_dim, img0, status, s)) != PRISM_OK) return st;
-  if ((st = launch_block_images(g, zone_shape, vb, in_stride, heads, head_dim, img1, status, s)) != PRISM_OK) return st;
+  if (!gather) {
+    if ((st = launch_block_images(g, zone_shape, kb, in_stride, heads, head_dim, img0, status, s)) != PRISM_OK)
+      return st;
+    if ((st = launch_block_images(g, zone_shape, vb, in_stride, heads, head_dim, img1, status, s)) != PRISM_OK)
+      return st;
+  }
   P.img0 = img0;
   P.img1 = img1;
   P.ptr = row_ptr;
   P.idx = col_idx;
   P.out0 = dq;
   P.out1 = nullptr;
+  if (dtype == PRISM_BF16)
+    for (int c = 0; c < g.n_cand; ++c)
+      if ((st = encode_block_map(&P.mo0[c], dq, g, heads, head_dim, tok_stride, g.cand[c][0], g.cand[c][1],
+                                 g.cand[c][2])) != PRISM_OK)
+        return st;
   if (head_dim == 128) {
     const size_t smem = DqSmem<128>::kTotal + 1024;
     if (cudaFuncSetAttribute(bsa_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
@@ -992,13 +1086,22 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   if (cudaGetLastError() != cudaSuccess) return PRISM_ERR_CUDA;
   // dK, dV: kv-stationary over the CSC, streaming Q and dO (the images
   // overwrite those of K and V once the dq pass is done: same stream)
-  if ((st = launch_block_images(g, zone_shape, qb, in_stride, heads, head_dim, img0, status, s)) != PRISM_OK) return st;
-  if ((st = launch_block_images(g, zone_shape, dob, in_stride, heads, head_dim, img1, status, s)) != PRISM_OK)
-    return st;
+  if (!gather) {
+    if ((st = launch_block_images(g, zone_shape, qb, in_stride, heads, head_dim, img0, status, s)) != PRISM_OK)
+      return st;
+    if ((st = launch_block_images(g, zone_shape, dob, in_stride, heads, head_dim, img1, status, s)) != PRISM_OK)
+      return st;
+  }
   P.ptr = cptr;
   P.idx = ridx;
   P.out0 = dk;
   P.out1 = dv;
+  if (dtype == PRISM_BF16)
+    for (int c = 0; c < g.n_cand; ++c) {
+      const int bt = g.cand[c][0], bh = g.cand[c][1], bw = g.cand[c][2];
+      if ((st = encode_block_map(&P.mo0[c], dk, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK) return st;
+      if ((st = encode_block_map(&P.mo1[c], dv, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK) return st;
+    }
   if (head_dim == 128) {
     const size_t smem = DkvSmem<128>::kTotal;
     if (cudaFuncSetAttribute(bsa_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=

@@ -146,16 +146,16 @@ __device__ __forceinline__ int4 block_box_coords(const Geo& g, const int32_t* zo
 // `cnt` blocks processed `step` (a power of two) per step: e < cnt is the
 // list's e-th block; a ragged tail (e >= cnt in the last step) repeats the
 // step's first block. An id out of range is reported and replaced by 0. With
-// `boxes` set, the same warp-wide pass also looks up each block's zone shape
-// and box origin (block_box_coords), so the thread that issues tensor-map
-// copies of the blocks has neither a dependent load nor the box arithmetic on
-// its path.
+// `zone_shape` set, the same warp-wide pass also looks up each block's zone
+// shape and box origin (block_box_coords) and keeps it in the register of
+// the lane that read the id, so the thread that issues tensor-map copies of
+// the blocks has neither a dependent load nor the box arithmetic on its path.
 struct IdCache {
   int* ring;  // shared memory, kDescRing entries
   int filled;
   int step = 2;
-  int4* boxes = nullptr;                // shared memory, kDescRing entries, or null
-  const int32_t* zone_shape = nullptr;  // with boxes
+  const int32_t* zone_shape = nullptr;  // non-null: keep box origins
+  int4 mybox = make_int4(0, 0, 0, 0);   // this lane's entry of the latest fill
   // Makes entries [0, e] available; the whole warp must call it.
   __device__ __forceinline__ void ensure(int e, const Geo& g, const int32_t* list, int beg, int cnt, int* status,
                                          int lane) {
@@ -169,13 +169,20 @@ struct IdCache {
         J = 0;
       }
       ring[ee % kDescRing] = J;
-      if (boxes) boxes[ee % kDescRing] = block_box_coords(g, zone_shape, J, status);
+      if (zone_shape) mybox = block_box_coords(g, zone_shape, J, status);
       __syncwarp();
       filled += 32;
     }
   }
   __device__ __forceinline__ int get(int e) const { return ring[e % kDescRing]; }
-  __device__ __forceinline__ int4 box(int e) const { return boxes[e % kDescRing]; }
+  // {shape, t0, h0, w0} of entry e, which must belong to the latest fill
+  // (fills are 32-entry aligned: entry e sits in lane e % 32); the whole warp
+  // calls it
+  __device__ __forceinline__ int4 box(int e) const {
+    const int l = e & 31;
+    return make_int4(__shfl_sync(0xffffffffu, mybox.x, l), __shfl_sync(0xffffffffu, mybox.y, l),
+                     __shfl_sync(0xffffffffu, mybox.z, l), __shfl_sync(0xffffffffu, mybox.w, l));
+  }
 };
 
 // Byte offset of the operand image of (head, block) in a block-major image

@@ -69,7 +69,7 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int kSmallSteps = 4;  // rows of up to 8 key blocks go to bsa_fwd_small_kernel
 // With at most this many selected key blocks per row on average the short-row
 // kernel takes every row (the sparse plan)
-constexpr int kSparseBlocksPerRow = 8;
+constexpr int kSparseBlocksPerRow = 32;
 
 struct FwdParams {
   CUtensorMap mq[kMaxCand];
@@ -589,8 +589,7 @@ struct FwdSmallSmem {
   static constexpr uint32_t kX = kRed + kRedBytes;
   static constexpr uint32_t kXBytes = 2 * 64 * kXPitch * 4;
   static_assert(kX % 1024 == 0 && kXBytes >= D * 128, "the exchange buffer holds one swizzled output tile");
-  static constexpr uint32_t kBox = kX + kXBytes;  // box origins of the ring's blocks (5-D copies)
-  static constexpr uint32_t kDesc = kBox + kDescRing * 16;  // block-id ring
+  static constexpr uint32_t kDesc = kX + kXBytes;  // block-id ring
   static constexpr uint32_t kBar = kDesc + kDescRing * 4;
   static constexpr uint32_t kTotal = kBar + 128;
   static_assert(2 * (kTotal + 2048) <= 228 * 1024, "two CTAs per SM");
@@ -713,10 +712,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
-    if (P.all_rows) {
-      dc.boxes = reinterpret_cast<int4*>(sm + L::kBox);
-      dc.zone_shape = P.zone_shape;
-    }
+    if (P.all_rows) dc.zone_shape = P.zone_shape;
     bool ok = true;
     int lq = 0, gs = 0, q_iss = 0, k_iss = 0, v_iss = 0;
     for (int row = blockIdx.x; row < rows && ok; row += gridDim.x) {
@@ -745,14 +741,16 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
       dc.filled = 0;
       for (int j = 0; j < nsteps && ok; ++j, ++gs) {
         dc.ensure(kKB * j + kKB - 1, g, P.col_idx, beg, cnt, status, lane);
+        int4 bx[kKB] = {};
+        if (P.all_rows)
+          for (int slot = 0; slot < kKB; ++slot) bx[slot] = dc.box(kKB * j + slot);
         if (lane == 0) {
           // the K slot last held step gs - 1: free once its S completed
           if (gs > 0) ok = mbar_wait_abortable(k_free, (gs - 1) & 1, status, abort_flag);
           if (ok) {
             mbar_arrive_expect_tx(k_full, L::kSlotBytes);
             for (int slot = 0; slot < kKB; ++slot)
-              small_load_kv<D>(P, false, sm + L::kK, slot, head, dc.get(kKB * j + slot),
-                               P.all_rows ? dc.box(kKB * j + slot) : int4{}, k_full);
+              small_load_kv<D>(P, false, sm + L::kK, slot, head, dc.get(kKB * j + slot), bx[slot], k_full);
             k_iss = gs + 1;
           }
           // the V slot last held step gs - 1: free once its PV completed
@@ -760,8 +758,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bsa_fwd_small_kernel(const _
           if (ok) {
             mbar_arrive_expect_tx(v_full, L::kSlotBytes);
             for (int slot = 0; slot < kKB; ++slot)
-              small_load_kv<D>(P, true, sm + L::kV, slot, head, dc.get(kKB * j + slot),
-                               P.all_rows ? dc.box(kKB * j + slot) : int4{}, v_full);
+              small_load_kv<D>(P, true, sm + L::kV, slot, head, dc.get(kKB * j + slot), bx[slot], v_full);
             v_iss = gs + 1;
           }
         }

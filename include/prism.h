@@ -364,7 +364,7 @@ PRISM_API prism_status prism_mask_to_csr(const uint32_t* mask, const int32_t* ro
  *       give O = 0 and lse = -inf).
  * nnz: row_ptr[heads*n_blocks] (the total_kept of prism_block_select), or -1
  *       when the caller does not know it. It only chooses how the work is
- *       laid out: with at most 8 selected key blocks per row on average the
+ *       laid out: with at most 32 selected key blocks per row on average the
  *       kernel gathers K and V straight from k and v, row after row, and the
  *       workspace's block images go unused; otherwise (and for -1) K and V
  *       are first made block images. Any value >= -1 gives the same result;
@@ -399,6 +399,9 @@ PRISM_API prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* z
  * outputs (with o_lo, D_i = dO_i . (O_i + O_lo_i)); dout is device
  * [N, heads, head_dim]; dq, dk, dv are device outs like q. nnz =
  * row_ptr[heads*n_blocks] (for workspace sizing; checked against ws_bytes).
+ * With at most 32 selected key blocks per row on average the passes gather
+ * their streamed blocks straight from the inputs and the block-major copies
+ * below go unused; the result is the same.
  * ws: at least prism_workspace_size(PRISM_OP_BSA_BWD, ...) bytes: D and the
  *       LSE in block order, the CSC of the selection (4 bytes per selected
  *       pair), two block-major operand copies (2 * heads * n_blocks *
