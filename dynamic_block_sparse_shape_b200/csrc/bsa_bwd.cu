@@ -75,7 +75,21 @@ struct BwdParams {
   float scale;
   int out_fp32;
   int gather;  // the streamed tiles come through the 5-D tensor maps (no block images)
+  int heads;
 };
+
+// List of row (or column) `row` of ptr / idx: its first entry and its length
+// (a malformed length is reported and read as 0).
+__device__ __forceinline__ int bwd_list(const BwdParams& P, int row, int* beg) {
+  const int b = __ldg(P.ptr + row);
+  int cnt = __ldg(P.ptr + row + 1) - b;
+  if (cnt < 0 || cnt > P.g.n_blocks) {
+    atomicOr(P.status, kDevErrBounds);
+    cnt = 0;
+  }
+  *beg = b;
+  return cnt;
+}
 
 // The rows of an output block leave as box stores for bf16 outputs: each
 // thread writes its NC channels (from `c`) of row m, rounded to bf16, into a
@@ -435,6 +449,349 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
+  }
+}
+
+// ------------------------------------------------------------ dq, short rows
+// The sparse plan's dQ pass (rows of few key blocks on average; every row): a
+// row of a few key blocks is mostly fixed cost (the Q / dO copies, the first
+// K / V copies, the epilogue), so each CTA takes about half the tensor memory
+// and 96 KB of shared memory, two CTAs share an SM, and each loops over the
+// rows of its stride with the copies of the next row started as soon as the
+// current one frees their buffers.
+//   warp 0      copies: per row Q and dO (5-D TMA) into two tiles that are the
+//               A operands of the row's S / dP products; per step K and V of
+//               the step's two key blocks (5-D TMA from the box origins the
+//               block-id prefetch keeps);
+//   warp 1      TMEM owner and issuer, per step: S_j = Q [K_j0 K_j1]^T and
+//               dP_j = dO [V_j0 V_j1]^T (.ws M=64, N=128, A from shared
+//               memory), then, once dS_j is written over S_j's first 32
+//               columns, dQ_parts += dS_j K_j (dS as the TMEM A operand);
+//   warps 2..5  dS = P (dP - D) with P = exp2(S scale log2e - LSE log2e),
+//               one thread per TMEM lane (row m, key block kh of the step),
+//               then the epilogue: the key-block parts of dQ added across
+//               the lane halves through shared memory (over the V slot, free
+//               once the row's last dP has completed), scaled, and stored.
+// TMEM: S (dS over its first 32 columns) at 0, dP at 64, the dQ parts at 128.
+// Barrier phases run on across rows (steps and rows of the CTA counted from
+// 0); every wait is placed so that the phase after the awaited one needs a
+// step the waiter has not yet enabled.
+constexpr int kDqSmallThreads = 64 + 128;
+
+template <int D>
+struct DqSmallSmem {
+  static constexpr uint32_t kQ = 0;                      // Q [dh][64][128 B]
+  static constexpr uint32_t kDO = D * 128;               // dO
+  static constexpr uint32_t kHalf = kKB * D * 128;       // K (or V) of one step, [dh][key block][64][128 B]
+  static constexpr uint32_t kK = 2 * D * 128;
+  static constexpr uint32_t kV = kK + kHalf;
+  static constexpr uint32_t kDesc = kV + kHalf;          // block-id ring
+  static constexpr uint32_t kBar = kDesc + kDescRing * 4;
+  static constexpr uint32_t kTotal = kBar + 128;
+  // epilogue over the V slot: exchange of half rows [lane half][64 rows][kXC + 4 floats] in rounds
+  // of kXC channels, then the bf16 dQ tile ([dh][64][128 B], swizzled)
+  static constexpr int kXC = D == 128 ? 32 : 16;
+  static constexpr uint32_t kXPitch = kXC + 4;
+  static_assert(2 * 64 * kXPitch * 4 <= kHalf && D * 128 <= kHalf, "epilogue buffers fit the V slot");
+  static_assert(2 * (kTotal + 2048) <= 228 * 1024, "two CTAs per SM");
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kTS = 0, kTP = 64, kTQ = 128;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kDqSmallThreads, 2) bsa_dq_small_kernel(const __grid_constant__ BwdParams P) {
+  using L = DqSmallSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  uint64_t* qd_full = bars + 0;     // Q and dO of the row landed
+  uint64_t* qd_free = bars + 1;     // the row's last S / dP products complete (Q, dO tiles free)
+  uint64_t* k_full = bars + 2;      // K of the step landed
+  uint64_t* v_full = bars + 3;      // V of the step landed
+  uint64_t* v_free = bars + 4;      // S / dP of the step complete (V slot free)
+  uint64_t* s_full = bars + 5;      // S / dP of the step complete
+  uint64_t* ds_full = bars + 6;     // dS of the step written (4 warps)
+  uint64_t* b_done = bars + 7;      // dQ product of the step complete (K slot, S / dP columns free)
+  uint64_t* dq_free = bars + 8;     // the row's dQ parts read by the epilogue (4 warps)
+  uint64_t* stage_free = bars + 9;  // the row's epilogue done with the V slot
+  uint64_t* mma_done = bars + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
+  const Geo& g = P.g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = P.status;
+  const int rows = P.heads * g.n_blocks;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 6 || i == 8) ? 4 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tS = tbase + L::kTS, tP = tbase + L::kTP, tdQ = tbase + L::kTQ;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    IdCache dc{reinterpret_cast<int*>(sm + L::kDesc), 0};
+    dc.zone_shape = P.zone_shape;
+    bool ok = true;
+    int lq = 0, gs = 0, q_iss = 0, k_iss = 0, v_iss = 0;
+    for (int row = blockIdx.x; row < rows && ok; row += gridDim.x) {
+      int beg;
+      const int cnt = bwd_list(P, row, &beg);
+      const int nsteps = (cnt + kKB - 1) / kKB;
+      if (nsteps == 0) continue;
+      const int I = row % g.n_blocks, head = row / g.n_blocks;
+      if (lane == 0) {
+        // the tiles held the previous row's Q / dO until its last S / dP completed
+        if (lq > 0) ok = mbar_wait_abortable(qd_free, (lq - 1) & 1, status, abort_flag);
+        if (ok) {
+          const int sI = safe_shape(g, P.zone_shape, I, status);
+          const BlockBox qb = block_box(g, sI, I);
+          mbar_arrive_expect_tx(qd_full, 2 * D * 128);
+          for (int dh = 0; dh < D / 64; ++dh) {
+            tma_load_5d(sm + L::kQ + dh * kBoxBytes, &P.mq[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+            tma_load_5d(sm + L::kDO + dh * kBoxBytes, &P.mdo[sI], qd_full, dh * 64, head, qb.w0, qb.h0, qb.t0);
+          }
+          q_iss = lq + 1;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      dc.filled = 0;
+      for (int j = 0; j < nsteps && ok; ++j, ++gs) {
+        dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, status, lane);
+        int4 bx[kKB];
+        for (int slot = 0; slot < kKB; ++slot) bx[slot] = dc.box(kKB * j + slot);
+        if (lane == 0) {
+          // the K slot last held step gs - 1: free once its dQ product completed
+          if (gs > 0) ok = mbar_wait_abortable(b_done, (gs - 1) & 1, status, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(k_full, L::kHalf);
+            for (int slot = 0; slot < kKB; ++slot)
+              for (int dh = 0; dh < D / 64; ++dh)
+                tma_load_5d(sm + L::kK + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &P.mk[bx[slot].x], k_full, dh * 64,
+                            head, bx[slot].w, bx[slot].z, bx[slot].y);
+            k_iss = gs + 1;
+          }
+          // the V slot last held step gs - 1 (free once its S / dP completed)
+          // and, before a row's first step, the previous row's epilogue
+          if (ok && gs > 0) ok = mbar_wait_abortable(v_free, (gs - 1) & 1, status, abort_flag);
+          if (ok && j == 0 && lq > 0) ok = mbar_wait_abortable(stage_free, (lq - 1) & 1, status, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(v_full, L::kHalf);
+            for (int slot = 0; slot < kKB; ++slot)
+              for (int dh = 0; dh < D / 64; ++dh)
+                tma_load_5d(sm + L::kV + dh * (kKB * kBoxBytes) + slot * kBoxBytes, &P.mv[bx[slot].x], v_full, dh * 64,
+                            head, bx[slot].w, bx[slot].z, bx[slot].y);
+            v_iss = gs + 1;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      ++lq;
+    }
+    if (lane == 0) {
+      // drain: every issued copy has landed before the CTA may exit (one buffer each: the last)
+      if (q_iss > 0) mbar_wait(qd_full, (q_iss - 1) & 1, status);
+      if (k_iss > 0) mbar_wait(k_full, (k_iss - 1) & 1, status);
+      if (v_iss > 0) mbar_wait(v_full, (v_iss - 1) & 1, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16_f32(64, 64 * kKB, false, false);
+      const uint64_t dQa = sdesc_sw128(smem_u32(sm + L::kQ), 16, 1024);    // Q as A of S
+      const uint64_t dDOa = sdesc_sw128(smem_u32(sm + L::kDO), 16, 1024);  // dO as A of dP
+      const uint64_t dKb = sdesc_sw128(smem_u32(sm + L::kK), 16, 1024);    // K as B of S
+      const uint64_t dVb = sdesc_sw128(smem_u32(sm + L::kV), 16, 1024);    // V as B of dP
+      // B of the dQ product = K of the step, MN-major, N = 128: 64 channels of
+      // key block 0 then the same channels of key block 1
+      const uint32_t idQ = idesc_bf16_f32(64, 128, false, true);
+      const uint64_t dKmn = sdesc_sw128(smem_u32(sm + L::kK), kBoxBytes, 1024);
+      bool ok = true;
+      int lq = 0, gs = 0;
+      for (int row = blockIdx.x; row < rows && ok; row += gridDim.x) {
+        int beg;
+        const int cnt = bwd_list(P, row, &beg);
+        const int nsteps = (cnt + kKB - 1) / kKB;
+        if (nsteps == 0) continue;
+        ok = mbar_wait_abortable(qd_full, lq & 1, status, abort_flag);
+        for (int j = 0; j < nsteps && ok; ++j, ++gs) {
+          // K and V of the step landed; the previous step's dQ product (which
+          // read dS from the S columns) complete
+          ok = mbar_wait_abortable(k_full, gs & 1, status, abort_flag) &&
+               mbar_wait_abortable(v_full, gs & 1, status, abort_flag) &&
+               (gs == 0 || mbar_wait_abortable(b_done, (gs - 1) & 1, status, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws(tS, dQa + kmajor_step(kk, kBoxBytes), dKb + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ws(tP, dDOa + kmajor_step(kk, kBoxBytes), dVb + kmajor_step(kk, kKB * kBoxBytes), idS, kk > 0 ? 1u : 0u);
+          mma_commit(s_full);
+          mma_commit(v_free);
+          if (j == nsteps - 1) mma_commit(qd_free);
+          // dS written; before a row's first dQ product the previous row's parts read
+          ok = mbar_wait_abortable(ds_full, gs & 1, status, abort_flag) &&
+               (j > 0 || lq == 0 || mbar_wait_abortable(dq_free, (lq - 1) & 1, status, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              mma_ws_ts(tdQ + c * 64, tS + kk * 8, dKmn + uint64_t((c * kKB * kBoxBytes + kk * 2048) >> 4), idQ,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(b_done);
+        }
+        ++lq;
+      }
+      // every product this thread issued has completed before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, status);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    // The four warps run the same control flow whatever their waits return
+    // (after a timeout the waits give up at once and the values are
+    // discarded), so their named barriers always match.
+    const int sp = warp & 3;  // TMEM lane quarter of this warp
+    const int Ln = sp * 32 + lane;
+    const int m = Ln & 63, kh = Ln >> 6;
+    const uint32_t lane_off = uint32_t(sp * 32) << 16;
+    const int tid = threadIdx.x - 64;
+    constexpr int NC = D / 2;
+    int lq = 0, gs = 0;
+    for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+      int beg;
+      const int cnt = bwd_list(P, row, &beg);
+      const int nsteps = (cnt + kKB - 1) / kKB;
+      const int I = row % g.n_blocks, head = row / g.n_blocks;
+      const int sI = safe_shape(g, P.zone_shape, I, status);
+      const BlockBox qb = block_box(g, sI, I);
+      if (nsteps == 0) {
+        // no key block: dQ = 0
+        if (!g.partial || block_slot_in_grid(g, qb, m)) {
+          float z[NC];
+#pragma unroll
+          for (int i = 0; i < NC; ++i) z[i] = 0.f;
+          store_row<NC>(P.out0, int64_t(block_token(g, qb, m)) * P.tok_stride + int64_t(head) * D + kh * NC, z,
+                        P.out_fp32);
+        }
+        continue;
+      }
+      const float lse2 = P.lse2[size_t(row) * 64 + m];
+      const float dm = P.dvec[size_t(row) * 64 + m];
+      for (int j = 0; j < nsteps; ++j, ++gs) {
+        const bool valid = (j * kKB + kh) < cnt;  // warp-uniform
+        // keys of a key block clipped by the grid's edge (read before the wait)
+        uint64_t members = ~uint64_t(0);
+        if (g.partial && valid) members = key_block_members(g, P.zone_shape, __ldg(P.idx + beg + j * kKB + kh));
+        mbar_wait_abortable(s_full, gs & 1, status, abort_flag);
+        tc_fence_after();
+        uint32_t pk[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t rs[32], rp[32];
+          tmem_ld32(tS + lane_off + h * 32, rs);
+          tmem_ld32(tP + lane_off + h * 32, rp);
+          tmem_ld_wait();
+          mask_scores32(rs, uint32_t(members >> (32 * h)));  // P = exp2(-inf) = 0 there, hence dS = 0
+          if (valid) {
+            const float c = P.scale_log2, nl = -lse2;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(rs[2 * i]), c, nl));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(rs[2 * i + 1]), c, nl));
+              pk[16 * h + i] =
+                  pack_bf16x2(p0 * (__uint_as_float(rp[2 * i]) - dm), p1 * (__uint_as_float(rp[2 * i + 1]) - dm));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[16 * h + i] = 0u;
+          }
+        }
+        // dS over the first 32 columns of S (every S / dP value of this lane was read above)
+        tmem_st16(tS + lane_off, pk);
+        tmem_st16(tS + lane_off + 16, pk + 16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full);
+      }
+      // ---------------------------------------------------------- epilogue
+      // the row's last dQ product complete: the dQ parts are final and the V
+      // slot is free (every dP of the row completed before it)
+      mbar_wait_abortable(b_done, (gs - 1) & 1, status, abort_flag);
+      tc_fence_after();
+      named_bar_sync(1, 128);
+      const bool ok = *abort_flag == 0;
+      // this thread holds the key-block-kh part of dQ row m; it keeps channel
+      // half kh and hands half kh ^ 1 to the other lane half, kXC channels per round
+      float* X = reinterpret_cast<float*>(sm + L::kV);
+      float v[NC];
+#pragma unroll
+      for (int c0 = 0; c0 < NC; c0 += L::kXC) {
+        float gv[L::kXC];
+        tmem_ld_f<L::kXC>(tdQ + lane_off + (kh ^ 1) * NC + c0, gv);
+        tmem_ld_f<L::kXC>(tdQ + lane_off + kh * NC + c0, v + c0);
+        if (c0 + L::kXC == NC) {
+          // this warp's last read of the dQ parts: the next row's first dQ product may overwrite them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dq_free);
+        }
+        float* xo = X + ((kh ^ 1) * 64 + m) * L::kXPitch;
+#pragma unroll
+        for (int i = 0; i < L::kXC / 4; ++i)
+          reinterpret_cast<float4*>(xo)[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
+        named_bar_sync(1, 128);
+        const float* xi = X + (kh * 64 + m) * L::kXPitch;
+#pragma unroll
+        for (int i = 0; i < L::kXC / 4; ++i) {
+          const float4 t = reinterpret_cast<const float4*>(xi)[i];
+          v[c0 + 4 * i] = (v[c0 + 4 * i] + t.x) * P.scale;
+          v[c0 + 4 * i + 1] = (v[c0 + 4 * i + 1] + t.y) * P.scale;
+          v[c0 + 4 * i + 2] = (v[c0 + 4 * i + 2] + t.z) * P.scale;
+          v[c0 + 4 * i + 3] = (v[c0 + 4 * i + 3] + t.w) * P.scale;
+        }
+        named_bar_sync(1, 128);  // the exchange buffer is free for the next round (and the tile)
+      }
+#pragma unroll
+      for (int i = 0; i < NC; ++i) v[i] = ok ? v[i] : 0.f;
+      if (!P.out_fp32) {
+        uint8_t* tile = sm + L::kV;
+        tile_put_row<NC>(tile, m, kh * NC, v);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (tid == 0) {
+          for (int h = 0; h < D / 64; ++h) tma_store_5d(&P.mo0[sI], tile + h * kBoxBytes, h * 64, head, qb.w0, qb.h0, qb.t0);
+          bulk_commit_group();
+          bulk_wait_group_read0();  // the tile stays valid until read
+        }
+      } else if (!g.partial || block_slot_in_grid(g, qb, m)) {
+        store_row<NC>(P.out0, int64_t(block_token(g, qb, m)) * P.tok_stride + int64_t(head) * D + kh * NC, v, true);
+      }
+      // the V slot is free for the next row's first V: after the tile was read
+      // (tid 0 waited above) or after every thread's last exchange read
+      named_bar_sync(1, 128);
+      if (tid == 0) mbar_arrive(stage_free);
+      ++lq;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, L::kTmemCols);
   }
 }
 
@@ -1046,6 +1403,7 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   P.scale_log2 = scale * 1.4426950408889634f;
   P.scale = scale;
   P.out_fp32 = dtype == PRISM_FP32;
+  P.heads = heads;
   uint8_t* img0 = w8 + W.img0;
   uint8_t* img1 = w8 + W.img1;
   // The plan: with at most kSparseBlocksPerRow kept key blocks per row on
@@ -1072,7 +1430,23 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
       if ((st = encode_block_map(&P.mo0[c], dq, g, heads, head_dim, tok_stride, g.cand[c][0], g.cand[c][1],
                                  g.cand[c][2])) != PRISM_OK)
         return st;
-  if (head_dim == 128) {
+  if (gather) {
+    // rows short on average: the short-row kernel, two CTAs per SM, each looping over its rows
+    const dim3 grid_small(unsigned(std::min<int64_t>(rows, 2 * device_sm_count())));
+    if (head_dim == 128) {
+      const size_t smem = DqSmallSmem<128>::kTotal + 1024;
+      if (cudaFuncSetAttribute(bsa_dq_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+          cudaSuccess)
+        return PRISM_ERR_CUDA;
+      bsa_dq_small_kernel<128><<<grid_small, kDqSmallThreads, smem, s>>>(P);
+    } else {
+      const size_t smem = DqSmallSmem<64>::kTotal + 1024;
+      if (cudaFuncSetAttribute(bsa_dq_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+          cudaSuccess)
+        return PRISM_ERR_CUDA;
+      bsa_dq_small_kernel<64><<<grid_small, kDqSmallThreads, smem, s>>>(P);
+    }
+  } else if (head_dim == 128) {
     const size_t smem = DqSmem<128>::kTotal + 1024;
     if (cudaFuncSetAttribute(bsa_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
       return PRISM_ERR_CUDA;
