@@ -159,6 +159,26 @@ def test_attention_row_lengths_across_the_short_row_kernel(d, plan):
     _check_attention(geo, zone_shape, q, k, v, do, mask, plan=plan)
 
 
+def test_attention_fp32_short_rows():
+    """fp32 inputs and outputs (rounded to bf16 operands inside) with rows of 0 to
+    12 key blocks at d = 128: the sparse plan's short-row forward and dQ kernels
+    and the gathering dK/dV pass on their fp32 output paths."""
+    grid, zone = (8, 16, 24), (8, 8, 8)
+    geo = P.Geometry(grid, zone, CAND)
+    nz, nb = geo.counts()
+    rng = np.random.default_rng(57)
+    zone_shape = rng.integers(0, len(CAND), nz)
+    H, d = 2, 128
+    mask = np.zeros((H, nb, nb), dtype=bool)
+    for h in range(H):
+        for i in range(nb):
+            mask[h, i, rng.choice(nb, size=(3 * i + h) % 13, replace=False)] = True
+    gen = torch.Generator().manual_seed(59)
+    dev = torch.device("cuda")
+    q, k, v, do = (torch.randn((geo.n_tokens, H, d), generator=gen).to(dev) for _ in range(4))
+    _check_attention(geo, zone_shape, q, k, v, do, mask, plan="sparse")
+
+
 @pytest.mark.parametrize("plan", ["dense", "sparse"])
 def test_attention_strided_tokens(plan):
     """Q/K/V/O as views with a token stride larger than heads*head_dim."""
