@@ -54,7 +54,7 @@ struct BwdParams {
   CUtensorMap mk[kMaxCand];
   CUtensorMap mv[kMaxCand];
   CUtensorMap mdo[kMaxCand];
-  // bf16 outputs: dq (dq pass) or dk and dv (dkdv pass), stored as 5-D boxes
+  // bf16 outputs in the sparse plan: dq (dq pass) or dk and dv (dkdv pass), stored as 5-D boxes
   CUtensorMap mo0[kMaxCand];
   CUtensorMap mo1[kMaxCand];
   // block images (layout in host.h) of the two operands a kernel streams:
@@ -74,7 +74,6 @@ struct BwdParams {
   float scale_log2;
   float scale;
   int out_fp32;
-  int gather;  // the streamed tiles come through the 5-D tensor maps (no block images)
   int heads;
 };
 
@@ -108,15 +107,17 @@ __device__ __forceinline__ void tile_put_row(uint8_t* tile, int m, int c, const 
   }
 }
 
-// One step slot of the two streamed operands (K and V for dq, Q and dO for
-// dkdv) of block b, each laid out [dh][block][64][128 B] from dst0 / dst1:
-// bulk copies of the block images, or (gather) 5-D tensor-map copies from the
-// box origin {shape, t0, h0, w0} cached with the block id.
-template <int D>
+// One step slot of the two streamed operands (Q and dO for dkdv) of block b,
+// each laid out [dh][block][64][128 B] from dst0 / dst1: bulk copies of the
+// block images, or (G, the sparse plan) 5-D tensor-map copies from the box
+// origin {shape, t0, h0, w0} cached with the block id. The plan is a template
+// parameter: a run-time test in the copy loop cost the dense plan's dK/dV and
+// dQ passes about 2 % at 2K.
+template <int D, bool G>
 __device__ __forceinline__ void stream_pair(const BwdParams& P, const CUtensorMap* map0, const CUtensorMap* map1,
                                             uint8_t* dst0, uint8_t* dst1, int slot, int head, int b, int4 box,
                                             uint64_t* bar) {
-  if (P.gather) {
+  if constexpr (G) {
     for (int dh = 0; dh < D / 64; ++dh) {
       const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
       tma_load_5d(dst0 + off, &map0[box.x], bar, dh * 64, head, box.w, box.z, box.y);
@@ -243,14 +244,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
                       qb.t0);
         }
       }
-      if (P.gather) dc.zone_shape = P.zone_shape;
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < nsteps && ok; ++j) {
         dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, status, lane);
-        int4 bx[kKB] = {};
-        if (P.gather)
-          for (int slot = 0; slot < kKB; ++slot) bx[slot] = dc.box(kKB * j + slot);
         if (lane == 0) {
           const int s = j % NS;
           // slot s last held step j - 3: free once its dQ product completed
@@ -258,9 +255,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
           if (ok) {
             uint8_t* dst = sm + L::kSlot0 + s * L::kSlotBytes;
             mbar_arrive_expect_tx(&kv_full[s], L::kSlotBytes);
-            for (int slot = 0; slot < kKB; ++slot)
-              stream_pair<D>(P, P.mk, P.mv, dst, dst + L::kHalf, slot, head, dc.get(kKB * j + slot), bx[slot],
-                             &kv_full[s]);
+            for (int slot = 0; slot < kKB; ++slot) {
+              const size_t io = image_offset(g, head, dc.get(kKB * j + slot), D);
+              for (int dh = 0; dh < D / 64; ++dh) {
+                const uint32_t off = dh * (kKB * kBoxBytes) + slot * kBoxBytes;
+                bulk_load(dst + off, P.img0 + io + dh * kBoxBytes, kBoxBytes, &kv_full[s]);
+                bulk_load(dst + L::kHalf + off, P.img1 + io + dh * kBoxBytes, kBoxBytes, &kv_full[s]);
+              }
+            }
             issued = j + 1;
           }
         }
@@ -427,22 +429,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_kernel(const __grid_con
     }
     const int sI = safe_shape(g, P.zone_shape, I, status);
     const BlockBox qb = block_box(g, sI, I);
-    if (!P.out_fp32) {
-      // the dQ tile after the exchange buffer (both in the slots)
-      uint8_t* tile = sm + L::kSlot0 + L::kXTile;
-      tile_put_row<NC>(tile, m, keep, v);
-      fence_proxy_async_smem();
-      named_bar_sync(1, 32 * kSoftWarps);
-      if (warp == 2 && lane == 0) {
-        for (int h = 0; h < D / 64; ++h) tma_store_5d(&P.mo0[sI], tile + h * kBoxBytes, h * 64, head, qb.w0, qb.h0, qb.t0);
-        bulk_commit_group();
-        bulk_wait_group_read0();  // the tile stays valid until read
-      }
-    } else {
-      const int tok = block_token(g, qb, m);
-      if (!g.partial || block_slot_in_grid(g, qb, m))  // a slot outside the grid has no row
-        store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, v, true);
-    }
+    const int tok = block_token(g, qb, m);
+    if (!g.partial || block_slot_in_grid(g, qb, m))  // a slot outside the grid has no row
+      store_row<NC>(P.out0, int64_t(tok) * P.tok_stride + int64_t(head) * D + keep, v, P.out_fp32);
   }
   tc_fence_before();
   __syncthreads();
@@ -842,7 +831,7 @@ struct DkvSmem {
   static_assert(kTotal <= 227 * 1024, "shared-memory budget");
 };
 
-template <int D>
+template <int D, bool G>
 __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_constant__ BwdParams P) {
   using L = DkvSmem<D>;
   constexpr int NS = L::kStages;
@@ -923,13 +912,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
                       kb.t0);
         }
       }
-      if (P.gather) dc.zone_shape = P.zone_shape;
+      if constexpr (G) dc.zone_shape = P.zone_shape;
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < nsteps && ok; ++j) {
         dc.ensure(kKB * j + kKB - 1, g, P.idx, beg, cnt, status, lane);
         int4 bx[kKB] = {};
-        if (P.gather)
+        if constexpr (G)
           for (int slot = 0; slot < kKB; ++slot) bx[slot] = dc.box(kKB * j + slot);
         if (lane == 0) {
           const int s = j % NS;
@@ -939,8 +928,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
             uint8_t* stage = sm + L::kStage0 + s * L::kStageBytes;
             mbar_arrive_expect_tx(&st_full[s], L::kStageBytes + L::kLDBytes);
             for (int slot = 0; slot < kKB; ++slot)
-              stream_pair<D>(P, P.mq, P.mdo, stage, stage + L::kHalf, slot, head, dc.get(kKB * j + slot), bx[slot],
-                             &st_full[s]);
+              stream_pair<D, G>(P, P.mq, P.mdo, stage, stage + L::kHalf, slot, head, dc.get(kKB * j + slot),
+                                bx[slot], &st_full[s]);
             issued = j + 1;
             // LSE / D buffer j % 2 last held step j - 2: free once its group read it.
             // The copies are issued even after a failed wait (an abort, results
@@ -1147,8 +1136,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     const BlockBox kb = block_box(g, sJ, J);
     // a key slot outside the grid (a block clipped by the edge) has no row; the
     // query slots outside the grid carry P = 0 (LSE = +inf from the prep pass)
-    if (!P.out_fp32) {
-      // the dK and dV tiles after the exchange buffer (all in the stages)
+    if (!P.out_fp32 && G) {
+      // sparse plan: the dK and dV tiles after the exchange buffer (all in the
+      // stages) leave as box stores (the dense plan keeps plain row stores,
+      // which do not hold the CTA until a tile is read)
       uint8_t* tk = sm + L::kStage0 + L::kXTile;
       uint8_t* tv = tk + D * 128;
       tile_put_row<NC>(tk, m, keep, vk);
@@ -1166,8 +1157,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_kernel(const __grid_c
     } else if (!g.partial || block_slot_in_grid(g, kb, m)) {
       const int tok = block_token(g, kb, m);
       const int64_t off = int64_t(tok) * P.tok_stride + int64_t(head) * D + keep;
-      store_row<NC>(P.out0, off, vk, true);
-      store_row<NC>(P.out1, off, vv, true);
+      store_row<NC>(P.out0, off, vk, P.out_fp32);
+      store_row<NC>(P.out1, off, vv, P.out_fp32);
     }
   }
   tc_fence_before();
@@ -1318,6 +1309,19 @@ size_t bsa_bwd_ws_bytes(const Geo& g, int heads, int head_dim, prism_dtype dtype
 
 using namespace prism;
 
+namespace prism {
+namespace {
+template <int D, bool G>
+cudaError_t launch_dkdv(const BwdParams& P, dim3 grid, cudaStream_t s) {
+  const size_t smem = DkvSmem<D>::kTotal;
+  const cudaError_t e = cudaFuncSetAttribute(bsa_dkdv_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  bsa_dkdv_kernel<D, G><<<grid, kBwdThreads, smem, s>>>(P);
+  return cudaGetLastError();
+}
+}  // namespace
+}  // namespace prism
+
 extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* zone_shape, const void* q,
                                       const void* k, const void* v, const void* o, const void* o_lo,
                                       const float* lse, const void* dout, prism_dtype dtype, int32_t heads,
@@ -1411,7 +1415,6 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   // passes gather them through the tensor maps instead of making block
   // images of K, V, Q and dO first. Both plans compute the same result.
   const bool gather = nnz <= int64_t(kSparseBlocksPerRow) * rows;
-  P.gather = gather ? 1 : 0;
   // dQ: q-stationary over the CSR, streaming K and V
   if (!gather) {
     if ((st = launch_block_images(g, zone_shape, kb, in_stride, heads, head_dim, img0, status, s)) != PRISM_OK)
@@ -1425,7 +1428,7 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   P.idx = col_idx;
   P.out0 = dq;
   P.out1 = nullptr;
-  if (dtype == PRISM_BF16)
+  if (dtype == PRISM_BF16 && gather)
     for (int c = 0; c < g.n_cand; ++c)
       if ((st = encode_block_map(&P.mo0[c], dq, g, heads, head_dim, tok_stride, g.cand[c][0], g.cand[c][1],
                                  g.cand[c][2])) != PRISM_OK)
@@ -1470,24 +1473,14 @@ extern "C" prism_status prism_bsa_bwd(const prism_geometry* geo, const int32_t* 
   P.idx = ridx;
   P.out0 = dk;
   P.out1 = dv;
-  if (dtype == PRISM_BF16)
+  if (dtype == PRISM_BF16 && gather)
     for (int c = 0; c < g.n_cand; ++c) {
       const int bt = g.cand[c][0], bh = g.cand[c][1], bw = g.cand[c][2];
       if ((st = encode_block_map(&P.mo0[c], dk, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK) return st;
       if ((st = encode_block_map(&P.mo1[c], dv, g, heads, head_dim, tok_stride, bt, bh, bw)) != PRISM_OK) return st;
     }
-  if (head_dim == 128) {
-    const size_t smem = DkvSmem<128>::kTotal;
-    if (cudaFuncSetAttribute(bsa_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-      return PRISM_ERR_CUDA;
-    bsa_dkdv_kernel<128><<<grid, kBwdThreads, smem, s>>>(P);
-  } else {
-    const size_t smem = DkvSmem<64>::kTotal;
-    if (cudaFuncSetAttribute(bsa_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-      return PRISM_ERR_CUDA;
-    bsa_dkdv_kernel<64><<<grid, kBwdThreads, smem, s>>>(P);
-  }
+  const cudaError_t e = head_dim == 128 ? (gather ? launch_dkdv<128, true>(P, grid, s) : launch_dkdv<128, false>(P, grid, s))
+                                        : (gather ? launch_dkdv<64, true>(P, grid, s) : launch_dkdv<64, false>(P, grid, s));
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
   return cuda_status(cudaGetLastError());
 }
