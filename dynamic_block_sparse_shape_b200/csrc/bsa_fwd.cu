@@ -1240,10 +1240,10 @@ extern "C" prism_status prism_bsa_fwd(const prism_geometry* geo, const int32_t* 
   P.heads = heads;
   P.all_rows = all_rows ? 1 : 0;
   // long rows: one CTA per row, launched in row order (neighbouring rows share key blocks in L2);
-  // short and empty rows: two CTAs per SM, each looping over its rows
+  // short and empty rows (every row in the sparse plan): two CTAs per SM, each looping over its rows
   const dim3 grid(g.n_blocks, heads);
   const dim3 grid_small(unsigned(std::min<int64_t>(rows, 2 * device_sm_count())));
-  // short and empty rows first (two CTAs per SM), then the long rows
+  // short and empty rows first (two CTAs per SM), then, in the dense plan, the long rows
   if (head_dim == 128) {
     const size_t smem = FwdSmallSmem<128>::kTotal + 1024;
     if (cudaFuncSetAttribute(bsa_fwd_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
