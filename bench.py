@@ -249,8 +249,9 @@ class Pipeline:
     # alone when the rows hold at most 32 key blocks on average; bsa_bwd: prep, CSC (3), K/V images, dQ,
     # Q/dO images, dK/dV, without the images in that case)
     # (block_select: the tf32 split of q and k, then per round of heads whose logits fit in 1 GiB a score
-    # GEMM and a selection launch, then the CSR scan; the rounds are counted in launches_per_step)
-    LAUNCHES = {"zone_shapes": 4, "block_pool": 1, "block_select": 3, "bsa_fwd": 4, "bsa_bwd": 11}
+    # GEMM and a selection launch, then the CSR scan and the list fill; the rounds are counted in
+    # launches_per_step)
+    LAUNCHES = {"zone_shapes": 4, "block_pool": 1, "block_select": 4, "bsa_fwd": 4, "bsa_bwd": 11}
 
     def step(self, record=None):
         fns = (self.stage_zone, self.stage_pool, self.stage_select, self.stage_fwd, self.stage_bwd)
@@ -275,10 +276,13 @@ class Pipeline:
 
     def launches_per_step(self):
         n = sum(self.LAUNCHES.values()) + 2 * self.select_rounds()
-        if self.nnz <= SPARSE_BLOCKS_PER_ROW * self.wl.heads * self.geo.counts()[1]:
-            n -= 3 + 4  # the sparse plan: no block images (2 + 4), no main forward kernel
+        sparse = self.nnz <= SPARSE_BLOCKS_PER_ROW * self.wl.heads * self.geo.counts()[1]
+        if sparse:
+            n -= 3  # the forward's sparse plan: no K/V block images, no main forward kernel
         if not self.backward:
             n -= self.LAUNCHES["bsa_bwd"]
+        elif sparse:
+            n -= 4  # the backward's sparse plan: no block images of K, V, Q, dO
         if self.feats is None:
             n -= 1
         if self.res is None:

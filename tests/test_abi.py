@@ -214,3 +214,28 @@ def test_bench_restates_the_plan_threshold():
         assert m and int(m.group(1)) == bench.SPARSE_BLOCKS_PER_ROW, name
     hdr = open(HEADER).read()
     assert hdr.count(f"at most {bench.SPARSE_BLOCKS_PER_ROW} selected key blocks per row") == 2
+
+
+def test_bench_launch_count_per_plan():
+    """The bench's claimed kernel launches per step, for the 2K layer (two
+    selection rounds of 12 heads): 28 in the dense plan (the launch list of one
+    step: 4 zone-shape, 1 pooling, 8 selection, 4 forward, 11 backward kernels),
+    21 in the sparse plan (no block images, no main forward kernel), 15 / 12
+    for a forward-only layer without the bridge residual."""
+    import types
+    import bench
+    from dynamic_block_sparse_shape_b200 import synth
+    wl = synth.WORKLOADS["2k"]
+    geo = P.Geometry(wl.grid, wl.zone, tuple(synth.candidates_for(wl)))
+    rows = wl.heads * geo.counts()[1]
+
+    def count(nnz, backward=True, res=True):
+        fake = types.SimpleNamespace(wl=wl, geo=geo, nnz=nnz, backward=backward, feats=object(),
+                                     res=object() if res else None, LAUNCHES=bench.Pipeline.LAUNCHES)
+        fake.select_rounds = lambda: bench.Pipeline.select_rounds(fake)
+        return bench.Pipeline.launches_per_step(fake)
+
+    assert count(60958374) == 28
+    assert count(4 * rows) == 21
+    assert count(60958374, backward=False, res=False) == 28 - 11 - 2
+    assert count(4 * rows, backward=False, res=False) == 28 - 11 - 2 - 3
