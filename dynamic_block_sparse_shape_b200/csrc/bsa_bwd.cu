@@ -45,9 +45,6 @@ constexpr int kSoftWarps = 8;
 constexpr int kGroupWarps = 4;  // the softmax warps form two groups taking alternate steps
 constexpr int kBwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kIssuerB = 2 + kSoftWarps;  // warp of the second MMA issuer
-// With at most this many kept key blocks per row on average the passes gather
-// their streamed tiles through the tensor maps (no block images)
-constexpr int kSparseBlocksPerRow = 32;
 
 struct BwdParams {
   CUtensorMap mq[kMaxCand];

@@ -18,6 +18,12 @@ namespace prism {
 
 constexpr int kBoxBytes = 64 * 128;  // one 64-row x 128-byte swizzled box
 
+// The attention's sparse plan: with at most this many kept key blocks per row
+// on average (kept pairs / rows) the forward and backward passes gather their
+// streamed blocks through 5-D tensor maps instead of making block images, and
+// the short-row kernels take every row.
+constexpr int kSparseBlocksPerRow = 32;
+
 __device__ __forceinline__ void mma_ws(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
   asm volatile(

@@ -67,9 +67,6 @@ constexpr int kFwdThreads = 64 + 32 * kSoftWarps + 32;
 constexpr int kPvWarp = 2 + kSoftWarps;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kSmallSteps = 4;  // rows of up to 8 key blocks go to bsa_fwd_small_kernel
-// With at most this many selected key blocks per row on average the short-row
-// kernel takes every row (the sparse plan)
-constexpr int kSparseBlocksPerRow = 32;
 
 struct FwdParams {
   CUtensorMap mq[kMaxCand];

@@ -203,15 +203,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 
 def test_bench_restates_the_plan_threshold():
     """bench.py counts its kernel launches per plan from a restated copy of the
-    library's sparse-plan threshold (kept blocks per row on average); both
-    passes of the library and the header's documentation must say the same."""
+    library's sparse-plan threshold (kept blocks per row on average); the
+    library's constant and the header's documentation must say the same."""
     import bench
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     csrc = os.path.join(root, "dynamic_block_sparse_shape_b200", "csrc")
-    for name in ("bsa_fwd.cu", "bsa_bwd.cu"):
-        txt = open(os.path.join(csrc, name)).read()
-        m = re.search(r"constexpr int kSparseBlocksPerRow = (\d+);", txt)
-        assert m and int(m.group(1)) == bench.SPARSE_BLOCKS_PER_ROW, name
+    txt = open(os.path.join(csrc, "bsa_common.cuh")).read()
+    m = re.search(r"constexpr int kSparseBlocksPerRow = (\d+);", txt)
+    assert m and int(m.group(1)) == bench.SPARSE_BLOCKS_PER_ROW
     hdr = open(HEADER).read()
     assert hdr.count(f"at most {bench.SPARSE_BLOCKS_PER_ROW} selected key blocks per row") == 2
 
